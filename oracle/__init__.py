@@ -1,0 +1,13 @@
+"""CPU float64 oracle for scaled-dot-product attention (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA path never does.
+"""
+from .sdpa_oracle import (  # noqa: F401
+    attention_backward,
+    attention_forward,
+    attention_probs,
+    head_scores,
+    t5_relative_bucket,
+    visibility_mask,
+)

@@ -1,0 +1,272 @@
+"""CPU float64 oracle for scaled-dot-product attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  This module is imported by ``tests/``, by
+``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py``; the
+product path (the CUDA library and its Python binding) never imports, calls or
+links it, and it imports nothing from the product.  It is deliberately plain
+and slow: one explicit L x L score matrix per (batch, query head), an explicit
+boolean mask matrix, an explicit softmax and explicit chain-rule gradients, all
+in numpy float64.  No blocking, no online softmax, no fusion.
+
+What it computes, and where each piece comes from:
+
+* The attention definition softmax(Q K^T / sqrt(d_k)) V, its four steps
+  (score, scale + softmax, weighted sum, output shaped like Q) -- codelab
+  "jax-gpu-05-attention-gpu", section 1 ("Dikkat nasil calisir?") and the
+  naive reference of section 4 ("Dikkat mekanizmasini sifirdan uygulama");
+  Medium "Simplified Explanation of Attention ...", "Scaled Dot Product
+  Operation" Steps 1-4.
+* (B, T, N, H) layout of Q, K, V and the output -- codelab section 3.
+* Causal masking (query i sees keys j <= i) -- codelab section 7 ("Nedensel
+  maskeleme ekleme").
+* Causal sliding window (Mistral, window 4096) -- HF transformers issue #30461
+  "Slowdown in Training Speed Due to SDPA Mask Fix in Version 4.40.0".
+  The pages never say whether the window bound is inclusive; this oracle takes
+  the bound explicitly: key j is visible from query i iff
+  i - window_left <= j <= i + window_right (a negative bound = unbounded).
+* MHA / GQA / MQA: KV heads shared by contiguous groups of query heads,
+  g = hq // (Hq / Hkv) -- codelab section 9 ("MHA, GQA ve MQA'yi
+  karsilastirma").
+* Additive attention biases: a full (dense) bias tensor and a T5-style
+  relative-position bias looked up from a [num_buckets, H] table -- catie-aq/
+  flashT5 README (the "Full attention biases" and "T5-like relative position
+  encoding biases" implementations, and the 3 October 2024 "fa2-rpe" item).
+  The bias is added after the 1/sqrt(d) scaling and is not itself scaled.
+* T5 bucketing: the pages name the bias but print no formula.  The oracle
+  uses the published T5 closed form (Raffel et al. 2020) in its log form,
+  evaluated in float64 (see ``t5_relative_bucket``).
+* Backward: the pages print no gradient formulas; the oracle applies the chain
+  rule to the definition above (dP = dO V^T, dS = P * (dP - rowsum(P*dP)),
+  dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO, with dK / dV summed over
+  the query heads that share a KV head).
+* LSE is the natural-log log-sum-exp of each score row (bias included); a row
+  with no visible key has LSE = -inf, output 0 and zero gradients.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "t5_relative_bucket",
+    "visibility_mask",
+    "head_scores",
+    "attention_forward",
+    "attention_backward",
+    "attention_probs",
+]
+
+
+# --------------------------------------------------------------------------
+# T5 relative-position bucketing (catie-aq/flashT5 README, "T5-like relative
+# position encoding biases"; closed form of Raffel et al. 2020).
+# --------------------------------------------------------------------------
+def t5_relative_bucket(rel, num_buckets: int = 32, max_distance: int = 128,
+                       bidirectional: bool = True) -> np.ndarray:
+    """Bucket id of the signed distance ``rel = key_pos - query_pos``.
+
+    Bidirectional: half the buckets hold keys after the query (rel > 0,
+    ids offset by num_buckets/2), half the rest; within a half, distances
+    below max_exact = half/2 get one bucket each, larger distances share
+    logarithmically wider buckets up to max_distance, beyond which all
+    distances fall in the last bucket of the half.
+
+    Unidirectional (decoder): only keys at or before the query matter,
+    n = max(-rel, 0), all num_buckets are used, max_exact = num_buckets/2.
+
+    The log is evaluated in float64 and truncated toward zero.
+    """
+    rel = np.asarray(rel, dtype=np.int64)
+    nb = int(num_buckets)
+    if bidirectional:
+        nb = nb // 2
+        offset = np.where(rel > 0, nb, 0).astype(np.int64)
+        n = np.abs(rel)
+    else:
+        offset = np.zeros_like(rel)
+        n = np.maximum(-rel, 0)
+    max_exact = nb // 2
+    out = np.empty_like(rel)
+    small = n < max_exact
+    out[small] = n[small]
+    big = ~small
+    if np.any(big):
+        nf = n[big].astype(np.float64)
+        v = np.log(nf / max_exact) / math.log(max_distance / max_exact) * (nb - max_exact)
+        large = max_exact + np.trunc(v).astype(np.int64)
+        out[big] = np.minimum(large, nb - 1)
+    return out + offset
+
+
+# --------------------------------------------------------------------------
+# Mask (codelab section 7; transformers issue #30461 sliding window).
+# --------------------------------------------------------------------------
+def visibility_mask(L: int, causal: bool, window_left: int = -1,
+                    window_right: int = -1, Lk: int | None = None) -> np.ndarray:
+    """Boolean [L, Lk] matrix, True where query i may attend to key j."""
+    Lk = L if Lk is None else Lk
+    i = np.arange(L)[:, None]
+    j = np.arange(Lk)[None, :]
+    m = np.ones((L, Lk), dtype=bool)
+    if causal:
+        m &= j <= i
+    if window_left is not None and window_left >= 0:
+        m &= j >= i - window_left
+    if window_right is not None and window_right >= 0:
+        m &= j <= i + window_right
+    return m
+
+
+def _as64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # a torch tensor
+        x = x.detach().to("cpu")
+        import torch  # local: only to read torch inputs
+        x = x.to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
+                 t5_max_distance, t5_bidirectional):
+    """Additive bias for one (batch, query head), [L, L] float64 (or 0)."""
+    out = 0.0
+    if bias is not None:
+        out = out + bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0]
+    if t5_table is not None:
+        i = np.arange(L)[:, None]
+        j = np.arange(L)[None, :]
+        bucket = t5_relative_bucket(j - i, t5_num_buckets, t5_max_distance, t5_bidirectional)
+        out = out + t5_table[bucket, hq]
+    return out
+
+
+def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
+                window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
+                t5_max_distance=128, t5_bidirectional=True):
+    """Masked score matrix S for one (b, hq): scale * Q K^T + bias, -inf where
+    masked.  q: [B, L, Hq, d], k: [B, L, Hkv, d] float64 arrays."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    g = hq // (Hq // Hkv)
+    S = scale * (q[b, :, hq, :] @ k[b, :, g, :].T)
+    S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets,
+                         t5_max_distance, t5_bidirectional)
+    M = visibility_mask(L, causal, window_left, window_right)
+    S = np.where(M, S, -np.inf)
+    return S
+
+
+def _softmax_rows(S):
+    """Row softmax of a masked score matrix and its natural-log LSE."""
+    m = np.max(S, axis=1)
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    E = np.exp(S - m_safe[:, None])           # exp(-inf) = 0 for masked
+    ssum = E.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse = np.where(ssum > 0, m_safe + np.log(ssum), -np.inf)
+        P = np.where(ssum[:, None] > 0, E / ssum[:, None], 0.0)
+    return P, lse
+
+
+def _select(B, Hkv, batches, kv_heads):
+    bs = range(B) if batches is None else list(batches)
+    gs = range(Hkv) if kv_heads is None else list(kv_heads)
+    return bs, gs
+
+
+def _scale_of(d, scale):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
+    """Probability matrix P (rows sum to 1 over visible keys) for one head."""
+    q = _as64(q)
+    k = _as64(k)
+    S = head_scores(q, k, b, hq, scale=_scale_of(q.shape[-1], scale), **mask_bias)
+    P, _ = _softmax_rows(S)
+    return P
+
+
+def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
+                      window_right=-1, bias=None, t5_table=None,
+                      t5_num_buckets=32, t5_max_distance=128,
+                      t5_bidirectional=True, batches=None, kv_heads=None):
+    """O = softmax(scale Q K^T + bias, masked) V and LSE, in float64.
+
+    q: [B, L, Hq, d]; k, v: [B, L, Hkv, d]; bias: [B|1, Hq|1, L, L] or None;
+    t5_table: [num_buckets, Hq] or None.  Returns O [B, L, Hq, d] and
+    LSE [B, Hq, L]; when ``batches`` / ``kv_heads`` restrict the work to a
+    subset, entries outside it are NaN.
+    """
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    bias, t5_table = _as64(bias), _as64(t5_table)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    assert Hq % Hkv == 0
+    G = Hq // Hkv
+    sc = _scale_of(d, scale)
+    O = np.full((B, L, Hq, v.shape[-1]), np.nan)
+    LSE = np.full((B, Hq, L), np.nan)
+    kw = dict(causal=causal, window_left=window_left, window_right=window_right,
+              bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
+              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional)
+    bs, gs = _select(B, Hkv, batches, kv_heads)
+    for b in bs:
+        for g in gs:
+            for hq in range(g * G, (g + 1) * G):
+                S = head_scores(q, k, b, hq, scale=sc, **kw)
+                P, lse = _softmax_rows(S)
+                O[b, :, hq, :] = P @ v[b, :, g, :]
+                LSE[b, hq, :] = lse
+    return O, LSE
+
+
+def attention_backward(q, k, v, do, *, scale=None, causal=False,
+                       window_left=-1, window_right=-1, bias=None,
+                       t5_table=None, t5_num_buckets=32, t5_max_distance=128,
+                       t5_bidirectional=True, batches=None, kv_heads=None,
+                       return_dbias=False):
+    """Gradients of sum(O * dO) with respect to Q, K, V (float64).
+
+    Returns dQ [B, L, Hq, d], dK and dV [B, L, Hkv, d] (and, with
+    ``return_dbias``, dS per head as [B, Hq, L, L], the gradient of a dense
+    additive bias).  Subset selection as in ``attention_forward``.
+    """
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    bias, t5_table = _as64(bias), _as64(t5_table)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    sc = _scale_of(d, scale)
+    dQ = np.full(q.shape, np.nan)
+    dK = np.full(k.shape, np.nan)
+    dV = np.full(v.shape, np.nan)
+    dB = np.full((B, Hq, L, L), np.nan) if return_dbias else None
+    kw = dict(causal=causal, window_left=window_left, window_right=window_right,
+              bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
+              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional)
+    bs, gs = _select(B, Hkv, batches, kv_heads)
+    for b in bs:
+        for g in gs:
+            dK[b, :, g, :] = 0.0
+            dV[b, :, g, :] = 0.0
+            Kg = k[b, :, g, :]
+            Vg = v[b, :, g, :]
+            for hq in range(g * G, (g + 1) * G):
+                S = head_scores(q, k, b, hq, scale=sc, **kw)
+                P, _ = _softmax_rows(S)
+                dO = do[b, :, hq, :]
+                dP = dO @ Vg.T                               # dL/dP
+                Dv = np.sum(P * dP, axis=1)                  # rowsum(P * dP)
+                dS = P * (dP - Dv[:, None])                  # softmax Jacobian
+                dQ[b, :, hq, :] = sc * (dS @ Kg)
+                dK[b, :, g, :] += sc * (dS.T @ q[b, :, hq, :])
+                dV[b, :, g, :] += P.T @ dO
+                if dB is not None:
+                    dB[b, hq] = dS
+    if return_dbias:
+        return dQ, dK, dV, dB
+    return dQ, dK, dV

@@ -1,0 +1,373 @@
+"""Pins for the float64 oracle, each against something other than the oracle.
+
+Every check here is a closed form, an invariant of the definition, a hand-
+worked value, brute force, finite differences, or an independent library
+routine (torch's float64 CPU SDPA with autograd).  A dropped term, a wrong
+sign, a wrong index or a transposed operand in the oracle fails at least one.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import (attention_backward, attention_forward, attention_probs,
+                    head_scores, t5_relative_bucket, visibility_mask)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def qkv(B=2, L=12, Hq=4, Hkv=2, d=8, seed=0):
+    return (rnd((B, L, Hq, d), seed), rnd((B, L, Hkv, d), seed + 1),
+            rnd((B, L, Hkv, d), seed + 2), rnd((B, L, Hq, d), seed + 3))
+
+
+# ---------------------------------------------------------------- buckets
+def test_t5_buckets_hand_worked():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "t5_buckets.txt"))
+            if l.strip() and not l.startswith("#")]
+    rel = np.array([int(r[0]) for r in rows])
+    want = np.array([int(r[1]) for r in rows])
+    got = t5_relative_bucket(rel, 32, 128, True)
+    assert np.array_equal(got, want), list(zip(rel, got, want))
+
+
+def test_t5_buckets_integer_thresholds():
+    # The log-form boundaries for (32, 128) are n = 8,12,16,23,32,46,64,91
+    # (solve 8*16^(k/8) for k = 0..7 and round up): every n in [0, 5000].
+    thr = [8, 12, 16, 23, 32, 46, 64, 91]
+    n = np.arange(0, 5001)
+    want = np.where(n < 8, n, 7 + np.searchsorted(thr, n, side="right"))
+    want = np.minimum(want, 15)
+    assert np.array_equal(t5_relative_bucket(-n, 32, 128, True), want)
+    want_pos = np.where(n > 0, want + 16, 0)
+    assert np.array_equal(t5_relative_bucket(n, 32, 128, True), want_pos)
+
+
+def test_t5_buckets_unidirectional_brute_force():
+    # Decoder form: n = max(i - j, 0); 32 buckets, max_exact 16; keys after
+    # the query all land in bucket 0.
+    rel = np.arange(-400, 401)
+    got = t5_relative_bucket(rel, 32, 128, False)
+    for r, b in zip(rel, got):
+        n = max(-r, 0)
+        if n < 16:
+            exp = n
+        else:
+            exp = min(16 + int(math.log(n / 16) / math.log(128 / 16) * 16), 31)
+        assert b == exp, (r, b, exp)
+
+
+# ---------------------------------------------------------------- masks
+def test_mask_brute_force():
+    L = 9
+    for causal in (False, True):
+        for wl in (-1, 0, 2, 8):
+            for wr in (-1, 0, 3):
+                m = visibility_mask(L, causal, wl, wr)
+                for i in range(L):
+                    for j in range(L):
+                        ok = (not causal or j <= i) and (wl < 0 or j >= i - wl) \
+                            and (wr < 0 or j <= i + wr)
+                        assert m[i, j] == ok
+
+
+# ---------------------------------------------------------------- softmax
+@pytest.mark.parametrize("causal,wl", [(False, -1), (True, -1), (True, 3)])
+def test_probability_rows_sum_to_one(causal, wl):
+    q, k, _, _ = qkv()
+    for b in range(2):
+        for hq in range(4):
+            P = attention_probs(q, k, b, hq, causal=causal, window_left=wl)
+            assert np.allclose(P.sum(1), 1.0, atol=1e-13)
+            assert (P >= 0).all()
+            M = visibility_mask(12, causal, wl)
+            assert (P[~M] == 0).all()
+
+
+def test_row_constant_bias_is_invariant():
+    q, k, v, do = qkv()
+    B, L, Hq = 2, 12, 4
+    c = rnd((B, Hq, L, 1), 7) * np.ones((1, 1, 1, L))
+    O0, _ = attention_forward(q, k, v, causal=True)
+    O1, _ = attention_forward(q, k, v, causal=True, bias=c)
+    g0 = attention_backward(q, k, v, do, causal=True)
+    g1 = attention_backward(q, k, v, do, causal=True, bias=c)
+    assert np.allclose(O0, O1, atol=1e-12)
+    for a, b_ in zip(g0, g1):
+        assert np.allclose(a, b_, atol=1e-11)
+
+
+# ---------------------------------------------------------------- causal
+def test_causal_first_and_last_rows():
+    # codelab section 7: the first query sees only itself, the last sees all.
+    q, k, v, _ = qkv()
+    Oc, _ = attention_forward(q, k, v, causal=True)
+    Of, _ = attention_forward(q, k, v, causal=False)
+    G = 2
+    for hq in range(4):
+        assert np.array_equal(Oc[:, 0, hq], v[:, 0, hq // G])
+    assert np.allclose(Oc[:, -1], Of[:, -1], atol=1e-14)
+    assert not np.allclose(Oc[:, 0], Of[:, 0], atol=1e-3)
+
+
+def test_lower_triangular_dense_bias_equals_causal():
+    q, k, v, do = qkv()
+    L = 12
+    tri = np.where(np.tril(np.ones((L, L), bool)), 0.0, -np.inf)[None, None]
+    Oc, Lc = attention_forward(q, k, v, causal=True)
+    Ob, Lb = attention_forward(q, k, v, causal=False, bias=tri)
+    assert np.allclose(Oc, Ob, atol=1e-14) and np.allclose(Lc, Lb, atol=1e-14)
+    gc = attention_backward(q, k, v, do, causal=True)
+    gb = attention_backward(q, k, v, do, causal=False, bias=tri)
+    for a, b_ in zip(gc, gb):
+        assert np.allclose(a, b_, atol=1e-13)
+
+
+# ---------------------------------------------------------------- window
+def test_window_at_least_L_minus_1_equals_causal():
+    q, k, v, do = qkv()
+    Oc, Lc = attention_forward(q, k, v, causal=True)
+    for wl in (11, 12, 4096):
+        Ow, Lw = attention_forward(q, k, v, causal=True, window_left=wl)
+        assert np.array_equal(Oc, Ow) and np.array_equal(Lc, Lw)
+    Ow, _ = attention_forward(q, k, v, causal=True, window_left=10)
+    assert not np.allclose(Oc, Ow)   # wl = L-2 drops key 0 from the last row
+
+
+def test_window_zero_closed_form():
+    # Each query sees only its own key: O = V_g, dQ = dK = 0, dV = group sum of dO.
+    q, k, v, do = qkv()
+    O, LSE = attention_forward(q, k, v, causal=True, window_left=0)
+    dq, dk, dv = attention_backward(q, k, v, do, causal=True, window_left=0)
+    G = 2
+    for hq in range(4):
+        assert np.allclose(O[:, :, hq], v[:, :, hq // G], atol=1e-15)
+        s = np.einsum("bld,bld->bl", q[:, :, hq], k[:, :, hq // G]) / math.sqrt(8)
+        assert np.allclose(LSE[:, hq], s, atol=1e-13)
+    assert np.allclose(dq, 0, atol=1e-15) and np.allclose(dk, 0, atol=1e-15)
+    want = do.reshape(2, 12, 2, G, 8).sum(3)
+    assert np.allclose(dv, want, atol=1e-13)
+
+
+# ---------------------------------------------------------------- closed forms
+def test_zero_q_gives_mean_of_visible_values():
+    _, k, v, _ = qkv()
+    q = np.zeros((2, 12, 4, 8))
+    O, LSE = attention_forward(q, k, v, causal=True, window_left=3)
+    M = visibility_mask(12, True, 3)
+    n = M.sum(1)
+    for hq in range(4):
+        want = np.einsum("ij,bjd->bid", M / n[:, None], v[:, :, hq // 2])
+        assert np.allclose(O[:, :, hq], want, atol=1e-14)
+        assert np.allclose(LSE[:, hq], np.log(n)[None], atol=1e-14)
+
+
+def test_constant_v_and_single_key():
+    q, k, _, _ = qkv()
+    v = np.full((2, 12, 2, 8), 3.25)
+    O, _ = attention_forward(q, k, v, causal=False)
+    assert np.allclose(O, 3.25, atol=1e-14)
+    q1, k1, v1, _ = qkv(L=1)
+    O1, L1 = attention_forward(q1, k1, v1)
+    for hq in range(4):
+        assert np.array_equal(O1[:, 0, hq], v1[:, 0, hq // 2])
+        s = (q1[:, 0, hq] * k1[:, 0, hq // 2]).sum(-1) / math.sqrt(8)
+        assert np.allclose(L1[:, hq, 0], s, atol=1e-14)
+
+
+def test_fully_masked_row_is_zero():
+    q, k, v, do = qkv()
+    bias = np.zeros((1, 1, 12, 12))
+    bias[..., 5, :] = -np.inf
+    O, LSE = attention_forward(q, k, v, bias=bias)
+    assert (O[:, 5] == 0).all() and np.isneginf(LSE[:, :, 5]).all()
+    dq, dk, dv = attention_backward(q, k, v, do, bias=bias)
+    assert (dq[:, 5] == 0).all()
+    assert np.isfinite(dk).all() and np.isfinite(dv).all()
+
+
+# ---------------------------------------------------------------- GQA / MQA
+@pytest.mark.parametrize("Hkv", [1, 2, 4])
+def test_gqa_equals_mha_with_repeated_kv(Hkv):
+    q, k, v, do = qkv(Hkv=Hkv)
+    G = 4 // Hkv
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    O, LSE = attention_forward(q, k, v, causal=True)
+    Or, LSEr = attention_forward(q, kr, vr, causal=True)
+    assert np.array_equal(O, Or) and np.array_equal(LSE, LSEr)
+    dq, dk, dv = attention_backward(q, k, v, do, causal=True)
+    dqr, dkr, dvr = attention_backward(q, kr, vr, do, causal=True)
+    assert np.allclose(dq, dqr, atol=1e-14)
+    assert np.allclose(dk, dkr.reshape(2, 12, Hkv, G, 8).sum(3), atol=1e-13)
+    assert np.allclose(dv, dvr.reshape(2, 12, Hkv, G, 8).sum(3), atol=1e-13)
+
+
+def test_subset_matches_full():
+    q, k, v, do = qkv()
+    O, LSE = attention_forward(q, k, v, causal=True)
+    Os, LSEs = attention_forward(q, k, v, causal=True, batches=[1], kv_heads=[0])
+    assert np.array_equal(Os[1, :, :2], O[1, :, :2]) and np.isnan(Os[0]).all()
+    g = attention_backward(q, k, v, do, causal=True)
+    gs = attention_backward(q, k, v, do, causal=True, batches=[1], kv_heads=[0])
+    assert np.array_equal(gs[0][1, :, :2], g[0][1, :, :2])
+    assert np.array_equal(gs[1][1, :, 0], g[1][1, :, 0])
+
+
+# ---------------------------------------------------------------- biases
+def test_constant_t5_table_is_no_bias():
+    q, k, v, do = qkv()
+    table = np.tile(rnd((1, 4), 3), (32, 1))      # constant per head
+    O0, _ = attention_forward(q, k, v)
+    O1, _ = attention_forward(q, k, v, t5_table=table)
+    assert np.allclose(O0, O1, atol=1e-13)
+
+
+def test_dense_bias_equals_expanded_t5_bias():
+    q, k, v, do = qkv(L=40)
+    table = rnd((32, 4), 5)
+    L = 40
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    # expand by brute force with the hand-worked threshold rule
+    thr = [8, 12, 16, 23, 32, 46, 64, 91]
+    dense = np.zeros((1, 4, L, L))
+    for a in range(L):
+        for c in range(L):
+            r = c - a
+            n = abs(r)
+            bk = n if n < 8 else min(7 + sum(n >= t for t in thr), 15)
+            bk += 16 if r > 0 else 0
+            dense[0, :, a, c] = table[bk, :]
+    O1, L1 = attention_forward(q, k, v, t5_table=table)
+    O2, L2 = attention_forward(q, k, v, bias=dense)
+    assert np.allclose(O1, O2, atol=1e-14) and np.allclose(L1, L2, atol=1e-14)
+    g1 = attention_backward(q, k, v, do, t5_table=table)
+    g2 = attention_backward(q, k, v, do, bias=dense)
+    for a, b_ in zip(g1, g2):
+        assert np.allclose(a, b_, atol=1e-13)
+
+
+# ---------------------------------------------------------------- gradients
+def _loss(q, k, v, do, kw):
+    O, _ = attention_forward(q, k, v, **kw)
+    return float(np.sum(O * do))
+
+
+@pytest.mark.parametrize("kw", [
+    dict(causal=True),
+    dict(causal=True, window_left=2),
+    dict(causal=False, window_left=1, window_right=3),
+    dict(causal=False, t5_table="t5"),
+    dict(causal=False, bias="dense"),
+])
+def test_gradients_central_differences(kw):
+    B, L, Hq, Hkv, d = 1, 6, 4, 2, 3
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=11)
+    kw = dict(kw)
+    if kw.get("t5_table") == "t5":
+        kw["t5_table"] = rnd((32, Hq), 4)
+    if kw.get("bias") == "dense":
+        kw["bias"] = rnd((B, Hq, L, L), 4)
+    dq, dk, dv = attention_backward(q, k, v, do, **kw)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            argm = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (_loss(*args, do, kw) - _loss(*argm, do, kw)) / (2 * h)
+        err = np.max(np.abs(num - g)) / max(1.0, np.max(np.abs(g)))
+        assert err < 1e-6, (name, err)
+
+
+def test_dense_bias_gradient_central_differences():
+    B, L, Hq, Hkv, d = 1, 5, 2, 1, 3
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=21)
+    bias = rnd((B, Hq, L, L), 9)
+    *_, dB = attention_backward(q, k, v, do, causal=True, bias=bias, return_dbias=True)
+    h = 1e-6
+    M = visibility_mask(L, True)
+    for hq in range(Hq):
+        for i in range(L):
+            for j in range(L):
+                bp = bias.copy(); bp[0, hq, i, j] += h
+                bm = bias.copy(); bm[0, hq, i, j] -= h
+                num = (_loss(q, k, v, do, dict(causal=True, bias=bp))
+                       - _loss(q, k, v, do, dict(causal=True, bias=bm))) / (2 * h)
+                want = dB[0, hq, i, j] if M[i, j] else 0.0
+                assert abs(num - want) < 1e-7
+
+
+def test_D_two_ways():
+    # rowsum(P * dP) = rowsum(dO * O) for every row.
+    q, k, v, do = qkv()
+    O, _ = attention_forward(q, k, v, causal=True)
+    for b in range(2):
+        for hq in range(4):
+            P = attention_probs(q, k, b, hq, causal=True)
+            dP = do[b, :, hq] @ v[b, :, hq // 2].T
+            assert np.allclose((P * dP).sum(1), (do[b, :, hq] * O[b, :, hq]).sum(1), atol=1e-13)
+
+
+# ---------------------------------------------------------------- library
+@pytest.mark.parametrize("causal,wl,wr,bias_kind,Hkv", [
+    (False, -1, -1, None, 4), (True, -1, -1, None, 2), (True, 5, -1, None, 1),
+    (False, 4, 2, None, 4), (False, -1, -1, "t5", 4), (True, -1, -1, "dense", 2),
+])
+def test_matches_torch_float64_sdpa(causal, wl, wr, bias_kind, Hkv):
+    B, L, Hq, d = 2, 33, 4, 16
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=3)
+    kw = dict(causal=causal, window_left=wl, window_right=wr)
+    add = np.where(visibility_mask(L, causal, wl, wr), 0.0, -np.inf)[None, None]
+    if bias_kind == "t5":
+        table = rnd((32, Hq), 8)
+        kw["t5_table"] = table
+        rel = np.arange(L)[None, :] - np.arange(L)[:, None]
+        # torch side indexes the table with its own integer bucket rule
+        thr = torch.tensor([8, 12, 16, 23, 32, 46, 64, 91])
+        n = torch.from_numpy(np.abs(rel))
+        bk = torch.where(n < 8, n, torch.clamp(7 + torch.bucketize(n, thr, right=True), max=15))
+        bk = bk + torch.from_numpy((rel > 0).astype(np.int64)) * 16
+        add = add + torch.from_numpy(table)[bk].permute(2, 0, 1).numpy()[None]
+    elif bias_kind == "dense":
+        bias = rnd((B, Hq, L, L), 8)
+        kw["bias"] = bias
+        add = add + bias
+    G = Hq // Hkv
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k, requires_grad=True)
+    tv = torch.tensor(v, requires_grad=True)
+    kr = tk.repeat_interleave(G, dim=2)
+    vr = tv.repeat_interleave(G, dim=2)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(1, 2), kr.transpose(1, 2), vr.transpose(1, 2),
+        attn_mask=torch.tensor(np.broadcast_to(add, (B, Hq, L, L)).copy()))
+    out = out.transpose(1, 2)
+    out.backward(torch.tensor(do))
+    O, LSE = attention_forward(q, k, v, **kw)
+    dq, dk, dv = attention_backward(q, k, v, do, **kw)
+    assert np.allclose(O, out.detach().numpy(), atol=1e-12)
+    assert np.allclose(dq, tq.grad.numpy(), atol=1e-11)
+    assert np.allclose(dk, tk.grad.numpy(), atol=1e-11)
+    assert np.allclose(dv, tv.grad.numpy(), atol=1e-11)
+    # LSE against torch's own logsumexp of the same scores
+    s = torch.einsum("blhd,bmhd->bhlm", tq.detach(), kr.detach()) / math.sqrt(d)
+    s = s + torch.tensor(add)
+    assert np.allclose(LSE, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
+
+
+def test_head_scores_masked_entries():
+    q, k, _, _ = qkv()
+    S = head_scores(q, k, 0, 1, scale=0.5, causal=True)
+    assert np.isneginf(S[0, 1:]).all()
+    assert math.isclose(S[3, 2], 0.5 * float(q[0, 3, 1] @ k[0, 2, 0]), rel_tol=1e-14)
