@@ -1,0 +1,188 @@
+/*
+ * sdpa.h -- C ABI of the B200 (sm_100a) fused scaled-dot-product attention
+ * library: forward and backward of
+ *
+ *     O = softmax(scale * Q K^T + bias, masked) V
+ *
+ * Definition: codelab "jax-gpu-05-attention-gpu", section 1 (how attention
+ * works: score, scale + softmax, weighted sum, output shaped like Q) and
+ * section 4 (the naive reference); Medium "Simplified Explanation of
+ * Attention ...", Steps 1-4 of "Scaled Dot Product Operation".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  Q, K, V, O, dO, dQ, dK, dV are bf16 tensors in (batch, sequence,
+ *   head, head_dim) order -- the (B, T, N, H) layout of the codelab, section
+ *   3 -- given by element strides; head_dim is contiguous.  Q, O, dO and dQ
+ *   share the strides sq_*, K, V, dK and dV share skv_*.  Query and key
+ *   sequences have the same length L.  LSE is float32 [B, Hq, L], contiguous.
+ * Heads.  Hq query heads share Hkv key/value heads in contiguous groups:
+ *   query head h reads KV head h / (Hq / Hkv) (MHA Hkv = Hq, GQA, MQA
+ *   Hkv = 1; codelab section 9).  Hq % Hkv must be 0.
+ * Supported.  head_dim d in {64, 128}; 1 <= L < 2^30; every bf16 base pointer
+ *   16-byte aligned; every stride a multiple of 8 elements (16 bytes) except
+ *   the contiguous head_dim.  Anything else returns SDPA_ERR_UNSUPPORTED or
+ *   SDPA_ERR_INVALID_ARG before any work is queued.
+ * Ownership.  The caller owns every buffer.  No entry point allocates,
+ *   frees, or synchronises the stream, except sdpa_read_device_status.
+ *   Outputs (O, LSE, dQ, dK, dV) are fully overwritten; no pre-zeroing.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream); work is queued on it and the call returns without waiting.
+ *   Device pointers must belong to the current CUDA device.
+ * Errors.  Argument errors are reported synchronously before any launch;
+ *   launch failures return SDPA_ERR_CUDA.  Waits inside the kernels are
+ *   bounded: a wait that runs out records SDPA_ERR_TIMEOUT in a per-device
+ *   status word (read with sdpa_read_device_status) and the kernel returns
+ *   instead of hanging.
+ * Determinism.  Results are bit-identical run to run for identical inputs
+ *   and launch configuration: every reduction is in a fixed order and no
+ *   floating-point atomics are used (HF transformers issue #31787,
+ *   "Transformer models are not deterministic when using Flash Attention 2",
+ *   is the problem this guards against).
+ */
+#ifndef SDPA_B200_SDPA_H
+#define SDPA_B200_SDPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sdpa_status_t {
+  SDPA_OK = 0,
+  SDPA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, stride or alignment  */
+  SDPA_ERR_UNSUPPORTED = 2,  /* valid but not built: e.g. head_dim 96        */
+  SDPA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small   */
+  SDPA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed           */
+  SDPA_ERR_TIMEOUT = 5       /* a bounded in-kernel wait ran out              */
+} sdpa_status_t;
+
+/*
+ * Mask specification -- replaces a dense mask tensor.  Key j is visible from
+ * query i iff
+ *     (!causal || j <= i) && (window_left < 0 || j >= i - window_left)
+ *                         && (window_right < 0 || j <= i + window_right).
+ * Causal masking: codelab section 7.  Causal sliding window (Mistral,
+ * window 4096): HF transformers issue #30461, "Slowdown in Training Speed Due
+ * to SDPA Mask Fix in Version 4.40.0", whose whole point is that handing this
+ * mask over as a dense tensor forfeits skipping fully masked key tiles.  The
+ * pages do not say whether the window bound is inclusive; here both bounds
+ * are inclusive and a negative bound means unbounded.
+ */
+typedef struct sdpa_mask_spec {
+  int32_t causal;
+  int64_t window_left;
+  int64_t window_right;
+} sdpa_mask_spec;
+
+typedef enum sdpa_bias_kind {
+  SDPA_BIAS_NONE = 0,
+  SDPA_BIAS_DENSE = 1, /* additive float32 bias[b, h, i, j]                  */
+  SDPA_BIAS_T5 = 2     /* additive table[bucket(j - i), h], bucketed in-kernel */
+} sdpa_bias_kind;
+
+/*
+ * Additive attention bias (catie-aq/flashT5 README: "Full attention biases"
+ * and "T5-like relative position encoding biases"; the 3 October 2024
+ * "fa2-rpe" item -- linear memory for the T5 bias).  The bias is added after
+ * the scale and is not itself scaled; it takes part in LSE.
+ *   DENSE: ptr -> float32 with element strides stride_b, stride_h, stride_i
+ *          (j contiguous; 0 broadcasts over that index); ptr 16-byte aligned,
+ *          stride_i a multiple of 4.  A value of -inf masks (i, j); a row
+ *          with no visible key yields O = 0, LSE = -inf, zero gradients.
+ *   T5:    ptr -> float32 table[num_buckets][Hq] (row-major), bucket of the
+ *          signed distance j - i by the T5 closed form (Raffel et al. 2020):
+ *          bidirectional splits the buckets by sign; 2 <= num_buckets <= 128,
+ *          num_buckets even when bidirectional, max_distance >= num_buckets/2
+ *          (bidirectional: /4).  Nothing L x L is materialised.
+ */
+typedef struct sdpa_bias_desc {
+  int32_t kind; /* sdpa_bias_kind */
+  const float* ptr;
+  int64_t stride_b, stride_h, stride_i;
+  int32_t num_buckets, max_distance, bidirectional;
+} sdpa_bias_desc;
+
+typedef struct sdpa_shape {
+  int64_t B, L, Hq, Hkv, d;
+  int64_t sq_b, sq_l, sq_h;    /* element strides of Q, O, dO, dQ */
+  int64_t skv_b, skv_l, skv_h; /* element strides of K, V, dK, dV */
+} sdpa_shape;
+
+/*
+ * Forward.  Writes O (bf16, Q's layout) and LSE[b, h, i] = natural-log
+ * log-sum-exp of score row i (float32, -inf for a row with no visible key).
+ * bias may be NULL (= no bias); mask may not be NULL.  Fully masked key
+ * tiles are never loaded.
+ */
+sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k,
+                       const void* v, const sdpa_bias_desc* bias,
+                       const sdpa_mask_spec* mask, float scale, void* o,
+                       float* lse, void* stream);
+
+/*
+ * Bytes of device workspace sdpa_bwd needs for this shape (the per-row
+ * D_i = sum_c dO[i,c] O[i,c] vector, float32 [B, Hq, L], plus alignment).
+ * Returns 0 for an invalid shape.
+ */
+size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic);
+
+/*
+ * Backward.  Given Q, K, V, the forward output O and its LSE, and the
+ * output gradient dO (Q's layout), writes dQ (Q's layout), dK and dV (K's
+ * layout, summed over the query heads that share each KV head).  The pages
+ * print no gradient formulas; these are the chain rule of the forward:
+ *   P = exp(S - LSE), dP = dO V^T, D_i = rowsum(dO * O), dS = P (dP - D),
+ *   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+ * deterministic: must be 1 (the only mode built; 0 returns UNSUPPORTED).
+ * workspace: device memory of at least sdpa_bwd_workspace_size() bytes,
+ * 256-byte aligned, owned by the caller, contents ignored on entry.
+ */
+sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k,
+                       const void* v, const void* o, const void* dout,
+                       const float* lse, const sdpa_bias_desc* bias,
+                       const sdpa_mask_spec* mask, float scale, void* dq,
+                       void* dk, void* dv, int32_t deterministic,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * T5 bucket ids of n signed distances rel[i] = key_pos - query_pos, computed
+ * by the same device function the kernels use (device pointers, int32).
+ * Exported so the bucketing can be checked bit-exactly on its own.
+ */
+sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n,
+                             int32_t num_buckets, int32_t max_distance,
+                             int32_t bidirectional, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the sticky device status of
+ * the current device: SDPA_OK, or SDPA_ERR_TIMEOUT if any kernel's bounded
+ * wait ran out since the last call (SDPA_ERR_CUDA if the reads fail).
+ */
+sdpa_status_t sdpa_read_device_status(void* stream);
+
+/*
+ * Sets the time limit of every bounded in-kernel wait, in nanoseconds
+ * (default 2e9; values below 1000 are raised to 1000).  Host-side setting,
+ * read at each launch.
+ */
+void sdpa_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Launches one CTA that waits on a barrier nothing ever completes, under the
+ * current wait limit, so the timeout path can be exercised without faulting
+ * or hanging the GPU.  Expect sdpa_read_device_status() == SDPA_ERR_TIMEOUT
+ * afterwards.
+ */
+sdpa_status_t sdpa_debug_wait_timeout(void* stream);
+
+/* Static English text for a status code. */
+const char* sdpa_status_string(sdpa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_SDPA_H */

@@ -1,0 +1,235 @@
+"""ctypes binding of the C ABI in include/sdpa.h (argument marshalling only).
+
+Every function here converts torch tensors into pointers, sizes and strides,
+calls the entry point of the same name in libsdpa_b200.so on the current CUDA
+stream, and turns a non-OK status into an exception.  All arithmetic runs in
+the library's kernels; there is no fallback: if the library is missing or
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsdpa_b200.so")
+
+SDPA_OK = 0
+STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
+                3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
+BIAS_NONE, BIAS_DENSE, BIAS_T5 = 0, 1, 2
+
+EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
+            "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
+            "sdpa_status_string")
+
+
+class SdpaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class MaskSpec(ctypes.Structure):
+    _fields_ = [("causal", ctypes.c_int32), ("window_left", ctypes.c_int64),
+                ("window_right", ctypes.c_int64)]
+
+
+class BiasDesc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("ptr", ctypes.c_void_p),
+                ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64),
+                ("stride_i", ctypes.c_int64), ("num_buckets", ctypes.c_int32),
+                ("max_distance", ctypes.c_int32), ("bidirectional", ctypes.c_int32)]
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("B", "L", "Hq", "Hkv", "d", "sq_b", "sq_l", "sq_h", "skv_b", "skv_l", "skv_h")]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libsdpa_b200.so once and declare the signatures.  Raises if absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"CUDA library not built: {p} (run scaled_dot_product_bwd_b200.build)")
+    lib = ctypes.CDLL(p)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    sp, bp, mp = ctypes.POINTER(Shape), ctypes.POINTER(BiasDesc), ctypes.POINTER(MaskSpec)
+    lib.sdpa_fwd.argtypes = [sp, vp, vp, vp, bp, mp, f32, vp, vp, vp]
+    lib.sdpa_fwd.restype = i32
+    lib.sdpa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, i32, vp, sz, vp]
+    lib.sdpa_bwd.restype = i32
+    lib.sdpa_bwd_workspace_size.argtypes = [sp, i32]
+    lib.sdpa_bwd_workspace_size.restype = sz
+    lib.sdpa_t5_bucket.argtypes = [vp, vp, i64, i32, i32, i32, vp]
+    lib.sdpa_t5_bucket.restype = i32
+    lib.sdpa_read_device_status.argtypes = [vp]
+    lib.sdpa_read_device_status.restype = i32
+    lib.sdpa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.sdpa_set_wait_limit_ns.restype = None
+    lib.sdpa_debug_wait_timeout.argtypes = [vp]
+    lib.sdpa_debug_wait_timeout.restype = i32
+    lib.sdpa_status_string.argtypes = [i32]
+    lib.sdpa_status_string.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != SDPA_OK:
+        raise SdpaError(status, where)
+
+
+def _stream(t: torch.Tensor | None = None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor) -> Shape:
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, L, H, d]")
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape[0] != B or k.shape[1] != L or k.shape[3] != d:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    if q.stride(-1) != 1 or k.stride(-1) != 1:
+        raise ValueError("head_dim must be contiguous")
+    return Shape(B, L, Hq, Hkv, d, q.stride(0), q.stride(1), q.stride(2),
+                 k.stride(0), k.stride(1), k.stride(2))
+
+
+def make_mask(causal: bool, window_left: int, window_right: int) -> MaskSpec:
+    return MaskSpec(1 if causal else 0, int(window_left), int(window_right))
+
+
+def make_bias(bias: torch.Tensor | None, t5_table: torch.Tensor | None, num_buckets: int,
+              max_distance: int, bidirectional: bool) -> BiasDesc:
+    if bias is not None and t5_table is not None:
+        raise ValueError("give either a dense bias or a T5 table, not both")
+    if bias is not None:
+        if bias.dtype != torch.float32 or bias.dim() != 4 or bias.stride(-1) != 1:
+            raise ValueError("dense bias must be float32 [B|1, H|1, L, L] with j contiguous")
+        sb = bias.stride(0) if bias.shape[0] > 1 else 0
+        sh = bias.stride(1) if bias.shape[1] > 1 else 0
+        return BiasDesc(BIAS_DENSE, bias.data_ptr(), sb, sh, bias.stride(2), 0, 0, 0)
+    if t5_table is not None:
+        if t5_table.dtype != torch.float32 or not t5_table.is_contiguous():
+            raise ValueError("T5 table must be contiguous float32 [num_buckets, Hq]")
+        if t5_table.shape[0] != num_buckets:
+            raise ValueError("T5 table rows must equal num_buckets")
+        return BiasDesc(BIAS_T5, t5_table.data_ptr(), 0, 0, 0, int(num_buckets),
+                        int(max_distance), 1 if bidirectional else 0)
+    return BiasDesc(BIAS_NONE, None, 0, 0, 0, 0, 0, 0)
+
+
+def _same_layout(a: torch.Tensor, ref: torch.Tensor, name: str):
+    if a.shape != ref.shape or a.stride() != ref.stride() or a.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bf16 with the shape and strides of its partner")
+
+
+def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=None,
+             t5_table=None, t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
+             scale=None, out=None, lse=None):
+    """O, LSE = attention forward (see sdpa_fwd in include/sdpa.h)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise ValueError(f"{n} must be a bf16 CUDA tensor")
+    shape = make_shape(q, k)
+    _same_layout(v, k, "v")
+    B, L, Hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _same_layout(out, q, "out")
+    if lse is None:
+        lse = torch.empty(B, Hq, L, device=q.device, dtype=torch.float32)
+    if lse.shape != (B, Hq, L) or not lse.is_contiguous() or lse.dtype != torch.float32:
+        raise ValueError("lse must be contiguous float32 [B, Hq, L]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bd),
+                      ctypes.byref(m), sc, _ptr(out), _ptr(lse), _stream(q))
+    _check(st, "sdpa_fwd")
+    return out, lse
+
+
+def sdpa_bwd_workspace_size(q, k, deterministic: bool = True) -> int:
+    lib = load_library()
+    shape = make_shape(q, k)
+    return int(lib.sdpa_bwd_workspace_size(ctypes.byref(shape), 1 if deterministic else 0))
+
+
+def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
+             bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
+             t5_bidirectional=True, scale=None, dq=None, dk=None, dv=None, workspace=None,
+             deterministic=True):
+    """dQ, dK, dV = attention backward (see sdpa_bwd in include/sdpa.h)."""
+    lib = load_library()
+    shape = make_shape(q, k)
+    _same_layout(v, k, "v")
+    _same_layout(o, q, "o")
+    _same_layout(do, q, "do")
+    d = q.shape[-1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _same_layout(dq, q, "dq")
+    _same_layout(dk, k, "dk")
+    _same_layout(dv, k, "dv")
+    need = int(lib.sdpa_bwd_workspace_size(ctypes.byref(shape), 1))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
+                      _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk),
+                      _ptr(dv), 1 if deterministic else 0, _ptr(workspace),
+                      workspace.numel() * workspace.element_size(), _stream(q))
+    _check(st, "sdpa_bwd")
+    return dq, dk, dv
+
+
+def sdpa_t5_bucket(rel: torch.Tensor, num_buckets=32, max_distance=128, bidirectional=True):
+    """Bucket ids of int32 signed distances (device tensor) by the kernels' own function."""
+    lib = load_library()
+    if rel.dtype != torch.int32 or not rel.is_cuda or not rel.is_contiguous():
+        raise ValueError("rel must be a contiguous int32 CUDA tensor")
+    out = torch.empty_like(rel)
+    st = lib.sdpa_t5_bucket(_ptr(rel), _ptr(out), rel.numel(), int(num_buckets),
+                            int(max_distance), 1 if bidirectional else 0, _stream(rel))
+    _check(st, "sdpa_t5_bucket")
+    return out
+
+
+def sdpa_read_device_status() -> int:
+    """Synchronise the current stream; return (and clear) the device status code."""
+    return int(load_library().sdpa_read_device_status(_stream()))
+
+
+def sdpa_set_wait_limit_ns(ns: int):
+    load_library().sdpa_set_wait_limit_ns(int(ns))
+
+
+def sdpa_debug_wait_timeout():
+    _check(load_library().sdpa_debug_wait_timeout(_stream()), "sdpa_debug_wait_timeout")
+
+
+def sdpa_status_string(status: int) -> str:
+    return load_library().sdpa_status_string(int(status)).decode()

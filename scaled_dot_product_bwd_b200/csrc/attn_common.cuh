@@ -1,0 +1,138 @@
+// attn_common.cuh -- kernel parameters, mask-band arithmetic and the T5
+// relative-position bucket function shared by the forward and backward
+// kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace sdpa {
+
+constexpr int kTile = 128;             // query rows and keys per tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxT5Thresholds = 64;
+
+enum BiasKind : int { kBiasNone = 0, kBiasDense = 1, kBiasT5 = 2 };
+
+// T5 bucketing with the log boundaries precomputed on the host (in float64,
+// the precision the closed form is evaluated in) as integer thresholds:
+// distance n >= max_exact falls in bucket max_exact - 1 + #{k : n >= thr[k]},
+// capped at half - 1.  `half` is num_buckets / 2 when bidirectional (then
+// keys after the query, rel > 0, are offset by `half`), else num_buckets.
+struct T5Spec {
+  int half;
+  int max_exact;
+  int nthr;
+  int bidirectional;
+  int thr[kMaxT5Thresholds];
+};
+
+__host__ __device__ __forceinline__ int t5_bucket(int rel, const T5Spec& s) {
+  int n, off = 0;
+  if (s.bidirectional) {
+    n = rel < 0 ? -rel : rel;
+    off = rel > 0 ? s.half : 0;
+  } else {
+    n = rel < 0 ? -rel : 0;
+  }
+  int b;
+  if (n < s.max_exact) {
+    b = n;
+  } else {
+    b = s.max_exact - 1;
+    for (int k = 0; k < s.nthr; ++k) b += (n >= s.thr[k]) ? 1 : 0;
+    b = b < s.half - 1 ? b : s.half - 1;
+  }
+  return b + off;
+}
+
+struct AttnParams {
+  int B, L, Hq, Hkv, G;
+  int causal, wl, wr;          // wl / wr < 0: unbounded
+  float scale;                 // softmax scale
+  float scale_log2;            // scale * log2(e)
+  int64_t sq_b, sq_l, sq_h;    // element strides: Q, O, dO, dQ
+  int64_t skv_b, skv_l, skv_h; // element strides: K, V, dK, dV
+  // forward outputs / backward inputs
+  __nv_bfloat16* o;
+  float* lse;                  // [B, Hq, L]
+  // backward
+  const __nv_bfloat16* dout;
+  float* dvec;                 // D = rowsum(dO * O), [B, Hq, L]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  // bias
+  int bias_kind;
+  const float* bias;           // dense
+  int64_t sb_b, sb_h, sb_i;
+  const float* t5_table;       // [num_buckets, Hq]
+  T5Spec t5;
+  uint64_t wait_limit_ns;
+};
+
+// Key tiles [nlo, nhi) that hold any key visible from query rows
+// [m0, m0 + rows) (clipped to L).  Empty when nhi <= nlo.
+__device__ __forceinline__ void key_tile_range(const AttnParams& p, int m0, int rows, int& nlo,
+                                               int& nhi) {
+  const int m_last = min(m0 + rows - 1, p.L - 1);
+  int jmin = 0;
+  if (p.wl >= 0) jmin = max(0, m0 - p.wl);
+  int jmax = p.L - 1;
+  if (p.causal) jmax = min(jmax, m_last);
+  if (p.wr >= 0) jmax = min(jmax, m_last + p.wr);
+  nlo = jmin / kTile;
+  nhi = (jmax >= jmin) ? jmax / kTile + 1 : nlo;
+}
+
+// Query tiles [mlo, mhi) holding any query that sees a key in
+// [n0, n0 + kTile) (clipped to L).
+__device__ __forceinline__ void query_tile_range(const AttnParams& p, int n0, int& mlo, int& mhi) {
+  const int n_last = min(n0 + kTile - 1, p.L - 1);
+  int imin = 0;
+  if (p.causal) imin = n0;
+  if (p.wr >= 0) imin = max(imin, n0 - p.wr);
+  int imax = p.L - 1;
+  if (p.wl >= 0) imax = min(imax, n_last + p.wl);
+  mlo = imin / kTile;
+  mhi = (imax >= imin) ? imax / kTile + 1 : mlo;
+}
+
+// True when every (query, key) pair of the tile (rows m0.., keys n0..) is
+// visible and in range, so no element needs masking.  `rows_in_range`
+// additionally requires every query row < L.
+__device__ __forceinline__ bool tile_is_full(const AttnParams& p, int m0, int n0,
+                                             bool rows_in_range) {
+  if (n0 + kTile > p.L) return false;
+  if (rows_in_range && m0 + kTile > p.L) return false;
+  if (p.causal && n0 + kTile - 1 > m0) return false;
+  if (p.wl >= 0 && n0 < m0 + kTile - 1 - p.wl) return false;
+  if (p.wr >= 0 && n0 + kTile - 1 > m0 + p.wr) return false;
+  return true;
+}
+
+// For query row i and a key tile starting at n0: the visible tile columns
+// are [lo, hi] (possibly empty).
+__device__ __forceinline__ void row_visible_cols(const AttnParams& p, int i, int n0, int& lo,
+                                                 int& hi) {
+  lo = 0;
+  if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
+  hi = min(kTile - 1, p.L - 1 - n0);
+  if (p.causal) hi = min(hi, i - n0);
+  if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
+}
+
+// For key j and a query tile starting at m0: the query columns that see j
+// are [lo, hi] (possibly empty).
+__device__ __forceinline__ void key_visible_rows(const AttnParams& p, int j, int m0, int& lo,
+                                                 int& hi) {
+  lo = 0;
+  if (p.causal) lo = max(lo, j - m0);
+  if (p.wr >= 0) lo = max(lo, j - p.wr - m0);
+  hi = min(kTile - 1, p.L - 1 - m0);
+  if (p.wl >= 0) hi = min(hi, j + p.wl - m0);
+}
+
+}  // namespace sdpa

@@ -1,0 +1,307 @@
+// sdpa_api.cu -- host side of the C ABI declared in include/sdpa.h:
+// argument validation (before anything is queued), TMA tensor maps,
+// T5 bucket thresholds, kernel launches, and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "sdpa.h"
+#include "attn_common.cuh"
+#include "bwd_kernels.cuh"
+#include "fwd_kernel.cuh"
+
+using namespace sdpa;
+
+namespace {
+
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 4-D map over a (batch, seq, head, head_dim) bf16 tensor, box = 64 head-dim
+// elements x 128 rows of one head of one batch, 128-byte swizzle.  Rows past
+// the sequence end read as zero.
+bool make_bshd_map(CUtensorMap* m, const void* base, int64_t B, int64_t L, int64_t H, int64_t D,
+                   int64_t s_b, int64_t s_l, int64_t s_h) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_l) * 2, static_cast<cuuint64_t>(s_h) * 2,
+                           static_cast<cuuint64_t>(s_b) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kTile), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Integer thresholds of the T5 log buckets, evaluated in float64 exactly as
+// the closed form reads: large(n) = max_exact + trunc(ln(n / max_exact) /
+// ln(max_distance / max_exact) * (half - max_exact)).
+bool fill_t5(T5Spec& t, int nb, int md, int bidir) {
+  const int half = bidir ? nb / 2 : nb;
+  const int me = half / 2;
+  if (me < 1 || md <= me) return false;
+  const int K = half - me;
+  if (K > kMaxT5Thresholds) return false;
+  t.half = half;
+  t.max_exact = me;
+  t.bidirectional = bidir ? 1 : 0;
+  t.nthr = K;
+  const double denom = std::log(static_cast<double>(md) / static_cast<double>(me));
+  auto large = [&](int64_t n) -> int64_t {
+    const double v = std::log(static_cast<double>(n) / static_cast<double>(me)) / denom *
+                     static_cast<double>(half - me);
+    return me + static_cast<int64_t>(v);
+  };
+  const int64_t limit = 4 * static_cast<int64_t>(md) + 1024;
+  int64_t n = me;
+  for (int k = 0; k < K; ++k) {
+    while (n < limit && large(n) < me + k) ++n;
+    t.thr[k] = (n < limit) ? static_cast<int>(n) : INT_MAX;
+  }
+  for (int k = K; k < kMaxT5Thresholds; ++k) t.thr[k] = INT_MAX;
+  return true;
+}
+
+int clamp_window(int64_t w, int64_t L) {
+  if (w < 0) return -1;
+  return static_cast<int>(w > L ? L : w);
+}
+
+// Shared validation of shape / mask / bias; fills the common fields of p.
+sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
+                      float scale, AttnParams& p) {
+  if (!s || !mask) return SDPA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->L < 1 || s->Hq < 1 || s->Hkv < 1) return SDPA_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return SDPA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return SDPA_ERR_UNSUPPORTED;
+  if (s->L >= (1ll << 30) || s->B > 65535 || s->Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  const int64_t st[6] = {s->sq_b, s->sq_l, s->sq_h, s->skv_b, s->skv_l, s->skv_h};
+  for (int64_t v : st)
+    if (v <= 0 || (v % 8) != 0 || v >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
+  std::memset(&p, 0, sizeof(p));
+  p.B = static_cast<int>(s->B);
+  p.L = static_cast<int>(s->L);
+  p.Hq = static_cast<int>(s->Hq);
+  p.Hkv = static_cast<int>(s->Hkv);
+  p.G = p.Hq / p.Hkv;
+  p.causal = mask->causal ? 1 : 0;
+  p.wl = clamp_window(mask->window_left, s->L);
+  p.wr = clamp_window(mask->window_right, s->L);
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.sq_b = s->sq_b;
+  p.sq_l = s->sq_l;
+  p.sq_h = s->sq_h;
+  p.skv_b = s->skv_b;
+  p.skv_l = s->skv_l;
+  p.skv_h = s->skv_h;
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.bias_kind = kBiasNone;
+  if (bias && bias->kind != SDPA_BIAS_NONE) {
+    if (bias->kind == SDPA_BIAS_DENSE) {
+      if (!bias->ptr || !aligned16(bias->ptr)) return SDPA_ERR_INVALID_ARG;
+      if (bias->stride_b < 0 || bias->stride_h < 0 || bias->stride_i < 0) return SDPA_ERR_INVALID_ARG;
+      if (bias->stride_i % 4 != 0) return SDPA_ERR_INVALID_ARG;
+      p.bias_kind = kBiasDense;
+      p.bias = bias->ptr;
+      p.sb_b = bias->stride_b;
+      p.sb_h = bias->stride_h;
+      p.sb_i = bias->stride_i;
+    } else if (bias->kind == SDPA_BIAS_T5) {
+      if (!bias->ptr) return SDPA_ERR_INVALID_ARG;
+      const int nb = bias->num_buckets;
+      if (nb < 2 || nb > 128) return SDPA_ERR_INVALID_ARG;
+      if (bias->bidirectional && (nb % 2) != 0) return SDPA_ERR_INVALID_ARG;
+      if (!fill_t5(p.t5, nb, bias->max_distance, bias->bidirectional)) return SDPA_ERR_INVALID_ARG;
+      p.bias_kind = kBiasT5;
+      p.t5_table = bias->ptr;
+    } else {
+      return SDPA_ERR_INVALID_ARG;
+    }
+  }
+  return SDPA_OK;
+}
+
+template <int D, int NQ, int BIAS>
+cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
+                       const CUtensorMap& v, cudaStream_t st) {
+  using Lay = FwdLayout<D, NQ>;
+  auto kern = fwd_kernel<D, NQ, BIAS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Lay::kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  const int rows = kTile * NQ;
+  dim3 grid((p.L + rows - 1) / rows, p.Hq, p.B);
+  kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v);
+  return cudaGetLastError();
+}
+
+template <int D, int NQ>
+cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
+                              const CUtensorMap& v, cudaStream_t st) {
+  switch (p.bias_kind) {
+    case kBiasDense: return launch_fwd<D, NQ, kBiasDense>(p, q, k, v, st);
+    case kBiasT5: return launch_fwd<D, NQ, kBiasT5>(p, q, k, v, st);
+    default: return launch_fwd<D, NQ, kBiasNone>(p, q, k, v, st);
+  }
+}
+
+__global__ void t5_bucket_kernel(const int32_t* rel, int32_t* out, int64_t n, T5Spec spec) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = t5_bucket(rel[i], spec);
+}
+
+// One barrier that nothing ever completes, waited on under the wait limit.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_storage), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl ctl{&abort_flag, limit_ns};
+    (void)mbar_wait(smem_u32(&bar_storage), 0, ctl);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sdpa_status_string(sdpa_status_t s) {
+  switch (s) {
+    case SDPA_OK: return "ok";
+    case SDPA_ERR_INVALID_ARG: return "invalid argument";
+    case SDPA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SDPA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SDPA_ERR_CUDA: return "CUDA error";
+    case SDPA_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+void sdpa_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns < 1000 ? 1000 : ns; }
+
+sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
+                       const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
+                       void* o, float* lse, void* stream) {
+  AttnParams p;
+  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  if (st != SDPA_OK) return st;
+  if (!q || !k || !v || !o || !lse) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return SDPA_ERR_INVALID_ARG;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  CUtensorMap mq, mk, mv;
+  const sdpa_shape& s = *shape;
+  if (!make_bshd_map(&mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h) ||
+      !make_bshd_map(&mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
+      !make_bshd_map(&mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h))
+    return SDPA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128, 2>(p, mq, mk, mv, cs)
+                               : dispatch_fwd_bias<64, 2>(p, mq, mk, mv, cs);
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic) {
+  (void)deterministic;
+  if (!shape || shape->B < 1 || shape->Hq < 1 || shape->L < 1) return 0;
+  const size_t rows = static_cast<size_t>(shape->B) * shape->Hq * shape->L;
+  return ((rows * sizeof(float) + 255) / 256) * 256;
+}
+
+sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse,
+                       const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
+                       void* dq, void* dk, void* dv, int32_t deterministic, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  AttnParams p;
+  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  if (st != SDPA_OK) return st;
+  if (deterministic != 1) return SDPA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return SDPA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sdpa_bwd_workspace_size(shape, deterministic))
+    return SDPA_ERR_WORKSPACE;
+  p.o = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(o));
+  p.lse = const_cast<float*>(lse);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dvec = static_cast<float*>(workspace);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  const sdpa_shape& s = *shape;
+  BwdMaps maps;
+  if (!make_bshd_map(&maps.q, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h) ||
+      !make_bshd_map(&maps.k, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
+      !make_bshd_map(&maps.v, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
+      !make_bshd_map(&maps.dout, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h))
+    return SDPA_ERR_CUDA;
+  cudaError_t e = launch_bwd(p, maps, static_cast<int>(s.d), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n, int32_t num_buckets,
+                             int32_t max_distance, int32_t bidirectional, void* stream) {
+  if (n < 0 || (n > 0 && (!rel || !out))) return SDPA_ERR_INVALID_ARG;
+  if (num_buckets < 2 || num_buckets > 128 || (bidirectional && (num_buckets % 2) != 0))
+    return SDPA_ERR_INVALID_ARG;
+  T5Spec spec;
+  if (!fill_t5(spec, num_buckets, max_distance, bidirectional)) return SDPA_ERR_INVALID_ARG;
+  if (n == 0) return SDPA_OK;
+  const int64_t blocks = (n + 255) / 256;
+  t5_bucket_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0,
+                     static_cast<cudaStream_t>(stream)>>>(rel, out, n, spec);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status_t sdpa_read_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SDPA_ERR_CUDA;
+  unsigned int h = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(h)) != cudaSuccess) return SDPA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SDPA_ERR_CUDA;
+  return (h & kStatusTimeout) ? SDPA_ERR_TIMEOUT : SDPA_OK;
+}
+
+sdpa_status_t sdpa_debug_wait_timeout(void* stream) {
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_limit_ns);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+}  // extern "C"

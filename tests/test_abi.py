@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/sdpa.h declares, and rejects bad arguments before
+queuing any work (those calls return before touching CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from scaled_dot_product_bwd_b200 import binding
+from scaled_dot_product_bwd_b200.build import LIB_PATH, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdpa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sdpa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "sdpa_fwd" in names and "sdpa_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding.EXPORTED)
+
+
+def test_library_is_in_tree():
+    build()
+    assert os.path.dirname(LIB_PATH) == os.path.join(ROOT, "scaled_dot_product_bwd_b200")
+    assert os.path.exists(LIB_PATH)
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert binding.sdpa_status_string(code)
+    assert binding.sdpa_status_string(5) == "in-kernel wait timed out"
+
+
+def _shape(**kw):
+    base = dict(B=1, L=128, Hq=4, Hkv=2, d=64, sq_b=128 * 4 * 64, sq_l=4 * 64, sq_h=64,
+                skv_b=128 * 2 * 64, skv_l=2 * 64, skv_h=64)
+    base.update(kw)
+    return binding.Shape(*[base[n] for n, _ in binding.Shape._fields_])
+
+
+FAKE = ctypes.c_void_p(0x10000)   # aligned, never dereferenced: validation fails first
+
+
+def _fwd(lib, shape, mask=None, bias=None, scale=0.125, ptr=FAKE, lse=FAKE):
+    mask = mask or binding.MaskSpec(1, -1, -1)
+    return lib.sdpa_fwd(ctypes.byref(shape), ptr, ptr, ptr,
+                        ctypes.byref(bias) if bias is not None else None,
+                        ctypes.byref(mask), scale, ptr, lse, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(d=32), 2), (dict(Hq=3, Hkv=2), 1), (dict(L=0), 1),
+    (dict(B=0), 1), (dict(sq_l=4 * 64 + 4), 1), (dict(skv_h=0), 1), (dict(Hkv=0), 1),
+])
+def test_fwd_rejects_bad_shapes(lib, kw, code):
+    assert _fwd(lib, _shape(**kw)) == code
+
+
+def test_fwd_rejects_null_and_misaligned(lib):
+    assert _fwd(lib, _shape(), ptr=ctypes.c_void_p(0)) == 1
+    assert _fwd(lib, _shape(), ptr=ctypes.c_void_p(0x10008)) == 1
+    assert lib.sdpa_fwd(None, FAKE, FAKE, FAKE, None, None, 0.1, FAKE, FAKE, None) == 1
+    assert _fwd(lib, _shape(), scale=float("nan")) == 1
+
+
+def test_fwd_rejects_bad_bias(lib):
+    bad = [binding.BiasDesc(7, 0x10000, 0, 0, 0, 0, 0, 0),           # unknown kind
+           binding.BiasDesc(1, 0, 0, 0, 128, 0, 0, 0),               # dense, null
+           binding.BiasDesc(1, 0x10004, 0, 0, 128, 0, 0, 0),         # dense, misaligned
+           binding.BiasDesc(1, 0x10000, 0, 0, 130, 0, 0, 0),         # dense, stride_i % 4
+           binding.BiasDesc(2, 0x10000, 0, 0, 0, 31, 128, 1),        # T5, odd buckets (bidir)
+           binding.BiasDesc(2, 0x10000, 0, 0, 0, 256, 128, 1),       # T5, too many buckets
+           binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 8, 1),          # T5, max_distance <= max_exact
+           binding.BiasDesc(2, 0, 0, 0, 0, 32, 128, 1)]              # T5, null table
+    for b in bad:
+        assert _fwd(lib, _shape(), bias=b) == 1, (b.kind, b.num_buckets)
+
+
+def test_bwd_rejects_bad_args(lib):
+    s = _shape()
+    m = binding.MaskSpec(1, -1, -1)
+    ws = lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1)
+    assert ws >= 128 * 4 * 4 and ws % 256 == 0
+
+    def call(det=1, wsp=FAKE, wsb=ws, shape=s):
+        return lib.sdpa_bwd(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                            ctypes.byref(m), 0.125, FAKE, FAKE, FAKE, det, wsp, wsb, None)
+    assert call(det=0) == 2                               # only deterministic mode is built
+    assert call(wsp=ctypes.c_void_p(0)) == 3
+    assert call(wsp=ctypes.c_void_p(0x10010)) == 3        # not 256-byte aligned
+    assert call(wsb=ws - 1) == 3
+    assert call(shape=_shape(d=80)) == 2
+    assert lib.sdpa_bwd_workspace_size(None, 1) == 0
+
+
+def test_t5_bucket_rejects_bad_args(lib):
+    assert lib.sdpa_t5_bucket(FAKE, FAKE, -1, 32, 128, 1, None) == 1
+    assert lib.sdpa_t5_bucket(None, None, 5, 32, 128, 1, None) == 1
+    assert lib.sdpa_t5_bucket(FAKE, FAKE, 4, 33, 128, 1, None) == 1
+    assert lib.sdpa_t5_bucket(FAKE, FAKE, 0, 32, 128, 1, None) == 0   # nothing to do
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError):
+        binding.load_library(str(tmp_path / "missing.so"))

@@ -1,0 +1,84 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs, element by element, at sizes that span several tiles
+with ragged tails, plus the degenerate cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import assert_close, case_inputs, run_cuda, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # the small configuration of the benchmark table
+    "tiny_causal_d64": dict(B=1, Hq=2, Hkv=2, L=128, d=64, causal=True),
+    "ragged_gqa_causal_d128": dict(B=2, Hq=4, Hkv=2, L=300, d=128, causal=True),
+    "window_mqa_d128": dict(B=1, Hq=4, Hkv=1, L=520, d=128, causal=True, wl=130),
+    "window_two_sided_d64": dict(B=1, Hq=2, Hkv=2, L=333, d=64, wl=100, wr=50),
+    "bidirectional_d64": dict(B=2, Hq=2, Hkv=2, L=257, d=64),
+    "bidirectional_d128_gqa": dict(B=1, Hq=4, Hkv=2, L=390, d=128),
+    "t5_bias_d64": dict(B=2, Hq=4, Hkv=4, L=300, d=64, bias="t5"),
+    "t5_bias_causal_d128": dict(B=1, Hq=2, Hkv=1, L=270, d=128, causal=True, bias="t5"),
+    "dense_bias_causal_d128": dict(B=2, Hq=2, Hkv=1, L=200, d=128, causal=True, bias="dense"),
+    "dense_bias_d64": dict(B=1, Hq=3, Hkv=3, L=260, d=64, bias="dense"),
+    "dense_bias_broadcast_batch": dict(B=2, Hq=2, Hkv=2, L=144, d=64, bias="dense",
+                                       bias_shape=(1, 2, 144, 144)),
+    "single_token": dict(B=1, Hq=2, Hkv=1, L=1, d=64, causal=True),
+    "window_zero": dict(B=1, Hq=2, Hkv=2, L=200, d=128, causal=True, wl=0),
+    "window_ge_L": dict(B=1, Hq=2, Hkv=1, L=300, d=128, causal=True, wl=4096),
+    "short_ragged_d64": dict(B=3, Hq=2, Hkv=1, L=37, d=64, causal=True),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity_small(name):
+    c = CASES[name]
+    inp = case_inputs(c)
+    got = run_cuda(c, inp)
+    ref = run_oracle(c, inp)
+    assert_close(got, ref)
+
+
+def test_fully_masked_rows_by_dense_bias():
+    c = dict(B=1, Hq=2, Hkv=2, L=160, d=64, bias="dense")
+    inp = case_inputs(c)
+    inp.bias[:, :, 7, :] = -float("inf")
+    inp.bias[:, :, 150, :] = -float("inf")
+    got = run_cuda(c, inp)
+    ref = run_oracle(c, inp)
+    assert (got["o"][:, [7, 150]] == 0).all()
+    assert np.isneginf(got["lse"][:, :, [7, 150]]).all()
+    assert (got["dq"][:, [7, 150]] == 0).all()
+    assert_close(got, ref)
+
+
+def test_window_ge_L_equals_causal_bitwise():
+    c = dict(B=1, Hq=4, Hkv=2, L=384, d=128, causal=True)
+    inp = case_inputs(c)
+    a = run_cuda(c, inp)
+    b = run_cuda(dict(c, wl=384), inp)
+    for n in a:
+        assert np.array_equal(a[n], b[n]), n
+
+
+def test_causal_first_row_is_v0():
+    # codelab section 7: the first query attends only to itself.
+    c = dict(B=1, Hq=2, Hkv=1, L=256, d=128, causal=True)
+    inp = case_inputs(c)
+    got = run_cuda(c, inp, backward=False)
+    v0 = inp.v[:, 0, 0].float().numpy()
+    for h in range(2):
+        assert np.array_equal(got["o"][:, 0, h], v0)
+
+
+@pytest.mark.parametrize("name", ["ragged_gqa_causal_d128", "t5_bias_d64",
+                                  "dense_bias_causal_d128"])
+def test_bitwise_repeatable(name):
+    # HF transformers issue #31787: repeat and compare with torch.equal.
+    c = CASES[name]
+    inp = case_inputs(c)
+    first = run_cuda(c, inp)
+    for _ in range(3):
+        again = run_cuda(c, inp)
+        for n in first:
+            assert np.array_equal(first[n], again[n]), n
