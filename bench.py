@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark: effective attention TFLOP/s of one fused forward + backward step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is one sdpa_fwd + sdpa_bwd over one batch of seeded synthetic inputs
+already resident in HBM.  Effective FLOPs count only unmasked (query, key)
+pairs P per (batch, query head): forward 4 d P, backward 10 d P (the
+recompute of the scores included), 14 d P in total.  With N > 1 (torchrun)
+every rank runs its own batch (replicas; no collective on the data path) and
+rank 0 prints the whole-job rate: all ranks' FLOPs / the slowest rank's time.
+
+--impl reference times the float64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (one KV head group of one batch per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective attention TFLOP/s fwd+bwd (unmasked FLOPs) and % of B200 BF16 peak"
+
+CONFIGS = {
+    "mistral4k": dict(B=4, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1, bias="none"),
+    "mistral8k": dict(B=2, Hq=32, Hkv=8, L=8192, d=128, causal=True, wl=4096, wr=-1, bias="none"),
+    "t5rpe": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="t5"),
+    "t5dense": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="dense"),
+    "tiny": dict(B=1, Hq=2, Hkv=2, L=128, d=64, causal=True, wl=-1, wr=-1, bias="none"),
+}
+
+
+def describe(c):
+    mask = "causal" if c["causal"] else "bidirectional"
+    if c["wl"] >= 0:
+        mask += f" window_left={c['wl']}"
+    return (f"B={c['B']} Hq={c['Hq']} Hkv={c['Hkv']} L={c['L']} d={c['d']} {mask} "
+            f"bias={c['bias']}")
+
+
+def visible_pairs(L, causal, wl, wr):
+    """Unmasked (i, j) pairs of one head: sum over rows of the visible key span."""
+    i = np.arange(L, dtype=np.int64)
+    lo = np.maximum(0, i - wl) if wl >= 0 else np.zeros(L, np.int64)
+    hi = np.full(L, L - 1, np.int64)
+    if causal:
+        hi = np.minimum(hi, i)
+    if wr >= 0:
+        hi = np.minimum(hi, i + wr)
+    return int(np.maximum(0, hi - lo + 1).sum())
+
+
+def flop_counts(c):
+    P = visible_pairs(c["L"], c["causal"], c["wl"], c["wr"])
+    heads = c["B"] * c["Hq"]
+    d = c["d"]
+    return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads,
+                dkdv=8 * d * P * heads, dq=2 * d * P * heads)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(tflops=pk["bf16_tflops"], tflops_sustained=pk.get("bf16_tflops_sustained"),
+                    hbm=pk["hbm_gbs"], source="measured")
+    return dict(tflops=1590.0, tflops_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def make_case(c, seed):
+    from scaled_dot_product_bwd_b200.inputs import make_inputs
+    return make_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], c["d"], seed=seed,
+                       t5_buckets=32 if c["bias"] == "t5" else 0,
+                       dense_bias=c["bias"] == "dense")
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample(c, inp):
+    """fwd + bwd of the oracle on batch 0, KV head 0 (all its query heads)."""
+    from oracle import attention_backward, attention_forward
+    kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"],
+              bias=inp.bias, t5_table=inp.t5_table, batches=[0], kv_heads=[0])
+    attention_forward(inp.q, inp.k, inp.v, **kw)
+    attention_backward(inp.q, inp.k, inp.v, inp.do, **kw)
+
+
+def sample_inputs(c, seed):
+    """The sample's slice of the workload: batch 0, KV head 0 and its query heads."""
+    G = c["Hq"] // c["Hkv"]
+    sc = dict(c, B=1, Hq=G, Hkv=1)
+    return sc, make_case(sc, seed)
+
+
+def time_oracle(c, steps, warmup):
+    sc, inp = sample_inputs(c, 0)
+    flops = flop_counts(sc)
+    total = flops["fwd"] + flops["bwd"]
+    for _ in range(warmup):
+        oracle_sample(sc, inp)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_sample(sc, inp)
+    dt = (time.perf_counter() - t0) / steps
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"batch 0, KV head 0 with its {sc['Hq']} query heads of {describe(c)}; "
+              f"float64 numpy, explicit L x L matrices")
+    return dict(value=total / dt / 1e12, seconds_per_sample=dt, cores=cores, sample=sample,
+                flops=total)
+
+
+def run_reference(args, c):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    r = time_oracle(c, max(1, args.steps), args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": r["seconds_per_sample"] * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.config}: {describe(c)}", "sample": r["sample"]},
+        "cpu_baseline": {"value": r["value"], "unit": "TFLOP/s", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": r["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- GPU
+def run_gpu(args, c):
+    import torch
+    import torch.distributed as dist
+
+    from scaled_dot_product_bwd_b200 import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, load_library,
+                                             sdpa_bwd, sdpa_bwd_workspace_size, sdpa_fwd,
+                                             sdpa_read_device_status)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    load_library()
+
+    inp = make_case(c, seed=rank)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    bias = inp.bias.to(dev) if inp.bias is not None else None
+    table = inp.t5_table.to(dev) if inp.t5_table is not None else None
+    kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"], bias=bias,
+              t5_table=table)
+    o = torch.empty_like(q)
+    lse = torch.empty(c["B"], c["Hq"], c["L"], device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(sdpa_bwd_workspace_size(q, k), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sdpa_fwd(q, k, v, out=o, lse=lse, **kw)
+        if ev is not None:
+            ev[1].record(stream)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws,
+                 phases=BWD_PREPROCESS, **kw)
+        if ev is not None:
+            ev[2].record(stream)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DQ, **kw)
+        if ev is not None:
+            ev[3].record(stream)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DKDV, **kw)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if sdpa_read_device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait during warm-up")
+
+    # ---------------- timed region: K steps, device-timed, max over ranks
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.1)
+    start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(end)
+    phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(4)]
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = sdpa_read_device_status()
+
+    # ---------------- end to end: pinned host buffers, copies inside the timed region
+    hq_, hk_, hv_, hdo_ = (t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.do))
+    ho, hlse = torch.empty_like(hq_).pin_memory(), torch.empty(lse.shape).pin_memory()
+    hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq_, hk_, hv_))
+    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo_))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        do.copy_(hdo_, non_blocking=True)
+        sdpa_fwd(q, k, v, out=o, lse=lse, **kw)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+        for h, d_ in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+            h.copy_(d_, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    for _ in range(min(args.warmup, 2)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    fl = flop_counts(c)
+    step_flops = fl["fwd"] + fl["bwd"]
+    ms_step = ms_total / args.steps
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    peaks = load_peaks()
+
+    # dominant kernel by mean duration; its algorithmic FLOPs per launch
+    names = ["fwd", "bwd_preprocess", "bwd_dq", "bwd_dkdv"]
+    algo = {"fwd": fl["fwd"], "bwd_dq": fl["dq"], "bwd_dkdv": fl["dkdv"]}
+    dom = max(range(4), key=lambda i: phase_ms[i])
+    dname = names[dom]
+    roofline = None
+    if dname in algo:
+        ach = algo[dname] / (phase_ms[dom] * 1e-3) / 1e12
+        roofline = {"kernel": dname, "bound": "tensor", "achieved": round(ach, 1),
+                    "peak": peaks["tflops"], "unit": "TFLOP/s",
+                    "frac": round(ach / peaks["tflops"], 4), "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"
+                    if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
+                    "flops_per_launch": algo[dname], "ms_per_launch": round(phase_ms[dom], 4)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: {describe(c)}", "global_batch": c["B"] * world,
+                   "seq_len": c["L"], "parallelism": f"replicas x{world} (batch shards)",
+                   "l2": "inputs larger than L2: no flush between steps",
+                   "flops_per_step": step_flops, "unmasked_pairs_per_head": fl["P"]},
+        "pct_of_peak": round(100 * value / world / peaks["tflops"], 2),
+        "value_strict": round(world * (fl["fwd"] + fl["bwd_strict"]) / (ms_step * 1e-3) / 1e12, 2),
+        "kernel_ms": {n: round(t, 4) for n, t in zip(names, phase_ms)},
+        "roofline": roofline,
+        "e2e": {"value": round(world * step_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            r = time_oracle(c, 1, 0)
+            line["cpu_baseline"] = {"value": r["value"], "unit": "TFLOP/s", "cores": r["cores"],
+                                    "kind": "oracle", "sample": r["sample"]}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="mistral4k", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    c = CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, c)
+    return run_gpu(args, c)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -148,6 +148,26 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The backward as its three launches, selected by a bitmask: PREPROCESS
+ * writes D = rowsum(dO * O) into the workspace; DQ writes dQ; DKDV writes dK
+ * and dV.  DQ and DKDV read D from the workspace, so PREPROCESS must have run
+ * on the same workspace earlier in stream order; DQ and DKDV are independent
+ * of each other and may run on different streams.  sdpa_bwd is
+ * sdpa_bwd_phases(SDPA_BWD_ALL, ...).  Arguments as sdpa_bwd; phases == 0 or
+ * unknown bits -> SDPA_ERR_INVALID_ARG.
+ */
+#define SDPA_BWD_PREPROCESS 1u
+#define SDPA_BWD_DQ 2u
+#define SDPA_BWD_DKDV 4u
+#define SDPA_BWD_ALL 7u
+sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const void* q,
+                              const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, const sdpa_bias_desc* bias,
+                              const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                              void* dv, int32_t deterministic, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * T5 bucket ids of n signed distances rel[i] = key_pos - query_pos, computed
  * by the same device function the kernels use (device pointers, int32).
  * Exported so the bucketing can be checked bit-exactly on its own.

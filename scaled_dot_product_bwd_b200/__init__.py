@@ -6,6 +6,10 @@ The shared library is loaded on first use; importing the package does not
 touch the GPU.
 """
 from .binding import (  # noqa: F401
+    BWD_ALL,
+    BWD_DKDV,
+    BWD_DQ,
+    BWD_PREPROCESS,
     EXPORTED,
     SdpaError,
     load_library,

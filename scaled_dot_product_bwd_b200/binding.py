@@ -22,7 +22,9 @@ STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTE
                 3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 BIAS_NONE, BIAS_DENSE, BIAS_T5 = 0, 1, 2
 
-EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
+BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
+
+EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
             "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
             "sdpa_status_string")
 
@@ -69,6 +71,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_fwd.restype = i32
     lib.sdpa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, i32, vp, sz, vp]
     lib.sdpa_bwd.restype = i32
+    lib.sdpa_bwd_phases.argtypes = [ctypes.c_uint32] + lib.sdpa_bwd.argtypes
+    lib.sdpa_bwd_phases.restype = i32
     lib.sdpa_bwd_workspace_size.argtypes = [sp, i32]
     lib.sdpa_bwd_workspace_size.restype = sz
     lib.sdpa_t5_bucket.argtypes = [vp, vp, i64, i32, i32, i32, vp]
@@ -178,8 +182,13 @@ def sdpa_bwd_workspace_size(q, k, deterministic: bool = True) -> int:
 def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
              bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
              t5_bidirectional=True, scale=None, dq=None, dk=None, dv=None, workspace=None,
-             deterministic=True):
-    """dQ, dK, dV = attention backward (see sdpa_bwd in include/sdpa.h)."""
+             deterministic=True, phases=BWD_ALL):
+    """dQ, dK, dV = attention backward (see sdpa_bwd / sdpa_bwd_phases in include/sdpa.h).
+
+    ``phases`` selects launches (BWD_PREPROCESS | BWD_DQ | BWD_DKDV); the
+    default runs all three in order.  A partial call needs the workspace of
+    an earlier PREPROCESS call.
+    """
     lib = load_library()
     shape = make_shape(q, k)
     _same_layout(v, k, "v")
@@ -198,11 +207,14 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
     m = make_mask(causal, window_left, window_right)
-    st = lib.sdpa_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
-                      _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk),
-                      _ptr(dv), 1 if deterministic else 0, _ptr(workspace),
-                      workspace.numel() * workspace.element_size(), _stream(q))
-    _check(st, "sdpa_bwd")
+    args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+            ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk), _ptr(dv),
+            1 if deterministic else 0, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(q))
+    if phases == BWD_ALL:
+        _check(lib.sdpa_bwd(*args), "sdpa_bwd")
+    else:
+        _check(lib.sdpa_bwd_phases(int(phases), *args), "sdpa_bwd_phases")
     return dq, dk, dv
 
 

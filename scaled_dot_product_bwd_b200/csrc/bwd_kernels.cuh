@@ -651,9 +651,12 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ------------------------------------------------------------- launchers
+constexpr uint32_t kPhasePre = 1u, kPhaseDq = 2u, kPhaseDkdv = 4u;
+
 template <int D, int BIAS>
-cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, cudaStream_t st) {
-  {
+cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, uint32_t phases,
+                         cudaStream_t st) {
+  if (phases & kPhasePre) {
     const int64_t threads = static_cast<int64_t>(p.B) * p.L * p.Hq * (D / 8);
     const int64_t blocks = (threads + 255) / 256;
     bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p);
@@ -661,7 +664,7 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, cudaStream_t st)
     if (e != cudaSuccess) return e;
   }
   const int ntiles = (p.L + kTile - 1) / kTile;
-  {
+  if (phases & kPhaseDq) {
     auto kern = bwd_dq_kernel<D, BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DqLayout<D>::kSmemAlloc);
@@ -671,28 +674,32 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, cudaStream_t st)
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  {
+  if (phases & kPhaseDkdv) {
     auto kern = bwd_dkdv_kernel<D, BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DkdvLayout<D>::kSmemAlloc);
     if (e != cudaSuccess) return e;
     kern<<<dim3(ntiles, p.Hkv, p.B), DkdvLayout<D>::kThreads, DkdvLayout<D>::kSmemAlloc, st>>>(
         p, m.q, m.k, m.v, m.dout);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const AttnParams& p, const BwdMaps& m, cudaStream_t st) {
+cudaError_t launch_bwd_d(const AttnParams& p, const BwdMaps& m, uint32_t phases,
+                         cudaStream_t st) {
   switch (p.bias_kind) {
-    case kBiasDense: return launch_bwd_t<D, kBiasDense>(p, m, st);
-    case kBiasT5: return launch_bwd_t<D, kBiasT5>(p, m, st);
-    default: return launch_bwd_t<D, kBiasNone>(p, m, st);
+    case kBiasDense: return launch_bwd_t<D, kBiasDense>(p, m, phases, st);
+    case kBiasT5: return launch_bwd_t<D, kBiasT5>(p, m, phases, st);
+    default: return launch_bwd_t<D, kBiasNone>(p, m, phases, st);
   }
 }
 
-inline cudaError_t launch_bwd(const AttnParams& p, const BwdMaps& m, int d, cudaStream_t st) {
-  return d == 128 ? launch_bwd_d<128>(p, m, st) : launch_bwd_d<64>(p, m, st);
+inline cudaError_t launch_bwd(const AttnParams& p, const BwdMaps& m, int d, uint32_t phases,
+                              cudaStream_t st) {
+  return d == 128 ? launch_bwd_d<128>(p, m, phases, st) : launch_bwd_d<64>(p, m, phases, st);
 }
 
 }  // namespace sdpa

@@ -244,11 +244,13 @@ size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic) {
   return ((rows * sizeof(float) + 255) / 256) * 256;
 }
 
-sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
-                       const void* o, const void* dout, const float* lse,
-                       const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
-                       void* dq, void* dk, void* dv, int32_t deterministic, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const void* q,
+                              const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, const sdpa_bias_desc* bias,
+                              const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                              void* dv, int32_t deterministic, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (phases == 0 || (phases & ~SDPA_BWD_ALL) != 0) return SDPA_ERR_INVALID_ARG;
   AttnParams p;
   sdpa_status_t st = prepare(shape, bias, mask, scale, p);
   if (st != SDPA_OK) return st;
@@ -273,8 +275,18 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, co
       !make_bshd_map(&maps.v, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
       !make_bshd_map(&maps.dout, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h))
     return SDPA_ERR_CUDA;
-  cudaError_t e = launch_bwd(p, maps, static_cast<int>(s.d), static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_bwd(p, maps, static_cast<int>(s.d), phases, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
+                       const void* o, const void* dout, const float* lse,
+                       const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
+                       void* dq, void* dk, void* dv, int32_t deterministic, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return sdpa_bwd_phases(SDPA_BWD_ALL, shape, q, k, v, o, dout, lse, bias, mask, scale, dq, dk,
+                         dv, deterministic, workspace, workspace_bytes, stream);
 }
 
 sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n, int32_t num_buckets,
