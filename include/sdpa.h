@@ -168,6 +168,37 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
                               size_t workspace_bytes, void* stream);
 
 /*
+ * Backward without a caller-supplied workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory around the call: kernel hosts and plugin
+ * interfaces that hand a library only its input and output buffers and own
+ * every other byte of device memory through their own pool, processes held
+ * to a hard memory cap where a late allocation can fail mid-step, and
+ * latency-bound loops that avoid cudaMalloc / cudaFree because those calls
+ * can synchronise the device and stall other streams.
+ *
+ * Same arguments and results as sdpa_bwd minus the workspace: the D vector
+ * lives in a fixed array of SDPA_NOALLOC_MAX_ROWS floats (4 MiB) compiled
+ * into the library, held by every GPU that loads it until the process exits.
+ *  - B * Hq * L must be <= SDPA_NOALLOC_MAX_ROWS, else SDPA_ERR_WORKSPACE
+ *    (nothing is launched).
+ *  - The first call on a device looks up the array's device address with
+ *    that device current (once per device); make that first call before
+ *    any stream capture on the device.  A failed lookup -> SDPA_ERR_CUDA.
+ *  - Every call, on every stream of a device, shares the one array, which
+ *    keeps the contents of the last call (nothing in it needs to start at
+ *    zero: each call writes the rows it reads).  Calls whose executions
+ *    overlap on the GPU race on it; order them on one stream or with events.
+ *  - Calls no allocating routine (no cudaMalloc / cudaFree).
+ */
+#define SDPA_NOALLOC_MAX_ROWS (1u << 20)
+sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const void* k,
+                               const void* v, const void* o, const void* dout,
+                               const float* lse, const sdpa_bias_desc* bias,
+                               const sdpa_mask_spec* mask, float scale, void* dq,
+                               void* dk, void* dv, int32_t deterministic, void* stream);
+
+/*
  * T5 bucket ids of n signed distances rel[i] = key_pos - query_pos, computed
  * by the same device function the kernels use (device pointers, int32).
  * Exported so the bucketing can be checked bit-exactly on its own.

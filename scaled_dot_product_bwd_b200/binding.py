@@ -24,7 +24,10 @@ BIAS_NONE, BIAS_DENSE, BIAS_T5 = 0, 1, 2
 
 BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 
-EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
+NOALLOC_MAX_ROWS = 1 << 20
+
+EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_noalloc",
+            "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
             "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
             "sdpa_status_string")
 
@@ -73,6 +76,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_bwd.restype = i32
     lib.sdpa_bwd_phases.argtypes = [ctypes.c_uint32] + lib.sdpa_bwd.argtypes
     lib.sdpa_bwd_phases.restype = i32
+    lib.sdpa_bwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, i32, vp]
+    lib.sdpa_bwd_noalloc.restype = i32
     lib.sdpa_bwd_workspace_size.argtypes = [sp, i32]
     lib.sdpa_bwd_workspace_size.restype = sz
     lib.sdpa_t5_bucket.argtypes = [vp, vp, i64, i32, i32, i32, vp]
@@ -215,6 +220,30 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
         _check(lib.sdpa_bwd(*args), "sdpa_bwd")
     else:
         _check(lib.sdpa_bwd_phases(int(phases), *args), "sdpa_bwd_phases")
+    return dq, dk, dv
+
+
+def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_left=-1,
+                     window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
+                     t5_max_distance=128, t5_bidirectional=True, scale=None):
+    """Backward into caller-given dQ, dK, dV with no workspace and no allocation.
+
+    For callers that cannot allocate device memory: the library's built-in
+    scratch array (NOALLOC_MAX_ROWS rows of B * Hq * L) stands in for the
+    workspace.  Calls that overlap on the GPU race on that array.
+    """
+    lib = load_library()
+    shape = make_shape(q, k)
+    for t, ref, n in ((v, k, "v"), (o, q, "o"), (do, q, "do"), (dq, q, "dq"), (dk, k, "dk"),
+                      (dv, k, "dv")):
+        _same_layout(t, ref, n)
+    sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_bwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
+                              _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq),
+                              _ptr(dk), _ptr(dv), 1, _stream(q))
+    _check(st, "sdpa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -289,6 +289,48 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, co
                          dv, deterministic, workspace, workspace_bytes, stream);
 }
 
+// ---------------------------------------------------------------------
+// sdpa_bwd_noalloc: the backward's D-vector scratch in a fixed device array
+// instead of a caller workspace, for callers that cannot allocate device
+// memory (see include/sdpa.h).  In host code `g_noalloc_scratch` names a
+// host-side stand-in, not device memory, so the kernels are given the
+// device address looked up with cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) float g_noalloc_scratch[SDPA_NOALLOC_MAX_ROWS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, or nullptr.
+void* noalloc_scratch_ptr() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const void* k,
+                               const void* v, const void* o, const void* dout, const float* lse,
+                               const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
+                               float scale, void* dq, void* dk, void* dv, int32_t deterministic,
+                               void* stream) {
+  if (!shape || shape->B < 1 || shape->Hq < 1 || shape->L < 1) return SDPA_ERR_INVALID_ARG;
+  const uint64_t rows = static_cast<uint64_t>(shape->B) * static_cast<uint64_t>(shape->Hq) *
+                        static_cast<uint64_t>(shape->L);
+  if (rows > SDPA_NOALLOC_MAX_ROWS) return SDPA_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return SDPA_ERR_CUDA;
+  return sdpa_bwd_phases(SDPA_BWD_ALL, shape, q, k, v, o, dout, lse, bias, mask, scale, dq, dk,
+                         dv, deterministic, scratch, sizeof(g_noalloc_scratch), stream);
+}
+
 sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n, int32_t num_buckets,
                              int32_t max_distance, int32_t bidirectional, void* stream) {
   if (n < 0 || (n > 0 && (!rel || !out))) return SDPA_ERR_INVALID_ARG;

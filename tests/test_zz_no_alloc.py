@@ -1,0 +1,57 @@
+"""The allocation-free backward entry point, sdpa_bwd_noalloc, for callers
+that cannot allocate device memory around the call (kernel hosts that hand a
+library only its inputs and outputs, processes under a hard memory cap,
+latency-bound loops that avoid cudaMalloc / cudaFree).  Its D-vector scratch
+is a fixed array inside the library instead of a caller workspace; its
+results must match sdpa_bwd's, call after call.
+
+Kept in its own file, named to be collected last.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import ATOL, RTOL
+from scaled_dot_product_bwd_b200 import SdpaError, sdpa_bwd, sdpa_bwd_noalloc, sdpa_fwd
+from scaled_dot_product_bwd_b200.binding import NOALLOC_MAX_ROWS
+from scaled_dot_product_bwd_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(a, b):
+    a = a.float().cpu().numpy()
+    b = b.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= ATOL + RTOL * np.abs(b))
+
+
+@pytest.mark.parametrize("kw", [dict(causal=True), dict(causal=False, t5=True)])
+def test_noalloc_matches_workspace_entry_point_twice(kw):
+    dev = torch.device("cuda")
+    t5 = kw.pop("t5", False)
+    for call, seed in enumerate((1, 2)):   # two calls in a row, different inputs
+        inp = make_inputs(2, 300, 4, 2, 128, seed=seed, t5_buckets=32 if t5 else 0)
+        q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+        extra = dict(kw)
+        if t5:
+            extra["t5_table"] = inp.t5_table.to(dev)
+        o, lse = sdpa_fwd(q, k, v, **extra)
+        ref = sdpa_bwd(q, k, v, o, do, lse, **extra)
+        out = (torch.full_like(q, float("nan")), torch.full_like(k, float("nan")),
+               torch.full_like(v, float("nan")))
+        got = sdpa_bwd_noalloc(q, k, v, o, do, lse, *out, **extra)
+        torch.cuda.synchronize()
+        for g, r in zip(got, ref):
+            _close(g, r)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    dev = torch.device("cuda")
+    L = NOALLOC_MAX_ROWS // 2 + 8          # B * Hq * L > max with B = 1, Hq = 2
+    q = torch.zeros(1, L, 2, 64, device=dev, dtype=torch.bfloat16)
+    k = torch.zeros(1, L, 1, 64, device=dev, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, L, device=dev)
+    with pytest.raises(SdpaError) as e:
+        sdpa_bwd_noalloc(q, k, k, q, q, lse, torch.empty_like(q), torch.empty_like(k),
+                         torch.empty_like(k), causal=True)
+    assert e.value.status == 3             # SDPA_ERR_WORKSPACE: nothing launched
