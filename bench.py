@@ -185,6 +185,23 @@ def run_reference(args, c):
     return 0
 
 
+# ------------------------------------------------------- multi-rank plumbing
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's time: all_reduce(MAX) when a process group is up."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank runs its own batch; all ranks' FLOPs / slowest time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------- GPU
 def run_gpu(args, c):
     import torch
@@ -258,10 +275,7 @@ def run_gpu(args, c):
     clocks = sampler.stop()
     ms_total = start.elapsed_time(end)
     phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(4)]
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     status = sdpa_read_device_status()
 
     # ---------------- end to end: pinned host buffers, copies inside the timed region
@@ -294,15 +308,12 @@ def run_gpu(args, c):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
 
     fl = flop_counts(c)
     step_flops = fl["fwd"] + fl["bwd"]
     ms_step = ms_total / args.steps
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, ms_step)
     peaks = load_peaks()
 
     # dominant kernel by mean duration; its algorithmic FLOPs per launch
@@ -333,7 +344,7 @@ def run_gpu(args, c):
         "value_strict": round(world * (fl["fwd"] + fl["bwd_strict"]) / (ms_step * 1e-3) / 1e12, 2),
         "kernel_ms": {n: round(t, 4) for n, t in zip(names, phase_ms)},
         "roofline": roofline,
-        "e2e": {"value": round(world * step_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_tflops(world, step_flops, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": 4 * args.steps,

@@ -95,8 +95,9 @@ typedef enum sdpa_bias_kind {
  *   T5:    ptr -> float32 table[num_buckets][Hq] (row-major), bucket of the
  *          signed distance j - i by the T5 closed form (Raffel et al. 2020):
  *          bidirectional splits the buckets by sign; 2 <= num_buckets <= 128,
- *          num_buckets even when bidirectional, max_distance >= num_buckets/2
- *          (bidirectional: /4).  Nothing L x L is materialised.
+ *          num_buckets even when bidirectional, max_distance > max_exact
+ *          (num_buckets/4 when bidirectional, num_buckets/2 otherwise).
+ *          Nothing L x L is materialised.
  */
 typedef struct sdpa_bias_desc {
   int32_t kind; /* sdpa_bias_kind */
