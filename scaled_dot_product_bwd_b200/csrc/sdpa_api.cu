@@ -40,17 +40,17 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a (batch, seq, head, head_dim) bf16 tensor, box = 64 head-dim
-// elements x 128 rows of one head of one batch, 128-byte swizzle.  Rows past
-// the sequence end read as zero.
+// elements x `rows` rows of one head of one batch, 128-byte swizzle.  Rows
+// past the sequence end read as zero.
 bool make_bshd_map(CUtensorMap* m, const void* base, int64_t B, int64_t L, int64_t H, int64_t D,
-                   int64_t s_b, int64_t s_l, int64_t s_h) {
+                   int64_t s_b, int64_t s_l, int64_t s_h, int rows = kTile) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                         static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_l) * 2, static_cast<cuuint64_t>(s_h) * 2,
                            static_cast<cuuint64_t>(s_b) * 2};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kTile), 1, 1};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -270,11 +270,18 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
   p.dv = static_cast<__nv_bfloat16*>(dv);
   const sdpa_shape& s = *shape;
   BwdMaps maps;
-  if (!make_bshd_map(&maps.q, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h) ||
-      !make_bshd_map(&maps.k, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
-      !make_bshd_map(&maps.v, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
-      !make_bshd_map(&maps.dout, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h))
-    return SDPA_ERR_CUDA;
+  bool ok = true;
+  for (int rows : {kTile, kBlk}) {
+    CUtensorMap* mq = rows == kTile ? &maps.q128 : &maps.q64;
+    CUtensorMap* mdo = rows == kTile ? &maps.dout128 : &maps.dout64;
+    CUtensorMap* mk = rows == kTile ? &maps.k128 : &maps.k64;
+    CUtensorMap* mv = rows == kTile ? &maps.v128 : &maps.v64;
+    ok = ok && make_bshd_map(mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
+         make_bshd_map(mdo, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
+         make_bshd_map(mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows) &&
+         make_bshd_map(mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows);
+  }
+  if (!ok) return SDPA_ERR_CUDA;
   cudaError_t e =
       launch_bwd(p, maps, static_cast<int>(s.d), phases, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
