@@ -209,9 +209,19 @@ sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n,
                              int32_t bidirectional, void* stream);
 
 /*
+ * y[i] = 2^x[i] by the kernels' FMA-pipe exponential (Cody-Waite reduction
+ * and a fitted cubic; relative error below 1.2e-4 for -125 <= x <= 125),
+ * device pointers, float32.  Exported so the approximation can be checked
+ * against exp2 on its own.
+ */
+sdpa_status_t sdpa_exp2_fma(const float* x, float* y, int64_t n, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the sticky device status of
- * the current device: SDPA_OK, or SDPA_ERR_TIMEOUT if any kernel's bounded
- * wait ran out since the last call (SDPA_ERR_CUDA if the reads fail).
+ * the current device: SDPA_OK; SDPA_ERR_TIMEOUT if any kernel's bounded wait
+ * ran out since the last call; SDPA_ERR_UNSUPPORTED if a kernel found its
+ * shared memory not 1024-byte aligned and returned without computing;
+ * SDPA_ERR_CUDA if the reads fail.
  */
 sdpa_status_t sdpa_read_device_status(void* stream);
 

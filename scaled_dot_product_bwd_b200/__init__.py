@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     sdpa_bwd_noalloc,
     sdpa_bwd_workspace_size,
     sdpa_debug_wait_timeout,
+    sdpa_exp2_fma,
     sdpa_fwd,
     sdpa_read_device_status,
     sdpa_set_wait_limit_ns,

@@ -27,7 +27,7 @@ BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 NOALLOC_MAX_ROWS = 1 << 20
 
 EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_noalloc",
-            "sdpa_bwd_workspace_size", "sdpa_t5_bucket",
+            "sdpa_bwd_workspace_size", "sdpa_t5_bucket", "sdpa_exp2_fma",
             "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
             "sdpa_status_string")
 
@@ -82,6 +82,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_bwd_workspace_size.restype = sz
     lib.sdpa_t5_bucket.argtypes = [vp, vp, i64, i32, i32, i32, vp]
     lib.sdpa_t5_bucket.restype = i32
+    lib.sdpa_exp2_fma.argtypes = [vp, vp, i64, vp]
+    lib.sdpa_exp2_fma.restype = i32
     lib.sdpa_read_device_status.argtypes = [vp]
     lib.sdpa_read_device_status.restype = i32
     lib.sdpa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -257,6 +259,16 @@ def sdpa_t5_bucket(rel: torch.Tensor, num_buckets=32, max_distance=128, bidirect
                             int(max_distance), 1 if bidirectional else 0, _stream(rel))
     _check(st, "sdpa_t5_bucket")
     return out
+
+
+def sdpa_exp2_fma(x: torch.Tensor) -> torch.Tensor:
+    """2^x by the kernels' FMA-pipe exponential (float32 CUDA tensor)."""
+    lib = load_library()
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(lib.sdpa_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(x)), "sdpa_exp2_fma")
+    return y
 
 
 def sdpa_read_device_status() -> int:

@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "exp2_poly.cuh"
+
 namespace sdpa {
 
 constexpr int kTile = 128;             // query rows and keys per tile
@@ -72,6 +74,16 @@ struct AttnParams {
   T5Spec t5;
   uint64_t wait_limit_ns;
 };
+
+// Whether column c of a fully visible tile takes the FMA-pipe exponential:
+// never with a dense bias, whose entries may be -inf (masked) even inside a
+// visible tile and must give exactly 0; otherwise columns c (mod 8) >=
+// MUFU_PER8 do -- a fixed split per kernel, so results stay bit-reproducible.
+// MUFU_PER8 = 8 keeps every exponential on the MUFU unit.
+template <int BIAS, int MUFU_PER8>
+__device__ __forceinline__ constexpr bool emu_exp2(int c) {
+  return BIAS != kBiasDense && (c & 7) >= MUFU_PER8;
+}
 
 // Key tiles [nlo, nhi) that hold any key visible from query rows
 // [m0, m0 + rows) (clipped to L).  Empty when nhi <= nlo.

@@ -9,27 +9,34 @@
 // result is bit-identical run to run (HF transformers issue #31787,
 // "Transformer models are not deterministic when using Flash Attention 2"):
 //   1. preprocess: D = rowsum(dO * O) into the workspace.
-//   2. dK/dV: one CTA per (128 keys, KV head, batch).  It walks 64-query
-//      blocks of the band, for every query head of the group, in a fixed
+//   2. dK/dV: one CTA per (128 keys, KV head, batch).  It walks 128-query
+//      tiles of the band, for every query head of the group, in a fixed
 //      order and accumulates dV and dK in tensor memory:
-//        S^T = K Q^T, dP^T = V dO^T           (SS MMAs, 128 x 64)
+//        S^T = K Q^T, dP^T = V dO^T           (SS MMAs, 128 x 128)
 //        P^T, dS^T -> tensor memory as bf16    (compute warpgroups)
 //        dV += P^T dO, dK += dS^T Q            (TS MMAs, 128 x d)
-//   3. dQ: one CTA per (128 queries, query head, batch), walking 64-key
-//      blocks of the band in order: S = Q K^T, dP = dO V^T, dQ += dS K.
-// In both, S and dP are double-buffered in tensor memory and the MMA warp
-// issues the scores of block i before the gradient MMAs of block i-1, so the
-// exponentials of one block overlap the tensor-core work of its neighbours.
-// Two compute warpgroups take alternate blocks.
+//   3. dQ: one CTA per (128 queries, query head, batch), walking 128-key
+//      tiles of the band in order: S = Q K^T, dP = dO V^T, dQ += dS K, with S
+//      double-buffered so the next tile's scores are ready while this tile's
+//      dS is formed.
+// All score MMAs are 128 x 128 (an N = 64 MMA with both operands in shared
+// memory is shared-memory-bandwidth bound on this part); the two compute
+// warpgroups split every tile's 128 columns between them.
 #pragma once
 
 #include "attn_common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100.cuh"
 #include "tmem_sync.cuh"
 
 namespace sdpa {
 
-constexpr int kBlk = 64;  // inner block: queries (dK/dV kernel) or keys (dQ kernel)
+constexpr int kBlk = 64;  // columns per compute warpgroup in a 128-wide tile
+// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all),
+// chosen by measurement: the dK/dV kernel gains from moving 3 of 8 to the
+// FMA pipe, the dQ kernel does not.
+constexpr int kDkdvMufuPer8 = 5;
+constexpr int kDqMufuPer8 = 8;
 
 struct BwdMaps {
   CUtensorMap q128, dout128, k128, v128;  // 128-row boxes (resident tiles)
@@ -75,41 +82,59 @@ __device__ __forceinline__ uint32_t kmajor_koff(int kk, int rows) {
 }
 
 // ------------------------------------------------------------------ dK / dV
-template <int D>
+// CTA = 128 keys of one (KV head, batch).  Blocks of 128 queries stream
+// through; both compute warpgroups work on every block, warpgroup w on the
+// query columns [64 w, 64 w + 64).  Tensor memory (512 columns):
+//   S^T 0..127 | dP^T 128..255 | dV 256.. | dK 256 + d..
+// P^T (bf16) overwrites the first half of each warpgroup's S^T columns, dS^T
+// the first half of its dP^T columns; the TS MMAs read them from there.
+template <int D, int BIAS>
 struct DkdvLayout {
-  static constexpr int kKVBytes = kTile * D * 2;  // resident K or V tile (128 keys)
-  static constexpr int kBlkBytes = kBlk * D * 2;  // one 64-query block of Q or dO
-  static constexpr int kStages = 3;
+  static constexpr int kTileBytes = kTile * D * 2;  // 128 rows x d bf16
+  // Q blocks are used until the block's dK MMA, dO blocks only until its dV
+  // MMA: the Q ring is the deeper one.  At d = 128 without a T5 table this
+  // fills the 227 KB of shared memory to the last kilobyte.
+  static constexpr int kSQ = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : 4;
+  static constexpr int kSO = (D == 128) ? 2 : 4;
   static constexpr int kKOff = 0;
-  static constexpr int kVOff = kKVBytes;
-  static constexpr int kQOff = 2 * kKVBytes;
-  static constexpr int kDOOff = kQOff + kStages * kBlkBytes;
-  static constexpr int kVecOff = kDOOff + kStages * kBlkBytes;  // stages x (lse2[64], D[64])
-  static constexpr int kLutOff = kVecOff + kStages * 2 * kBlk * 4;  // 2 WG x 2 x 256 floats
-  static constexpr int kBarOff = kLutOff + 4 * 256 * 4;
-  // kv_full, q_full[S], q_empty[S], s_full[2], dp_full[2], p_full[2], ds_full[2],
-  // buf_free[2], acc_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 10 + 2;
+  static constexpr int kVOff = kTileBytes;
+  static constexpr int kQOff = 2 * kTileBytes;                  // Q ring
+  static constexpr int kDOOff = kQOff + kSQ * kTileBytes;       // dO ring
+  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;     // 2 x (lse2[128], D[128])
+  static constexpr int kLutOff = kVecOff + 2 * 2 * kTile * 4;   // T5 only: 2 WG x 2 x 256
+  static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
+  static constexpr int kBarOff = kLutOff + kLutBytes;
+  // kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], vec_full[2],
+  // vec_empty[2], s_full, dp_full, p_full, ds_full, s_free, dp_free, acc_done, drain
+  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
-  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr int kSmemAlloc = kMiscOff + 16;
   static constexpr int kThreads = 320;  // 2 compute warpgroups, producer, MMA
   static constexpr int kTmemCols = 512;
-  // S^T[x] at 64 x, dP^T[x] at 128 + 64 x, dV at 256, dK at 256 + D
-  static constexpr int kDVCol = 256, kDKCol = 256 + D;
+  static constexpr int kSCol = 0, kDPCol = 128, kDVCol = 256, kDKCol = 256 + D;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
+
+// TMEM column of the bf16 A operand for the 16-row K step kk of a 128-wide
+// block whose two 64-wide halves were written by the two warpgroups into the
+// first 32 columns of their own 64-column regions starting at `base`.
+__device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
+  return base + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+}
 
 template <int D, int BIAS>
 __global__ void __launch_bounds__(320, 1)
     bwd_dkdv_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmDO) {
-  using Lay = DkdvLayout<D>;
-  constexpr int S = Lay::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  using Lay = DkdvLayout<D, BIAS>;
+  constexpr int SQ = Lay::kSQ;
+  constexpr int SO = Lay::kSO;
+  extern __shared__ uint8_t smem[];
+  if (!smem_base_ok(smem)) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusMisaligned);
+    return;
+  }
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -118,47 +143,50 @@ __global__ void __launch_bounds__(320, 1)
   const int b = blockIdx.z;
   const int n0 = static_cast<int>(blockIdx.x) * kTile;  // causal: low key tiles are heaviest
   int mlo, mhi;
-  {
-    // 64-query blocks that hold any query seeing a key of this tile
-    const int n_last = min(n0 + kTile - 1, p.L - 1);
-    int imin = 0;
-    if (p.causal) imin = n0;
-    if (p.wr >= 0) imin = max(imin, n0 - p.wr);
-    int imax = p.L - 1;
-    if (p.wl >= 0) imax = min(imax, n_last + p.wl);
-    mlo = imin / kBlk;
-    mhi = (imax >= imin) ? imax / kBlk + 1 : mlo;
-  }
-  const int nm = mhi - mlo;
-  const int total = nm * p.G;  // blocks: query head (outer) x query block (inner)
+  query_tile_range(p, n0, mlo, mhi);
+  const int nm = mhi > mlo ? mhi - mlo : 0;
+  const int total = nm * p.G;  // blocks: query head (outer) x query tile (inner)
 
   auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
   const uint32_t kv_full = bar(0);
   auto q_full = [&](int s) { return bar(1 + s); };
-  auto q_empty = [&](int s) { return bar(1 + S + s); };
-  auto s_full = [&](int x) { return bar(1 + 2 * S + x); };
-  auto dp_full = [&](int x) { return bar(3 + 2 * S + x); };
-  auto p_full = [&](int x) { return bar(5 + 2 * S + x); };
-  auto ds_full = [&](int x) { return bar(7 + 2 * S + x); };
-  auto buf_free = [&](int x) { return bar(9 + 2 * S + x); };
-  const uint32_t acc_done = bar(11 + 2 * S);
-  const uint32_t drain = bar(12 + 2 * S);
+  auto q_empty = [&](int s) { return bar(1 + SQ + s); };
+  auto o_full = [&](int s) { return bar(1 + 2 * SQ + s); };
+  auto o_empty = [&](int s) { return bar(1 + 2 * SQ + SO + s); };
+  constexpr int kB = 1 + 2 * SQ + 2 * SO;
+  auto vec_full = [&](int x) { return bar(kB + x); };
+  auto vec_empty = [&](int x) { return bar(kB + 2 + x); };
+  const uint32_t s_full = bar(kB + 4);
+  const uint32_t dp_full = bar(kB + 5);
+  const uint32_t p_full = bar(kB + 6);
+  const uint32_t ds_full = bar(kB + 7);
+  const uint32_t s_free = bar(kB + 8);
+  const uint32_t dp_free = bar(kB + 9);
+  const uint32_t acc_done = bar(kB + 10);
+  const uint32_t drain = bar(kB + 11);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(q_full(s), 32);  // the producer warp's lanes (lane 0 with the tx count)
+    for (int s = 0; s < SQ; ++s) {
+      mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(s_full(x), 1);
-      mbar_init(dp_full(x), 1);
-      mbar_init(p_full(x), kTile);
-      mbar_init(ds_full(x), kTile);
-      mbar_init(buf_free(x), 1);
+    for (int s = 0; s < SO; ++s) {
+      mbar_init(o_full(s), 1);
+      mbar_init(o_empty(s), 1);
     }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(vec_full(x), 32);          // the producer warp's lanes
+      mbar_init(vec_empty(x), 2 * kTile);  // both compute warpgroups
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 2 * kTile);
+    mbar_init(ds_full, 2 * kTile);
+    mbar_init(s_free, 1);
+    mbar_init(dp_free, 1);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -181,115 +209,147 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmDO);
-        mbar_expect_tx(kv_full, 2 * Lay::kKVBytes);
+        mbar_expect_tx(kv_full, 2 * Lay::kTileBytes);
         for (int h = 0; h < D / 64; ++h) {
           tma_load_4d(sb + Lay::kKOff + h * kTile * 128, &tmK, kv_full, h * 64, n0, g, b);
           tma_load_4d(sb + Lay::kVOff + h * kTile * 128, &tmV, kv_full, h * 64, n0, g, b);
         }
       }
-      int issued[S];
-      for (int s = 0; s < S; ++s) issued[s] = -1;
-      bool ok = true;
-      for (int it = 0; it < total; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
+      // LSE (log2 units) and D of one block's 128 queries, four per lane,
+      // loaded one block ahead of the slot they go to.
+      float l2v[4], ddv[4];
+      auto load_vec = [&](int it) {
         const int hq = g * p.G + it / nm;
-        const int m0 = (mlo + it % nm) * kBlk;
-        if (ok) ok = mbar_wait(q_empty(s), ph ^ 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        // LSE (log2 units) and D of the block's 64 queries, two per lane
-        float* lse2 = vec + s * 2 * kBlk;
-        float* dvv = lse2 + kBlk;
+        const int m0 = (mlo + it % nm) * kTile;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = lane + 32 * e;
-          const int i = m0 + c;
-          float l2 = INFINITY, dd = 0.f;  // queries past L: P = 0
+        for (int e = 0; e < 4; ++e) {
+          const int i = m0 + lane + 32 * e;
+          l2v[e] = INFINITY;  // queries past L: P = 0
+          ddv[e] = 0.f;
           if (i < p.L) {
             const int64_t idx = (static_cast<int64_t>(b) * p.Hq + hq) * p.L + i;
-            l2 = p.lse[idx] * kLog2e;
-            dd = p.dvec[idx];
-            if (l2 == -INFINITY) l2 = INFINITY;  // row with no visible key
+            l2v[e] = p.lse[idx] * kLog2e;
+            ddv[e] = p.dvec[idx];
+            if (l2v[e] == -INFINITY) l2v[e] = INFINITY;  // row with no visible key
           }
-          lse2[c] = l2;
-          dvv[c] = dd;
         }
-        __syncwarp();
+      };
+      load_vec(0);
+      int issued_q[SQ], issued_o[SO];
+      for (int s = 0; s < SQ; ++s) issued_q[s] = -1;
+      for (int s = 0; s < SO; ++s) issued_o[s] = -1;
+      bool ok = true;
+      for (int it = 0; it < total; ++it) {
+        const int hq = g * p.G + it / nm;
+        const int m0 = (mlo + it % nm) * kTile;
+        const int x = it & 1;
+        if (ok) ok = mbar_wait(vec_empty(x), ((it >> 1) & 1) ^ 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float* lse2 = vec + x * 2 * kTile;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          lse2[lane + 32 * e] = l2v[e];
+          lse2[kTile + lane + 32 * e] = ddv[e];
+        }
+        mbar_arrive(vec_full(x));
         if (lane == 0) {
-          mbar_expect_tx(q_full(s), 2 * Lay::kBlkBytes);
-          for (int h = 0; h < D / 64; ++h) {
-            tma_load_4d(sb + Lay::kQOff + s * Lay::kBlkBytes + h * kBlk * 128, &tmQ, q_full(s),
-                        h * 64, m0, hq, b);
-            tma_load_4d(sb + Lay::kDOOff + s * Lay::kBlkBytes + h * kBlk * 128, &tmDO, q_full(s),
-                        h * 64, m0, hq, b);
+          const int sq = it % SQ, so = it % SO;
+          ok = mbar_wait(q_empty(sq), ((it / SQ) & 1) ^ 1, ctl);
+          if (ok) {
+            mbar_expect_tx(q_full(sq), Lay::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(sb + Lay::kQOff + sq * Lay::kTileBytes + h * kTile * 128, &tmQ,
+                          q_full(sq), h * 64, m0, hq, b);
+            issued_q[sq] = (it / SQ) & 1;
+            ok = mbar_wait(o_empty(so), ((it / SO) & 1) ^ 1, ctl);
           }
-        } else {
-          mbar_arrive(q_full(s));
+          if (ok) {
+            mbar_expect_tx(o_full(so), Lay::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(sb + Lay::kDOOff + so * Lay::kTileBytes + h * kTile * 128, &tmDO,
+                          o_full(so), h * 64, m0, hq, b);
+            issued_o[so] = (it / SO) & 1;
+          }
         }
-        issued[s] = ph;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (it + 1 < total) load_vec(it + 1);
       }
       if (!ok && lane == 0) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
         mbar_wait(kv_full, 0, ign);
-        for (int s = 0; s < S; ++s)
-          if (issued[s] >= 0) mbar_wait(q_full(s), issued[s], ign);
+        for (int s = 0; s < SQ; ++s)
+          if (issued_q[s] >= 0) mbar_wait(q_full(s), issued_q[s], ign);
+        for (int s = 0; s < SO; ++s)
+          if (issued_o[s] >= 0) mbar_wait(o_full(s), issued_o[s], ign);
       }
     }
   } else if (warp == 9) {
     // ============================ MMA issuer ============================
     if (lane == 0 && total > 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kBlk, 0, 0);  // 128 keys x 64 queries
-      constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);     // 128 keys x d
-      auto grads = [&](int jb) -> bool {
-        const int x = jb & 1;
-        const int s = jb % S;
-        const uint32_t ph = (jb >> 1) & 1;
-        const uint32_t qs = sb + Lay::kQOff + s * Lay::kBlkBytes;
-        const uint32_t dos = sb + Lay::kDOOff + s * Lay::kBlkBytes;
-        if (!mbar_wait(p_full(x), ph, ctl)) return false;
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 keys x 128 queries
+      constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // 128 keys x d
+      auto issue_s = [&](int jb) -> bool {
+        const int sq = jb % SQ;
+        const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
+        if (!mbar_wait(q_full(sq), (jb / SQ) & 1, ctl)) return false;
+        // S^T held P^T of the previous block: wait for that block's dV MMA
+        if (jb > 0 && !mbar_wait(s_free, (jb - 1) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ts(tmem + Lay::kDVCol, tmem + 64 * x + kk * 8,
-                 smem_desc_sw128(dos + kk * 2048, kBlk * 128, 1024), kIdG,
-                 (jb > 0 || kk > 0) ? 1u : 0u);
-        if (!mbar_wait(ds_full(x), ph, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ts(tmem + Lay::kDKCol, tmem + 128 + 64 * x + kk * 8,
-                 smem_desc_sw128(qs + kk * 2048, kBlk * 128, 1024), kIdG,
-                 (jb > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(buf_free(x));
-        mma_commit(q_empty(s));
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + Lay::kSCol, smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
+                 smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
         return true;
       };
-      bool ok = mbar_wait(kv_full, 0, ctl);
-      for (int it = 0; it < total && ok; ++it) {
-        const int x = it & 1;
-        const int s = it % S;
-        const uint32_t qs = sb + Lay::kQOff + s * Lay::kBlkBytes;
-        const uint32_t dos = sb + Lay::kDOOff + s * Lay::kBlkBytes;
-        if (!(ok = mbar_wait(q_full(s), (it / S) & 1, ctl))) break;
-        // buffer x last held block it-2: its P^T / dS^T must have been consumed
-        if (it >= 2 && !(ok = mbar_wait(buf_free(x), ((it >> 1) - 1) & 1, ctl))) break;
+      auto issue_dp = [&](int jb) -> bool {
+        const int so = jb % SO;
+        const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
+        if (!mbar_wait(o_full(so), (jb / SO) & 1, ctl)) return false;
+        // dP^T held dS^T of the previous block: wait for that block's dK MMA
+        if (jb > 0 && !mbar_wait(dp_free, (jb - 1) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + 64 * x, smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(qs + kmajor_koff(kk, kBlk), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(s_full(x));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + 128 + 64 * x,
+          mma_ss(tmem + Lay::kDPCol,
                  smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(dos + kmajor_koff(kk, kBlk), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(dp_full(x));
-        if (it >= 1 && !(ok = grads(it - 1))) break;
+                 smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(dp_full);
+        return true;
+      };
+      // Order per block: dV(i), S(i+1), dK(i), dP(i+1): the scores of the
+      // next block are ready while this block's dK runs, so its exponentials
+      // overlap dK(i) and dP(i+1).
+      bool ok = mbar_wait(kv_full, 0, ctl);
+      ok = ok && issue_s(0) && issue_dp(0);
+      for (int it = 0; it < total && ok; ++it) {
+        const int sq = it % SQ, so = it % SO;
+        const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
+        const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
+        if (!(ok = mbar_wait(p_full, it & 1, ctl))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
+                 smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(s_free);
+        mma_commit(o_empty(so));
+        if (it + 1 < total && !(ok = issue_s(it + 1))) break;
+        if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk),
+                 smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(dp_free);
+        mma_commit(q_empty(sq));
+        if (it + 1 < total && !(ok = issue_dp(it + 1))) break;
       }
-      if (ok) ok = grads(total - 1);
       if (ok) mma_commit(acc_done);
       if (!ok) {
         volatile int never = 0;
@@ -299,31 +359,31 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // ======= compute warpgroup wg: blocks it = wg, wg + 2, ...; thread = key =======
+    // ===== compute warpgroup wg: query columns [64 wg, 64 wg + 64); thread = key =====
     const int wg = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const int j = n0 + row;
+    const int c0w = kBlk * wg;  // first query column of this warpgroup
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_bits + 64 * wg;
-    const uint32_t tDP = tmem + lane_bits + 128 + 64 * wg;
+    const uint32_t tS = tmem + lane_bits + Lay::kSCol + c0w;
+    const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + wg * 512;
     bool ok = true;
-    for (int it = wg; it < total; it += 2) {
-      const int k = it >> 1;
-      const int s = it % S;
+    for (int it = 0; it < total; ++it) {
+      const int x = it & 1;
       const int hq = g * p.G + it / nm;
-      const int m0 = (mlo + it % nm) * kBlk;
+      const int m0 = (mlo + it % nm) * kTile + c0w;  // first query of this warpgroup
       const float* lut_row = nullptr;
       if constexpr (BIAS == kBiasT5) {
         // j - i = (n0 - m0) + (row - c): entry r = row - c + 63, r in [0, 190]
-        float* lt = lut + (k & 1) * 256;
+        float* lt = lut + (it & 1) * 256;
         const int base = n0 - m0 - (kBlk - 1);
         for (int r = row; r < kTile + kBlk - 1; r += kTile)
           lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
         named_barrier(1 + wg, kTile);
         lut_row = lt + row + (kBlk - 1);
       }
-      // visible queries of this key inside the block: [lo, hi]
+      // visible queries of this key among the warpgroup's 64: [lo, hi]
       int lo = 0, hi = kBlk - 1;
       bool full = (m0 + kBlk <= p.L) && (n0 + kTile <= p.L);
       if (p.causal) full = full && (n0 + kTile - 1 <= m0);
@@ -338,57 +398,86 @@ __global__ void __launch_bounds__(320, 1)
       const float* bcol = nullptr;
       if constexpr (BIAS == kBiasDense)
         bcol = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
-               static_cast<int64_t>(m0) * p.sb_i + min(j, p.L - 1);
-      if (ok) ok = mbar_wait(q_full(s), (it / S) & 1, ctl);  // LSE / D staged
-      if (ok) ok = mbar_wait(s_full(wg), k & 1, ctl);
+               static_cast<int64_t>(min(m0, p.L - 1)) * p.sb_i + min(j, p.L - 1);
+      if (ok) ok = mbar_wait(vec_full(x), (it >> 1) & 1, ctl);  // LSE / D staged
+      if (ok) ok = mbar_wait(s_full, it & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
-      const float* lse2 = vec + s * 2 * kBlk;
-      const float* dvv = lse2 + kBlk;
+      const float* lse2 = vec + x * 2 * kTile + c0w;
+      const float* dvv = vec + x * 2 * kTile + kTile + c0w;
       uint32_t pr[64];  // S^T row, then P^T (fp32 bits)
       tmem_ld64_sync(tS, pr);
+      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < kBlk; ++c) {
-        float x = __uint_as_float(pr[c]) * p.scale_log2 - lse2[c];
-        const bool vis = full || (c >= lo && c <= hi);
-        if constexpr (BIAS == kBiasT5) x += lut_row[-c];
-        if constexpr (BIAS == kBiasDense)
-          x += vis ? bcol[static_cast<int64_t>(c) * p.sb_i] * kLog2e : 0.f;
-        pr[c] = __float_as_uint(vis ? fast_exp2(x) : 0.f);
+        for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+          const float4 l = lse4[c4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            if constexpr (BIAS == kBiasDense)
+              xv = fmaf(bcol[static_cast<int64_t>(c) * p.sb_i], kLog2e, xv);
+            pr[c] = __float_as_uint(emu_exp2<BIAS, kDkdvMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+          const float4 l = lse4[c4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const bool vis = (c >= lo) && (c <= hi);
+            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            if constexpr (BIAS == kBiasDense)
+              xv = fmaf(bcol[static_cast<int64_t>(vis ? c : 0) * p.sb_i], kLog2e, xv);
+            pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+          }
+        }
       }
 #pragma unroll
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+      for (int cc = 0; cc < kBlk; cc += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2)
-          pk[c >> 1] = pack_bf16x2(__uint_as_float(pr[c0 + c]), __uint_as_float(pr[c0 + c + 1]));
-        tmem_st16(tS + (c0 >> 1), pk);  // P^T over the first 32 columns of S^T[wg]
+          pk[c >> 1] = pack_bf16x2(__uint_as_float(pr[cc + c]), __uint_as_float(pr[cc + c + 1]));
+        tmem_st16(tS + (cc >> 1), pk);  // P^T over the first 32 of this warpgroup's columns
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full(wg));
-      if (ok) ok = mbar_wait(dp_full(wg), k & 1, ctl);
+      mbar_arrive(p_full);
+      if (ok) ok = mbar_wait(dp_full, it & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+      for (int cc = 0; cc < kBlk; cc += 32) {
         uint32_t dr[32];
-        tmem_ld32_sync(tDP + c0, dr);
+        tmem_ld32_sync(tDP + cc, dr);
         uint32_t pk[16];
+        const float4* d4v = reinterpret_cast<const float4*>(dvv + cc);
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float d0 = __uint_as_float(pr[c0 + c]) * (__uint_as_float(dr[c]) - dvv[c0 + c]);
-          const float d1 =
-              __uint_as_float(pr[c0 + c + 1]) * (__uint_as_float(dr[c + 1]) - dvv[c0 + c + 1]);
+        for (int c = 0; c < 32; c += 4) {
+          const float4 dv4 = d4v[c >> 2];
+          const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dv4.x);
+          const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dv4.y);
+          const float d2 = __uint_as_float(pr[cc + c + 2]) * (__uint_as_float(dr[c + 2]) - dv4.z);
+          const float d3 = __uint_as_float(pr[cc + c + 3]) * (__uint_as_float(dr[c + 3]) - dv4.w);
           pk[c >> 1] = pack_bf16x2(d0, d1);
+          pk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
         }
-        tmem_st16(tDP + (c0 >> 1), pk);  // dS^T over the first 32 columns of dP^T[wg]
+        tmem_st16(tDP + (cc >> 1), pk);  // dS^T over the first 32 of this warpgroup's columns
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_full(wg));
+      mbar_arrive(ds_full);
+      mbar_arrive(vec_empty(x));
     }
     // ---------------- epilogue: warpgroup 0 stores dV, warpgroup 1 stores dK ----------------
     if (ok && total > 0) ok = mbar_wait(acc_done, 0, ctl);
@@ -432,27 +521,33 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // --------------------------------------------------------------------- dQ
-template <int D>
+// CTA = 128 queries of one (query head, batch); blocks of 128 keys stream
+// through; warpgroup w takes the key columns [64 w, 64 w + 64).  Tensor
+// memory: S[0] 0..127 | S[1] 128..255 | dP 256..383 | dQ 384..  The scores
+// are double-buffered, so S of block i + 1 is computed while block i's dS is
+// formed; dS (bf16) overwrites the first half of each warpgroup's dP columns.
+template <int D, int BIAS>
 struct DqLayout {
-  static constexpr int kQBytes = kTile * D * 2;   // resident Q or dO tile (128 queries)
-  static constexpr int kBlkBytes = kBlk * D * 2;  // one 64-key block of K or V
-  static constexpr int kStages = 3;
+  static constexpr int kTileBytes = kTile * D * 2;
+  // K blocks are used until the block's dQ MMA, V blocks only until its dP
+  // MMA: the K ring is the deeper one.
+  static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : 4;
+  static constexpr int kSV = (D == 128) ? 2 : 3;
   static constexpr int kQOff = 0;
-  static constexpr int kDOOff = kQBytes;
-  static constexpr int kKOff = 2 * kQBytes;
-  static constexpr int kVOff = kKOff + kStages * kBlkBytes;
-  static constexpr int kLutOff = kVOff + kStages * kBlkBytes;  // 2 WG x 2 x 256 floats
-  static constexpr int kBarOff = kLutOff + 4 * 256 * 4;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], dp_full[2], ds_full[2], buf_free[2],
-  // acc_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 8 + 2;
+  static constexpr int kDOOff = kTileBytes;
+  static constexpr int kKOff = 2 * kTileBytes;                // K ring
+  static constexpr int kVOff = kKOff + kSK * kTileBytes;      // V ring
+  static constexpr int kLutOff = kVOff + kSV * kTileBytes;    // T5 only: 2 WG x 2 x 256 floats
+  static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
+  static constexpr int kBarOff = kLutOff + kLutBytes;
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_used[2],
+  // dp_full, ds_full, dq_done, acc_done, drain
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 9;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
-  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr int kSmemAlloc = kMiscOff + 16;
   static constexpr int kThreads = 320;
   static constexpr int kTmemCols = 512;
-  // S[x] at 64 x, dP[x] at 128 + 64 x, dQ at 256
-  static constexpr int kDQCol = 256;
+  static constexpr int kDPCol = 256, kDQCol = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
@@ -461,11 +556,14 @@ __global__ void __launch_bounds__(320, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmDO) {
-  using Lay = DqLayout<D>;
-  constexpr int S = Lay::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  using Lay = DqLayout<D, BIAS>;
+  constexpr int SK = Lay::kSK;
+  constexpr int SV = Lay::kSV;
+  extern __shared__ uint8_t smem[];
+  if (!smem_base_ok(smem)) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusMisaligned);
+    return;
+  }
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -477,44 +575,43 @@ __global__ void __launch_bounds__(320, 1)
   const int g = hq / p.G;
   const int m0 = qt * kTile;
   int nlo, nhi;
-  {
-    // 64-key blocks holding any key visible from rows [m0, m0 + 128)
-    const int m_last = min(m0 + kTile - 1, p.L - 1);
-    int jmin = 0;
-    if (p.wl >= 0) jmin = max(0, m0 - p.wl);
-    int jmax = p.L - 1;
-    if (p.causal) jmax = min(jmax, m_last);
-    if (p.wr >= 0) jmax = min(jmax, m_last + p.wr);
-    nlo = jmin / kBlk;
-    nhi = (jmax >= jmin) ? jmax / kBlk + 1 : nlo;
-  }
-  const int nt = nhi - nlo;
+  key_tile_range(p, m0, kTile, nlo, nhi);
+  const int nt = nhi > nlo ? nhi - nlo : 0;
 
   auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
   const uint32_t q_full = bar(0);
-  auto kv_full = [&](int s) { return bar(1 + s); };
-  auto kv_empty = [&](int s) { return bar(1 + S + s); };
-  auto s_full = [&](int x) { return bar(1 + 2 * S + x); };
-  auto dp_full = [&](int x) { return bar(3 + 2 * S + x); };
-  auto ds_full = [&](int x) { return bar(5 + 2 * S + x); };
-  auto buf_free = [&](int x) { return bar(7 + 2 * S + x); };
-  const uint32_t acc_done = bar(9 + 2 * S);
-  const uint32_t drain = bar(10 + 2 * S);
+  auto k_full = [&](int s) { return bar(1 + s); };
+  auto k_empty = [&](int s) { return bar(1 + SK + s); };
+  auto v_full = [&](int s) { return bar(1 + 2 * SK + s); };
+  auto v_empty = [&](int s) { return bar(1 + 2 * SK + SV + s); };
+  constexpr int kB = 1 + 2 * SK + 2 * SV;
+  auto s_full = [&](int x) { return bar(kB + x); };
+  auto s_used = [&](int x) { return bar(kB + 2 + x); };
+  const uint32_t dp_full = bar(kB + 4);
+  const uint32_t ds_full = bar(kB + 5);
+  const uint32_t dq_done = bar(kB + 6);
+  const uint32_t acc_done = bar(kB + 7);
+  const uint32_t drain = bar(kB + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+    for (int s = 0; s < SK; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < SV; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full(x), 1);
-      mbar_init(dp_full(x), 1);
-      mbar_init(ds_full(x), kTile);
-      mbar_init(buf_free(x), 1);
+      mbar_init(s_used(x), 2 * kTile);
     }
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 2 * kTile);
+    mbar_init(dq_done, 1);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -535,79 +632,99 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0 && nt > 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(q_full, 2 * Lay::kQBytes);
+      mbar_expect_tx(q_full, 2 * Lay::kTileBytes);
       for (int h = 0; h < D / 64; ++h) {
         tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, m0, hq, b);
         tma_load_4d(sb + Lay::kDOOff + h * kTile * 128, &tmDO, q_full, h * 64, m0, hq, b);
       }
-      int issued[S];
-      for (int s = 0; s < S; ++s) issued[s] = -1;
+      int issued_k[SK], issued_v[SV];
+      for (int s = 0; s < SK; ++s) issued_k[s] = -1;
+      for (int s = 0; s < SV; ++s) issued_v[s] = -1;
       bool ok = true;
       for (int it = 0; it < nt; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        const int n0 = (nlo + it) * kBlk;
-        if (!(ok = mbar_wait(kv_empty(s), ph ^ 1, ctl))) break;
-        mbar_expect_tx(kv_full(s), 2 * Lay::kBlkBytes);
-        for (int h = 0; h < D / 64; ++h) {
-          tma_load_4d(sb + Lay::kKOff + s * Lay::kBlkBytes + h * kBlk * 128, &tmK, kv_full(s),
+        const int sk = it % SK, sv = it % SV;
+        const int n0 = (nlo + it) * kTile;
+        if (!(ok = mbar_wait(k_empty(sk), ((it / SK) & 1) ^ 1, ctl))) break;
+        mbar_expect_tx(k_full(sk), Lay::kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK, k_full(sk),
                       h * 64, n0, g, b);
-          tma_load_4d(sb + Lay::kVOff + s * Lay::kBlkBytes + h * kBlk * 128, &tmV, kv_full(s),
+        issued_k[sk] = (it / SK) & 1;
+        if (!(ok = mbar_wait(v_empty(sv), ((it / SV) & 1) ^ 1, ctl))) break;
+        mbar_expect_tx(v_full(sv), Lay::kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(sb + Lay::kVOff + sv * Lay::kTileBytes + h * kTile * 128, &tmV, v_full(sv),
                       h * 64, n0, g, b);
-        }
-        issued[s] = ph;
+        issued_v[sv] = (it / SV) & 1;
       }
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
         mbar_wait(q_full, 0, ign);
-        for (int s = 0; s < S; ++s)
-          if (issued[s] >= 0) mbar_wait(kv_full(s), issued[s], ign);
+        for (int s = 0; s < SK; ++s)
+          if (issued_k[s] >= 0) mbar_wait(k_full(s), issued_k[s], ign);
+        for (int s = 0; s < SV; ++s)
+          if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
       }
     }
   } else if (warp == 9) {
     // ============================ MMA issuer ============================
     if (lane == 0 && nt > 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kBlk, 0, 0);  // 128 queries x 64 keys
-      constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);     // 128 queries x d
-      auto grad = [&](int jb) -> bool {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
+      constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
+      auto issue_s = [&](int jb) -> bool {
         const int x = jb & 1;
-        const int s = jb % S;
-        const uint32_t ks = sb + Lay::kKOff + s * Lay::kBlkBytes;
-        if (!mbar_wait(ds_full(x), (jb >> 1) & 1, ctl)) return false;
+        const int sk = jb % SK;
+        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+        if (!mbar_wait(k_full(sk), (jb / SK) & 1, ctl)) return false;
+        // S[x] held block jb-2: both warpgroups must have loaded it
+        if (jb >= 2 && !mbar_wait(s_used(x), ((jb >> 1) - 1) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ts(tmem + Lay::kDQCol, tmem + 64 * x + kk * 8,
-                 smem_desc_sw128(ks + kk * 2048, kBlk * 128, 1024), kIdQ,
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kTile * x,
+                 smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
+                 smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(s_full(x));
+        return true;
+      };
+      auto issue_dp = [&](int jb) -> bool {
+        const int sv = jb % SV;
+        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+        if (!mbar_wait(v_full(sv), (jb / SV) & 1, ctl)) return false;
+        // dP held dS of block jb-1: wait for that block's dQ MMA
+        if (jb >= 1 && !mbar_wait(dq_done, (jb - 1) & 1, ctl)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + Lay::kDPCol,
+                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
+                 smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(dp_full);
+        mma_commit(v_empty(sv));
+        return true;
+      };
+      auto issue_dq = [&](int jb) -> bool {
+        const int sk = jb % SK;
+        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+        if (!mbar_wait(ds_full, jb & 1, ctl)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + Lay::kDPCol, kk),
+                 smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
                  (jb > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(buf_free(x));
-        mma_commit(kv_empty(s));
+        mma_commit(dq_done);
+        mma_commit(k_empty(sk));
         return true;
       };
       bool ok = mbar_wait(q_full, 0, ctl);
+      ok = ok && issue_s(0) && issue_dp(0);
       for (int it = 0; it < nt && ok; ++it) {
-        const int x = it & 1;
-        const int s = it % S;
-        const uint32_t ks = sb + Lay::kKOff + s * Lay::kBlkBytes;
-        const uint32_t vs = sb + Lay::kVOff + s * Lay::kBlkBytes;
-        if (!(ok = mbar_wait(kv_full(s), (it / S) & 1, ctl))) break;
-        if (it >= 2 && !(ok = mbar_wait(buf_free(x), ((it >> 1) - 1) & 1, ctl))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + 64 * x, smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(ks + kmajor_koff(kk, kBlk), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(s_full(x));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + 128 + 64 * x,
-                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(vs + kmajor_koff(kk, kBlk), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(dp_full(x));
-        if (it >= 1 && !(ok = grad(it - 1))) break;
+        if (it + 1 < nt && !(ok = issue_s(it + 1))) break;
+        if (!(ok = issue_dq(it))) break;
+        if (it + 1 < nt && !(ok = issue_dp(it + 1))) break;
       }
-      if (ok) ok = grad(nt - 1);
       if (ok) mma_commit(acc_done);
       if (!ok) {
         volatile int never = 0;
@@ -617,13 +734,13 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // ===== compute warpgroup wg: blocks it = wg, wg + 2, ...; thread = query row =====
+    // ===== compute warpgroup wg: key columns [64 wg, 64 wg + 64); thread = query row =====
     const int wg = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const int i = m0 + row;
+    const int c0w = kBlk * wg;
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_bits + 64 * wg;
-    const uint32_t tDP = tmem + lane_bits + 128 + 64 * wg;
+    const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + wg * 512;
     float l2 = INFINITY, dd = 0.f;
     if (i < p.L) {
@@ -637,13 +754,13 @@ __global__ void __launch_bounds__(320, 1)
       brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
              static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
     bool ok = true;
-    for (int it = wg; it < nt; it += 2) {
-      const int k = it >> 1;
-      const int n0 = (nlo + it) * kBlk;
+    for (int it = 0; it < nt; ++it) {
+      const int x = it & 1;
+      const int n0 = (nlo + it) * kTile + c0w;  // first key of this warpgroup
       const float* lut_row = nullptr;
       if constexpr (BIAS == kBiasT5) {
         // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
-        float* lt = lut + (k & 1) * 256;
+        float* lt = lut + (it & 1) * 256;
         const int base = n0 - m0 - (kTile - 1);
         for (int r = row; r < kTile + kBlk - 1; r += kTile)
           lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
@@ -661,40 +778,52 @@ __global__ void __launch_bounds__(320, 1)
         if (p.causal) hi = min(hi, i - n0);
         if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
       }
-      if (ok) ok = mbar_wait(s_full(wg), k & 1, ctl);
+      if (ok) ok = mbar_wait(s_full(x), (it >> 1) & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
       uint32_t pr[64];  // S row, then P (fp32 bits)
-      tmem_ld64_sync(tS, pr);
+      tmem_ld64_sync(tmem + lane_bits + kTile * x + c0w, pr);
+      tc_fence_before();
+      mbar_arrive(s_used(x));  // S[x] may now take block it + 2
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < kBlk; ++c) {
-        float x = __uint_as_float(pr[c]) * p.scale_log2 - l2;
-        const bool vis = full || (c >= lo && c <= hi);
-        if constexpr (BIAS == kBiasT5) x += lut_row[c];
-        if constexpr (BIAS == kBiasDense) x += vis ? brow[n0 + c] * kLog2e : 0.f;
-        pr[c] = __float_as_uint(vis ? fast_exp2(x) : 0.f);
+        for (int c = 0; c < kBlk; ++c) {
+          float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -l2);
+          if constexpr (BIAS == kBiasT5) xv += lut_row[c];
+          if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + c], kLog2e, xv);
+          pr[c] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBlk; ++c) {
+          const bool vis = (c >= lo) && (c <= hi);
+          float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -l2);
+          if constexpr (BIAS == kBiasT5) xv += lut_row[c];
+          if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + (vis ? c : 0)], kLog2e, xv);
+          pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+        }
       }
-      if (ok) ok = mbar_wait(dp_full(wg), k & 1, ctl);
+      if (ok) ok = mbar_wait(dp_full, it & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+      for (int cc = 0; cc < kBlk; cc += 32) {
         uint32_t dr[32];
-        tmem_ld32_sync(tDP + c0, dr);
+        tmem_ld32_sync(tDP + cc, dr);
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float d0 = __uint_as_float(pr[c0 + c]) * (__uint_as_float(dr[c]) - dd);
-          const float d1 = __uint_as_float(pr[c0 + c + 1]) * (__uint_as_float(dr[c + 1]) - dd);
+          const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dd);
+          const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dd);
           pk[c >> 1] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tS + (c0 >> 1), pk);  // dS over the first 32 columns of S[wg]
+        tmem_st16(tDP + (cc >> 1), pk);  // dS over the first 32 of this warpgroup's dP columns
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_full(wg));
+      mbar_arrive(ds_full);
     }
     // ------------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -------------
     if (ok && nt > 0) ok = mbar_wait(acc_done, 0, ctl);
@@ -750,22 +879,24 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, uint32_t phases,
   }
   const int ntiles = (p.L + kTile - 1) / kTile;
   if (phases & kPhaseDq) {
+    using Lay = DqLayout<D, BIAS>;
     auto kern = bwd_dq_kernel<D, BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DqLayout<D>::kSmemAlloc);
+                                         Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(ntiles, p.Hq, p.B), DqLayout<D>::kThreads, DqLayout<D>::kSmemAlloc, st>>>(
-        p, m.q128, m.k64, m.v64, m.dout128);
+    kern<<<dim3(ntiles, p.Hq, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(
+        p, m.q128, m.k128, m.v128, m.dout128);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (phases & kPhaseDkdv) {
+    using Lay = DkdvLayout<D, BIAS>;
     auto kern = bwd_dkdv_kernel<D, BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DkdvLayout<D>::kSmemAlloc);
+                                         Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(ntiles, p.Hkv, p.B), DkdvLayout<D>::kThreads, DkdvLayout<D>::kSmemAlloc, st>>>(
-        p, m.q64, m.k128, m.v128, m.dout64);
+    kern<<<dim3(ntiles, p.Hkv, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(
+        p, m.q128, m.k128, m.v128, m.dout128);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

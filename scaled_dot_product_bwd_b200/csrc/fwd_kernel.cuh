@@ -24,12 +24,16 @@
 #pragma once
 
 #include "attn_common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100.cuh"
 #include "tmem_sync.cuh"
 
 namespace sdpa {
 
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
+constexpr float kRescaleThreshold = 8.0f;
+// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all): the
+// forward measured fastest with every exponential on MUFU.
+constexpr int kFwdMufuPer8 = 8;  // log2 units: rescale O when max grows > 2^8
 
 template <int D, int NQ>
 struct FwdLayout {
@@ -280,7 +284,8 @@ __global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
       // x: scores in log2 units, in place over the raw accumulator bits
       uint32_t x[128];
       tmem_ld128_sync(tS, x);
-      float tmax = -INFINITY;
+      // four independent max / sum chains instead of one 128 long
+      float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       const float* bcol = brow ? brow + n0 : nullptr;
       if (full) {
 #pragma unroll
@@ -288,7 +293,7 @@ __global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
           float v = __uint_as_float(x[c]) * p.scale_log2;
           if constexpr (BIAS != kBiasNone) v += bias_log2<BIAS>(lut_row, bcol, c);
           x[c] = __float_as_uint(v);
-          tmax = fmaxf(tmax, v);
+          tm[c & 3] = fmaxf(tm[c & 3], v);
         }
       } else {
 #pragma unroll
@@ -299,27 +304,47 @@ __global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
           if constexpr (BIAS == kBiasDense) v += vis ? bcol[c] * kLog2e : 0.f;
           v = vis ? v : -INFINITY;
           x[c] = __float_as_uint(v);
-          tmax = fmaxf(tmax, v);
+          tm[c & 3] = fmaxf(tm[c & 3], v);
         }
       }
+      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
       const float m_new = fmaxf(m_run, tmax);
       const bool grow = m_new > m_run + kRescaleThreshold;
       const float m_use = grow ? m_new : m_run;
       const float alpha = grow ? fast_exp2(m_run - m_use) : 1.f;
       const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-      float sum = 0.f;
+      float sm[4] = {0.f, 0.f, 0.f, 0.f};
+      if (full) {
+        // every entry is finite: a fixed share of the exponentials on the FMA pipe
 #pragma unroll
-      for (int c0 = 0; c0 < kTile; c0 += 32) {
-        uint32_t pk[16];
+        for (int c0 = 0; c0 < kTile; c0 += 32) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float e0 = fast_exp2(__uint_as_float(x[c0 + c]) - m_sub);
-          const float e1 = fast_exp2(__uint_as_float(x[c0 + c + 1]) - m_sub);
-          sum += e0 + e1;
-          pk[c >> 1] = pack_bf16x2(e0, e1);
+          for (int c = 0; c < 32; c += 2) {
+            const float v0 = __uint_as_float(x[c0 + c]) - m_sub;
+            const float v1 = __uint_as_float(x[c0 + c + 1]) - m_sub;
+            const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
+            const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
+            sm[(c >> 1) & 3] += e0 + e1;
+            pk[c >> 1] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
         }
-        tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < kTile; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float e0 = fast_exp2(__uint_as_float(x[c0 + c]) - m_sub);
+            const float e1 = fast_exp2(__uint_as_float(x[c0 + c + 1]) - m_sub);
+            sm[(c >> 1) & 3] += e0 + e1;
+            pk[c >> 1] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + (c0 >> 1), pk);
+        }
       }
+      const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
       l_run = l_run * alpha + sum;
       m_run = m_use;
       tmem_st_wait();

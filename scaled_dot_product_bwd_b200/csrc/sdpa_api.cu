@@ -173,6 +173,12 @@ cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const C
   }
 }
 
+__global__ void exp2_fma_kernel(const float* x, float* y, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = exp2_fma(x[i]);
+}
+
 __global__ void t5_bucket_kernel(const int32_t* rel, int32_t* out, int64_t n, T5Spec spec) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
@@ -352,12 +358,23 @@ sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n, int32_
   return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
+sdpa_status_t sdpa_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return SDPA_ERR_INVALID_ARG;
+  if (n == 0) return SDPA_OK;
+  const int64_t blocks = (n + 255) / 256;
+  exp2_fma_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0,
+                    static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
 sdpa_status_t sdpa_read_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SDPA_ERR_CUDA;
   unsigned int h = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(h)) != cudaSuccess) return SDPA_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SDPA_ERR_CUDA;
-  return (h & kStatusTimeout) ? SDPA_ERR_TIMEOUT : SDPA_OK;
+  if (h & kStatusTimeout) return SDPA_ERR_TIMEOUT;
+  if (h & kStatusMisaligned) return SDPA_ERR_UNSUPPORTED;
+  return SDPA_OK;
 }
 
 sdpa_status_t sdpa_debug_wait_timeout(void* stream) {

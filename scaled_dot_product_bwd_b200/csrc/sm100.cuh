@@ -15,6 +15,15 @@ namespace sdpa {
 // library is one translation unit, so the definition lives here.
 __device__ unsigned int g_device_status = 0;
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusMisaligned = 2u;
+
+// Dynamic shared memory starts right after the 1 KB the driver reserves per
+// CTA, so it is 1024-byte aligned -- what the 128-byte swizzle atoms need.
+// Kernels check it on entry and, if it ever is not, record kStatusMisaligned
+// and return before touching anything.
+__device__ __forceinline__ bool smem_base_ok(const void* p) {
+  return (static_cast<uint32_t>(__cvta_generic_to_shared(p)) & 1023u) == 0;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -56,6 +65,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete sleeps until it
+// completes or `hint_ns` passes, instead of returning at once: waiting warps
+// then leave their issue slots to the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared state every role of a CTA consults while waiting: once one wait
 // runs out, `abort` is set and every other wait returns false at once, so
 // all roles fall through to the common teardown instead of hanging.
@@ -65,15 +90,14 @@ struct WaitCtl {
 };
 
 // Wait for phase `parity` of barrier `bar` to complete, for at most
-// ctl.limit_ns.  Returns false (and raises the abort flag and the device
-// status) when the limit is reached, or at once if another wait aborted.
+// ctl.limit_ns (checked between sleeps of at most 0.5 ms).  Returns false
+// (and raises the abort flag and the device status) when the limit is
+// reached, or at once if another wait aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
     if (*ctl.abort) return false;
     if (globaltimer_ns() - t0 > ctl.limit_ns) {
       *ctl.abort = 1;

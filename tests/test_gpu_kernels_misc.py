@@ -5,8 +5,9 @@ import pytest
 import torch
 
 from oracle import t5_relative_bucket
-from scaled_dot_product_bwd_b200 import (sdpa_debug_wait_timeout, sdpa_read_device_status,
-                                         sdpa_set_wait_limit_ns, sdpa_t5_bucket)
+from scaled_dot_product_bwd_b200 import (sdpa_debug_wait_timeout, sdpa_exp2_fma,
+                                         sdpa_read_device_status, sdpa_set_wait_limit_ns,
+                                         sdpa_t5_bucket)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,3 +32,19 @@ def test_wait_timeout_reports_status_and_context_survives():
         sdpa_set_wait_limit_ns(2_000_000_000)
     x = torch.ones(1024, device="cuda")
     assert float(x.sum()) == 1024.0            # the context is still usable
+
+
+def test_exp2_fma_within_its_bound():
+    # The FMA-pipe exponential against float64 exp2 (and CUDA's exp2f) over the
+    # range the kernels feed it: relative error below the stated 1.2e-4.
+    x = torch.cat([torch.linspace(-125, 125, 1_000_001), torch.linspace(-0.5, 0.5, 100_001),
+                   torch.tensor([-200.0, float("-inf")])]).cuda()
+    y = sdpa_exp2_fma(x).double().cpu()
+    xs = x.double().cpu()
+    ref = torch.exp2(xs)
+    rel = ((y[:-2] / ref[:-2]) - 1).abs().max().item()
+    assert rel < 1.2e-4, rel
+    cuda_rel = ((y[:-2] / torch.exp2(x[:-2]).double().cpu()) - 1).abs().max().item()
+    assert cuda_rel < 1.3e-4, cuda_rel
+    # inputs below -125 clamp to 2^-125, never wrap into large values
+    assert 0 < y[-2].item() < 1e-37 and 0 < y[-1].item() < 1e-37
