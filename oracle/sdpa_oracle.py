@@ -144,16 +144,19 @@ def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
 
 def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
                 window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
-                t5_max_distance=128, t5_bidirectional=True):
+                t5_max_distance=128, t5_bidirectional=True, rows=None):
     """Masked score matrix S for one (b, hq): scale * Q K^T + bias, -inf where
-    masked.  q: [B, L, Hq, d], k: [B, L, Hkv, d] float64 arrays."""
+    masked.  q: [B, L, Hq, d], k: [B, L, Hkv, d] float64 arrays.  With
+    ``rows`` (an index array), only those query rows of S are formed."""
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     g = hq // (Hq // Hkv)
-    S = scale * (q[b, :, hq, :] @ k[b, :, g, :].T)
+    r = np.arange(L) if rows is None else np.asarray(rows)
+    S = scale * (q[b, r, hq, :] @ k[b, :, g, :].T)
     S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets,
-                         t5_max_distance, t5_bidirectional)
-    M = visibility_mask(L, causal, window_left, window_right)
+                         t5_max_distance, t5_bidirectional)[r] \
+        if (bias is not None or t5_table is not None) else S
+    M = visibility_mask(L, causal, window_left, window_right)[r]
     S = np.where(M, S, -np.inf)
     return S
 
@@ -193,7 +196,8 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
 def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
                       window_right=-1, bias=None, t5_table=None,
                       t5_num_buckets=32, t5_max_distance=128,
-                      t5_bidirectional=True, batches=None, kv_heads=None):
+                      t5_bidirectional=True, batches=None, kv_heads=None,
+                      query_rows=None):
     """O = softmax(scale Q K^T + bias, masked) V and LSE, in float64.
 
     q: [B, L, Hq, d]; k, v: [B, L, Hkv, d]; bias: [B|1, Hq|1, L, L] or None;
@@ -213,14 +217,15 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
               t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional)
+    r = np.arange(L) if query_rows is None else np.asarray(query_rows)
     bs, gs = _select(B, Hkv, batches, kv_heads)
     for b in bs:
         for g in gs:
             for hq in range(g * G, (g + 1) * G):
-                S = head_scores(q, k, b, hq, scale=sc, **kw)
+                S = head_scores(q, k, b, hq, scale=sc, rows=r, **kw)
                 P, lse = _softmax_rows(S)
-                O[b, :, hq, :] = P @ v[b, :, g, :]
-                LSE[b, hq, :] = lse
+                O[b, r, hq, :] = P @ v[b, :, g, :]
+                LSE[b, hq, r] = lse
     return O, LSE
 
 

@@ -29,25 +29,41 @@ def nvcc_path() -> str:
 
 
 def _deps():
-    out = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
+    out = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))]
     out.append(os.path.join(INCLUDE, "sdpa.h"))
     return out
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+STAMP_PATH = LIB_PATH + ".stamp"
+
+
+def _source_hash(flags) -> str:
+    import hashlib
+    h = hashlib.sha256(" ".join(flags).encode())
+    for d in sorted(_deps()):
+        if os.path.isfile(d):
+            h.update(os.path.relpath(d, ROOT).encode())
+            with open(d, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def up_to_date(flags=()) -> bool:
+    """The library exists and was built from exactly these sources and flags."""
+    if not (os.path.exists(LIB_PATH) and os.path.exists(STAMP_PATH)):
         return False
-    t = os.path.getmtime(LIB_PATH)
-    return all(os.path.getmtime(d) <= t for d in _deps())
+    with open(STAMP_PATH) as fh:
+        return fh.read().strip() == _source_hash(flags)
+
+
+FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
+         "-Xcompiler", "-fPIC", "-shared", "-cudart", "static"]
 
 
 def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and up_to_date():
+    if not force and up_to_date(FLAGS):
         return LIB_PATH
-    cmd = [
-        nvcc_path(), "-std=c++17", "-O3", "-lineinfo",
-        "-gencode", "arch=compute_100a,code=sm_100a",
-        "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
+    cmd = [nvcc_path()] + FLAGS + [
         "-I", INCLUDE, "-I", CSRC,
         "-o", LIB_PATH + ".tmp",
     ] + [os.path.join(CSRC, s) for s in SOURCES]
@@ -60,6 +76,8 @@ def build(verbose: bool = False, force: bool = False) -> str:
     if verbose:
         sys.stderr.write(r.stderr)
     os.replace(LIB_PATH + ".tmp", LIB_PATH)
+    with open(STAMP_PATH, "w") as fh:
+        fh.write(_source_hash(FLAGS) + "\n")
     return LIB_PATH
 
 

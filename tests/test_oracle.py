@@ -208,6 +208,17 @@ def test_gqa_equals_mha_with_repeated_kv(Hkv):
     assert np.allclose(dv, dvr.reshape(2, 12, Hkv, G, 8).sum(3), atol=1e-13)
 
 
+def test_row_subset_matches_full():
+    q, k, v, _ = qkv(L=20)
+    table = rnd((32, 4), 2)
+    O, LSE = attention_forward(q, k, v, causal=True, window_left=6, t5_table=table)
+    rows = [0, 3, 19, 7]
+    Os, LSEs = attention_forward(q, k, v, causal=True, window_left=6, t5_table=table,
+                                 query_rows=rows, batches=[1])
+    assert np.array_equal(Os[1, rows], O[1, rows]) and np.array_equal(LSEs[1][:, rows], LSE[1][:, rows])
+    assert np.isnan(Os[1, 1]).all() and np.isnan(Os[0]).all()
+
+
 def test_subset_matches_full():
     q, k, v, do = qkv()
     O, LSE = attention_forward(q, k, v, causal=True)
