@@ -33,7 +33,12 @@ namespace sdpa {
 constexpr float kRescaleThreshold = 8.0f;
 // Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all): the
 // forward measured fastest with every exponential on MUFU.
-constexpr int kFwdMufuPer8 = 8;  // log2 units: rescale O when max grows > 2^8
+constexpr int kFwdMufuPer8 = 8;
+// Full tiles without a bias take the lean path: the row max is taken on the
+// raw scores (scale > 0 preserves the order), the scale folds into the one
+// fused multiply-add that forms each exponent, and pairs of columns go
+// through the packed fp32x2 FMA / add of sm_100.
+constexpr bool kFwdLeanSoftmax = true;  // log2 units: rescale O when max grows > 2^8
 
 template <int D, int NQ>
 struct FwdLayout {
@@ -284,67 +289,113 @@ __global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
       // x: scores in log2 units, in place over the raw accumulator bits
       uint32_t x[128];
       tmem_ld128_sync(tS, x);
-      // four independent max / sum chains instead of one 128 long
-      float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      const float* bcol = brow ? brow + n0 : nullptr;
-      if (full) {
+      float sum, alpha, m_use;
+      bool grow;
+      if (kFwdLeanSoftmax && BIAS == kBiasNone && full && p.scale_log2 > 0.f) {
+        // ---- lean path: raw max (3-input), exponent = fma(s, c, -m)
+        float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          float v = __uint_as_float(x[c]) * p.scale_log2;
-          if constexpr (BIAS != kBiasNone) v += bias_log2<BIAS>(lut_row, bcol, c);
-          x[c] = __float_as_uint(v);
-          tm[c & 3] = fmaxf(tm[c & 3], v);
+        for (int c = 0; c < kTile; c += 4) {
+          ma = fmax3(ma, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+          mb = fmax3(mb, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const bool vis = (c >= lo) && (c <= hi);
-          float v = __uint_as_float(x[c]) * p.scale_log2;
-          if constexpr (BIAS == kBiasT5) v += lut_row[c];
-          if constexpr (BIAS == kBiasDense) v += vis ? bcol[c] * kLog2e : 0.f;
-          v = vis ? v : -INFINITY;
-          x[c] = __float_as_uint(v);
-          tm[c & 3] = fmaxf(tm[c & 3], v);
-        }
-      }
-      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
-      const float m_new = fmaxf(m_run, tmax);
-      const bool grow = m_new > m_run + kRescaleThreshold;
-      const float m_use = grow ? m_new : m_run;
-      const float alpha = grow ? fast_exp2(m_run - m_use) : 1.f;
-      const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-      float sm[4] = {0.f, 0.f, 0.f, 0.f};
-      if (full) {
-        // every entry is finite: a fixed share of the exponentials on the FMA pipe
+        const float tmax = fmaxf(ma, mb) * p.scale_log2;
+        const float m_new = fmaxf(m_run, tmax);
+        grow = m_new > m_run + kRescaleThreshold;
+        m_use = grow ? m_new : m_run;
+        alpha = grow ? fast_exp2(m_run - m_use) : 1.f;
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-m_use, -m_use);  // m_use is finite in a full tile
+        uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int c0 = 0; c0 < kTile; c0 += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float v0 = __uint_as_float(x[c0 + c]) - m_sub;
-            const float v1 = __uint_as_float(x[c0 + c + 1]) - m_sub;
+            const uint64_t arg = f2_fma(f2_pack(__uint_as_float(x[c0 + c]), __uint_as_float(x[c0 + c + 1])),
+                                        c2, nm2);
+            float v0, v1;
+            f2_unpack(arg, v0, v1);
             const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
             const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
-            sm[(c >> 1) & 3] += e0 + e1;
+            const uint64_t e2 = f2_pack(e0, e1);
+            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e2);
             pk[c >> 1] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
         }
+        float s0, s1, s2, s3, s4, s5, s6, s7;
+        f2_unpack(acc[0], s0, s1);
+        f2_unpack(acc[1], s2, s3);
+        f2_unpack(acc[2], s4, s5);
+        f2_unpack(acc[3], s6, s7);
+        sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       } else {
-#pragma unroll
-        for (int c0 = 0; c0 < kTile; c0 += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float e0 = fast_exp2(__uint_as_float(x[c0 + c]) - m_sub);
-            const float e1 = fast_exp2(__uint_as_float(x[c0 + c + 1]) - m_sub);
-            sm[(c >> 1) & 3] += e0 + e1;
-            pk[c >> 1] = pack_bf16x2(e0, e1);
+        // four independent max / sum chains instead of one 128 long
+        float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const float* bcol = brow ? brow + n0 : nullptr;
+        if (full) {
+  #pragma unroll
+          for (int c = 0; c < kTile; ++c) {
+            float v = __uint_as_float(x[c]) * p.scale_log2;
+            if constexpr (BIAS != kBiasNone) v += bias_log2<BIAS>(lut_row, bcol, c);
+            x[c] = __float_as_uint(v);
+            tm[c & 3] = fmaxf(tm[c & 3], v);
           }
-          tmem_st16(tS + (c0 >> 1), pk);
+        } else {
+  #pragma unroll
+          for (int c = 0; c < kTile; ++c) {
+            const bool vis = (c >= lo) && (c <= hi);
+            float v = __uint_as_float(x[c]) * p.scale_log2;
+            if constexpr (BIAS == kBiasT5) v += lut_row[c];
+            if constexpr (BIAS == kBiasDense) v += vis ? bcol[c] * kLog2e : 0.f;
+            v = vis ? v : -INFINITY;
+            x[c] = __float_as_uint(v);
+            tm[c & 3] = fmaxf(tm[c & 3], v);
+          }
         }
+        const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+        const float m_new = fmaxf(m_run, tmax);
+        const bool grow_g = m_new > m_run + kRescaleThreshold;
+        const float m_use_g = grow_g ? m_new : m_run;
+        const float alpha_g = grow_g ? fast_exp2(m_run - m_use_g) : 1.f;
+        const float m_sub = (m_use_g == -INFINITY) ? 0.f : m_use_g;
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
+        if (full) {
+          // every entry is finite: a fixed share of the exponentials on the FMA pipe
+  #pragma unroll
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float v0 = __uint_as_float(x[c0 + c]) - m_sub;
+              const float v1 = __uint_as_float(x[c0 + c + 1]) - m_sub;
+              const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
+              const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
+              sm[(c >> 1) & 3] += e0 + e1;
+              pk[c >> 1] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
+          }
+        } else {
+  #pragma unroll
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float e0 = fast_exp2(__uint_as_float(x[c0 + c]) - m_sub);
+              const float e1 = fast_exp2(__uint_as_float(x[c0 + c + 1]) - m_sub);
+              sm[(c >> 1) & 3] += e0 + e1;
+              pk[c >> 1] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + (c0 >> 1), pk);
+          }
+        }
+        sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+        grow = grow_g;
+        alpha = alpha_g;
+        m_use = m_use_g;
       }
-      const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
       l_run = l_run * alpha + sum;
       m_run = m_use;
       tmem_st_wait();
