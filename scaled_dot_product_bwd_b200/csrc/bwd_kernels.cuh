@@ -105,11 +105,13 @@ struct DkdvLayout {
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], vec_full[2],
-  // vec_empty[2], s_full, dp_full, p_full, ds_full, s_free, dp_free, acc_done, drain
-  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 8;
+  // vec_empty[2], s_full, dp_full, p_full, ds_full, s_free, dp_free, acc_done,
+  // drain[2]
+  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 9;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
-  static constexpr int kThreads = 320;  // 2 compute warpgroups, producer, MMA
+  // 2 compute warpgroups, producer, two MMA issuers
+  static constexpr int kThreads = 352;
   static constexpr int kTmemCols = 512;
   static constexpr int kSCol = 0, kDPCol = 128, kDVCol = 256, kDKCol = 256 + D;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -123,7 +125,7 @@ __device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
 }
 
 template <int D, int BIAS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_dkdv_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmDO) {
@@ -163,19 +165,21 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t s_free = bar(kB + 8);
   const uint32_t dp_free = bar(kB + 9);
   const uint32_t acc_done = bar(kB + 10);
-  const uint32_t drain = bar(kB + 11);
+  auto drain = [&](int x) { return bar(kB + 11 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    // Q blocks are read by both issuers (S^T and dK), dO blocks too (dP^T and
+    // dV): a slot is free once each issuer's last MMA on it has completed.
     for (int s = 0; s < SQ; ++s) {
       mbar_init(q_full(s), 1);
-      mbar_init(q_empty(s), 1);
+      mbar_init(q_empty(s), 2);
     }
     for (int s = 0; s < SO; ++s) {
       mbar_init(o_full(s), 1);
-      mbar_init(o_empty(s), 1);
+      mbar_init(o_empty(s), 2);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(vec_full(x), 32);          // the producer warp's lanes
@@ -187,8 +191,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(ds_full, 2 * kTile);
     mbar_init(s_free, 1);
     mbar_init(dp_free, 1);
-    mbar_init(acc_done, 1);
-    mbar_init(drain, 1);
+    mbar_init(acc_done, 2);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -243,16 +248,8 @@ __global__ void __launch_bounds__(320, 1)
         const int hq = g * p.G + it / nm;
         const int m0 = (mlo + it % nm) * kTile;
         const int x = it & 1;
-        if (ok) ok = mbar_wait(vec_empty(x), ((it >> 1) & 1) ^ 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        float* lse2 = vec + x * 2 * kTile;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          lse2[lane + 32 * e] = l2v[e];
-          lse2[kTile + lane + 32 * e] = ddv[e];
-        }
-        mbar_arrive(vec_full(x));
+        // The Q / dO copies go first: they wait only for their ring slots,
+        // not for the compute warps, so they run as far ahead as the rings allow.
         if (lane == 0) {
           const int sq = it % SQ, so = it % SO;
           ok = mbar_wait(q_empty(sq), ((it / SQ) & 1) ^ 1, ctl);
@@ -274,6 +271,16 @@ __global__ void __launch_bounds__(320, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
+        if (ok) ok = mbar_wait(vec_empty(x), ((it >> 1) & 1) ^ 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float* lse2 = vec + x * 2 * kTile;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          lse2[lane + 32 * e] = l2v[e];
+          lse2[kTile + lane + 32 * e] = ddv[e];
+        }
+        mbar_arrive(vec_full(x));
         if (it + 1 < total) load_vec(it + 1);
       }
       if (!ok && lane == 0) {
@@ -286,76 +293,72 @@ __global__ void __launch_bounds__(320, 1)
           if (issued_o[s] >= 0) mbar_wait(o_full(s), issued_o[s], ign);
       }
     }
-  } else if (warp == 9) {
-    // ============================ MMA issuer ============================
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers (one thread each) =====================
+    // Warp 9 owns the S^T chain: S^T(i), then dV(i) once P^T(i) is ready, then
+    // S^T(i+1) once dV(i) has read P^T(i) out of the S^T columns.  Warp 10 owns
+    // the dP^T chain: dP^T(i), dK(i) once dS^T(i) is ready, dP^T(i+1) once dK(i)
+    // is done.  Neither waits on the other's barriers, so a stalled chain does
+    // not hold up MMAs that are ready in the other.
     if (lane == 0 && total > 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 keys x 128 queries
       constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // 128 keys x d
-      auto issue_s = [&](int jb) -> bool {
-        const int sq = jb % SQ;
-        const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
-        if (!mbar_wait(q_full(sq), (jb / SQ) & 1, ctl)) return false;
-        // S^T held P^T of the previous block: wait for that block's dV MMA
-        if (jb > 0 && !mbar_wait(s_free, (jb - 1) & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + Lay::kSCol, smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        return true;
-      };
-      auto issue_dp = [&](int jb) -> bool {
-        const int so = jb % SO;
-        const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
-        if (!mbar_wait(o_full(so), (jb / SO) & 1, ctl)) return false;
-        // dP^T held dS^T of the previous block: wait for that block's dK MMA
-        if (jb > 0 && !mbar_wait(dp_free, (jb - 1) & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + Lay::kDPCol,
-                 smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(dp_full);
-        return true;
-      };
-      // Order per block: dV(i), S(i+1), dK(i), dP(i+1): the scores of the
-      // next block are ready while this block's dK runs, so its exponentials
-      // overlap dK(i) and dP(i+1).
+      const bool chain_s = (warp == 9);
       bool ok = mbar_wait(kv_full, 0, ctl);
-      ok = ok && issue_s(0) && issue_dp(0);
       for (int it = 0; it < total && ok; ++it) {
         const int sq = it % SQ, so = it % SO;
         const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
         const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
-        if (!(ok = mbar_wait(p_full, it & 1, ctl))) break;
-        tc_fence_after();
+        if (chain_s) {
+          if (!(ok = mbar_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (it > 0 && !(ok = mbar_wait(s_free, (it - 1) & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
-                 smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(s_free);
-        mma_commit(o_empty(so));
-        if (it + 1 < total && !(ok = issue_s(it + 1))) break;
-        if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
-        tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + Lay::kSCol,
+                   smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(s_full);
+          mma_commit(q_empty(sq));
+          if (!(ok = mbar_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (!(ok = mbar_wait(p_full, it & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk),
-                 smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(dp_free);
-        mma_commit(q_empty(sq));
-        if (it + 1 < total && !(ok = issue_dp(it + 1))) break;
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
+                   smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(s_free);
+          mma_commit(o_empty(so));
+        } else {
+          if (!(ok = mbar_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (it > 0 && !(ok = mbar_wait(dp_free, (it - 1) & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + Lay::kDPCol,
+                   smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(dp_full);
+          mma_commit(o_empty(so));
+          if (!(ok = mbar_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk),
+                   smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(dp_free);
+          mma_commit(q_empty(sq));
+        }
       }
       if (ok) mma_commit(acc_done);
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mma_commit(drain);
-        mbar_wait(drain, 0, ign);
+        mma_commit(drain(chain_s ? 0 : 1));
+        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
       }
     }
   } else {
@@ -541,18 +544,18 @@ struct DqLayout {
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_used[2],
-  // dp_full, ds_full, dq_done, acc_done, drain
-  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 9;
+  // dp_full, ds_full, dq_done, acc_done, drain[2]
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;  // 2 compute warpgroups, producer, two MMA issuers
   static constexpr int kTmemCols = 512;
   static constexpr int kDPCol = 256, kDQCol = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
 template <int D, int BIAS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmDO) {
@@ -591,15 +594,17 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t ds_full = bar(kB + 5);
   const uint32_t dq_done = bar(kB + 6);
   const uint32_t acc_done = bar(kB + 7);
-  const uint32_t drain = bar(kB + 8);
+  auto drain = [&](int x) { return bar(kB + 8 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    // K blocks are read by both issuers (S and dQ): a slot is free once each
+    // issuer's last MMA on it has completed.
     for (int s = 0; s < SK; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
+      mbar_init(k_empty(s), 2);
     }
     for (int s = 0; s < SV; ++s) {
       mbar_init(v_full(s), 1);
@@ -613,7 +618,8 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(ds_full, 2 * kTile);
     mbar_init(dq_done, 1);
     mbar_init(acc_done, 1);
-    mbar_init(drain, 1);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -667,70 +673,61 @@ __global__ void __launch_bounds__(320, 1)
           if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
       }
     }
-  } else if (warp == 9) {
-    // ============================ MMA issuer ============================
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers (one thread each) =====================
+    // Warp 9 runs the score chain ahead: S(i) into buffer i % 2 as soon as K(i)
+    // has landed and both warpgroups have loaded S(i-2) out of that buffer.
+    // Warp 10 runs dP(i), then dQ(i) once dS(i) is ready, then dP(i+1) once
+    // dQ(i) has read dS(i) out of the dP columns.
     if (lane == 0 && nt > 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
-      auto issue_s = [&](int jb) -> bool {
-        const int x = jb & 1;
-        const int sk = jb % SK;
-        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
-        if (!mbar_wait(k_full(sk), (jb / SK) & 1, ctl)) return false;
-        // S[x] held block jb-2: both warpgroups must have loaded it
-        if (jb >= 2 && !mbar_wait(s_used(x), ((jb >> 1) - 1) & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kTile * x,
-                 smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(s_full(x));
-        return true;
-      };
-      auto issue_dp = [&](int jb) -> bool {
-        const int sv = jb % SV;
-        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
-        if (!mbar_wait(v_full(sv), (jb / SV) & 1, ctl)) return false;
-        // dP held dS of block jb-1: wait for that block's dQ MMA
-        if (jb >= 1 && !mbar_wait(dq_done, (jb - 1) & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + Lay::kDPCol,
-                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(dp_full);
-        mma_commit(v_empty(sv));
-        return true;
-      };
-      auto issue_dq = [&](int jb) -> bool {
-        const int sk = jb % SK;
-        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
-        if (!mbar_wait(ds_full, jb & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + Lay::kDPCol, kk),
-                 smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
-                 (jb > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(dq_done);
-        mma_commit(k_empty(sk));
-        return true;
-      };
+      const bool chain_s = (warp == 9);
       bool ok = mbar_wait(q_full, 0, ctl);
-      ok = ok && issue_s(0) && issue_dp(0);
       for (int it = 0; it < nt && ok; ++it) {
-        if (it + 1 < nt && !(ok = issue_s(it + 1))) break;
-        if (!(ok = issue_dq(it))) break;
-        if (it + 1 < nt && !(ok = issue_dp(it + 1))) break;
+        const int x = it & 1;
+        const int sk = it % SK, sv = it % SV;
+        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+        if (!(ok = mbar_wait(k_full(sk), (it / SK) & 1, ctl))) break;
+        if (chain_s) {
+          if (it >= 2 && !(ok = mbar_wait(s_used(x), ((it >> 1) - 1) & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + kTile * x,
+                   smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(s_full(x));
+          mma_commit(k_empty(sk));
+        } else {
+          if (!(ok = mbar_wait(v_full(sv), (it / SV) & 1, ctl))) break;
+          if (it > 0 && !(ok = mbar_wait(dq_done, (it - 1) & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + Lay::kDPCol,
+                   smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(dp_full);
+          mma_commit(v_empty(sv));
+          if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + Lay::kDPCol, kk),
+                   smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(dq_done);
+          mma_commit(k_empty(sk));
+        }
       }
-      if (ok) mma_commit(acc_done);
+      if (ok && !chain_s) mma_commit(acc_done);
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mma_commit(drain);
-        mbar_wait(drain, 0, ign);
+        mma_commit(drain(chain_s ? 0 : 1));
+        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
       }
     }
   } else {
