@@ -19,9 +19,10 @@
  * Heads.  Hq query heads share Hkv key/value heads in contiguous groups:
  *   query head h reads KV head h / (Hq / Hkv) (MHA Hkv = Hq, GQA, MQA
  *   Hkv = 1; codelab section 9).  Hq % Hkv must be 0.
- * Supported.  head_dim d in {64, 128}; 1 <= L < 2^30; every bf16 base pointer
- *   16-byte aligned; every stride a multiple of 8 elements (16 bytes) except
- *   the contiguous head_dim.  Anything else returns SDPA_ERR_UNSUPPORTED or
+ * Supported.  head_dim d in {64, 128}; 1 <= L < 2^30; B, Hq <= 65535;
+ *   ceil(L / 128) * Hq * B < 2^31 (query tiles are counted in 32 bits);
+ *   every bf16 base pointer 16-byte aligned; every stride a multiple of 8
+ *   elements (16 bytes) except the contiguous head_dim.  Anything else returns SDPA_ERR_UNSUPPORTED or
  *   SDPA_ERR_INVALID_ARG before any work is queued.
  * Ownership.  The caller owns every buffer.  No entry point allocates,
  *   frees, or synchronises the stream, except sdpa_read_device_status.

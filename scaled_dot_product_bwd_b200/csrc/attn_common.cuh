@@ -12,6 +12,7 @@
 namespace sdpa {
 
 constexpr int kTile = 128;             // query rows and keys per tile
+constexpr int kBlk = 64;               // columns per compute warpgroup in a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxT5Thresholds = 64;
@@ -145,6 +146,19 @@ __device__ __forceinline__ void key_visible_rows(const AttnParams& p, int j, int
   if (p.wr >= 0) lo = max(lo, j - p.wr - m0);
   hi = min(kTile - 1, p.L - 1 - m0);
   if (p.wl >= 0) hi = min(hi, j + p.wl - m0);
+}
+
+// Byte offset of the 16-element K step kk inside a K-major SW128 tile of
+// `rows` rows: a d = 128 tile is two 64-column halves of rows x 128 bytes.
+__device__ __forceinline__ uint32_t kmajor_koff(int kk, int rows) {
+  return static_cast<uint32_t>((kk >> 2) * rows * 128 + (kk & 3) * 32);
+}
+
+// TMEM column of the bf16 A operand for the 16-row K step kk of a 128-wide
+// block whose two 64-wide halves were written by the two warpgroups into the
+// first 32 columns of their own 64-column regions starting at `base`.
+__device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
+  return base + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
 }
 
 }  // namespace sdpa

@@ -31,7 +31,6 @@
 
 namespace sdpa {
 
-constexpr int kBlk = 64;  // columns per compute warpgroup in a 128-wide tile
 // Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all),
 // chosen by measurement: the dK/dV kernel gains from moving 3 of 8 to the
 // FMA pipe, the dQ kernel does not.
@@ -75,11 +74,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p)
   if (part == 0 && r < nrows) p.dvec[(static_cast<int64_t>(b) * p.Hq + h) * p.L + i] = acc;
 }
 
-// Byte offset of the 16-element K step kk inside a K-major SW128 tile of
-// `rows` rows: a d = 128 tile is two 64-column halves of rows x 128 bytes.
-__device__ __forceinline__ uint32_t kmajor_koff(int kk, int rows) {
-  return static_cast<uint32_t>((kk >> 2) * rows * 128 + (kk & 3) * 32);
-}
 
 // ------------------------------------------------------------------ dK / dV
 // CTA = 128 keys of one (KV head, batch).  Blocks of 128 queries stream
@@ -117,12 +111,6 @@ struct DkdvLayout {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-// TMEM column of the bf16 A operand for the 16-row K step kk of a 128-wide
-// block whose two 64-wide halves were written by the two warpgroups into the
-// first 32 columns of their own 64-column regions starting at `base`.
-__device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
-  return base + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-}
 
 template <int D, int BIAS>
 __global__ void __launch_bounds__(352, 1)
@@ -304,14 +292,14 @@ __global__ void __launch_bounds__(352, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 keys x 128 queries
       constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // 128 keys x d
       const bool chain_s = (warp == 9);
-      bool ok = mbar_wait(kv_full, 0, ctl);
+      bool ok = issuer_wait(kv_full, 0, ctl);
       for (int it = 0; it < total && ok; ++it) {
         const int sq = it % SQ, so = it % SO;
         const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
         const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
         if (chain_s) {
-          if (!(ok = mbar_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
-          if (it > 0 && !(ok = mbar_wait(s_free, (it - 1) & 1, ctl))) break;
+          if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (it > 0 && !(ok = issuer_wait(s_free, (it - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -320,8 +308,8 @@ __global__ void __launch_bounds__(352, 1)
                    smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
           mma_commit(s_full);
           mma_commit(q_empty(sq));
-          if (!(ok = mbar_wait(o_full(so), (it / SO) & 1, ctl))) break;
-          if (!(ok = mbar_wait(p_full, it & 1, ctl))) break;
+          if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (!(ok = issuer_wait(p_full, it & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
@@ -331,8 +319,8 @@ __global__ void __launch_bounds__(352, 1)
           mma_commit(s_free);
           mma_commit(o_empty(so));
         } else {
-          if (!(ok = mbar_wait(o_full(so), (it / SO) & 1, ctl))) break;
-          if (it > 0 && !(ok = mbar_wait(dp_free, (it - 1) & 1, ctl))) break;
+          if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (it > 0 && !(ok = issuer_wait(dp_free, (it - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -341,8 +329,8 @@ __global__ void __launch_bounds__(352, 1)
                    smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
           mma_commit(dp_full);
           mma_commit(o_empty(so));
-          if (!(ok = mbar_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
-          if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
+          if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (!(ok = issuer_wait(ds_full, it & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
@@ -683,15 +671,15 @@ __global__ void __launch_bounds__(352, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
       const bool chain_s = (warp == 9);
-      bool ok = mbar_wait(q_full, 0, ctl);
+      bool ok = issuer_wait(q_full, 0, ctl);
       for (int it = 0; it < nt && ok; ++it) {
         const int x = it & 1;
         const int sk = it % SK, sv = it % SV;
         const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
         const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
-        if (!(ok = mbar_wait(k_full(sk), (it / SK) & 1, ctl))) break;
+        if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
         if (chain_s) {
-          if (it >= 2 && !(ok = mbar_wait(s_used(x), ((it >> 1) - 1) & 1, ctl))) break;
+          if (it >= 2 && !(ok = issuer_wait(s_used(x), ((it >> 1) - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -701,8 +689,8 @@ __global__ void __launch_bounds__(352, 1)
           mma_commit(s_full(x));
           mma_commit(k_empty(sk));
         } else {
-          if (!(ok = mbar_wait(v_full(sv), (it / SV) & 1, ctl))) break;
-          if (it > 0 && !(ok = mbar_wait(dq_done, (it - 1) & 1, ctl))) break;
+          if (!(ok = issuer_wait(v_full(sv), (it / SV) & 1, ctl))) break;
+          if (it > 0 && !(ok = issuer_wait(dq_done, (it - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -711,7 +699,7 @@ __global__ void __launch_bounds__(352, 1)
                    smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
           mma_commit(dp_full);
           mma_commit(v_empty(sv));
-          if (!(ok = mbar_wait(ds_full, it & 1, ctl))) break;
+          if (!(ok = issuer_wait(ds_full, it & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)

@@ -1,21 +1,38 @@
 // fwd_kernel.cuh -- fused attention forward for sm_100a.
 //
-// One CTA owns NQ query tiles of 128 rows of one (batch, query head) and
-// streams the key/value tiles of the mask band through shared memory:
+// Persistent: one CTA per SM walks a list of work items -- a tile of 128
+// query rows of one (batch, query head), heaviest causal tiles first -- and
+// for each streams the key/value tiles of the mask band through shared memory.
+// Every ring and buffer index below counts across items, so the producers and
+// the S issuer run on into the next item while the softmax warps finish the
+// current one:
 //
-//   producer warp   TMA: the NQ Q tiles once, then K_j and V_j into a ring of
-//                   kStages stages (fully masked key tiles are never loaded --
-//                   the point of HF transformers issue #30461: a mask handed
-//                   over as a dense tensor forfeits this skipping).
-//   MMA warp        one thread issues tcgen05.mma: S_t = Q_t K_j^T into tensor
-//                   memory, then O_t += P_t V_j with P_t read from tensor memory.
-//   softmax warps   one warpgroup per Q tile, one thread per query row (its
-//                   TMEM lane): scale (log2e folded in), bias, mask at band
-//                   edges, running max / sum, exp2, P_t back to tensor memory as
-//                   bf16; O_t is rescaled in tensor memory only when the row
-//                   max grows by more than 2^8 (exact: O and the sum always
-//                   share the same reference max).  Epilogue: O = acc / sum ->
-//                   bf16, LSE = (max + log2 sum) ln 2.
+//   K producer warp   TMA: the item's Q tile (once the previous item's last S
+//                     MMA has read the single Q buffer), then K_j into a ring
+//                     of kSK stages
+//                     (fully masked key tiles are never loaded -- the point of
+//                     HF transformers issue #30461: a mask handed over as a
+//                     dense tensor forfeits this skipping).
+//   V producer warp   TMA: V_j into a ring of kSV stages.
+//   S issuer          one thread: S_j = Q K_j^T into tensor-memory buffer
+//                     j mod 3, as soon as K_j has landed and the P V MMA of
+//                     tile j - 3 has finished reading that buffer.
+//   PV issuer         one thread: O += P_j V_j with P_j read from tensor memory.
+//   softmax warps     two warpgroups, thread = query row (its TMEM lane);
+//                     warpgroup w owns the key columns [64 w, 64 w + 64) of
+//                     every tile.  Per tile: load its half of S_j, take the
+//                     partial row max, exchange it with the other warpgroup
+//                     through shared memory, then scale (log2 e folded in),
+//                     bias, band-edge mask, exp2, P_j back to tensor memory as
+//                     bf16 over its own S columns.  O is rescaled in tensor
+//                     memory only when the row max grows by more than 2^8
+//                     (exact: O and the row sum always share one reference
+//                     max); each warpgroup rescales half of O's columns.
+//                     Epilogue: O = acc / sum -> bf16, LSE = (max + log2 sum) ln 2.
+//
+// Tensor memory (512 columns): S buffers at 0, 128, 256; O at 384 (d columns).
+// Three S buffers let the tensor core compute S_{j+1} and S_{j+2} while the
+// softmax of tile j runs, so neither side waits on the other's latency.
 //
 // Definition: codelab "jax-gpu-05-attention-gpu", sections 1 and 4 (score,
 // scale, softmax, weighted sum); section 7 (causal masking); transformers
@@ -30,108 +47,125 @@
 
 namespace sdpa {
 
-constexpr float kRescaleThreshold = 8.0f;
-// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all): the
-// forward measured fastest with every exponential on MUFU.
-constexpr int kFwdMufuPer8 = 8;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
+// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all): with
+// both warpgroups on one tile, 6 of 8 on MUFU and 2 on the FMA pipe measured
+// fastest (5 and 4 were slower).
+constexpr int kFwdMufuPer8 = 6;
 // Full tiles without a bias take the lean path: the row max is taken on the
 // raw scores (scale > 0 preserves the order), the scale folds into the one
 // fused multiply-add that forms each exponent, and pairs of columns go
 // through the packed fp32x2 FMA / add of sm_100.
-constexpr bool kFwdLeanSoftmax = true;  // log2 units: rescale O when max grows > 2^8
+constexpr bool kFwdLeanSoftmax = true;
+// Named barriers: 1, 2 guard each warpgroup's T5 bias table; 3 is the
+// row-max / row-sum exchange between the two warpgroups.
+constexpr uint32_t kXchgBar = 3;
 
-template <int D, int NQ>
+template <int D, int BIAS>
 struct FwdLayout {
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kNS = 3;                     // S buffers in tensor memory
+  // K is needed up to three tiles ahead of V (the S buffers run ahead of P V).
+  static constexpr int kSK = (D == 128) ? 3 : 4;
+  static constexpr int kSV = (D == 128) ? 2 : 4;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + NQ * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kLutOff = kVOff + kStages * kTileBytes;  // NQ x 2 x 256 floats
-  static constexpr int kBarOff = kLutOff + NQ * 2 * 256 * 4;
-  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQ], p_full[NQ], o_done[NQ],
-  // drain
-  static constexpr int kNumBars = 2 + 4 * kStages + 3 * NQ;
+  static constexpr int kKOff = kTileBytes;
+  static constexpr int kVOff = kKOff + kSK * kTileBytes;
+  static constexpr int kRedOff = kVOff + kSV * kTileBytes;  // max[2][2][128], sum[2][2][128]
+  static constexpr int kRedBytes = 8 * kTile * 4;
+  static constexpr int kLutOff = kRedOff + kRedBytes;       // T5 only: 2 WG x 2 x 256 floats
+  static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
+  static constexpr int kBarOff = kLutOff + kLutBytes;
+  // q_full, q_empty, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
+  // s_full[NS], p_full[NS], pv_done[NS], acc_done, drain[2]
+  static constexpr int kNumBars = 2 + 2 * kSK + 2 * kSV + 3 * kNS + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
-  static constexpr int kSmemAlloc = kBytes + 1024;  // slack for 1024-byte alignment
-  static constexpr int kThreads = NQ * 128 + 64;
-  static constexpr int kTmemCols = (NQ * (128 + D) <= 256) ? 256 : 512;
-  static constexpr int kOCol = NQ * 128;            // O_t at kOCol + t * D, S_t at t * 128
+  static constexpr int kSmemAlloc = kMiscOff + 16;
+  // 2 softmax warpgroups; warp 8 K producer, 9 S issuer, 10 PV issuer, 11 V producer
+  static constexpr int kThreads = 384;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol = kNS * kTile;
+  static_assert(kOCol + D <= kTmemCols, "tensor memory budget");
+  static_assert(kSK <= 4 && kSV <= 4, "producer bookkeeping");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-// Bias term of one score row, in log2 units, for the 128 columns of a tile.
-template <int BIAS>
-__device__ __forceinline__ float bias_log2(const float* lut_row, const float* brow, int c) {
-  if constexpr (BIAS == kBiasT5) return lut_row[c];
-  if constexpr (BIAS == kBiasDense) return brow[c] * kLog2e;
-  return 0.f;
-}
-
-template <int D, int NQ, int BIAS>
-__global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
+template <int D, int BIAS>
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
-  using Lay = FwdLayout<D, NQ>;
-  constexpr int S = Lay::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  using Lay = FwdLayout<D, BIAS>;
+  constexpr int SK = Lay::kSK;
+  constexpr int SV = Lay::kSV;
+  constexpr int NS = Lay::kNS;
+  extern __shared__ uint8_t smem[];
+  if (!smem_base_ok(smem)) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusMisaligned);
+    return;
+  }
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- tile coordinates: heaviest causal query blocks first
-  const int rows_cta = kTile * NQ;
-  const int nqb = (p.L + rows_cta - 1) / rows_cta;
-  const int qb = p.causal ? (nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int hq = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = hq / p.G;
-  const int m0 = qb * rows_cta;
-  int nlo, nhi;
-  key_tile_range(p, m0, rows_cta, nlo, nhi);
-  int tlo[NQ], thi[NQ];  // key-tile range of each Q tile (a sub-range of [nlo, nhi))
-#pragma unroll
-  for (int t = 0; t < NQ; ++t) {
-    if (m0 + t * kTile < p.L) {
-      key_tile_range(p, m0 + t * kTile, kTile, tlo[t], thi[t]);
-    } else {
-      tlo[t] = nlo;
-      thi[t] = nlo;  // entirely past L: nothing to compute
-    }
-  }
-  const int nt = nhi - nlo;
+  // ---- work items: (query tile, head, batch), heaviest causal query tiles
+  // first; consecutive items are neighbouring heads, which share K / V in L2.
+  const int nqt = (p.L + kTile - 1) / kTile;
+  const int heads = p.Hq * p.B;
+  const int n_items = nqt * heads;
+  struct Item {
+    int m0, hq, b, g, nlo, nt;
+  };
+  auto item_at = [&](int id) {
+    Item w;
+    const int r = id / heads;
+    const int rem = id - r * heads;
+    const int qt = p.causal ? nqt - 1 - r : r;
+    w.m0 = qt * kTile;
+    w.hq = rem % p.Hq;
+    w.b = rem / p.Hq;
+    w.g = w.hq / p.G;
+    int nhi;
+    key_tile_range(p, w.m0, kTile, w.nlo, nhi);
+    w.nt = nhi > w.nlo ? nhi - w.nlo : 0;
+    return w;
+  };
 
   // ---- barriers
   auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
   const uint32_t q_full = bar(0);
-  auto k_full = [&](int s) { return bar(1 + s); };
-  auto k_empty = [&](int s) { return bar(1 + S + s); };
-  auto v_full = [&](int s) { return bar(1 + 2 * S + s); };
-  auto v_empty = [&](int s) { return bar(1 + 3 * S + s); };
-  auto s_full = [&](int t) { return bar(1 + 4 * S + t); };
-  auto p_full = [&](int t) { return bar(1 + 4 * S + NQ + t); };
-  auto o_done = [&](int t) { return bar(1 + 4 * S + 2 * NQ + t); };
-  const uint32_t drain = bar(1 + 4 * S + 3 * NQ);
+  const uint32_t q_empty = bar(1);
+  auto k_full = [&](int s) { return bar(2 + s); };
+  auto k_empty = [&](int s) { return bar(2 + SK + s); };
+  auto v_full = [&](int s) { return bar(2 + 2 * SK + s); };
+  auto v_empty = [&](int s) { return bar(2 + 2 * SK + SV + s); };
+  constexpr int kB = 2 + 2 * SK + 2 * SV;
+  auto s_full = [&](int x) { return bar(kB + x); };
+  auto p_full = [&](int x) { return bar(kB + NS + x); };
+  auto pv_done = [&](int x) { return bar(kB + 2 * NS + x); };
+  const uint32_t acc_done = bar(kB + 3 * NS);
+  auto drain = [&](int x) { return bar(kB + 3 * NS + 1 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < SK; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < SV; ++s) {
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    for (int t = 0; t < NQ; ++t) {
-      mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), kTile);
-      mbar_init(o_done(t), 1);
+    for (int x = 0; x < NS; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(p_full(x), 2 * kTile);
+      mbar_init(pv_done(x), 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(acc_done, 1);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -145,309 +179,351 @@ __global__ void __launch_bounds__(FwdLayout<D, NQ>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.wait_limit_ns};
 
-  if (warp == 4 * NQ) {
-    // =========================== producer (TMA) ===========================
-    if (lane == 0 && nt > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_expect_tx(q_full, NQ * Lay::kTileBytes);
-      for (int t = 0; t < NQ; ++t)
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(sb + Lay::kQOff + t * Lay::kTileBytes + h * 16384, &tmQ, q_full, h * 64,
-                      m0 + t * kTile, hq, b);
-      int issued_k[S], issued_v[S];
-      for (int s = 0; s < S; ++s) issued_k[s] = issued_v[s] = -1;
+  if (warp == 8 || warp == 11) {
+    // ===================== producers (TMA): K (+Q) and V =====================
+    const bool is_k = (warp == 8);
+    if (lane == 0) {
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      const int stages = is_k ? SK : SV;
+      const uint32_t ring = sb + (is_k ? Lay::kKOff : Lay::kVOff);
+      tma_prefetch_desc(map);
+      if (is_k) tma_prefetch_desc(&tmQ);
+      int issued[4] = {-1, -1, -1, -1};
+      int q_issued = -1;
+      int c = 0;  // tiles loaded so far, over all items
+      int u = 0;  // items with a non-empty band so far
       bool ok = true;
-      for (int it = 0; it < nt && ok; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        const int n0 = (nlo + it) * kTile;
-        if (!(ok = mbar_wait(k_empty(s), ph ^ 1, ctl))) break;
-        mbar_expect_tx(k_full(s), Lay::kTileBytes);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(sb + Lay::kKOff + s * Lay::kTileBytes + h * 16384, &tmK, k_full(s), h * 64,
-                      n0, g, b);
-        issued_k[s] = ph;
-        if (!(ok = mbar_wait(v_empty(s), ph ^ 1, ctl))) break;
-        mbar_expect_tx(v_full(s), Lay::kTileBytes);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(sb + Lay::kVOff + s * Lay::kTileBytes + h * 16384, &tmV, v_full(s), h * 64,
-                      n0, g, b);
-        issued_v[s] = ph;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (is_k) {
+          // the single Q buffer is free once the previous item's S MMAs are done
+          if (u > 0 && !(ok = mbar_wait(q_empty, (u - 1) & 1, ctl))) break;
+          mbar_expect_tx(q_full, Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, w.m0, w.hq, w.b);
+          q_issued = u & 1;
+        }
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int s = c % stages;
+          const uint32_t ph = (c / stages) & 1;
+          const uint32_t full = is_k ? k_full(s) : v_full(s);
+          const uint32_t empty = is_k ? k_empty(s) : v_empty(s);
+          if (!(ok = mbar_wait(empty, ph ^ 1, ctl))) break;
+          mbar_expect_tx(full, Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(ring + s * Lay::kTileBytes + h * kTile * 128, map, full, h * 64,
+                        (w.nlo + it) * kTile, w.g, w.b);
+          issued[s] = static_cast<int>(ph);
+        }
+        ++u;
       }
       if (!ok) {
         // Aborted: let every copy already issued land before the CTA exits.
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mbar_wait(q_full, 0, ign);
-        for (int s = 0; s < S; ++s) {
-          if (issued_k[s] >= 0) mbar_wait(k_full(s), issued_k[s], ign);
-          if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
-        }
+        if (q_issued >= 0) mbar_wait(q_full, q_issued, ign);
+        for (int s = 0; s < stages; ++s)
+          if (issued[s] >= 0) mbar_wait(is_k ? k_full(s) : v_full(s), issued[s], ign);
       }
     }
-  } else if (warp == 4 * NQ + 1) {
-    // ============================ MMA issuer =============================
-    if (lane == 0 && nt > 0) {
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers (one thread each) =====================
+    if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_bf16_f32(kTile, D, 0, 1);      // V is N(=d)-major
-      int cnt[NQ];
-      for (int t = 0; t < NQ; ++t) cnt[t] = 0;
-      bool ok = mbar_wait(q_full, 0, ctl);
-      for (int it = 0; it < nt && ok; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        const int n = nlo + it;
-        if (!(ok = mbar_wait(k_full(s), ph, ctl))) break;
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (n < tlo[t] || n >= thi[t]) continue;
-          // S_t's columns held P_t of the previous tile: wait until P_t V was done.
-          if (cnt[t] > 0 && !(ok = mbar_wait(o_done(t), (cnt[t] - 1) & 1, ctl))) break;
-          tc_fence_after();
+      const bool chain_s = (warp == 9);
+      int c = 0;  // tiles so far, over all items
+      int u = 0;  // items with a non-empty band so far
+      bool ok = true;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (chain_s && !(ok = issuer_wait(q_full, u & 1, ctl))) break;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int x = c % NS;
+          if (chain_s) {
+            const int sk = c % SK;
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            // buffer x held P of tile c - NS: wait until its P V MMA is done
+            if (c >= NS && !(ok = issuer_wait(pv_done(x), ((c / NS) - 1) & 1, ctl))) break;
+            tc_fence_after();
+            const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t qa = sb + Lay::kQOff + t * Lay::kTileBytes + (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t ka = sb + Lay::kKOff + s * Lay::kTileBytes + (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + t * kTile, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024),
-                   kIdS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + x * kTile,
+                     smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
+                     smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+            mma_commit(s_full(x));
+            mma_commit(k_empty(sk));
+          } else {
+            // P V of an item's first tile overwrites O: every softmax thread
+            // read the previous item's O before it marked this P ready.
+            const int sv = c % SV;
+            if (!(ok = issuer_wait(v_full(sv), (c / SV) & 1, ctl))) break;
+            if (!(ok = issuer_wait(p_full(x), (c / NS) & 1, ctl))) break;
+            tc_fence_after();
+            const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(tmem + Lay::kOCol, split_a_col(tmem + x * kTile, kk),
+                     smem_desc_sw128(vs + kk * 2048, kTile * 128, 1024), kIdO,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(pv_done(x));
+            mma_commit(v_empty(sv));
           }
-          mma_commit(s_full(t));
         }
         if (!ok) break;
-        mma_commit(k_empty(s));
-        if (!(ok = mbar_wait(v_full(s), ph, ctl))) break;
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (n < tlo[t] || n >= thi[t]) continue;
-          if (!(ok = mbar_wait(p_full(t), cnt[t] & 1, ctl))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t va = sb + Lay::kVOff + s * Lay::kTileBytes + kk * 2048;
-            mma_ts(tmem + Lay::kOCol + t * D, tmem + t * kTile + kk * 8,
-                   smem_desc_sw128(va, 16384, 1024), kIdO, (cnt[t] > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(o_done(t));
-          ++cnt[t];
-        }
-        if (!ok) break;
-        mma_commit(v_empty(s));
+        mma_commit(chain_s ? q_empty : acc_done);
+        ++u;
       }
       if (!ok) {
-        // Aborted: wait until every MMA already issued has finished with
+        // Aborted: wait until every MMA this thread issued has finished with
         // tensor memory before the CTA frees it.
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mma_commit(drain);
-        mbar_wait(drain, 0, ign);
+        mma_commit(drain(chain_s ? 0 : 1));
+        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
       }
     }
   } else {
-    // ===================== softmax warpgroup t (rows) =====================
-    const int t = warp >> 2;
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const int m0t = m0 + t * kTile;
-    const int i = m0t + row;  // query row
-    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_bits + t * kTile;
-    const uint32_t tO = tmem + lane_bits + Lay::kOCol + t * D;
-    float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + t * 512;
-    const float* brow = nullptr;
-    if constexpr (BIAS == kBiasDense) {
-      // rows past L read row L-1 (in bounds); their outputs are never stored
-      brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
-             static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
-    }
-    float m_run = -INFINITY;  // running max, log2 units
-    float l_run = 0.f;        // running sum relative to m_run
-    // `ok` is kept warp-uniform; after an abort the loop still runs to the
-    // end (every wait then returns at once) so that no thread of the
-    // warpgroup is left waiting at a named barrier.
+    // ===== softmax warpgroup wg: key columns [64 wg, 64 wg + 64); thread = query row =====
+    const int wg = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const int c0w = kBlk * wg;
+    const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + lane_bits + Lay::kOCol + wg * (D / 2);
+    float* red = reinterpret_cast<float*>(smem + Lay::kRedOff);  // max [parity][wg][row]
+    float* rsum = red + 4 * kTile;                               // sum [parity][wg][row]
+    float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + wg * 512;
+    // `ok` is kept warp-uniform.  After an abort every wait returns at once,
+    // but every tile of every item still passes the exchange barrier, so no
+    // thread of the CTA is left waiting at a named barrier.
     bool ok = true;
-    int cnt = 0;
-    for (int n = tlo[t]; n < thi[t]; ++n, ++cnt) {
-      const int n0 = n * kTile;
-      const bool full = tile_is_full(p, m0t, n0, false);
-      int lo = 0, hi = kTile - 1;
-      if (!full) row_visible_cols(p, i, n0, lo, hi);
-      const float* lut_row = nullptr;
-      if constexpr (BIAS == kBiasT5) {
-        // bias of every distance this tile spans: j - i = (n0 - m0t) + (c - row)
-        float* lt = lut + (cnt & 1) * 256;
-        const int base = n0 - m0t - (kTile - 1);
-        lt[row] = p.t5_table[t5_bucket(base + row, p.t5) * p.Hq + hq] * kLog2e;
-        if (row < kTile - 1)
-          lt[row + kTile] = p.t5_table[t5_bucket(base + row + kTile, p.t5) * p.Hq + hq] * kLog2e;
-        named_barrier(1 + t, kTile);
-        lut_row = lt + (kTile - 1) - row;
+    int gc = 0;  // tiles so far, over all items
+    int u = 0;   // items with a non-empty band so far
+    for (int id = blockIdx.x; id < n_items; id += gridDim.x) {
+      const Item w = item_at(id);
+      const int m0 = w.m0, hq = w.hq, b = w.b, nt = w.nt;
+      const int i = m0 + row;  // query row
+      const float* brow = nullptr;
+      if constexpr (BIAS == kBiasDense) {
+        // rows past L read row L-1 (in bounds); their outputs are never stored
+        brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
+               static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
       }
-      if (ok) ok = mbar_wait(s_full(t), cnt & 1, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) continue;
-      tc_fence_after();
-      // x: scores in log2 units, in place over the raw accumulator bits
-      uint32_t x[128];
-      tmem_ld128_sync(tS, x);
-      float sum, alpha, m_use;
-      bool grow;
-      if (kFwdLeanSoftmax && BIAS == kBiasNone && full && p.scale_log2 > 0.f) {
-        // ---- lean path: raw max (3-input), exponent = fma(s, c, -m)
-        float ma = -INFINITY, mb = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kTile; c += 4) {
-          ma = fmax3(ma, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-          mb = fmax3(mb, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+      float m_run = -INFINITY;  // running row max, log2 units (identical in both warpgroups)
+      float l_run = 0.f;        // this warpgroup's share of the row sum, relative to m_run
+      for (int it = 0; it < nt; ++it, ++gc) {
+        const int x = gc % NS;
+        const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup's columns
+        const uint32_t tS = tmem + lane_bits + x * kTile + c0w;
+        const float* lut_row = nullptr;
+        if constexpr (BIAS == kBiasT5) {
+          // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
+          float* lt = lut + (gc & 1) * 256;
+          const int base = n0 - m0 - (kTile - 1);
+          for (int r = row; r < kTile + kBlk - 1; r += kTile)
+            lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
+          named_barrier(1 + wg, kTile);
+          lut_row = lt + (kTile - 1) - row;
         }
-        const float tmax = fmaxf(ma, mb) * p.scale_log2;
+        int lo = 0, hi = kBlk - 1;
+        bool full = n0 + kBlk <= p.L;
+        if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
+        if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
+        if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
+        if (!full) {
+          if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
+          hi = min(hi, p.L - 1 - n0);
+          if (p.causal) hi = min(hi, i - n0);
+          if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
+        }
+        const bool lean = kFwdLeanSoftmax && BIAS == kBiasNone && full && p.scale_log2 > 0.f;
+
+        // ---- phase A: this warpgroup's half of S_j and its partial row max
+        if (ok) ok = mbar_wait(s_full(x), (gc / NS) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        const bool live = ok;
+        uint32_t xs[kBlk];  // raw accumulator bits (lean) or log2-unit scores
+        float pmax = -INFINITY;
+        if (live) {
+          tc_fence_after();
+          tmem_ld64_sync(tS, xs);
+          if (lean) {
+            float ma = -INFINITY, mb = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kBlk; c += 4) {
+              ma = fmax3(ma, __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
+              mb = fmax3(mb, __uint_as_float(xs[c + 2]), __uint_as_float(xs[c + 3]));
+            }
+            pmax = fmaxf(ma, mb) * p.scale_log2;
+          } else {
+            float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (full) {
+#pragma unroll
+              for (int c = 0; c < kBlk; ++c) {
+                float v = __uint_as_float(xs[c]) * p.scale_log2;
+                if constexpr (BIAS == kBiasT5) v += lut_row[c];
+                if constexpr (BIAS == kBiasDense) v = fmaf(brow[n0 + c], kLog2e, v);
+                xs[c] = __float_as_uint(v);
+                tm[c & 3] = fmaxf(tm[c & 3], v);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < kBlk; ++c) {
+                const bool vis = (c >= lo) && (c <= hi);
+                float v = __uint_as_float(xs[c]) * p.scale_log2;
+                if constexpr (BIAS == kBiasT5) v += lut_row[c];
+                if constexpr (BIAS == kBiasDense) v += vis ? brow[n0 + c] * kLog2e : 0.f;
+                v = vis ? v : -INFINITY;
+                xs[c] = __float_as_uint(v);
+                tm[c & 3] = fmaxf(tm[c & 3], v);
+              }
+            }
+            pmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+          }
+        }
+        // ---- exchange the partial maxima (double-buffered by tile parity)
+        red[((gc & 1) * 2 + wg) * kTile + row] = pmax;
+        named_barrier(kXchgBar, 2 * kTile);
+        if (!live) continue;
+        const float tmax = fmaxf(pmax, red[((gc & 1) * 2 + (1 - wg)) * kTile + row]);
         const float m_new = fmaxf(m_run, tmax);
-        grow = m_new > m_run + kRescaleThreshold;
-        m_use = grow ? m_new : m_run;
-        alpha = grow ? fast_exp2(m_run - m_use) : 1.f;
-        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-m_use, -m_use);  // m_use is finite in a full tile
-        uint64_t acc[4] = {0, 0, 0, 0};
+        const bool grow = m_new > m_run + kRescaleThreshold;
+        const float m_use = grow ? m_new : m_run;
+        const float alpha = grow ? fast_exp2(m_run - m_use) : 1.f;
+        const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;  // finite on every lean tile
+
+        // ---- phase B: exponentials, P_j (bf16) over the first 32 of this warpgroup's S columns
+        float sum;
+        if (lean) {
+          const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
+          uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int c0 = 0; c0 < kTile; c0 += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const uint64_t arg = f2_fma(f2_pack(__uint_as_float(x[c0 + c]), __uint_as_float(x[c0 + c + 1])),
-                                        c2, nm2);
-            float v0, v1;
-            f2_unpack(arg, v0, v1);
-            const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
-            const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
-            const uint64_t e2 = f2_pack(e0, e1);
-            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e2);
-            pk[c >> 1] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
-        }
-        float s0, s1, s2, s3, s4, s5, s6, s7;
-        f2_unpack(acc[0], s0, s1);
-        f2_unpack(acc[1], s2, s3);
-        f2_unpack(acc[2], s4, s5);
-        f2_unpack(acc[3], s6, s7);
-        sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-      } else {
-        // four independent max / sum chains instead of one 128 long
-        float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        const float* bcol = brow ? brow + n0 : nullptr;
-        if (full) {
-  #pragma unroll
-          for (int c = 0; c < kTile; ++c) {
-            float v = __uint_as_float(x[c]) * p.scale_log2;
-            if constexpr (BIAS != kBiasNone) v += bias_log2<BIAS>(lut_row, bcol, c);
-            x[c] = __float_as_uint(v);
-            tm[c & 3] = fmaxf(tm[c & 3], v);
-          }
-        } else {
-  #pragma unroll
-          for (int c = 0; c < kTile; ++c) {
-            const bool vis = (c >= lo) && (c <= hi);
-            float v = __uint_as_float(x[c]) * p.scale_log2;
-            if constexpr (BIAS == kBiasT5) v += lut_row[c];
-            if constexpr (BIAS == kBiasDense) v += vis ? bcol[c] * kLog2e : 0.f;
-            v = vis ? v : -INFINITY;
-            x[c] = __float_as_uint(v);
-            tm[c & 3] = fmaxf(tm[c & 3], v);
-          }
-        }
-        const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
-        const float m_new = fmaxf(m_run, tmax);
-        const bool grow_g = m_new > m_run + kRescaleThreshold;
-        const float m_use_g = grow_g ? m_new : m_run;
-        const float alpha_g = grow_g ? fast_exp2(m_run - m_use_g) : 1.f;
-        const float m_sub = (m_use_g == -INFINITY) ? 0.f : m_use_g;
-        float sm[4] = {0.f, 0.f, 0.f, 0.f};
-        if (full) {
-          // every entry is finite: a fixed share of the exponentials on the FMA pipe
-  #pragma unroll
-          for (int c0 = 0; c0 < kTile; c0 += 32) {
+          for (int c0 = 0; c0 < kBlk; c0 += 32) {
             uint32_t pk[16];
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              const float v0 = __uint_as_float(x[c0 + c]) - m_sub;
-              const float v1 = __uint_as_float(x[c0 + c + 1]) - m_sub;
+              const uint64_t arg = f2_fma(
+                  f2_pack(__uint_as_float(xs[c0 + c]), __uint_as_float(xs[c0 + c + 1])), c2, nm2);
+              float v0, v1;
+              f2_unpack(arg, v0, v1);
               const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
               const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
-              sm[(c >> 1) & 3] += e0 + e1;
-              pk[c >> 1] = pack_bf16x2(e0, e1);
-            }
-            tmem_st16(tS + (c0 >> 1), pk);  // P_t (bf16 pairs) over the first 64 columns of S_t
-          }
-        } else {
-  #pragma unroll
-          for (int c0 = 0; c0 < kTile; c0 += 32) {
-            uint32_t pk[16];
-  #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float e0 = fast_exp2(__uint_as_float(x[c0 + c]) - m_sub);
-              const float e1 = fast_exp2(__uint_as_float(x[c0 + c + 1]) - m_sub);
-              sm[(c >> 1) & 3] += e0 + e1;
+              acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(e0, e1));
               pk[c >> 1] = pack_bf16x2(e0, e1);
             }
             tmem_st16(tS + (c0 >> 1), pk);
           }
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(acc[0], s0, s1);
+          f2_unpack(acc[1], s2, s3);
+          f2_unpack(acc[2], s4, s5);
+          f2_unpack(acc[3], s6, s7);
+          sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        } else {
+          float sm[4] = {0.f, 0.f, 0.f, 0.f};
+          if (full) {
+            // every entry is finite: a fixed share of the exponentials on the FMA pipe
+#pragma unroll
+            for (int c0 = 0; c0 < kBlk; c0 += 32) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                const float v0 = __uint_as_float(xs[c0 + c]) - m_sub;
+                const float v1 = __uint_as_float(xs[c0 + c + 1]) - m_sub;
+                const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
+                const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
+                sm[(c >> 1) & 3] += e0 + e1;
+                pk[c >> 1] = pack_bf16x2(e0, e1);
+              }
+              tmem_st16(tS + (c0 >> 1), pk);
+            }
+          } else {
+#pragma unroll
+            for (int c0 = 0; c0 < kBlk; c0 += 32) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                const float e0 = fast_exp2(__uint_as_float(xs[c0 + c]) - m_sub);
+                const float e1 = fast_exp2(__uint_as_float(xs[c0 + c + 1]) - m_sub);
+                sm[(c >> 1) & 3] += e0 + e1;
+                pk[c >> 1] = pack_bf16x2(e0, e1);
+              }
+              tmem_st16(tS + (c0 >> 1), pk);
+            }
+          }
+          sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
         }
-        sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
-        grow = grow_g;
-        alpha = alpha_g;
-        m_use = m_use_g;
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
+        tmem_st_wait();
+        if (it > 0 && __any_sync(0xffffffffu, grow)) {
+          // O holds earlier tiles: rescale this warpgroup's half of its columns
+          // once P V of the previous tile has landed.
+          ok = mbar_wait(pv_done((gc - 1) % NS), ((gc - 1) / NS) & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) continue;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 2; c += 32) {
+            uint32_t r[32];
+            tmem_ld32_sync(tO + c, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32_sync(tO + c, r);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(p_full(x));
       }
-      l_run = l_run * alpha + sum;
-      m_run = m_use;
-      tmem_st_wait();
-      if (cnt > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_t holds earlier tiles: rescale it once P_t V of the previous tile landed.
-        ok = mbar_wait(o_done(t), (cnt - 1) & 1, ctl);
+
+      // ------------------------------ epilogue ------------------------------
+      // Items without a visible key (none exist for the masks accepted at the
+      // boundary) write O = 0 and LSE = -inf without touching tensor memory.
+      float l_tot = 0.f;
+      if (nt > 0) {
+        rsum[((u & 1) * 2 + wg) * kTile + row] = l_run;
+        named_barrier(kXchgBar, 2 * kTile);
+        l_tot = l_run + rsum[((u & 1) * 2 + (1 - wg)) * kTile + row];
+        if (ok) ok = mbar_wait(acc_done, u & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
-        if (!ok) continue;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32_sync(tO + c, r);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32_sync(tO + c, r);
-        }
+        ++u;
       }
-      tc_fence_before();
-      mbar_arrive(p_full(t));
-    }
-    // ------------------------------ epilogue ------------------------------
-    if (ok && cnt > 0) ok = mbar_wait(o_done(t), (cnt - 1) & 1, ctl);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.sq_b +
-                            static_cast<int64_t>(i) * p.sq_l + static_cast<int64_t>(hq) * p.sq_h;
+      if (ok) {
+        // this warpgroup's half of the O row; once read, the next item's first
+        // P V may overwrite O (this thread marks that P ready only after this)
+        uint32_t r[D / 2];
+        if (nt > 0) {
+          tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t r[32];
-        if (cnt > 0) {
-          tmem_ld32_sync(tO + c, r);
+          for (int c = 0; c < D / 2; c += 32)
+            tmem_ld32_sync(tO + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+          for (int e = 0; e < D / 2; ++e) r[e] = 0u;
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+        const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         if (i < p.L) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.sq_b +
+                                static_cast<int64_t>(i) * p.sq_l + static_cast<int64_t>(hq) * p.sq_h +
+                                wg * (D / 2);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int c = 0; c < D / 2; c += 8) {
+            uint4 v4;
+            v4.x = pack_bf16x2(__uint_as_float(r[c]) * inv, __uint_as_float(r[c + 1]) * inv);
+            v4.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv, __uint_as_float(r[c + 3]) * inv);
+            v4.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv, __uint_as_float(r[c + 5]) * inv);
+            v4.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv, __uint_as_float(r[c + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c) = v4;
+          }
+          if (wg == 0) {
+            p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + i] =
+                l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
+          }
         }
-      }
-      if (i < p.L) {
-        p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + i] =
-            l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
   }

@@ -101,6 +101,7 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
   if (s->Hq % s->Hkv != 0) return SDPA_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return SDPA_ERR_UNSUPPORTED;
   if (s->L >= (1ll << 30) || s->B > 65535 || s->Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  if ((s->L + 127) / 128 * s->Hq * s->B >= (1ll << 31)) return SDPA_ERR_UNSUPPORTED;
   const int64_t st[6] = {s->sq_b, s->sq_l, s->sq_h, s->skv_b, s->skv_l, s->skv_h};
   for (int64_t v : st)
     if (v <= 0 || (v % 8) != 0 || v >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
@@ -149,27 +150,44 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
   return SDPA_OK;
 }
 
-template <int D, int NQ, int BIAS>
+// Streaming multiprocessors of the current device (persistent grids), cached
+// per device.
+int sm_count() {
+  constexpr int kDevs = 64;
+  static int cached[kDevs] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevs && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevs) cached[dev] = n;
+  return n;
+}
+
+template <int D, int BIAS>
 cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
                        const CUtensorMap& v, cudaStream_t st) {
-  using Lay = FwdLayout<D, NQ>;
-  auto kern = fwd_kernel<D, NQ, BIAS>;
+  using Lay = FwdLayout<D, BIAS>;
+  auto kern = fwd_kernel<D, BIAS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Lay::kSmemAlloc);
   if (e != cudaSuccess) return e;
-  const int rows = kTile * NQ;
-  dim3 grid((p.L + rows - 1) / rows, p.Hq, p.B);
+  // persistent: one CTA per SM (or per work item, if fewer)
+  const int64_t items = static_cast<int64_t>((p.L + kTile - 1) / kTile) * p.Hq * p.B;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = static_cast<int>(items < sms ? items : sms);
   kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v);
   return cudaGetLastError();
 }
 
-template <int D, int NQ>
+template <int D>
 cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
                               const CUtensorMap& v, cudaStream_t st) {
   switch (p.bias_kind) {
-    case kBiasDense: return launch_fwd<D, NQ, kBiasDense>(p, q, k, v, st);
-    case kBiasT5: return launch_fwd<D, NQ, kBiasT5>(p, q, k, v, st);
-    default: return launch_fwd<D, NQ, kBiasNone>(p, q, k, v, st);
+    case kBiasDense: return launch_fwd<D, kBiasDense>(p, q, k, v, st);
+    case kBiasT5: return launch_fwd<D, kBiasT5>(p, q, k, v, st);
+    default: return launch_fwd<D, kBiasNone>(p, q, k, v, st);
   }
 }
 
@@ -238,8 +256,8 @@ sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k, co
       !make_bshd_map(&mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h))
     return SDPA_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128, 2>(p, mq, mk, mv, cs)
-                               : dispatch_fwd_bias<64, 2>(p, mq, mk, mv, cs);
+  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128>(p, mq, mk, mv, cs)
+                               : dispatch_fwd_bias<64>(p, mq, mk, mv, cs);
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 

@@ -107,9 +107,64 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait, but polling without ever suspending the thread: for the
+// single-thread roles (MMA issue) whose reaction time is on the critical path
+// of every tile.  The time limit is checked every 1024 polls.
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t k = 1;; ++k) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((k & 1023u) == 0) {
+      if (*ctl.abort) return false;
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort = 1;
+        atomicOr(&g_device_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait used by the MMA-issuing threads.
+constexpr bool kIssuerPoll = true;
+__device__ __forceinline__ bool issuer_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+  return kIssuerPoll ? mbar_wait_poll(bar, parity, ctl) : mbar_wait(bar, parity, ctl);
+}
+
 // Named barrier over `count` threads (multiple of 32), id 1..15.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Warpgroup register reallocation: every warp of a warpgroup executes the
+// same one.  The grown warpgroups draw on registers the shrunk ones release;
+// the totals must fit the registers the block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Arrive on a named barrier without waiting (the other `count - arrivals`
+// threads wait on it with named_barrier).
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---------------------------------------------------------------------- TMA
