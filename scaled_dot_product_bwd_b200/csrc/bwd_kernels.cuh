@@ -516,7 +516,10 @@ __global__ void __launch_bounds__(352, 1)
 // through; warpgroup w takes the key columns [64 w, 64 w + 64).  Tensor
 // memory: S[0] 0..127 | S[1] 128..255 | dP 256..383 | dQ 384..  The scores
 // are double-buffered, so S of block i + 1 is computed while block i's dS is
-// formed; dS (bf16) overwrites the first half of each warpgroup's dP columns.
+// formed.  dS (bf16) goes over the first half of each warpgroup's columns of
+// its own, already loaded, S buffer: dP of block i + 1 can then be computed
+// as soon as block i's dP has been loaded, and S of block i + 2 waits only
+// for the dQ MMA of block i.
 template <int D, int BIAS>
 struct DqLayout {
   static constexpr int kTileBytes = kTile * D * 2;
@@ -531,8 +534,8 @@ struct DqLayout {
   static constexpr int kLutOff = kVOff + kSV * kTileBytes;    // T5 only: 2 WG x 2 x 256 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
-  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_used[2],
-  // dp_full, ds_full, dq_done, acc_done, drain[2]
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
+  // dp_full, dp_used, ds_full, acc_done, drain[2]
   static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
@@ -577,10 +580,10 @@ __global__ void __launch_bounds__(352, 1)
   auto v_empty = [&](int s) { return bar(1 + 2 * SK + SV + s); };
   constexpr int kB = 1 + 2 * SK + 2 * SV;
   auto s_full = [&](int x) { return bar(kB + x); };
-  auto s_used = [&](int x) { return bar(kB + 2 + x); };
+  auto dq_done = [&](int x) { return bar(kB + 2 + x); };  // dQ MMA of a block in buffer x done
   const uint32_t dp_full = bar(kB + 4);
-  const uint32_t ds_full = bar(kB + 5);
-  const uint32_t dq_done = bar(kB + 6);
+  const uint32_t dp_used = bar(kB + 5);
+  const uint32_t ds_full = bar(kB + 6);
   const uint32_t acc_done = bar(kB + 7);
   auto drain = [&](int x) { return bar(kB + 8 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
@@ -600,11 +603,11 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full(x), 1);
-      mbar_init(s_used(x), 2 * kTile);
+      mbar_init(dq_done(x), 1);
     }
     mbar_init(dp_full, 1);
+    mbar_init(dp_used, 2 * kTile);
     mbar_init(ds_full, 2 * kTile);
-    mbar_init(dq_done, 1);
     mbar_init(acc_done, 1);
     mbar_init(drain(0), 1);
     mbar_init(drain(1), 1);
@@ -663,23 +666,39 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else if (warp == 9 || warp == 10) {
     // ===================== MMA issuers (one thread each) =====================
-    // Warp 9 runs the score chain ahead: S(i) into buffer i % 2 as soon as K(i)
-    // has landed and both warpgroups have loaded S(i-2) out of that buffer.
-    // Warp 10 runs dP(i), then dQ(i) once dS(i) is ready, then dP(i+1) once
-    // dQ(i) has read dS(i) out of the dP columns.
+    // Warp 9 runs the score chain: S(i) into buffer i % 2 once K(i) has landed
+    // and the dQ MMA of block i - 2 has read dS out of that buffer.  Warp 10
+    // runs dP one block ahead of dQ: dP(i + 1) as soon as both warpgroups have
+    // loaded dP(i), then dQ(i) once dS(i) is ready.
     if (lane == 0 && nt > 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
       const bool chain_s = (warp == 9);
+      auto issue_dp = [&](int it) {
+        const uint32_t vs = sb + Lay::kVOff + (it % SV) * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + Lay::kDPCol,
+                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
+                 smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(dp_full);
+        mma_commit(v_empty(it % SV));
+      };
       bool ok = issuer_wait(q_full, 0, ctl);
+      if (ok && !chain_s) {
+        ok = issuer_wait(v_full(0), 0, ctl);
+        if (ok) {
+          tc_fence_after();
+          issue_dp(0);
+        }
+      }
       for (int it = 0; it < nt && ok; ++it) {
         const int x = it & 1;
-        const int sk = it % SK, sv = it % SV;
+        const int sk = it % SK;
         const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
-        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
-        if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
         if (chain_s) {
-          if (it >= 2 && !(ok = issuer_wait(s_used(x), ((it >> 1) - 1) & 1, ctl))) break;
+          if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
+          if (it >= 2 && !(ok = issuer_wait(dq_done(x), ((it >> 1) - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -689,24 +708,22 @@ __global__ void __launch_bounds__(352, 1)
           mma_commit(s_full(x));
           mma_commit(k_empty(sk));
         } else {
-          if (!(ok = issuer_wait(v_full(sv), (it / SV) & 1, ctl))) break;
-          if (it > 0 && !(ok = issuer_wait(dq_done, (it - 1) & 1, ctl))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + Lay::kDPCol,
-                   smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
-                   smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-          mma_commit(dp_full);
-          mma_commit(v_empty(sv));
+          if (it + 1 < nt) {
+            const int sv = (it + 1) % SV;
+            if (!(ok = issuer_wait(v_full(sv), ((it + 1) / SV) & 1, ctl))) break;
+            if (!(ok = issuer_wait(dp_used, it & 1, ctl))) break;
+            tc_fence_after();
+            issue_dp(it + 1);
+          }
+          if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
           if (!(ok = issuer_wait(ds_full, it & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + Lay::kDPCol, kk),
+            mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk),
                    smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
                    (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(dq_done);
+          mma_commit(dq_done(x));
           mma_commit(k_empty(sk));
         }
       }
@@ -767,10 +784,9 @@ __global__ void __launch_bounds__(352, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
+      const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
       uint32_t pr[64];  // S row, then P (fp32 bits)
-      tmem_ld64_sync(tmem + lane_bits + kTile * x + c0w, pr);
-      tc_fence_before();
-      mbar_arrive(s_used(x));  // S[x] may now take block it + 2
+      tmem_ld64_sync(tSx, pr);
       if (full) {
 #pragma unroll
         for (int c = 0; c < kBlk; ++c) {
@@ -793,19 +809,25 @@ __global__ void __launch_bounds__(352, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
+      uint32_t pk[32];  // dS as bf16 pairs
 #pragma unroll
       for (int cc = 0; cc < kBlk; cc += 32) {
         uint32_t dr[32];
         tmem_ld32_sync(tDP + cc, dr);
-        uint32_t pk[16];
+        if (cc + 32 == kBlk) {
+          tc_fence_before();
+          mbar_arrive(dp_used);  // the dP columns may now take block it + 1
+        }
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dd);
           const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dd);
-          pk[c >> 1] = pack_bf16x2(d0, d1);
+          pk[(cc + c) >> 1] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tDP + (cc >> 1), pk);  // dS over the first 32 of this warpgroup's dP columns
       }
+      // dS over the first 32 of this warpgroup's columns of its S buffer
+      tmem_st16(tSx, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+      tmem_st16(tSx + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
