@@ -36,7 +36,37 @@ CONFIGS = {
     "t5rpe": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="t5"),
     "t5dense": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="dense"),
     "tiny": dict(B=1, Hq=2, Hkv=2, L=128, d=64, causal=True, wl=-1, wr=-1, bias="none"),
+    # the mistral4k shape at batch 2: the case the ncu captures run on (inputs
+    # still larger than L2, a few hundred MB on the device)
+    "mistral4k_small": dict(B=2, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1,
+                            bias="none"),
 }
+
+# DRAM bytes per launch of a kernel (dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture, divided by the captured batch size), keyed by workload
+# shape and kernel, with the hash of the kernel sources the counters were taken
+# on.  A bench workload of the same shape reports them scaled to its batch, and
+# only while the library is built from exactly those sources.
+NCU_TRAFFIC = {
+    # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
+    # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
+    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_164_480 + 22_958_848) / 2,
+                                    source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
+    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(169_956_608 + 43_143_168) / 2,
+                                  source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
+    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_805_120 + 33_030_400) / 2,
+                               source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
+}
+
+
+def traffic_per_launch(config_name, kernel, batch):
+    """ncu DRAM bytes of one launch of `kernel` on this workload, else None."""
+    from scaled_dot_product_bwd_b200.build import source_hash
+    shape = config_name.replace("_small", "")
+    rec = NCU_TRAFFIC.get((shape, kernel))
+    if rec is None or rec["source_hash"] != source_hash():
+        return None
+    return int(round(rec["bytes_per_batch"] * batch))
 
 
 def describe(c):
@@ -326,7 +356,8 @@ def run_gpu(args, c):
         ach = algo[dname] / (phase_ms[dom] * 1e-3) / 1e12
         roofline = {"kernel": dname, "bound": "tensor", "achieved": round(ach, 1),
                     "peak": peaks["tflops"], "unit": "TFLOP/s",
-                    "frac": round(ach / peaks["tflops"], 4), "traffic": None,
+                    "frac": round(ach / peaks["tflops"], 4),
+                    "traffic": traffic_per_launch(args.config, dname, c["B"]),
                     "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"
                     if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
                     "flops_per_launch": algo[dname], "ms_per_launch": round(phase_ms[dom], 4)}

@@ -60,6 +60,11 @@ FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=s
          "-Xcompiler", "-fPIC", "-shared", "-cudart", "static"]
 
 
+def source_hash() -> str:
+    """Hash of the kernel sources and build flags the library is built from."""
+    return _source_hash(FLAGS)
+
+
 def build(verbose: bool = False, force: bool = False) -> str:
     if not force and up_to_date(FLAGS):
         return LIB_PATH
