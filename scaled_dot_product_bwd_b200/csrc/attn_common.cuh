@@ -161,4 +161,18 @@ __device__ __forceinline__ uint32_t split_a_col(uint32_t base, int kk) {
   return base + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
 }
 
+// Streaming multiprocessors of the current device (persistent grids), cached
+// per device.
+inline int sm_count() {
+  constexpr int kDevs = 64;
+  static int cached[kDevs] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevs && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kDevs) cached[dev] = n;
+  return n;
+}
+
 }  // namespace sdpa

@@ -512,8 +512,11 @@ __global__ void __launch_bounds__(352, 1)
 }
 
 // --------------------------------------------------------------------- dQ
-// CTA = 128 queries of one (query head, batch); blocks of 128 keys stream
-// through; warpgroup w takes the key columns [64 w, 64 w + 64).  Tensor
+// Persistent: one CTA per SM walks a heavy-first list of work items, each 128
+// queries of one (query head, batch); blocks of 128 keys stream through;
+// warpgroup w takes the key columns [64 w, 64 w + 64).  Ring, buffer and
+// barrier indices count across items, so the next item's Q / dO load and
+// first scores overlap the current item's last blocks and epilogue.  Tensor
 // memory: S[0] 0..127 | S[1] 128..255 | dP 256..383 | dQ 384..  The scores
 // are double-buffered, so S of block i + 1 is computed while block i's dS is
 // formed.  dS (bf16) goes over the first half of each warpgroup's columns of
@@ -535,8 +538,8 @@ struct DqLayout {
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
-  // dp_full, dp_used, ds_full, acc_done, drain[2]
-  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 10;
+  // dp_full, dp_used, ds_full, acc_done, drain[2], q_empty, o_full, o_empty
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 13;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
   static constexpr int kThreads = 352;  // 2 compute warpgroups, producer, two MMA issuers
@@ -562,15 +565,28 @@ __global__ void __launch_bounds__(352, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // ---- work items: (query tile, head, batch), heaviest causal query tiles
+  // first; consecutive items are neighbouring heads, which share K / V in L2.
   const int nqt = (p.L + kTile - 1) / kTile;
-  const int qt = p.causal ? (nqt - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int hq = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = hq / p.G;
-  const int m0 = qt * kTile;
-  int nlo, nhi;
-  key_tile_range(p, m0, kTile, nlo, nhi);
-  const int nt = nhi > nlo ? nhi - nlo : 0;
+  const int heads = p.Hq * p.B;
+  const int n_items = nqt * heads;
+  struct Item {
+    int m0, hq, b, g, nlo, nt;
+  };
+  auto item_at = [&](int id) {
+    Item w;
+    const int r = id / heads;
+    const int rem = id - r * heads;
+    const int qt = p.causal ? nqt - 1 - r : r;
+    w.m0 = qt * kTile;
+    w.hq = rem % p.Hq;
+    w.b = rem / p.Hq;
+    w.g = w.hq / p.G;
+    int nhi;
+    key_tile_range(p, w.m0, kTile, w.nlo, nhi);
+    w.nt = nhi > w.nlo ? nhi - w.nlo : 0;
+    return w;
+  };
 
   auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
   const uint32_t q_full = bar(0);
@@ -586,11 +602,19 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t ds_full = bar(kB + 6);
   const uint32_t acc_done = bar(kB + 7);
   auto drain = [&](int x) { return bar(kB + 8 + x); };
+  // Q is read only by the score issuer, dO only by the dP issuer: each tile is
+  // released as soon as its one reader is done with the item
+  const uint32_t q_empty = bar(kB + 10);
+  const uint32_t o_full = bar(kB + 11);
+  const uint32_t o_empty = bar(kB + 12);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 1);
     // K blocks are read by both issuers (S and dQ): a slot is free once each
     // issuer's last MMA on it has completed.
     for (int s = 0; s < SK; ++s) {
@@ -626,38 +650,56 @@ __global__ void __launch_bounds__(352, 1)
 
   if (warp == 8) {
     // ============================ producer ============================
-    if (lane == 0 && nt > 0) {
+    // Per item: Q and dO once (each after its reader is done with the
+    // previous item's), then K and V of every key block into their rings.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(q_full, 2 * Lay::kTileBytes);
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, m0, hq, b);
-        tma_load_4d(sb + Lay::kDOOff + h * kTile * 128, &tmDO, q_full, h * 64, m0, hq, b);
-      }
       int issued_k[SK], issued_v[SV];
       for (int s = 0; s < SK; ++s) issued_k[s] = -1;
       for (int s = 0; s < SV; ++s) issued_v[s] = -1;
+      int q_issued = -1, o_issued = -1;
+      int c = 0;  // key blocks so far, over all items
+      int u = 0;  // items with a non-empty band so far
       bool ok = true;
-      for (int it = 0; it < nt; ++it) {
-        const int sk = it % SK, sv = it % SV;
-        const int n0 = (nlo + it) * kTile;
-        if (!(ok = mbar_wait(k_empty(sk), ((it / SK) & 1) ^ 1, ctl))) break;
-        mbar_expect_tx(k_full(sk), Lay::kTileBytes);
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (u > 0 && !(ok = mbar_wait(q_empty, (u - 1) & 1, ctl))) break;
+        mbar_expect_tx(q_full, Lay::kTileBytes);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK, k_full(sk),
-                      h * 64, n0, g, b);
-        issued_k[sk] = (it / SK) & 1;
-        if (!(ok = mbar_wait(v_empty(sv), ((it / SV) & 1) ^ 1, ctl))) break;
-        mbar_expect_tx(v_full(sv), Lay::kTileBytes);
+          tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, w.m0, w.hq, w.b);
+        q_issued = u & 1;
+        if (u > 0 && !(ok = mbar_wait(o_empty, (u - 1) & 1, ctl))) break;
+        mbar_expect_tx(o_full, Lay::kTileBytes);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(sb + Lay::kVOff + sv * Lay::kTileBytes + h * kTile * 128, &tmV, v_full(sv),
-                      h * 64, n0, g, b);
-        issued_v[sv] = (it / SV) & 1;
+          tma_load_4d(sb + Lay::kDOOff + h * kTile * 128, &tmDO, o_full, h * 64, w.m0, w.hq, w.b);
+        o_issued = u & 1;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int sk = c % SK, sv = c % SV;
+          const int n0 = (w.nlo + it) * kTile;
+          if (!(ok = mbar_wait(k_empty(sk), ((c / SK) & 1) ^ 1, ctl))) break;
+          mbar_expect_tx(k_full(sk), Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
+                        k_full(sk), h * 64, n0, w.g, w.b);
+          issued_k[sk] = (c / SK) & 1;
+          if (!(ok = mbar_wait(v_empty(sv), ((c / SV) & 1) ^ 1, ctl))) break;
+          mbar_expect_tx(v_full(sv), Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kVOff + sv * Lay::kTileBytes + h * kTile * 128, &tmV,
+                        v_full(sv), h * 64, n0, w.g, w.b);
+          issued_v[sv] = (c / SV) & 1;
+        }
+        ++u;
       }
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mbar_wait(q_full, 0, ign);
+        if (q_issued >= 0) mbar_wait(q_full, q_issued, ign);
+        if (o_issued >= 0) mbar_wait(o_full, o_issued, ign);
         for (int s = 0; s < SK; ++s)
           if (issued_k[s] >= 0) mbar_wait(k_full(s), issued_k[s], ign);
         for (int s = 0; s < SV; ++s)
@@ -668,66 +710,73 @@ __global__ void __launch_bounds__(352, 1)
     // ===================== MMA issuers (one thread each) =====================
     // Warp 9 runs the score chain: S(i) into buffer i % 2 once K(i) has landed
     // and the dQ MMA of block i - 2 has read dS out of that buffer.  Warp 10
-    // runs dP one block ahead of dQ: dP(i + 1) as soon as both warpgroups have
-    // loaded dP(i), then dQ(i) once dS(i) is ready.
-    if (lane == 0 && nt > 0) {
+    // runs dP one block ahead of dQ within an item: dP(i + 1) as soon as both
+    // warpgroups have loaded dP(i), then dQ(i) once dS(i) is ready.  Block
+    // indices run on across items.
+    if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
       const bool chain_s = (warp == 9);
-      auto issue_dp = [&](int it) {
-        const uint32_t vs = sb + Lay::kVOff + (it % SV) * Lay::kTileBytes;
+      auto issue_dp = [&](int c) -> bool {
+        const int sv = c % SV;
+        if (!issuer_wait(v_full(sv), (c / SV) & 1, ctl)) return false;
+        if (c > 0 && !issuer_wait(dp_used, (c - 1) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + Lay::kDPCol,
                  smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
                  smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
         mma_commit(dp_full);
-        mma_commit(v_empty(it % SV));
+        mma_commit(v_empty(sv));
+        return true;
       };
-      bool ok = issuer_wait(q_full, 0, ctl);
-      if (ok && !chain_s) {
-        ok = issuer_wait(v_full(0), 0, ctl);
-        if (ok) {
-          tc_fence_after();
-          issue_dp(0);
-        }
-      }
-      for (int it = 0; it < nt && ok; ++it) {
-        const int x = it & 1;
-        const int sk = it % SK;
-        const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
-        if (chain_s) {
-          if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
-          if (it >= 2 && !(ok = issuer_wait(dq_done(x), ((it >> 1) - 1) & 1, ctl))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + kTile * x,
-                   smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
-                   smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-          mma_commit(s_full(x));
-          mma_commit(k_empty(sk));
-        } else {
-          if (it + 1 < nt) {
-            const int sv = (it + 1) % SV;
-            if (!(ok = issuer_wait(v_full(sv), ((it + 1) / SV) & 1, ctl))) break;
-            if (!(ok = issuer_wait(dp_used, it & 1, ctl))) break;
+      int c = 0;  // key blocks so far, over all items
+      int u = 0;  // items with a non-empty band so far
+      bool ok = true;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (!(ok = issuer_wait(chain_s ? q_full : o_full, u & 1, ctl))) break;
+        if (!chain_s && !(ok = issue_dp(c))) break;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int x = c & 1;
+          const int sk = c % SK;
+          const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+          if (chain_s) {
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (c >= 2 && !(ok = issuer_wait(dq_done(x), ((c >> 1) - 1) & 1, ctl))) break;
             tc_fence_after();
-            issue_dp(it + 1);
-          }
-          if (!(ok = issuer_wait(k_full(sk), (it / SK) & 1, ctl))) break;
-          if (!(ok = issuer_wait(ds_full, it & 1, ctl))) break;
-          tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk),
-                   smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(dq_done(x));
-          mma_commit(k_empty(sk));
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + kTile * x,
+                     smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
+                     smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(s_full(x));
+            mma_commit(k_empty(sk));
+          } else {
+            if (it + 1 < w.nt && !(ok = issue_dp(c + 1))) break;
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (!(ok = issuer_wait(ds_full, c & 1, ctl))) break;
+            tc_fence_after();
+            // the item's first dQ MMA overwrites the accumulator: every
+            // warpgroup thread read the previous item's dQ before marking dS ready
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk),
+                     smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(dq_done(x));
+            mma_commit(k_empty(sk));
+          }
         }
+        if (!ok) break;
+        mma_commit(chain_s ? q_empty : o_empty);  // the item's Q / dO is read
+        if (!chain_s) mma_commit(acc_done);
+        ++u;
       }
-      if (ok && !chain_s) mma_commit(acc_done);
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
@@ -739,125 +788,137 @@ __global__ void __launch_bounds__(352, 1)
     // ===== compute warpgroup wg: key columns [64 wg, 64 wg + 64); thread = query row =====
     const int wg = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
-    const int i = m0 + row;
     const int c0w = kBlk * wg;
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + wg * 512;
-    float l2 = INFINITY, dd = 0.f;
-    if (i < p.L) {
-      const int64_t idx = (static_cast<int64_t>(b) * p.Hq + hq) * p.L + i;
-      l2 = p.lse[idx] * kLog2e;
-      dd = p.dvec[idx];
-      if (l2 == -INFINITY) l2 = INFINITY;
-    }
-    const float* brow = nullptr;
-    if constexpr (BIAS == kBiasDense)
-      brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
-             static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
     bool ok = true;
-    for (int it = 0; it < nt; ++it) {
-      const int x = it & 1;
-      const int n0 = (nlo + it) * kTile + c0w;  // first key of this warpgroup
-      const float* lut_row = nullptr;
-      if constexpr (BIAS == kBiasT5) {
-        // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
-        float* lt = lut + (it & 1) * 256;
-        const int base = n0 - m0 - (kTile - 1);
-        for (int r = row; r < kTile + kBlk - 1; r += kTile)
-          lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
-        named_barrier(1 + wg, kTile);
-        lut_row = lt + (kTile - 1) - row;
+    int c = 0;  // key blocks so far, over all items
+    int u = 0;  // items with a non-empty band so far
+    for (int id = blockIdx.x; id < n_items; id += gridDim.x) {
+      const Item w = item_at(id);
+      const int m0 = w.m0, hq = w.hq, b = w.b, nt = w.nt;
+      const int i = m0 + row;
+      float l2 = INFINITY, dd = 0.f;
+      if (i < p.L) {
+        const int64_t idx = (static_cast<int64_t>(b) * p.Hq + hq) * p.L + i;
+        l2 = p.lse[idx] * kLog2e;
+        dd = p.dvec[idx];
+        if (l2 == -INFINITY) l2 = INFINITY;
       }
-      int lo = 0, hi = kBlk - 1;
-      bool full = n0 + kBlk <= p.L;
-      if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
-      if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
-      if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
-      if (!full) {
-        if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
-        hi = min(hi, p.L - 1 - n0);
-        if (p.causal) hi = min(hi, i - n0);
-        if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
-      }
-      if (ok) ok = mbar_wait(s_full(x), (it >> 1) & 1, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) continue;
-      tc_fence_after();
-      const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
-      uint32_t pr[64];  // S row, then P (fp32 bits)
-      tmem_ld64_sync(tSx, pr);
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < kBlk; ++c) {
-          float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -l2);
-          if constexpr (BIAS == kBiasT5) xv += lut_row[c];
-          if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + c], kLog2e, xv);
-          pr[c] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
+      const float* brow = nullptr;
+      if constexpr (BIAS == kBiasDense)
+        brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
+               static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
+      for (int it = 0; it < nt; ++it, ++c) {
+        const int x = c & 1;
+        const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup
+        const float* lut_row = nullptr;
+        if constexpr (BIAS == kBiasT5) {
+          // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
+          float* lt = lut + (c & 1) * 256;
+          const int base = n0 - m0 - (kTile - 1);
+          for (int r = row; r < kTile + kBlk - 1; r += kTile)
+            lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
+          named_barrier(1 + wg, kTile);
+          lut_row = lt + (kTile - 1) - row;
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBlk; ++c) {
-          const bool vis = (c >= lo) && (c <= hi);
-          float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -l2);
-          if constexpr (BIAS == kBiasT5) xv += lut_row[c];
-          if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + (vis ? c : 0)], kLog2e, xv);
-          pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+        int lo = 0, hi = kBlk - 1;
+        bool full = n0 + kBlk <= p.L;
+        if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
+        if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
+        if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
+        if (!full) {
+          if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
+          hi = min(hi, p.L - 1 - n0);
+          if (p.causal) hi = min(hi, i - n0);
+          if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
         }
-      }
-      if (ok) ok = mbar_wait(dp_full, it & 1, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) continue;
-      tc_fence_after();
-      uint32_t pk[32];  // dS as bf16 pairs
+        if (ok) ok = mbar_wait(s_full(x), (c >> 1) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) continue;
+        tc_fence_after();
+        const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
+        uint32_t pr[64];  // S row, then P (fp32 bits)
+        tmem_ld64_sync(tSx, pr);
+        if (full) {
 #pragma unroll
-      for (int cc = 0; cc < kBlk; cc += 32) {
-        uint32_t dr[32];
-        tmem_ld32_sync(tDP + cc, dr);
-        if (cc + 32 == kBlk) {
-          tc_fence_before();
-          mbar_arrive(dp_used);  // the dP columns may now take block it + 1
-        }
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dd);
-          const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dd);
-          pk[(cc + c) >> 1] = pack_bf16x2(d0, d1);
-        }
-      }
-      // dS over the first 32 of this warpgroup's columns of its S buffer
-      tmem_st16(tSx, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-      tmem_st16(tSx + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(ds_full);
-    }
-    // ------------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -------------
-    if (ok && nt > 0) ok = mbar_wait(acc_done, 0, ctl);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after();
-      __nv_bfloat16* dst = p.dq + static_cast<int64_t>(b) * p.sq_b + static_cast<int64_t>(i) * p.sq_l +
-                           static_cast<int64_t>(hq) * p.sq_h;
-#pragma unroll
-      for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
-        uint32_t r[32];
-        if (nt > 0) {
-          tmem_ld32_sync(tmem + lane_bits + Lay::kDQCol + c, r);
+          for (int cc = 0; cc < kBlk; ++cc) {
+            float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
+            if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + cc], kLog2e, xv);
+            pr[cc] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(cc) ? exp2_fma(xv) : fast_exp2(xv));
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+          for (int cc = 0; cc < kBlk; ++cc) {
+            const bool vis = (cc >= lo) && (cc <= hi);
+            float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
+            if constexpr (BIAS == kBiasDense) xv += vis ? brow[n0 + cc] * kLog2e : 0.f;
+            pr[cc] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+          }
         }
-        uint32_t pk[16];
+        if (ok) ok = mbar_wait(dp_full, c & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) continue;
+        tc_fence_after();
+        uint32_t pk[32];  // dS as bf16 pairs
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale,
-                              __uint_as_float(r[2 * e + 1]) * p.scale);
+        for (int cc = 0; cc < kBlk; cc += 32) {
+          uint32_t dr[32];
+          tmem_ld32_sync(tDP + cc, dr);
+          if (cc + 32 == kBlk) {
+            tc_fence_before();
+            mbar_arrive(dp_used);  // the dP columns may now take the next block
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float d0 = __uint_as_float(pr[cc + e]) * (__uint_as_float(dr[e]) - dd);
+            const float d1 = __uint_as_float(pr[cc + e + 1]) * (__uint_as_float(dr[e + 1]) - dd);
+            pk[(cc + e) >> 1] = pack_bf16x2(d0, d1);
+          }
+        }
+        // dS over the first 32 of this warpgroup's columns of its S buffer
+        tmem_st16(tSx, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        tmem_st16(tSx + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(ds_full);
+      }
+      // ----------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -----------
+      // Items without a visible key (none exist for the masks accepted at the
+      // boundary) store zeros without touching tensor memory.
+      if (nt > 0) {
+        if (ok) ok = mbar_wait(acc_done, u & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        ++u;
+      }
+      if (ok) {
+        uint32_t r[D / 2];
+        if (nt > 0) {
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 2; cc += 32)
+            tmem_ld32_sync(tmem + lane_bits + Lay::kDQCol + wg * (D / 2) + cc,
+                           *reinterpret_cast<uint32_t(*)[32]>(r + cc));
+        } else {
+#pragma unroll
+          for (int e = 0; e < D / 2; ++e) r[e] = 0u;
+        }
         if (i < p.L) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+          __nv_bfloat16* dst = p.dq + static_cast<int64_t>(b) * p.sq_b +
+                               static_cast<int64_t>(i) * p.sq_l + static_cast<int64_t>(hq) * p.sq_h +
+                               wg * (D / 2);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int cc = 0; cc < D / 2; cc += 8) {
+            uint4 v4;
+            v4.x = pack_bf16x2(__uint_as_float(r[cc]) * p.scale, __uint_as_float(r[cc + 1]) * p.scale);
+            v4.y = pack_bf16x2(__uint_as_float(r[cc + 2]) * p.scale, __uint_as_float(r[cc + 3]) * p.scale);
+            v4.z = pack_bf16x2(__uint_as_float(r[cc + 4]) * p.scale, __uint_as_float(r[cc + 5]) * p.scale);
+            v4.w = pack_bf16x2(__uint_as_float(r[cc + 6]) * p.scale, __uint_as_float(r[cc + 7]) * p.scale);
+            *reinterpret_cast<uint4*>(dst + cc) = v4;
+          }
         }
       }
     }
@@ -872,6 +933,7 @@ __global__ void __launch_bounds__(352, 1)
 }
 
 // ------------------------------------------------------------- launchers
+// Launch selection bits of the backward (sdpa_bwd_phases).
 constexpr uint32_t kPhasePre = 1u, kPhaseDq = 2u, kPhaseDkdv = 4u;
 
 template <int D, int BIAS>
@@ -891,7 +953,11 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, uint32_t phases,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(ntiles, p.Hq, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(
+    // persistent: one CTA per SM (or per work item, if fewer)
+    const int64_t items = static_cast<int64_t>(ntiles) * p.Hq * p.B;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    kern<<<static_cast<int>(items < sms ? items : sms), Lay::kThreads, Lay::kSmemAlloc, st>>>(
         p, m.q128, m.k128, m.v128, m.dout128);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -150,20 +150,6 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
   return SDPA_OK;
 }
 
-// Streaming multiprocessors of the current device (persistent grids), cached
-// per device.
-int sm_count() {
-  constexpr int kDevs = 64;
-  static int cached[kDevs] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < kDevs && cached[dev] > 0) return cached[dev];
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < kDevs) cached[dev] = n;
-  return n;
-}
-
 template <int D, int BIAS>
 cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
                        const CUtensorMap& v, cudaStream_t st) {
