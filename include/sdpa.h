@@ -91,7 +91,8 @@ typedef enum sdpa_bias_kind {
  * the scale and is not itself scaled; it takes part in LSE.
  *   DENSE: ptr -> float32 with element strides stride_b, stride_h, stride_i
  *          (j contiguous; 0 broadcasts over that index); ptr 16-byte aligned,
- *          stride_i a multiple of 4.  A value of -inf masks (i, j); a row
+ *          stride_b, stride_h, stride_i multiples of 4 (rows are read in
+ *          16-byte pieces).  A value of -inf masks (i, j); a row
  *          with no visible key yields O = 0, LSE = -inf, zero gradients.
  *   T5:    ptr -> float32 table[num_buckets][Hq] (row-major), bucket of the
  *          signed distance j - i by the T5 closed form (Raffel et al. 2020):

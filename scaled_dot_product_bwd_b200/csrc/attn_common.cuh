@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "exp2_poly.cuh"
+#include "sm100.cuh"
 
 namespace sdpa {
 
@@ -111,6 +112,19 @@ __device__ __forceinline__ void query_tile_range(const AttnParams& p, int n0, in
   if (p.wl >= 0) imax = min(imax, n_last + p.wl);
   mlo = imin / kTile;
   mhi = (imax >= imin) ? imax / kTile + 1 : mlo;
+}
+
+// L2 prefetch of the dense-bias rows [m0, m0 + 128) x keys [n0, n0 + 128) of
+// one (batch, query head), clipped to L (rounded up to 16 bytes, which stays
+// inside the row: row strides are multiples of 4 floats).  One thread issues.
+__device__ __forceinline__ void prefetch_bias_tile(const AttnParams& p, int b, int hq, int m0,
+                                                   int n0) {
+  const int cols = min(kTile, p.L - n0);
+  if (cols <= 0) return;
+  const uint32_t bytes = static_cast<uint32_t>((cols + 3) & ~3) * 4u;
+  const float* base = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h + n0;
+  const int rows = min(kTile, p.L - m0);
+  for (int r = 0; r < rows; ++r) prefetch_l2(base + static_cast<int64_t>(m0 + r) * p.sb_i, bytes);
 }
 
 // True when every (query, key) pair of the tile (rows m0.., keys n0..) is

@@ -686,6 +686,7 @@ __global__ void __launch_bounds__(352, 1)
             tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
                         k_full(sk), h * 64, n0, w.g, w.b);
           issued_k[sk] = (c / SK) & 1;
+          if constexpr (BIAS == kBiasDense) prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
           if (!(ok = mbar_wait(v_empty(sv), ((c / SV) & 1) ^ 1, ctl))) break;
           mbar_expect_tx(v_full(sv), Lay::kTileBytes);
           for (int h = 0; h < D / 64; ++h)
@@ -841,12 +842,30 @@ __global__ void __launch_bounds__(352, 1)
         const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
         uint32_t pr[64];  // S row, then P (fp32 bits)
         tmem_ld64_sync(tSx, pr);
-        if (full) {
+        if (full && BIAS == kBiasDense) {
+          // the row's 64 bias values as 16-byte loads, 32 at a time
+          const float4* b4 = reinterpret_cast<const float4*>(brow + n0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float4 bb[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) bb[q] = b4[8 * h + q];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float bv[4] = {bb[q].x, bb[q].y, bb[q].z, bb[q].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int cc = 32 * h + 4 * q + e;
+                const float xv = fmaf(bv[e], kLog2e, fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2));
+                pr[cc] = __float_as_uint(fast_exp2(xv));
+              }
+            }
+          }
+        } else if (full) {
 #pragma unroll
           for (int cc = 0; cc < kBlk; ++cc) {
             float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
             if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
-            if constexpr (BIAS == kBiasDense) xv = fmaf(brow[n0 + cc], kLog2e, xv);
             pr[cc] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(cc) ? exp2_fma(xv) : fast_exp2(xv));
           }
         } else {

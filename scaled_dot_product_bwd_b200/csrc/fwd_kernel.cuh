@@ -215,6 +215,9 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_4d(ring + s * Lay::kTileBytes + h * kTile * 128, map, full, h * 64,
                         (w.nlo + it) * kTile, w.g, w.b);
           issued[s] = static_cast<int>(ph);
+          if constexpr (BIAS == kBiasDense) {
+            if (is_k) prefetch_bias_tile(p, w.b, w.hq, w.m0, (w.nlo + it) * kTile);
+          }
         }
         ++u;
       }
@@ -360,12 +363,31 @@ __global__ void __launch_bounds__(384, 1)
             pmax = fmaxf(ma, mb) * p.scale_log2;
           } else {
             float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (full) {
+            if (full && BIAS == kBiasDense) {
+              // the row's 64 bias values as 16-byte loads, 32 at a time
+              const float4* b4 = reinterpret_cast<const float4*>(brow + n0);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                float4 bb[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) bb[q] = b4[8 * h + q];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const float bv[4] = {bb[q].x, bb[q].y, bb[q].z, bb[q].w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int c = 32 * h + 4 * q + e;
+                    const float v = fmaf(bv[e], kLog2e, __uint_as_float(xs[c]) * p.scale_log2);
+                    xs[c] = __float_as_uint(v);
+                    tm[c & 3] = fmaxf(tm[c & 3], v);
+                  }
+                }
+              }
+            } else if (full) {
 #pragma unroll
               for (int c = 0; c < kBlk; ++c) {
                 float v = __uint_as_float(xs[c]) * p.scale_log2;
                 if constexpr (BIAS == kBiasT5) v += lut_row[c];
-                if constexpr (BIAS == kBiasDense) v = fmaf(brow[n0 + c], kLog2e, v);
                 xs[c] = __float_as_uint(v);
                 tm[c & 3] = fmaxf(tm[c & 3], v);
               }

@@ -129,7 +129,8 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
     if (bias->kind == SDPA_BIAS_DENSE) {
       if (!bias->ptr || !aligned16(bias->ptr)) return SDPA_ERR_INVALID_ARG;
       if (bias->stride_b < 0 || bias->stride_h < 0 || bias->stride_i < 0) return SDPA_ERR_INVALID_ARG;
-      if (bias->stride_i % 4 != 0) return SDPA_ERR_INVALID_ARG;
+      if (bias->stride_b % 4 != 0 || bias->stride_h % 4 != 0 || bias->stride_i % 4 != 0)
+        return SDPA_ERR_INVALID_ARG;
       p.bias_kind = kBiasDense;
       p.bias = bias->ptr;
       p.sb_b = bias->stride_b;

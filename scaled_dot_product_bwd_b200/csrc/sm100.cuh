@@ -144,6 +144,12 @@ __device__ __forceinline__ bool issuer_wait(uint32_t bar, uint32_t parity, const
   return kIssuerPoll ? mbar_wait_poll(bar, parity, ctl) : mbar_wait(bar, parity, ctl);
 }
 
+// Ask L2 to fetch `bytes` (a multiple of 16) of global memory at `src`
+// (16-byte aligned); no data is returned.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Named barrier over `count` threads (multiple of 32), id 1..15.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -83,6 +83,8 @@ def test_fwd_rejects_bad_bias(lib):
            binding.BiasDesc(1, 0, 0, 0, 128, 0, 0, 0),               # dense, null
            binding.BiasDesc(1, 0x10004, 0, 0, 128, 0, 0, 0),         # dense, misaligned
            binding.BiasDesc(1, 0x10000, 0, 0, 130, 0, 0, 0),         # dense, stride_i % 4
+           binding.BiasDesc(1, 0x10000, 0, 2, 128, 0, 0, 0),         # dense, stride_h % 4
+           binding.BiasDesc(1, 0x10000, 6, 0, 128, 0, 0, 0),         # dense, stride_b % 4
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 31, 128, 1),        # T5, odd buckets (bidir)
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 256, 128, 1),       # T5, too many buckets
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 8, 1),          # T5, max_distance <= max_exact
