@@ -50,12 +50,12 @@ CONFIGS = {
 NCU_TRAFFIC = {
     # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
     # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
-    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_164_480 + 22_958_848) / 2,
-                                    source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
-    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(169_956_608 + 43_143_168) / 2,
-                                  source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
-    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_805_120 + 33_030_400) / 2,
-                               source_hash="0f42eb422f58356721b9f91e644b204a6f0e1839def0159fbb872be16fee7389"),
+    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_165_248 + 22_864_896) / 2,
+                                    source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
+    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_898_176 + 42_148_352) / 2,
+                                  source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
+    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_808_448 + 32_648_960) / 2,
+                               source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
 }
 
 
