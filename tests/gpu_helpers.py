@@ -21,8 +21,14 @@ def case_inputs(c):
 
 
 def mask_kw(c):
-    return dict(causal=c.get("causal", False), window_left=c.get("wl", -1),
-                window_right=c.get("wr", -1))
+    """Mask, scale and T5 options of a case (the same keywords on both sides)."""
+    kw = dict(causal=c.get("causal", False), window_left=c.get("wl", -1),
+              window_right=c.get("wr", -1))
+    if "scale" in c:
+        kw["scale"] = c["scale"]
+    if "t5_bidirectional" in c:
+        kw["t5_bidirectional"] = c["t5_bidirectional"]
+    return kw
 
 
 def run_cuda(c, inp, backward=True):

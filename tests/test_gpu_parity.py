@@ -27,6 +27,21 @@ CASES = {
     "window_zero": dict(B=1, Hq=2, Hkv=2, L=200, d=128, causal=True, wl=0),
     "window_ge_L": dict(B=1, Hq=2, Hkv=1, L=300, d=128, causal=True, wl=4096),
     "short_ragged_d64": dict(B=3, Hq=2, Hkv=1, L=37, d=64, causal=True),
+    # dense bias broadcast over heads / over batch and heads; L = 132 leaves the
+    # second warpgroup's key columns of the last tile entirely past L
+    "dense_bias_broadcast_heads": dict(B=2, Hq=2, Hkv=1, L=132, d=64, causal=True, bias="dense",
+                                       bias_shape=(2, 1, 132, 132)),
+    "dense_bias_broadcast_all_d128": dict(B=2, Hq=2, Hkv=2, L=132, d=128, bias="dense",
+                                          bias_shape=(1, 1, 132, 132)),
+    # a scale other than 1/sqrt(d), and a negative one (the raw-max shortcut of
+    # full tiles applies to positive scales only).  Much larger scales make the
+    # softmax so peaked that dQ's bf16 rounding of dS and of O (in the row sums
+    # D) exceeds the fixed 1e-2 absolute tolerance on small entries.
+    "scale_0p15_causal_d128": dict(B=1, Hq=2, Hkv=1, L=300, d=128, causal=True, scale=0.15),
+    "negative_scale_d64": dict(B=1, Hq=2, Hkv=2, L=260, d=64, scale=-0.08),
+    # decoder-style T5 buckets (distance folded to one sign) under a causal mask
+    "t5_unidirectional_causal_d64": dict(B=2, Hq=2, Hkv=2, L=280, d=64, causal=True, bias="t5",
+                                         t5_bidirectional=False),
 }
 
 
