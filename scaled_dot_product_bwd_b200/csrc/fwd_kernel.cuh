@@ -65,20 +65,26 @@ template <int D, int BIAS>
 struct FwdLayout {
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
   static constexpr int kNS = 3;                     // S buffers in tensor memory
+  // Dense bias at d = 64: each tile's 128 x 128 fp32 bias block comes by TMA
+  // into a 2-stage ring (4 boxes of 128 rows x 32 columns, 128-byte swizzle).
+  static constexpr bool kBiasTma = (BIAS == kBiasDense && D == 64);
+  static constexpr int kBiasTileBytes = kTile * kTile * 4;
+  static constexpr int kSB = kBiasTma ? 2 : 0;
   // K is needed up to three tiles ahead of V (the S buffers run ahead of P V).
-  static constexpr int kSK = (D == 128) ? 3 : 4;
-  static constexpr int kSV = (D == 128) ? 2 : 4;
+  static constexpr int kSK = (D == 128) ? 3 : (kBiasTma ? 2 : 4);
+  static constexpr int kSV = (D == 128) ? 2 : (kBiasTma ? 2 : 4);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kTileBytes;
   static constexpr int kVOff = kKOff + kSK * kTileBytes;
-  static constexpr int kRedOff = kVOff + kSV * kTileBytes;  // max[2][2][128], sum[2][2][128]
+  static constexpr int kBOff = kVOff + kSV * kTileBytes;    // bias ring (kBiasTma)
+  static constexpr int kRedOff = kBOff + kSB * kBiasTileBytes;  // max[2][2][128], sum[2][2][128]
   static constexpr int kRedBytes = 8 * kTile * 4;
   static constexpr int kLutOff = kRedOff + kRedBytes;       // T5 only: 2 WG x 2 x 256 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // q_full, q_empty, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
-  // s_full[NS], p_full[NS], pv_done[NS], acc_done, drain[2]
-  static constexpr int kNumBars = 2 + 2 * kSK + 2 * kSV + 3 * kNS + 3;
+  // s_full[NS], p_full[NS], pv_done[NS], acc_done, drain[2], b_full[2], b_empty[2]
+  static constexpr int kNumBars = 2 + 2 * kSK + 2 * kSV + 3 * kNS + 3 + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
   // 2 softmax warpgroups; warp 8 K producer, 9 S issuer, 10 PV issuer, 11 V producer
@@ -93,7 +99,8 @@ struct FwdLayout {
 template <int D, int BIAS>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmB) {
   using Lay = FwdLayout<D, BIAS>;
   constexpr int SK = Lay::kSK;
   constexpr int SV = Lay::kSV;
@@ -144,6 +151,9 @@ __global__ void __launch_bounds__(384, 1)
   auto pv_done = [&](int x) { return bar(kB + 2 * NS + x); };
   const uint32_t acc_done = bar(kB + 3 * NS);
   auto drain = [&](int x) { return bar(kB + 3 * NS + 1 + x); };
+  auto b_full = [&](int x) { return bar(kB + 3 * NS + 3 + x); };
+  auto b_empty = [&](int x) { return bar(kB + 3 * NS + 5 + x); };
+  constexpr bool BT = Lay::kBiasTma;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -166,6 +176,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(acc_done, 1);
     mbar_init(drain(0), 1);
     mbar_init(drain(1), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(b_full(x), 1);
+      mbar_init(b_empty(x), 2 * kTile);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -189,6 +203,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(map);
       if (is_k) tma_prefetch_desc(&tmQ);
       int issued[4] = {-1, -1, -1, -1};
+      int b_issued[2] = {-1, -1};
       int q_issued = -1;
       int c = 0;  // tiles loaded so far, over all items
       int u = 0;  // items with a non-empty band so far
@@ -215,7 +230,21 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_4d(ring + s * Lay::kTileBytes + h * kTile * 128, map, full, h * 64,
                         (w.nlo + it) * kTile, w.g, w.b);
           issued[s] = static_cast<int>(ph);
-          if constexpr (BIAS == kBiasDense) {
+          if constexpr (BT) {
+            if (is_k) {
+              // this tile's bias block: rows m0.., keys n0.. of (b, hq), 4 boxes
+              const int x = c & 1;
+              const uint32_t bph = (c >> 1) & 1;
+              if (!(ok = mbar_wait(b_empty(x), bph ^ 1, ctl))) break;
+              mbar_expect_tx(b_full(x), Lay::kBiasTileBytes);
+              const int n0 = (w.nlo + it) * kTile;
+              const int hb = p.sb_h ? w.hq : 0, bb = p.sb_b ? w.b : 0;
+              for (int q4 = 0; q4 < 4; ++q4)
+                tma_load_4d(sb + Lay::kBOff + x * Lay::kBiasTileBytes + q4 * (kTile * 128), &tmB,
+                            b_full(x), n0 + 32 * q4, w.m0, hb, bb);
+              b_issued[x] = static_cast<int>(bph);
+            }
+          } else if constexpr (BIAS == kBiasDense) {
             if (is_k) prefetch_bias_tile(p, w.b, w.hq, w.m0, (w.nlo + it) * kTile);
           }
         }
@@ -228,6 +257,8 @@ __global__ void __launch_bounds__(384, 1)
         if (q_issued >= 0) mbar_wait(q_full, q_issued, ign);
         for (int s = 0; s < stages; ++s)
           if (issued[s] >= 0) mbar_wait(is_k ? k_full(s) : v_full(s), issued[s], ign);
+        for (int x = 0; x < 2; ++x)
+          if (b_issued[x] >= 0) mbar_wait(b_full(x), b_issued[x], ign);
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -346,6 +377,9 @@ __global__ void __launch_bounds__(384, 1)
 
         // ---- phase A: this warpgroup's half of S_j and its partial row max
         if (ok) ok = mbar_wait(s_full(x), (gc / NS) & 1, ctl);
+        if constexpr (BT) {
+          if (ok) ok = mbar_wait(b_full(gc & 1), (gc >> 1) & 1, ctl);
+        }
         ok = __all_sync(0xffffffffu, ok);
         const bool live = ok;
         uint32_t xs[kBlk];  // raw accumulator bits (lean) or log2-unit scores
@@ -363,7 +397,29 @@ __global__ void __launch_bounds__(384, 1)
             pmax = fmaxf(ma, mb) * p.scale_log2;
           } else {
             float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (full && BIAS == kBiasDense) {
+            if constexpr (BT) {
+              // this warpgroup's 64 bias columns from the staged block: boxes
+              // 2 wg and 2 wg + 1, row `row`, 8 swizzled 16-byte chunks each
+              const uint8_t* bt = smem + Lay::kBOff + (gc & 1) * Lay::kBiasTileBytes;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint8_t* brw = bt + (2 * wg + h) * (kTile * 128) + row * 128;
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                  const float4 b4 = *reinterpret_cast<const float4*>(brw + ((k4 ^ (row & 7)) << 4));
+                  const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int c = 32 * h + 4 * k4 + e;
+                    float v = fmaf(bv[e], kLog2e, __uint_as_float(xs[c]) * p.scale_log2);
+                    if (!full) v = (c >= lo && c <= hi) ? v : -INFINITY;
+                    xs[c] = __float_as_uint(v);
+                    tm[c & 3] = fmaxf(tm[c & 3], v);
+                  }
+                }
+              }
+              mbar_arrive(b_empty(gc & 1));  // the bias block is read
+            } else if (full && BIAS == kBiasDense) {
               // the row's 64 bias values as 16-byte loads, 32 at a time
               const float4* b4 = reinterpret_cast<const float4*>(brow + n0);
 #pragma unroll

@@ -57,6 +57,26 @@ bool make_bshd_map(CUtensorMap* m, const void* base, int64_t B, int64_t L, int64
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dense fp32 bias [B|1, Hq|1, L, L] as a 4-D map (j, i, head, batch) with
+// boxes of 32 keys x 128 queries (128-byte swizzle); a broadcast index has
+// extent 1 and is always addressed at 0.
+bool make_bias_map(CUtensorMap* m, const AttnParams& p) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(p.sb_i) * 4;
+  const cuuint64_t head = p.sb_h ? static_cast<cuuint64_t>(p.sb_h) * 4 : row * p.L;
+  const cuuint64_t batch = p.sb_b ? static_cast<cuuint64_t>(p.sb_b) * 4 : head * (p.sb_h ? p.Hq : 1);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(p.L), static_cast<cuuint64_t>(p.L),
+                        static_cast<cuuint64_t>(p.sb_h ? p.Hq : 1),
+                        static_cast<cuuint64_t>(p.sb_b ? p.B : 1)};
+  cuuint64_t strides[3] = {row, head, batch};
+  cuuint32_t box[4] = {32, static_cast<cuuint32_t>(kTile), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(p.bias), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Integer thresholds of the T5 log buckets, evaluated in float64 exactly as
@@ -153,7 +173,7 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
 
 template <int D, int BIAS>
 cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
-                       const CUtensorMap& v, cudaStream_t st) {
+                       const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
   using Lay = FwdLayout<D, BIAS>;
   auto kern = fwd_kernel<D, BIAS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -164,17 +184,17 @@ cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensor
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int grid = static_cast<int>(items < sms ? items : sms);
-  kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v);
+  kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v, bmap);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
-                              const CUtensorMap& v, cudaStream_t st) {
+                              const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
   switch (p.bias_kind) {
-    case kBiasDense: return launch_fwd<D, kBiasDense>(p, q, k, v, st);
-    case kBiasT5: return launch_fwd<D, kBiasT5>(p, q, k, v, st);
-    default: return launch_fwd<D, kBiasNone>(p, q, k, v, st);
+    case kBiasDense: return launch_fwd<D, kBiasDense>(p, q, k, v, bmap, st);
+    case kBiasT5: return launch_fwd<D, kBiasT5>(p, q, k, v, bmap, st);
+    default: return launch_fwd<D, kBiasNone>(p, q, k, v, bmap, st);
   }
 }
 
@@ -243,8 +263,11 @@ sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k, co
       !make_bshd_map(&mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h))
     return SDPA_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128>(p, mq, mk, mv, cs)
-                               : dispatch_fwd_bias<64>(p, mq, mk, mv, cs);
+  CUtensorMap mb;
+  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias kernels
+  if (p.bias_kind == kBiasDense && !make_bias_map(&mb, p)) return SDPA_ERR_CUDA;
+  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128>(p, mq, mk, mv, mb, cs)
+                               : dispatch_fwd_bias<64>(p, mq, mk, mv, mb, cs);
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
