@@ -50,12 +50,12 @@ CONFIGS = {
 NCU_TRAFFIC = {
     # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
     # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
-    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_165_248 + 22_864_896) / 2,
-                                    source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
-    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_898_176 + 42_148_352) / 2,
-                                  source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
-    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_808_448 + 32_648_960) / 2,
-                               source_hash="e7fd7b11f4e520d045b2cfbc12d8c33a60dde6c2a5c344c5e13f18e82b15fd30"),
+    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(169_944_832 + 23_383_040) / 2,
+                                    source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
+    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_331_136 + 41_576_192) / 2,
+                                  source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
+    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_764_160 + 32_813_056) / 2,
+                               source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
 }
 
 
