@@ -40,6 +40,7 @@ constexpr int kDqMufuPer8 = 8;
 struct BwdMaps {
   CUtensorMap q128, dout128, k128, v128;  // 128-row boxes (resident tiles)
   CUtensorMap q64, dout64, k64, v64;      // 64-row boxes (streamed blocks)
+  CUtensorMap bias;                       // dense fp32 bias, 32 x 128 boxes
 };
 
 // ------------------------------------------------------------ preprocess
@@ -526,20 +527,27 @@ __global__ void __launch_bounds__(352, 1)
 template <int D, int BIAS>
 struct DqLayout {
   static constexpr int kTileBytes = kTile * D * 2;
+  // Dense bias at d = 64: each block's 128 x 128 fp32 bias comes by TMA into
+  // a 2-stage ring (4 boxes of 128 rows x 32 columns, 128-byte swizzle).
+  static constexpr bool kBiasTma = (BIAS == kBiasDense && D == 64);
+  static constexpr int kBiasTileBytes = kTile * kTile * 4;
+  static constexpr int kSB = kBiasTma ? 2 : 0;
   // K blocks are used until the block's dQ MMA, V blocks only until its dP
   // MMA: the K ring is the deeper one.
-  static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : 4;
-  static constexpr int kSV = (D == 128) ? 2 : 3;
+  static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : (kBiasTma ? 2 : 4);
+  static constexpr int kSV = (D == 128) ? 2 : (kBiasTma ? 2 : 3);
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTileBytes;
   static constexpr int kKOff = 2 * kTileBytes;                // K ring
   static constexpr int kVOff = kKOff + kSK * kTileBytes;      // V ring
-  static constexpr int kLutOff = kVOff + kSV * kTileBytes;    // T5 only: 2 WG x 2 x 256 floats
+  static constexpr int kBOff = kVOff + kSV * kTileBytes;      // bias ring (kBiasTma)
+  static constexpr int kLutOff = kBOff + kSB * kBiasTileBytes;  // T5 only: 2 WG x 2 x 256 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 4 * 256 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
-  // dp_full, dp_used, ds_full, acc_done, drain[2], q_empty, o_full, o_empty
-  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 13;
+  // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
+  // b_full[2], b_empty[2]
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 18;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
   static constexpr int kThreads = 352;  // 2 compute warpgroups, producer, two MMA issuers
@@ -552,7 +560,7 @@ template <int D, int BIAS>
 __global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __grid_constant__ CUtensorMap tmDO) {
+                  const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
   using Lay = DqLayout<D, BIAS>;
   constexpr int SK = Lay::kSK;
   constexpr int SV = Lay::kSV;
@@ -599,7 +607,11 @@ __global__ void __launch_bounds__(352, 1)
   auto dq_done = [&](int x) { return bar(kB + 2 + x); };  // dQ MMA of a block in buffer x done
   const uint32_t dp_full = bar(kB + 4);
   const uint32_t dp_used = bar(kB + 5);
-  const uint32_t ds_full = bar(kB + 6);
+  // dS of block i ready, by block parity: the dQ issuer issues dP(i + 1)
+  // before it waits for dS(i), so the warpgroups can finish dS(i + 1) before
+  // it looks; a single barrier would then have completed two phases and the
+  // wait for block i's parity would never succeed.
+  auto ds_full = [&](int x) { return x == 0 ? bar(kB + 6) : bar(kB + 13); };
   const uint32_t acc_done = bar(kB + 7);
   auto drain = [&](int x) { return bar(kB + 8 + x); };
   // Q is read only by the score issuer, dO only by the dP issuer: each tile is
@@ -607,6 +619,9 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t q_empty = bar(kB + 10);
   const uint32_t o_full = bar(kB + 11);
   const uint32_t o_empty = bar(kB + 12);
+  auto b_full = [&](int x) { return bar(kB + 14 + x); };
+  auto b_empty = [&](int x) { return bar(kB + 16 + x); };
+  constexpr bool BT = Lay::kBiasTma;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -615,6 +630,10 @@ __global__ void __launch_bounds__(352, 1)
     mbar_init(q_empty, 1);
     mbar_init(o_full, 1);
     mbar_init(o_empty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(b_full(x), 1);
+      mbar_init(b_empty(x), 2 * kTile);
+    }
     // K blocks are read by both issuers (S and dQ): a slot is free once each
     // issuer's last MMA on it has completed.
     for (int s = 0; s < SK; ++s) {
@@ -631,7 +650,8 @@ __global__ void __launch_bounds__(352, 1)
     }
     mbar_init(dp_full, 1);
     mbar_init(dp_used, 2 * kTile);
-    mbar_init(ds_full, 2 * kTile);
+    mbar_init(ds_full(0), 2 * kTile);
+    mbar_init(ds_full(1), 2 * kTile);
     mbar_init(acc_done, 1);
     mbar_init(drain(0), 1);
     mbar_init(drain(1), 1);
@@ -661,6 +681,7 @@ __global__ void __launch_bounds__(352, 1)
       for (int s = 0; s < SK; ++s) issued_k[s] = -1;
       for (int s = 0; s < SV; ++s) issued_v[s] = -1;
       int q_issued = -1, o_issued = -1;
+      int b_issued[2] = {-1, -1};
       int c = 0;  // key blocks so far, over all items
       int u = 0;  // items with a non-empty band so far
       bool ok = true;
@@ -686,7 +707,20 @@ __global__ void __launch_bounds__(352, 1)
             tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
                         k_full(sk), h * 64, n0, w.g, w.b);
           issued_k[sk] = (c / SK) & 1;
-          if constexpr (BIAS == kBiasDense) prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
+          if constexpr (BT) {
+            // this block's bias: rows m0.., keys n0.. of (b, hq), 4 boxes
+            const int x = c & 1;
+            const uint32_t bph = (c >> 1) & 1;
+            if (!(ok = mbar_wait(b_empty(x), bph ^ 1, ctl))) break;
+            mbar_expect_tx(b_full(x), Lay::kBiasTileBytes);
+            const int hb = p.sb_h ? w.hq : 0, bb = p.sb_b ? w.b : 0;
+            for (int q4 = 0; q4 < 4; ++q4)
+              tma_load_4d(sb + Lay::kBOff + x * Lay::kBiasTileBytes + q4 * (kTile * 128), &tmB,
+                          b_full(x), n0 + 32 * q4, w.m0, hb, bb);
+            b_issued[x] = static_cast<int>(bph);
+          } else if constexpr (BIAS == kBiasDense) {
+            prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
+          }
           if (!(ok = mbar_wait(v_empty(sv), ((c / SV) & 1) ^ 1, ctl))) break;
           mbar_expect_tx(v_full(sv), Lay::kTileBytes);
           for (int h = 0; h < D / 64; ++h)
@@ -701,6 +735,8 @@ __global__ void __launch_bounds__(352, 1)
         const WaitCtl ign{&never, p.wait_limit_ns};
         if (q_issued >= 0) mbar_wait(q_full, q_issued, ign);
         if (o_issued >= 0) mbar_wait(o_full, o_issued, ign);
+        for (int x = 0; x < 2; ++x)
+          if (b_issued[x] >= 0) mbar_wait(b_full(x), b_issued[x], ign);
         for (int s = 0; s < SK; ++s)
           if (issued_k[s] >= 0) mbar_wait(k_full(s), issued_k[s], ign);
         for (int s = 0; s < SV; ++s)
@@ -760,7 +796,7 @@ __global__ void __launch_bounds__(352, 1)
           } else {
             if (it + 1 < w.nt && !(ok = issue_dp(c + 1))) break;
             if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
-            if (!(ok = issuer_wait(ds_full, c & 1, ctl))) break;
+            if (!(ok = issuer_wait(ds_full(c & 1), (c >> 1) & 1, ctl))) break;
             tc_fence_after();
             // the item's first dQ MMA overwrites the accumulator: every
             // warpgroup thread read the previous item's dQ before marking dS ready
@@ -836,13 +872,36 @@ __global__ void __launch_bounds__(352, 1)
           if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
         }
         if (ok) ok = mbar_wait(s_full(x), (c >> 1) & 1, ctl);
+        if constexpr (BT) {
+          if (ok) ok = mbar_wait(b_full(c & 1), (c >> 1) & 1, ctl);
+        }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) continue;
         tc_fence_after();
         const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
         uint32_t pr[64];  // S row, then P (fp32 bits)
         tmem_ld64_sync(tSx, pr);
-        if (full && BIAS == kBiasDense) {
+        if constexpr (BT) {
+          // this warpgroup's 64 bias columns from the staged block: boxes
+          // 2 wg and 2 wg + 1, row `row`, 8 swizzled 16-byte chunks each
+          const uint8_t* bt = smem + Lay::kBOff + (c & 1) * Lay::kBiasTileBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t* brw = bt + (2 * wg + h) * (kTile * 128) + row * 128;
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 b4 = *reinterpret_cast<const float4*>(brw + ((k4 ^ (row & 7)) << 4));
+              const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int cc = 32 * h + 4 * k4 + e;
+                const float xv = fmaf(bv[e], kLog2e, fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2));
+                pr[cc] = __float_as_uint(fast_exp2(full || (cc >= lo && cc <= hi) ? xv : -INFINITY));
+              }
+            }
+          }
+          mbar_arrive(b_empty(c & 1));  // the bias block is read
+        } else if (full && BIAS == kBiasDense) {
           // the row's 64 bias values as 16-byte loads, 32 at a time
           const float4* b4 = reinterpret_cast<const float4*>(brow + n0);
 #pragma unroll
@@ -903,7 +962,7 @@ __global__ void __launch_bounds__(352, 1)
         tmem_st16(tSx + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(ds_full);
+        mbar_arrive(ds_full(c & 1));
       }
       // ----------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -----------
       // Items without a visible key (none exist for the masks accepted at the
@@ -977,7 +1036,7 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, uint32_t phases,
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
     kern<<<static_cast<int>(items < sms ? items : sms), Lay::kThreads, Lay::kSmemAlloc, st>>>(
-        p, m.q128, m.k128, m.v128, m.dout128);
+        p, m.q128, m.k128, m.v128, m.dout128, m.bias);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

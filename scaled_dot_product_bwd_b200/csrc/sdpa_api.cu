@@ -315,6 +315,8 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
          make_bshd_map(mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows) &&
          make_bshd_map(mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows);
   }
+  std::memset(&maps.bias, 0, sizeof(maps.bias));  // read only by the dense-bias kernels
+  if (ok && p.bias_kind == kBiasDense) ok = make_bias_map(&maps.bias, p);
   if (!ok) return SDPA_ERR_CUDA;
   cudaError_t e =
       launch_bwd(p, maps, static_cast<int>(s.d), phases, static_cast<cudaStream_t>(stream));
