@@ -50,12 +50,12 @@ CONFIGS = {
 NCU_TRAFFIC = {
     # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
     # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
-    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(169_944_832 + 23_383_040) / 2,
-                                    source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
-    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_331_136 + 41_576_192) / 2,
-                                  source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
-    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_764_160 + 32_813_056) / 2,
-                               source_hash="e286bd2ff5a5f0c3d9df5ddb4cd34d28edee4d8c9b01c3d9ebcaead8bac14173"),
+    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(169_943_808 + 22_621_952) / 2,
+                                    source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
+    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_351_616 + 43_025_920) / 2,
+                                  source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
+    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_755_712 + 33_460_992) / 2,
+                               source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
 }
 
 
