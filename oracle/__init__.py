@@ -7,7 +7,9 @@ from .sdpa_oracle import (  # noqa: F401
     attention_backward,
     attention_forward,
     attention_probs,
+    dense_bias_gradient,
     head_scores,
     t5_relative_bucket,
+    t5_table_gradient,
     visibility_mask,
 )

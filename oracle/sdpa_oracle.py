@@ -39,6 +39,13 @@ What it computes, and where each piece comes from:
   rule to the definition above (dP = dO V^T, dS = P * (dP - rowsum(P*dP)),
   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO, with dK / dV summed over
   the query heads that share a KV head).
+* Bias gradients: the scores are linear in the bias with coefficient 1, so
+  the gradient of a dense bias is dS itself, summed over every index along
+  which the bias is broadcast, and the gradient of a T5 table entry
+  table[k, h] is the sum of dS over all (b, i, j) with bucket(j - i) = k in
+  head h (chain rule through the table lookup).  The pages name a learnable
+  relative-position bias for training (catie-aq/flashT5 README, "T5-like
+  relative position encoding biases") but print no gradient.
 * LSE is the natural-log log-sum-exp of each score row (bias included); a row
   with no visible key has LSE = -inf, output 0 and zero gradients.
 """
@@ -55,6 +62,8 @@ __all__ = [
     "attention_forward",
     "attention_backward",
     "attention_probs",
+    "dense_bias_gradient",
+    "t5_table_gradient",
 ]
 
 
@@ -133,7 +142,9 @@ def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
     """Additive bias for one (batch, query head), [L, L] float64 (or 0)."""
     out = 0.0
     if bias is not None:
-        out = out + bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0]
+        # a bias row of extent 1 is broadcast over the query rows
+        out = out + np.broadcast_to(
+            bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0], (L, L))
     if t5_table is not None:
         i = np.arange(L)[:, None]
         j = np.arange(L)[None, :]
@@ -275,3 +286,36 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     if return_dbias:
         return dQ, dK, dV, dB
     return dQ, dK, dV
+
+
+# --------------------------------------------------------------------------
+# Bias gradients (chain rule through the additive bias; catie-aq/flashT5
+# README, "Full attention biases" and "T5-like relative position encoding
+# biases").
+# --------------------------------------------------------------------------
+def dense_bias_gradient(dS, bias_shape):
+    """Gradient of a dense bias of shape ``bias_shape`` = [B|1, Hq|1, L|1, L]
+    from dS [B, Hq, L, L]: dS summed over each index where the bias has
+    extent 1 (it was broadcast there), in float64."""
+    dS = np.asarray(dS, dtype=np.float64)
+    assert len(bias_shape) == 4 and bias_shape[3] == dS.shape[3]
+    axes = tuple(a for a in range(3) if bias_shape[a] == 1 and dS.shape[a] != 1)
+    out = dS.sum(axis=axes, keepdims=True) if axes else dS.copy()
+    assert out.shape == tuple(bias_shape)
+    return out
+
+
+def t5_table_gradient(dS, num_buckets: int = 32, max_distance: int = 128,
+                      bidirectional: bool = True):
+    """Gradient of a T5 table [num_buckets, Hq] from dS [B, Hq, L, L]:
+    grad[k, h] = sum of dS[b, h, i, j] over every (b, i, j) whose distance
+    j - i falls in bucket k (one explicit scatter-add per head)."""
+    dS = np.asarray(dS, dtype=np.float64)
+    B, Hq, L, Lk = dS.shape
+    i = np.arange(L)[:, None]
+    j = np.arange(Lk)[None, :]
+    bucket = t5_relative_bucket(j - i, num_buckets, max_distance, bidirectional)
+    grad = np.zeros((num_buckets, Hq))
+    for h in range(Hq):
+        np.add.at(grad[:, h], bucket.ravel(), dS[:, h].sum(axis=0).ravel())
+    return grad

@@ -13,7 +13,8 @@ import pytest
 import torch
 
 from oracle import (attention_backward, attention_forward, attention_probs,
-                    head_scores, t5_relative_bucket, visibility_mask)
+                    dense_bias_gradient, head_scores, t5_relative_bucket,
+                    t5_table_gradient, visibility_mask)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -317,6 +318,55 @@ def test_dense_bias_gradient_central_differences():
                        - _loss(q, k, v, do, dict(causal=True, bias=bm))) / (2 * h)
                 want = dB[0, hq, i, j] if M[i, j] else 0.0
                 assert abs(num - want) < 1e-7
+
+
+@pytest.mark.parametrize("bias_shape", [(1, 2, 5, 5), (2, 1, 5, 5), (1, 1, 5, 5),
+                                        (2, 2, 1, 5), (1, 1, 1, 5)])
+def test_broadcast_bias_gradient_central_differences(bias_shape):
+    # A broadcast bias feeds every (b, h, i) it is broadcast over, so its
+    # gradient is the sum of dS over those copies.
+    B, L, Hq, Hkv, d = 2, 5, 2, 1, 3
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=23)
+    bias = rnd(bias_shape, 10)
+    kw = dict(causal=False, window_left=3, window_right=1, bias=bias)
+    *_, dS = attention_backward(q, k, v, do, return_dbias=True, **kw)
+    g = dense_bias_gradient(dS, bias_shape)
+    assert g.shape == bias_shape
+    h = 1e-6
+    it = np.nditer(bias, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        bp = bias.copy(); bp[idx] += h
+        bm = bias.copy(); bm[idx] -= h
+        num = (_loss(q, k, v, do, {**kw, "bias": bp})
+               - _loss(q, k, v, do, {**kw, "bias": bm})) / (2 * h)
+        assert abs(num - g[idx]) < 1e-7, (idx, num, g[idx])
+
+
+@pytest.mark.parametrize("bidirectional,causal", [(True, False), (True, True), (False, True),
+                                                  (False, False)])
+def test_t5_table_gradient_central_differences(bidirectional, causal):
+    # 8 buckets over distances up to 11 with max_distance 6: exact, log-wide
+    # and clamped buckets all occur, on both sides when bidirectional.
+    B, L, Hq, Hkv, d = 2, 12, 2, 2, 3
+    nb, md = 8, 6
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=31)
+    table = rnd((nb, Hq), 12)
+    kw = dict(causal=causal, t5_table=table, t5_num_buckets=nb, t5_max_distance=md,
+              t5_bidirectional=bidirectional)
+    *_, dS = attention_backward(q, k, v, do, return_dbias=True, **kw)
+    g = t5_table_gradient(dS, nb, md, bidirectional)
+    h = 1e-6
+    for kb in range(nb):
+        for hq in range(Hq):
+            tp = table.copy(); tp[kb, hq] += h
+            tm = table.copy(); tm[kb, hq] -= h
+            num = (_loss(q, k, v, do, {**kw, "t5_table": tp})
+                   - _loss(q, k, v, do, {**kw, "t5_table": tm})) / (2 * h)
+            assert abs(num - g[kb, hq]) < 1e-7, (kb, hq, num, g[kb, hq])
+    # softmax rows sum to one, so each row of dS sums to zero, and so do the
+    # table gradient's columns (every (i, j) lands in exactly one bucket)
+    assert np.allclose(g.sum(axis=0), 0.0, atol=1e-12)
 
 
 def test_D_two_ways():
