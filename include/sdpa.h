@@ -92,7 +92,8 @@ typedef enum sdpa_bias_kind {
  *   DENSE: ptr -> float32 with element strides stride_b, stride_h, stride_i
  *          (j contiguous; 0 broadcasts over that index); ptr 16-byte aligned,
  *          stride_b, stride_h, stride_i multiples of 4 (rows are read in
- *          16-byte pieces).  A value of -inf masks (i, j); a row
+ *          16-byte pieces); stride_i = 0 (one row for every query) ->
+ *          SDPA_ERR_UNSUPPORTED.  A value of -inf masks (i, j); a row
  *          with no visible key yields O = 0, LSE = -inf, zero gradients.
  *   T5:    ptr -> float32 table[num_buckets][Hq] (row-major), bucket of the
  *          signed distance j - i by the T5 closed form (Raffel et al. 2020):
@@ -200,6 +201,39 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
                                const float* lse, const sdpa_bias_desc* bias,
                                const sdpa_mask_spec* mask, float scale, void* dq,
                                void* dk, void* dv, int32_t deterministic, void* stream);
+
+/*
+ * Backward plus the gradient of the additive bias, for training a learnable
+ * bias (catie-aq/flashT5 README: "Full attention biases" and "T5-like
+ * relative position encoding biases").  The scores are linear in the bias,
+ * so with dS = P (dP - D) as in sdpa_bwd:
+ *   DENSE: dbias[b, h, i, j] = sum of dS[b', h', i, j] over the (b', h')
+ *          that read bias[b, h, i, j]: dS itself for a full-shape bias,
+ *          summed over batch and / or heads where stride_b / stride_h = 0.
+ *          dbias is float32 with the bias's own strides (a padded bias
+ *          gives an equally padded dbias; padding is not written), 16-byte
+ *          aligned.  The bias's kept indices must nest b > h > i without
+ *          overlap (stride_i >= L, stride_h >= L stride_i, stride_b >= Hq
+ *          stride_h, skipping broadcast indices), else SDPA_ERR_UNSUPPORTED.
+ *          Masked (i, j), and keys of tiles the mask skips, get 0.
+ *   T5:    dbias[k * Hq + h] = sum of dS[b, h, i, j] over every (b, i, j)
+ *          with bucket(j - i) = k: float32 [num_buckets, Hq] like the table,
+ *          16-byte aligned.
+ *   NONE:  SDPA_ERR_UNSUPPORTED.
+ * dq, dk, dv as sdpa_bwd.  Deterministic: every sum is taken in one fixed
+ * order, so repeated calls give identical bits.
+ * workspace: at least sdpa_bwd_bias_grad_workspace_size(shape, bias) bytes,
+ * 256-byte aligned, contents ignored on entry.  Except for a full-shape dense
+ * bias, it holds an fp32 copy of dS, B * Hq * L * ceil4(L) floats, that the
+ * gradient is reduced from.  dbias must not overlap any other argument.
+ */
+size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias);
+sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,
+                                 const void* v, const void* o, const void* dout,
+                                 const float* lse, const sdpa_bias_desc* bias,
+                                 const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                                 void* dv, float* dbias, int32_t deterministic, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /*
  * T5 bucket ids of n signed distances rel[i] = key_pos - query_pos, computed

@@ -199,6 +199,9 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
     """Probability matrix P (rows sum to 1 over visible keys) for one head."""
     q = _as64(q)
     k = _as64(k)
+    for name in ("bias", "t5_table"):
+        if name in mask_bias:
+            mask_bias[name] = _as64(mask_bias[name])
     S = head_scores(q, k, b, hq, scale=_scale_of(q.shape[-1], scale), **mask_bias)
     P, _ = _softmax_rows(S)
     return P

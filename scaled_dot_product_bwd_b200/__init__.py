@@ -14,6 +14,8 @@ from .binding import (  # noqa: F401
     SdpaError,
     load_library,
     sdpa_bwd,
+    sdpa_bwd_bias_grad,
+    sdpa_bwd_bias_grad_workspace_size,
     sdpa_bwd_noalloc,
     sdpa_bwd_workspace_size,
     sdpa_debug_wait_timeout,

@@ -27,7 +27,8 @@ BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 NOALLOC_MAX_ROWS = 1 << 20
 
 EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_noalloc",
-            "sdpa_bwd_workspace_size", "sdpa_t5_bucket", "sdpa_exp2_fma",
+            "sdpa_bwd_workspace_size", "sdpa_bwd_bias_grad",
+            "sdpa_bwd_bias_grad_workspace_size", "sdpa_t5_bucket", "sdpa_exp2_fma",
             "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
             "sdpa_status_string")
 
@@ -80,6 +81,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_bwd_noalloc.restype = i32
     lib.sdpa_bwd_workspace_size.argtypes = [sp, i32]
     lib.sdpa_bwd_workspace_size.restype = sz
+    lib.sdpa_bwd_bias_grad.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, vp,
+                                       i32, vp, sz, vp]
+    lib.sdpa_bwd_bias_grad.restype = i32
+    lib.sdpa_bwd_bias_grad_workspace_size.argtypes = [sp, bp]
+    lib.sdpa_bwd_bias_grad_workspace_size.restype = sz
     lib.sdpa_t5_bucket.argtypes = [vp, vp, i64, i32, i32, i32, vp]
     lib.sdpa_t5_bucket.restype = i32
     lib.sdpa_exp2_fma.argtypes = [vp, vp, i64, vp]
@@ -129,20 +135,29 @@ def make_mask(causal: bool, window_left: int, window_right: int) -> MaskSpec:
 
 
 def make_bias(bias: torch.Tensor | None, t5_table: torch.Tensor | None, num_buckets: int,
-              max_distance: int, bidirectional: bool) -> BiasDesc:
+              max_distance: int, bidirectional: bool, dims: tuple | None = None) -> BiasDesc:
+    """Bias descriptor; ``dims`` = (B, Hq, L) of the attention checks the shapes."""
     if bias is not None and t5_table is not None:
         raise ValueError("give either a dense bias or a T5 table, not both")
     if bias is not None:
         if bias.dtype != torch.float32 or bias.dim() != 4 or bias.stride(-1) != 1:
             raise ValueError("dense bias must be float32 [B|1, H|1, L, L] with j contiguous")
+        if dims is not None:
+            B, Hq, L = dims
+            if (bias.shape[0] not in (1, B) or bias.shape[1] not in (1, Hq)
+                    or tuple(bias.shape[2:]) != (L, L)):
+                raise ValueError(f"dense bias shape {tuple(bias.shape)} is not "
+                                 f"[{B}|1, {Hq}|1, {L}, {L}]")
         sb = bias.stride(0) if bias.shape[0] > 1 else 0
         sh = bias.stride(1) if bias.shape[1] > 1 else 0
         return BiasDesc(BIAS_DENSE, bias.data_ptr(), sb, sh, bias.stride(2), 0, 0, 0)
     if t5_table is not None:
         if t5_table.dtype != torch.float32 or not t5_table.is_contiguous():
             raise ValueError("T5 table must be contiguous float32 [num_buckets, Hq]")
-        if t5_table.shape[0] != num_buckets:
-            raise ValueError("T5 table rows must equal num_buckets")
+        if t5_table.dim() != 2 or t5_table.shape[0] != num_buckets:
+            raise ValueError("T5 table must be [num_buckets, Hq]")
+        if dims is not None and t5_table.shape[1] != dims[1]:
+            raise ValueError("T5 table columns must equal the query heads")
         return BiasDesc(BIAS_T5, t5_table.data_ptr(), 0, 0, 0, int(num_buckets),
                         int(max_distance), 1 if bidirectional else 0)
     return BiasDesc(BIAS_NONE, None, 0, 0, 0, 0, 0, 0)
@@ -172,7 +187,8 @@ def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=Non
     if lse.shape != (B, Hq, L) or not lse.is_contiguous() or lse.dtype != torch.float32:
         raise ValueError("lse must be contiguous float32 [B, Hq, L]")
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (B, Hq, L))
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bd),
                       ctypes.byref(m), sc, _ptr(out), _ptr(lse), _stream(q))
@@ -212,7 +228,8 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
     if workspace is None:
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (q.shape[0], q.shape[2], q.shape[1]))
     m = make_mask(causal, window_left, window_right)
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
             ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk), _ptr(dv),
@@ -240,13 +257,67 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
                       (dv, k, "dv")):
         _same_layout(t, ref, n)
     sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
-    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (q.shape[0], q.shape[2], q.shape[1]))
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_bwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
                               _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq),
                               _ptr(dk), _ptr(dv), 1, _stream(q))
     _check(st, "sdpa_bwd_noalloc")
     return dq, dk, dv
+
+
+def sdpa_bwd_bias_grad_workspace_size(q, k, *, bias=None, t5_table=None, t5_num_buckets=32,
+                                      t5_max_distance=128, t5_bidirectional=True) -> int:
+    lib = load_library()
+    shape = make_shape(q, k)
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (q.shape[0], q.shape[2], q.shape[1]))
+    return int(lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(shape), ctypes.byref(bd)))
+
+
+def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
+                       bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
+                       t5_bidirectional=True, scale=None, dq=None, dk=None, dv=None, dbias=None,
+                       workspace=None):
+    """dQ, dK, dV and the bias gradient (see sdpa_bwd_bias_grad in include/sdpa.h).
+
+    The bias gradient has the dense bias's shape and strides, or the T5
+    table's [num_buckets, Hq] shape.
+    """
+    lib = load_library()
+    shape = make_shape(q, k)
+    _same_layout(v, k, "v")
+    _same_layout(o, q, "o")
+    _same_layout(do, q, "do")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _same_layout(dq, q, "dq")
+    _same_layout(dk, k, "dk")
+    _same_layout(dv, k, "dv")
+    bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (q.shape[0], q.shape[2], q.shape[1]))
+    ref = bias if bias is not None else t5_table
+    if ref is None:
+        raise ValueError("a bias gradient needs a dense bias or a T5 table")
+    if dbias is None:
+        dbias = torch.empty_strided(ref.shape, ref.stride(), device=q.device,
+                                    dtype=torch.float32)
+    if (dbias.shape != ref.shape or dbias.stride() != ref.stride()
+            or dbias.dtype != torch.float32):
+        raise ValueError("dbias must be float32 with the shape and strides of the bias")
+    need = int(lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(shape), ctypes.byref(bd)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_bwd_bias_grad(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                _ptr(do), _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc,
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbias), 1, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(q))
+    _check(st, "sdpa_bwd_bias_grad")
+    return dq, dk, dv, dbias
 
 
 def sdpa_t5_bucket(rel: torch.Tensor, num_buckets=32, max_distance=128, bidirectional=True):

@@ -68,6 +68,10 @@ struct AttnParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  // optional fp32 dS (the gradient of the logits, = of an additive bias),
+  // element strides sd_b, sd_h, sd_i (multiples of 4), j contiguous
+  float* ds_out;
+  int64_t sd_b, sd_h, sd_i;
   // bias
   int bias_kind;
   const float* bias;           // dense

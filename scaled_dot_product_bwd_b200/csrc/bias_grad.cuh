@@ -1,0 +1,203 @@
+// Bias gradients from the fp32 dS the dQ kernel stores (bwd_dq_kernel with
+// DS_OUT): the scores are linear in an additive bias, so a dense bias's
+// gradient is dS summed over each index the bias is broadcast along, and a
+// T5 table entry's gradient is dS summed over every (b, i, j) whose distance
+// j - i falls in its bucket (catie-aq/flashT5 README, "Full attention
+// biases" and "T5-like relative position encoding biases": a learnable
+// bias needs these to train).
+//
+// Every kernel here is bandwidth-bound and deterministic: each output is a
+// sum taken in one fixed order (fixed chunking of the reduced index, chunks
+// added in ascending order, a fixed shared-memory tree), independent of
+// timing, so repeated calls give identical bits.
+#pragma once
+
+#include "attn_common.cuh"
+
+namespace sdpa {
+
+// Blocks the reduction grids aim for (8 per SM on a 148-SM part); a constant,
+// not the device's SM count, so the chunking -- and with it the rounding of
+// every sum -- is the same on every device.
+constexpr int64_t kReduceTargetBlocks = 1184;
+
+// ---------------------------------------------------------------------
+// dS entries the backward never visits: for query row i, the key tiles
+// outside [nlo, nhi) of i's query tile (key_tile_range), which hold no key
+// visible from any row of the tile.  The dQ kernel writes every column of
+// the tiles inside the band (masked keys as 0); this fills the rest with 0.
+__device__ __forceinline__ void zero_span(float* row, int j0, int j1) {
+  // j0 is 0 or a multiple of the tile width, so row + j0 is 16-byte aligned
+  for (int j = j0 + 4 * static_cast<int>(threadIdx.x); j < j1; j += 4 * static_cast<int>(blockDim.x)) {
+    if (j + 4 <= j1) {
+      *reinterpret_cast<float4*>(row + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      for (int t = j; t < j1; ++t) row[t] = 0.f;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) ds_zero_outside_band_kernel(const AttnParams p) {
+  const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.L;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int i = static_cast<int>(r % p.L);
+    const int64_t bh = r / p.L;
+    const int hq = static_cast<int>(bh % p.Hq);
+    const int b = static_cast<int>(bh / p.Hq);
+    int nlo, nhi;
+    key_tile_range(p, (i / kTile) * kTile, kTile, nlo, nhi);
+    float* row = p.ds_out + static_cast<int64_t>(b) * p.sd_b + static_cast<int64_t>(hq) * p.sd_h +
+                 static_cast<int64_t>(i) * p.sd_i;
+    // [0, nlo * 128) and [nhi * 128, L); with an empty band the two cover the row
+    zero_span(row, 0, min(nlo * kTile, p.L));
+    zero_span(row, min(nhi * kTile, p.L), p.L);
+  }
+}
+
+// ---------------------------------------------------------------------
+// Dense bias broadcast along some of (b, h, i): out[b', h', i', j] = sum of
+// dS[b, h, i, j] over the broadcast indices.  Output rows o enumerate the
+// kept indices (extents eb, eh, ei: the full extent where kept, else 1);
+// the reduced index t enumerates the broadcast ones (extents rb, rh, ri).
+struct DenseReduce {
+  const float* ds;               // [B, Hq, L, lp] fp32, row stride lp
+  int64_t ds_b, ds_h, ds_i;
+  float* out;                    // the bias gradient, element strides o_b, o_h, o_i
+  int64_t o_b, o_h, o_i;
+  int L;
+  int eb, eh, ei;                // kept extents
+  int rb, rh, ri;                // reduced extents
+  int64_t n_out, n_red;          // eb*eh*ei, rb*rh*ri
+  int jblocks;                   // ceil(L / 256)
+  int chunks;                    // pieces of the reduced index (grid y)
+  int64_t rchunk;                // reduced indices per piece
+  float* partial;                // [chunks, n_out, lp] when chunks > 1
+  int64_t lp;
+};
+
+__device__ __forceinline__ void dense_out_index(const DenseReduce& a, int64_t o, int& b, int& h,
+                                                int& i) {
+  i = static_cast<int>(o % a.ei);
+  const int64_t r = o / a.ei;
+  h = static_cast<int>(r % a.eh);
+  b = static_cast<int>(r / a.eh);
+}
+
+__global__ void __launch_bounds__(256) dense_bias_reduce_kernel(const DenseReduce a) {
+  const int z = blockIdx.y;
+  const int64_t t0 = static_cast<int64_t>(z) * a.rchunk;
+  const int64_t t1 = min(a.n_red, t0 + a.rchunk);
+  const int64_t work = a.n_out * a.jblocks;
+  for (int64_t w = blockIdx.x; w < work; w += gridDim.x) {
+    const int64_t o = w / a.jblocks;
+    const int j = static_cast<int>(w % a.jblocks) * 256 + static_cast<int>(threadIdx.x);
+    if (j >= a.L) continue;
+    int ob, oh, oi;
+    dense_out_index(a, o, ob, oh, oi);
+    float acc = 0.f;
+    // reduced index t = (tb, th, ti), ti fastest; exactly one of o's and t's
+    // coordinate is non-zero along each axis
+    int ti = static_cast<int>(t0 % a.ri);
+    int th = static_cast<int>((t0 / a.ri) % a.rh);
+    int tb = static_cast<int>(t0 / (static_cast<int64_t>(a.ri) * a.rh));
+    for (int64_t t = t0; t < t1; ++t) {
+      acc += a.ds[static_cast<int64_t>(ob + tb) * a.ds_b + static_cast<int64_t>(oh + th) * a.ds_h +
+                  static_cast<int64_t>(oi + ti) * a.ds_i + j];
+      if (++ti == a.ri) {
+        ti = 0;
+        if (++th == a.rh) {
+          th = 0;
+          ++tb;
+        }
+      }
+    }
+    if (a.chunks == 1)
+      a.out[ob * a.o_b + oh * a.o_h + oi * a.o_i + j] = acc;
+    else
+      a.partial[(static_cast<int64_t>(z) * a.n_out + o) * a.lp + j] = acc;
+  }
+}
+
+// Second stage when the reduced index was split: add the pieces in order.
+__global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseReduce a) {
+  const int64_t work = a.n_out * a.jblocks;
+  for (int64_t w = blockIdx.x; w < work; w += gridDim.x) {
+    const int64_t o = w / a.jblocks;
+    const int j = static_cast<int>(w % a.jblocks) * 256 + static_cast<int>(threadIdx.x);
+    if (j >= a.L) continue;
+    float acc = 0.f;
+    for (int z = 0; z < a.chunks; ++z) acc += a.partial[(static_cast<int64_t>(z) * a.n_out + o) * a.lp + j];
+    int ob, oh, oi;
+    dense_out_index(a, o, ob, oh, oi);
+    a.out[ob * a.o_b + oh * a.o_h + oi * a.o_i + j] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------
+// T5 table gradient.  The bucket depends on j - i alone, so first sum dS
+// along each diagonal r = j - i (r in [-(L-1), L-1]), then add up the
+// diagonals of each bucket.  Every bucket covers one contiguous range of r
+// (the bucket is monotone in |r| on each side of 0, and the two sides use
+// disjoint ids when bidirectional), given to the second kernel as [lo, hi].
+struct T5Reduce {
+  const float* ds;               // [B, Hq, L, lp] fp32
+  int64_t ds_b, ds_h, ds_i;
+  int B, Hq, L;
+  int chunks;                    // pieces of the (b, i) range (grid z)
+  int64_t uchunk;                // (b, i) pairs per piece
+  float* partial;                // [chunks, Hq, 2L - 1]
+  float* out;                    // table gradient [num_buckets, Hq]
+  int num_buckets;
+};
+
+struct T5Ranges {
+  int lo[128];                   // first r of bucket k (r = j - i)
+  int hi[128];                   // last r of bucket k; hi < lo: bucket unused
+};
+
+// partial[z, h, r + L - 1] = sum of dS[b, h, i, i + r] over the (b, i) of piece z
+__global__ void __launch_bounds__(128) t5_diag_kernel(const T5Reduce a) {
+  const int nd = 2 * a.L - 1;
+  const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
+  if (dr >= nd) return;
+  const int r = dr - (a.L - 1);
+  const int h = blockIdx.y;
+  const int z = blockIdx.z;
+  const int64_t u0 = static_cast<int64_t>(z) * a.uchunk;
+  const int64_t u1 = min(static_cast<int64_t>(a.B) * a.L, u0 + a.uchunk);
+  int b = static_cast<int>(u0 / a.L);
+  int i = static_cast<int>(u0 % a.L);
+  float acc = 0.f;
+  for (int64_t u = u0; u < u1; ++u) {
+    const int j = i + r;
+    if (j >= 0 && j < a.L)
+      acc += a.ds[static_cast<int64_t>(b) * a.ds_b + static_cast<int64_t>(h) * a.ds_h +
+                  static_cast<int64_t>(i) * a.ds_i + j];
+    if (++i == a.L) {
+      i = 0;
+      ++b;
+    }
+  }
+  a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + dr] = acc;
+}
+
+// out[k, h] = sum over r in bucket k's range, over the pieces, of the
+// diagonal sums: one block per (k, h), a fixed tree over its 256 threads.
+__global__ void __launch_bounds__(256) t5_bucket_sum_kernel(const T5Reduce a, const T5Ranges rg) {
+  __shared__ float red[256];
+  const int k = blockIdx.x;
+  const int h = blockIdx.y;
+  const int nd = 2 * a.L - 1;
+  float acc = 0.f;
+  for (int r = rg.lo[k] + static_cast<int>(threadIdx.x); r <= rg.hi[k]; r += 256)
+    for (int z = 0; z < a.chunks; ++z)
+      acc += a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + (r + a.L - 1)];
+  red[threadIdx.x] = acc;
+  for (int w = 128; w > 0; w >>= 1) {
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
+  }
+  if (threadIdx.x == 0) a.out[static_cast<int64_t>(k) * a.Hq + h] = red[0];
+}
+
+}  // namespace sdpa

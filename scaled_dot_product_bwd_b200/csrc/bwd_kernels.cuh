@@ -556,7 +556,8 @@ struct DqLayout {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-template <int D, int BIAS>
+// DS_OUT: also store dS in fp32 through p.ds_out (the bias gradient path).
+template <int D, int BIAS, bool DS_OUT = false>
 __global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -955,6 +956,10 @@ __global__ void __launch_bounds__(352, 1)
             const float d0 = __uint_as_float(pr[cc + e]) * (__uint_as_float(dr[e]) - dd);
             const float d1 = __uint_as_float(pr[cc + e + 1]) * (__uint_as_float(dr[e + 1]) - dd);
             pk[(cc + e) >> 1] = pack_bf16x2(d0, d1);
+            if constexpr (DS_OUT) {  // P is spent: keep the fp32 dS in its place
+              pr[cc + e] = __float_as_uint(d0);
+              pr[cc + e + 1] = __float_as_uint(d1);
+            }
           }
         }
         // dS over the first 32 of this warpgroup's columns of its S buffer
@@ -963,6 +968,25 @@ __global__ void __launch_bounds__(352, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(ds_full(c & 1));
+        if constexpr (DS_OUT) {
+          // fp32 dS of this row's 64 keys while the dQ MMA runs; masked keys
+          // have P = 0 and so dS = 0
+          if (i < p.L) {
+            float* dst = p.ds_out + static_cast<int64_t>(b) * p.sd_b +
+                         static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(i) * p.sd_i + n0;
+            if (n0 + kBlk <= p.L) {
+#pragma unroll
+              for (int e = 0; e < kBlk; e += 4)
+                *reinterpret_cast<float4*>(dst + e) =
+                    make_float4(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1]),
+                                __uint_as_float(pr[e + 2]), __uint_as_float(pr[e + 3]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < kBlk; ++e)
+                if (n0 + e < p.L) dst[e] = __uint_as_float(pr[e]);
+            }
+          }
+        }
       }
       // ----------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -----------
       // Items without a visible key (none exist for the masks accepted at the
@@ -1028,6 +1052,9 @@ cudaError_t launch_bwd_t(const AttnParams& p, const BwdMaps& m, uint32_t phases,
   if (phases & kPhaseDq) {
     using Lay = DqLayout<D, BIAS>;
     auto kern = bwd_dq_kernel<D, BIAS>;
+    if constexpr (BIAS != kBiasNone) {
+      if (p.ds_out) kern = bwd_dq_kernel<D, BIAS, true>;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;

@@ -8,9 +8,11 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "sdpa.h"
 #include "attn_common.cuh"
+#include "bias_grad.cuh"
 #include "bwd_kernels.cuh"
 #include "fwd_kernel.cuh"
 
@@ -151,6 +153,9 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
       if (bias->stride_b < 0 || bias->stride_h < 0 || bias->stride_i < 0) return SDPA_ERR_INVALID_ARG;
       if (bias->stride_b % 4 != 0 || bias->stride_h % 4 != 0 || bias->stride_i % 4 != 0)
         return SDPA_ERR_INVALID_ARG;
+      // a bias broadcast over query rows has no 2-D tile layout for the
+      // tensor-memory copies that stage bias blocks
+      if (bias->stride_i == 0) return SDPA_ERR_UNSUPPORTED;
       p.bias_kind = kBiasDense;
       p.bias = bias->ptr;
       p.sb_b = bias->stride_b;
@@ -169,6 +174,123 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
     }
   }
   return SDPA_OK;
+}
+
+// Tensor maps for the backward's three launches, then the launches selected
+// by `phases`; p carries every pointer and size.
+sdpa_status_t run_bwd(uint32_t phases, const AttnParams& p, const sdpa_shape& s, const void* q,
+                      const void* k, const void* v, const void* dout, cudaStream_t stream) {
+  BwdMaps maps;
+  bool ok = true;
+  for (int rows : {kTile, kBlk}) {
+    CUtensorMap* mq = rows == kTile ? &maps.q128 : &maps.q64;
+    CUtensorMap* mdo = rows == kTile ? &maps.dout128 : &maps.dout64;
+    CUtensorMap* mk = rows == kTile ? &maps.k128 : &maps.k64;
+    CUtensorMap* mv = rows == kTile ? &maps.v128 : &maps.v64;
+    ok = ok && make_bshd_map(mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
+         make_bshd_map(mdo, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
+         make_bshd_map(mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows) &&
+         make_bshd_map(mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows);
+  }
+  std::memset(&maps.bias, 0, sizeof(maps.bias));  // read only by the dense-bias kernels
+  if (ok && p.bias_kind == kBiasDense) ok = make_bias_map(&maps.bias, p);
+  if (!ok) return SDPA_ERR_CUDA;
+  cudaError_t e = launch_bwd(p, maps, static_cast<int>(s.d), phases, stream);
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+// ----- bias gradients: workspace plan (sdpa_bwd_bias_grad) -----
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct BiasGradPlan {
+  size_t d_bytes = 0;     // D vector
+  bool ds_ws = false;     // dS staged in the workspace (else written into dbias)
+  int64_t lp = 0;         // row stride of the staged dS
+  size_t ds_bytes = 0;
+  int chunks = 1;         // pieces of the reduced index
+  int64_t per_chunk = 0;  // reduced indices per piece
+  size_t part_bytes = 0;  // partial sums of the pieces
+  size_t total = 0;
+};
+
+// Splits n_red reduced indices into pieces so that `blocks` output blocks per
+// piece give about kReduceTargetBlocks blocks in all (at most 65535 pieces).
+void split_reduction(int64_t n_red, int64_t blocks, int& chunks, int64_t& per_chunk) {
+  int64_t c = (kReduceTargetBlocks + blocks - 1) / blocks;
+  c = c < 1 ? 1 : c;
+  c = c > n_red ? n_red : c;
+  c = c > 65535 ? 65535 : c;
+  per_chunk = (n_red + c - 1) / c;
+  chunks = static_cast<int>((n_red + per_chunk - 1) / per_chunk);
+}
+
+sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, BiasGradPlan& pl) {
+  if (!s || !bias || s->B < 1 || s->L < 1 || s->Hq < 1) return SDPA_ERR_INVALID_ARG;
+  if (s->L >= (1ll << 30) || s->B > 65535 || s->Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  const int64_t B = s->B, Hq = s->Hq, L = s->L;
+  pl = BiasGradPlan{};
+  pl.d_bytes = round256(static_cast<size_t>(B * Hq * L) * sizeof(float));
+  pl.lp = (L + 3) / 4 * 4;
+  // B * Hq * L * lp floats must stay far from 2^63 bytes
+  const double ds_elems = static_cast<double>(B) * Hq * L * pl.lp;
+  if (bias->kind == SDPA_BIAS_DENSE) {
+    // the kept indices must nest b > h > i without overlap, so that each
+    // gradient entry has exactly one address
+    int64_t span = L;
+    const int64_t st[3] = {bias->stride_i, bias->stride_h, bias->stride_b};
+    const int64_t ex[3] = {L, Hq, B};
+    for (int a = 0; a < 3; ++a) {
+      if (st[a] < 0) return SDPA_ERR_INVALID_ARG;
+      if (st[a] == 0) continue;
+      if (st[a] < span) return SDPA_ERR_UNSUPPORTED;
+      span = st[a] * ex[a];
+    }
+    if (bias->stride_i == 0) return SDPA_ERR_UNSUPPORTED;
+    pl.ds_ws = bias->stride_b == 0 || bias->stride_h == 0;
+    if (pl.ds_ws) {
+      if (ds_elems > 1e17) return SDPA_ERR_UNSUPPORTED;
+      pl.ds_bytes = round256(static_cast<size_t>(B * Hq * L * pl.lp) * sizeof(float));
+      const int64_t n_out = (bias->stride_b ? B : 1) * (bias->stride_h ? Hq : 1) * L;
+      const int64_t n_red = (bias->stride_b ? 1 : B) * (bias->stride_h ? 1 : Hq);
+      split_reduction(n_red, n_out * ((L + 255) / 256), pl.chunks, pl.per_chunk);
+      if (pl.chunks > 1)
+        pl.part_bytes = round256(static_cast<size_t>(pl.chunks * n_out * pl.lp) * sizeof(float));
+    }
+  } else if (bias->kind == SDPA_BIAS_T5) {
+    if (ds_elems > 1e17) return SDPA_ERR_UNSUPPORTED;
+    pl.ds_ws = true;
+    pl.ds_bytes = round256(static_cast<size_t>(B * Hq * L * pl.lp) * sizeof(float));
+    split_reduction(B * L, ((2 * L - 1 + 127) / 128) * Hq, pl.chunks, pl.per_chunk);
+    pl.part_bytes = round256(static_cast<size_t>(pl.chunks * Hq * (2 * L - 1)) * sizeof(float));
+  } else {
+    return SDPA_ERR_UNSUPPORTED;  // no bias: nothing to differentiate
+  }
+  pl.total = pl.d_bytes + pl.ds_bytes + pl.part_bytes;
+  return SDPA_OK;
+}
+
+// The contiguous range [lo, hi] of distances r = j - i in [-(L-1), L-1]
+// that fall in each T5 bucket (hi < lo when none does).  False if some
+// bucket's distances are not contiguous, which the bucket function rules out.
+bool t5_ranges(const T5Spec& t, int L, int num_buckets, T5Ranges& rg) {
+  for (int k = 0; k < 128; ++k) {
+    rg.lo[k] = 0;
+    rg.hi[k] = -1;
+  }
+  std::vector<char> seen(num_buckets, 0);
+  int prev = -1;
+  for (int r = -(L - 1); r <= L - 1; ++r) {
+    const int k = t5_bucket(r, t);
+    if (k < 0 || k >= num_buckets) return false;
+    if (k != prev) {
+      if (seen[k]) return false;
+      seen[k] = 1;
+      rg.lo[k] = r;
+      prev = k;
+    }
+    rg.hi[k] = r;
+  }
+  return true;
 }
 
 template <int D, int BIAS>
@@ -302,25 +424,7 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  const sdpa_shape& s = *shape;
-  BwdMaps maps;
-  bool ok = true;
-  for (int rows : {kTile, kBlk}) {
-    CUtensorMap* mq = rows == kTile ? &maps.q128 : &maps.q64;
-    CUtensorMap* mdo = rows == kTile ? &maps.dout128 : &maps.dout64;
-    CUtensorMap* mk = rows == kTile ? &maps.k128 : &maps.k64;
-    CUtensorMap* mv = rows == kTile ? &maps.v128 : &maps.v64;
-    ok = ok && make_bshd_map(mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
-         make_bshd_map(mdo, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
-         make_bshd_map(mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows) &&
-         make_bshd_map(mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows);
-  }
-  std::memset(&maps.bias, 0, sizeof(maps.bias));  // read only by the dense-bias kernels
-  if (ok && p.bias_kind == kBiasDense) ok = make_bias_map(&maps.bias, p);
-  if (!ok) return SDPA_ERR_CUDA;
-  cudaError_t e =
-      launch_bwd(p, maps, static_cast<int>(s.d), phases, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  return run_bwd(phases, p, *shape, q, k, v, dout, static_cast<cudaStream_t>(stream));
 }
 
 sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
@@ -330,6 +434,120 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, co
                        size_t workspace_bytes, void* stream) {
   return sdpa_bwd_phases(SDPA_BWD_ALL, shape, q, k, v, o, dout, lse, bias, mask, scale, dq, dk,
                          dv, deterministic, workspace, workspace_bytes, stream);
+}
+
+size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias) {
+  BiasGradPlan pl;
+  return plan_bias_grad(shape, bias, pl) == SDPA_OK ? pl.total : 0;
+}
+
+sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,
+                                 const void* v, const void* o, const void* dout,
+                                 const float* lse, const sdpa_bias_desc* bias,
+                                 const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                                 void* dv, float* dbias, int32_t deterministic, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  AttnParams p;
+  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  if (st != SDPA_OK) return st;
+  if (p.bias_kind == kBiasNone) return SDPA_ERR_UNSUPPORTED;
+  if (deterministic != 1) return SDPA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv, dbias};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return SDPA_ERR_INVALID_ARG;
+  BiasGradPlan pl;
+  st = plan_bias_grad(shape, bias, pl);
+  if (st != SDPA_OK) return st;
+  T5Ranges rg;
+  if (p.bias_kind == kBiasT5 && !t5_ranges(p.t5, p.L, bias->num_buckets, rg))
+    return SDPA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < pl.total)
+    return SDPA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.o = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(o));
+  p.lse = const_cast<float*>(lse);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dvec = reinterpret_cast<float*>(ws);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  if (pl.ds_ws) {
+    p.ds_out = reinterpret_cast<float*>(ws + pl.d_bytes);
+    p.sd_i = pl.lp;
+    p.sd_h = pl.lp * p.L;
+    p.sd_b = p.sd_h * p.Hq;
+  } else {
+    p.ds_out = dbias;
+    p.sd_b = p.sb_b;
+    p.sd_h = p.sb_h;
+    p.sd_i = p.sb_i;
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int sms = sm_count();
+  if (sms <= 0) return SDPA_ERR_CUDA;
+  if (p.causal || p.wl >= 0 || p.wr >= 0) {
+    const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.L;
+    const int64_t grid = rows < 8ll * sms ? rows : 8ll * sms;
+    ds_zero_outside_band_kernel<<<static_cast<unsigned>(grid), 256, 0, cs>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+  }
+  st = run_bwd(SDPA_BWD_ALL, p, *shape, q, k, v, dout, cs);
+  if (st != SDPA_OK || !pl.ds_ws) return st;
+  float* part = reinterpret_cast<float*>(ws + pl.d_bytes + pl.ds_bytes);
+  if (p.bias_kind == kBiasDense) {
+    DenseReduce a;
+    a.ds = p.ds_out;
+    a.ds_b = p.sd_b;
+    a.ds_h = p.sd_h;
+    a.ds_i = p.sd_i;
+    a.out = dbias;
+    a.o_b = p.sb_b;
+    a.o_h = p.sb_h;
+    a.o_i = p.sb_i;
+    a.L = p.L;
+    a.eb = p.sb_b ? p.B : 1;
+    a.eh = p.sb_h ? p.Hq : 1;
+    a.ei = p.L;
+    a.rb = p.sb_b ? 1 : p.B;
+    a.rh = p.sb_h ? 1 : p.Hq;
+    a.ri = 1;
+    a.n_out = static_cast<int64_t>(a.eb) * a.eh * a.ei;
+    a.n_red = static_cast<int64_t>(a.rb) * a.rh * a.ri;
+    a.jblocks = (p.L + 255) / 256;
+    a.chunks = pl.chunks;
+    a.rchunk = pl.per_chunk;
+    a.partial = part;
+    a.lp = pl.lp;
+    const int64_t work = a.n_out * a.jblocks;
+    const int64_t g1 = work < kReduceTargetBlocks ? work : kReduceTargetBlocks;
+    dense_bias_reduce_kernel<<<dim3(static_cast<unsigned>(g1), a.chunks), 256, 0, cs>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    if (a.chunks > 1) {
+      dense_bias_combine_kernel<<<static_cast<unsigned>(g1), 256, 0, cs>>>(a);
+      if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    }
+  } else {
+    T5Reduce a;
+    a.ds = p.ds_out;
+    a.ds_b = p.sd_b;
+    a.ds_h = p.sd_h;
+    a.ds_i = p.sd_i;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.L = p.L;
+    a.chunks = pl.chunks;
+    a.uchunk = pl.per_chunk;
+    a.partial = part;
+    a.out = dbias;
+    a.num_buckets = bias->num_buckets;
+    const unsigned rblocks = static_cast<unsigned>((2 * p.L - 1 + 127) / 128);
+    t5_diag_kernel<<<dim3(rblocks, p.Hq, a.chunks), 128, 0, cs>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+  }
+  return SDPA_OK;
 }
 
 // ---------------------------------------------------------------------

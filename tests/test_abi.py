@@ -110,6 +110,68 @@ def test_bwd_rejects_bad_args(lib):
     assert lib.sdpa_bwd_workspace_size(None, 1) == 0
 
 
+def _dense(sb, sh, si, ptr=0x10000):
+    return binding.BiasDesc(1, ptr, sb, sh, si, 0, 0, 0)
+
+
+def test_bias_grad_workspace_size(lib):
+    B, L, Hq = 2, 128, 4
+    s = _shape(B=B, sq_b=128 * 4 * 64, skv_b=128 * 2 * 64)
+    ws = lambda bias: lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(s), ctypes.byref(bias))
+    d_bytes = lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1)
+    ds_bytes = B * Hq * L * L * 4
+    # full-shape dense bias: dS goes straight into dbias, only D is staged
+    assert ws(_dense(Hq * L * L, L * L, L)) == d_bytes
+    # a padded full-shape bias needs no more
+    assert ws(_dense(Hq * L * (L + 4), L * (L + 4), L + 4)) == d_bytes
+    # broadcast over heads, over batch, over both: dS is staged and reduced
+    for b in (_dense(L * L, 0, L), _dense(0, L * L, L), _dense(0, 0, L)):
+        n = ws(b)
+        assert n >= d_bytes + ds_bytes and n % 256 == 0
+    t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
+    n = ws(t5)
+    assert n >= d_bytes + ds_bytes + Hq * (2 * L - 1) * 4 and n % 256 == 0
+    assert ws(binding.BiasDesc(0, None, 0, 0, 0, 0, 0, 0)) == 0       # nothing to differentiate
+    assert ws(_dense(L * L, L * L, L)) == 0                          # heads overlap batches
+    assert ws(_dense(Hq * L * L, L * L, 0)) == 0                      # one row for all queries
+    assert lib.sdpa_bwd_bias_grad_workspace_size(None, ctypes.byref(t5)) == 0
+
+
+def test_bias_grad_rejects_bad_args(lib):
+    B, L, Hq = 2, 128, 4
+    s = _shape(B=B)
+    m = binding.MaskSpec(1, -1, -1)
+    full = _dense(Hq * L * L, L * L, L)
+    need = lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(s), ctypes.byref(full))
+
+    def call(bias=full, dbias=FAKE, det=1, wsb=need, wsp=FAKE):
+        return lib.sdpa_bwd_bias_grad(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                      ctypes.byref(bias) if bias is not None else None,
+                                      ctypes.byref(m), 0.125, FAKE, FAKE, FAKE, dbias, det, wsp,
+                                      wsb, None)
+    assert call(bias=None) == 2                                      # no bias
+    assert call(bias=binding.BiasDesc(0, None, 0, 0, 0, 0, 0, 0)) == 2
+    assert call(bias=_dense(Hq * L * L, L * L, 0)) == 2              # row-broadcast bias
+    assert call(bias=_dense(L * L, L * L, L)) == 2                   # overlapping layout
+    assert call(dbias=ctypes.c_void_p(0)) == 1
+    assert call(dbias=ctypes.c_void_p(0x10008)) == 1                 # not 16-byte aligned
+    assert call(det=0) == 2
+    assert call(wsb=need - 1) == 3
+    assert call(wsp=ctypes.c_void_p(0x10040)) == 3                   # not 256-byte aligned
+
+
+def test_binding_checks_bias_shapes():
+    import torch
+    ok = torch.zeros(1, 4, 16, 16)
+    binding.make_bias(ok, None, 32, 128, True, (2, 4, 16))
+    for bad in (torch.zeros(2, 4, 1, 16), torch.zeros(3, 4, 16, 16), torch.zeros(1, 2, 16, 16),
+                torch.zeros(1, 4, 16, 8)):
+        with pytest.raises(ValueError):
+            binding.make_bias(bad, None, 32, 128, True, (2, 4, 16))
+    with pytest.raises(ValueError):
+        binding.make_bias(None, torch.zeros(32, 3), 32, 128, True, (2, 4, 16))
+
+
 def test_t5_bucket_rejects_bad_args(lib):
     assert lib.sdpa_t5_bucket(FAKE, FAKE, -1, 32, 128, 1, None) == 1
     assert lib.sdpa_t5_bucket(None, None, 5, 32, 128, 1, None) == 1
