@@ -12,6 +12,10 @@ rank 0 prints the whole-job rate: all ranks' FLOPs / the slowest rank's time.
 
 --impl reference times the float64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload (one KV head group of one batch per step).
+
+--bias-grad (a workload with a bias) times the step with the bias gradient
+(sdpa_bwd_bias_grad) beside the plain step on the same inputs, and reports
+the gradient's extra cost against its extra HBM traffic.
 """
 from __future__ import annotations
 
@@ -416,6 +420,114 @@ def run_gpu(args, c):
     return 0
 
 
+def bias_grad_extra_bytes(c):
+    """HBM bytes the bias gradient adds to the backward: the fp32 dS written
+    once, plus -- when it is staged (T5 table, broadcast dense bias) -- read
+    back once by the reduction and the gradient written."""
+    B, H, L = c["B"], c["Hq"], c["L"]
+    ds = B * H * L * L * 4
+    if c["bias"] == "t5":
+        return 2 * ds + 32 * H * 4
+    return ds                      # a full-shape dense bias: dS goes straight out
+
+
+def run_bias_grad(args, c):
+    import torch
+
+    from scaled_dot_product_bwd_b200 import (load_library, sdpa_bwd, sdpa_bwd_bias_grad,
+                                             sdpa_bwd_bias_grad_workspace_size,
+                                             sdpa_bwd_workspace_size, sdpa_fwd,
+                                             sdpa_read_device_status)
+    if c["bias"] == "none":
+        raise SystemExit("--bias-grad needs a workload with a bias")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    load_library()
+    inp = make_case(c, seed=0)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    bias = inp.bias.to(dev) if inp.bias is not None else None
+    table = inp.t5_table.to(dev) if inp.t5_table is not None else None
+    kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"], bias=bias,
+              t5_table=table)
+    o = torch.empty_like(q)
+    lse = torch.empty(c["B"], c["Hq"], c["L"], device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ref = bias if bias is not None else table
+    dbias = torch.empty_strided(ref.shape, ref.stride(), device=dev, dtype=torch.float32)
+    ws = torch.empty(sdpa_bwd_workspace_size(q, k), device=dev, dtype=torch.uint8)
+    wsg = torch.empty(max(256, sdpa_bwd_bias_grad_workspace_size(q, k, bias=bias,
+                                                                 t5_table=table)),
+                      device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(grad, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sdpa_fwd(q, k, v, out=o, lse=lse, **kw)
+        if ev is not None:
+            ev[1].record(stream)
+        if grad:
+            sdpa_bwd_bias_grad(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, dbias=dbias,
+                               workspace=wsg, **kw)
+        else:
+            sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+        if ev is not None:
+            ev[2].record(stream)
+
+    res = {}
+    for grad in (False, True):
+        for _ in range(args.warmup):
+            step(grad)
+        torch.cuda.synchronize(dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+               for _ in range(args.steps)]
+        sampler = ClockSampler(0) if grad else None
+        if sampler is not None:
+            time.sleep(0.1)
+        for s_i in range(args.steps):
+            step(grad, evs[s_i])
+        torch.cuda.synchronize(dev)
+        clocks = sampler.stop() if sampler is not None else None
+        res[grad] = dict(fwd=statistics.fmean(e[0].elapsed_time(e[1]) for e in evs),
+                         bwd=statistics.fmean(e[1].elapsed_time(e[2]) for e in evs),
+                         clocks=clocks)
+    status = sdpa_read_device_status()
+    fl = flop_counts(c)
+    step_flops = fl["fwd"] + fl["bwd"]
+    ms_step = res[True]["fwd"] + res[True]["bwd"]
+    extra_ms = res[True]["bwd"] - res[False]["bwd"]
+    extra = bias_grad_extra_bytes(c)
+    peaks = load_peaks()
+    ach = extra / (extra_ms * 1e-3) / 1e9 if extra_ms > 0 else None
+    line = {
+        "metric": METRIC + ", backward with the bias gradient",
+        "value": round(step_flops / (ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: {describe(c)}, with bias gradient",
+                   "global_batch": c["B"], "seq_len": c["L"], "parallelism": "replicas x1",
+                   "l2": "inputs larger than L2: no flush between steps",
+                   "flops_per_step": step_flops},
+        "kernel_ms": {"fwd": round(res[True]["fwd"], 4),
+                      "bwd_bias_grad": round(res[True]["bwd"], 4),
+                      "bwd_plain": round(res[False]["bwd"], 4)},
+        "bias_grad_extra_ms": round(extra_ms, 4),
+        "roofline": {"kernel": "bias-gradient extra (dS store + reduction)", "bound": "hbm",
+                     "achieved": None if ach is None else round(ach, 1),
+                     "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": None if ach is None else round(ach / peaks["hbm"], 4),
+                     "traffic": None, "bytes_per_step": extra,
+                     "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json)"
+                     if peaks["source"] == "measured" else "fallback 6.65 TB/s"},
+        "gpu_launches": None,
+        "clocks": res[True]["clocks"],
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -424,10 +536,13 @@ def main():
     ap.add_argument("--config", default="mistral4k", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bias-grad", action="store_true")
     args = ap.parse_args()
     c = CONFIGS[args.config]
     if args.impl == "reference":
         return run_reference(args, c)
+    if args.bias_grad:
+        return run_bias_grad(args, c)
     return run_gpu(args, c)
 
 

@@ -21,6 +21,9 @@ namespace sdpa {
 // every sum -- is the same on every device.
 constexpr int64_t kReduceTargetBlocks = 1184;
 
+// (b, i) rows per piece of the T5 diagonal sums.
+constexpr int64_t kT5RowsPerPiece = 128;
+
 // ---------------------------------------------------------------------
 // dS entries the backward never visits: for query row i, the key tiles
 // outside [nlo, nhi) of i's query tile (key_tile_range), which hold no key
@@ -138,7 +141,7 @@ __global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseRedu
 // along each diagonal r = j - i (r in [-(L-1), L-1]), then add up the
 // diagonals of each bucket.  Every bucket covers one contiguous range of r
 // (the bucket is monotone in |r| on each side of 0, and the two sides use
-// disjoint ids when bidirectional), given to the second kernel as [lo, hi].
+// disjoint ids when bidirectional), given to the last kernel as [lo, hi].
 struct T5Reduce {
   const float* ds;               // [B, Hq, L, lp] fp32
   int64_t ds_b, ds_h, ds_i;
@@ -155,7 +158,11 @@ struct T5Ranges {
   int hi[128];                   // last r of bucket k; hi < lo: bucket unused
 };
 
-// partial[z, h, r + L - 1] = sum of dS[b, h, i, i + r] over the (b, i) of piece z
+// partial[z, h, r + L - 1] = sum of dS[b, h, i, i + r] over the (b, i) of
+// piece z.  A thread walks only the rows that have a key at distance r, with
+// eight accumulators (the e-th of every eight consecutive rows goes to
+// accumulator e, an order fixed by the shape alone) so that eight loads are
+// in flight at a time.
 __global__ void __launch_bounds__(128) t5_diag_kernel(const T5Reduce a) {
   const int nd = 2 * a.L - 1;
   const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
@@ -163,35 +170,72 @@ __global__ void __launch_bounds__(128) t5_diag_kernel(const T5Reduce a) {
   const int r = dr - (a.L - 1);
   const int h = blockIdx.y;
   const int z = blockIdx.z;
+  const int row_lo = max(0, -r), row_hi = min(a.L, a.L - r);  // rows i with 0 <= i + r < L
   const int64_t u0 = static_cast<int64_t>(z) * a.uchunk;
   const int64_t u1 = min(static_cast<int64_t>(a.B) * a.L, u0 + a.uchunk);
-  int b = static_cast<int>(u0 / a.L);
-  int i = static_cast<int>(u0 % a.L);
-  float acc = 0.f;
-  for (int64_t u = u0; u < u1; ++u) {
-    const int j = i + r;
-    if (j >= 0 && j < a.L)
-      acc += a.ds[static_cast<int64_t>(b) * a.ds_b + static_cast<int64_t>(h) * a.ds_h +
-                  static_cast<int64_t>(i) * a.ds_i + j];
-    if (++i == a.L) {
-      i = 0;
-      ++b;
+  const int b_first = static_cast<int>(u0 / a.L);
+  const int b_last = static_cast<int>((u1 - 1) / a.L);
+  const int64_t step = a.ds_i + 1;  // (i, i + r) -> (i + 1, i + 1 + r)
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int b = b_first; b <= b_last; ++b) {
+    int ia = row_lo, ib = row_hi;
+    if (b == b_first) ia = max(ia, static_cast<int>(u0 - static_cast<int64_t>(b) * a.L));
+    if (b == b_last) ib = min(ib, static_cast<int>(u1 - static_cast<int64_t>(b) * a.L));
+    const float* base = a.ds + static_cast<int64_t>(b) * a.ds_b +
+                        static_cast<int64_t>(h) * a.ds_h + r;
+    int i = ia;
+    for (; i + 8 <= ib; i += 8) {
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = base[static_cast<int64_t>(i + e) * step];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += x[e];
     }
+#pragma unroll
+    for (int e = 0; e < 7; ++e)
+      if (i + e < ib) acc[e] += base[static_cast<int64_t>(i + e) * step];
   }
-  a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + dr] = acc;
+  const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + dr] = sum;
 }
 
-// out[k, h] = sum over r in bucket k's range, over the pieces, of the
-// diagonal sums: one block per (k, h), a fixed tree over its 256 threads.
+// Folds the pieces: partial[0, h, dr] = sum over z of partial[z, h, dr], the
+// pieces taken in eight interleaved accumulators (piece z to accumulator
+// z mod 8) and the eight added in a fixed tree.  A thread owns one (h, dr)
+// across all pieces, so it may overwrite piece 0 in place.
+__global__ void __launch_bounds__(128) t5_piece_sum_kernel(const T5Reduce a) {
+  const int nd = 2 * a.L - 1;
+  const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
+  if (dr >= nd) return;
+  const int h = blockIdx.y;
+  const int64_t stride = static_cast<int64_t>(a.Hq) * nd;
+  const float* src = a.partial + static_cast<int64_t>(h) * nd + dr;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int z = 0;
+  for (; z + 8 <= a.chunks; z += 8) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = src[(z + e) * stride];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += x[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 7; ++e)
+    if (z + e < a.chunks) acc[e] += src[(z + e) * stride];
+  a.partial[static_cast<int64_t>(h) * nd + dr] =
+      ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// out[k, h] = sum of the diagonal sums over bucket k's range of r: one block
+// per (k, h), a fixed tree over its 256 threads.
 __global__ void __launch_bounds__(256) t5_bucket_sum_kernel(const T5Reduce a, const T5Ranges rg) {
   __shared__ float red[256];
   const int k = blockIdx.x;
   const int h = blockIdx.y;
   const int nd = 2 * a.L - 1;
+  const float* diag = a.partial + static_cast<int64_t>(h) * nd + (a.L - 1);  // diag[r]
   float acc = 0.f;
-  for (int r = rg.lo[k] + static_cast<int>(threadIdx.x); r <= rg.hi[k]; r += 256)
-    for (int z = 0; z < a.chunks; ++z)
-      acc += a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + (r + a.L - 1)];
+  for (int r = rg.lo[k] + static_cast<int>(threadIdx.x); r <= rg.hi[k]; r += 256) acc += diag[r];
   red[threadIdx.x] = acc;
   for (int w = 128; w > 0; w >>= 1) {
     __syncthreads();

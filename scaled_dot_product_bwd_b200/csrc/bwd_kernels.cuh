@@ -970,20 +970,22 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive(ds_full(c & 1));
         if constexpr (DS_OUT) {
           // fp32 dS of this row's 64 keys while the dQ MMA runs; masked keys
-          // have P = 0 and so dS = 0
+          // have P = 0 and so dS = 0.  Streaming stores: dS is not read again
+          // by this kernel, and should not evict the K / V tiles that
+          // neighbouring heads reuse from L2.
           if (i < p.L) {
             float* dst = p.ds_out + static_cast<int64_t>(b) * p.sd_b +
                          static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(i) * p.sd_i + n0;
             if (n0 + kBlk <= p.L) {
 #pragma unroll
               for (int e = 0; e < kBlk; e += 4)
-                *reinterpret_cast<float4*>(dst + e) =
-                    make_float4(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1]),
-                                __uint_as_float(pr[e + 2]), __uint_as_float(pr[e + 3]));
+                __stcs(reinterpret_cast<float4*>(dst + e),
+                       make_float4(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1]),
+                                   __uint_as_float(pr[e + 2]), __uint_as_float(pr[e + 3])));
             } else {
 #pragma unroll
               for (int e = 0; e < kBlk; ++e)
-                if (n0 + e < p.L) dst[e] = __uint_as_float(pr[e]);
+                if (n0 + e < p.L) __stcs(dst + e, __uint_as_float(pr[e]));
             }
           }
         }

@@ -260,7 +260,13 @@ sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, Bi
     if (ds_elems > 1e17) return SDPA_ERR_UNSUPPORTED;
     pl.ds_ws = true;
     pl.ds_bytes = round256(static_cast<size_t>(B * Hq * L * pl.lp) * sizeof(float));
-    split_reduction(B * L, ((2 * L - 1 + 127) / 128) * Hq, pl.chunks, pl.per_chunk);
+    // pieces of kT5RowsPerPiece (b, i) rows: the diagonals near the middle
+    // hold L rows per batch entry and the outer ones few, so short pieces keep
+    // every thread's chain of loads short and the grid balanced; the
+    // partial sums are then 1/64 of dS or less
+    pl.per_chunk = kT5RowsPerPiece;
+    if ((B * L + pl.per_chunk - 1) / pl.per_chunk > 65535) pl.per_chunk = (B * L + 65534) / 65535;
+    pl.chunks = static_cast<int>((B * L + pl.per_chunk - 1) / pl.per_chunk);
     pl.part_bytes = round256(static_cast<size_t>(pl.chunks * Hq * (2 * L - 1)) * sizeof(float));
   } else {
     return SDPA_ERR_UNSUPPORTED;  // no bias: nothing to differentiate
@@ -543,6 +549,8 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.num_buckets = bias->num_buckets;
     const unsigned rblocks = static_cast<unsigned>((2 * p.L - 1 + 127) / 128);
     t5_diag_kernel<<<dim3(rblocks, p.Hq, a.chunks), 128, 0, cs>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    t5_piece_sum_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(a);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
