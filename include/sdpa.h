@@ -224,8 +224,8 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
  * order, so repeated calls give identical bits.
  * workspace: at least sdpa_bwd_bias_grad_workspace_size(shape, bias) bytes,
  * 256-byte aligned, contents ignored on entry.  Except for a full-shape dense
- * bias, it holds an fp32 copy of dS, B * Hq * L * ceil4(L) floats, that the
- * gradient is reduced from.  dbias must not overlap any other argument.
+ * bias, it holds an fp32 copy of dS, B * Hq * L rows of L floats padded to a
+ * multiple of 8, that the gradient is reduced from.  dbias must not overlap any other argument.
  */
 size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias);
 sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,

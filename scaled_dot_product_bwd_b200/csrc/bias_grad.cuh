@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(256) ds_zero_outside_band_kernel(const AttnPar
 // kept indices (extents eb, eh, ei: the full extent where kept, else 1);
 // the reduced index t enumerates the broadcast ones (extents rb, rh, ri).
 struct DenseReduce {
-  const float* ds;               // [B, Hq, L, lp] fp32, row stride lp
+  const float* ds;               // [B, Hq, L, lp] fp32, row stride lp (a multiple of 8)
   int64_t ds_b, ds_h, ds_i;
   float* out;                    // the bias gradient, element strides o_b, o_h, o_i
   int64_t o_b, o_h, o_i;

@@ -970,23 +970,44 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive(ds_full(c & 1));
         if constexpr (DS_OUT) {
           // fp32 dS of this row's 64 keys while the dQ MMA runs; masked keys
-          // have P = 0 and so dS = 0.  Streaming stores: dS is not read again
-          // by this kernel, and should not evict the K / V tiles that
+          // have P = 0 and so dS = 0.  Lanes 2m and 2m + 1 hold neighbouring
+          // rows; for every 8 keys they swap four values so that each store
+          // writes one whole 32-byte piece of a row from two lanes (the even
+          // lane's row first, then the odd lane's), rather than every lane
+          // half a piece of its own row.  Streaming stores: dS is not read
+          // again here and should not evict the K / V tiles that
           // neighbouring heads reuse from L2.
-          if (i < p.L) {
-            float* dst = p.ds_out + static_cast<int64_t>(b) * p.sd_b +
-                         static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(i) * p.sd_i + n0;
-            if (n0 + kBlk <= p.L) {
+          const int64_t head_off = static_cast<int64_t>(b) * p.sd_b + static_cast<int64_t>(hq) * p.sd_h;
+          if (n0 + kBlk <= p.L) {
+            const bool odd = (lane & 1) != 0;
+            const int i_a = odd ? i - 1 : i;  // the even lane's row
+            const int i_b = odd ? i : i + 1;  // the odd lane's row
+            const int c_off = n0 + (odd ? 4 : 0);
+            float* row_a = p.ds_out + head_off + static_cast<int64_t>(i_a) * p.sd_i + c_off;
+            float* row_b = p.ds_out + head_off + static_cast<int64_t>(i_b) * p.sd_i + c_off;
 #pragma unroll
-              for (int e = 0; e < kBlk; e += 4)
-                __stcs(reinterpret_cast<float4*>(dst + e),
-                       make_float4(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1]),
-                                   __uint_as_float(pr[e + 2]), __uint_as_float(pr[e + 3])));
-            } else {
+            for (int g = 0; g < kBlk; g += 8) {
+              float lo[4], hi[4], got[4];
 #pragma unroll
-              for (int e = 0; e < kBlk; ++e)
-                if (n0 + e < p.L) __stcs(dst + e, __uint_as_float(pr[e]));
+              for (int t = 0; t < 4; ++t) {
+                lo[t] = __uint_as_float(pr[g + t]);
+                hi[t] = __uint_as_float(pr[g + 4 + t]);
+              }
+              // the even lane sends its keys g+4..g+7, the odd lane its g..g+3
+#pragma unroll
+              for (int t = 0; t < 4; ++t) got[t] = __shfl_xor_sync(0xffffffffu, odd ? lo[t] : hi[t], 1);
+              const float4 va = odd ? make_float4(got[0], got[1], got[2], got[3])
+                                    : make_float4(lo[0], lo[1], lo[2], lo[3]);
+              const float4 vb = odd ? make_float4(hi[0], hi[1], hi[2], hi[3])
+                                    : make_float4(got[0], got[1], got[2], got[3]);
+              if (i_a < p.L) __stcs(reinterpret_cast<float4*>(row_a + g), va);
+              if (i_b < p.L) __stcs(reinterpret_cast<float4*>(row_b + g), vb);
             }
+          } else if (i < p.L) {
+            float* dst = p.ds_out + head_off + static_cast<int64_t>(i) * p.sd_i + n0;
+#pragma unroll
+            for (int e = 0; e < kBlk; ++e)
+              if (n0 + e < p.L) __stcs(dst + e, __uint_as_float(pr[e]));
           }
         }
       }

@@ -230,7 +230,7 @@ sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, Bi
   const int64_t B = s->B, Hq = s->Hq, L = s->L;
   pl = BiasGradPlan{};
   pl.d_bytes = round256(static_cast<size_t>(B * Hq * L) * sizeof(float));
-  pl.lp = (L + 3) / 4 * 4;
+  pl.lp = (L + 7) / 8 * 8;  // staged dS rows start on 32-byte boundaries
   // B * Hq * L * lp floats must stay far from 2^63 bytes
   const double ds_elems = static_cast<double>(B) * Hq * L * pl.lp;
   if (bias->kind == SDPA_BIAS_DENSE) {
