@@ -4,6 +4,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA path never does.
 """
 from .sdpa_oracle import (  # noqa: F401
+    alibi_slope_gradient,
     attention_backward,
     attention_forward,
     attention_probs,

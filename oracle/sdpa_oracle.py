@@ -39,6 +39,12 @@ What it computes, and where each piece comes from:
   rule to the definition above (dP = dO V^T, dS = P * (dP - rowsum(P*dP)),
   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO, with dK / dV summed over
   the query heads that share a KV head).
+* ALiBi: the flashT5 README names it among the supported positional
+  schemes but prints no formula.  The oracle takes the linear bias of Press
+  et al. 2022 ("Train Short, Test Long"), bias = -m_h |j - i| with one slope
+  m_h per query head given by the caller; under a causal mask this is the
+  paper's -m_h (i - j), and the absolute value extends it to keys after the
+  query.
 * Bias gradients: the scores are linear in the bias with coefficient 1, so
   the gradient of a dense bias is dS itself, summed over every index along
   which the bias is broadcast, and the gradient of a T5 table entry
@@ -64,6 +70,7 @@ __all__ = [
     "attention_probs",
     "dense_bias_gradient",
     "t5_table_gradient",
+    "alibi_slope_gradient",
 ]
 
 
@@ -138,9 +145,13 @@ def _as64(x):
 
 
 def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
-                 t5_max_distance, t5_bidirectional):
+                 t5_max_distance, t5_bidirectional, alibi_slopes=None):
     """Additive bias for one (batch, query head), [L, L] float64 (or 0)."""
     out = 0.0
+    if alibi_slopes is not None:
+        i = np.arange(L)[:, None]
+        j = np.arange(L)[None, :]
+        out = out - alibi_slopes[hq] * np.abs(j - i)
     if bias is not None:
         # a bias row of extent 1 is broadcast over the query rows
         out = out + np.broadcast_to(
@@ -155,7 +166,8 @@ def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
 
 def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
                 window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
-                t5_max_distance=128, t5_bidirectional=True, rows=None):
+                t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None,
+                rows=None):
     """Masked score matrix S for one (b, hq): scale * Q K^T + bias, -inf where
     masked.  q: [B, L, Hq, d], k: [B, L, Hkv, d] float64 arrays.  With
     ``rows`` (an index array), only those query rows of S are formed."""
@@ -165,8 +177,8 @@ def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
     r = np.arange(L) if rows is None else np.asarray(rows)
     S = scale * (q[b, r, hq, :] @ k[b, :, g, :].T)
     S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets,
-                         t5_max_distance, t5_bidirectional)[r] \
-        if (bias is not None or t5_table is not None) else S
+                         t5_max_distance, t5_bidirectional, alibi_slopes)[r] \
+        if (bias is not None or t5_table is not None or alibi_slopes is not None) else S
     M = visibility_mask(L, causal, window_left, window_right)[r]
     S = np.where(M, S, -np.inf)
     return S
@@ -199,7 +211,7 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
     """Probability matrix P (rows sum to 1 over visible keys) for one head."""
     q = _as64(q)
     k = _as64(k)
-    for name in ("bias", "t5_table"):
+    for name in ("bias", "t5_table", "alibi_slopes"):
         if name in mask_bias:
             mask_bias[name] = _as64(mask_bias[name])
     S = head_scores(q, k, b, hq, scale=_scale_of(q.shape[-1], scale), **mask_bias)
@@ -210,17 +222,18 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
 def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
                       window_right=-1, bias=None, t5_table=None,
                       t5_num_buckets=32, t5_max_distance=128,
-                      t5_bidirectional=True, batches=None, kv_heads=None,
-                      query_rows=None):
+                      t5_bidirectional=True, alibi_slopes=None, batches=None,
+                      kv_heads=None, query_rows=None):
     """O = softmax(scale Q K^T + bias, masked) V and LSE, in float64.
 
     q: [B, L, Hq, d]; k, v: [B, L, Hkv, d]; bias: [B|1, Hq|1, L, L] or None;
-    t5_table: [num_buckets, Hq] or None.  Returns O [B, L, Hq, d] and
+    t5_table: [num_buckets, Hq] or None; alibi_slopes: [Hq] or None.
+    Returns O [B, L, Hq, d] and
     LSE [B, Hq, L]; when ``batches`` / ``kv_heads`` restrict the work to a
     subset, entries outside it are NaN.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
-    bias, t5_table = _as64(bias), _as64(t5_table)
+    bias, t5_table, alibi_slopes = _as64(bias), _as64(t5_table), _as64(alibi_slopes)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     assert Hq % Hkv == 0
@@ -230,7 +243,8 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
     LSE = np.full((B, Hq, L), np.nan)
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
-              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional)
+              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional,
+              alibi_slopes=alibi_slopes)
     r = np.arange(L) if query_rows is None else np.asarray(query_rows)
     bs, gs = _select(B, Hkv, batches, kv_heads)
     for b in bs:
@@ -246,8 +260,8 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
 def attention_backward(q, k, v, do, *, scale=None, causal=False,
                        window_left=-1, window_right=-1, bias=None,
                        t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-                       t5_bidirectional=True, batches=None, kv_heads=None,
-                       return_dbias=False):
+                       t5_bidirectional=True, alibi_slopes=None, batches=None,
+                       kv_heads=None, return_dbias=False):
     """Gradients of sum(O * dO) with respect to Q, K, V (float64).
 
     Returns dQ [B, L, Hq, d], dK and dV [B, L, Hkv, d] (and, with
@@ -255,7 +269,7 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     additive bias).  Subset selection as in ``attention_forward``.
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
-    bias, t5_table = _as64(bias), _as64(t5_table)
+    bias, t5_table, alibi_slopes = _as64(bias), _as64(t5_table), _as64(alibi_slopes)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
@@ -266,7 +280,8 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     dB = np.full((B, Hq, L, L), np.nan) if return_dbias else None
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
-              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional)
+              t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional,
+              alibi_slopes=alibi_slopes)
     bs, gs = _select(B, Hkv, batches, kv_heads)
     for b in bs:
         for g in gs:
@@ -322,3 +337,13 @@ def t5_table_gradient(dS, num_buckets: int = 32, max_distance: int = 128,
     for h in range(Hq):
         np.add.at(grad[:, h], bucket.ravel(), dS[:, h].sum(axis=0).ravel())
     return grad
+
+
+def alibi_slope_gradient(dS):
+    """Gradient of the ALiBi slopes [Hq] from dS [B, Hq, L, L]: the bias
+    -m_h |j - i| is linear in m_h, so dm_h = -sum over (b, i, j) of
+    |j - i| dS[b, h, i, j]."""
+    dS = np.asarray(dS, dtype=np.float64)
+    L, Lk = dS.shape[2], dS.shape[3]
+    dist = np.abs(np.arange(Lk)[None, :] - np.arange(L)[:, None])
+    return -np.einsum("bhij,ij->h", dS, dist)

@@ -12,8 +12,8 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (attention_backward, attention_forward, attention_probs,
-                    dense_bias_gradient, head_scores, t5_relative_bucket,
+from oracle import (alibi_slope_gradient, attention_backward, attention_forward,
+                    attention_probs, dense_bias_gradient, head_scores, t5_relative_bucket,
                     t5_table_gradient, visibility_mask)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -367,6 +367,67 @@ def test_t5_table_gradient_central_differences(bidirectional, causal):
     # softmax rows sum to one, so each row of dS sums to zero, and so do the
     # table gradient's columns (every (i, j) lands in exactly one bucket)
     assert np.allclose(g.sum(axis=0), 0.0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- ALiBi
+def test_alibi_zero_slopes_is_no_bias():
+    q, k, v, do = qkv(1, 9, 2, 1, 4, seed=41)
+    a = attention_forward(q, k, v, causal=True, alibi_slopes=np.zeros(2))
+    b = attention_forward(q, k, v, causal=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_causal_alibi_is_a_key_position_bias():
+    # Softmax ignores a constant added to a whole row, and under a causal
+    # mask -m (i - j) = m j - m i: causal ALiBi must equal the bias m j, with
+    # LSE lower by m i.  A sign error or a dropped |.| breaks this.
+    B, L, Hq, Hkv, d = 2, 11, 3, 1, 5
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=43)
+    m = np.array([0.5, 0.25, 0.125])
+    O1, lse1 = attention_forward(q, k, v, causal=True, alibi_slopes=m)
+    keybias = m[None, :, None, None] * np.arange(L)[None, None, None, :] * np.ones((1, Hq, L, L))
+    O2, lse2 = attention_forward(q, k, v, causal=True, bias=keybias)
+    assert np.allclose(O1, O2, atol=1e-12)
+    shift = m[None, :, None] * np.arange(L)[None, None, :]
+    assert np.allclose(lse1, lse2 - shift, atol=1e-12)
+
+
+def test_bidirectional_alibi_is_symmetric_under_reversal():
+    # |j - i| is unchanged when both positions are mirrored, so reversing the
+    # sequence reverses the outputs; a one-sided (j - i) form would not.
+    B, L, Hq, Hkv, d = 1, 10, 2, 2, 4
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=47)
+    m = np.array([0.7, 0.3])
+    O, lse = attention_forward(q, k, v, alibi_slopes=m)
+    Or, lser = attention_forward(q[:, ::-1], k[:, ::-1], v[:, ::-1], alibi_slopes=m)
+    assert np.allclose(O, Or[:, ::-1], atol=1e-12)
+    assert np.allclose(lse, lser[:, :, ::-1], atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_alibi_slope_gradient_central_differences(causal):
+    B, L, Hq, Hkv, d = 2, 8, 2, 1, 3
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=53)
+    m = np.array([0.6, 0.2])
+    kw = dict(causal=causal, alibi_slopes=m)
+    dq, dk, dv, dS = attention_backward(q, k, v, do, return_dbias=True, **kw)
+    g = alibi_slope_gradient(dS)
+    h = 1e-6
+    for hq in range(Hq):
+        mp = m.copy(); mp[hq] += h
+        mm = m.copy(); mm[hq] -= h
+        num = (_loss(q, k, v, do, {**kw, "alibi_slopes": mp})
+               - _loss(q, k, v, do, {**kw, "alibi_slopes": mm})) / (2 * h)
+        assert abs(num - g[hq]) < 1e-7, (hq, num, g[hq])
+    # and dQ / dK / dV through the ALiBi bias, as for the other biases
+    for name, x, gx in (("q", q, dq), ("k", k, dk)):
+        idx = (1, 3, 1 if name == "q" else 0, 2)
+        xp = x.copy(); xp[idx] += h
+        xm = x.copy(); xm[idx] -= h
+        args = (xp, k, v) if name == "q" else (q, xp, v)
+        argm = (xm, k, v) if name == "q" else (q, xm, v)
+        num = (_loss(*args, do, kw) - _loss(*argm, do, kw)) / (2 * h)
+        assert abs(num - gx[idx]) < 1e-7
 
 
 def test_D_two_ways():
