@@ -40,6 +40,9 @@ CONFIGS = {
     "t5rpe": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="t5"),
     "t5dense": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="dense"),
     "tiny": dict(B=1, Hq=2, Hkv=2, L=128, d=64, causal=True, wl=-1, wr=-1, bias="none"),
+    # the Mistral GQA shape with an in-kernel ALiBi bias (slopes 2^(-8 (h+1) / 32))
+    "alibi_causal_4k": dict(B=4, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=-1, wr=-1,
+                            bias="alibi"),
     # the mistral4k shape at batch 2: the case the ncu captures run on (inputs
     # still larger than L2, a few hundred MB on the device)
     "mistral4k_small": dict(B=2, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1,
@@ -162,7 +165,7 @@ def make_case(c, seed):
     from scaled_dot_product_bwd_b200.inputs import make_inputs
     return make_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], c["d"], seed=seed,
                        t5_buckets=32 if c["bias"] == "t5" else 0,
-                       dense_bias=c["bias"] == "dense")
+                       dense_bias=c["bias"] == "dense", alibi=c["bias"] == "alibi")
 
 
 # ------------------------------------------------------------------ oracle
@@ -170,7 +173,8 @@ def oracle_sample(c, inp):
     """fwd + bwd of the oracle on batch 0, KV head 0 (all its query heads)."""
     from oracle import attention_backward, attention_forward
     kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"],
-              bias=inp.bias, t5_table=inp.t5_table, batches=[0], kv_heads=[0])
+              bias=inp.bias, t5_table=inp.t5_table, alibi_slopes=inp.alibi_slopes,
+              batches=[0], kv_heads=[0])
     attention_forward(inp.q, inp.k, inp.v, **kw)
     attention_backward(inp.q, inp.k, inp.v, inp.do, **kw)
 
@@ -260,8 +264,9 @@ def run_gpu(args, c):
     q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
     bias = inp.bias.to(dev) if inp.bias is not None else None
     table = inp.t5_table.to(dev) if inp.t5_table is not None else None
+    slopes = inp.alibi_slopes.to(dev) if inp.alibi_slopes is not None else None
     kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"], bias=bias,
-              t5_table=table)
+              t5_table=table, alibi_slopes=slopes)
     o = torch.empty_like(q)
     lse = torch.empty(c["B"], c["Hq"], c["L"], device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -428,6 +433,8 @@ def bias_grad_extra_bytes(c):
     ds = B * H * L * L * 4
     if c["bias"] == "t5":
         return 2 * ds + 32 * H * 4
+    if c["bias"] == "alibi":
+        return 2 * ds + H * 4
     return ds                      # a full-shape dense bias: dS goes straight out
 
 
@@ -447,17 +454,17 @@ def run_bias_grad(args, c):
     q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
     bias = inp.bias.to(dev) if inp.bias is not None else None
     table = inp.t5_table.to(dev) if inp.t5_table is not None else None
+    slopes = inp.alibi_slopes.to(dev) if inp.alibi_slopes is not None else None
     kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"], bias=bias,
-              t5_table=table)
+              t5_table=table, alibi_slopes=slopes)
     o = torch.empty_like(q)
     lse = torch.empty(c["B"], c["Hq"], c["L"], device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ref = bias if bias is not None else table
+    ref = next(x for x in (bias, table, slopes) if x is not None)
     dbias = torch.empty_strided(ref.shape, ref.stride(), device=dev, dtype=torch.float32)
     ws = torch.empty(sdpa_bwd_workspace_size(q, k), device=dev, dtype=torch.uint8)
-    wsg = torch.empty(max(256, sdpa_bwd_bias_grad_workspace_size(q, k, bias=bias,
-                                                                 t5_table=table)),
-                      device=dev, dtype=torch.uint8)
+    wsg = torch.empty(max(256, sdpa_bwd_bias_grad_workspace_size(
+        q, k, bias=bias, t5_table=table, alibi_slopes=slopes)), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
 
     def step(grad, ev=None):

@@ -81,7 +81,8 @@ typedef struct sdpa_mask_spec {
 typedef enum sdpa_bias_kind {
   SDPA_BIAS_NONE = 0,
   SDPA_BIAS_DENSE = 1, /* additive float32 bias[b, h, i, j]                  */
-  SDPA_BIAS_T5 = 2     /* additive table[bucket(j - i), h], bucketed in-kernel */
+  SDPA_BIAS_T5 = 2,    /* additive table[bucket(j - i), h], bucketed in-kernel */
+  SDPA_BIAS_ALIBI = 3  /* additive -slope[h] |j - i|, computed in-kernel       */
 } sdpa_bias_kind;
 
 /*
@@ -101,6 +102,11 @@ typedef enum sdpa_bias_kind {
  *          num_buckets even when bidirectional, max_distance > max_exact
  *          (num_buckets/4 when bidirectional, num_buckets/2 otherwise).
  *          Nothing L x L is materialised.
+ *   ALIBI: ptr -> float32 slopes[Hq]; bias[h, i, j] = -slopes[h] |j - i|.
+ *          The README names ALiBi among its positional schemes without a
+ *          formula; this is the linear bias of Press et al. 2022 ("Train
+ *          Short, Test Long"), equal to their -m (i - j) on the keys a causal
+ *          mask leaves.  Strides and T5 fields are ignored.
  */
 typedef struct sdpa_bias_desc {
   int32_t kind; /* sdpa_bias_kind */
@@ -219,6 +225,8 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
  *   T5:    dbias[k * Hq + h] = sum of dS[b, h, i, j] over every (b, i, j)
  *          with bucket(j - i) = k: float32 [num_buckets, Hq] like the table,
  *          16-byte aligned.
+ *   ALIBI: dbias[h] = -sum of |j - i| dS[b, h, i, j] over every (b, i, j):
+ *          the gradient of the slopes, float32 [Hq], 16-byte aligned.
  *   NONE:  SDPA_ERR_UNSUPPORTED.
  * dq, dk, dv as sdpa_bwd.  Deterministic: every sum is taken in one fixed
  * order, so repeated calls give identical bits.

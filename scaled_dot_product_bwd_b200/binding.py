@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsdpa_b200.so")
 SDPA_OK = 0
 STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
                 3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
-BIAS_NONE, BIAS_DENSE, BIAS_T5 = 0, 1, 2
+BIAS_NONE, BIAS_DENSE, BIAS_T5, BIAS_ALIBI = 0, 1, 2, 3
 
 BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 
@@ -135,10 +135,18 @@ def make_mask(causal: bool, window_left: int, window_right: int) -> MaskSpec:
 
 
 def make_bias(bias: torch.Tensor | None, t5_table: torch.Tensor | None, num_buckets: int,
-              max_distance: int, bidirectional: bool, dims: tuple | None = None) -> BiasDesc:
+              max_distance: int, bidirectional: bool, dims: tuple | None = None,
+              alibi_slopes: torch.Tensor | None = None) -> BiasDesc:
     """Bias descriptor; ``dims`` = (B, Hq, L) of the attention checks the shapes."""
-    if bias is not None and t5_table is not None:
-        raise ValueError("give either a dense bias or a T5 table, not both")
+    if sum(x is not None for x in (bias, t5_table, alibi_slopes)) > 1:
+        raise ValueError("give one of a dense bias, a T5 table or ALiBi slopes")
+    if alibi_slopes is not None:
+        if (alibi_slopes.dtype != torch.float32 or alibi_slopes.dim() != 1
+                or not alibi_slopes.is_contiguous()):
+            raise ValueError("ALiBi slopes must be a contiguous float32 [Hq] vector")
+        if dims is not None and alibi_slopes.shape[0] != dims[1]:
+            raise ValueError("ALiBi slopes must have one entry per query head")
+        return BiasDesc(BIAS_ALIBI, alibi_slopes.data_ptr(), 0, 0, 0, 0, 0, 0)
     if bias is not None:
         if bias.dtype != torch.float32 or bias.dim() != 4 or bias.stride(-1) != 1:
             raise ValueError("dense bias must be float32 [B|1, H|1, L, L] with j contiguous")
@@ -170,7 +178,7 @@ def _same_layout(a: torch.Tensor, ref: torch.Tensor, name: str):
 
 def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=None,
              t5_table=None, t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
-             scale=None, out=None, lse=None):
+             alibi_slopes=None, scale=None, out=None, lse=None):
     """O, LSE = attention forward (see sdpa_fwd in include/sdpa.h)."""
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -188,7 +196,7 @@ def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=Non
         raise ValueError("lse must be contiguous float32 [B, Hq, L]")
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (B, Hq, L))
+                   (B, Hq, L), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bd),
                       ctypes.byref(m), sc, _ptr(out), _ptr(lse), _stream(q))
@@ -204,8 +212,8 @@ def sdpa_bwd_workspace_size(q, k, deterministic: bool = True) -> int:
 
 def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
              bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-             t5_bidirectional=True, scale=None, dq=None, dk=None, dv=None, workspace=None,
-             deterministic=True, phases=BWD_ALL):
+             t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None, dv=None,
+             workspace=None, deterministic=True, phases=BWD_ALL):
     """dQ, dK, dV = attention backward (see sdpa_bwd / sdpa_bwd_phases in include/sdpa.h).
 
     ``phases`` selects launches (BWD_PREPROCESS | BWD_DQ | BWD_DKDV); the
@@ -229,7 +237,7 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]))
+                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
             ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk), _ptr(dv),
@@ -244,7 +252,7 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
 
 def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_left=-1,
                      window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
-                     t5_max_distance=128, t5_bidirectional=True, scale=None):
+                     t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None, scale=None):
     """Backward into caller-given dQ, dK, dV with no workspace and no allocation.
 
     For callers that cannot allocate device memory: the library's built-in
@@ -258,7 +266,7 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
         _same_layout(t, ref, n)
     sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]))
+                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_bwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
                               _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq),
@@ -268,22 +276,23 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
 
 
 def sdpa_bwd_bias_grad_workspace_size(q, k, *, bias=None, t5_table=None, t5_num_buckets=32,
-                                      t5_max_distance=128, t5_bidirectional=True) -> int:
+                                      t5_max_distance=128, t5_bidirectional=True,
+                                      alibi_slopes=None) -> int:
     lib = load_library()
     shape = make_shape(q, k)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]))
+                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
     return int(lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(shape), ctypes.byref(bd)))
 
 
 def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
                        bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-                       t5_bidirectional=True, scale=None, dq=None, dk=None, dv=None, dbias=None,
-                       workspace=None):
+                       t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None,
+                       dv=None, dbias=None, workspace=None):
     """dQ, dK, dV and the bias gradient (see sdpa_bwd_bias_grad in include/sdpa.h).
 
-    The bias gradient has the dense bias's shape and strides, or the T5
-    table's [num_buckets, Hq] shape.
+    The bias gradient has the dense bias's shape and strides, the T5 table's
+    [num_buckets, Hq] shape, or the ALiBi slopes' [Hq] shape.
     """
     lib = load_library()
     shape = make_shape(q, k)
@@ -297,10 +306,10 @@ def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, win
     _same_layout(dk, k, "dk")
     _same_layout(dv, k, "dv")
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]))
-    ref = bias if bias is not None else t5_table
+                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
+    ref = next((x for x in (bias, t5_table, alibi_slopes) if x is not None), None)
     if ref is None:
-        raise ValueError("a bias gradient needs a dense bias or a T5 table")
+        raise ValueError("a bias gradient needs a dense bias, a T5 table or ALiBi slopes")
     if dbias is None:
         dbias = torch.empty_strided(ref.shape, ref.stride(), device=q.device,
                                     dtype=torch.float32)

@@ -78,8 +78,22 @@ struct AttnParams {
   int64_t sb_b, sb_h, sb_i;
   const float* t5_table;       // [num_buckets, Hq]
   T5Spec t5;
+  // ALiBi runs in the kBiasT5 kernels: both biases are functions of j - i
+  // that the kernels tabulate per tile
+  int alibi;                   // 1: bias = -alibi_slopes[h] |j - i| instead of T5
+  const float* alibi_slopes;   // [Hq]
   uint64_t wait_limit_ns;
 };
+
+// Relative-position bias of distance rel = j - i for query head hq, in log2
+// units (times log2 e), as the kBiasT5 kernels tabulate it per tile: the
+// T5 table entry of rel's bucket (catie-aq/flashT5 README, "T5-like relative
+// position encoding biases"), or ALiBi's -m_h |rel| (Press et al. 2022;
+// named by the same README among the supported positional schemes).
+__device__ __forceinline__ float rel_bias_log2(const AttnParams& p, int rel, int hq) {
+  if (p.alibi) return -(p.alibi_slopes[hq] * kLog2e) * fabsf(static_cast<float>(rel));
+  return p.t5_table[t5_bucket(rel, p.t5) * p.Hq + hq] * kLog2e;
+}
 
 // Whether column c of a fully visible tile takes the FMA-pipe exponential:
 // never with a dense bias, whose entries may be -inf (masked) even inside a

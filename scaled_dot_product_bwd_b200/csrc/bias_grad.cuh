@@ -137,11 +137,12 @@ __global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseRedu
 }
 
 // ---------------------------------------------------------------------
-// T5 table gradient.  The bucket depends on j - i alone, so first sum dS
-// along each diagonal r = j - i (r in [-(L-1), L-1]), then add up the
-// diagonals of each bucket.  Every bucket covers one contiguous range of r
-// (the bucket is monotone in |r| on each side of 0, and the two sides use
-// disjoint ids when bidirectional), given to the last kernel as [lo, hi].
+// T5 table (and ALiBi slope) gradient.  The bias depends on j - i alone, so
+// first sum dS along each diagonal r = j - i (r in [-(L-1), L-1]), then add
+// up the diagonals of each bucket (or weigh them by -|r| for ALiBi).  Every
+// bucket covers one contiguous range of r (the bucket is monotone in |r| on
+// each side of 0, and the two sides use disjoint ids when bidirectional),
+// given to the last kernel as [lo, hi].
 struct T5Reduce {
   const float* ds;               // [B, Hq, L, lp] fp32
   int64_t ds_b, ds_h, ds_i;
@@ -242,6 +243,25 @@ __global__ void __launch_bounds__(256) t5_bucket_sum_kernel(const T5Reduce a, co
     if (static_cast<int>(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
   }
   if (threadIdx.x == 0) a.out[static_cast<int64_t>(k) * a.Hq + h] = red[0];
+}
+
+// ALiBi: the bias -m_h |r| is linear in the slope, so
+// out[h] = -sum over r of |r| times the diagonal sum of r; one block per
+// head, a fixed tree over its 256 threads.
+__global__ void __launch_bounds__(256) alibi_slope_grad_kernel(const T5Reduce a) {
+  __shared__ float red[256];
+  const int h = blockIdx.x;
+  const int nd = 2 * a.L - 1;
+  const float* diag = a.partial + static_cast<int64_t>(h) * nd;  // diag[r + L - 1]
+  float acc = 0.f;
+  for (int dr = static_cast<int>(threadIdx.x); dr < nd; dr += 256)
+    acc += fabsf(static_cast<float>(dr - (a.L - 1))) * diag[dr];
+  red[threadIdx.x] = acc;
+  for (int w = 128; w > 0; w >>= 1) {
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
+  }
+  if (threadIdx.x == 0) a.out[h] = -red[0];
 }
 
 }  // namespace sdpa

@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(352, 1)
         float* lt = lut + (it & 1) * 256;
         const int base = n0 - m0 - (kBlk - 1);
         for (int r = row; r < kTile + kBlk - 1; r += kTile)
-          lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
+          lt[r] = rel_bias_log2(p, base + r, hq);
         named_barrier(1 + wg, kTile);
         lut_row = lt + row + (kBlk - 1);
       }
@@ -857,7 +857,7 @@ __global__ void __launch_bounds__(352, 1)
           float* lt = lut + (c & 1) * 256;
           const int base = n0 - m0 - (kTile - 1);
           for (int r = row; r < kTile + kBlk - 1; r += kTile)
-            lt[r] = p.t5_table[t5_bucket(base + r, p.t5) * p.Hq + hq] * kLog2e;
+            lt[r] = rel_bias_log2(p, base + r, hq);
           named_barrier(1 + wg, kTile);
           lut_row = lt + (kTile - 1) - row;
         }

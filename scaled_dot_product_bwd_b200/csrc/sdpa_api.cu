@@ -169,6 +169,11 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
       if (!fill_t5(p.t5, nb, bias->max_distance, bias->bidirectional)) return SDPA_ERR_INVALID_ARG;
       p.bias_kind = kBiasT5;
       p.t5_table = bias->ptr;
+    } else if (bias->kind == SDPA_BIAS_ALIBI) {
+      if (!bias->ptr) return SDPA_ERR_INVALID_ARG;
+      p.bias_kind = kBiasT5;  // the relative-position kernels, with the ALiBi table
+      p.alibi = 1;
+      p.alibi_slopes = bias->ptr;
     } else {
       return SDPA_ERR_INVALID_ARG;
     }
@@ -256,7 +261,7 @@ sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, Bi
       if (pl.chunks > 1)
         pl.part_bytes = round256(static_cast<size_t>(pl.chunks * n_out * pl.lp) * sizeof(float));
     }
-  } else if (bias->kind == SDPA_BIAS_T5) {
+  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_ALIBI) {
     if (ds_elems > 1e17) return SDPA_ERR_UNSUPPORTED;
     pl.ds_ws = true;
     pl.ds_bytes = round256(static_cast<size_t>(B * Hq * L * pl.lp) * sizeof(float));
@@ -465,7 +470,7 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   st = plan_bias_grad(shape, bias, pl);
   if (st != SDPA_OK) return st;
   T5Ranges rg;
-  if (p.bias_kind == kBiasT5 && !t5_ranges(p.t5, p.L, bias->num_buckets, rg))
+  if (p.bias_kind == kBiasT5 && !p.alibi && !t5_ranges(p.t5, p.L, bias->num_buckets, rg))
     return SDPA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < pl.total)
@@ -546,13 +551,16 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.uchunk = pl.per_chunk;
     a.partial = part;
     a.out = dbias;
-    a.num_buckets = bias->num_buckets;
+    a.num_buckets = p.alibi ? 0 : bias->num_buckets;
     const unsigned rblocks = static_cast<unsigned>((2 * p.L - 1 + 127) / 128);
     t5_diag_kernel<<<dim3(rblocks, p.Hq, a.chunks), 128, 0, cs>>>(a);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     t5_piece_sum_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(a);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
-    t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
+    if (p.alibi)
+      alibi_slope_grad_kernel<<<p.Hq, 256, 0, cs>>>(a);
+    else
+      t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
   }
   return SDPA_OK;

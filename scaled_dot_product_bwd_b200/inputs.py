@@ -9,7 +9,8 @@ a parity check see the same values.
 
 Layouts: Q, dO [B, L, Hq, d]; K, V [B, L, Hkv, d] (batch, sequence, heads,
 head dim -- the (B, T, N, H) layout of the codelab "jax-gpu-05-attention-gpu",
-section 3); T5 table [num_buckets, Hq]; dense bias [B, Hq, L, L].
+section 3); T5 table [num_buckets, Hq]; dense bias [B, Hq, L, L]; ALiBi
+slopes [Hq].
 """
 from __future__ import annotations
 
@@ -26,12 +27,16 @@ class Inputs:
     do: torch.Tensor
     t5_table: torch.Tensor | None = None
     bias: torch.Tensor | None = None
+    alibi_slopes: torch.Tensor | None = None
 
 
 def make_inputs(B: int, L: int, Hq: int, Hkv: int, d: int, *, seed: int = 0,
                 t5_buckets: int = 0, dense_bias: bool = False,
-                bias_shape: tuple | None = None) -> Inputs:
-    """Draw Q, K, V, dO (bf16) and optionally a T5 table / dense bias (fp32)."""
+                bias_shape: tuple | None = None, alibi: bool = False) -> Inputs:
+    """Draw Q, K, V, dO (bf16) and optionally a T5 table / dense bias (fp32).
+
+    ALiBi slopes are not drawn: they are the geometric sequence of Press et
+    al. 2022, 2^(-8 (h + 1) / Hq) for head h (fp32)."""
     g = torch.Generator().manual_seed(seed)
 
     def randn(*shape):
@@ -45,7 +50,11 @@ def make_inputs(B: int, L: int, Hq: int, Hkv: int, d: int, *, seed: int = 0,
     bias = None
     if dense_bias:
         bias = randn(*(bias_shape or (B, Hq, L, L)))
-    return Inputs(q, k, v, do, table, bias)
+    slopes = None
+    if alibi:
+        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)],
+                              dtype=torch.float32)
+    return Inputs(q, k, v, do, table, bias, slopes)
 
 
 # The workloads of the benchmark table, by name.  Each entry: shapes, mask and

@@ -17,7 +17,7 @@ def case_inputs(c):
     return make_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], c["d"], seed=c.get("seed", 0),
                        t5_buckets=32 if c.get("bias") == "t5" else 0,
                        dense_bias=c.get("bias") == "dense",
-                       bias_shape=c.get("bias_shape"))
+                       bias_shape=c.get("bias_shape"), alibi=c.get("bias") == "alibi")
 
 
 def mask_kw(c):
@@ -36,7 +36,8 @@ def run_cuda(c, inp, backward=True):
     q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
     bias = inp.bias.to(dev) if inp.bias is not None else None
     table = inp.t5_table.to(dev) if inp.t5_table is not None else None
-    kw = dict(mask_kw(c), bias=bias, t5_table=table)
+    slopes = inp.alibi_slopes.to(dev) if inp.alibi_slopes is not None else None
+    kw = dict(mask_kw(c), bias=bias, t5_table=table, alibi_slopes=slopes)
     o, lse = sdpa_fwd(q, k, v, **kw)
     out = {"o": o, "lse": lse}
     if backward:
@@ -47,8 +48,8 @@ def run_cuda(c, inp, backward=True):
 
 
 def run_oracle(c, inp, backward=True, batches=None, kv_heads=None):
-    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table, batches=batches,
-              kv_heads=kv_heads)
+    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table,
+              alibi_slopes=inp.alibi_slopes, batches=batches, kv_heads=kv_heads)
     O, LSE = attention_forward(inp.q, inp.k, inp.v, **kw)
     out = {"o": O, "lse": LSE}
     if backward:

@@ -88,7 +88,8 @@ def test_fwd_rejects_bad_bias(lib):
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 31, 128, 1),        # T5, odd buckets (bidir)
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 256, 128, 1),       # T5, too many buckets
            binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 8, 1),          # T5, max_distance <= max_exact
-           binding.BiasDesc(2, 0, 0, 0, 0, 32, 128, 1)]              # T5, null table
+           binding.BiasDesc(2, 0, 0, 0, 0, 32, 128, 1),              # T5, null table
+           binding.BiasDesc(3, 0, 0, 0, 0, 0, 0, 0)]                 # ALiBi, null slopes
     for b in bad:
         assert _fwd(lib, _shape(), bias=b) == 1, (b.kind, b.num_buckets)
 
@@ -131,6 +132,8 @@ def test_bias_grad_workspace_size(lib):
     t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
     n = ws(t5)
     assert n >= d_bytes + ds_bytes + Hq * (2 * L - 1) * 4 and n % 256 == 0
+    alibi = binding.BiasDesc(3, 0x10000, 0, 0, 0, 0, 0, 0)
+    assert ws(alibi) >= d_bytes + ds_bytes and ws(alibi) % 256 == 0
     assert ws(binding.BiasDesc(0, None, 0, 0, 0, 0, 0, 0)) == 0       # nothing to differentiate
     assert ws(_dense(L * L, L * L, L)) == 0                          # heads overlap batches
     assert ws(_dense(Hq * L * L, L * L, 0)) == 0                      # one row for all queries
@@ -170,6 +173,21 @@ def test_binding_checks_bias_shapes():
             binding.make_bias(bad, None, 32, 128, True, (2, 4, 16))
     with pytest.raises(ValueError):
         binding.make_bias(None, torch.zeros(32, 3), 32, 128, True, (2, 4, 16))
+    binding.make_bias(None, None, 32, 128, True, (2, 4, 16), torch.zeros(4))
+    with pytest.raises(ValueError):                                   # one slope per head
+        binding.make_bias(None, None, 32, 128, True, (2, 4, 16), torch.zeros(3))
+    with pytest.raises(ValueError):                                   # one bias at a time
+        binding.make_bias(ok, None, 32, 128, True, (2, 4, 16), torch.zeros(4))
+
+
+def test_binding_entry_points_share_the_bias_keywords():
+    import inspect
+    keys = {"causal", "window_left", "window_right", "bias", "t5_table", "t5_num_buckets",
+            "t5_max_distance", "t5_bidirectional", "alibi_slopes", "scale"}
+    for fn in (binding.sdpa_fwd, binding.sdpa_bwd, binding.sdpa_bwd_noalloc,
+               binding.sdpa_bwd_bias_grad):
+        missing = keys - set(inspect.signature(fn).parameters)
+        assert not missing, (fn.__name__, missing)
 
 
 def test_t5_bucket_rejects_bad_args(lib):

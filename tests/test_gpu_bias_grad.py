@@ -1,6 +1,7 @@
 """GPU parity of the bias gradients (sdpa_bwd_bias_grad) against the float64
 oracle: a dense bias's gradient is dS, summed over the indices the bias is
-broadcast along; a T5 table's gradient is dS summed per bucket of j - i.
+broadcast along; a T5 table's gradient is dS summed per bucket of j - i; the
+ALiBi slopes' gradient is -sum |j - i| dS per head.
 
 Tolerances.  dS = P (dP - D) with D = rowsum(dO * O) formed from the stored
 bf16 O, so D_i carries the rounding of O: with unit roundoff u = 2^-8 (bf16,
@@ -12,7 +13,8 @@ by sqrt(d), which is why the other gradients do not feel it.  Let
     e_i = 4 u sqrt(sum_d (dO_id O_id)^2)      (about seven standard deviations).
 An output that sums dS over a set of entries takes, from each query row
 (b, h, i), the row's one D error times the P mass of its entries in the set:
-w_row = e_i * sum of P_ij over those entries.  Rows round independently, so
+w_row = e_i * sum of P_ij over those entries (weighted by |j - i| for the
+ALiBi slopes).  Rows round independently, so
 the rows' terms add in quadrature, and the bound is
     |err| <= 1e-2 + 1e-2 |ref| + sqrt(sum over rows of w_row^2)
 (for a full-shape dense bias one row and one entry: 1e-2 + 1e-2 |dS| + P e).
@@ -24,9 +26,9 @@ import pytest
 import torch
 
 from gpu_helpers import ATOL, RTOL, assert_close, case_inputs, mask_kw
-from oracle import (attention_backward, attention_forward, attention_probs,
-                    dense_bias_gradient, t5_relative_bucket, t5_table_gradient,
-                    visibility_mask)
+from oracle import (alibi_slope_gradient, attention_backward, attention_forward,
+                    attention_probs, dense_bias_gradient, t5_relative_bucket,
+                    t5_table_gradient, visibility_mask)
 from scaled_dot_product_bwd_b200 import sdpa_bwd, sdpa_bwd_bias_grad, sdpa_fwd
 from scaled_dot_product_bwd_b200.inputs import Inputs
 
@@ -50,6 +52,9 @@ CASES = {
     "t5_bidir_causal_gqa_d128": dict(B=1, Hq=2, Hkv=1, L=270, d=128, causal=True, bias="t5"),
     "t5_unidir_causal_d64": dict(B=2, Hq=2, Hkv=2, L=280, d=64, causal=True, bias="t5",
                                  t5_bidirectional=False),
+    # ALiBi slopes: dm_h = -sum |j - i| dS
+    "alibi_bidir_d64": dict(B=2, Hq=4, Hkv=4, L=301, d=64, bias="alibi"),
+    "alibi_causal_gqa_d128": dict(B=1, Hq=2, Hkv=1, L=270, d=128, causal=True, bias="alibi"),
 }
 
 
@@ -59,7 +64,8 @@ def run_cuda_bias_grad(c, inp, bias=None):
     if bias is None and inp.bias is not None:
         bias = inp.bias.to(dev)
     table = inp.t5_table.to(dev) if inp.t5_table is not None else None
-    kw = dict(mask_kw(c), bias=bias, t5_table=table)
+    slopes = inp.alibi_slopes.to(dev) if inp.alibi_slopes is not None else None
+    kw = dict(mask_kw(c), bias=bias, t5_table=table, alibi_slopes=slopes)
     o, lse = sdpa_fwd(q, k, v, **kw)
     dq, dk, dv, dbias = sdpa_bwd_bias_grad(q, k, v, o, do, lse, **kw)
     dq0, dk0, dv0 = sdpa_bwd(q, k, v, o, do, lse, **kw)
@@ -71,7 +77,8 @@ def run_cuda_bias_grad(c, inp, bias=None):
 
 
 def oracle_ds(c, inp):
-    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table)
+    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table,
+              alibi_slopes=inp.alibi_slopes)
     dq, dk, dv, dS = attention_backward(inp.q, inp.k, inp.v, inp.do, return_dbias=True, **kw)
     return dict(dq=dq, dk=dk, dv=dv), dS
 
@@ -81,7 +88,8 @@ U_BF16 = 2.0 ** -8
 
 def row_error_scale(c, inp):
     """e_i of the module docstring, [B, Hq, L], from the oracle's O and dO."""
-    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table)
+    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table,
+              alibi_slopes=inp.alibi_slopes)
     O, _ = attention_forward(inp.q, inp.k, inp.v, **kw)          # [B, L, Hq, d]
     dO = inp.do.double().numpy()
     e = 4 * U_BF16 * np.sqrt(np.sum((dO * O) ** 2, axis=-1))     # [B, L, Hq]
@@ -90,7 +98,8 @@ def row_error_scale(c, inp):
 
 def expected_bias_grad(c, inp, dS):
     """Oracle gradient and the sum over rows of w_row^2 (module docstring)."""
-    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table)
+    kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table,
+              alibi_slopes=inp.alibi_slopes)
     e = row_error_scale(c, inp)
     B, Hq, L = e.shape
     if c["bias"] == "dense":
@@ -100,6 +109,14 @@ def expected_bias_grad(c, inp, dS):
             for h in range(Hq):
                 w2[b, h] = (attention_probs(inp.q, inp.k, b, h, **kw) * e[b, h, :, None]) ** 2
         return dense_bias_gradient(dS, shape), dense_bias_gradient(w2, shape)
+    if c["bias"] == "alibi":
+        dist = np.abs(np.arange(L)[None, :] - np.arange(L)[:, None])
+        q2 = np.zeros(Hq)
+        for b in range(B):
+            for h in range(Hq):
+                P = attention_probs(inp.q, inp.k, b, h, **kw)
+                q2[h] += np.sum((e[b, h] * (P * dist).sum(axis=1)) ** 2)
+        return alibi_slope_gradient(dS), q2
     bidir = c.get("t5_bidirectional", True)
     nb = 32
     i = np.arange(L)[:, None]

@@ -40,6 +40,10 @@ CASES = {
     "scale_0p05_causal_d128": dict(B=1, Hq=2, Hkv=1, L=300, d=128, causal=True, scale=0.05),
     "negative_scale_d64": dict(B=1, Hq=2, Hkv=2, L=260, d=64, scale=-0.08),
     # decoder-style T5 buckets (distance folded to one sign) under a causal mask
+    # ALiBi (-slope_h |j - i|, slopes 2^(-8 (h + 1) / Hq)) through the relative-position kernels
+    "alibi_bidir_gqa_d64": dict(B=2, Hq=4, Hkv=2, L=300, d=64, bias="alibi"),
+    "alibi_causal_window_mqa_d128": dict(B=1, Hq=4, Hkv=1, L=390, d=128, causal=True, wl=200,
+                                         bias="alibi"),
     "t5_unidirectional_causal_d64": dict(B=2, Hq=2, Hkv=2, L=280, d=64, causal=True, bias="t5",
                                          t5_bidirectional=False),
 }
