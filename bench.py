@@ -57,12 +57,12 @@ CONFIGS = {
 NCU_TRAFFIC = {
     # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
     # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
-    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(169_943_808 + 22_621_952) / 2,
-                                    source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
-    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(170_351_616 + 43_025_920) / 2,
-                                  source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
-    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_755_712 + 33_460_992) / 2,
-                               source_hash="022b2b419da8a5be80c2029f8cf4f03e03aa79fbbc43a47a961c9d81bbca9700"),
+    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_241_024 + 22_872_064) / 2,
+                                    source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
+    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(171_017_728 + 43_307_776) / 2,
+                                  source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
+    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_843_008 + 34_080_000) / 2,
+                               source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
 }
 
 
