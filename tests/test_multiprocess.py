@@ -2,7 +2,13 @@
 each.  Every rank runs its own batch (replicas), the step time is the max over
 ranks, and the whole-job rate counts all ranks' FLOPs.  Also checks that the
 per-rank inputs differ (each rank draws its own seeded batch) and that a rank
-which raises is reported to the launcher rather than hanging the other."""
+which raises is reported to the launcher rather than hanging the other.
+
+The bias gradients (a T5 table's, the ALiBi slopes') are weight gradients:
+each replica's covers its own batch shard, and the training framework's
+weight-gradient all-reduce sums them.  The last test checks, with the
+oracle on two gloo ranks, that the sum of the shards' gradients is the
+gradient of the whole batch."""
 import os
 import socket
 
@@ -73,3 +79,58 @@ def test_failing_rank_is_reported_not_hung():
     out, codes = _run(fail_rank=1)
     assert codes[1] != 0                             # the failing rank exits non-zero
     assert all(c is not None for c in codes)         # nobody is left hanging
+
+
+def _grad_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import datetime
+
+    from oracle import alibi_slope_gradient, attention_backward, t5_table_gradient
+    from scaled_dot_product_bwd_b200.inputs import make_inputs
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        full = make_inputs(2 * world, 24, 2, 1, 8, seed=5, t5_buckets=8, alibi=True)
+        sl = slice(2 * rank, 2 * rank + 2)            # this rank's batch shard
+        args = (full.q[sl], full.k[sl], full.v[sl], full.do[sl])
+        *_, dS = attention_backward(*args, causal=True, t5_table=full.t5_table,
+                                    t5_num_buckets=8, t5_max_distance=12, return_dbias=True)
+        table = torch.from_numpy(t5_table_gradient(dS, 8, 12, True))
+        *_, dS2 = attention_backward(*args, causal=True, alibi_slopes=full.alibi_slopes,
+                                     return_dbias=True)
+        slopes = torch.from_numpy(alibi_slope_gradient(dS2))
+        dist.all_reduce(table)
+        dist.all_reduce(slopes)
+        out[rank] = (table.numpy(), slopes.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bias_gradients_of_batch_shards_sum_to_the_full_batch():
+    import numpy as np
+
+    from oracle import alibi_slope_gradient, attention_backward, t5_table_gradient
+    from scaled_dot_product_bwd_b200.inputs import make_inputs
+    world = 2
+    mgr = mp.Manager()
+    out = mgr.dict()
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_grad_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert [p.exitcode for p in procs] == [0, 0]
+    full = make_inputs(2 * world, 24, 2, 1, 8, seed=5, t5_buckets=8, alibi=True)
+    args = (full.q, full.k, full.v, full.do)
+    *_, dS = attention_backward(*args, causal=True, t5_table=full.t5_table, t5_num_buckets=8,
+                                t5_max_distance=12, return_dbias=True)
+    *_, dS2 = attention_backward(*args, causal=True, alibi_slopes=full.alibi_slopes,
+                                 return_dbias=True)
+    want_table = t5_table_gradient(dS, 8, 12, True)
+    want_slopes = alibi_slope_gradient(dS2)
+    for r in range(world):
+        assert np.allclose(out[r][0], want_table, atol=1e-12)
+        assert np.allclose(out[r][1], want_slopes, atol=1e-10)

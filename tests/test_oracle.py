@@ -369,6 +369,23 @@ def test_t5_table_gradient_central_differences(bidirectional, causal):
     assert np.allclose(g.sum(axis=0), 0.0, atol=1e-12)
 
 
+@pytest.mark.parametrize("bidirectional", [True, False])
+def test_every_t5_bucket_is_one_range_of_distances(bidirectional):
+    # The T5 table gradient adds up per-diagonal sums over one contiguous
+    # range of r = j - i per bucket; that needs the bucket to be monotone in
+    # |r| on each side of 0 with disjoint ids across the sides.
+    L = 3000
+    r = np.arange(-(L - 1), L)
+    for nb in (4, 8, 16, 32, 64, 128):
+        for md in (nb, 2 * nb, 128, 1000, 5000):
+            if md <= (nb // 2 if bidirectional else nb) // 2:
+                continue
+            b = t5_relative_bucket(r, nb, md, bidirectional)
+            for k in np.unique(b):
+                idx = np.nonzero(b == k)[0]
+                assert idx[-1] - idx[0] + 1 == idx.size, (nb, md, k)
+
+
 # ---------------------------------------------------------------- ALiBi
 def test_alibi_zero_slopes_is_no_bias():
     q, k, v, do = qkv(1, 9, 2, 1, 4, seed=41)
