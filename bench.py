@@ -43,6 +43,9 @@ CONFIGS = {
     # the Mistral GQA shape with an in-kernel ALiBi bias (slopes 2^(-8 (h+1) / 32))
     "alibi_causal_4k": dict(B=4, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=-1, wr=-1,
                             bias="alibi"),
+    # the t5rpe shape at batch 4: the case the bias-gradient ncu capture runs
+    # on (its fp32 dS, 200 MB, still larger than L2)
+    "t5rpe_small": dict(B=4, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="t5"),
     # the mistral4k shape at batch 2: the case the ncu captures run on (inputs
     # still larger than L2, a few hundred MB on the device)
     "mistral4k_small": dict(B=2, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1,
@@ -64,6 +67,28 @@ NCU_TRAFFIC = {
     ("mistral4k", "fwd"): dict(bytes_per_batch=(100_843_008 + 34_080_000) / 2,
                                source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
 }
+
+
+# DRAM bytes the T5 table gradient adds to one backward, per batch entry:
+# (dQ kernel with dS output - plain dQ kernel) + diagonal sums + piece fold +
+# bucket sums, each as dram__bytes.sum.per_second x gpu__time_duration of one
+# launch from one ncu capture of
+#   python bench.py --config t5rpe_small --bias-grad --steps 1 --warmup 1
+# under ncu --section SpeedOfLight --section MemoryWorkloadAnalysis
+#   -k regex:"bwd_dq_kernel|t5_" -c 6 (batch 4).
+BIAS_GRAD_TRAFFIC = {
+    "t5rpe": dict(bytes_per_batch=90_910_618,
+                  source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
+}
+
+
+def bias_grad_traffic(config_name, batch):
+    """ncu DRAM bytes the bias gradient adds to one step of this workload, else None."""
+    from scaled_dot_product_bwd_b200.build import source_hash
+    rec = BIAS_GRAD_TRAFFIC.get(config_name.replace("_small", ""))
+    if rec is None or rec["source_hash"] != source_hash():
+        return None
+    return int(round(rec["bytes_per_batch"] * batch))
 
 
 def traffic_per_launch(config_name, kernel, batch):
@@ -524,7 +549,7 @@ def run_bias_grad(args, c):
                      "achieved": None if ach is None else round(ach, 1),
                      "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": None if ach is None else round(ach / peaks["hbm"], 4),
-                     "traffic": None, "bytes_per_step": extra,
+                     "traffic": bias_grad_traffic(args.config, c["B"]), "bytes_per_step": extra,
                      "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json)"
                      if peaks["source"] == "measured" else "fallback 6.65 TB/s"},
         "gpu_launches": None,
