@@ -52,6 +52,12 @@ What it computes, and where each piece comes from:
   head h (chain rule through the table lookup).  The pages name a learnable
   relative-position bias for training (catie-aq/flashT5 README, "T5-like
   relative position encoding biases") but print no gradient.
+* Cross-attention (a query sequence attending to a key/value sequence of
+  another length, as in T5's encoder-decoder): the same definition with
+  K, V of Lk rows.  The pages do not say how positions of the two
+  sequences line up; the oracle counts both from 0, so masks and
+  relative-position biases read the absolute indices i and j.  (T5's own
+  cross-attention uses neither a causal mask nor a position bias.)
 * LSE is the natural-log log-sum-exp of each score row (bias included); a row
   with no visible key has LSE = -inf, output 0 and zero gradients.
 """
@@ -145,20 +151,21 @@ def _as64(x):
 
 
 def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
-                 t5_max_distance, t5_bidirectional, alibi_slopes=None):
-    """Additive bias for one (batch, query head), [L, L] float64 (or 0)."""
+                 t5_max_distance, t5_bidirectional, alibi_slopes=None, Lk=None):
+    """Additive bias for one (batch, query head), [L, Lk] float64 (or 0)."""
+    Lk = L if Lk is None else Lk
     out = 0.0
     if alibi_slopes is not None:
         i = np.arange(L)[:, None]
-        j = np.arange(L)[None, :]
+        j = np.arange(Lk)[None, :]
         out = out - alibi_slopes[hq] * np.abs(j - i)
     if bias is not None:
         # a bias row of extent 1 is broadcast over the query rows
         out = out + np.broadcast_to(
-            bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0], (L, L))
+            bias[b if bias.shape[0] > 1 else 0, hq if bias.shape[1] > 1 else 0], (L, Lk))
     if t5_table is not None:
         i = np.arange(L)[:, None]
-        j = np.arange(L)[None, :]
+        j = np.arange(Lk)[None, :]
         bucket = t5_relative_bucket(j - i, t5_num_buckets, t5_max_distance, t5_bidirectional)
         out = out + t5_table[bucket, hq]
     return out
@@ -169,17 +176,19 @@ def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
                 t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None,
                 rows=None):
     """Masked score matrix S for one (b, hq): scale * Q K^T + bias, -inf where
-    masked.  q: [B, L, Hq, d], k: [B, L, Hkv, d] float64 arrays.  With
+    masked.  q: [B, L, Hq, d], k: [B, Lk, Hkv, d] float64 arrays (Lk = L for
+    self-attention; positions of both sequences count from 0).  With
     ``rows`` (an index array), only those query rows of S are formed."""
     B, L, Hq, d = q.shape
+    Lk = k.shape[1]
     Hkv = k.shape[2]
     g = hq // (Hq // Hkv)
     r = np.arange(L) if rows is None else np.asarray(rows)
     S = scale * (q[b, r, hq, :] @ k[b, :, g, :].T)
     S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets,
-                         t5_max_distance, t5_bidirectional, alibi_slopes)[r] \
+                         t5_max_distance, t5_bidirectional, alibi_slopes, Lk)[r] \
         if (bias is not None or t5_table is not None or alibi_slopes is not None) else S
-    M = visibility_mask(L, causal, window_left, window_right)[r]
+    M = visibility_mask(L, causal, window_left, window_right, Lk)[r]
     S = np.where(M, S, -np.inf)
     return S
 
@@ -226,7 +235,8 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
                       kv_heads=None, query_rows=None):
     """O = softmax(scale Q K^T + bias, masked) V and LSE, in float64.
 
-    q: [B, L, Hq, d]; k, v: [B, L, Hkv, d]; bias: [B|1, Hq|1, L, L] or None;
+    q: [B, L, Hq, d]; k, v: [B, Lk, Hkv, d] (Lk = L for self-attention);
+    bias: [B|1, Hq|1, L|1, Lk] or None;
     t5_table: [num_buckets, Hq] or None; alibi_slopes: [Hq] or None.
     Returns O [B, L, Hq, d] and
     LSE [B, Hq, L]; when ``batches`` / ``kv_heads`` restrict the work to a
@@ -264,8 +274,8 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
                        kv_heads=None, return_dbias=False):
     """Gradients of sum(O * dO) with respect to Q, K, V (float64).
 
-    Returns dQ [B, L, Hq, d], dK and dV [B, L, Hkv, d] (and, with
-    ``return_dbias``, dS per head as [B, Hq, L, L], the gradient of a dense
+    Returns dQ [B, L, Hq, d], dK and dV [B, Lk, Hkv, d] (and, with
+    ``return_dbias``, dS per head as [B, Hq, L, Lk], the gradient of a dense
     additive bias).  Subset selection as in ``attention_forward``.
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
@@ -277,7 +287,7 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     dQ = np.full(q.shape, np.nan)
     dK = np.full(k.shape, np.nan)
     dV = np.full(v.shape, np.nan)
-    dB = np.full((B, Hq, L, L), np.nan) if return_dbias else None
+    dB = np.full((B, Hq, L, k.shape[1]), np.nan) if return_dbias else None
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
               t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional,

@@ -447,6 +447,76 @@ def test_alibi_slope_gradient_central_differences(causal):
         assert abs(num - gx[idx]) < 1e-7
 
 
+# ------------------------------------------------- cross-attention (Lk != L)
+def test_cross_attention_single_query_brute_force():
+    # one query row over 7 keys of another sequence, summed term by term
+    rng = np.random.default_rng(61)
+    q = rng.standard_normal((1, 1, 2, 3))
+    k = rng.standard_normal((1, 7, 1, 3))
+    v = rng.standard_normal((1, 7, 1, 4))
+    bias = rng.standard_normal((1, 2, 1, 7))
+    O, lse = attention_forward(q, k, v, bias=bias)
+    for h in range(2):
+        s = [sum(q[0, 0, h, c] * k[0, j, 0, c] for c in range(3)) / math.sqrt(3)
+             + bias[0, h, 0, j] for j in range(7)]
+        w = [math.exp(x) for x in s]
+        z = sum(w)
+        assert abs(lse[0, h, 0] - math.log(z)) < 1e-12
+        for c in range(4):
+            assert abs(O[0, 0, h, c] - sum(w[j] * v[0, j, 0, c] for j in range(7)) / z) < 1e-12
+
+
+def test_cross_attention_key_permutation():
+    # permuting keys, values and the bias's key axis together leaves O and
+    # LSE unchanged; a bias read along the wrong axis would not follow
+    rng = np.random.default_rng(67)
+    q = rng.standard_normal((2, 5, 2, 4))
+    k = rng.standard_normal((2, 9, 1, 4))
+    v = rng.standard_normal((2, 9, 1, 4))
+    bias = rng.standard_normal((2, 2, 5, 9))
+    perm = rng.permutation(9)
+    O, lse = attention_forward(q, k, v, bias=bias)
+    Op, lsep = attention_forward(q, k[:, perm], v[:, perm], bias=bias[..., perm])
+    assert np.allclose(O, Op, atol=1e-12) and np.allclose(lse, lsep, atol=1e-12)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(bias="dense"), dict(t5="t5"),
+                                dict(window_left=2, window_right=3)])
+def test_cross_attention_gradients_central_differences(kw):
+    B, Lq, Lk, Hq, Hkv, d = 1, 4, 7, 2, 1, 3
+    rng = np.random.default_rng(71)
+    q = rng.standard_normal((B, Lq, Hq, d))
+    k = rng.standard_normal((B, Lk, Hkv, d))
+    v = rng.standard_normal((B, Lk, Hkv, d))
+    do = rng.standard_normal((B, Lq, Hq, d))
+    kw = dict(kw)
+    if kw.pop("bias", None):
+        kw["bias"] = rng.standard_normal((B, Hq, Lq, Lk))
+    if kw.pop("t5", None):
+        kw.update(t5_table=rng.standard_normal((8, Hq)), t5_num_buckets=8, t5_max_distance=6)
+    dq, dk, dv, dS = attention_backward(q, k, v, do, return_dbias=True, **kw)
+    assert dq.shape == q.shape and dk.shape == k.shape and dS.shape == (B, Hq, Lq, Lk)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            argm = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (_loss(*args, do, kw) - _loss(*argm, do, kw)) / (2 * h)
+        assert np.max(np.abs(num - g)) < 1e-6 * max(1.0, np.max(np.abs(g))), name
+    if "bias" in kw:
+        for idx in ((0, 0, 1, 5), (0, 1, 3, 0)):
+            bp = kw["bias"].copy(); bp[idx] += h
+            bm = kw["bias"].copy(); bm[idx] -= h
+            num = (_loss(q, k, v, do, {**kw, "bias": bp})
+                   - _loss(q, k, v, do, {**kw, "bias": bm})) / (2 * h)
+            assert abs(num - dS[idx]) < 1e-7
+
+
 def test_D_two_ways():
     # rowsum(P * dP) = rowsum(dO * O) for every row.
     q, k, v, do = qkv()
