@@ -463,6 +463,20 @@ def bias_grad_extra_bytes(c):
     return ds                      # a full-shape dense bias: dS goes straight out
 
 
+def bias_grad_launches(c):
+    """Kernels one timed step of the bias-gradient leg launches: the forward,
+    preprocess, dQ (with dS output) and dK/dV, the zero fill of skipped key
+    tiles under a mask, and the reductions (T5 / ALiBi: diagonal sums, their
+    fold and the per-bucket or per-slope sums; a full-shape dense bias needs
+    none)."""
+    n = 4
+    if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
+        n += 1
+    if c["bias"] in ("t5", "alibi"):
+        n += 3
+    return n
+
+
 def run_bias_grad(args, c):
     import torch
 
@@ -552,7 +566,7 @@ def run_bias_grad(args, c):
                      "traffic": bias_grad_traffic(args.config, c["B"]), "bytes_per_step": extra,
                      "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json)"
                      if peaks["source"] == "measured" else "fallback 6.65 TB/s"},
-        "gpu_launches": None,
+        "gpu_launches": args.steps * bias_grad_launches(c),
         "clocks": res[True]["clocks"],
         "device_status": status,
     }
