@@ -35,6 +35,14 @@
  *   bounded: a wait that runs out records SDPA_ERR_TIMEOUT in a per-device
  *   status word (read with sdpa_read_device_status) and the kernel returns
  *   instead of hanging.
+ * Accuracy.  bf16 inputs and outputs with float32 accumulation.  Against an
+ *   exact (float64) evaluation, O, dQ, dK and dV are within
+ *   1e-2 + 1e-2 |ref| element-wise and LSE within 1e-3 for N(0, 1) inputs at
+ *   scales up to 1 / sqrt(d) (and at smaller or negative scales).  Larger
+ *   scales -- T5's historical scale 1, say -- make the softmax peaked, and
+ *   the bf16 rounding of dS (the operand of the dQ and dK products) and of
+ *   the stored O (in D = rowsum(dO * O)) can then exceed that bound on a few
+ *   gradient entries where large terms cancel.
  * Determinism.  Results are bit-identical run to run for identical inputs
  *   and launch configuration: every reduction is in a fixed order and no
  *   floating-point atomics are used (HF transformers issue #31787,
@@ -199,6 +207,10 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
  *    keeps the contents of the last call (nothing in it needs to start at
  *    zero: each call writes the rows it reads).  Calls whose executions
  *    overlap on the GPU race on it; order them on one stream or with events.
+ *  - The looked-up address is cached per device for the life of the
+ *    process; it does not survive cudaDeviceReset (or any other teardown of
+ *    the device's primary context), after which this entry point must not
+ *    be called again in that process.
  *  - Calls no allocating routine (no cudaMalloc / cudaFree).
  */
 #define SDPA_NOALLOC_MAX_ROWS (1u << 20)

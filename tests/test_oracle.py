@@ -50,18 +50,47 @@ def test_t5_buckets_integer_thresholds():
     assert np.array_equal(t5_relative_bucket(n, 32, 128, True), want_pos)
 
 
-def test_t5_buckets_unidirectional_brute_force():
-    # Decoder form: n = max(i - j, 0); 32 buckets, max_exact 16; keys after
-    # the query all land in bucket 0.
-    rel = np.arange(-400, 401)
-    got = t5_relative_bucket(rel, 32, 128, False)
-    for r, b in zip(rel, got):
-        n = max(-r, 0)
-        if n < 16:
-            exp = n
-        else:
-            exp = min(16 + int(math.log(n / 16) / math.log(128 / 16) * 16), 31)
-        assert b == exp, (r, b, exp)
+def _golden_sections(name):
+    """{(num_buckets, max_distance, bidirectional): (rel, bucket)} of a golden file."""
+    out, cur = {}, None
+    for line in open(os.path.join(GOLDEN, name)):
+        f = line.split()
+        if not f or f[0].startswith("#"):
+            continue
+        if f[0] == "config":
+            cur = (int(f[1]), int(f[2]), bool(int(f[3])))
+            out[cur] = ([], [])
+            continue
+        out[cur][0].append(int(f[0]))
+        out[cur][1].append(int(f[1]))
+    return out
+
+
+def test_t5_buckets_other_settings_hand_worked():
+    # The decoder (unidirectional) form and the non-default bucket settings
+    # the GPU bucket test uses, against thresholds solved by hand: both sides
+    # of every threshold of the 32-bucket decoder table, keys after the query
+    # (bucket 0), the caps, and the exact-tie distances 32, 64, 128 of the
+    # (64, 256) table.
+    secs = _golden_sections("t5_buckets_more.txt")
+    assert set(secs) == {(32, 128, False), (16, 40, True), (64, 256, True), (8, 20, True),
+                         (128, 1000, False)}
+    for (nb, md, bidir), (rel, want) in secs.items():
+        got = t5_relative_bucket(np.array(rel), nb, md, bidir)
+        assert np.array_equal(got, np.array(want)), \
+            [(r, g, w) for r, g, w in zip(rel, got, want) if g != w]
+
+
+def test_t5_buckets_decoder_thresholds_every_distance():
+    # 32 decoder buckets: the hand-solved first distance of each log bucket
+    # (16 * 8^(k/16) rounded up), checked for every n in [0, 5000]; every key
+    # after the query is bucket 0.
+    thr = [16, 19, 21, 24, 27, 31, 35, 40, 46, 52, 59, 67, 77, 87, 99, 113]
+    n = np.arange(0, 5001)
+    want = np.where(n < 16, n, 15 + np.searchsorted(thr, n, side="right"))
+    want = np.minimum(want, 31)
+    assert np.array_equal(t5_relative_bucket(-n, 32, 128, False), want)
+    assert (t5_relative_bucket(np.arange(1, 3000), 32, 128, False) == 0).all()
 
 
 # ---------------------------------------------------------------- masks

@@ -19,20 +19,29 @@ from scaled_dot_product_bwd_b200.inputs import make_inputs
 pytestmark = pytest.mark.gpu
 
 
-def _close(a, b):
-    a = a.float().cpu().numpy()
-    b = b.float().cpu().numpy()
-    assert np.all(np.abs(a - b) <= ATOL + RTOL * np.abs(b))
+def _same(got, ref, name):
+    """Bit-identical: both entry points run the same kernels on the same inputs,
+    so any difference means the scratch array fed a kernel stale or foreign
+    data.  The tolerance figure is only there to describe a mismatch."""
+    if torch.equal(got, ref):
+        return
+    a = got.float().cpu().numpy()
+    b = ref.float().cpu().numpy()
+    within = bool(np.all(np.abs(a - b) <= ATOL + RTOL * np.abs(b)))
+    raise AssertionError(f"{name}: not bit-identical to sdpa_bwd "
+                         f"(max |diff| {np.nanmax(np.abs(a - b)):.3e}, "
+                         f"{'within' if within else 'outside'} the oracle tolerance)")
 
 
 @pytest.mark.parametrize("kw", [dict(causal=True), dict(causal=False, t5=True)])
 def test_noalloc_matches_workspace_entry_point_twice(kw):
     dev = torch.device("cuda")
-    t5 = kw.pop("t5", False)
+    t5 = kw.get("t5", False)
+    mask = {n: v for n, v in kw.items() if n != "t5"}
     for call, seed in enumerate((1, 2)):   # two calls in a row, different inputs
         inp = make_inputs(2, 300, 4, 2, 128, seed=seed, t5_buckets=32 if t5 else 0)
         q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
-        extra = dict(kw)
+        extra = dict(mask)
         if t5:
             extra["t5_table"] = inp.t5_table.to(dev)
         o, lse = sdpa_fwd(q, k, v, **extra)
@@ -41,8 +50,8 @@ def test_noalloc_matches_workspace_entry_point_twice(kw):
                torch.full_like(v, float("nan")))
         got = sdpa_bwd_noalloc(q, k, v, o, do, lse, *out, **extra)
         torch.cuda.synchronize()
-        for g, r in zip(got, ref):
-            _close(g, r)
+        for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+            _same(g, r, f"call {call + 1} {name}")
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
