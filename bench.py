@@ -58,14 +58,6 @@ CONFIGS = {
 # on.  A bench workload of the same shape reports them scaled to its batch, and
 # only while the library is built from exactly those sources.
 NCU_TRAFFIC = {
-    # python bench.py --config mistral4k_small --steps 1 --warmup 1 --no-cpu-baseline
-    # under ncu --set full -k regex:<kernel> -s 1 -c 1 (batch 2)
-    ("mistral4k", "bwd_dkdv"): dict(bytes_per_batch=(170_241_024 + 22_872_064) / 2,
-                                    source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
-    ("mistral4k", "bwd_dq"): dict(bytes_per_batch=(171_017_728 + 43_307_776) / 2,
-                                  source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
-    ("mistral4k", "fwd"): dict(bytes_per_batch=(100_843_008 + 34_080_000) / 2,
-                               source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
 }
 
 
@@ -77,8 +69,6 @@ NCU_TRAFFIC = {
 # under ncu --section SpeedOfLight --section MemoryWorkloadAnalysis
 #   -k regex:"bwd_dq_kernel|t5_" -c 6 (batch 4).
 BIAS_GRAD_TRAFFIC = {
-    "t5rpe": dict(bytes_per_batch=90_910_618,
-                  source_hash="bc6170e958f452a05a70084f376dabe8297ab051168e9b45562fe1479a2739df"),
 }
 
 
@@ -125,8 +115,7 @@ def flop_counts(c):
     P = visible_pairs(c["L"], c["causal"], c["wl"], c["wr"])
     heads = c["B"] * c["Hq"]
     d = c["d"]
-    return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads,
-                dkdv=8 * d * P * heads, dq=2 * d * P * heads)
+    return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads)
 
 
 def load_peaks():
@@ -270,7 +259,7 @@ def run_gpu(args, c):
     import torch
     import torch.distributed as dist
 
-    from scaled_dot_product_bwd_b200 import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, load_library,
+    from scaled_dot_product_bwd_b200 import (BWD_GRADS, BWD_PREPROCESS, load_library,
                                              sdpa_bwd, sdpa_bwd_workspace_size, sdpa_fwd,
                                              sdpa_read_device_status)
 
@@ -308,12 +297,9 @@ def run_gpu(args, c):
                  phases=BWD_PREPROCESS, **kw)
         if ev is not None:
             ev[2].record(stream)
-        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DQ, **kw)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_GRADS, **kw)
         if ev is not None:
             ev[3].record(stream)
-        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DKDV, **kw)
-        if ev is not None:
-            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -322,7 +308,7 @@ def run_gpu(args, c):
         raise RuntimeError("device status reports a timed-out wait during warm-up")
 
     # ---------------- timed region: K steps, device-timed, max over ranks
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -338,7 +324,7 @@ def run_gpu(args, c):
         dist.barrier()
     clocks = sampler.stop()
     ms_total = start.elapsed_time(end)
-    phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(4)]
+    phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(3)]
     ms_total = max_over_ranks(ms_total, dev)
     status = sdpa_read_device_status()
 
@@ -403,9 +389,9 @@ def run_gpu(args, c):
     peaks = load_peaks()
 
     # dominant kernel by mean duration; its algorithmic FLOPs per launch
-    names = ["fwd", "bwd_preprocess", "bwd_dq", "bwd_dkdv"]
-    algo = {"fwd": fl["fwd"], "bwd_dq": fl["dq"], "bwd_dkdv": fl["dkdv"]}
-    dom = max(range(4), key=lambda i: phase_ms[i])
+    names = ["fwd", "bwd_preprocess", "bwd"]
+    algo = {"fwd": fl["fwd"], "bwd": fl["bwd"]}
+    dom = max(range(3), key=lambda i: phase_ms[i])
     dname = names[dom]
     roofline = None
     if dname in algo:
@@ -435,7 +421,7 @@ def run_gpu(args, c):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3),
                 "pipelining": "3 streams, 2 device buffer sets: H2D(s+1) | compute(s) | D2H(s-1)"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks,
         "device_status": status,
     }
@@ -465,11 +451,11 @@ def bias_grad_extra_bytes(c):
 
 def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
-    preprocess, dQ (with dS output) and dK/dV, the zero fill of skipped key
-    tiles under a mask, and the reductions (T5 / ALiBi: diagonal sums, their
-    fold and the per-bucket or per-slope sums; a full-shape dense bias needs
-    none)."""
-    n = 4
+    preprocess and the backward kernel (with dS output), the zero fill of
+    skipped key tiles under a mask, and the reductions (T5 / ALiBi: diagonal
+    sums, their fold and the per-bucket or per-slope sums; a full-shape dense
+    bias needs none)."""
+    n = 3
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1
     if c["bias"] in ("t5", "alibi"):

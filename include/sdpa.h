@@ -14,12 +14,18 @@
  * Layout.  Q, K, V, O, dO, dQ, dK, dV are bf16 tensors in (batch, sequence,
  *   head, head_dim) order -- the (B, T, N, H) layout of the codelab, section
  *   3 -- given by element strides; head_dim is contiguous.  Q, O, dO and dQ
- *   share the strides sq_*, K, V, dK and dV share skv_*.  Query and key
- *   sequences have the same length L.  LSE is float32 [B, Hq, L], contiguous.
+ *   share the strides sq_*, K, V, dK and dV share skv_*.  Queries have L rows,
+ *   keys and values Lk (Lk = L for self-attention; cross-attention, as in a
+ *   T5 decoder attending to its encoder, may differ).  Positions of both
+ *   sequences count from 0: the causal and window masks and the relative-
+ *   position biases compare the query index i with the key index j as they
+ *   are.  LSE is float32 [B, Hq, L], contiguous.  Packed variable-length
+ *   batches (sdpa_fwd_varlen / sdpa_bwd_varlen) lay the sequences end to end
+ *   along one sequence axis instead, described by sdpa_varlen.
  * Heads.  Hq query heads share Hkv key/value heads in contiguous groups:
  *   query head h reads KV head h / (Hq / Hkv) (MHA Hkv = Hq, GQA, MQA
  *   Hkv = 1; codelab section 9).  Hq % Hkv must be 0.
- * Supported.  head_dim d in {64, 128}; 1 <= L < 2^30; B, Hq <= 65535;
+ * Supported.  head_dim d in {64, 128}; 1 <= L, Lk < 2^30; B, Hq <= 65535;
  *   ceil(L / 128) * Hq * B < 2^31 (query tiles are counted in 32 bits);
  *   every bf16 base pointer 16-byte aligned; every stride a multiple of 8
  *   elements (16 bytes) except the contiguous head_dim.  Anything else returns SDPA_ERR_UNSUPPORTED or
@@ -127,7 +133,36 @@ typedef struct sdpa_shape {
   int64_t B, L, Hq, Hkv, d;
   int64_t sq_b, sq_l, sq_h;    /* element strides of Q, O, dO, dQ */
   int64_t skv_b, skv_l, skv_h; /* element strides of K, V, dK, dV */
+  int64_t Lk;                  /* key / value length; 0 = L */
 } sdpa_shape;
+
+/*
+ * Packed variable-length sequences (HF transformers issue #30461: the Mistral
+ * fine-tune packs its examples, `packing=True`; catie-aq/flashT5 README:
+ * dynamic batching to cut padding).  Batch entry b owns query rows
+ * [cu_seqlens_q[b], cu_seqlens_q[b + 1]) and key rows [cu_seqlens_k[b],
+ * cu_seqlens_k[b + 1]) of one shared sequence axis; its positions count from
+ * 0 at its first row and no query attends to another entry's keys.
+ *   cu_seqlens_q, cu_seqlens_k: device int32 [B + 1], non-decreasing, first
+ *     entry 0, last entry total_q / total_k, read by the kernels (entries
+ *     that leave [0, total] or give a sequence longer than max_seqlen make
+ *     that entry empty and are reported by sdpa_read_device_status as
+ *     SDPA_ERR_UNSUPPORTED).
+ *   max_seqlen_q / max_seqlen_k: upper bounds of the lengths (>= 1).
+ *   total_q / total_k: rows of the packed axes (>= 1, < 2^30).
+ * With a packed batch the shape's B is the number of sequences, its L and Lk
+ * and batch strides sq_b / skv_b are ignored: Q, O, dO, dQ are
+ * [total_q, Hq, d] with strides sq_l, sq_h, K, V, dK, dV [total_k, Hkv, d]
+ * with skv_l, skv_h, and LSE is float32 [Hq, total_q].  Dense biases have no
+ * packed form (SDPA_ERR_UNSUPPORTED); T5 and ALiBi biases are relative
+ * positions within each sequence.
+ */
+typedef struct sdpa_varlen {
+  const int32_t* cu_seqlens_q;
+  const int32_t* cu_seqlens_k;
+  int64_t max_seqlen_q, max_seqlen_k;
+  int64_t total_q, total_k;
+} sdpa_varlen;
 
 /*
  * Forward.  Writes O (bf16, Q's layout) and LSE[b, h, i] = natural-log
@@ -140,12 +175,21 @@ sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k,
                        const sdpa_mask_spec* mask, float scale, void* o,
                        float* lse, void* stream);
 
+/* Forward of a packed variable-length batch (see sdpa_varlen). */
+sdpa_status_t sdpa_fwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen,
+                              const void* q, const void* k, const void* v,
+                              const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
+                              float scale, void* o, float* lse, void* stream);
+
 /*
- * Bytes of device workspace sdpa_bwd needs for this shape (the per-row
- * D_i = sum_c dO[i,c] O[i,c] vector, float32 [B, Hq, L], plus alignment).
- * Returns 0 for an invalid shape.
+ * Bytes of device workspace sdpa_bwd needs for this shape: the per-row
+ * D_i = sum_c dO[i,c] O[i,c] vector (float32, one per LSE entry), the dQ
+ * turn counters (4 bytes per 32 query rows of each head), and the float32
+ * dQ accumulator (d floats per LSE entry), each 256-byte aligned.  Returns 0
+ * for an invalid shape.
  */
 size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic);
+size_t sdpa_bwd_varlen_workspace_size(const sdpa_shape* shape, const sdpa_varlen* varlen);
 
 /*
  * Backward.  Given Q, K, V, the forward output O and its LSE, and the
@@ -154,6 +198,13 @@ size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic);
  * print no gradient formulas; these are the chain rule of the forward:
  *   P = exp(S - LSE), dP = dO V^T, D_i = rowsum(dO * O), dS = P (dP - D),
  *   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+ * One kernel computes all three: for each block of 128 keys it walks the
+ * query tiles of the mask band and keeps dK and dV on chip; every dQ
+ * partial is added into the workspace's float32 accumulator in ascending
+ * key-tile order, gated by a turn counter per 32 query rows (a fixed-order
+ * split-K sum, no floating-point atomics; HF transformers issue #31787 is
+ * the non-determinism this avoids).  The waits for a turn are bounded like
+ * every other in-kernel wait.
  * deterministic: must be 1 (the only mode built; 0 returns UNSUPPORTED).
  * workspace: device memory of at least sdpa_bwd_workspace_size() bytes,
  * 256-byte aligned, owned by the caller, contents ignored on entry.
@@ -166,21 +217,28 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The backward as its three launches, selected by a bitmask: PREPROCESS
- * writes D = rowsum(dO * O) into the workspace; DQ writes dQ; DKDV writes dK
- * and dV.  DQ and DKDV read D from the workspace, so PREPROCESS must have run
- * on the same workspace earlier in stream order; DQ and DKDV are independent
- * of each other and may run on different streams.  sdpa_bwd is
- * sdpa_bwd_phases(SDPA_BWD_ALL, ...).  Arguments as sdpa_bwd; phases == 0 or
- * unknown bits -> SDPA_ERR_INVALID_ARG.
+ * The backward as its two launches, selected by a bitmask: PREPROCESS
+ * writes D = rowsum(dO * O) into the workspace and clears its counters;
+ * GRADS writes dQ, dK and dV and needs a PREPROCESS on the same workspace
+ * earlier in stream order (once per GRADS launch: the counters it clears are
+ * used up).  sdpa_bwd is sdpa_bwd_phases(SDPA_BWD_ALL, ...).  Arguments as
+ * sdpa_bwd; phases == 0 or unknown bits -> SDPA_ERR_INVALID_ARG.
  */
 #define SDPA_BWD_PREPROCESS 1u
-#define SDPA_BWD_DQ 2u
-#define SDPA_BWD_DKDV 4u
-#define SDPA_BWD_ALL 7u
+#define SDPA_BWD_GRADS 2u
+#define SDPA_BWD_ALL 3u
 sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const void* q,
                               const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, const sdpa_bias_desc* bias,
+                              const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                              void* dv, int32_t deterministic, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Backward of a packed variable-length batch (see sdpa_varlen); workspace of
+ * at least sdpa_bwd_varlen_workspace_size() bytes. */
+sdpa_status_t sdpa_bwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen,
+                              const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, const sdpa_bias_desc* bias,
                               const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
                               void* dv, int32_t deterministic, void* workspace,
                               size_t workspace_bytes, void* stream);
@@ -195,17 +253,18 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
  * latency-bound loops that avoid cudaMalloc / cudaFree because those calls
  * can synchronise the device and stall other streams.
  *
- * Same arguments and results as sdpa_bwd minus the workspace: the D vector
- * lives in a fixed array of SDPA_NOALLOC_MAX_ROWS floats (4 MiB) compiled
- * into the library, held by every GPU that loads it until the process exits.
- *  - B * Hq * L must be <= SDPA_NOALLOC_MAX_ROWS, else SDPA_ERR_WORKSPACE
- *    (nothing is launched).
+ * Same arguments and results as sdpa_bwd minus the workspace: the workspace
+ * lives in a fixed array of SDPA_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into
+ * the library, held by every GPU that loads it until the process exits.
+ *  - sdpa_bwd_workspace_size(shape) must be <= SDPA_NOALLOC_SCRATCH_BYTES
+ *    (about B * Hq * L * (d + 1) * 4 bytes: B * Hq * L up to 32512 at
+ *    d = 128), else SDPA_ERR_WORKSPACE (nothing is launched).
  *  - The first call on a device looks up the array's device address with
  *    that device current (once per device); make that first call before
  *    any stream capture on the device.  A failed lookup -> SDPA_ERR_CUDA.
  *  - Every call, on every stream of a device, shares the one array, which
- *    keeps the contents of the last call (nothing in it needs to start at
- *    zero: each call writes the rows it reads).  Calls whose executions
+ *    keeps the contents of the last call (each call clears the counters it
+ *    uses and writes every other entry before reading it).  Calls whose executions
  *    overlap on the GPU race on it; order them on one stream or with events.
  *  - The looked-up address is cached per device for the life of the
  *    process; it does not survive cudaDeviceReset (or any other teardown of
@@ -213,7 +272,7 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
  *    be called again in that process.
  *  - Calls no allocating routine (no cudaMalloc / cudaFree).
  */
-#define SDPA_NOALLOC_MAX_ROWS (1u << 20)
+#define SDPA_NOALLOC_SCRATCH_BYTES (16u << 20)
 sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const void* k,
                                const void* v, const void* o, const void* dout,
                                const float* lse, const sdpa_bias_desc* bias,
@@ -295,6 +354,15 @@ void sdpa_set_wait_limit_ns(uint64_t ns);
  * afterwards.
  */
 sdpa_status_t sdpa_debug_wait_timeout(void* stream);
+
+/*
+ * Launches one warp that waits for a dQ turn that never comes: it polls the
+ * device word *counter (caller-owned, any value but 0xffffffff) for the value
+ * 0xffffffff under the current wait limit, the way the backward's reducer
+ * warps wait for their turn.  Expect sdpa_read_device_status() ==
+ * SDPA_ERR_TIMEOUT afterwards.
+ */
+sdpa_status_t sdpa_debug_turn_timeout(const uint32_t* counter, void* stream);
 
 /* Static English text for a status code. */
 const char* sdpa_status_string(sdpa_status_t status);

@@ -6,10 +6,14 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 from .sdpa_oracle import (  # noqa: F401
     alibi_slope_gradient,
     attention_backward,
+    attention_backward_packed,
     attention_forward,
+    attention_forward_packed,
     attention_probs,
     dense_bias_gradient,
     head_scores,
+    packed_positions,
+    packed_visibility_mask,
     t5_relative_bucket,
     t5_table_gradient,
     visibility_mask,

@@ -58,6 +58,16 @@ What it computes, and where each piece comes from:
   sequences line up; the oracle counts both from 0, so masks and
   relative-position biases read the absolute indices i and j.  (T5's own
   cross-attention uses neither a causal mask nor a position bias.)
+* Packed variable-length sequences (HF transformers issue #30461: the
+  reporter's fine-tune packs its examples, ``packing=True``; catie-aq/flashT5
+  README: dynamic batching to cut padding): the pages do not say how
+  attention treats the boundaries of packed examples.  The oracle's reading:
+  the sequences lie end to end on one axis, cut by cumulative lengths
+  ``cu_seqlens``; a query attends only to keys of its own sequence; positions
+  count from 0 at each sequence's first row, and the masks and relative-
+  position biases use those local positions.  ``attention_forward_packed``
+  and ``attention_backward_packed`` write this out over the whole packed
+  axis with one explicit block-diagonal mask.
 * LSE is the natural-log log-sum-exp of each score row (bias included); a row
   with no visible key has LSE = -inf, output 0 and zero gradients.
 """
@@ -77,6 +87,10 @@ __all__ = [
     "dense_bias_gradient",
     "t5_table_gradient",
     "alibi_slope_gradient",
+    "packed_positions",
+    "packed_visibility_mask",
+    "attention_forward_packed",
+    "attention_backward_packed",
 ]
 
 
@@ -357,3 +371,111 @@ def alibi_slope_gradient(dS):
     L, Lk = dS.shape[2], dS.shape[3]
     dist = np.abs(np.arange(Lk)[None, :] - np.arange(L)[:, None])
     return -np.einsum("bhij,ij->h", dS, dist)
+
+
+# --------------------------------------------------------------------------
+# Packed variable-length sequences (transformers issue #30461, packing=True;
+# catie-aq/flashT5 README, dynamic batching).
+# --------------------------------------------------------------------------
+def packed_positions(cu_seqlens):
+    """Sequence id and local position (from 0) of every row of a packed axis."""
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    total = cu[-1]
+    seq = np.empty(total, dtype=np.int64)
+    pos = np.empty(total, dtype=np.int64)
+    for b in range(len(cu) - 1):
+        seq[cu[b]:cu[b + 1]] = b
+        pos[cu[b]:cu[b + 1]] = np.arange(cu[b + 1] - cu[b])
+    return seq, pos
+
+
+def packed_visibility_mask(cu_seqlens_q, cu_seqlens_k, causal, window_left=-1,
+                           window_right=-1):
+    """Boolean [total_q, total_k]: packed query row r sees packed key row c
+    iff both belong to the same sequence and their local positions i, j
+    satisfy the mask (j <= i if causal, j >= i - window_left, j <= i +
+    window_right; negative bounds unbounded)."""
+    sq, i = packed_positions(cu_seqlens_q)
+    sk, j = packed_positions(cu_seqlens_k)
+    i = i[:, None]
+    j = j[None, :]
+    m = sq[:, None] == sk[None, :]
+    if causal:
+        m &= j <= i
+    if window_left is not None and window_left >= 0:
+        m &= j >= i - window_left
+    if window_right is not None and window_right >= 0:
+        m &= j <= i + window_right
+    return m
+
+
+def _packed_scores(q, k, hq, G, sc, M, rel, t5_table, t5_num_buckets, t5_max_distance,
+                   t5_bidirectional, alibi_slopes):
+    S = sc * (q[:, hq, :] @ k[:, hq // G, :].T)
+    if t5_table is not None:
+        S = S + t5_table[t5_relative_bucket(rel, t5_num_buckets, t5_max_distance,
+                                            t5_bidirectional), hq]
+    if alibi_slopes is not None:
+        S = S - alibi_slopes[hq] * np.abs(rel)
+    return np.where(M, S, -np.inf)
+
+
+def attention_forward_packed(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None,
+                             causal=False, window_left=-1, window_right=-1, t5_table=None,
+                             t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
+                             alibi_slopes=None):
+    """O [total_q, Hq, d] and LSE [Hq, total_q] of a packed batch: the
+    definition over the whole packed axis with the block-diagonal mask of
+    ``packed_visibility_mask`` and the relative position j - i of the local
+    positions.  q: [total_q, Hq, d]; k, v: [total_k, Hkv, d]."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    t5_table, alibi_slopes = _as64(t5_table), _as64(alibi_slopes)
+    Tq, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    sc = _scale_of(d, scale)
+    M = packed_visibility_mask(cu_seqlens_q, cu_seqlens_k, causal, window_left, window_right)
+    _, pi = packed_positions(cu_seqlens_q)
+    _, pj = packed_positions(cu_seqlens_k)
+    rel = pj[None, :] - pi[:, None]
+    O = np.zeros((Tq, Hq, v.shape[-1]))
+    LSE = np.zeros((Hq, Tq))
+    for hq in range(Hq):
+        S = _packed_scores(q, k, hq, G, sc, M, rel, t5_table, t5_num_buckets, t5_max_distance,
+                           t5_bidirectional, alibi_slopes)
+        P, lse = _softmax_rows(S)
+        O[:, hq, :] = P @ v[:, hq // G, :]
+        LSE[hq] = lse
+    return O, LSE
+
+
+def attention_backward_packed(q, k, v, do, cu_seqlens_q, cu_seqlens_k, *, scale=None,
+                              causal=False, window_left=-1, window_right=-1, t5_table=None,
+                              t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
+                              alibi_slopes=None):
+    """dQ [total_q, Hq, d], dK and dV [total_k, Hkv, d] of sum(O * dO) for a
+    packed batch, by the chain rule over the packed axis (as in
+    ``attention_backward``)."""
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    t5_table, alibi_slopes = _as64(t5_table), _as64(alibi_slopes)
+    Tq, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    sc = _scale_of(d, scale)
+    M = packed_visibility_mask(cu_seqlens_q, cu_seqlens_k, causal, window_left, window_right)
+    _, pi = packed_positions(cu_seqlens_q)
+    _, pj = packed_positions(cu_seqlens_k)
+    rel = pj[None, :] - pi[:, None]
+    dQ = np.zeros(q.shape)
+    dK = np.zeros(k.shape)
+    dV = np.zeros(v.shape)
+    for hq in range(Hq):
+        g = hq // G
+        S = _packed_scores(q, k, hq, G, sc, M, rel, t5_table, t5_num_buckets, t5_max_distance,
+                           t5_bidirectional, alibi_slopes)
+        P, _ = _softmax_rows(S)
+        dP = do[:, hq, :] @ v[:, g, :].T
+        Dv = np.sum(P * dP, axis=1)
+        dS = P * (dP - Dv[:, None])
+        dQ[:, hq, :] = sc * (dS @ k[:, g, :])
+        dK[:, g, :] += sc * (dS.T @ q[:, hq, :])
+        dV[:, g, :] += P.T @ do[:, hq, :]
+    return dQ, dK, dV

@@ -7,8 +7,7 @@ touch the GPU.
 """
 from .binding import (  # noqa: F401
     BWD_ALL,
-    BWD_DKDV,
-    BWD_DQ,
+    BWD_GRADS,
     BWD_PREPROCESS,
     EXPORTED,
     SdpaError,
@@ -17,10 +16,13 @@ from .binding import (  # noqa: F401
     sdpa_bwd_bias_grad,
     sdpa_bwd_bias_grad_workspace_size,
     sdpa_bwd_noalloc,
+    sdpa_bwd_varlen,
     sdpa_bwd_workspace_size,
+    sdpa_debug_turn_timeout,
     sdpa_debug_wait_timeout,
     sdpa_exp2_fma,
     sdpa_fwd,
+    sdpa_fwd_varlen,
     sdpa_read_device_status,
     sdpa_set_wait_limit_ns,
     sdpa_status_string,

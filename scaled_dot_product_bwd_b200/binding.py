@@ -22,15 +22,15 @@ STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTE
                 3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 BIAS_NONE, BIAS_DENSE, BIAS_T5, BIAS_ALIBI = 0, 1, 2, 3
 
-BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
+BWD_PREPROCESS, BWD_GRADS, BWD_ALL = 1, 2, 3
 
-NOALLOC_MAX_ROWS = 1 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
-EXPORTED = ("sdpa_fwd", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_noalloc",
-            "sdpa_bwd_workspace_size", "sdpa_bwd_bias_grad",
-            "sdpa_bwd_bias_grad_workspace_size", "sdpa_t5_bucket", "sdpa_exp2_fma",
-            "sdpa_read_device_status", "sdpa_set_wait_limit_ns", "sdpa_debug_wait_timeout",
-            "sdpa_status_string")
+EXPORTED = ("sdpa_fwd", "sdpa_fwd_varlen", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_bwd_varlen",
+            "sdpa_bwd_noalloc", "sdpa_bwd_workspace_size", "sdpa_bwd_varlen_workspace_size",
+            "sdpa_bwd_bias_grad", "sdpa_bwd_bias_grad_workspace_size", "sdpa_t5_bucket",
+            "sdpa_exp2_fma", "sdpa_read_device_status", "sdpa_set_wait_limit_ns",
+            "sdpa_debug_wait_timeout", "sdpa_debug_turn_timeout", "sdpa_status_string")
 
 
 class SdpaError(RuntimeError):
@@ -53,7 +53,14 @@ class BiasDesc(ctypes.Structure):
 
 class Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in
-                ("B", "L", "Hq", "Hkv", "d", "sq_b", "sq_l", "sq_h", "skv_b", "skv_l", "skv_h")]
+                ("B", "L", "Hq", "Hkv", "d", "sq_b", "sq_l", "sq_h", "skv_b", "skv_l", "skv_h",
+                 "Lk")]
+
+
+class Varlen(ctypes.Structure):
+    _fields_ = [("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+                ("max_seqlen_q", ctypes.c_int64), ("max_seqlen_k", ctypes.c_int64),
+                ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64)]
 
 
 _lib = None
@@ -71,10 +78,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                              ctypes.c_size_t)
     sp, bp, mp = ctypes.POINTER(Shape), ctypes.POINTER(BiasDesc), ctypes.POINTER(MaskSpec)
+    vlp = ctypes.POINTER(Varlen)
     lib.sdpa_fwd.argtypes = [sp, vp, vp, vp, bp, mp, f32, vp, vp, vp]
     lib.sdpa_fwd.restype = i32
+    lib.sdpa_fwd_varlen.argtypes = [sp, vlp, vp, vp, vp, bp, mp, f32, vp, vp, vp]
+    lib.sdpa_fwd_varlen.restype = i32
     lib.sdpa_bwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, i32, vp, sz, vp]
     lib.sdpa_bwd.restype = i32
+    lib.sdpa_bwd_varlen.argtypes = [sp, vlp] + lib.sdpa_bwd.argtypes[1:]
+    lib.sdpa_bwd_varlen.restype = i32
+    lib.sdpa_bwd_varlen_workspace_size.argtypes = [sp, vlp]
+    lib.sdpa_bwd_varlen_workspace_size.restype = sz
     lib.sdpa_bwd_phases.argtypes = [ctypes.c_uint32] + lib.sdpa_bwd.argtypes
     lib.sdpa_bwd_phases.restype = i32
     lib.sdpa_bwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, bp, mp, f32, vp, vp, vp, i32, vp]
@@ -96,6 +110,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_set_wait_limit_ns.restype = None
     lib.sdpa_debug_wait_timeout.argtypes = [vp]
     lib.sdpa_debug_wait_timeout.restype = i32
+    lib.sdpa_debug_turn_timeout.argtypes = [vp, vp]
+    lib.sdpa_debug_turn_timeout.restype = i32
     lib.sdpa_status_string.argtypes = [i32]
     lib.sdpa_status_string.restype = ctypes.c_char_p
     if path is None:
@@ -118,16 +134,40 @@ def _ptr(t):
 
 
 def make_shape(q: torch.Tensor, k: torch.Tensor) -> Shape:
+    """Shape of q [B, L, Hq, d] against k [B, Lk, Hkv, d] (Lk may differ from L)."""
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be [B, L, H, d]")
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
-    if k.shape[0] != B or k.shape[1] != L or k.shape[3] != d:
+    if k.shape[0] != B or k.shape[3] != d:
         raise ValueError(f"k shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
     if q.stride(-1) != 1 or k.stride(-1) != 1:
         raise ValueError("head_dim must be contiguous")
     return Shape(B, L, Hq, Hkv, d, q.stride(0), q.stride(1), q.stride(2),
-                 k.stride(0), k.stride(1), k.stride(2))
+                 k.stride(0), k.stride(1), k.stride(2), k.shape[1])
+
+
+def make_varlen_shape(q: torch.Tensor, k: torch.Tensor, batch: int) -> Shape:
+    """Shape of packed q [total_q, Hq, d] and k [total_k, Hkv, d] with `batch` sequences."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed q and k must be [total, H, d]")
+    if q.shape[2] != k.shape[2]:
+        raise ValueError("q and k head dims differ")
+    if q.stride(-1) != 1 or k.stride(-1) != 1:
+        raise ValueError("head_dim must be contiguous")
+    return Shape(int(batch), 0, q.shape[1], k.shape[1], q.shape[2], 0, q.stride(0), q.stride(1),
+                 0, k.stride(0), k.stride(1), 0)
+
+
+def make_varlen(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
+                max_seqlen_k: int, total_q: int, total_k: int) -> Varlen:
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{n} must be a contiguous int32 CUDA vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel():
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    return Varlen(cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), int(max_seqlen_q),
+                  int(max_seqlen_k), int(total_q), int(total_k))
 
 
 def make_mask(causal: bool, window_left: int, window_right: int) -> MaskSpec:
@@ -151,11 +191,12 @@ def make_bias(bias: torch.Tensor | None, t5_table: torch.Tensor | None, num_buck
         if bias.dtype != torch.float32 or bias.dim() != 4 or bias.stride(-1) != 1:
             raise ValueError("dense bias must be float32 [B|1, H|1, L, L] with j contiguous")
         if dims is not None:
-            B, Hq, L = dims
+            B, Hq, L = dims[:3]
+            Lk = dims[3] if len(dims) > 3 else L
             if (bias.shape[0] not in (1, B) or bias.shape[1] not in (1, Hq)
-                    or tuple(bias.shape[2:]) != (L, L)):
+                    or tuple(bias.shape[2:]) != (L, Lk)):
                 raise ValueError(f"dense bias shape {tuple(bias.shape)} is not "
-                                 f"[{B}|1, {Hq}|1, {L}, {L}]")
+                                 f"[{B}|1, {Hq}|1, {L}, {Lk}]")
         sb = bias.stride(0) if bias.shape[0] > 1 else 0
         sh = bias.stride(1) if bias.shape[1] > 1 else 0
         return BiasDesc(BIAS_DENSE, bias.data_ptr(), sb, sh, bias.stride(2), 0, 0, 0)
@@ -196,7 +237,7 @@ def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=Non
         raise ValueError("lse must be contiguous float32 [B, Hq, L]")
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (B, Hq, L), alibi_slopes)
+                   (B, Hq, L, k.shape[1]), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bd),
                       ctypes.byref(m), sc, _ptr(out), _ptr(lse), _stream(q))
@@ -216,9 +257,9 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
              workspace=None, deterministic=True, phases=BWD_ALL):
     """dQ, dK, dV = attention backward (see sdpa_bwd / sdpa_bwd_phases in include/sdpa.h).
 
-    ``phases`` selects launches (BWD_PREPROCESS | BWD_DQ | BWD_DKDV); the
-    default runs all three in order.  A partial call needs the workspace of
-    an earlier PREPROCESS call.
+    ``phases`` selects launches (BWD_PREPROCESS | BWD_GRADS); the default
+    runs both in order.  A GRADS call needs the workspace of an earlier
+    PREPROCESS call (one per GRADS call).
     """
     lib = load_library()
     shape = make_shape(q, k)
@@ -237,7 +278,7 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
             ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk), _ptr(dv),
@@ -256,8 +297,9 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
     """Backward into caller-given dQ, dK, dV with no workspace and no allocation.
 
     For callers that cannot allocate device memory: the library's built-in
-    scratch array (NOALLOC_MAX_ROWS rows of B * Hq * L) stands in for the
-    workspace.  Calls that overlap on the GPU race on that array.
+    scratch array (NOALLOC_SCRATCH_BYTES) stands in for the workspace, so the
+    shape's sdpa_bwd_workspace_size must fit in it.  Calls that overlap on
+    the GPU race on that array.
     """
     lib = load_library()
     shape = make_shape(q, k)
@@ -266,12 +308,79 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
         _same_layout(t, ref, n)
     sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_bwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
                               _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq),
                               _ptr(dk), _ptr(dv), 1, _stream(q))
     _check(st, "sdpa_bwd_noalloc")
+    return dq, dk, dv
+
+
+def sdpa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
+                    causal=False, window_left=-1, window_right=-1, t5_table=None,
+                    t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
+                    alibi_slopes=None, scale=None, out=None, lse=None):
+    """O [total_q, Hq, d], LSE [Hq, total_q] of a packed batch (sdpa_fwd_varlen)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise ValueError(f"{n} must be a bf16 CUDA tensor")
+    _same_layout(v, k, "v")
+    B = cu_seqlens_q.numel() - 1
+    shape = make_varlen_shape(q, k, B)
+    vl = make_varlen(cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, q.shape[0],
+                     k.shape[0])
+    total_q, Hq, d = q.shape
+    out = torch.empty_like(q) if out is None else out
+    _same_layout(out, q, "out")
+    if lse is None:
+        lse = torch.empty(Hq, total_q, device=q.device, dtype=torch.float32)
+    if lse.shape != (Hq, total_q) or not lse.is_contiguous() or lse.dtype != torch.float32:
+        raise ValueError("lse must be contiguous float32 [Hq, total_q]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    bd = make_bias(None, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (B, q.shape[1], 0, 0), alibi_slopes)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_fwd_varlen(ctypes.byref(shape), ctypes.byref(vl), _ptr(q), _ptr(k), _ptr(v),
+                             ctypes.byref(bd), ctypes.byref(m), sc, _ptr(out), _ptr(lse),
+                             _stream(q))
+    _check(st, "sdpa_fwd_varlen")
+    return out, lse
+
+
+def sdpa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, *, causal=False, window_left=-1, window_right=-1,
+                    t5_table=None, t5_num_buckets=32, t5_max_distance=128,
+                    t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None,
+                    dv=None, workspace=None):
+    """dQ, dK, dV of a packed batch (sdpa_bwd_varlen)."""
+    lib = load_library()
+    _same_layout(v, k, "v")
+    _same_layout(o, q, "o")
+    _same_layout(do, q, "do")
+    B = cu_seqlens_q.numel() - 1
+    shape = make_varlen_shape(q, k, B)
+    vl = make_varlen(cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, q.shape[0],
+                     k.shape[0])
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _same_layout(dq, q, "dq")
+    _same_layout(dk, k, "dk")
+    _same_layout(dv, k, "dv")
+    need = int(lib.sdpa_bwd_varlen_workspace_size(ctypes.byref(shape), ctypes.byref(vl)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+    bd = make_bias(None, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
+                   (B, q.shape[1], 0, 0), alibi_slopes)
+    m = make_mask(causal, window_left, window_right)
+    st = lib.sdpa_bwd_varlen(ctypes.byref(shape), ctypes.byref(vl), _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(o), _ptr(do), _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc,
+                             _ptr(dq), _ptr(dk), _ptr(dv), 1, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(q))
+    _check(st, "sdpa_bwd_varlen")
     return dq, dk, dv
 
 
@@ -281,7 +390,7 @@ def sdpa_bwd_bias_grad_workspace_size(q, k, *, bias=None, t5_table=None, t5_num_
     lib = load_library()
     shape = make_shape(q, k)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
     return int(lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(shape), ctypes.byref(bd)))
 
 
@@ -306,7 +415,7 @@ def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, win
     _same_layout(dk, k, "dk")
     _same_layout(dv, k, "dv")
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
     ref = next((x for x in (bias, t5_table, alibi_slopes) if x is not None), None)
     if ref is None:
         raise ValueError("a bias gradient needs a dense bias, a T5 table or ALiBi slopes")
@@ -362,6 +471,14 @@ def sdpa_set_wait_limit_ns(ns: int):
 
 def sdpa_debug_wait_timeout():
     _check(load_library().sdpa_debug_wait_timeout(_stream()), "sdpa_debug_wait_timeout")
+
+
+def sdpa_debug_turn_timeout(counter: torch.Tensor):
+    """One warp waits, under the wait limit, for a dQ turn that never comes."""
+    if counter.dtype != torch.int32 or not counter.is_cuda or counter.numel() < 1:
+        raise ValueError("counter must be an int32 CUDA tensor")
+    _check(load_library().sdpa_debug_turn_timeout(_ptr(counter), _stream(counter)),
+           "sdpa_debug_turn_timeout")
 
 
 def sdpa_status_string(status: int) -> str:

@@ -53,21 +53,36 @@ __host__ __device__ __forceinline__ int t5_bucket(int rel, const T5Spec& s) {
 }
 
 struct AttnParams {
-  int B, L, Hq, Hkv, G;
+  // Batch entries, query / key sequence lengths (the longest, for packed
+  // sequences), heads (G = Hq / Hkv query heads per KV head).
+  int B, Lq, Lk, Hq, Hkv, G;
   int causal, wl, wr;          // wl / wr < 0: unbounded
   float scale;                 // softmax scale
   float scale_log2;            // scale * log2(e)
   int64_t sq_b, sq_l, sq_h;    // element strides: Q, O, dO, dQ
   int64_t skv_b, skv_l, skv_h; // element strides: K, V, dK, dV
+  // Packed variable-length sequences: batch entry b holds query rows
+  // [cu_q[b], cu_q[b + 1]) and key rows [cu_k[b], cu_k[b + 1]) of one
+  // sequence axis (sq_b = skv_b = 0).  nullptr: every entry has Lq / Lk rows.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;        // rows of the packed sequence axes (cu_q != nullptr)
+  // element strides of the per-row float arrays LSE, D and the dQ
+  // accumulator's rows: entry (b, h, row) is at b * lse_sb + h * lse_sh + row,
+  // row counted along the (packed) query sequence axis
+  int64_t lse_sb, lse_sh;
   // forward outputs / backward inputs
   __nv_bfloat16* o;
-  float* lse;                  // [B, Hq, L]
+  float* lse;
   // backward
   const __nv_bfloat16* dout;
-  float* dvec;                 // D = rowsum(dO * O), [B, Hq, L]
+  float* dvec;                 // D = rowsum(dO * O), laid out as LSE
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dq_acc;               // fp32 dQ partial sums, row r at dq_acc + r * d
+  unsigned int* turns;         // per (b, hq, query tile): key tiles already added
+  unsigned int* tickets;       // work-item counter of the persistent backward
   // optional fp32 dS (the gradient of the logits, = of an additive bias),
   // element strides sd_b, sd_h, sd_i (multiples of 4), j contiguous
   float* ds_out;
@@ -84,6 +99,46 @@ struct AttnParams {
   const float* alibi_slopes;   // [Hq]
   uint64_t wait_limit_ns;
 };
+
+// One batch entry's sequences: row offsets along the (packed) sequence axes,
+// lengths, and the batch coordinate of the tensor maps (0 when packed).
+struct SeqView {
+  int q0, k0, Lq, Lk, bc;
+};
+
+// Offsets that are not non-decreasing, leave the packed axis, or give a
+// sequence longer than the stated maximum record kStatusBadSeqlens and make
+// the entry empty, so no kernel addresses memory outside its tensors.
+__device__ __forceinline__ SeqView seq_view(const AttnParams& p, int b) {
+  SeqView s;
+  if (p.cu_q != nullptr) {
+    s.q0 = p.cu_q[b];
+    s.Lq = p.cu_q[b + 1] - s.q0;
+    s.k0 = p.cu_k[b];
+    s.Lk = p.cu_k[b + 1] - s.k0;
+    s.bc = 0;
+    const bool bad = s.q0 < 0 || s.Lq < 0 || s.Lq > p.Lq || s.q0 > p.total_q - s.Lq ||
+                     s.k0 < 0 || s.Lk < 0 || s.Lk > p.Lk || s.k0 > p.total_k - s.Lk;
+    if (bad) {
+      atomicOr(&g_device_status, kStatusBadSeqlens);
+      s.q0 = s.k0 = s.Lq = s.Lk = 0;
+    }
+  } else {
+    s.q0 = 0;
+    s.k0 = 0;
+    s.Lq = p.Lq;
+    s.Lk = p.Lk;
+    s.bc = b;
+  }
+  return s;
+}
+
+// Index of (b, h, query row i of b's sequence) in LSE, D and the dQ
+// accumulator's rows.
+__device__ __forceinline__ int64_t row_index(const AttnParams& p, const SeqView& s, int b, int h,
+                                             int i) {
+  return static_cast<int64_t>(b) * p.lse_sb + static_cast<int64_t>(h) * p.lse_sh + s.q0 + i;
+}
 
 // Relative-position bias of distance rel = j - i for query head hq, in log2
 // units (times log2 e), as the kBiasT5 kernels tabulate it per tile: the
@@ -106,78 +161,46 @@ __device__ __forceinline__ constexpr bool emu_exp2(int c) {
 }
 
 // Key tiles [nlo, nhi) that hold any key visible from query rows
-// [m0, m0 + rows) (clipped to L).  Empty when nhi <= nlo.
-__device__ __forceinline__ void key_tile_range(const AttnParams& p, int m0, int rows, int& nlo,
-                                               int& nhi) {
-  const int m_last = min(m0 + rows - 1, p.L - 1);
+// [m0, m0 + rows) (clipped to Lq), keys clipped to Lk.  Empty when nhi <= nlo.
+// Positions of both sequences count from 0.
+__device__ __forceinline__ void key_tile_range(const AttnParams& p, int Lq, int Lk, int m0,
+                                               int rows, int& nlo, int& nhi) {
+  const int m_last = min(m0 + rows - 1, Lq - 1);
   int jmin = 0;
   if (p.wl >= 0) jmin = max(0, m0 - p.wl);
-  int jmax = p.L - 1;
+  int jmax = Lk - 1;
   if (p.causal) jmax = min(jmax, m_last);
   if (p.wr >= 0) jmax = min(jmax, m_last + p.wr);
   nlo = jmin / kTile;
-  nhi = (jmax >= jmin) ? jmax / kTile + 1 : nlo;
+  nhi = (jmax >= jmin && m_last >= m0) ? jmax / kTile + 1 : nlo;
 }
 
-// Query tiles [mlo, mhi) holding any query that sees a key in
-// [n0, n0 + kTile) (clipped to L).
-__device__ __forceinline__ void query_tile_range(const AttnParams& p, int n0, int& mlo, int& mhi) {
-  const int n_last = min(n0 + kTile - 1, p.L - 1);
+// Query tiles [mlo, mhi) holding any query (< Lq) that sees a key in
+// [n0, n0 + kTile) (clipped to Lk).
+__device__ __forceinline__ void query_tile_range(const AttnParams& p, int Lq, int Lk, int n0,
+                                                 int& mlo, int& mhi) {
+  const int n_last = min(n0 + kTile - 1, Lk - 1);
   int imin = 0;
   if (p.causal) imin = n0;
   if (p.wr >= 0) imin = max(imin, n0 - p.wr);
-  int imax = p.L - 1;
+  int imax = Lq - 1;
   if (p.wl >= 0) imax = min(imax, n_last + p.wl);
   mlo = imin / kTile;
-  mhi = (imax >= imin) ? imax / kTile + 1 : mlo;
+  mhi = (imax >= imin && n_last >= n0) ? imax / kTile + 1 : mlo;
 }
 
 // L2 prefetch of the dense-bias rows [m0, m0 + 128) x keys [n0, n0 + 128) of
-// one (batch, query head), clipped to L (rounded up to 16 bytes, which stays
-// inside the row: row strides are multiples of 4 floats).  One thread issues.
+// one (batch, query head), clipped to Lq x Lk (rounded up to 16 bytes, which
+// stays inside the row: row strides are multiples of 4 floats).  One thread
+// issues.
 __device__ __forceinline__ void prefetch_bias_tile(const AttnParams& p, int b, int hq, int m0,
                                                    int n0) {
-  const int cols = min(kTile, p.L - n0);
+  const int cols = min(kTile, p.Lk - n0);
   if (cols <= 0) return;
   const uint32_t bytes = static_cast<uint32_t>((cols + 3) & ~3) * 4u;
   const float* base = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h + n0;
-  const int rows = min(kTile, p.L - m0);
+  const int rows = min(kTile, p.Lq - m0);
   for (int r = 0; r < rows; ++r) prefetch_l2(base + static_cast<int64_t>(m0 + r) * p.sb_i, bytes);
-}
-
-// True when every (query, key) pair of the tile (rows m0.., keys n0..) is
-// visible and in range, so no element needs masking.  `rows_in_range`
-// additionally requires every query row < L.
-__device__ __forceinline__ bool tile_is_full(const AttnParams& p, int m0, int n0,
-                                             bool rows_in_range) {
-  if (n0 + kTile > p.L) return false;
-  if (rows_in_range && m0 + kTile > p.L) return false;
-  if (p.causal && n0 + kTile - 1 > m0) return false;
-  if (p.wl >= 0 && n0 < m0 + kTile - 1 - p.wl) return false;
-  if (p.wr >= 0 && n0 + kTile - 1 > m0 + p.wr) return false;
-  return true;
-}
-
-// For query row i and a key tile starting at n0: the visible tile columns
-// are [lo, hi] (possibly empty).
-__device__ __forceinline__ void row_visible_cols(const AttnParams& p, int i, int n0, int& lo,
-                                                 int& hi) {
-  lo = 0;
-  if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
-  hi = min(kTile - 1, p.L - 1 - n0);
-  if (p.causal) hi = min(hi, i - n0);
-  if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
-}
-
-// For key j and a query tile starting at m0: the query columns that see j
-// are [lo, hi] (possibly empty).
-__device__ __forceinline__ void key_visible_rows(const AttnParams& p, int j, int m0, int& lo,
-                                                 int& hi) {
-  lo = 0;
-  if (p.causal) lo = max(lo, j - m0);
-  if (p.wr >= 0) lo = max(lo, j - p.wr - m0);
-  hi = min(kTile - 1, p.L - 1 - m0);
-  if (p.wl >= 0) hi = min(hi, j + p.wl - m0);
 }
 
 // Byte offset of the 16-element K step kk inside a K-major SW128 tile of

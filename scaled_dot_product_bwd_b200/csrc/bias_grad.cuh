@@ -1,5 +1,5 @@
-// Bias gradients from the fp32 dS the dQ kernel stores (bwd_dq_kernel with
-// DS_OUT): the scores are linear in an additive bias, so a dense bias's
+// Bias gradients from the fp32 dS the backward kernel stores (bwd_kernel
+// with DS_OUT): the scores are linear in an additive bias, so a dense bias's
 // gradient is dS summed over each index the bias is broadcast along, and a
 // T5 table entry's gradient is dS summed over every (b, i, j) whose distance
 // j - i falls in its bucket (catie-aq/flashT5 README, "Full attention
@@ -27,8 +27,8 @@ constexpr int64_t kT5RowsPerPiece = 128;
 // ---------------------------------------------------------------------
 // dS entries the backward never visits: for query row i, the key tiles
 // outside [nlo, nhi) of i's query tile (key_tile_range), which hold no key
-// visible from any row of the tile.  The dQ kernel writes every column of
-// the tiles inside the band (masked keys as 0); this fills the rest with 0.
+// visible from any row of the tile.  The backward kernel writes every column
+// of the tiles inside the band (masked keys as 0); this fills the rest with 0.
 __device__ __forceinline__ void zero_span(float* row, int j0, int j1) {
   // j0 is 0 or a multiple of the tile width, so row + j0 is 16-byte aligned
   for (int j = j0 + 4 * static_cast<int>(threadIdx.x); j < j1; j += 4 * static_cast<int>(blockDim.x)) {
@@ -41,19 +41,19 @@ __device__ __forceinline__ void zero_span(float* row, int j0, int j1) {
 }
 
 __global__ void __launch_bounds__(256) ds_zero_outside_band_kernel(const AttnParams p) {
-  const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.L;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.Lq;
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int i = static_cast<int>(r % p.L);
-    const int64_t bh = r / p.L;
+    const int i = static_cast<int>(r % p.Lq);
+    const int64_t bh = r / p.Lq;
     const int hq = static_cast<int>(bh % p.Hq);
     const int b = static_cast<int>(bh / p.Hq);
     int nlo, nhi;
-    key_tile_range(p, (i / kTile) * kTile, kTile, nlo, nhi);
+    key_tile_range(p, p.Lq, p.Lk, (i / kTile) * kTile, kTile, nlo, nhi);
     float* row = p.ds_out + static_cast<int64_t>(b) * p.sd_b + static_cast<int64_t>(hq) * p.sd_h +
                  static_cast<int64_t>(i) * p.sd_i;
-    // [0, nlo * 128) and [nhi * 128, L); with an empty band the two cover the row
-    zero_span(row, 0, min(nlo * kTile, p.L));
-    zero_span(row, min(nhi * kTile, p.L), p.L);
+    // [0, nlo * 128) and [nhi * 128, Lk); with an empty band the two cover the row
+    zero_span(row, 0, min(nlo * kTile, p.Lk));
+    zero_span(row, min(nhi * kTile, p.Lk), p.Lk);
   }
 }
 

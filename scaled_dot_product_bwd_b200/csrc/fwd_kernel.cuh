@@ -116,11 +116,13 @@ __global__ void __launch_bounds__(384, 1)
 
   // ---- work items: (query tile, head, batch), heaviest causal query tiles
   // first; consecutive items are neighbouring heads, which share K / V in L2.
-  const int nqt = (p.L + kTile - 1) / kTile;
+  // Query tiles past a (packed) sequence's end are empty items.
+  const int nqt = (p.Lq + kTile - 1) / kTile;
   const int heads = p.Hq * p.B;
   const int n_items = nqt * heads;
   struct Item {
     int m0, hq, b, g, nlo, nt;
+    SeqView s;
   };
   auto item_at = [&](int id) {
     Item w;
@@ -131,9 +133,10 @@ __global__ void __launch_bounds__(384, 1)
     w.hq = rem % p.Hq;
     w.b = rem / p.Hq;
     w.g = w.hq / p.G;
+    w.s = seq_view(p, w.b);
     int nhi;
-    key_tile_range(p, w.m0, kTile, w.nlo, nhi);
-    w.nt = nhi > w.nlo ? nhi - w.nlo : 0;
+    key_tile_range(p, w.s.Lq, w.s.Lk, w.m0, kTile, w.nlo, nhi);
+    w.nt = (w.m0 < w.s.Lq && nhi > w.nlo) ? nhi - w.nlo : 0;
     return w;
   };
 
@@ -216,7 +219,8 @@ __global__ void __launch_bounds__(384, 1)
           if (u > 0 && !(ok = mbar_wait(q_empty, (u - 1) & 1, ctl))) break;
           mbar_expect_tx(q_full, Lay::kTileBytes);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, w.m0, w.hq, w.b);
+            tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, w.s.q0 + w.m0,
+                        w.hq, w.s.bc);
           q_issued = u & 1;
         }
         for (int it = 0; it < w.nt; ++it, ++c) {
@@ -228,7 +232,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_expect_tx(full, Lay::kTileBytes);
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(ring + s * Lay::kTileBytes + h * kTile * 128, map, full, h * 64,
-                        (w.nlo + it) * kTile, w.g, w.b);
+                        w.s.k0 + (w.nlo + it) * kTile, w.g, w.s.bc);
           issued[s] = static_cast<int>(ph);
           if constexpr (BT) {
             if (is_k) {
@@ -339,12 +343,13 @@ __global__ void __launch_bounds__(384, 1)
     for (int id = blockIdx.x; id < n_items; id += gridDim.x) {
       const Item w = item_at(id);
       const int m0 = w.m0, hq = w.hq, b = w.b, nt = w.nt;
+      const int Lq = w.s.Lq, Lk = w.s.Lk;
       const int i = m0 + row;  // query row
       const float* brow = nullptr;
       if constexpr (BIAS == kBiasDense) {
-        // rows past L read row L-1 (in bounds); their outputs are never stored
+        // rows past Lq read row Lq-1 (in bounds); their outputs are never stored
         brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
-               static_cast<int64_t>(min(i, p.L - 1)) * p.sb_i;
+               static_cast<int64_t>(min(i, Lq - 1)) * p.sb_i;
       }
       float m_run = -INFINITY;  // running row max, log2 units (identical in both warpgroups)
       float l_run = 0.f;        // this warpgroup's share of the row sum, relative to m_run
@@ -363,13 +368,13 @@ __global__ void __launch_bounds__(384, 1)
           lut_row = lt + (kTile - 1) - row;
         }
         int lo = 0, hi = kBlk - 1;
-        bool full = n0 + kBlk <= p.L;
+        bool full = n0 + kBlk <= Lk;
         if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
         if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
         if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
         if (!full) {
           if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
-          hi = min(hi, p.L - 1 - n0);
+          hi = min(hi, Lk - 1 - n0);
           if (p.causal) hi = min(hi, i - n0);
           if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
         }
@@ -559,8 +564,10 @@ __global__ void __launch_bounds__(384, 1)
       }
 
       // ------------------------------ epilogue ------------------------------
-      // Items without a visible key (none exist for the masks accepted at the
-      // boundary) write O = 0 and LSE = -inf without touching tensor memory.
+      // Rows that see no key (a left window that starts past the end of a
+      // shorter key sequence, an empty packed key sequence) get O = 0 and
+      // LSE = -inf without touching tensor memory; rows past the end of the
+      // query sequence are not written.
       float l_tot = 0.f;
       if (nt > 0) {
         rsum[((u & 1) * 2 + wg) * kTile + row] = l_run;
@@ -584,22 +591,56 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < D / 2; ++e) r[e] = 0u;
         }
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-        if (i < p.L) {
-          __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.sq_b +
-                                static_cast<int64_t>(i) * p.sq_l + static_cast<int64_t>(hq) * p.sq_h +
-                                wg * (D / 2);
+        // O: lanes 2m and 2m + 1 hold rows i and i + 1.  For every 16
+        // columns (32 bytes of bf16) they trade halves, so each 16-byte
+        // store of the pair writes one whole 32-byte sector of one row: the
+        // even lane's row first, then the odd lane's.
+        const bool odd = (lane & 1) != 0;
+        const int i_a = odd ? i - 1 : i, i_b = odd ? i : i + 1;
+        __nv_bfloat16* row_a = p.o + static_cast<int64_t>(b) * p.sq_b +
+                               static_cast<int64_t>(w.s.q0 + i_a) * p.sq_l +
+                               static_cast<int64_t>(hq) * p.sq_h + wg * (D / 2) + (odd ? 8 : 0);
+        __nv_bfloat16* row_b = row_a + p.sq_l;
 #pragma unroll
-          for (int c = 0; c < D / 2; c += 8) {
-            uint4 v4;
-            v4.x = pack_bf16x2(__uint_as_float(r[c]) * inv, __uint_as_float(r[c + 1]) * inv);
-            v4.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv, __uint_as_float(r[c + 3]) * inv);
-            v4.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv, __uint_as_float(r[c + 5]) * inv);
-            v4.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv, __uint_as_float(r[c + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c) = v4;
-          }
-          if (wg == 0) {
-            p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + i] =
-                l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
+        for (int c = 0; c < D / 2; c += 16) {
+          uint4 lo, hi;
+          lo.x = pack_bf16x2(__uint_as_float(r[c]) * inv, __uint_as_float(r[c + 1]) * inv);
+          lo.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv, __uint_as_float(r[c + 3]) * inv);
+          lo.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv, __uint_as_float(r[c + 5]) * inv);
+          lo.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv, __uint_as_float(r[c + 7]) * inv);
+          hi.x = pack_bf16x2(__uint_as_float(r[c + 8]) * inv, __uint_as_float(r[c + 9]) * inv);
+          hi.y = pack_bf16x2(__uint_as_float(r[c + 10]) * inv, __uint_as_float(r[c + 11]) * inv);
+          hi.z = pack_bf16x2(__uint_as_float(r[c + 12]) * inv, __uint_as_float(r[c + 13]) * inv);
+          hi.w = pack_bf16x2(__uint_as_float(r[c + 14]) * inv, __uint_as_float(r[c + 15]) * inv);
+          // the even lane sends its columns c+8.., the odd lane its columns c..
+          const uint4 snd = odd ? lo : hi;
+          uint4 got;
+          got.x = __shfl_xor_sync(0xffffffffu, snd.x, 1);
+          got.y = __shfl_xor_sync(0xffffffffu, snd.y, 1);
+          got.z = __shfl_xor_sync(0xffffffffu, snd.z, 1);
+          got.w = __shfl_xor_sync(0xffffffffu, snd.w, 1);
+          const uint4 va = odd ? got : lo;  // row i_a
+          const uint4 vb = odd ? hi : got;  // row i_b
+          if (i_a < Lq) *reinterpret_cast<uint4*>(row_a + c) = va;
+          if (i_b < Lq) *reinterpret_cast<uint4*>(row_b + c) = vb;
+        }
+        if (wg == 0) {
+          // LSE: each group of four lanes gathers its four rows into the first
+          // lane, which writes them as one 16-byte store when all four rows
+          // exist and the address is 16-byte aligned (scalar stores otherwise).
+          const float lse = l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
+          float4 l4;
+          l4.x = __shfl_sync(0xffffffffu, lse, lane & ~3);
+          l4.y = __shfl_sync(0xffffffffu, lse, (lane & ~3) + 1);
+          l4.z = __shfl_sync(0xffffffffu, lse, (lane & ~3) + 2);
+          l4.w = __shfl_sync(0xffffffffu, lse, (lane & ~3) + 3);
+          const int64_t li = row_index(p, w.s, b, hq, i);
+          const int i0 = i - (lane & 3);
+          const bool vec = (((li - (lane & 3)) & 3) == 0) && (i0 + 3 < Lq);
+          if (vec) {
+            if ((lane & 3) == 0) *reinterpret_cast<float4*>(p.lse + li) = l4;
+          } else if (i < Lq) {
+            p.lse[li] = lse;
           }
         }
       }

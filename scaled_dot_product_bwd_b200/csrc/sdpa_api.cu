@@ -1,9 +1,11 @@
 // sdpa_api.cu -- host side of the C ABI declared in include/sdpa.h:
 // argument validation (before anything is queued), TMA tensor maps,
-// T5 bucket thresholds, kernel launches, and the device status word.
+// T5 bucket thresholds, workspace plans, kernel launches, and the device
+// status word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -41,34 +43,106 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D map over a (batch, seq, head, head_dim) bf16 tensor, box = 64 head-dim
-// elements x `rows` rows of one head of one batch, 128-byte swizzle.  Rows
-// past the sequence end read as zero.
-bool make_bshd_map(CUtensorMap* m, const void* base, int64_t B, int64_t L, int64_t H, int64_t D,
-                   int64_t s_b, int64_t s_l, int64_t s_h, int rows = kTile) {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shapes of one call: B sequences of Lq query and Lk key rows (padded), or
+// B packed sequences along one axis of total_q / total_k rows whose
+// lengths are at most Lq / Lk.
+struct Geometry {
+  int64_t B, Lq, Lk, Hq, Hkv, d;
+  bool packed;
+  int64_t total_q, total_k;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int64_t sq_b, sq_l, sq_h, skv_b, skv_l, skv_h;
+  // positions along the query / key sequence axis (per head)
+  int64_t axis_q() const { return packed ? total_q : B * Lq; }
+  int64_t axis_k() const { return packed ? total_k : B * Lk; }
+  // rows of LSE, D and the dQ accumulator
+  int64_t rows() const { return Hq * axis_q(); }
+};
+
+sdpa_status_t make_geometry(const sdpa_shape* s, const sdpa_varlen* vl, Geometry& g) {
+  if (!s) return SDPA_ERR_INVALID_ARG;
+  g = Geometry{};
+  g.B = s->B;
+  g.Hq = s->Hq;
+  g.Hkv = s->Hkv;
+  g.d = s->d;
+  if (g.B < 1 || g.Hq < 1 || g.Hkv < 1) return SDPA_ERR_INVALID_ARG;
+  if (g.Hq % g.Hkv != 0) return SDPA_ERR_INVALID_ARG;
+  if (g.d != 64 && g.d != 128) return SDPA_ERR_UNSUPPORTED;
+  if (g.B > 65535 || g.Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  g.sq_l = s->sq_l;
+  g.sq_h = s->sq_h;
+  g.skv_l = s->skv_l;
+  g.skv_h = s->skv_h;
+  if (vl) {
+    if (!vl->cu_seqlens_q || !vl->cu_seqlens_k) return SDPA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(vl->cu_seqlens_q) & 3u) ||
+        (reinterpret_cast<uintptr_t>(vl->cu_seqlens_k) & 3u))
+      return SDPA_ERR_INVALID_ARG;
+    g.packed = true;
+    g.cu_q = vl->cu_seqlens_q;
+    g.cu_k = vl->cu_seqlens_k;
+    g.Lq = vl->max_seqlen_q;
+    g.Lk = vl->max_seqlen_k;
+    g.total_q = vl->total_q;
+    g.total_k = vl->total_k;
+    if (g.Lq < 1 || g.Lk < 1 || g.total_q < 1 || g.total_k < 1) return SDPA_ERR_INVALID_ARG;
+    if (g.total_q >= (1ll << 30) || g.total_k >= (1ll << 30)) return SDPA_ERR_UNSUPPORTED;
+    g.sq_b = 0;
+    g.skv_b = 0;
+  } else {
+    g.Lq = s->L;
+    g.Lk = s->Lk > 0 ? s->Lk : s->L;
+    if (g.Lq < 1 || s->Lk < 0) return SDPA_ERR_INVALID_ARG;
+    g.sq_b = s->sq_b;
+    g.skv_b = s->skv_b;
+    if (g.sq_b <= 0 || (g.sq_b % 8) != 0 || g.sq_b >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
+    if (g.skv_b <= 0 || (g.skv_b % 8) != 0 || g.skv_b >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
+  }
+  if (g.Lq >= (1ll << 30) || g.Lk >= (1ll << 30)) return SDPA_ERR_UNSUPPORTED;
+  if ((g.Lq + 127) / 128 * g.Hq * g.B >= (1ll << 31)) return SDPA_ERR_UNSUPPORTED;
+  if ((g.Lk + 127) / 128 * g.Hkv * g.B >= (1ll << 31)) return SDPA_ERR_UNSUPPORTED;
+  const int64_t st[4] = {g.sq_l, g.sq_h, g.skv_l, g.skv_h};
+  for (int64_t v : st)
+    if (v <= 0 || (v % 8) != 0 || v >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
+  return SDPA_OK;
+}
+
+// 4-D map over a bf16 tensor along (head_dim, sequence axis, head, batch),
+// box = 64 head-dim elements x 128 rows of one head, 128-byte swizzle.  Rows
+// past the axis end read as zero.  Packed sequences: one batch entry over
+// the whole packed axis.
+bool make_axis_map(CUtensorMap* m, const void* base, const Geometry& g, bool query) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
-                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_l) * 2, static_cast<cuuint64_t>(s_h) * 2,
-                           static_cast<cuuint64_t>(s_b) * 2};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), 1, 1};
+  const int64_t axis = g.packed ? (query ? g.total_q : g.total_k) : (query ? g.Lq : g.Lk);
+  const int64_t H = query ? g.Hq : g.Hkv;
+  const int64_t sl = query ? g.sq_l : g.skv_l, sh = query ? g.sq_h : g.skv_h;
+  const int64_t sbt = g.packed ? sl * axis : (query ? g.sq_b : g.skv_b);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(axis),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(g.packed ? 1 : g.B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(sl) * 2, static_cast<cuuint64_t>(sh) * 2,
+                           static_cast<cuuint64_t>(sbt) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kTile), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Dense fp32 bias [B|1, Hq|1, L, L] as a 4-D map (j, i, head, batch) with
+// Dense fp32 bias [B|1, Hq|1, Lq, Lk] as a 4-D map (j, i, head, batch) with
 // boxes of 32 keys x 128 queries (128-byte swizzle); a broadcast index has
 // extent 1 and is always addressed at 0.
 bool make_bias_map(CUtensorMap* m, const AttnParams& p) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t row = static_cast<cuuint64_t>(p.sb_i) * 4;
-  const cuuint64_t head = p.sb_h ? static_cast<cuuint64_t>(p.sb_h) * 4 : row * p.L;
+  const cuuint64_t head = p.sb_h ? static_cast<cuuint64_t>(p.sb_h) * 4 : row * p.Lq;
   const cuuint64_t batch = p.sb_b ? static_cast<cuuint64_t>(p.sb_b) * 4 : head * (p.sb_h ? p.Hq : 1);
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(p.L), static_cast<cuuint64_t>(p.L),
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(p.Lk), static_cast<cuuint64_t>(p.Lq),
                         static_cast<cuuint64_t>(p.sb_h ? p.Hq : 1),
                         static_cast<cuuint64_t>(p.sb_b ? p.B : 1)};
   cuuint64_t strides[3] = {row, head, batch};
@@ -78,8 +152,6 @@ bool make_bias_map(CUtensorMap* m, const AttnParams& p) {
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Integer thresholds of the T5 log buckets, evaluated in float64 exactly as
 // the closed form reads: large(n) = max_exact + trunc(ln(n / max_exact) /
@@ -115,40 +187,46 @@ int clamp_window(int64_t w, int64_t L) {
   return static_cast<int>(w > L ? L : w);
 }
 
-// Shared validation of shape / mask / bias; fills the common fields of p.
-sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
+// Validation of mask / bias and the common fields of p for geometry g.
+sdpa_status_t prepare(const Geometry& g, const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
                       float scale, AttnParams& p) {
-  if (!s || !mask) return SDPA_ERR_INVALID_ARG;
-  if (s->B < 1 || s->L < 1 || s->Hq < 1 || s->Hkv < 1) return SDPA_ERR_INVALID_ARG;
-  if (s->Hq % s->Hkv != 0) return SDPA_ERR_INVALID_ARG;
-  if (s->d != 64 && s->d != 128) return SDPA_ERR_UNSUPPORTED;
-  if (s->L >= (1ll << 30) || s->B > 65535 || s->Hq > 65535) return SDPA_ERR_UNSUPPORTED;
-  if ((s->L + 127) / 128 * s->Hq * s->B >= (1ll << 31)) return SDPA_ERR_UNSUPPORTED;
-  const int64_t st[6] = {s->sq_b, s->sq_l, s->sq_h, s->skv_b, s->skv_l, s->skv_h};
-  for (int64_t v : st)
-    if (v <= 0 || (v % 8) != 0 || v >= (1ll << 38)) return SDPA_ERR_INVALID_ARG;
+  if (!mask) return SDPA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
   std::memset(&p, 0, sizeof(p));
-  p.B = static_cast<int>(s->B);
-  p.L = static_cast<int>(s->L);
-  p.Hq = static_cast<int>(s->Hq);
-  p.Hkv = static_cast<int>(s->Hkv);
+  p.B = static_cast<int>(g.B);
+  p.Lq = static_cast<int>(g.Lq);
+  p.Lk = static_cast<int>(g.Lk);
+  p.Hq = static_cast<int>(g.Hq);
+  p.Hkv = static_cast<int>(g.Hkv);
   p.G = p.Hq / p.Hkv;
+  const int64_t span = std::max(g.Lq, g.Lk);
   p.causal = mask->causal ? 1 : 0;
-  p.wl = clamp_window(mask->window_left, s->L);
-  p.wr = clamp_window(mask->window_right, s->L);
+  p.wl = clamp_window(mask->window_left, span);
+  p.wr = clamp_window(mask->window_right, span);
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  p.sq_b = s->sq_b;
-  p.sq_l = s->sq_l;
-  p.sq_h = s->sq_h;
-  p.skv_b = s->skv_b;
-  p.skv_l = s->skv_l;
-  p.skv_h = s->skv_h;
+  p.sq_b = g.sq_b;
+  p.sq_l = g.sq_l;
+  p.sq_h = g.sq_h;
+  p.skv_b = g.skv_b;
+  p.skv_l = g.skv_l;
+  p.skv_h = g.skv_h;
+  if (g.packed) {
+    p.cu_q = g.cu_q;
+    p.cu_k = g.cu_k;
+    p.total_q = static_cast<int>(g.total_q);
+    p.total_k = static_cast<int>(g.total_k);
+    p.lse_sb = 0;
+    p.lse_sh = g.total_q;
+  } else {
+    p.lse_sb = g.Hq * g.Lq;
+    p.lse_sh = g.Lq;
+  }
   p.wait_limit_ns = g_wait_limit_ns;
   p.bias_kind = kBiasNone;
   if (bias && bias->kind != SDPA_BIAS_NONE) {
     if (bias->kind == SDPA_BIAS_DENSE) {
+      if (g.packed) return SDPA_ERR_UNSUPPORTED;  // a [B, H, L, L] tensor has no packed form
       if (!bias->ptr || !aligned16(bias->ptr)) return SDPA_ERR_INVALID_ARG;
       if (bias->stride_b < 0 || bias->stride_h < 0 || bias->stride_i < 0) return SDPA_ERR_INVALID_ARG;
       if (bias->stride_b % 4 != 0 || bias->stride_h % 4 != 0 || bias->stride_i % 4 != 0)
@@ -181,34 +259,120 @@ sdpa_status_t prepare(const sdpa_shape* s, const sdpa_bias_desc* bias, const sdp
   return SDPA_OK;
 }
 
-// Tensor maps for the backward's three launches, then the launches selected
-// by `phases`; p carries every pointer and size.
-sdpa_status_t run_bwd(uint32_t phases, const AttnParams& p, const sdpa_shape& s, const void* q,
-                      const void* k, const void* v, const void* dout, cudaStream_t stream) {
-  BwdMaps maps;
-  bool ok = true;
-  for (int rows : {kTile, kBlk}) {
-    CUtensorMap* mq = rows == kTile ? &maps.q128 : &maps.q64;
-    CUtensorMap* mdo = rows == kTile ? &maps.dout128 : &maps.dout64;
-    CUtensorMap* mk = rows == kTile ? &maps.k128 : &maps.k64;
-    CUtensorMap* mv = rows == kTile ? &maps.v128 : &maps.v64;
-    ok = ok && make_bshd_map(mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
-         make_bshd_map(mdo, dout, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h, rows) &&
-         make_bshd_map(mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows) &&
-         make_bshd_map(mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h, rows);
+// ------------------------------------------------------------- forward
+template <int D, int BIAS>
+cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
+                       const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
+  using Lay = FwdLayout<D, BIAS>;
+  auto kern = fwd_kernel<D, BIAS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Lay::kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  // persistent: one CTA per SM (or per work item, if fewer)
+  const int64_t items = static_cast<int64_t>((p.Lq + kTile - 1) / kTile) * p.Hq * p.B;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v, bmap);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
+                              const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
+  switch (p.bias_kind) {
+    case kBiasDense: return launch_fwd<D, kBiasDense>(p, q, k, v, bmap, st);
+    case kBiasT5: return launch_fwd<D, kBiasT5>(p, q, k, v, bmap, st);
+    default: return launch_fwd<D, kBiasNone>(p, q, k, v, bmap, st);
   }
-  std::memset(&maps.bias, 0, sizeof(maps.bias));  // read only by the dense-bias kernels
-  if (ok && p.bias_kind == kBiasDense) ok = make_bias_map(&maps.bias, p);
-  if (!ok) return SDPA_ERR_CUDA;
-  cudaError_t e = launch_bwd(p, maps, static_cast<int>(s.d), phases, stream);
+}
+
+sdpa_status_t run_fwd(const Geometry& g, const void* q, const void* k, const void* v,
+                      const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
+                      void* o, float* lse, void* stream) {
+  AttnParams p;
+  sdpa_status_t st = prepare(g, bias, mask, scale, p);
+  if (st != SDPA_OK) return st;
+  if (!q || !k || !v || !o || !lse) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return SDPA_ERR_INVALID_ARG;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  CUtensorMap mq, mk, mv, mb;
+  if (!make_axis_map(&mq, q, g, true) || !make_axis_map(&mk, k, g, false) ||
+      !make_axis_map(&mv, v, g, false))
+    return SDPA_ERR_CUDA;
+  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias kernels
+  if (p.bias_kind == kBiasDense && !make_bias_map(&mb, p)) return SDPA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (g.d == 128) ? dispatch_fwd_bias<128>(p, mq, mk, mv, mb, cs)
+                               : dispatch_fwd_bias<64>(p, mq, mk, mv, mb, cs);
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ backward
+BwdWorkspace plan_of(const Geometry& g) {
+  return bwd_workspace_plan(g.rows(), g.B, g.Hq, g.Lq, g.d);
+}
+
+// The backward's pointers, with its workspace (laid out by plan_of) at ws.
+sdpa_status_t bind_bwd(AttnParams& p, const Geometry& g, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* ws) {
+  const BwdWorkspace pl = plan_of(g);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.o = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(o));
+  p.lse = const_cast<float*>(lse);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dvec = reinterpret_cast<float*>(w + pl.d_off);
+  p.turns = reinterpret_cast<unsigned int*>(w + pl.turn_off);
+  p.tickets = p.turns + pl.n_turns;
+  p.dq_acc = reinterpret_cast<float*>(w + pl.acc_off);
+  return SDPA_OK;
+}
+
+// Tensor maps, then the launches selected by `phases`.
+sdpa_status_t run_bwd(uint32_t phases, const AttnParams& p, const Geometry& g, const void* q,
+                      const void* k, const void* v, const void* dout, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_axis_map(&mq, q, g, true) || !make_axis_map(&mdo, dout, g, true) ||
+      !make_axis_map(&mk, k, g, false) || !make_axis_map(&mv, v, g, false))
+    return SDPA_ERR_CUDA;
+  const BwdWorkspace pl = plan_of(g);
+  cudaError_t e =
+      g.d == 128 ? launch_bwd_d<128>(p, mq, mk, mv, mdo, phases, g.axis_q(), pl.n_turns, stream)
+                 : launch_bwd_d<64>(p, mq, mk, mv, mdo, phases, g.axis_q(), pl.n_turns, stream);
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status_t core_bwd(uint32_t phases, const Geometry& g, const void* q, const void* k,
+                       const void* v, const void* o, const void* dout, const float* lse,
+                       const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
+                       void* dq, void* dk, void* dv, int32_t deterministic, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (phases == 0 || (phases & ~static_cast<uint32_t>(SDPA_BWD_ALL)) != 0)
+    return SDPA_ERR_INVALID_ARG;
+  AttnParams p;
+  sdpa_status_t st = prepare(g, bias, mask, scale, p);
+  if (st != SDPA_OK) return st;
+  if (deterministic != 1) return SDPA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return SDPA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < plan_of(g).total)
+    return SDPA_ERR_WORKSPACE;
+  bind_bwd(p, g, o, dout, lse, dq, dk, dv, workspace);
+  return run_bwd(phases, p, g, q, k, v, dout, static_cast<cudaStream_t>(stream));
 }
 
 // ----- bias gradients: workspace plan (sdpa_bwd_bias_grad) -----
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct BiasGradPlan {
-  size_t d_bytes = 0;     // D vector
+  size_t bwd_bytes = 0;   // the backward's own workspace
   bool ds_ws = false;     // dS staged in the workspace (else written into dbias)
   int64_t lp = 0;         // row stride of the staged dS
   size_t ds_bytes = 0;
@@ -229,12 +393,13 @@ void split_reduction(int64_t n_red, int64_t blocks, int& chunks, int64_t& per_ch
   chunks = static_cast<int>((n_red + per_chunk - 1) / per_chunk);
 }
 
-sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, BiasGradPlan& pl) {
-  if (!s || !bias || s->B < 1 || s->L < 1 || s->Hq < 1) return SDPA_ERR_INVALID_ARG;
-  if (s->L >= (1ll << 30) || s->B > 65535 || s->Hq > 65535) return SDPA_ERR_UNSUPPORTED;
-  const int64_t B = s->B, Hq = s->Hq, L = s->L;
+// The bias gradient is built for self-attention of one padded length.
+sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, BiasGradPlan& pl) {
+  if (!bias) return SDPA_ERR_INVALID_ARG;
+  if (g.packed || g.Lq != g.Lk) return SDPA_ERR_UNSUPPORTED;
+  const int64_t B = g.B, Hq = g.Hq, L = g.Lq;
   pl = BiasGradPlan{};
-  pl.d_bytes = round256(static_cast<size_t>(B * Hq * L) * sizeof(float));
+  pl.bwd_bytes = plan_of(g).total;
   pl.lp = (L + 7) / 8 * 8;  // staged dS rows start on 32-byte boundaries
   // B * Hq * L * lp floats must stay far from 2^63 bytes
   const double ds_elems = static_cast<double>(B) * Hq * L * pl.lp;
@@ -276,7 +441,7 @@ sdpa_status_t plan_bias_grad(const sdpa_shape* s, const sdpa_bias_desc* bias, Bi
   } else {
     return SDPA_ERR_UNSUPPORTED;  // no bias: nothing to differentiate
   }
-  pl.total = pl.d_bytes + pl.ds_bytes + pl.part_bytes;
+  pl.total = pl.bwd_bytes + pl.ds_bytes + pl.part_bytes;
   return SDPA_OK;
 }
 
@@ -302,33 +467,6 @@ bool t5_ranges(const T5Spec& t, int L, int num_buckets, T5Ranges& rg) {
     rg.hi[k] = r;
   }
   return true;
-}
-
-template <int D, int BIAS>
-cudaError_t launch_fwd(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
-                       const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
-  using Lay = FwdLayout<D, BIAS>;
-  auto kern = fwd_kernel<D, BIAS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Lay::kSmemAlloc);
-  if (e != cudaSuccess) return e;
-  // persistent: one CTA per SM (or per work item, if fewer)
-  const int64_t items = static_cast<int64_t>((p.L + kTile - 1) / kTile) * p.Hq * p.B;
-  const int sms = sm_count();
-  if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = static_cast<int>(items < sms ? items : sms);
-  kern<<<grid, Lay::kThreads, Lay::kSmemAlloc, st>>>(p, q, k, v, bmap);
-  return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t dispatch_fwd_bias(const AttnParams& p, const CUtensorMap& q, const CUtensorMap& k,
-                              const CUtensorMap& v, const CUtensorMap& bmap, cudaStream_t st) {
-  switch (p.bias_kind) {
-    case kBiasDense: return launch_fwd<D, kBiasDense>(p, q, k, v, bmap, st);
-    case kBiasT5: return launch_fwd<D, kBiasT5>(p, q, k, v, bmap, st);
-    default: return launch_fwd<D, kBiasNone>(p, q, k, v, bmap, st);
-  }
 }
 
 __global__ void exp2_fma_kernel(const float* x, float* y, int64_t n) {
@@ -360,6 +498,16 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
   __syncthreads();
 }
 
+// One dQ turn that nothing ever passes, waited on under the wait limit by
+// one warp, the way the backward's reducer warps wait for theirs.
+__global__ void turn_timeout_kernel(const unsigned int* ctr, uint64_t limit_ns) {
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) abort_flag = 0;
+  __syncwarp();
+  const WaitCtl ctl{&abort_flag, limit_ns};
+  (void)wait_turn(ctr, 0xffffffffu, ctl);
+}
+
 }  // namespace
 
 extern "C" {
@@ -381,34 +529,34 @@ void sdpa_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns < 1000 ? 1000 : 
 sdpa_status_t sdpa_fwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
                        const sdpa_bias_desc* bias, const sdpa_mask_spec* mask, float scale,
                        void* o, float* lse, void* stream) {
-  AttnParams p;
-  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, nullptr, g);
   if (st != SDPA_OK) return st;
-  if (!q || !k || !v || !o || !lse) return SDPA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-    return SDPA_ERR_INVALID_ARG;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  CUtensorMap mq, mk, mv;
-  const sdpa_shape& s = *shape;
-  if (!make_bshd_map(&mq, q, s.B, s.L, s.Hq, s.d, s.sq_b, s.sq_l, s.sq_h) ||
-      !make_bshd_map(&mk, k, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h) ||
-      !make_bshd_map(&mv, v, s.B, s.L, s.Hkv, s.d, s.skv_b, s.skv_l, s.skv_h))
-    return SDPA_ERR_CUDA;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  CUtensorMap mb;
-  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias kernels
-  if (p.bias_kind == kBiasDense && !make_bias_map(&mb, p)) return SDPA_ERR_CUDA;
-  cudaError_t e = (s.d == 128) ? dispatch_fwd_bias<128>(p, mq, mk, mv, mb, cs)
-                               : dispatch_fwd_bias<64>(p, mq, mk, mv, mb, cs);
-  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  return run_fwd(g, q, k, v, bias, mask, scale, o, lse, stream);
+}
+
+sdpa_status_t sdpa_fwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen, const void* q,
+                              const void* k, const void* v, const sdpa_bias_desc* bias,
+                              const sdpa_mask_spec* mask, float scale, void* o, float* lse,
+                              void* stream) {
+  if (!varlen) return SDPA_ERR_INVALID_ARG;
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, varlen, g);
+  if (st != SDPA_OK) return st;
+  return run_fwd(g, q, k, v, bias, mask, scale, o, lse, stream);
 }
 
 size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic) {
   (void)deterministic;
-  if (!shape || shape->B < 1 || shape->Hq < 1 || shape->L < 1) return 0;
-  const size_t rows = static_cast<size_t>(shape->B) * shape->Hq * shape->L;
-  return ((rows * sizeof(float) + 255) / 256) * 256;
+  Geometry g;
+  if (make_geometry(shape, nullptr, g) != SDPA_OK) return 0;
+  return plan_of(g).total;
+}
+
+size_t sdpa_bwd_varlen_workspace_size(const sdpa_shape* shape, const sdpa_varlen* varlen) {
+  Geometry g;
+  if (!varlen || make_geometry(shape, varlen, g) != SDPA_OK) return 0;
+  return plan_of(g).total;
 }
 
 sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const void* q,
@@ -417,25 +565,11 @@ sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const vo
                               const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
                               void* dv, int32_t deterministic, void* workspace,
                               size_t workspace_bytes, void* stream) {
-  if (phases == 0 || (phases & ~SDPA_BWD_ALL) != 0) return SDPA_ERR_INVALID_ARG;
-  AttnParams p;
-  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, nullptr, g);
   if (st != SDPA_OK) return st;
-  if (deterministic != 1) return SDPA_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
-  for (const void* ptr : ptrs)
-    if (!ptr || !aligned16(ptr)) return SDPA_ERR_INVALID_ARG;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      workspace_bytes < sdpa_bwd_workspace_size(shape, deterministic))
-    return SDPA_ERR_WORKSPACE;
-  p.o = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(o));
-  p.lse = const_cast<float*>(lse);
-  p.dout = static_cast<const __nv_bfloat16*>(dout);
-  p.dvec = static_cast<float*>(workspace);
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  return run_bwd(phases, p, *shape, q, k, v, dout, static_cast<cudaStream_t>(stream));
+  return core_bwd(phases, g, q, k, v, o, dout, lse, bias, mask, scale, dq, dk, dv, deterministic,
+                  workspace, workspace_bytes, stream);
 }
 
 sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, const void* v,
@@ -447,9 +581,25 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k, co
                          dv, deterministic, workspace, workspace_bytes, stream);
 }
 
+sdpa_status_t sdpa_bwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen, const void* q,
+                              const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, const sdpa_bias_desc* bias,
+                              const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
+                              void* dv, int32_t deterministic, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!varlen) return SDPA_ERR_INVALID_ARG;
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, varlen, g);
+  if (st != SDPA_OK) return st;
+  return core_bwd(SDPA_BWD_ALL, g, q, k, v, o, dout, lse, bias, mask, scale, dq, dk, dv,
+                  deterministic, workspace, workspace_bytes, stream);
+}
+
 size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias) {
+  Geometry g;
+  if (make_geometry(shape, nullptr, g) != SDPA_OK) return 0;
   BiasGradPlan pl;
-  return plan_bias_grad(shape, bias, pl) == SDPA_OK ? pl.total : 0;
+  return plan_bias_grad(g, bias, pl) == SDPA_OK ? pl.total : 0;
 }
 
 sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,
@@ -458,8 +608,11 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
                                  const sdpa_mask_spec* mask, float scale, void* dq, void* dk,
                                  void* dv, float* dbias, int32_t deterministic, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, nullptr, g);
+  if (st != SDPA_OK) return st;
   AttnParams p;
-  sdpa_status_t st = prepare(shape, bias, mask, scale, p);
+  st = prepare(g, bias, mask, scale, p);
   if (st != SDPA_OK) return st;
   if (p.bias_kind == kBiasNone) return SDPA_ERR_UNSUPPORTED;
   if (deterministic != 1) return SDPA_ERR_UNSUPPORTED;
@@ -467,26 +620,21 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   for (const void* ptr : ptrs)
     if (!ptr || !aligned16(ptr)) return SDPA_ERR_INVALID_ARG;
   BiasGradPlan pl;
-  st = plan_bias_grad(shape, bias, pl);
+  st = plan_bias_grad(g, bias, pl);
   if (st != SDPA_OK) return st;
   T5Ranges rg;
-  if (p.bias_kind == kBiasT5 && !p.alibi && !t5_ranges(p.t5, p.L, bias->num_buckets, rg))
+  if (p.bias_kind == kBiasT5 && !p.alibi && !t5_ranges(p.t5, p.Lq, bias->num_buckets, rg))
     return SDPA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < pl.total)
     return SDPA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.o = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(o));
-  p.lse = const_cast<float*>(lse);
-  p.dout = static_cast<const __nv_bfloat16*>(dout);
-  p.dvec = reinterpret_cast<float*>(ws);
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  bind_bwd(p, g, o, dout, lse, dq, dk, dv, ws);
+  const int L = p.Lq;
   if (pl.ds_ws) {
-    p.ds_out = reinterpret_cast<float*>(ws + pl.d_bytes);
+    p.ds_out = reinterpret_cast<float*>(ws + pl.bwd_bytes);
     p.sd_i = pl.lp;
-    p.sd_h = pl.lp * p.L;
+    p.sd_h = pl.lp * L;
     p.sd_b = p.sd_h * p.Hq;
   } else {
     p.ds_out = dbias;
@@ -498,14 +646,14 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   const int sms = sm_count();
   if (sms <= 0) return SDPA_ERR_CUDA;
   if (p.causal || p.wl >= 0 || p.wr >= 0) {
-    const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.L;
+    const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * L;
     const int64_t grid = rows < 8ll * sms ? rows : 8ll * sms;
     ds_zero_outside_band_kernel<<<static_cast<unsigned>(grid), 256, 0, cs>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
   }
-  st = run_bwd(SDPA_BWD_ALL, p, *shape, q, k, v, dout, cs);
+  st = run_bwd(SDPA_BWD_ALL, p, g, q, k, v, dout, cs);
   if (st != SDPA_OK || !pl.ds_ws) return st;
-  float* part = reinterpret_cast<float*>(ws + pl.d_bytes + pl.ds_bytes);
+  float* part = reinterpret_cast<float*>(ws + pl.bwd_bytes + pl.ds_bytes);
   if (p.bias_kind == kBiasDense) {
     DenseReduce a;
     a.ds = p.ds_out;
@@ -516,16 +664,16 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.o_b = p.sb_b;
     a.o_h = p.sb_h;
     a.o_i = p.sb_i;
-    a.L = p.L;
+    a.L = L;
     a.eb = p.sb_b ? p.B : 1;
     a.eh = p.sb_h ? p.Hq : 1;
-    a.ei = p.L;
+    a.ei = L;
     a.rb = p.sb_b ? 1 : p.B;
     a.rh = p.sb_h ? 1 : p.Hq;
     a.ri = 1;
     a.n_out = static_cast<int64_t>(a.eb) * a.eh * a.ei;
     a.n_red = static_cast<int64_t>(a.rb) * a.rh * a.ri;
-    a.jblocks = (p.L + 255) / 256;
+    a.jblocks = (L + 255) / 256;
     a.chunks = pl.chunks;
     a.rchunk = pl.per_chunk;
     a.partial = part;
@@ -546,13 +694,13 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.ds_i = p.sd_i;
     a.B = p.B;
     a.Hq = p.Hq;
-    a.L = p.L;
+    a.L = L;
     a.chunks = pl.chunks;
     a.uchunk = pl.per_chunk;
     a.partial = part;
     a.out = dbias;
     a.num_buckets = p.alibi ? 0 : bias->num_buckets;
-    const unsigned rblocks = static_cast<unsigned>((2 * p.L - 1 + 127) / 128);
+    const unsigned rblocks = static_cast<unsigned>((2 * L - 1 + 127) / 128);
     t5_diag_kernel<<<dim3(rblocks, p.Hq, a.chunks), 128, 0, cs>>>(a);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     t5_piece_sum_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(a);
@@ -567,12 +715,12 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
 }
 
 // ---------------------------------------------------------------------
-// sdpa_bwd_noalloc: the backward's D-vector scratch in a fixed device array
-// instead of a caller workspace, for callers that cannot allocate device
-// memory (see include/sdpa.h).  In host code `g_noalloc_scratch` names a
-// host-side stand-in, not device memory, so the kernels are given the
-// device address looked up with cudaGetSymbolAddress, once per device.
-static __device__ __align__(256) float g_noalloc_scratch[SDPA_NOALLOC_MAX_ROWS];
+// sdpa_bwd_noalloc: the backward's workspace in a fixed device array
+// instead of caller memory, for callers that cannot allocate device memory
+// (see include/sdpa.h).  In host code `g_noalloc_scratch` names a host-side
+// stand-in, not device memory, so the kernels are given the device address
+// looked up with cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SDPA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -598,14 +746,14 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
                                const sdpa_bias_desc* bias, const sdpa_mask_spec* mask,
                                float scale, void* dq, void* dk, void* dv, int32_t deterministic,
                                void* stream) {
-  if (!shape || shape->B < 1 || shape->Hq < 1 || shape->L < 1) return SDPA_ERR_INVALID_ARG;
-  const uint64_t rows = static_cast<uint64_t>(shape->B) * static_cast<uint64_t>(shape->Hq) *
-                        static_cast<uint64_t>(shape->L);
-  if (rows > SDPA_NOALLOC_MAX_ROWS) return SDPA_ERR_WORKSPACE;
+  Geometry g;
+  sdpa_status_t st = make_geometry(shape, nullptr, g);
+  if (st != SDPA_OK) return st;
+  if (plan_of(g).total > sizeof(g_noalloc_scratch)) return SDPA_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_ptr();
   if (!scratch) return SDPA_ERR_CUDA;
-  return sdpa_bwd_phases(SDPA_BWD_ALL, shape, q, k, v, o, dout, lse, bias, mask, scale, dq, dk,
-                         dv, deterministic, scratch, sizeof(g_noalloc_scratch), stream);
+  return core_bwd(SDPA_BWD_ALL, g, q, k, v, o, dout, lse, bias, mask, scale, dq, dk, dv,
+                  deterministic, scratch, sizeof(g_noalloc_scratch), stream);
 }
 
 sdpa_status_t sdpa_t5_bucket(const int32_t* rel, int32_t* out, int64_t n, int32_t num_buckets,
@@ -637,12 +785,18 @@ sdpa_status_t sdpa_read_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(h)) != cudaSuccess) return SDPA_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SDPA_ERR_CUDA;
   if (h & kStatusTimeout) return SDPA_ERR_TIMEOUT;
-  if (h & kStatusMisaligned) return SDPA_ERR_UNSUPPORTED;
+  if (h & (kStatusMisaligned | kStatusBadSeqlens)) return SDPA_ERR_UNSUPPORTED;
   return SDPA_OK;
 }
 
 sdpa_status_t sdpa_debug_wait_timeout(void* stream) {
   wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_limit_ns);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+sdpa_status_t sdpa_debug_turn_timeout(const uint32_t* counter, void* stream) {
+  if (!counter || (reinterpret_cast<uintptr_t>(counter) & 3u)) return SDPA_ERR_INVALID_ARG;
+  turn_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(counter, g_wait_limit_ns);
   return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 

@@ -16,6 +16,7 @@ namespace sdpa {
 __device__ unsigned int g_device_status = 0;
 constexpr unsigned int kStatusTimeout = 1u;
 constexpr unsigned int kStatusMisaligned = 2u;
+constexpr unsigned int kStatusBadSeqlens = 4u;  // packed-sequence offsets out of range
 
 // Dynamic shared memory starts right after the 1 KB the driver reserves per
 // CTA, so it is 1024-byte aligned -- what the 128-byte swizzle atoms need.

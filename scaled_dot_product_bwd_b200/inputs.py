@@ -7,10 +7,11 @@ Q, K, V and dO are rounded to bfloat16 (round-to-nearest-even), the bias and
 table stay float32.  Everything is generated on the CPU so that both sides of
 a parity check see the same values.
 
-Layouts: Q, dO [B, L, Hq, d]; K, V [B, L, Hkv, d] (batch, sequence, heads,
+Layouts: Q, dO [B, L, Hq, d]; K, V [B, Lk, Hkv, d] (batch, sequence, heads,
 head dim -- the (B, T, N, H) layout of the codelab "jax-gpu-05-attention-gpu",
-section 3); T5 table [num_buckets, Hq]; dense bias [B, Hq, L, L]; ALiBi
-slopes [Hq].
+section 3); T5 table [num_buckets, Hq]; dense bias [B, Hq, L, Lk]; ALiBi
+slopes [Hq].  Packed variable-length batches draw one sequence axis
+(B = 1) and are cut by cumulative lengths (``cu_seqlens``).
 """
 from __future__ import annotations
 
@@ -32,24 +33,27 @@ class Inputs:
 
 def make_inputs(B: int, L: int, Hq: int, Hkv: int, d: int, *, seed: int = 0,
                 t5_buckets: int = 0, dense_bias: bool = False,
-                bias_shape: tuple | None = None, alibi: bool = False) -> Inputs:
+                bias_shape: tuple | None = None, alibi: bool = False,
+                Lk: int | None = None) -> Inputs:
     """Draw Q, K, V, dO (bf16) and optionally a T5 table / dense bias (fp32).
 
-    ALiBi slopes are not drawn: they are the geometric sequence of Press et
-    al. 2022, 2^(-8 (h + 1) / Hq) for head h (fp32)."""
+    K and V have Lk rows (default L).  ALiBi slopes are not drawn: they are
+    the geometric sequence of Press et al. 2022, 2^(-8 (h + 1) / Hq) for head
+    h (fp32)."""
     g = torch.Generator().manual_seed(seed)
+    Lk = L if Lk is None else Lk
 
     def randn(*shape):
         return torch.randn(*shape, generator=g, dtype=torch.float32)
 
     q = randn(B, L, Hq, d).to(torch.bfloat16)
-    k = randn(B, L, Hkv, d).to(torch.bfloat16)
-    v = randn(B, L, Hkv, d).to(torch.bfloat16)
+    k = randn(B, Lk, Hkv, d).to(torch.bfloat16)
+    v = randn(B, Lk, Hkv, d).to(torch.bfloat16)
     do = randn(B, L, Hq, d).to(torch.bfloat16)
     table = randn(t5_buckets, Hq) if t5_buckets else None
     bias = None
     if dense_bias:
-        bias = randn(*(bias_shape or (B, Hq, L, L)))
+        bias = randn(*(bias_shape or (B, Hq, L, Lk)))
     slopes = None
     if alibi:
         slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)],
@@ -66,3 +70,11 @@ WORKLOADS = {
     "t5rpe": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, window_left=-1, bias="t5"),
     "t5dense": dict(B=16, Hq=12, Hkv=12, L=1024, d=64, causal=False, window_left=-1, bias="dense"),
 }
+
+
+def cu_seqlens(lengths) -> torch.Tensor:
+    """Cumulative offsets [0, l0, l0 + l1, ...] (int32) of packed sequences."""
+    out = [0]
+    for n in lengths:
+        out.append(out[-1] + int(n))
+    return torch.tensor(out, dtype=torch.int32)

@@ -17,7 +17,8 @@ def case_inputs(c):
     return make_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], c["d"], seed=c.get("seed", 0),
                        t5_buckets=32 if c.get("bias") == "t5" else 0,
                        dense_bias=c.get("bias") == "dense",
-                       bias_shape=c.get("bias_shape"), alibi=c.get("bias") == "alibi")
+                       bias_shape=c.get("bias_shape"), alibi=c.get("bias") == "alibi",
+                       Lk=c.get("Lk"))
 
 
 def mask_kw(c):

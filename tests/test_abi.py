@@ -48,7 +48,7 @@ def test_status_strings(lib):
 
 def _shape(**kw):
     base = dict(B=1, L=128, Hq=4, Hkv=2, d=64, sq_b=128 * 4 * 64, sq_l=4 * 64, sq_h=64,
-                skv_b=128 * 2 * 64, skv_l=2 * 64, skv_h=64)
+                skv_b=128 * 2 * 64, skv_l=2 * 64, skv_h=64, Lk=0)
     base.update(kw)
     return binding.Shape(*[base[n] for n, _ in binding.Shape._fields_])
 
@@ -109,6 +109,70 @@ def test_bwd_rejects_bad_args(lib):
     assert call(wsb=ws - 1) == 3
     assert call(shape=_shape(d=80)) == 2
     assert lib.sdpa_bwd_workspace_size(None, 1) == 0
+
+
+def test_bwd_workspace_layout(lib):
+    # D (one float per LSE entry), the dQ turn counters (4 per 128 query rows
+    # of each head) plus the ticket word, and the float32 dQ accumulator
+    # (d floats per LSE entry), each rounded up to 256 bytes.
+    r256 = lambda x: (x + 255) // 256 * 256
+    for B, L, Hq, d, Lk in ((1, 128, 4, 64, 0), (2, 300, 4, 128, 0), (3, 37, 2, 64, 1000)):
+        s = _shape(B=B, L=L, Hq=Hq, d=d, Lk=Lk)
+        rows = B * Hq * L
+        turns = B * Hq * ((L + 127) // 128) * 4
+        want = r256(rows * 4) + r256((turns + 1) * 4) + r256(rows * d * 4)
+        assert lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1) == want
+    assert lib.sdpa_bwd_workspace_size(ctypes.byref(_shape(Lk=-1)), 1) == 0
+
+
+def test_bwd_phases_rejects_bad_bits(lib):
+    s = _shape()
+    m = binding.MaskSpec(1, -1, -1)
+    ws = lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1)
+    for ph in (0, 4, 7):
+        assert lib.sdpa_bwd_phases(ph, ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                   ctypes.byref(m), 0.125, FAKE, FAKE, FAKE, 1, FAKE, ws,
+                                   None) == 1
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
+    m = binding.MaskSpec(1, -1, -1)
+    big = _shape(B=1, L=65536, Hq=4, d=128, sq_b=65536 * 4 * 128, sq_l=4 * 128, sq_h=128,
+                 skv_b=65536 * 2 * 128, skv_l=2 * 128, skv_h=128)
+    assert lib.sdpa_bwd_workspace_size(ctypes.byref(big), 1) > binding.NOALLOC_SCRATCH_BYTES
+    assert lib.sdpa_bwd_noalloc(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                ctypes.byref(m), 0.1, FAKE, FAKE, FAKE, 1, None) == 3
+
+
+def _varlen(**kw):
+    base = dict(cu_seqlens_q=0x20000, cu_seqlens_k=0x20100, max_seqlen_q=300, max_seqlen_k=300,
+                total_q=1000, total_k=1000)
+    base.update(kw)
+    return binding.Varlen(*[base[n] for n, _ in binding.Varlen._fields_])
+
+
+def test_varlen_rejects_bad_args(lib):
+    s = binding.Shape(3, 0, 4, 2, 64, 0, 4 * 64, 64, 0, 2 * 64, 64, 0)
+    m = binding.MaskSpec(1, -1, -1)
+
+    def fwd(vl, bias=None, shape=s):
+        return lib.sdpa_fwd_varlen(ctypes.byref(shape), ctypes.byref(vl) if vl else None, FAKE,
+                                   FAKE, FAKE, ctypes.byref(bias) if bias else None,
+                                   ctypes.byref(m), 0.125, FAKE, FAKE, None)
+    assert fwd(None) == 1
+    for bad in (dict(cu_seqlens_q=0), dict(cu_seqlens_k=0x20102), dict(max_seqlen_q=0),
+                dict(max_seqlen_k=-3), dict(total_q=0), dict(total_k=0)):
+        assert fwd(_varlen(**bad)) == 1, bad
+    assert fwd(_varlen(total_q=1 << 30)) == 2
+    assert fwd(_varlen(), bias=_dense(0, 0, 300)) == 2       # no packed form of a dense bias
+    assert fwd(_varlen(), shape=binding.Shape(3, 0, 4, 2, 96, 0, 4 * 96, 96, 0, 2 * 96, 96, 0)) == 2
+    assert lib.sdpa_bwd_varlen_workspace_size(ctypes.byref(s), None) == 0
+    # rows of LSE, D and the dQ accumulator: Hq * total_q; counters per B * Hq * max tiles
+    r256 = lambda x: (x + 255) // 256 * 256
+    rows = 4 * 1000
+    turns = 3 * 4 * 3 * 4
+    want = r256(rows * 4) + r256((turns + 1) * 4) + r256(rows * 64 * 4)
+    assert lib.sdpa_bwd_varlen_workspace_size(ctypes.byref(s), ctypes.byref(_varlen())) == want
 
 
 def _dense(sb, sh, si, ptr=0x10000):
@@ -187,6 +251,9 @@ def test_binding_entry_points_share_the_bias_keywords():
     for fn in (binding.sdpa_fwd, binding.sdpa_bwd, binding.sdpa_bwd_noalloc,
                binding.sdpa_bwd_bias_grad):
         missing = keys - set(inspect.signature(fn).parameters)
+        assert not missing, (fn.__name__, missing)
+    for fn in (binding.sdpa_fwd_varlen, binding.sdpa_bwd_varlen):   # no dense bias when packed
+        missing = (keys - {"bias"}) - set(inspect.signature(fn).parameters)
         assert not missing, (fn.__name__, missing)
 
 

@@ -46,6 +46,16 @@ CASES = {
                                          bias="alibi"),
     "t5_unidirectional_causal_d64": dict(B=2, Hq=2, Hkv=2, L=280, d=64, causal=True, bias="t5",
                                          t5_bidirectional=False),
+    # cross-attention (keys of another length; positions of both sequences from 0)
+    "cross_longer_keys_gqa_d64": dict(B=2, Hq=4, Hkv=2, L=200, Lk=333, d=64),
+    "cross_shorter_keys_causal_d128": dict(B=1, Hq=2, Hkv=1, L=300, Lk=140, d=128, causal=True),
+    "cross_t5_d64": dict(B=2, Hq=2, Hkv=2, L=130, Lk=260, d=64, bias="t5"),
+    "cross_dense_bias_d64": dict(B=1, Hq=2, Hkv=2, L=150, Lk=200, d=64, bias="dense"),
+    "cross_alibi_causal_d128": dict(B=1, Hq=4, Hkv=2, L=257, Lk=129, d=128, causal=True,
+                                    bias="alibi"),
+    "cross_decoder_t5_causal_d64": dict(B=1, Hq=2, Hkv=1, L=100, Lk=300, d=64, causal=True,
+                                        bias="t5", t5_bidirectional=False),
+    "cross_one_key_d128": dict(B=2, Hq=2, Hkv=2, L=140, Lk=1, d=128),
 }
 
 
@@ -98,6 +108,31 @@ def test_bitwise_repeatable(name):
     inp = case_inputs(c)
     first = run_cuda(c, inp)
     for _ in range(3):
+        again = run_cuda(c, inp)
+        for n in first:
+            assert np.array_equal(first[n], again[n]), n
+
+
+def test_cross_window_past_the_keys():
+    # Queries whose left window starts past the last key see nothing: O = 0,
+    # LSE = -inf and zero gradients, while the others match the oracle.
+    c = dict(B=1, Hq=2, Hkv=1, L=400, Lk=150, d=128, causal=True, wl=100)
+    inp = case_inputs(c)
+    got = run_cuda(c, inp)
+    ref = run_oracle(c, inp)
+    dead = np.arange(250, 400)
+    assert (got["o"][:, dead] == 0).all() and np.isneginf(got["lse"][:, :, dead]).all()
+    assert (got["dq"][:, dead] == 0).all()
+    assert_close(got, ref)
+
+
+@pytest.mark.parametrize("name", ["cross_t5_d64", "cross_shorter_keys_causal_d128",
+                                  "alibi_causal_window_mqa_d128"])
+def test_bitwise_repeatable_more(name):
+    c = CASES[name]
+    inp = case_inputs(c)
+    first = run_cuda(c, inp)
+    for _ in range(2):
         again = run_cuda(c, inp)
         for n in first:
             assert np.array_equal(first[n], again[n]), n

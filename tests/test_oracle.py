@@ -609,3 +609,103 @@ def test_head_scores_masked_entries():
     S = head_scores(q, k, 0, 1, scale=0.5, causal=True)
     assert np.isneginf(S[0, 1:]).all()
     assert math.isclose(S[3, 2], 0.5 * float(q[0, 3, 1] @ k[0, 2, 0]), rel_tol=1e-14)
+
+
+# ------------------------------------------------------ packed sequences
+from oracle import (attention_backward_packed, attention_forward_packed,  # noqa: E402
+                    packed_positions, packed_visibility_mask)
+
+
+def _packed(lq, lk, Hq=4, Hkv=2, d=8, seed=0):
+    cq = np.concatenate([[0], np.cumsum(lq)]).astype(int)
+    ck = np.concatenate([[0], np.cumsum(lk)]).astype(int)
+    q = rnd((cq[-1], Hq, d), seed)
+    k = rnd((ck[-1], Hkv, d), seed + 1)
+    v = rnd((ck[-1], Hkv, d), seed + 2)
+    do = rnd((cq[-1], Hq, d), seed + 3)
+    return cq, ck, q, k, v, do
+
+
+def test_packed_mask_brute_force():
+    cq, ck = [0, 3, 3, 7], [0, 2, 5, 9]
+    for causal, wl, wr in ((False, -1, -1), (True, -1, -1), (True, 1, -1), (False, 0, 2)):
+        m = packed_visibility_mask(cq, ck, causal, wl, wr)
+        for r in range(7):
+            for c in range(9):
+                bq = max(b for b in range(3) if cq[b] <= r and r < cq[b + 1])
+                bk = max(b for b in range(3) if ck[b] <= c and c < ck[b + 1])
+                i, j = r - cq[bq], c - ck[bk]
+                ok = bq == bk and (not causal or j <= i) and (wl < 0 or j >= i - wl) \
+                    and (wr < 0 or j <= i + wr)
+                assert m[r, c] == ok, (r, c)
+    seq, pos = packed_positions([0, 2, 2, 5])
+    assert seq.tolist() == [0, 0, 2, 2, 2] and pos.tolist() == [0, 1, 0, 1, 2]
+
+
+@pytest.mark.parametrize("kw", [dict(causal=True), dict(causal=False),
+                                dict(causal=True, window_left=2),
+                                dict(causal=False, t5_table=True),
+                                dict(causal=True, alibi=True)])
+def test_packed_equals_each_sequence_alone(kw):
+    # The packed reading reduces to the pinned dense oracle run on each
+    # sequence by itself (positions from 0), including an empty sequence, a
+    # single-row one and sequences of keys longer / shorter than the queries.
+    lq, lk = [5, 0, 1, 9, 4], [5, 0, 3, 9, 2]
+    cq, ck, q, k, v, do = _packed(lq, lk)
+    extra = dict(kw)
+    if extra.pop("t5_table", False):
+        extra["t5_table"] = rnd((32, 4), 9)
+    if extra.pop("alibi", False):
+        extra["alibi_slopes"] = np.array([0.5, 0.25, 0.125, 0.0625])
+    O, LSE = attention_forward_packed(q, k, v, cq, ck, **extra)
+    dQ, dK, dV = attention_backward_packed(q, k, v, do, cq, ck, **extra)
+    for b in range(len(lq)):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0:
+            continue
+        if k1 == k0:
+            assert (O[q0:q1] == 0).all() and np.isneginf(LSE[:, q0:q1]).all()
+            continue
+        Ob, Lb = attention_forward(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], **extra)
+        gq, gk, gv = attention_backward(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1],
+                                        do[None, q0:q1], **extra)
+        assert np.allclose(O[q0:q1], Ob[0], atol=1e-12)
+        assert np.allclose(LSE[:, q0:q1], Lb[0], atol=1e-12)
+        assert np.allclose(dQ[q0:q1], gq[0], atol=1e-11)
+        assert np.allclose(dK[k0:k1], gk[0], atol=1e-11)
+        assert np.allclose(dV[k0:k1], gv[0], atol=1e-11)
+
+
+def test_packed_sequences_do_not_see_each_other():
+    cq, ck, q, k, v, do = _packed([6, 4, 7], [6, 4, 7])
+    O0, _ = attention_forward_packed(q, k, v, cq, ck, causal=True)
+    g0 = attention_backward_packed(q, k, v, do, cq, ck, causal=True)
+    k2, v2 = k.copy(), v.copy()
+    k2[ck[1]:ck[2]] += 5.0          # change every key and value of the middle sequence
+    v2[ck[1]:ck[2]] -= 3.0
+    O1, _ = attention_forward_packed(q, k2, v2, cq, ck, causal=True)
+    g1 = attention_backward_packed(q, k2, v2, do, cq, ck, causal=True)
+    for lo, hi in ((cq[0], cq[1]), (cq[2], cq[3])):
+        assert np.array_equal(O0[lo:hi], O1[lo:hi])
+        assert np.array_equal(g0[0][lo:hi], g1[0][lo:hi])
+    assert not np.allclose(O0[cq[1]:cq[2]], O1[cq[1]:cq[2]])
+
+
+def test_packed_gradients_central_differences():
+    cq, ck, q, k, v, do = _packed([3, 2], [2, 4], Hq=2, Hkv=1, d=3, seed=4)
+    kw = dict(causal=False, t5_table=rnd((8, 2), 5), t5_num_buckets=8, t5_max_distance=20)
+
+    def loss(q_, k_, v_):
+        O, _ = attention_forward_packed(q_, k_, v_, cq, ck, **kw)
+        return float(np.sum(O * do))
+    dQ, dK, dV = attention_backward_packed(q, k, v, do, cq, ck, **kw)
+    h = 1e-6
+    for arr, grad, which in ((q, dQ, 0), (k, dK, 1), (v, dV, 2)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a = [q.copy(), k.copy(), v.copy()]
+            a[which][idx] += h
+            up = loss(*a)
+            a[which][idx] -= 2 * h
+            num[idx] = (up - loss(*a)) / (2 * h)
+        assert np.allclose(grad, num, rtol=1e-6, atol=1e-8), which

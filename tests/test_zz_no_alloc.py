@@ -1,9 +1,10 @@
 """The allocation-free backward entry point, sdpa_bwd_noalloc, for callers
 that cannot allocate device memory around the call (kernel hosts that hand a
 library only its inputs and outputs, processes under a hard memory cap,
-latency-bound loops that avoid cudaMalloc / cudaFree).  Its D-vector scratch
-is a fixed array inside the library instead of a caller workspace; its
-results must match sdpa_bwd's, call after call.
+latency-bound loops that avoid cudaMalloc / cudaFree).  Its workspace (the
+D vector, the dQ turn counters and the dQ accumulator) is a fixed array
+inside the library instead of caller memory; its results must match
+sdpa_bwd's bit for bit, call after call.
 
 Kept in its own file, named to be collected last.
 """
@@ -13,7 +14,8 @@ import torch
 
 from gpu_helpers import ATOL, RTOL
 from scaled_dot_product_bwd_b200 import SdpaError, sdpa_bwd, sdpa_bwd_noalloc, sdpa_fwd
-from scaled_dot_product_bwd_b200.binding import NOALLOC_MAX_ROWS
+from scaled_dot_product_bwd_b200 import sdpa_bwd_workspace_size
+from scaled_dot_product_bwd_b200.binding import NOALLOC_SCRATCH_BYTES
 from scaled_dot_product_bwd_b200.inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -56,9 +58,10 @@ def test_noalloc_matches_workspace_entry_point_twice(kw):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     dev = torch.device("cuda")
-    L = NOALLOC_MAX_ROWS // 2 + 8          # B * Hq * L > max with B = 1, Hq = 2
+    L = 40000                              # workspace ~ 2 * 40000 * 65 * 4 bytes > 16 MiB
     q = torch.zeros(1, L, 2, 64, device=dev, dtype=torch.bfloat16)
     k = torch.zeros(1, L, 1, 64, device=dev, dtype=torch.bfloat16)
+    assert sdpa_bwd_workspace_size(q, k) > NOALLOC_SCRATCH_BYTES
     lse = torch.zeros(1, 2, L, device=dev)
     with pytest.raises(SdpaError) as e:
         sdpa_bwd_noalloc(q, k, k, q, q, lse, torch.empty_like(q), torch.empty_like(k),
