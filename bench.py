@@ -51,6 +51,13 @@ CONFIGS = {
     "mistral4k_small": dict(B=2, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1,
                             bias="none"),
 }
+# The head-sharing and sequence-length sweep, forward only: Hq 32, d 128,
+# causal, Hkv 32 (MHA) / 8 (GQA) / 1 (MQA), B * L = 32768 tokens.
+for _hkv, _tag in ((32, "mha"), (8, "gqa"), (1, "mqa")):
+    for _L in (512, 2048, 8192, 16384):
+        CONFIGS[f"sweep_{_tag}_{_L}"] = dict(B=32768 // _L, Hq=32, Hkv=_hkv, L=_L, d=128,
+                                             causal=True, wl=-1, wr=-1, bias="none",
+                                             fwd_only=True)
 
 # DRAM bytes per launch of a kernel (dram__bytes_read.sum + dram__bytes_write.sum
 # from one ncu capture, divided by the captured batch size), keyed by workload
@@ -95,8 +102,9 @@ def describe(c):
     mask = "causal" if c["causal"] else "bidirectional"
     if c["wl"] >= 0:
         mask += f" window_left={c['wl']}"
+    fwd = ", forward only" if c.get("fwd_only") else ""
     return (f"B={c['B']} Hq={c['Hq']} Hkv={c['Hkv']} L={c['L']} d={c['d']} {mask} "
-            f"bias={c['bias']}")
+            f"bias={c['bias']}{fwd}")
 
 
 def visible_pairs(L, causal, wl, wr):
@@ -116,6 +124,19 @@ def flop_counts(c):
     heads = c["B"] * c["Hq"]
     d = c["d"]
     return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads)
+
+
+def kernel_bytes(c):
+    """Algorithmic HBM bytes of one launch of each kernel: every input read
+    once and every output written once (bf16 tensors, fp32 LSE / D / bias)."""
+    B, L, Hq, Hkv, d = c["B"], c["L"], c["Hq"], c["Hkv"], c["d"]
+    q = B * L * Hq * d * 2
+    kv = B * L * Hkv * d * 2
+    vec = B * Hq * L * 4
+    bias = B * Hq * L * L * 4 if c["bias"] == "dense" else 0
+    return {"fwd": q + 2 * kv + q + vec + bias,
+            "bwd_preprocess": 2 * q + vec,
+            "bwd": q + 2 * kv + q + 2 * vec + bias + q + 2 * kv}
 
 
 def load_peaks():
@@ -183,36 +204,62 @@ def make_case(c, seed):
 
 
 # ------------------------------------------------------------------ oracle
-def oracle_sample(c, inp):
-    """fwd + bwd of the oracle on batch 0, KV head 0 (all its query heads)."""
+def oracle_plan(c):
+    """Bounded sample of a workload for the float64 oracle: batch 0, KV head 0
+    and `heads` of its query heads; for a forward-only workload longer than
+    2048, an evenly spaced set of 1024 query rows (the oracle then forms only
+    those rows of S).  The sample's effective FLOPs count its unmasked pairs."""
+    G = c["Hq"] // c["Hkv"]
+    L = c["L"]
+    fwd_only = c.get("fwd_only", False)
+    heads = min(G, 2) if fwd_only else (G if L <= 4096 else 1)
+    rows = None
+    if fwd_only and L > 2048:
+        rows = np.unique(np.linspace(0, L - 1, 1024).astype(np.int64))
+    return heads, rows
+
+
+def oracle_sample(c, inp, rows):
+    """fwd (+ bwd) of the oracle on the sample's slice of the workload."""
     from oracle import attention_backward, attention_forward
     kw = dict(causal=c["causal"], window_left=c["wl"], window_right=c["wr"],
-              bias=inp.bias, t5_table=inp.t5_table, alibi_slopes=inp.alibi_slopes,
-              batches=[0], kv_heads=[0])
-    attention_forward(inp.q, inp.k, inp.v, **kw)
-    attention_backward(inp.q, inp.k, inp.v, inp.do, **kw)
+              bias=inp.bias, t5_table=inp.t5_table, alibi_slopes=inp.alibi_slopes)
+    attention_forward(inp.q, inp.k, inp.v, query_rows=rows, **kw)
+    if not c.get("fwd_only", False):
+        attention_backward(inp.q, inp.k, inp.v, inp.do, **kw)
 
 
-def sample_inputs(c, seed):
-    """The sample's slice of the workload: batch 0, KV head 0 and its query heads."""
-    G = c["Hq"] // c["Hkv"]
-    sc = dict(c, B=1, Hq=G, Hkv=1)
-    return sc, make_case(sc, seed)
+def sample_pairs(c, rows):
+    """Unmasked (i, j) pairs of the sampled query rows of one head."""
+    L = c["L"]
+    i = np.arange(L, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    lo = np.maximum(0, i - c["wl"]) if c["wl"] >= 0 else np.zeros_like(i)
+    hi = np.full_like(i, L - 1)
+    if c["causal"]:
+        hi = np.minimum(hi, i)
+    if c["wr"] >= 0:
+        hi = np.minimum(hi, i + c["wr"])
+    return int(np.maximum(0, hi - lo + 1).sum())
 
 
 def time_oracle(c, steps, warmup):
-    sc, inp = sample_inputs(c, 0)
-    flops = flop_counts(sc)
-    total = flops["fwd"] + flops["bwd"]
+    heads, rows = oracle_plan(c)
+    sc = dict(c, B=1, Hq=heads, Hkv=1)
+    inp = make_case(sc, 0)
+    per = 4 if c.get("fwd_only", False) else 14
+    total = per * c["d"] * sample_pairs(c, rows) * heads
     for _ in range(warmup):
-        oracle_sample(sc, inp)
+        oracle_sample(sc, inp, rows)
     t0 = time.perf_counter()
     for _ in range(steps):
-        oracle_sample(sc, inp)
+        oracle_sample(sc, inp, rows)
     dt = (time.perf_counter() - t0) / steps
     cores = len(os.sched_getaffinity(0))
-    sample = (f"batch 0, KV head 0 with its {sc['Hq']} query heads of {describe(c)}; "
-              f"float64 numpy, explicit L x L matrices")
+    what = "fwd" if c.get("fwd_only", False) else "fwd + bwd"
+    rows_txt = "all query rows" if rows is None else f"{len(rows)} evenly spaced query rows"
+    sample = (f"{what} of batch 0, KV head 0 with {heads} of its query heads, {rows_txt}, "
+              f"of {describe(c)}; float64 numpy, explicit score matrices; effective FLOPs of "
+              f"the sample's unmasked pairs")
     return dict(value=total / dt / 1e12, seconds_per_sample=dt, cores=cores, sample=sample,
                 flops=total)
 
@@ -287,12 +334,17 @@ def run_gpu(args, c):
     ws = torch.empty(sdpa_bwd_workspace_size(q, k), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
 
+    fwd_only = c.get("fwd_only", False)
+    names = ["fwd"] if fwd_only else ["fwd", "bwd_preprocess", "bwd"]
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
         sdpa_fwd(q, k, v, out=o, lse=lse, **kw)
         if ev is not None:
             ev[1].record(stream)
+        if fwd_only:
+            return
         sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws,
                  phases=BWD_PREPROCESS, **kw)
         if ev is not None:
@@ -308,7 +360,8 @@ def run_gpu(args, c):
         raise RuntimeError("device status reports a timed-out wait during warm-up")
 
     # ---------------- timed region: K steps, device-timed, max over ranks
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+           for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -324,7 +377,8 @@ def run_gpu(args, c):
         dist.barrier()
     clocks = sampler.stop()
     ms_total = start.elapsed_time(end)
-    phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(3)]
+    phase_ms = [statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i in range(len(names))]
     ms_total = max_over_ranks(ms_total, dev)
     status = sdpa_read_device_status()
 
@@ -337,8 +391,11 @@ def run_gpu(args, c):
     hq_, hk_, hv_, hdo_ = (t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.do))
     ho, hlse = torch.empty_like(hq_).pin_memory(), torch.empty(lse.shape).pin_memory()
     hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq_, hk_, hv_))
-    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo_))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+    ups = (("q", hq_), ("k", hk_), ("v", hv_)) + (() if fwd_only else (("do", hdo_),))
+    downs = ((ho, "o"), (hlse, "lse")) + (() if fwd_only else ((hdq, "dq"), (hdk, "dk"),
+                                                               (hdv, "dv")))
+    h2d = sum(h.numel() * h.element_size() for _, h in ups)
+    d2h = sum(h.numel() * h.element_size() for h, _ in downs)
     sets = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)]
     sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
     s_up, s_cmp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
@@ -351,7 +408,7 @@ def run_gpu(args, c):
             with torch.cuda.stream(s_up):
                 if s_i >= 2:
                     s_up.wait_event(cmp_done[x])  # step s-2 is done reading these inputs
-                for d_, h in (("q", hq_), ("k", hk_), ("v", hv_), ("do", hdo_)):
+                for d_, h in ups:
                     S[d_].copy_(h, non_blocking=True)
                 up_done[x].record(s_up)
             with torch.cuda.stream(s_cmp):
@@ -359,12 +416,13 @@ def run_gpu(args, c):
                 if s_i >= 2:
                     s_cmp.wait_event(down_done[x])  # step s-2's results are copied out
                 sdpa_fwd(S["q"], S["k"], S["v"], out=S["o"], lse=S["lse"], **kw)
-                sdpa_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], dq=S["dq"],
-                         dk=S["dk"], dv=S["dv"], workspace=S["ws"], **kw)
+                if not fwd_only:
+                    sdpa_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], dq=S["dq"],
+                             dk=S["dk"], dv=S["dv"], workspace=S["ws"], **kw)
                 cmp_done[x].record(s_cmp)
             with torch.cuda.stream(s_down):
                 s_down.wait_event(cmp_done[x])
-                for h, d_ in ((ho, "o"), (hlse, "lse"), (hdq, "dq"), (hdk, "dk"), (hdv, "dv")):
+                for h, d_ in downs:
                     h.copy_(S[d_], non_blocking=True)
                 down_done[x].record(s_down)
 
@@ -383,26 +441,37 @@ def run_gpu(args, c):
     e2e_ms = max_over_ranks(e2e_ms, dev)
 
     fl = flop_counts(c)
-    step_flops = fl["fwd"] + fl["bwd"]
+    step_flops = fl["fwd"] + (0 if fwd_only else fl["bwd"])
     ms_step = ms_total / args.steps
     value = whole_job_tflops(world, step_flops, ms_step)
     peaks = load_peaks()
+    peak_src = ("measured bf16 burst / copy bandwidth (MEASURED_PEAKS.json)"
+                if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s, 6.65 TB/s")
 
-    # dominant kernel by mean duration; its algorithmic FLOPs per launch
-    names = ["fwd", "bwd_preprocess", "bwd"]
-    algo = {"fwd": fl["fwd"], "bwd": fl["bwd"]}
-    dom = max(range(3), key=lambda i: phase_ms[i])
-    dname = names[dom]
-    roofline = None
-    if dname in algo:
-        ach = algo[dname] / (phase_ms[dom] * 1e-3) / 1e12
-        roofline = {"kernel": dname, "bound": "tensor", "achieved": round(ach, 1),
-                    "peak": peaks["tflops"], "unit": "TFLOP/s",
-                    "frac": round(ach / peaks["tflops"], 4),
-                    "traffic": traffic_per_launch(args.config, dname, c["B"]),
-                    "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"
-                    if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
-                    "flops_per_launch": algo[dname], "ms_per_launch": round(phase_ms[dom], 4)}
+    # Per kernel: algorithmic FLOPs and HBM bytes per launch against the mean
+    # event time, as fractions of the tensor and HBM peaks.  The roofline
+    # object is the dominant kernel's, bound by whichever roof is nearer.
+    algo = {"fwd": fl["fwd"], "bwd_preprocess": 0, "bwd": fl["bwd"]}
+    nbytes = kernel_bytes(c)
+    kernels = {}
+    for n, t in zip(names, phase_ms):
+        tf = algo[n] / (t * 1e-3) / 1e12
+        gbs = nbytes[n] / (t * 1e-3) / 1e9
+        kernels[n] = {"ms": round(t, 4), "tflops": round(tf, 1),
+                      "frac_tensor": round(tf / peaks["tflops"], 4), "gbs": round(gbs, 1),
+                      "frac_hbm": round(gbs / peaks["hbm"], 4), "flops": algo[n],
+                      "bytes": nbytes[n]}
+    dname = max(kernels, key=lambda n: kernels[n]["ms"])
+    kd = kernels[dname]
+    hbm_bound = kd["frac_hbm"] > kd["frac_tensor"]
+    roofline = {"kernel": dname, "bound": "hbm" if hbm_bound else "tensor",
+                "achieved": kd["gbs"] if hbm_bound else kd["tflops"],
+                "peak": peaks["hbm"] if hbm_bound else peaks["tflops"],
+                "unit": "GB/s" if hbm_bound else "TFLOP/s",
+                "frac": kd["frac_hbm"] if hbm_bound else kd["frac_tensor"],
+                "traffic": traffic_per_launch(args.config, dname, c["B"]),
+                "peak_source": peak_src, "flops_per_launch": kd["flops"],
+                "bytes_per_launch": kd["bytes"], "ms_per_launch": kd["ms"]}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -414,14 +483,16 @@ def run_gpu(args, c):
                    "l2": "inputs larger than L2: no flush between steps",
                    "flops_per_step": step_flops, "unmasked_pairs_per_head": fl["P"]},
         "pct_of_peak": round(100 * value / world / peaks["tflops"], 2),
-        "value_strict": round(world * (fl["fwd"] + fl["bwd_strict"]) / (ms_step * 1e-3) / 1e12, 2),
+        "value_strict": round(world * (fl["fwd"] + (0 if fwd_only else fl["bwd_strict"]))
+                              / (ms_step * 1e-3) / 1e12, 2),
         "kernel_ms": {n: round(t, 4) for n, t in zip(names, phase_ms)},
+        "kernels": kernels,
         "roofline": roofline,
         "e2e": {"value": round(whole_job_tflops(world, step_flops, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3),
                 "pipelining": "3 streams, 2 device buffer sets: H2D(s+1) | compute(s) | D2H(s-1)"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": len(names) * args.steps,
         "clocks": clocks,
         "device_status": status,
     }

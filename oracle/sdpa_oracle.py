@@ -451,10 +451,11 @@ def attention_forward_packed(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None,
 def attention_backward_packed(q, k, v, do, cu_seqlens_q, cu_seqlens_k, *, scale=None,
                               causal=False, window_left=-1, window_right=-1, t5_table=None,
                               t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
-                              alibi_slopes=None):
+                              alibi_slopes=None, return_intermediates=False):
     """dQ [total_q, Hq, d], dK and dV [total_k, Hkv, d] of sum(O * dO) for a
     packed batch, by the chain rule over the packed axis (as in
-    ``attention_backward``)."""
+    ``attention_backward``).  With ``return_intermediates`` also P and dS,
+    each [Hq, total_q, total_k]."""
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
     t5_table, alibi_slopes = _as64(t5_table), _as64(alibi_slopes)
     Tq, Hq, d = q.shape
@@ -467,6 +468,7 @@ def attention_backward_packed(q, k, v, do, cu_seqlens_q, cu_seqlens_k, *, scale=
     dQ = np.zeros(q.shape)
     dK = np.zeros(k.shape)
     dV = np.zeros(v.shape)
+    Ps, dSs = [], []
     for hq in range(Hq):
         g = hq // G
         S = _packed_scores(q, k, hq, G, sc, M, rel, t5_table, t5_num_buckets, t5_max_distance,
@@ -478,4 +480,9 @@ def attention_backward_packed(q, k, v, do, cu_seqlens_q, cu_seqlens_k, *, scale=
         dQ[:, hq, :] = sc * (dS @ k[:, g, :])
         dK[:, g, :] += sc * (dS.T @ q[:, hq, :])
         dV[:, g, :] += P.T @ do[:, hq, :]
+        if return_intermediates:
+            Ps.append(P)
+            dSs.append(dS)
+    if return_intermediates:
+        return dQ, dK, dV, np.stack(Ps), np.stack(dSs)
     return dQ, dK, dV

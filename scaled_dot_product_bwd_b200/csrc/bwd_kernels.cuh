@@ -16,7 +16,7 @@
 //        dV += P^T dO (TS), dK += dS^T Q (SS), dQ_part = dS K (SS)
 //      dV and dK stay in tensor memory for the whole item.  Each dQ_part is
 //      added into an fp32 accumulator in global memory, the contributions to
-//      one query tile in ascending key-tile order: a turn counter per
+//      one query tile in descending key-tile order: a turn counter per
 //      (query tile, 32-row quarter) holds the number of key tiles already
 //      added, the first key tile stores, the last one writes
 //      dQ = scale * sum as bf16.  A fixed-order split-K reduction with no
@@ -25,14 +25,15 @@
 //      deterministic when using Flash Attention 2").
 //
 // Work items are handed out by an atomic ticket counter, group by group
-// ((batch, KV head) major) and within a group in ascending key tile, which
-// is also the order of the dQ sums.  A waiting item only waits for items
-// with smaller tickets, all of which are held by CTAs that are running or
-// done, so the waits always end.  Within an item the query tiles run from
-// the last to the first: every key tile of a group then reaches a query tile
-// about as many blocks after its start as the others do, so the key tiles
-// taken earlier -- the earlier contributors -- stay ahead and a turn is
-// usually free when it is needed.
+// ((batch, KV head) major) and within a group from the last key tile to the
+// first, which is also the order of the dQ sums.  A waiting item only waits
+// for items with smaller tickets, all of which are held by CTAs that are
+// running or done, so the waits always end.  Within an item the query tiles
+// run from the first of its band to the last, every head of the group at
+// each: under a causal or windowed mask key tile n + 1 then reaches each
+// query tile G blocks before key tile n does, so the contributions to a
+// tile arrive spaced out and in order, and a turn is usually free when it
+// is needed.
 #pragma once
 
 #include "attn_common.cuh"
@@ -125,7 +126,7 @@ __device__ __forceinline__ bool wait_turn(const unsigned int* ctr, unsigned int 
   if (__shfl_sync(0xffffffffu, ld_acquire_u32(ctr), 0) == want) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t k = 1;; ++k) {
-    __nanosleep(100);
+    if (k > 32) __nanosleep(64);
     if (__shfl_sync(0xffffffffu, ld_acquire_u32(ctr), 0) == want) return true;
     if ((k & 255u) == 0) {
       const bool stop = *ctl.abort || (globaltimer_ns() - t0 > ctl.limit_ns);
@@ -212,8 +213,8 @@ struct BwdLayout {
 
 // Registers per thread after the warpgroups reallocate (launched with 128
 // each, 512 threads = 65536): compute warpgroups, reducer, producer/issuers.
-// 2 x 128 + 184 + 72 = 512 = 4 x 128 (ptxas -v: no spills at d = 64).
-constexpr uint32_t kRegsCompute = 128, kRegsReducer = 184, kRegsIssue = 72;
+// 2 x 152 + 128 + 80 = 512 = 4 x 128.
+constexpr uint32_t kRegsCompute = 152, kRegsReducer = 128, kRegsIssue = 80;
 static_assert(2 * kRegsCompute + kRegsReducer + kRegsIssue == 4 * 128, "register split");
 
 template <int D, int BIAS, bool DS_OUT>
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(512, 1)
   auto item_at = [&](int t) {
     Item w;
     const int grp = t / ntk;
-    w.n = t - grp * ntk;
+    w.n = ntk - 1 - (t - grp * ntk);  // key tiles of a group from the last to the first
     w.b = grp / p.Hkv;
     w.g = grp - w.b * p.Hkv;
     w.s = seq_view(p, w.b);
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(512, 1)
         // loaded one block ahead of the slot they go to.
         float l2v[4], ddv[4];
         auto load_vec = [&](int blk) {
-          const int mi = w.mhi - 1 - blk / p.G;
+          const int mi = w.mlo + blk / p.G;
           const int hq = w.g * p.G + blk % p.G;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(512, 1)
         };
         load_vec(0);
         for (int blk = 0; blk < w.nb; ++blk, ++i) {
-          const int mi = w.mhi - 1 - blk / p.G;
+          const int mi = w.mlo + blk / p.G;
           const int hq = w.g * p.G + blk % p.G;
           const int x = i & 1;
           if (lane == 0) {
@@ -579,6 +580,56 @@ __global__ void __launch_bounds__(512, 1)
     const int rq = warp - 8;
     const uint32_t lane_bits = static_cast<uint32_t>(rq * 32) << 16;
     const bool odd = (lane & 1) != 0;
+    const int co = odd ? 4 : 0;  // this lane's columns in each group of 8
+    // One block's share of the reduction: its query tile's place in the key
+    // tiles' order (idx, first, last) and which of this lane's two rows exist.
+    struct Red {
+      unsigned int idx;
+      int mi, hq;
+      bool first, last, va, vb;
+    };
+    auto red_at = [&](const Item& w, int blk) {
+      Red r;
+      r.mi = w.mlo + blk / p.G;
+      r.hq = w.g * p.G + blk % p.G;
+      int nlo, nhi;
+      key_tile_range(p, w.s.Lq, w.s.Lk, r.mi * kTile, kTile, nlo, nhi);
+      // key tiles add in descending order: nhi - 1 first, nlo last
+      r.idx = static_cast<unsigned int>(nhi - 1 - w.n);
+      r.first = r.idx == 0;
+      r.last = w.n == nlo;
+      const int ra = r.mi * kTile + rq * 32 + (lane & ~1);  // the lane pair's first row
+      r.va = ra < w.s.Lq;
+      r.vb = ra + 1 < w.s.Lq;
+      return r;
+    };
+    auto ctr_of = [&](const Item& w, const Red& r) {
+      return p.turns + ((static_cast<int64_t>(w.b) * p.Hq + r.hq) * ntq + r.mi) * 4 + rq;
+    };
+    auto acc_of = [&](const Item& w, const Red& r) {
+      return p.dq_acc + row_index(p, w.s, w.b, r.hq, r.mi * kTile + rq * 32 + (lane & ~1)) * D + co;
+    };
+    // This lane's running sums of one 64-column half of the block's two
+    // rows: group g (8 columns) of the half at [2g] (row a) and [2g + 1].
+    float4 old[16];
+    auto load_half = [&](const Item& w, const Red& r, int half) {
+      if (r.first) return;
+      const float* acc_a = acc_of(w, r) + 64 * half;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        old[2 * g] = r.va ? __ldcg(reinterpret_cast<const float4*>(acc_a + 8 * g))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        old[2 * g + 1] = r.vb ? __ldcg(reinterpret_cast<const float4*>(acc_a + D + 8 * g))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    // wait for the block's turn, then fetch the first half's running sums
+    auto fetch = [&](const Item& w, const Red& r) -> bool {
+      if (r.first) return true;
+      if (!wait_turn(ctr_of(w, r), r.idx, ctl)) return false;
+      load_half(w, r, 0);
+      return true;
+    };
     bool ok = true;
     int i = 0, k = 0;
     while (true) {
@@ -588,82 +639,77 @@ __global__ void __launch_bounds__(512, 1)
       if (t < 0) break;
       const Item w = item_at(t);
       if (w.nb == 0) continue;
+      Red cur = red_at(w, 0);
+      if (!(ok = fetch(w, cur))) break;
       for (int blk = 0; blk < w.nb; ++blk, ++i) {
-        const int mi = w.mhi - 1 - blk / p.G;
-        const int hq = w.g * p.G + blk % p.G;
-        int nlo, nhi;
-        key_tile_range(p, w.s.Lq, w.s.Lk, mi * kTile, kTile, nlo, nhi);
-        const unsigned int idx = static_cast<unsigned int>(w.n - nlo);
-        const bool first = idx == 0;
-        const bool last = (w.n == nhi - 1);
-        const int ra = mi * kTile + rq * 32 + (lane & ~1);  // the pair's first row
-        const bool va = ra < w.s.Lq, vb = ra + 1 < w.s.Lq;
-        const int co = odd ? 4 : 0;                          // this lane's columns in each 8
-        float* acc_a = p.dq_acc + row_index(p, w.s, w.b, hq, ra) * D + co;
-        float* acc_b = acc_a + D;
-        unsigned int* ctr =
-            p.turns + ((static_cast<int64_t>(w.b) * p.Hq + hq) * ntq + mi) * 4 + rq;
-        float4 old[D / 4];  // group g: [2g] row a, [2g + 1] row b
-        if (!first) {
-          if (!(ok = wait_turn(ctr, idx, ctl))) break;
-#pragma unroll
-          for (int g = 0; g < D / 8; ++g) {
-            old[2 * g] = va ? __ldcg(reinterpret_cast<const float4*>(acc_a + 8 * g))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-            old[2 * g + 1] = vb ? __ldcg(reinterpret_cast<const float4*>(acc_b + 8 * g))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
         ok = mbar_wait(dq_full(i & 1), (i >> 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
         const uint32_t tq =
             tmem + lane_bits + (Lay::kDQShared ? Lay::kDPCol : Lay::kDQCol + D * (i & 1));
+        float* acc_a = acc_of(w, cur);
         __nv_bfloat16* dq_a = p.dq + static_cast<int64_t>(w.b) * p.sq_b +
-                              static_cast<int64_t>(w.s.q0 + ra) * p.sq_l +
-                              static_cast<int64_t>(hq) * p.sq_h + co;
-        __nv_bfloat16* dq_b = dq_a + p.sq_l;
+                              static_cast<int64_t>(w.s.q0 + cur.mi * kTile + rq * 32 + (lane & ~1)) * p.sq_l +
+                              static_cast<int64_t>(cur.hq) * p.sq_h + co;
 #pragma unroll
-        for (int c = 0; c < D; c += 16) {
-          uint32_t v[16];
-          tmem_ld16_sync(tq + c, v);
-          if (c + 16 == D) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dq_free(i & 1));  // the partial is out of tensor memory
-          }
+        for (int half = 0; half < D / 64; ++half) {
+          // at d = 128 the second half's running sums come once the first
+          // half's are spent (registers), while the partial is still held
+          if (half > 0) load_half(w, cur, half);
 #pragma unroll
-          for (int g4 = 0; g4 < 2; ++g4) {
-            const int g = c / 8 + g4;
-            const float4 lo = make_float4(__uint_as_float(v[8 * g4]), __uint_as_float(v[8 * g4 + 1]),
-                                          __uint_as_float(v[8 * g4 + 2]), __uint_as_float(v[8 * g4 + 3]));
-            const float4 hi = make_float4(__uint_as_float(v[8 * g4 + 4]), __uint_as_float(v[8 * g4 + 5]),
-                                          __uint_as_float(v[8 * g4 + 6]), __uint_as_float(v[8 * g4 + 7]));
-            // the even lane sends its columns 4..7, the odd lane its 0..3
-            const float4 got = shfl_xor_f4(odd ? lo : hi, 1);
-            float4 sa = odd ? got : lo;  // row a, columns co..co+3 of group g
-            float4 sbv = odd ? hi : got; // row b
-            if (!first) {
-              sa = f4_add(old[2 * g], sa);
-              sbv = f4_add(old[2 * g + 1], sbv);
+          for (int c = 0; c < 64; c += 16) {
+            uint32_t v[16];
+            tmem_ld16_sync(tq + 64 * half + c, v);
+            if (half + 1 == D / 64 && c + 16 == 64) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(dq_free(i & 1));  // the partial is out of tensor memory
             }
-            if (last) {
-              const float sc = p.scale;
-              const uint2 pa = make_uint2(pack_bf16x2(sa.x * sc, sa.y * sc), pack_bf16x2(sa.z * sc, sa.w * sc));
-              const uint2 pb = make_uint2(pack_bf16x2(sbv.x * sc, sbv.y * sc), pack_bf16x2(sbv.z * sc, sbv.w * sc));
-              if (va) *reinterpret_cast<uint2*>(dq_a + 8 * g) = pa;
-              if (vb) *reinterpret_cast<uint2*>(dq_b + 8 * g) = pb;
-            } else {
-              if (va) __stcg(reinterpret_cast<float4*>(acc_a + 8 * g), sa);
-              if (vb) __stcg(reinterpret_cast<float4*>(acc_b + 8 * g), sbv);
+#pragma unroll
+            for (int g2 = 0; g2 < 2; ++g2) {
+              const int g = c / 8 + g2;        // group of the half
+              const int col = 64 * half + 8 * g;
+              const float4 lo = make_float4(__uint_as_float(v[8 * g2]), __uint_as_float(v[8 * g2 + 1]),
+                                            __uint_as_float(v[8 * g2 + 2]), __uint_as_float(v[8 * g2 + 3]));
+              const float4 hi = make_float4(__uint_as_float(v[8 * g2 + 4]), __uint_as_float(v[8 * g2 + 5]),
+                                            __uint_as_float(v[8 * g2 + 6]), __uint_as_float(v[8 * g2 + 7]));
+              // the even lane sends its columns 4..7, the odd lane its 0..3
+              const float4 got = shfl_xor_f4(odd ? lo : hi, 1);
+              float4 sa = odd ? got : lo;   // row a, columns col + co ..
+              float4 sbv = odd ? hi : got;  // row b
+              if (!cur.first) {
+                sa = f4_add(old[2 * g], sa);
+                sbv = f4_add(old[2 * g + 1], sbv);
+              }
+              if (cur.last) {
+                const float sc = p.scale;
+                const uint2 pa = make_uint2(pack_bf16x2(sa.x * sc, sa.y * sc), pack_bf16x2(sa.z * sc, sa.w * sc));
+                const uint2 pb = make_uint2(pack_bf16x2(sbv.x * sc, sbv.y * sc), pack_bf16x2(sbv.z * sc, sbv.w * sc));
+                if (cur.va) *reinterpret_cast<uint2*>(dq_a + col) = pa;
+                if (cur.vb) *reinterpret_cast<uint2*>(dq_a + p.sq_l + col) = pb;
+              } else {
+                if (cur.va) __stcg(reinterpret_cast<float4*>(acc_a + col), sa);
+                if (cur.vb) __stcg(reinterpret_cast<float4*>(acc_a + D + col), sbv);
+              }
             }
           }
         }
-        if (!last) {
+        // The next block of the item is another query tile (or head), whose
+        // turn only ever waits on key tiles handed out earlier: take it and
+        // start its loads before passing this block's turn on, so their
+        // latencies overlap.
+        unsigned int* ctr = ctr_of(w, cur);
+        const unsigned int pass = cur.idx + 1u;
+        const bool release = !cur.last;
+        if (blk + 1 < w.nb) {
+          cur = red_at(w, blk + 1);
+          if (!(ok = fetch(w, cur))) break;
+        }
+        if (release) {
           __threadfence();
           __syncwarp();
-          if (lane == 0) st_release_u32(ctr, idx + 1u);
+          if (lane == 0) st_release_u32(ctr, pass);
         }
       }
       if (!ok) break;
@@ -693,7 +739,7 @@ __global__ void __launch_bounds__(512, 1)
       const int j = n0 + row;  // this thread's key
       for (int blk = 0; blk < w.nb; ++blk, ++i) {
         const int x = i & 1;
-        const int mi = w.mhi - 1 - blk / p.G;
+        const int mi = w.mlo + blk / p.G;
         const int hq = w.g * p.G + blk % p.G;
         const int m0 = mi * kTile + c0w;  // first query of this warpgroup's columns
         const float* lut_row = nullptr;
@@ -730,7 +776,7 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         const float* lse2 = vec + x * 2 * kTile + c0w;
         const float* dvv = vec + x * 2 * kTile + kTile + c0w;
-        uint32_t pr[64];  // S^T row, then P^T (fp32 bits), then dS (DS_OUT)
+        uint32_t pr[64];  // S^T row, then P^T (fp32 bits)
         tmem_ld64_sync(tS, pr);
         const float4* lse4 = reinterpret_cast<const float4*>(lse2);
         if (full) {
@@ -784,14 +830,20 @@ __global__ void __launch_bounds__(512, 1)
         if (i > 0) ok = mbar_wait(ds_free, (i - 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+        float* ds_dst = nullptr;  // DS_OUT: fp32 dS of (query m0 + c, key j)
+        if constexpr (DS_OUT) {
+          if (j < Lk)
+            ds_dst = p.ds_out + static_cast<int64_t>(w.b) * p.sd_b +
+                     static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(m0) * p.sd_i + j;
+        }
 #pragma unroll
-        for (int cc = 0; cc < kBlk; cc += 32) {
-          uint32_t dr[32];
-          tmem_ld32_sync(tDP + cc, dr);
+        for (int cc = 0; cc < kBlk; cc += 16) {
+          uint32_t dr[16];
+          tmem_ld16_sync(tDP + cc, dr);
           const float4* d4v = reinterpret_cast<const float4*>(dvv + cc);
-          uint32_t pk[16];  // dS as bf16 pairs, queries cc..cc+31
+          uint32_t pk[8];  // dS as bf16 pairs, queries cc..cc+15
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
+          for (int c = 0; c < 16; c += 4) {
             const float4 dv4 = d4v[c >> 2];
             const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dv4.x);
             const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dv4.y);
@@ -799,20 +851,26 @@ __global__ void __launch_bounds__(512, 1)
             const float d3 = __uint_as_float(pr[cc + c + 3]) * (__uint_as_float(dr[c + 3]) - dv4.w);
             pk[c >> 1] = pack_bf16x2(d0, d1);
             pk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
-            if constexpr (DS_OUT) {  // P is spent: keep the fp32 dS in its place
-              pr[cc + c] = __float_as_uint(d0);
-              pr[cc + c + 1] = __float_as_uint(d1);
-              pr[cc + c + 2] = __float_as_uint(d2);
-              pr[cc + c + 3] = __float_as_uint(d3);
+            if constexpr (DS_OUT) {
+              // neighbouring lanes hold neighbouring keys: each store of the
+              // warp writes 128 contiguous bytes of one query row; masked
+              // and out-of-range entries are 0 (P = 0); rows past Lq are skipped
+              if (ds_dst) {
+                const float dd[4] = {d0, d1, d2, d3};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (m0 + cc + c + e < Lq)
+                    __stcs(ds_dst + static_cast<int64_t>(cc + c + e) * p.sd_i, dd[e]);
+              }
             }
           }
           // into this thread's row of the 128-byte swizzled dS tile (64
           // queries = 128 bytes): 16-byte chunk q goes to position q ^ (row % 8)
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int q = (cc >> 3) + q4;
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const int q = (cc >> 3) + q2;
             *reinterpret_cast<uint4*>(ds_row + ((q ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                make_uint4(pk[4 * q2], pk[4 * q2 + 1], pk[4 * q2 + 2], pk[4 * q2 + 3]);
           }
         }
         // dP^T is read: at d = 128 the dQ MMA writes those columns next
@@ -820,19 +878,6 @@ __global__ void __launch_bounds__(512, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(ds_full);
         mbar_arrive(vec_empty(x));
-        if constexpr (DS_OUT) {
-          // fp32 dS of (query m0 + c, key j) for this thread's 64 queries;
-          // neighbouring lanes hold neighbouring keys, so every store of the
-          // warp writes 128 contiguous bytes of one query row.  Masked and
-          // out-of-range entries are 0 (P = 0); rows past Lq are not stored.
-          if (j < Lk) {
-            float* dst = p.ds_out + static_cast<int64_t>(w.b) * p.sd_b +
-                         static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(m0) * p.sd_i + j;
-#pragma unroll
-            for (int c = 0; c < kBlk; ++c)
-              if (m0 + c < Lq) __stcs(dst + static_cast<int64_t>(c) * p.sd_i, __uint_as_float(pr[c]));
-          }
-        }
       }
       if (!ok) break;
       // ---------- item epilogue: warpgroup 0 stores dV, warpgroup 1 stores dK ----------

@@ -160,15 +160,18 @@ def fwd_protocol(items, SK, SV, NS=3, bias_ring=False, rng=None):
 def bwd_items(groups, ntk, G, causal):
     """Work items of the fused backward in ticket order: (group, key tile n,
     blocks), each block (query tile m, head) with its dQ turn index, first
-    and last flags -- query tiles from the last to the first, heads inner."""
+    and last flags.  Within a group the key tiles come from the last to the
+    first, and the dQ contributions to a query tile are added in that same
+    (descending) order; an item walks its query tiles from the first of its
+    band up, heads inner."""
     ntq = ntk
     items = []
     for grp in range(groups):
-        for n in range(ntk):
+        for n in range(ntk - 1, -1, -1):
             mlo = n if causal else 0
             blocks = []
-            for m in range(ntq - 1, mlo - 1, -1):
-                contrib = list(range(0, m + 1)) if causal else list(range(ntk))
+            for m in range(mlo, ntq):
+                contrib = list(range(m, -1, -1)) if causal else list(range(ntk - 1, -1, -1))
                 for h in range(G):
                     idx = contrib.index(n)
                     blocks.append(((grp, h, m), idx, idx == 0, idx == len(contrib) - 1))
@@ -324,17 +327,22 @@ def bwd_protocol(items, ctas, SQ, SO, dq_shared, reducers=2):
                     u += 1
 
         def reducer(r, c=c, B=B, consume=consume):
+            # the next block's turn is taken (and its sums fetched) before
+            # this block's turn is passed on
             k = i = 0
             while True:
                 t = yield from consume(k)
                 k += 1
                 if t is None:
                     return
-                for tile, idx, first, last in items[t]:
-                    if not first:
-                        yield ("turn_wait", (tile, r), idx)
+                blocks = items[t]
+                if blocks and not blocks[0][2]:
+                    yield ("turn_wait", (blocks[0][0], r), blocks[0][1])
+                for j, (tile, idx, first, last) in enumerate(blocks):
                     yield ("wait", B(f"dq_full{i & 1}"), (i >> 1) & 1)
                     yield ("arrive", B(f"dq_free{i & 1}"))
+                    if j + 1 < len(blocks) and not blocks[j + 1][2]:
+                        yield ("turn_wait", (blocks[j + 1][0], r), blocks[j + 1][1])
                     if not last:
                         yield ("turn_set", (tile, r), idx + 1)
                     i += 1
@@ -429,8 +437,8 @@ def test_fused_backward_protocol_has_no_deadlock(SQ, SO, dq_shared, causal):
 
 
 def test_fused_backward_turns_follow_key_tile_order():
-    # The dQ contributions to every (query tile, quarter) arrive in ascending
-    # key-tile order: turn indices are consecutive from 0 to the last.
+    # The dQ contributions to every (query tile, quarter) come in the order
+    # the key tiles are handed out: turn indices consecutive from 0.
     items = bwd_items(2, 4, 2, True)
     seen = {}
     for blocks in items:
@@ -443,8 +451,8 @@ def test_fused_backward_turns_follow_key_tile_order():
 
 
 def test_fused_backward_model_catches_a_wrong_turn_order():
-    # Planting a reversed contribution order in the model makes the waits
-    # cycle: the explorer reports the deadlock.
+    # Planting the contribution order opposite to the ticket order in the
+    # model makes the waits cycle: the explorer reports the deadlock.
     items = bwd_items(1, 3, 1, True)
     rev = []
     for blocks in items:
