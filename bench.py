@@ -6,7 +6,10 @@
 A step is one sdpa_fwd + sdpa_bwd over one batch of seeded synthetic inputs
 already resident in HBM.  Effective FLOPs count only unmasked (query, key)
 pairs P per (batch, query head): forward 4 d P, backward 10 d P (the
-recompute of the scores included), 14 d P in total.  With N > 1 (torchrun)
+recompute of the scores included), 14 d P in total.  Per kernel, the
+FLOPs are the matrix products that kernel needs for its own outputs over the
+unmasked pairs: forward 4 d P, dQ 6 d P (S, dP, dQ), dK/dV 8 d P (S, dP, dV,
+dK).  With N > 1 (torchrun)
 every rank runs its own batch (replicas; no collective on the data path) and
 rank 0 prints the whole-job rate: all ranks' FLOPs / the slowest rank's time.
 
@@ -123,7 +126,8 @@ def flop_counts(c):
     P = visible_pairs(c["L"], c["causal"], c["wl"], c["wr"])
     heads = c["B"] * c["Hq"]
     d = c["d"]
-    return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads)
+    return dict(P=P, fwd=4 * d * P * heads, bwd=10 * d * P * heads, bwd_strict=8 * d * P * heads,
+                bwd_dq=6 * d * P * heads, bwd_dkdv=8 * d * P * heads)
 
 
 def kernel_bytes(c):
@@ -136,7 +140,8 @@ def kernel_bytes(c):
     bias = B * Hq * L * L * 4 if c["bias"] == "dense" else 0
     return {"fwd": q + 2 * kv + q + vec + bias,
             "bwd_preprocess": 2 * q + vec,
-            "bwd": q + 2 * kv + q + 2 * vec + bias + q + 2 * kv}
+            "bwd_dq": q + 2 * kv + q + 2 * vec + bias + q,
+            "bwd_dkdv": q + 2 * kv + q + 2 * vec + bias + 2 * kv}
 
 
 def load_peaks():
@@ -306,7 +311,7 @@ def run_gpu(args, c):
     import torch
     import torch.distributed as dist
 
-    from scaled_dot_product_bwd_b200 import (BWD_GRADS, BWD_PREPROCESS, load_library,
+    from scaled_dot_product_bwd_b200 import (BWD_DKDV, BWD_DQ, BWD_PREPROCESS, load_library,
                                              sdpa_bwd, sdpa_bwd_workspace_size, sdpa_fwd,
                                              sdpa_read_device_status)
 
@@ -335,7 +340,7 @@ def run_gpu(args, c):
     stream = torch.cuda.current_stream(dev)
 
     fwd_only = c.get("fwd_only", False)
-    names = ["fwd"] if fwd_only else ["fwd", "bwd_preprocess", "bwd"]
+    names = ["fwd"] if fwd_only else ["fwd", "bwd_preprocess", "bwd_dq", "bwd_dkdv"]
 
     def step(ev=None):
         if ev is not None:
@@ -349,9 +354,12 @@ def run_gpu(args, c):
                  phases=BWD_PREPROCESS, **kw)
         if ev is not None:
             ev[2].record(stream)
-        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_GRADS, **kw)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DQ, **kw)
         if ev is not None:
             ev[3].record(stream)
+        sdpa_bwd(q, k, v, o, do, lse, dq=dq, dk=dk, dv=dv, workspace=ws, phases=BWD_DKDV, **kw)
+        if ev is not None:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -451,7 +459,8 @@ def run_gpu(args, c):
     # Per kernel: algorithmic FLOPs and HBM bytes per launch against the mean
     # event time, as fractions of the tensor and HBM peaks.  The roofline
     # object is the dominant kernel's, bound by whichever roof is nearer.
-    algo = {"fwd": fl["fwd"], "bwd_preprocess": 0, "bwd": fl["bwd"]}
+    algo = {"fwd": fl["fwd"], "bwd_preprocess": 0, "bwd_dq": fl["bwd_dq"],
+            "bwd_dkdv": fl["bwd_dkdv"]}
     nbytes = kernel_bytes(c)
     kernels = {}
     for n, t in zip(names, phase_ms):
@@ -522,11 +531,11 @@ def bias_grad_extra_bytes(c):
 
 def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
-    preprocess and the backward kernel (with dS output), the zero fill of
+    preprocess, the dQ kernel (with dS output) and the dK/dV kernel, the zero fill of
     skipped key tiles under a mask, and the reductions (T5 / ALiBi: diagonal
     sums, their fold and the per-bucket or per-slope sums; a full-shape dense
     bias needs none)."""
-    n = 3
+    n = 4
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1
     if c["bias"] in ("t5", "alibi"):

@@ -183,10 +183,8 @@ sdpa_status_t sdpa_fwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen
 
 /*
  * Bytes of device workspace sdpa_bwd needs for this shape: the per-row
- * D_i = sum_c dO[i,c] O[i,c] vector (float32, one per LSE entry), the dQ
- * turn counters (4 bytes per 32 query rows of each head), and the float32
- * dQ accumulator (d floats per LSE entry), each 256-byte aligned.  Returns 0
- * for an invalid shape.
+ * D_i = sum_c dO[i,c] O[i,c] vector (float32, one per LSE entry), rounded
+ * up to 256 bytes.  Returns 0 for an invalid shape.
  */
 size_t sdpa_bwd_workspace_size(const sdpa_shape* shape, int32_t deterministic);
 size_t sdpa_bwd_varlen_workspace_size(const sdpa_shape* shape, const sdpa_varlen* varlen);
@@ -198,13 +196,13 @@ size_t sdpa_bwd_varlen_workspace_size(const sdpa_shape* shape, const sdpa_varlen
  * print no gradient formulas; these are the chain rule of the forward:
  *   P = exp(S - LSE), dP = dO V^T, D_i = rowsum(dO * O), dS = P (dP - D),
  *   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
- * One kernel computes all three: for each block of 128 keys it walks the
- * query tiles of the mask band and keeps dK and dV on chip; every dQ
- * partial is added into the workspace's float32 accumulator in ascending
- * key-tile order, gated by a turn counter per 32 query rows (a fixed-order
- * split-K sum, no floating-point atomics; HF transformers issue #31787 is
- * the non-determinism this avoids).  The waits for a turn are bounded like
- * every other in-kernel wait.
+ * Three launches: D into the workspace; dQ, one CTA per 128 query rows
+ * summing over the key tiles of the mask band in ascending order on chip;
+ * dK and dV, one CTA per 128 keys summing over the query tiles and the
+ * query heads of its group in a fixed order on chip.  Every sum has a fixed
+ * order and none uses floating-point atomics, so repeated calls give
+ * bit-identical results (HF transformers issue #31787 is the
+ * non-determinism this avoids).
  * deterministic: must be 1 (the only mode built; 0 returns UNSUPPORTED).
  * workspace: device memory of at least sdpa_bwd_workspace_size() bytes,
  * 256-byte aligned, owned by the caller, contents ignored on entry.
@@ -217,16 +215,18 @@ sdpa_status_t sdpa_bwd(const sdpa_shape* shape, const void* q, const void* k,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The backward as its two launches, selected by a bitmask: PREPROCESS
- * writes D = rowsum(dO * O) into the workspace and clears its counters;
- * GRADS writes dQ, dK and dV and needs a PREPROCESS on the same workspace
- * earlier in stream order (once per GRADS launch: the counters it clears are
- * used up).  sdpa_bwd is sdpa_bwd_phases(SDPA_BWD_ALL, ...).  Arguments as
- * sdpa_bwd; phases == 0 or unknown bits -> SDPA_ERR_INVALID_ARG.
+ * The backward as its three launches, selected by a bitmask: PREPROCESS
+ * writes D = rowsum(dO * O) into the workspace; DQ writes dQ and DKDV
+ * writes dK and dV, both reading D, so they need a PREPROCESS on the same
+ * workspace (with the same O and dO) earlier in stream order; D stays valid
+ * for any number of DQ / DKDV launches after it.  sdpa_bwd is
+ * sdpa_bwd_phases(SDPA_BWD_ALL, ...).  Arguments as sdpa_bwd; phases == 0
+ * or unknown bits -> SDPA_ERR_INVALID_ARG.
  */
 #define SDPA_BWD_PREPROCESS 1u
-#define SDPA_BWD_GRADS 2u
-#define SDPA_BWD_ALL 3u
+#define SDPA_BWD_DQ 2u
+#define SDPA_BWD_DKDV 4u
+#define SDPA_BWD_ALL 7u
 sdpa_status_t sdpa_bwd_phases(uint32_t phases, const sdpa_shape* shape, const void* q,
                               const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, const sdpa_bias_desc* bias,
@@ -257,14 +257,14 @@ sdpa_status_t sdpa_bwd_varlen(const sdpa_shape* shape, const sdpa_varlen* varlen
  * lives in a fixed array of SDPA_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into
  * the library, held by every GPU that loads it until the process exits.
  *  - sdpa_bwd_workspace_size(shape) must be <= SDPA_NOALLOC_SCRATCH_BYTES
- *    (about B * Hq * L * (d + 1) * 4 bytes: B * Hq * L up to 32512 at
- *    d = 128), else SDPA_ERR_WORKSPACE (nothing is launched).
+ *    (4 bytes per LSE entry: B * Hq * L up to 4194304, or Hq times the
+ *    packed rows), else SDPA_ERR_WORKSPACE (nothing is launched).
  *  - The first call on a device looks up the array's device address with
  *    that device current (once per device); make that first call before
  *    any stream capture on the device.  A failed lookup -> SDPA_ERR_CUDA.
  *  - Every call, on every stream of a device, shares the one array, which
- *    keeps the contents of the last call (each call clears the counters it
- *    uses and writes every other entry before reading it).  Calls whose executions
+ *    keeps the contents of the last call (each call writes every entry it
+ *    reads before reading it).  Calls whose executions
  *    overlap on the GPU race on it; order them on one stream or with events.
  *  - The looked-up address is cached per device for the life of the
  *    process; it does not survive cudaDeviceReset (or any other teardown of
@@ -354,15 +354,6 @@ void sdpa_set_wait_limit_ns(uint64_t ns);
  * afterwards.
  */
 sdpa_status_t sdpa_debug_wait_timeout(void* stream);
-
-/*
- * Launches one warp that waits for a dQ turn that never comes: it polls the
- * device word *counter (caller-owned, any value but 0xffffffff) for the value
- * 0xffffffff under the current wait limit, the way the backward's reducer
- * warps wait for their turn.  Expect sdpa_read_device_status() ==
- * SDPA_ERR_TIMEOUT afterwards.
- */
-sdpa_status_t sdpa_debug_turn_timeout(const uint32_t* counter, void* stream);
 
 /* Static English text for a status code. */
 const char* sdpa_status_string(sdpa_status_t status);

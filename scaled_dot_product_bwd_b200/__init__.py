@@ -7,7 +7,8 @@ touch the GPU.
 """
 from .binding import (  # noqa: F401
     BWD_ALL,
-    BWD_GRADS,
+    BWD_DKDV,
+    BWD_DQ,
     BWD_PREPROCESS,
     EXPORTED,
     SdpaError,
@@ -18,7 +19,6 @@ from .binding import (  # noqa: F401
     sdpa_bwd_noalloc,
     sdpa_bwd_varlen,
     sdpa_bwd_workspace_size,
-    sdpa_debug_turn_timeout,
     sdpa_debug_wait_timeout,
     sdpa_exp2_fma,
     sdpa_fwd,

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTE
                 3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
 BIAS_NONE, BIAS_DENSE, BIAS_T5, BIAS_ALIBI = 0, 1, 2, 3
 
-BWD_PREPROCESS, BWD_GRADS, BWD_ALL = 1, 2, 3
+BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -30,7 +30,7 @@ EXPORTED = ("sdpa_fwd", "sdpa_fwd_varlen", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_
             "sdpa_bwd_noalloc", "sdpa_bwd_workspace_size", "sdpa_bwd_varlen_workspace_size",
             "sdpa_bwd_bias_grad", "sdpa_bwd_bias_grad_workspace_size", "sdpa_t5_bucket",
             "sdpa_exp2_fma", "sdpa_read_device_status", "sdpa_set_wait_limit_ns",
-            "sdpa_debug_wait_timeout", "sdpa_debug_turn_timeout", "sdpa_status_string")
+            "sdpa_debug_wait_timeout", "sdpa_status_string")
 
 
 class SdpaError(RuntimeError):
@@ -110,8 +110,6 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_set_wait_limit_ns.restype = None
     lib.sdpa_debug_wait_timeout.argtypes = [vp]
     lib.sdpa_debug_wait_timeout.restype = i32
-    lib.sdpa_debug_turn_timeout.argtypes = [vp, vp]
-    lib.sdpa_debug_turn_timeout.restype = i32
     lib.sdpa_status_string.argtypes = [i32]
     lib.sdpa_status_string.restype = ctypes.c_char_p
     if path is None:
@@ -257,9 +255,9 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
              workspace=None, deterministic=True, phases=BWD_ALL):
     """dQ, dK, dV = attention backward (see sdpa_bwd / sdpa_bwd_phases in include/sdpa.h).
 
-    ``phases`` selects launches (BWD_PREPROCESS | BWD_GRADS); the default
-    runs both in order.  A GRADS call needs the workspace of an earlier
-    PREPROCESS call (one per GRADS call).
+    ``phases`` selects launches (BWD_PREPROCESS | BWD_DQ | BWD_DKDV); the
+    default runs all three in order.  DQ and DKDV read D from the workspace
+    of an earlier PREPROCESS call on the same O and dO.
     """
     lib = load_library()
     shape = make_shape(q, k)
@@ -471,14 +469,6 @@ def sdpa_set_wait_limit_ns(ns: int):
 
 def sdpa_debug_wait_timeout():
     _check(load_library().sdpa_debug_wait_timeout(_stream()), "sdpa_debug_wait_timeout")
-
-
-def sdpa_debug_turn_timeout(counter: torch.Tensor):
-    """One warp waits, under the wait limit, for a dQ turn that never comes."""
-    if counter.dtype != torch.int32 or not counter.is_cuda or counter.numel() < 1:
-        raise ValueError("counter must be an int32 CUDA tensor")
-    _check(load_library().sdpa_debug_turn_timeout(_ptr(counter), _stream(counter)),
-           "sdpa_debug_turn_timeout")
 
 
 def sdpa_status_string(status: int) -> str:

@@ -67,9 +67,9 @@ struct AttnParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;        // rows of the packed sequence axes (cu_q != nullptr)
-  // element strides of the per-row float arrays LSE, D and the dQ
-  // accumulator's rows: entry (b, h, row) is at b * lse_sb + h * lse_sh + row,
-  // row counted along the (packed) query sequence axis
+  // element strides of the per-row float arrays LSE and D: entry (b, h, row)
+  // is at b * lse_sb + h * lse_sh + row, row counted along the (packed) query
+  // sequence axis
   int64_t lse_sb, lse_sh;
   // forward outputs / backward inputs
   __nv_bfloat16* o;
@@ -80,9 +80,6 @@ struct AttnParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* dq_acc;               // fp32 dQ partial sums, row r at dq_acc + r * d
-  unsigned int* turns;         // per (b, hq, query tile): key tiles already added
-  unsigned int* tickets;       // work-item counter of the persistent backward
   // optional fp32 dS (the gradient of the logits, = of an additive bias),
   // element strides sd_b, sd_h, sd_i (multiples of 4), j contiguous
   float* ds_out;
@@ -133,8 +130,7 @@ __device__ __forceinline__ SeqView seq_view(const AttnParams& p, int b) {
   return s;
 }
 
-// Index of (b, h, query row i of b's sequence) in LSE, D and the dQ
-// accumulator's rows.
+// Index of (b, h, query row i of b's sequence) in LSE and D.
 __device__ __forceinline__ int64_t row_index(const AttnParams& p, const SeqView& s, int b, int h,
                                              int i) {
   return static_cast<int64_t>(b) * p.lse_sb + static_cast<int64_t>(h) * p.lse_sh + s.q0 + i;

@@ -1,5 +1,5 @@
-// Bias gradients from the fp32 dS the backward kernel stores (bwd_kernel
-// with DS_OUT): the scores are linear in an additive bias, so a dense bias's
+// Bias gradients from the fp32 dS the dQ kernel stores (bwd_dq_kernel with
+// DS_OUT): the scores are linear in an additive bias, so a dense bias's
 // gradient is dS summed over each index the bias is broadcast along, and a
 // T5 table entry's gradient is dS summed over every (b, i, j) whose distance
 // j - i falls in its bucket (catie-aq/flashT5 README, "Full attention
@@ -27,8 +27,8 @@ constexpr int64_t kT5RowsPerPiece = 128;
 // ---------------------------------------------------------------------
 // dS entries the backward never visits: for query row i, the key tiles
 // outside [nlo, nhi) of i's query tile (key_tile_range), which hold no key
-// visible from any row of the tile.  The backward kernel writes every column
-// of the tiles inside the band (masked keys as 0); this fills the rest with 0.
+// visible from any row of the tile.  The dQ kernel writes every column of
+// the tiles inside the band (masked keys as 0); this fills the rest with 0.
 __device__ __forceinline__ void zero_span(float* row, int j0, int j1) {
   // j0 is 0 or a multiple of the tile width, so row + j0 is 16-byte aligned
   for (int j = j0 + 4 * static_cast<int>(threadIdx.x); j < j1; j += 4 * static_cast<int>(blockDim.x)) {

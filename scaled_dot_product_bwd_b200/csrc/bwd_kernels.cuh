@@ -1,39 +1,34 @@
-// bwd_kernels.cuh -- fused attention backward for sm_100a.
+// bwd_kernels.cuh -- attention backward for sm_100a.
 //
 // The pages print no gradient formulas; these kernels apply the chain rule
 // to the forward (codelab "jax-gpu-05-attention-gpu", sections 1 and 4):
 //   P = exp(S - LSE)  (S recomputed with the forward's mask and bias)
 //   dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO_i * O_i),  dS = P (dP - D)
 //   dK = scale dS^T Q,  dQ = scale dS K
-// Two launches:
-//   1. preprocess: D = rowsum(dO * O); zeroes the dQ turn counters and the
-//      work-item counter of launch 2.
-//   2. one persistent kernel for all three gradients.  A work item is 128
-//      keys of one (batch, KV head); it walks the 128-query tiles of the
-//      mask band, every query head of the group at each tile, and per block
-//        S^T = K Q^T, dP^T = V dO^T            (SS MMAs, 128 x 128)
-//        P^T -> tensor memory (bf16), dS -> shared memory (bf16)
-//        dV += P^T dO (TS), dK += dS^T Q (SS), dQ_part = dS K (SS)
-//      dV and dK stay in tensor memory for the whole item.  Each dQ_part is
-//      added into an fp32 accumulator in global memory, the contributions to
-//      one query tile in descending key-tile order: a turn counter per
-//      (query tile, 32-row quarter) holds the number of key tiles already
-//      added, the first key tile stores, the last one writes
-//      dQ = scale * sum as bf16.  A fixed-order split-K reduction with no
-//      floating-point atomics, so the result is bit-identical run to run
-//      (HF transformers issue #31787, "Transformer models are not
-//      deterministic when using Flash Attention 2").
-//
-// Work items are handed out by an atomic ticket counter, group by group
-// ((batch, KV head) major) and within a group from the last key tile to the
-// first, which is also the order of the dQ sums.  A waiting item only waits
-// for items with smaller tickets, all of which are held by CTAs that are
-// running or done, so the waits always end.  Within an item the query tiles
-// run from the first of its band to the last, every head of the group at
-// each: under a causal or windowed mask key tile n + 1 then reaches each
-// query tile G blocks before key tile n does, so the contributions to a
-// tile arrive spaced out and in order, and a turn is usually free when it
-// is needed.
+// Three launches, each reducing in a fixed order with no atomics, so the
+// result is bit-identical run to run (HF transformers issue #31787,
+// "Transformer models are not deterministic when using Flash Attention 2"):
+//   1. preprocess: D = rowsum(dO * O) into the workspace.
+//   2. dQ: one CTA per SM walks (128 queries, query head, batch entry) items,
+//      each over the 128-key tiles of its mask band in ascending order:
+//        S = Q K^T, dP = dO V^T                 (SS MMAs, 128 x 128)
+//        dS -> tensor memory (bf16), dQ += dS K (TS MMA, 128 x d)
+//      with S double-buffered, so the next tile's scores are ready while
+//      this tile's dS is formed.  The split-K sum over key tiles runs inside
+//      one CTA's tensor memory, in tile order.
+//   3. dK / dV: one CTA per (128 keys, KV head, batch entry) walks the
+//      128-query tiles of the band for every query head of the group, in a
+//      fixed order, and accumulates dV and dK in tensor memory:
+//        S^T = K Q^T, dP^T = V dO^T             (SS MMAs, 128 x 128)
+//        P^T, dS^T -> tensor memory (bf16)
+//        dV += P^T dO, dK += dS^T Q             (TS MMAs, 128 x d)
+// The dQ launch recomputes S and dP, 2 of the 7 MMAs of the pair: the price
+// of summing dQ without atomics or a cross-CTA ordering protocol.  All score
+// MMAs are 128 x 128 (an N = 64 MMA with both operands in shared memory is
+// shared-memory-bandwidth bound on this part); the two compute warpgroups
+// split every tile's 128 columns between them.  Rows of both sequences are
+// addressed through the batch entry's SeqView, so cross-attention lengths
+// and packed sequences take the same kernels.
 #pragma once
 
 #include "attn_common.cuh"
@@ -43,31 +38,28 @@
 
 namespace sdpa {
 
-// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all).
-constexpr int kBwdMufuPer8 = 5;
+// Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all),
+// chosen by measurement: the dK/dV kernel gains from moving 3 of 8 to the
+// FMA pipe, the dQ kernel does not.
+constexpr int kDkdvMufuPer8 = 5;
+constexpr int kDqMufuPer8 = 8;
 
 // ------------------------------------------------------------ preprocess
 // D = rowsum(dO * O) for every query row along the (padded or packed)
-// sequence axis, and zeroes `n_zero` words of turn counters plus the ticket.
-// Rows of query tiles that no key tile reaches (a left window that starts
-// past the end of a shorter key sequence, an empty packed key sequence)
-// get no dQ contribution from the main kernel: their dQ is zeroed here.
+// sequence axis, D / 8 threads per row.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p, int64_t n_axis,
-                                                             int64_t n_zero) {
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p, int64_t n_axis) {
   constexpr int kTpr = D / 8;  // threads per row, 8 bf16 (16 bytes) each
   const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (gt < n_zero) p.turns[gt] = 0u;
-  if (gt == 0) *p.tickets = 0u;
   const int64_t nrows = n_axis * p.Hq;
   const int64_t r = gt / kTpr;
   const int part = static_cast<int>(gt % kTpr);
   float acc = 0.f;
   int h = 0;
-  int64_t a = 0, b = 0, i = 0;
+  int64_t b = 0, i = 0;
   if (r < nrows) {
     h = static_cast<int>(r % p.Hq);
-    a = r / p.Hq;                         // position along the sequence axis
+    const int64_t a = r / p.Hq;  // position along the sequence axis
     b = p.cu_q ? 0 : a / p.Lq;
     i = p.cu_q ? a : a % p.Lq;
     const int64_t off = b * p.sq_b + i * p.sq_l + h * p.sq_h + part * 8;
@@ -85,60 +77,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p,
   }
 #pragma unroll
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (r < nrows) {
-    if (part == 0) p.dvec[b * p.lse_sb + h * p.lse_sh + i] = acc;
-    // the sequence of this row: b itself, or (packed) the last entry whose
-    // first row is at or before it
-    int bb = static_cast<int>(b);
-    if (p.cu_q) {
-      int lo = 0, hi = p.B;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (p.cu_q[mid] <= a) lo = mid; else hi = mid;
-      }
-      bb = lo;
-    }
-    const SeqView sv = seq_view(p, bb);
-    const int il = static_cast<int>(p.cu_q ? a - sv.q0 : i);
-    int nlo, nhi;
-    key_tile_range(p, sv.Lq, sv.Lk, (il / kTile) * kTile, kTile, nlo, nhi);
-    if (nhi <= nlo || il < 0 || il >= sv.Lq)
-      *reinterpret_cast<uint4*>(p.dq + b * p.sq_b + i * p.sq_l + h * p.sq_h + part * 8) =
-          make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-// ------------------------------------------------------------ turn counters
-__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Whole warp: wait until *ctr == want, for at most ctl.limit_ns.  On expiry
-// (or if another wait of the CTA aborted) raises the abort flag and the
-// device status and returns false.
-__device__ __forceinline__ bool wait_turn(const unsigned int* ctr, unsigned int want,
-                                          const WaitCtl& ctl) {
-  if (__shfl_sync(0xffffffffu, ld_acquire_u32(ctr), 0) == want) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t k = 1;; ++k) {
-    if (k > 32) __nanosleep(64);
-    if (__shfl_sync(0xffffffffu, ld_acquire_u32(ctr), 0) == want) return true;
-    if ((k & 255u) == 0) {
-      const bool stop = *ctl.abort || (globaltimer_ns() - t0 > ctl.limit_ns);
-      if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) {
-        if ((threadIdx.x & 31) == 0) {
-          *ctl.abort = 1;
-          atomicOr(&g_device_status, kStatusTimeout);
-        }
-        return false;
-      }
-    }
-  }
+  if (r < nrows && part == 0) p.dvec[b * p.lse_sb + h * p.lse_sh + i] = acc;
 }
 
 // 16 columns of one row, bf16, as two uint4 (columns c..c+7, c+8..c+15)
@@ -161,68 +100,49 @@ __device__ __forceinline__ uint4 shfl_xor_u4(uint4 v, int m) {
   return v;
 }
 
-__device__ __forceinline__ float4 shfl_xor_f4(float4 v, int m) {
-  v.x = __shfl_xor_sync(0xffffffffu, v.x, m);
-  v.y = __shfl_xor_sync(0xffffffffu, v.y, m);
-  v.z = __shfl_xor_sync(0xffffffffu, v.z, m);
-  v.w = __shfl_xor_sync(0xffffffffu, v.w, m);
-  return v;
-}
-
-__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
-  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-}
-
-// ---------------------------------------------------------------- layout
-// Tensor memory (512 columns): S^T 0..127 | dP^T 128..255 | dV 256.. | dK
-// 256 + d..  P^T (bf16) overwrites the first half of each compute
-// warpgroup's S^T columns and feeds the dV MMA from there.  The dQ partial
-// (128 queries x d fp32) goes over the dP^T columns at d = 128 (the compute
-// warpgroups have read dP^T by then) and into two buffers of its own at
-// 384 and 448 at d = 64.
+// ------------------------------------------------------------------ dK / dV
+// CTA = 128 keys of one (KV head, batch entry).  Blocks of 128 queries
+// stream through; both compute warpgroups work on every block, warpgroup w
+// on the query columns [64 w, 64 w + 64).  Tensor memory (512 columns):
+//   S^T 0..127 | dP^T 128..255 | dV 256.. | dK 256 + d..
+// P^T (bf16) overwrites the first half of each warpgroup's S^T columns, dS^T
+// the first half of its dP^T columns; the TS MMAs read them from there.
 template <int D, int BIAS>
-struct BwdLayout {
+struct DkdvLayout {
   static constexpr int kTileBytes = kTile * D * 2;  // 128 rows x d bf16
-  static constexpr int kDSBytes = kTile * kTile * 2;  // dS, 128 keys x 128 queries bf16
-  // Q blocks are read by S^T and dK, dO blocks by dP^T and dV.  At d = 128
-  // K, V, dS and two stages of each ring fill the 227 KB of shared memory.
-  static constexpr int kSQ = (D == 128) ? 2 : 4;
-  static constexpr int kSO = (D == 128) ? (BIAS == kBiasT5 ? 1 : 2) : 4;
+  // Q blocks are used until the block's dK MMA, dO blocks only until its dV
+  // MMA: the Q ring is the deeper one.  At d = 128 without a T5 table this
+  // fills the 227 KB of shared memory to the last kilobyte.
+  static constexpr int kSQ = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : 4;
+  static constexpr int kSO = (D == 128) ? 2 : 4;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
-  static constexpr int kDSOff = 2 * kTileBytes;
-  static constexpr int kQOff = kDSOff + kDSBytes;
-  static constexpr int kDOOff = kQOff + kSQ * kTileBytes;
-  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;      // 2 x (lse2[128], D[128])
-  static constexpr int kLutOff = kVecOff + 2 * 2 * kTile * 4;    // T5 only: 8 warps x 96 floats
+  static constexpr int kQOff = 2 * kTileBytes;                  // Q ring
+  static constexpr int kDOOff = kQOff + kSQ * kTileBytes;       // dO ring
+  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;     // 2 x (lse2[128], D[128])
+  static constexpr int kLutOff = kVecOff + 2 * 2 * kTile * 4;   // T5 only: 8 warps x 96 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
-  static constexpr int kNumBars = 2 + 2 * kSQ + 2 * kSO + 22;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;        // tmem slot, abort, item slots
-  static constexpr int kSmemAlloc = kMiscOff + 32;
-  // warps 0-7: two compute warpgroups; 8-11: dQ reducer; 12 producer,
-  // 13 / 14 MMA issuers, 15 spare
-  static constexpr int kThreads = 512;
+  // kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], vec_full[2],
+  // vec_empty[2], s_full, dp_full, p_full, ds_full, s_free, dp_free, acc_done,
+  // drain[2]
+  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 9;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemAlloc = kMiscOff + 16;
+  // 2 compute warpgroups, producer, two MMA issuers
+  static constexpr int kThreads = 352;
   static constexpr int kTmemCols = 512;
   static constexpr int kSCol = 0, kDPCol = 128, kDVCol = 256, kDKCol = 256 + D;
-  static constexpr bool kDQShared = (D == 128);
-  static constexpr int kDQCol = kDQShared ? kDPCol : 256 + 2 * D;
-  static_assert(kDQShared || kDQCol + 2 * D <= kTmemCols, "tensor memory budget");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-// Registers per thread after the warpgroups reallocate (launched with 128
-// each, 512 threads = 65536): compute warpgroups, reducer, producer/issuers.
-// 2 x 152 + 128 + 80 = 512 = 4 x 128.
-constexpr uint32_t kRegsCompute = 152, kRegsReducer = 128, kRegsIssue = 80;
-static_assert(2 * kRegsCompute + kRegsReducer + kRegsIssue == 4 * 128, "register split");
 
-template <int D, int BIAS, bool DS_OUT>
-__global__ void __launch_bounds__(512, 1)
-    bwd_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmDO) {
-  using Lay = BwdLayout<D, BIAS>;
+template <int D, int BIAS>
+__global__ void __launch_bounds__(352, 1)
+    bwd_dkdv_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmDO) {
+  using Lay = DkdvLayout<D, BIAS>;
   constexpr int SQ = Lay::kSQ;
   constexpr int SO = Lay::kSO;
   extern __shared__ uint8_t smem[];
@@ -234,63 +154,41 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work items: (batch, KV head) groups, key tiles ascending within one
-  const int ntk = (p.Lk + kTile - 1) / kTile;
-  const int ntq = (p.Lq + kTile - 1) / kTile;
-  const int n_items = p.B * p.Hkv * ntk;
-  struct Item {
-    int b, g, n, mlo, mhi, nb;
-    bool rows;  // the key tile holds keys of the sequence
-    SeqView s;
-  };
-  auto item_at = [&](int t) {
-    Item w;
-    const int grp = t / ntk;
-    w.n = ntk - 1 - (t - grp * ntk);  // key tiles of a group from the last to the first
-    w.b = grp / p.Hkv;
-    w.g = grp - w.b * p.Hkv;
-    w.s = seq_view(p, w.b);
-    w.mlo = w.mhi = 0;
-    w.nb = 0;
-    w.rows = w.n * kTile < w.s.Lk;
-    if (w.rows) {
-      query_tile_range(p, w.s.Lq, w.s.Lk, w.n * kTile, w.mlo, w.mhi);
-      if (w.mhi > w.mlo) w.nb = (w.mhi - w.mlo) * p.G;
-    }
-    return w;
-  };
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int n0 = static_cast<int>(blockIdx.x) * kTile;  // causal: low key tiles are heaviest
+  const SeqView s = seq_view(p, b);
+  if (n0 >= s.Lk) return;  // past this entry's key sequence (packed, or a shorter one)
+  const int Lq = s.Lq, Lk = s.Lk;
+  int mlo, mhi;
+  query_tile_range(p, Lq, Lk, n0, mlo, mhi);
+  const int nm = mhi > mlo ? mhi - mlo : 0;
+  const int total = nm * p.G;  // blocks: query head (outer) x query tile (inner)
 
-  // ---- barriers
   auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
   const uint32_t kv_full = bar(0);
-  const uint32_t kv_empty = bar(1);
-  auto q_full = [&](int s) { return bar(2 + s); };
-  auto q_empty = [&](int s) { return bar(2 + SQ + s); };
-  auto o_full = [&](int s) { return bar(2 + 2 * SQ + s); };
-  auto o_empty = [&](int s) { return bar(2 + 2 * SQ + SO + s); };
-  constexpr int kB = 2 + 2 * SQ + 2 * SO;
+  auto q_full = [&](int s) { return bar(1 + s); };
+  auto q_empty = [&](int s) { return bar(1 + SQ + s); };
+  auto o_full = [&](int s) { return bar(1 + 2 * SQ + s); };
+  auto o_empty = [&](int s) { return bar(1 + 2 * SQ + SO + s); };
+  constexpr int kB = 1 + 2 * SQ + 2 * SO;
   auto vec_full = [&](int x) { return bar(kB + x); };
   auto vec_empty = [&](int x) { return bar(kB + 2 + x); };
   const uint32_t s_full = bar(kB + 4);
-  const uint32_t p_full = bar(kB + 5);
-  const uint32_t s_free = bar(kB + 6);
-  const uint32_t dp_full = bar(kB + 7);
-  const uint32_t ds_full = bar(kB + 8);
-  const uint32_t ds_free = bar(kB + 9);
-  auto dq_full = [&](int x) { return bar(kB + 10 + x); };
-  auto dq_free = [&](int x) { return bar(kB + 12 + x); };
-  const uint32_t acc_done = bar(kB + 14);
-  const uint32_t acc_free = bar(kB + 15);
-  auto item_full = [&](int x) { return bar(kB + 16 + x); };
-  auto item_empty = [&](int x) { return bar(kB + 18 + x); };
-  auto drain = [&](int x) { return bar(kB + 20 + x); };
+  const uint32_t dp_full = bar(kB + 5);
+  const uint32_t p_full = bar(kB + 6);
+  const uint32_t ds_full = bar(kB + 7);
+  const uint32_t s_free = bar(kB + 8);
+  const uint32_t dp_free = bar(kB + 9);
+  const uint32_t acc_done = bar(kB + 10);
+  auto drain = [&](int x) { return bar(kB + 11 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
-  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 8);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 2);  // both issuers, after their last MMA of the item
+    // Q blocks are read by both issuers (S^T and dK), dO blocks too (dP^T and
+    // dV): a slot is free once each issuer's last MMA on it has completed.
     for (int s = 0; s < SQ; ++s) {
       mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 2);
@@ -302,20 +200,16 @@ __global__ void __launch_bounds__(512, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(vec_full(x), 32);          // the producer warp's lanes
       mbar_init(vec_empty(x), 2 * kTile);  // both compute warpgroups
-      mbar_init(dq_full(x), 1);
-      mbar_init(dq_free(x), 4);            // the reducer warps
-      mbar_init(item_full(x), 1);
-      mbar_init(item_empty(x), 14);        // 2 issuers, 8 compute and 4 reducer warps
-      mbar_init(drain(x), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 2 * kTile);
-    mbar_init(s_free, 1);
     mbar_init(dp_full, 1);
+    mbar_init(p_full, 2 * kTile);
     mbar_init(ds_full, 2 * kTile);
-    mbar_init(ds_free, 1);
+    mbar_init(s_free, 1);
+    mbar_init(dp_free, 1);
     mbar_init(acc_done, 2);
-    mbar_init(acc_free, 2 * kTile);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -330,569 +224,293 @@ __global__ void __launch_bounds__(512, 1)
   const WaitCtl ctl{abort_flag, p.wait_limit_ns};
   float* vec = reinterpret_cast<float*>(smem + Lay::kVecOff);
 
-  // Item ids from the producer's ring of two slots.  Returns false on abort.
-  auto next_item = [&](int k, int& t) -> bool {
-    bool ok = mbar_wait(item_full(k & 1), (k >> 1) & 1, ctl);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) return false;
-    t = item_slot[k & 1];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(item_empty(k & 1));
-    return true;
-  };
-
-  if (warp >= 12) {
-    regs_shrink<kRegsIssue>();
-    if (warp == 12) {
-      // ============================ producer ============================
+  if (warp == 8) {
+    // ============================ producer ============================
+    if (total > 0) {
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmDO);
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
+        mbar_expect_tx(kv_full, 2 * Lay::kTileBytes);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_4d(sb + Lay::kKOff + h * kTile * 128, &tmK, kv_full, h * 64, s.k0 + n0, g, s.bc);
+          tma_load_4d(sb + Lay::kVOff + h * kTile * 128, &tmV, kv_full, h * 64, s.k0 + n0, g, s.bc);
+        }
       }
+      // LSE (log2 units) and D of one block's 128 queries, four per lane,
+      // loaded one block ahead of the slot they go to.
+      float l2v[4], ddv[4];
+      auto load_vec = [&](int it) {
+        const int hq = g * p.G + it / nm;
+        const int m0 = (mlo + it % nm) * kTile;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = m0 + lane + 32 * e;
+          l2v[e] = INFINITY;  // queries past the sequence: P = 0
+          ddv[e] = 0.f;
+          if (i < Lq) {
+            const int64_t idx = row_index(p, s, b, hq, i);
+            l2v[e] = p.lse[idx] * kLog2e;
+            ddv[e] = p.dvec[idx];
+            if (l2v[e] == -INFINITY) l2v[e] = INFINITY;  // row with no visible key
+          }
+        }
+      };
+      load_vec(0);
       int issued_q[SQ], issued_o[SO];
       for (int s = 0; s < SQ; ++s) issued_q[s] = -1;
       for (int s = 0; s < SO; ++s) issued_o[s] = -1;
-      int kv_issued = -1;
       bool ok = true;
-      int i = 0, k = 0, u = 0;
-      while (ok) {
-        int t = -1;
+      for (int it = 0; it < total; ++it) {
+        const int hq = g * p.G + it / nm;
+        const int m0 = (mlo + it % nm) * kTile;
+        const int x = it & 1;
+        // The Q / dO copies go first: they wait only for their ring slots,
+        // not for the compute warps, so they run as far ahead as the rings allow.
         if (lane == 0) {
-          t = static_cast<int>(atomicAdd(p.tickets, 1u));
-          if (t >= n_items) t = -1;
-        }
-        t = __shfl_sync(0xffffffffu, t, 0);
-        ok = mbar_wait(item_empty(k & 1), ((k >> 1) & 1) ^ 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        if (lane == 0) {
-          item_slot[k & 1] = t;
-          mbar_arrive(item_full(k & 1));
-        }
-        ++k;
-        if (t < 0) break;
-        const Item w = item_at(t);
-        if (w.nb == 0) continue;
-        if (lane == 0) {
-          if (u > 0) ok = mbar_wait(kv_empty, (u - 1) & 1, ctl);
+          const int sq = it % SQ, so = it % SO;
+          ok = mbar_wait(q_empty(sq), ((it / SQ) & 1) ^ 1, ctl);
           if (ok) {
-            mbar_expect_tx(kv_full, 2 * Lay::kTileBytes);
-            for (int h = 0; h < D / 64; ++h) {
-              tma_load_4d(sb + Lay::kKOff + h * kTile * 128, &tmK, kv_full, h * 64,
-                          w.s.k0 + w.n * kTile, w.g, w.s.bc);
-              tma_load_4d(sb + Lay::kVOff + h * kTile * 128, &tmV, kv_full, h * 64,
-                          w.s.k0 + w.n * kTile, w.g, w.s.bc);
-            }
-            kv_issued = u & 1;
+            mbar_expect_tx(q_full(sq), Lay::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(sb + Lay::kQOff + sq * Lay::kTileBytes + h * kTile * 128, &tmQ,
+                          q_full(sq), h * 64, s.q0 + m0, hq, s.bc);
+            issued_q[sq] = (it / SQ) & 1;
+            ok = mbar_wait(o_empty(so), ((it / SO) & 1) ^ 1, ctl);
+          }
+          if (ok) {
+            mbar_expect_tx(o_full(so), Lay::kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(sb + Lay::kDOOff + so * Lay::kTileBytes + h * kTile * 128, &tmDO,
+                          o_full(so), h * 64, s.q0 + m0, hq, s.bc);
+            issued_o[so] = (it / SO) & 1;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        // LSE (log2 units) and D of one block's 128 queries, four per lane,
-        // loaded one block ahead of the slot they go to.
-        float l2v[4], ddv[4];
-        auto load_vec = [&](int blk) {
-          const int mi = w.mlo + blk / p.G;
-          const int hq = w.g * p.G + blk % p.G;
+        if (ok) ok = mbar_wait(vec_empty(x), ((it >> 1) & 1) ^ 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float* lse2 = vec + x * 2 * kTile;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int iq = mi * kTile + lane + 32 * e;
-            l2v[e] = INFINITY;  // queries past the sequence: P = 0
-            ddv[e] = 0.f;
-            if (iq < w.s.Lq) {
-              const int64_t idx = row_index(p, w.s, w.b, hq, iq);
-              l2v[e] = p.lse[idx] * kLog2e;
-              ddv[e] = p.dvec[idx];
-              if (l2v[e] == -INFINITY) l2v[e] = INFINITY;  // row with no visible key
-            }
-          }
-        };
-        load_vec(0);
-        for (int blk = 0; blk < w.nb; ++blk, ++i) {
-          const int mi = w.mlo + blk / p.G;
-          const int hq = w.g * p.G + blk % p.G;
-          const int x = i & 1;
-          if (lane == 0) {
-            const int sq = i % SQ, so = i % SO;
-            ok = mbar_wait(q_empty(sq), ((i / SQ) & 1) ^ 1, ctl);
-            if (ok) {
-              mbar_expect_tx(q_full(sq), Lay::kTileBytes);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_4d(sb + Lay::kQOff + sq * Lay::kTileBytes + h * kTile * 128, &tmQ,
-                            q_full(sq), h * 64, w.s.q0 + mi * kTile, hq, w.s.bc);
-              issued_q[sq] = (i / SQ) & 1;
-              ok = mbar_wait(o_empty(so), ((i / SO) & 1) ^ 1, ctl);
-            }
-            if (ok) {
-              mbar_expect_tx(o_full(so), Lay::kTileBytes);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_4d(sb + Lay::kDOOff + so * Lay::kTileBytes + h * kTile * 128, &tmDO,
-                            o_full(so), h * 64, w.s.q0 + mi * kTile, hq, w.s.bc);
-              issued_o[so] = (i / SO) & 1;
-              if constexpr (BIAS == kBiasDense) prefetch_bias_tile(p, w.b, hq, mi * kTile, w.n * kTile);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (ok) ok = mbar_wait(vec_empty(x), ((i >> 1) & 1) ^ 1, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          float* lse2 = vec + x * 2 * kTile;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            lse2[lane + 32 * e] = l2v[e];
-            lse2[kTile + lane + 32 * e] = ddv[e];
-          }
-          mbar_arrive(vec_full(x));
-          if (blk + 1 < w.nb) load_vec(blk + 1);
+        for (int e = 0; e < 4; ++e) {
+          lse2[lane + 32 * e] = l2v[e];
+          lse2[kTile + lane + 32 * e] = ddv[e];
         }
-        ++u;
+        mbar_arrive(vec_full(x));
+        if (it + 1 < total) load_vec(it + 1);
       }
       if (!ok && lane == 0) {
-        // Aborted: let every copy already issued land before the CTA exits.
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        if (kv_issued >= 0) mbar_wait(kv_full, kv_issued, ign);
+        mbar_wait(kv_full, 0, ign);
         for (int s = 0; s < SQ; ++s)
           if (issued_q[s] >= 0) mbar_wait(q_full(s), issued_q[s], ign);
         for (int s = 0; s < SO; ++s)
           if (issued_o[s] >= 0) mbar_wait(o_full(s), issued_o[s], ign);
       }
-    } else if (warp == 13 || warp == 14) {
-      // ===================== MMA issuers (one thread each) =====================
-      // Warp 13: S^T(i) = K Q^T once dV(i - 1) has read P^T(i - 1) out of the
-      // S^T columns, then dV(i) += P^T(i) dO(i) once P^T(i) is written.
-      // Warp 14: dP^T(i) = V dO^T into its columns (at d = 128 once the
-      // reducer has read dQ(i - 1) from them), then, once dS(i) is in shared
-      // memory, dQ(i) = dS(i) K and dK += dS(i)^T Q(i).
-      const bool chain_s = (warp == 13);
-      bool ok = true;
-      int i = 0, k = 0, u = 0;
+    }
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers (one thread each) =====================
+    // Warp 9 owns the S^T chain: S^T(i), then dV(i) once P^T(i) is ready, then
+    // S^T(i+1) once dV(i) has read P^T(i) out of the S^T columns.  Warp 10 owns
+    // the dP^T chain: dP^T(i), dK(i) once dS^T(i) is ready, dP^T(i+1) once dK(i)
+    // is done.  Neither waits on the other's barriers, so a stalled chain does
+    // not hold up MMAs that are ready in the other.
+    if (lane == 0 && total > 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 keys x 128 queries
-      constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // dV, dK: 128 keys x d
-      constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 1, 1);      // dQ: 128 queries x d
-      while (true) {
-        int t = -1;
-        if (!(ok = next_item(k, t))) break;
-        ++k;
-        if (t < 0) break;
-        const Item w = item_at(t);
-        if (w.nb == 0) continue;
-        if (lane == 0) {
-          ok = issuer_wait(kv_full, u & 1, ctl);
-          for (int blk = 0; blk < w.nb && ok; ++blk, ++i) {
-            const int sq = i % SQ, so = i % SO;
-            const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
-            const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
-            const uint32_t dss = sb + Lay::kDSOff;
-            if (chain_s) {
-              if (!(ok = issuer_wait(q_full(sq), (i / SQ) & 1, ctl))) break;
-              if (i > 0 && !(ok = issuer_wait(s_free, (i - 1) & 1, ctl))) break;
-              tc_fence_after();
+      constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // 128 keys x d
+      const bool chain_s = (warp == 9);
+      bool ok = issuer_wait(kv_full, 0, ctl);
+      for (int it = 0; it < total && ok; ++it) {
+        const int sq = it % SQ, so = it % SO;
+        const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
+        const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
+        if (chain_s) {
+          if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (it > 0 && !(ok = issuer_wait(s_free, (it - 1) & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk)
-                mma_ss(tmem + Lay::kSCol,
-                       smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
-                       smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS,
-                       kk > 0 ? 1u : 0u);
-              mma_commit(s_full);
-              mma_commit(q_empty(sq));
-              if (!(ok = issuer_wait(o_full(so), (i / SO) & 1, ctl))) break;
-              if (!(ok = issuer_wait(p_full, i & 1, ctl))) break;
-              // the item's first dV MMA overwrites the accumulator
-              if (blk == 0 && u > 0 && !(ok = issuer_wait(acc_free, (u - 1) & 1, ctl))) break;
-              tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + Lay::kSCol,
+                   smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(s_full);
+          mma_commit(q_empty(sq));
+          if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (!(ok = issuer_wait(p_full, it & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < kTile / 16; ++kk)
-                mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
-                       smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
-                       (blk > 0 || kk > 0) ? 1u : 0u);
-              mma_commit(s_free);
-              mma_commit(o_empty(so));
-            } else {
-              if (!(ok = issuer_wait(o_full(so), (i / SO) & 1, ctl))) break;
-              if (Lay::kDQShared && i > 0 &&
-                  !(ok = issuer_wait(dq_free((i - 1) & 1), ((i - 1) >> 1) & 1, ctl)))
-                break;
-              tc_fence_after();
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
+                   smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(s_free);
+          mma_commit(o_empty(so));
+        } else {
+          if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
+          if (it > 0 && !(ok = issuer_wait(dp_free, (it - 1) & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk)
-                mma_ss(tmem + Lay::kDPCol,
-                       smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
-                       smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS,
-                       kk > 0 ? 1u : 0u);
-              mma_commit(dp_full);
-              mma_commit(o_empty(so));
-              if (!(ok = issuer_wait(ds_full, i & 1, ctl))) break;
-              if (!(ok = issuer_wait(q_full(sq), (i / SQ) & 1, ctl))) break;
-              if (!Lay::kDQShared && i >= 2 &&
-                  !(ok = issuer_wait(dq_free(i & 1), ((i >> 1) - 1) & 1, ctl)))
-                break;
-              tc_fence_after();
-              // dQ(i) = dS(i) K: A = dS (queries contiguous), B = K (d contiguous)
-              const uint32_t dqc = Lay::kDQShared ? Lay::kDPCol : Lay::kDQCol + D * (i & 1);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + Lay::kDPCol,
+                   smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
+                   smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_commit(dp_full);
+          mma_commit(o_empty(so));
+          if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
+          if (!(ok = issuer_wait(ds_full, it & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < kTile / 16; ++kk)
-                mma_ss(tmem + dqc, smem_desc_sw128(dss + kk * 2048, kTile * 128, 1024),
-                       smem_desc_sw128(sb + Lay::kKOff + kk * 2048, kTile * 128, 1024), kIdQ,
-                       kk > 0 ? 1u : 0u);
-              mma_commit(dq_full(i & 1));
-              if (blk == 0 && u > 0 && !(ok = issuer_wait(acc_free, (u - 1) & 1, ctl))) break;
-              // dK += dS(i)^T Q(i): A = dS^T (queries contiguous), B = Q (d contiguous)
-#pragma unroll
-              for (int kk = 0; kk < kTile / 16; ++kk)
-                mma_ss(tmem + Lay::kDKCol, smem_desc_sw128(dss + kmajor_koff(kk, kTile), 16, 1024),
-                       smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
-                       (blk > 0 || kk > 0) ? 1u : 0u);
-              mma_commit(ds_free);
-              mma_commit(q_empty(sq));
-            }
-          }
-          if (ok) {
-            mma_commit(acc_done);
-            mma_commit(kv_empty);
-          }
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk),
+                   smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(dp_free);
+          mma_commit(q_empty(sq));
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        i = __shfl_sync(0xffffffffu, i, 0);
-        if (!ok) break;
-        ++u;
       }
-      if (!ok && lane == 0) {
-        // Aborted: wait until every MMA this thread issued has finished with
-        // tensor memory before the CTA frees it.
+      if (ok) mma_commit(acc_done);
+      if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
         mma_commit(drain(chain_s ? 0 : 1));
         mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
       }
     }
-  } else if (warp >= 8) {
-    regs_grow<kRegsReducer>();
-    // ======== dQ reducer: thread = query row 32 (warp - 8) + lane of the tile ========
-    // Per block: read the dQ partial out of tensor memory, wait for this
-    // (query tile, quarter)'s turn, add it to the fp32 accumulator (or store
-    // it, for the first key tile; or write dQ = scale * sum as bf16, for the
-    // last), then pass the turn on.  Lanes 2m and 2m + 1 hold rows r and
-    // r + 1; for every 8 columns they trade halves, so that each 16-byte
-    // access of the pair covers one whole 32-byte sector of one row.
-    const int rq = warp - 8;
-    const uint32_t lane_bits = static_cast<uint32_t>(rq * 32) << 16;
-    const bool odd = (lane & 1) != 0;
-    const int co = odd ? 4 : 0;  // this lane's columns in each group of 8
-    // One block's share of the reduction: its query tile's place in the key
-    // tiles' order (idx, first, last) and which of this lane's two rows exist.
-    struct Red {
-      unsigned int idx;
-      int mi, hq;
-      bool first, last, va, vb;
-    };
-    auto red_at = [&](const Item& w, int blk) {
-      Red r;
-      r.mi = w.mlo + blk / p.G;
-      r.hq = w.g * p.G + blk % p.G;
-      int nlo, nhi;
-      key_tile_range(p, w.s.Lq, w.s.Lk, r.mi * kTile, kTile, nlo, nhi);
-      // key tiles add in descending order: nhi - 1 first, nlo last
-      r.idx = static_cast<unsigned int>(nhi - 1 - w.n);
-      r.first = r.idx == 0;
-      r.last = w.n == nlo;
-      const int ra = r.mi * kTile + rq * 32 + (lane & ~1);  // the lane pair's first row
-      r.va = ra < w.s.Lq;
-      r.vb = ra + 1 < w.s.Lq;
-      return r;
-    };
-    auto ctr_of = [&](const Item& w, const Red& r) {
-      return p.turns + ((static_cast<int64_t>(w.b) * p.Hq + r.hq) * ntq + r.mi) * 4 + rq;
-    };
-    auto acc_of = [&](const Item& w, const Red& r) {
-      return p.dq_acc + row_index(p, w.s, w.b, r.hq, r.mi * kTile + rq * 32 + (lane & ~1)) * D + co;
-    };
-    // This lane's running sums of one 64-column half of the block's two
-    // rows: group g (8 columns) of the half at [2g] (row a) and [2g + 1].
-    float4 old[16];
-    auto load_half = [&](const Item& w, const Red& r, int half) {
-      if (r.first) return;
-      const float* acc_a = acc_of(w, r) + 64 * half;
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        old[2 * g] = r.va ? __ldcg(reinterpret_cast<const float4*>(acc_a + 8 * g))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        old[2 * g + 1] = r.vb ? __ldcg(reinterpret_cast<const float4*>(acc_a + D + 8 * g))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    };
-    // wait for the block's turn, then fetch the first half's running sums
-    auto fetch = [&](const Item& w, const Red& r) -> bool {
-      if (r.first) return true;
-      if (!wait_turn(ctr_of(w, r), r.idx, ctl)) return false;
-      load_half(w, r, 0);
-      return true;
-    };
-    bool ok = true;
-    int i = 0, k = 0;
-    while (true) {
-      int t = -1;
-      if (!(ok = next_item(k, t))) break;
-      ++k;
-      if (t < 0) break;
-      const Item w = item_at(t);
-      if (w.nb == 0) continue;
-      Red cur = red_at(w, 0);
-      if (!(ok = fetch(w, cur))) break;
-      for (int blk = 0; blk < w.nb; ++blk, ++i) {
-        ok = mbar_wait(dq_full(i & 1), (i >> 1) & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t tq =
-            tmem + lane_bits + (Lay::kDQShared ? Lay::kDPCol : Lay::kDQCol + D * (i & 1));
-        float* acc_a = acc_of(w, cur);
-        __nv_bfloat16* dq_a = p.dq + static_cast<int64_t>(w.b) * p.sq_b +
-                              static_cast<int64_t>(w.s.q0 + cur.mi * kTile + rq * 32 + (lane & ~1)) * p.sq_l +
-                              static_cast<int64_t>(cur.hq) * p.sq_h + co;
-#pragma unroll
-        for (int half = 0; half < D / 64; ++half) {
-          // at d = 128 the second half's running sums come once the first
-          // half's are spent (registers), while the partial is still held
-          if (half > 0) load_half(w, cur, half);
-#pragma unroll
-          for (int c = 0; c < 64; c += 16) {
-            uint32_t v[16];
-            tmem_ld16_sync(tq + 64 * half + c, v);
-            if (half + 1 == D / 64 && c + 16 == 64) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(dq_free(i & 1));  // the partial is out of tensor memory
-            }
-#pragma unroll
-            for (int g2 = 0; g2 < 2; ++g2) {
-              const int g = c / 8 + g2;        // group of the half
-              const int col = 64 * half + 8 * g;
-              const float4 lo = make_float4(__uint_as_float(v[8 * g2]), __uint_as_float(v[8 * g2 + 1]),
-                                            __uint_as_float(v[8 * g2 + 2]), __uint_as_float(v[8 * g2 + 3]));
-              const float4 hi = make_float4(__uint_as_float(v[8 * g2 + 4]), __uint_as_float(v[8 * g2 + 5]),
-                                            __uint_as_float(v[8 * g2 + 6]), __uint_as_float(v[8 * g2 + 7]));
-              // the even lane sends its columns 4..7, the odd lane its 0..3
-              const float4 got = shfl_xor_f4(odd ? lo : hi, 1);
-              float4 sa = odd ? got : lo;   // row a, columns col + co ..
-              float4 sbv = odd ? hi : got;  // row b
-              if (!cur.first) {
-                sa = f4_add(old[2 * g], sa);
-                sbv = f4_add(old[2 * g + 1], sbv);
-              }
-              if (cur.last) {
-                const float sc = p.scale;
-                const uint2 pa = make_uint2(pack_bf16x2(sa.x * sc, sa.y * sc), pack_bf16x2(sa.z * sc, sa.w * sc));
-                const uint2 pb = make_uint2(pack_bf16x2(sbv.x * sc, sbv.y * sc), pack_bf16x2(sbv.z * sc, sbv.w * sc));
-                if (cur.va) *reinterpret_cast<uint2*>(dq_a + col) = pa;
-                if (cur.vb) *reinterpret_cast<uint2*>(dq_a + p.sq_l + col) = pb;
-              } else {
-                if (cur.va) __stcg(reinterpret_cast<float4*>(acc_a + col), sa);
-                if (cur.vb) __stcg(reinterpret_cast<float4*>(acc_a + D + col), sbv);
-              }
-            }
-          }
-        }
-        // The next block of the item is another query tile (or head), whose
-        // turn only ever waits on key tiles handed out earlier: take it and
-        // start its loads before passing this block's turn on, so their
-        // latencies overlap.
-        unsigned int* ctr = ctr_of(w, cur);
-        const unsigned int pass = cur.idx + 1u;
-        const bool release = !cur.last;
-        if (blk + 1 < w.nb) {
-          cur = red_at(w, blk + 1);
-          if (!(ok = fetch(w, cur))) break;
-        }
-        if (release) {
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) st_release_u32(ctr, pass);
-        }
-      }
-      if (!ok) break;
-    }
   } else {
-    if constexpr (kRegsCompute > 128) regs_grow<kRegsCompute>();
     // ===== compute warpgroup wg: query columns [64 wg, 64 wg + 64); thread = key =====
     const int wg = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
-    const int c0w = kBlk * wg;
+    const int j = n0 + row;
+    const int c0w = kBlk * wg;  // first query column of this warpgroup
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_bits + Lay::kSCol + c0w;
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
-    uint8_t* ds_row = smem + Lay::kDSOff + wg * (kTile * 128) + row * 128;
     bool ok = true;
-    int i = 0, k = 0, u = 0;
-    while (true) {
-      int t = -1;
-      if (!(ok = next_item(k, t))) break;
-      ++k;
-      if (t < 0) break;
-      const Item w = item_at(t);
-      if (!w.rows) continue;
-      const int Lq = w.s.Lq, Lk = w.s.Lk;
-      const int n0 = w.n * kTile;
-      const int j = n0 + row;  // this thread's key
-      for (int blk = 0; blk < w.nb; ++blk, ++i) {
-        const int x = i & 1;
-        const int mi = w.mlo + blk / p.G;
-        const int hq = w.g * p.G + blk % p.G;
-        const int m0 = mi * kTile + c0w;  // first query of this warpgroup's columns
-        const float* lut_row = nullptr;
-        if constexpr (BIAS == kBiasT5) {
-          // this warp's keys jw..jw+31 and queries m0..m0+63: j - i = (jw - m0 - 63) + e,
-          // e in [0, 94]; the thread reads entry lane + 63 - c for column c
-          const int base = n0 + (warp & 3) * 32 - m0 - (kBlk - 1);
-          __syncwarp();
-          for (int e = lane; e < 32 + kBlk - 1; e += 32) lut[e] = rel_bias_log2(p, base + e, hq);
-          __syncwarp();
-          lut_row = lut + lane + (kBlk - 1);
-        }
-        // visible queries of this key among the warpgroup's 64: [lo, hi]
-        int lo = 0, hi = kBlk - 1;
-        bool full = (m0 + kBlk <= Lq) && (n0 + kTile <= Lk);
-        if (p.causal) full = full && (n0 + kTile - 1 <= m0);
-        if (p.wl >= 0) full = full && (m0 + kBlk - 1 <= n0 + p.wl);
-        if (p.wr >= 0) full = full && (n0 + kTile - 1 <= m0 + p.wr);
-        if (!full) {
-          if (p.causal) lo = max(lo, j - m0);
-          if (p.wr >= 0) lo = max(lo, j - p.wr - m0);
-          hi = min(hi, Lq - 1 - m0);
-          if (p.wl >= 0) hi = min(hi, j + p.wl - m0);
-          if (j >= Lk) hi = -1;  // past the key sequence: no query sees it
-        }
-        const float* bcol = nullptr;
-        if constexpr (BIAS == kBiasDense)
-          bcol = p.bias + static_cast<int64_t>(w.b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
-                 static_cast<int64_t>(min(m0, Lq - 1)) * p.sb_i + min(j, Lk - 1);
-        if (ok) ok = mbar_wait(vec_full(x), (i >> 1) & 1, ctl);  // LSE / D staged
-        if (ok) ok = mbar_wait(s_full, i & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const float* lse2 = vec + x * 2 * kTile + c0w;
-        const float* dvv = vec + x * 2 * kTile + kTile + c0w;
-        uint32_t pr[64];  // S^T row, then P^T (fp32 bits)
-        tmem_ld64_sync(tS, pr);
-        const float4* lse4 = reinterpret_cast<const float4*>(lse2);
-        if (full) {
-#pragma unroll
-          for (int c4 = 0; c4 < kBlk / 4; ++c4) {
-            const float4 l = lse4[c4];
-            const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
-              if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
-              if constexpr (BIAS == kBiasDense)
-                xv = fmaf(bcol[static_cast<int64_t>(c) * p.sb_i], kLog2e, xv);
-              pr[c] = __float_as_uint(emu_exp2<BIAS, kBwdMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int c4 = 0; c4 < kBlk / 4; ++c4) {
-            const float4 l = lse4[c4];
-            const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              const bool vis = (c >= lo) && (c <= hi);
-              float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
-              if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
-              if constexpr (BIAS == kBiasDense)
-                xv = fmaf(bcol[static_cast<int64_t>(vis ? c : 0) * p.sb_i], kLog2e, xv);
-              pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
-            }
-          }
-        }
-#pragma unroll
-        for (int cc = 0; cc < kBlk; cc += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2)
-            pk[c >> 1] = pack_bf16x2(__uint_as_float(pr[cc + c]), __uint_as_float(pr[cc + c + 1]));
-          tmem_st16(tS + (cc >> 1), pk);  // P^T over the first 32 of this warpgroup's columns
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(p_full);
-        if (ok) ok = mbar_wait(dp_full, i & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        // the dS buffer is free once dQ(i - 1) and dK(i - 1) have read it
-        if (i > 0) ok = mbar_wait(ds_free, (i - 1) & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        float* ds_dst = nullptr;  // DS_OUT: fp32 dS of (query m0 + c, key j)
-        if constexpr (DS_OUT) {
-          if (j < Lk)
-            ds_dst = p.ds_out + static_cast<int64_t>(w.b) * p.sd_b +
-                     static_cast<int64_t>(hq) * p.sd_h + static_cast<int64_t>(m0) * p.sd_i + j;
-        }
-#pragma unroll
-        for (int cc = 0; cc < kBlk; cc += 16) {
-          uint32_t dr[16];
-          tmem_ld16_sync(tDP + cc, dr);
-          const float4* d4v = reinterpret_cast<const float4*>(dvv + cc);
-          uint32_t pk[8];  // dS as bf16 pairs, queries cc..cc+15
-#pragma unroll
-          for (int c = 0; c < 16; c += 4) {
-            const float4 dv4 = d4v[c >> 2];
-            const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dv4.x);
-            const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dv4.y);
-            const float d2 = __uint_as_float(pr[cc + c + 2]) * (__uint_as_float(dr[c + 2]) - dv4.z);
-            const float d3 = __uint_as_float(pr[cc + c + 3]) * (__uint_as_float(dr[c + 3]) - dv4.w);
-            pk[c >> 1] = pack_bf16x2(d0, d1);
-            pk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
-            if constexpr (DS_OUT) {
-              // neighbouring lanes hold neighbouring keys: each store of the
-              // warp writes 128 contiguous bytes of one query row; masked
-              // and out-of-range entries are 0 (P = 0); rows past Lq are skipped
-              if (ds_dst) {
-                const float dd[4] = {d0, d1, d2, d3};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (m0 + cc + c + e < Lq)
-                    __stcs(ds_dst + static_cast<int64_t>(cc + c + e) * p.sd_i, dd[e]);
-              }
-            }
-          }
-          // into this thread's row of the 128-byte swizzled dS tile (64
-          // queries = 128 bytes): 16-byte chunk q goes to position q ^ (row % 8)
-#pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            const int q = (cc >> 3) + q2;
-            *reinterpret_cast<uint4*>(ds_row + ((q ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * q2], pk[4 * q2 + 1], pk[4 * q2 + 2], pk[4 * q2 + 3]);
-          }
-        }
-        // dP^T is read: at d = 128 the dQ MMA writes those columns next
-        tc_fence_before();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(ds_full);
-        mbar_arrive(vec_empty(x));
+    for (int it = 0; it < total; ++it) {
+      const int x = it & 1;
+      const int hq = g * p.G + it / nm;
+      const int m0 = (mlo + it % nm) * kTile + c0w;  // first query of this warpgroup
+      const float* lut_row = nullptr;
+      if constexpr (BIAS == kBiasT5) {
+        // this warp's keys jw..jw+31 and queries m0..m0+63: j - i = (jw - m0 - 63) + e,
+        // e in [0, 94]; the thread reads entry lane + 63 - c for column c
+        const int base = n0 + (warp & 3) * 32 - m0 - (kBlk - 1);
+        __syncwarp();
+        for (int e = lane; e < 32 + kBlk - 1; e += 32) lut[e] = rel_bias_log2(p, base + e, hq);
+        __syncwarp();
+        lut_row = lut + lane + (kBlk - 1);
       }
-      if (!ok) break;
-      // ---------- item epilogue: warpgroup 0 stores dV, warpgroup 1 stores dK ----------
-      if (w.nb > 0) {
-        ok = mbar_wait(acc_done, u & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
+      // visible queries of this key among the warpgroup's 64: [lo, hi]
+      int lo = 0, hi = kBlk - 1;
+      bool full = (m0 + kBlk <= Lq) && (n0 + kTile <= Lk);
+      if (p.causal) full = full && (n0 + kTile - 1 <= m0);
+      if (p.wl >= 0) full = full && (m0 + kBlk - 1 <= n0 + p.wl);
+      if (p.wr >= 0) full = full && (n0 + kTile - 1 <= m0 + p.wr);
+      if (!full) {
+        if (p.causal) lo = max(lo, j - m0);
+        if (p.wr >= 0) lo = max(lo, j - p.wr - m0);
+        hi = min(hi, Lq - 1 - m0);
+        if (p.wl >= 0) hi = min(hi, j + p.wl - m0);
+        if (j >= Lk) hi = -1;  // past the key sequence: no query sees it
       }
+      const float* bcol = nullptr;
+      if constexpr (BIAS == kBiasDense)
+        bcol = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
+               static_cast<int64_t>(min(m0, Lq - 1)) * p.sb_i + min(j, Lk - 1);
+      if (ok) ok = mbar_wait(vec_full(x), (it >> 1) & 1, ctl);  // LSE / D staged
+      if (ok) ok = mbar_wait(s_full, it & 1, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      tc_fence_after();
+      const float* lse2 = vec + x * 2 * kTile + c0w;
+      const float* dvv = vec + x * 2 * kTile + kTile + c0w;
+      uint32_t pr[64];  // S^T row, then P^T (fp32 bits)
+      tmem_ld64_sync(tS, pr);
+      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+      if (full) {
+#pragma unroll
+        for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+          const float4 l = lse4[c4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            if constexpr (BIAS == kBiasDense)
+              xv = fmaf(bcol[static_cast<int64_t>(c) * p.sb_i], kLog2e, xv);
+            pr[c] = __float_as_uint(emu_exp2<BIAS, kDkdvMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+          const float4 l = lse4[c4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const bool vis = (c >= lo) && (c <= hi);
+            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            if constexpr (BIAS == kBiasDense)
+              xv = fmaf(bcol[static_cast<int64_t>(vis ? c : 0) * p.sb_i], kLog2e, xv);
+            pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+          }
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < kBlk; cc += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2)
+          pk[c >> 1] = pack_bf16x2(__uint_as_float(pr[cc + c]), __uint_as_float(pr[cc + c + 1]));
+        tmem_st16(tS + (cc >> 1), pk);  // P^T over the first 32 of this warpgroup's columns
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      if (ok) ok = mbar_wait(dp_full, it & 1, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < kBlk; cc += 32) {
+        uint32_t dr[32];
+        tmem_ld32_sync(tDP + cc, dr);
+        uint32_t pk[16];
+        const float4* d4v = reinterpret_cast<const float4*>(dvv + cc);
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 dv4 = d4v[c >> 2];
+          const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dv4.x);
+          const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dv4.y);
+          const float d2 = __uint_as_float(pr[cc + c + 2]) * (__uint_as_float(dr[c + 2]) - dv4.z);
+          const float d3 = __uint_as_float(pr[cc + c + 3]) * (__uint_as_float(dr[c + 3]) - dv4.w);
+          pk[c >> 1] = pack_bf16x2(d0, d1);
+          pk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
+        }
+        tmem_st16(tDP + (cc >> 1), pk);  // dS^T over the first 32 of this warpgroup's columns
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+      mbar_arrive(vec_empty(x));
+    }
+    // ---------------- epilogue: warpgroup 0 stores dV, warpgroup 1 stores dK ----------------
+    if (ok && total > 0) ok = mbar_wait(acc_done, 0, ctl);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
       // lanes 2m, 2m + 1 hold keys j, j + 1 and trade halves of every 16
       // columns, so each 16-byte store of the pair fills one 32-byte sector
       const bool odd = (lane & 1) != 0;
       const int ja = j - (odd ? 1 : 0);
-      const int64_t off = static_cast<int64_t>(w.b) * p.skv_b + static_cast<int64_t>(w.s.k0 + ja) * p.skv_l +
-                          static_cast<int64_t>(w.g) * p.skv_h + (odd ? 8 : 0);
+      const int64_t off = static_cast<int64_t>(s.bc) * p.skv_b +
+                          static_cast<int64_t>(s.k0 + ja) * p.skv_l +
+                          static_cast<int64_t>(g) * p.skv_h + (odd ? 8 : 0);
       __nv_bfloat16* dst_a = (wg == 0 ? p.dv : p.dk) + off;
       __nv_bfloat16* dst_b = dst_a + p.skv_l;
       const float mul = wg == 0 ? 1.f : p.scale;
@@ -900,7 +518,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
-        if (w.nb > 0) {
+        if (total > 0) {
           tmem_ld32_sync(tcol + c, r);
         } else {
 #pragma unroll
@@ -917,10 +535,566 @@ __global__ void __launch_bounds__(512, 1)
           if (ja + 1 < Lk) *reinterpret_cast<uint4*>(dst_b + c + h) = vb;
         }
       }
-      if (w.nb > 0) {
-        tc_fence_before();
-        mbar_arrive(acc_free);  // the next item's first dV / dK MMA may overwrite
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------------- dQ
+// Persistent: one CTA per SM walks a heavy-first list of work items, each 128
+// queries of one (query head, batch entry); blocks of 128 keys stream through;
+// warpgroup w takes the key columns [64 w, 64 w + 64).  Ring, buffer and
+// barrier indices count across items, so the next item's Q / dO load and
+// first scores overlap the current item's last blocks and epilogue.  Tensor
+// memory: S[0] 0..127 | S[1] 128..255 | dP 256..383 | dQ 384..  The scores
+// are double-buffered, so S of block i + 1 is computed while block i's dS is
+// formed.  dS (bf16) goes over the first half of each warpgroup's columns of
+// its own, already loaded, S buffer: dP of block i + 1 can then be computed
+// as soon as block i's dP has been loaded, and S of block i + 2 waits only
+// for the dQ MMA of block i.
+template <int D, int BIAS>
+struct DqLayout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  // Dense bias at d = 64: each block's 128 x 128 fp32 bias comes by TMA into
+  // a 2-stage ring (4 boxes of 128 rows x 32 columns, 128-byte swizzle).
+  static constexpr bool kBiasTma = (BIAS == kBiasDense && D == 64);
+  static constexpr int kBiasTileBytes = kTile * kTile * 4;
+  static constexpr int kSB = kBiasTma ? 2 : 0;
+  // K blocks are used until the block's dQ MMA, V blocks only until its dP
+  // MMA: the K ring is the deeper one.
+  static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : (kBiasTma ? 2 : 4);
+  static constexpr int kSV = (D == 128) ? 2 : (kBiasTma ? 2 : 3);
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kTileBytes;
+  static constexpr int kKOff = 2 * kTileBytes;                // K ring
+  static constexpr int kVOff = kKOff + kSK * kTileBytes;      // V ring
+  static constexpr int kBOff = kVOff + kSV * kTileBytes;      // bias ring (kBiasTma)
+  static constexpr int kLutOff = kBOff + kSB * kBiasTileBytes;  // T5 only: 8 warps x 96 floats
+  static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
+  static constexpr int kBarOff = kLutOff + kLutBytes;
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
+  // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
+  // b_full[2], b_empty[2]
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 18;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemAlloc = kMiscOff + 16;
+  static constexpr int kThreads = 352;  // 2 compute warpgroups, producer, two MMA issuers
+  static constexpr int kTmemCols = 512;
+  static constexpr int kDPCol = 256, kDQCol = 384;
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+};
+
+// DS_OUT: also store dS in fp32 through p.ds_out (the bias gradient path).
+template <int D, int BIAS, bool DS_OUT = false>
+__global__ void __launch_bounds__(352, 1)
+    bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
+  using Lay = DqLayout<D, BIAS>;
+  constexpr int SK = Lay::kSK;
+  constexpr int SV = Lay::kSV;
+  extern __shared__ uint8_t smem[];
+  if (!smem_base_ok(smem)) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusMisaligned);
+    return;
+  }
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work items: (query tile, head, batch), heaviest causal query tiles
+  // first; consecutive items are neighbouring heads, which share K / V in L2.
+  const int nqt = (p.Lq + kTile - 1) / kTile;
+  const int heads = p.Hq * p.B;
+  const int n_items = nqt * heads;
+  struct Item {
+    int m0, hq, b, g, nlo, nt;
+    bool rows;  // the query tile holds queries of the sequence
+    SeqView s;
+  };
+  auto item_at = [&](int id) {
+    Item w;
+    const int r = id / heads;
+    const int rem = id - r * heads;
+    const int qt = p.causal ? nqt - 1 - r : r;
+    w.m0 = qt * kTile;
+    w.hq = rem % p.Hq;
+    w.b = rem / p.Hq;
+    w.g = w.hq / p.G;
+    w.s = seq_view(p, w.b);
+    w.rows = w.m0 < w.s.Lq;
+    w.nlo = 0;
+    w.nt = 0;
+    if (w.rows) {
+      int nhi;
+      key_tile_range(p, w.s.Lq, w.s.Lk, w.m0, kTile, w.nlo, nhi);
+      w.nt = nhi > w.nlo ? nhi - w.nlo : 0;
+    }
+    return w;
+  };
+
+  auto bar = [&](int idx) -> uint32_t { return sb + Lay::kBarOff + 8 * idx; };
+  const uint32_t q_full = bar(0);
+  auto k_full = [&](int s) { return bar(1 + s); };
+  auto k_empty = [&](int s) { return bar(1 + SK + s); };
+  auto v_full = [&](int s) { return bar(1 + 2 * SK + s); };
+  auto v_empty = [&](int s) { return bar(1 + 2 * SK + SV + s); };
+  constexpr int kB = 1 + 2 * SK + 2 * SV;
+  auto s_full = [&](int x) { return bar(kB + x); };
+  auto dq_done = [&](int x) { return bar(kB + 2 + x); };  // dQ MMA of a block in buffer x done
+  const uint32_t dp_full = bar(kB + 4);
+  const uint32_t dp_used = bar(kB + 5);
+  // dS of block i ready, by block parity: the dQ issuer issues dP(i + 1)
+  // before it waits for dS(i), so the warpgroups can finish dS(i + 1) before
+  // it looks; a single barrier would then have completed two phases and the
+  // wait for block i's parity would never succeed.
+  auto ds_full = [&](int x) { return x == 0 ? bar(kB + 6) : bar(kB + 13); };
+  const uint32_t acc_done = bar(kB + 7);
+  auto drain = [&](int x) { return bar(kB + 8 + x); };
+  // Q is read only by the score issuer, dO only by the dP issuer: each tile is
+  // released as soon as its one reader is done with the item
+  const uint32_t q_empty = bar(kB + 10);
+  const uint32_t o_full = bar(kB + 11);
+  const uint32_t o_empty = bar(kB + 12);
+  auto b_full = [&](int x) { return bar(kB + 14 + x); };
+  auto b_empty = [&](int x) { return bar(kB + 16 + x); };
+  constexpr bool BT = Lay::kBiasTma;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(b_full(x), 1);
+      mbar_init(b_empty(x), 2 * kTile);
+    }
+    // K blocks are read by both issuers (S and dQ): a slot is free once each
+    // issuer's last MMA on it has completed.
+    for (int s = 0; s < SK; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 2);
+    }
+    for (int s = 0; s < SV; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(dq_done(x), 1);
+    }
+    mbar_init(dp_full, 1);
+    mbar_init(dp_used, 2 * kTile);
+    mbar_init(ds_full(0), 2 * kTile);
+    mbar_init(ds_full(1), 2 * kTile);
+    mbar_init(acc_done, 1);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.wait_limit_ns};
+
+  if (warp == 8) {
+    // ============================ producer ============================
+    // Per item: Q and dO once (each after its reader is done with the
+    // previous item's), then K and V of every key block into their rings.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int issued_k[SK], issued_v[SV];
+      for (int s = 0; s < SK; ++s) issued_k[s] = -1;
+      for (int s = 0; s < SV; ++s) issued_v[s] = -1;
+      int q_issued = -1, o_issued = -1;
+      int b_issued[2] = {-1, -1};
+      int c = 0;  // key blocks so far, over all items
+      int u = 0;  // items with a non-empty band so far
+      bool ok = true;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (u > 0 && !(ok = mbar_wait(q_empty, (u - 1) & 1, ctl))) break;
+        mbar_expect_tx(q_full, Lay::kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(sb + Lay::kQOff + h * kTile * 128, &tmQ, q_full, h * 64, w.s.q0 + w.m0,
+                      w.hq, w.s.bc);
+        q_issued = u & 1;
+        if (u > 0 && !(ok = mbar_wait(o_empty, (u - 1) & 1, ctl))) break;
+        mbar_expect_tx(o_full, Lay::kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(sb + Lay::kDOOff + h * kTile * 128, &tmDO, o_full, h * 64, w.s.q0 + w.m0,
+                      w.hq, w.s.bc);
+        o_issued = u & 1;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int sk = c % SK, sv = c % SV;
+          const int n0 = (w.nlo + it) * kTile;
+          if (!(ok = mbar_wait(k_empty(sk), ((c / SK) & 1) ^ 1, ctl))) break;
+          mbar_expect_tx(k_full(sk), Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
+                        k_full(sk), h * 64, w.s.k0 + n0, w.g, w.s.bc);
+          issued_k[sk] = (c / SK) & 1;
+          if constexpr (BT) {
+            // this block's bias: rows m0.., keys n0.. of (b, hq), 4 boxes
+            const int x = c & 1;
+            const uint32_t bph = (c >> 1) & 1;
+            if (!(ok = mbar_wait(b_empty(x), bph ^ 1, ctl))) break;
+            mbar_expect_tx(b_full(x), Lay::kBiasTileBytes);
+            const int hb = p.sb_h ? w.hq : 0, bb = p.sb_b ? w.b : 0;
+            for (int q4 = 0; q4 < 4; ++q4)
+              tma_load_4d(sb + Lay::kBOff + x * Lay::kBiasTileBytes + q4 * (kTile * 128), &tmB,
+                          b_full(x), n0 + 32 * q4, w.m0, hb, bb);
+            b_issued[x] = static_cast<int>(bph);
+          } else if constexpr (BIAS == kBiasDense) {
+            prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
+          }
+          if (!(ok = mbar_wait(v_empty(sv), ((c / SV) & 1) ^ 1, ctl))) break;
+          mbar_expect_tx(v_full(sv), Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kVOff + sv * Lay::kTileBytes + h * kTile * 128, &tmV,
+                        v_full(sv), h * 64, w.s.k0 + n0, w.g, w.s.bc);
+          issued_v[sv] = (c / SV) & 1;
+        }
         ++u;
+      }
+      if (!ok) {
+        volatile int never = 0;
+        const WaitCtl ign{&never, p.wait_limit_ns};
+        if (q_issued >= 0) mbar_wait(q_full, q_issued, ign);
+        if (o_issued >= 0) mbar_wait(o_full, o_issued, ign);
+        for (int x = 0; x < 2; ++x)
+          if (b_issued[x] >= 0) mbar_wait(b_full(x), b_issued[x], ign);
+        for (int s = 0; s < SK; ++s)
+          if (issued_k[s] >= 0) mbar_wait(k_full(s), issued_k[s], ign);
+        for (int s = 0; s < SV; ++s)
+          if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
+      }
+    }
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers (one thread each) =====================
+    // Warp 9 runs the score chain: S(i) into buffer i % 2 once K(i) has landed
+    // and the dQ MMA of block i - 2 has read dS out of that buffer.  Warp 10
+    // runs dP one block ahead of dQ within an item: dP(i + 1) as soon as both
+    // warpgroups have loaded dP(i), then dQ(i) once dS(i) is ready.  Block
+    // indices run on across items.
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
+      constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
+      const bool chain_s = (warp == 9);
+      auto issue_dp = [&](int c) -> bool {
+        const int sv = c % SV;
+        if (!issuer_wait(v_full(sv), (c / SV) & 1, ctl)) return false;
+        if (c > 0 && !issuer_wait(dp_used, (c - 1) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + Lay::kDPCol,
+                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
+                 smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(dp_full);
+        mma_commit(v_empty(sv));
+        return true;
+      };
+      int c = 0;  // key blocks so far, over all items
+      int u = 0;  // items with a non-empty band so far
+      bool ok = true;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (!(ok = issuer_wait(chain_s ? q_full : o_full, u & 1, ctl))) break;
+        if (!chain_s && !(ok = issue_dp(c))) break;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int x = c & 1;
+          const int sk = c % SK;
+          const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+          if (chain_s) {
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (c >= 2 && !(ok = issuer_wait(dq_done(x), ((c >> 1) - 1) & 1, ctl))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + kTile * x,
+                     smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
+                     smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(s_full(x));
+            mma_commit(k_empty(sk));
+          } else {
+            if (it + 1 < w.nt && !(ok = issue_dp(c + 1))) break;
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (!(ok = issuer_wait(ds_full(c & 1), (c >> 1) & 1, ctl))) break;
+            tc_fence_after();
+            // the item's first dQ MMA overwrites the accumulator: every
+            // warpgroup thread read the previous item's dQ before marking dS ready
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk),
+                     smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(dq_done(x));
+            mma_commit(k_empty(sk));
+          }
+        }
+        if (!ok) break;
+        mma_commit(chain_s ? q_empty : o_empty);  // the item's Q / dO is read
+        if (!chain_s) mma_commit(acc_done);
+        ++u;
+      }
+      if (!ok) {
+        volatile int never = 0;
+        const WaitCtl ign{&never, p.wait_limit_ns};
+        mma_commit(drain(chain_s ? 0 : 1));
+        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
+      }
+    }
+  } else {
+    // ===== compute warpgroup wg: key columns [64 wg, 64 wg + 64); thread = query row =====
+    const int wg = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const int c0w = kBlk * wg;
+    const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
+    float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
+    bool ok = true;
+    int c = 0;  // key blocks so far, over all items
+    int u = 0;  // items with a non-empty band so far
+    for (int id = blockIdx.x; id < n_items; id += gridDim.x) {
+      const Item w = item_at(id);
+      if (!w.rows) continue;  // past this entry's query sequence: nothing to write
+      const int m0 = w.m0, hq = w.hq, b = w.b, nt = w.nt;
+      const int Lq = w.s.Lq, Lk = w.s.Lk;
+      const int i = m0 + row;
+      float l2 = INFINITY, dd = 0.f;
+      if (i < Lq) {
+        const int64_t idx = row_index(p, w.s, b, hq, i);
+        l2 = p.lse[idx] * kLog2e;
+        dd = p.dvec[idx];
+        if (l2 == -INFINITY) l2 = INFINITY;
+      }
+      const float* brow = nullptr;
+      if constexpr (BIAS == kBiasDense)
+        brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
+               static_cast<int64_t>(min(i, Lq - 1)) * p.sb_i;
+      for (int it = 0; it < nt; ++it, ++c) {
+        const int x = c & 1;
+        const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup
+        const float* lut_row = nullptr;
+        if constexpr (BIAS == kBiasT5) {
+          // this warp's queries iw..iw+31 and keys n0..n0+63: j - i = (n0 - iw - 31) + e,
+          // e in [0, 94]; the thread reads entry 31 - lane + cc for column cc
+          const int base = n0 - m0 - (warp & 3) * 32 - 31;
+          __syncwarp();
+          for (int e = lane; e < 32 + kBlk - 1; e += 32) lut[e] = rel_bias_log2(p, base + e, hq);
+          __syncwarp();
+          lut_row = lut + 31 - lane;
+        }
+        int lo = 0, hi = kBlk - 1;
+        bool full = n0 + kBlk <= Lk;
+        if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
+        if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
+        if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
+        if (!full) {
+          if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
+          hi = min(hi, Lk - 1 - n0);
+          if (p.causal) hi = min(hi, i - n0);
+          if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
+        }
+        if (ok) ok = mbar_wait(s_full(x), (c >> 1) & 1, ctl);
+        if constexpr (BT) {
+          if (ok) ok = mbar_wait(b_full(c & 1), (c >> 1) & 1, ctl);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) continue;
+        tc_fence_after();
+        const uint32_t tSx = tmem + lane_bits + kTile * x + c0w;
+        uint32_t pr[64];  // S row, then P (fp32 bits)
+        tmem_ld64_sync(tSx, pr);
+        if constexpr (BT) {
+          // this warpgroup's 64 bias columns from the staged block: boxes
+          // 2 wg and 2 wg + 1, row `row`, 8 swizzled 16-byte chunks each
+          const uint8_t* bt = smem + Lay::kBOff + (c & 1) * Lay::kBiasTileBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t* brw = bt + (2 * wg + h) * (kTile * 128) + row * 128;
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 b4 = *reinterpret_cast<const float4*>(brw + ((k4 ^ (row & 7)) << 4));
+              const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int cc = 32 * h + 4 * k4 + e;
+                const float xv = fmaf(bv[e], kLog2e, fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2));
+                pr[cc] = __float_as_uint(fast_exp2(full || (cc >= lo && cc <= hi) ? xv : -INFINITY));
+              }
+            }
+          }
+          mbar_arrive(b_empty(c & 1));  // the bias block is read
+        } else if (full && BIAS == kBiasDense) {
+          // the row's 64 bias values as 16-byte loads, 32 at a time
+          const float4* b4 = reinterpret_cast<const float4*>(brow + n0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float4 bb[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) bb[q] = b4[8 * h + q];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float bv[4] = {bb[q].x, bb[q].y, bb[q].z, bb[q].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int cc = 32 * h + 4 * q + e;
+                const float xv = fmaf(bv[e], kLog2e, fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2));
+                pr[cc] = __float_as_uint(fast_exp2(xv));
+              }
+            }
+          }
+        } else if (full) {
+#pragma unroll
+          for (int cc = 0; cc < kBlk; ++cc) {
+            float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
+            pr[cc] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(cc) ? exp2_fma(xv) : fast_exp2(xv));
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < kBlk; ++cc) {
+            const bool vis = (cc >= lo) && (cc <= hi);
+            float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
+            if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
+            if constexpr (BIAS == kBiasDense) xv += vis ? brow[n0 + cc] * kLog2e : 0.f;
+            pr[cc] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+          }
+        }
+        if (ok) ok = mbar_wait(dp_full, c & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) continue;
+        tc_fence_after();
+        uint32_t pk[32];  // dS as bf16 pairs
+#pragma unroll
+        for (int cc = 0; cc < kBlk; cc += 32) {
+          uint32_t dr[32];
+          tmem_ld32_sync(tDP + cc, dr);
+          if (cc + 32 == kBlk) {
+            tc_fence_before();
+            mbar_arrive(dp_used);  // the dP columns may now take the next block
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float d0 = __uint_as_float(pr[cc + e]) * (__uint_as_float(dr[e]) - dd);
+            const float d1 = __uint_as_float(pr[cc + e + 1]) * (__uint_as_float(dr[e + 1]) - dd);
+            pk[(cc + e) >> 1] = pack_bf16x2(d0, d1);
+            if constexpr (DS_OUT) {  // P is spent: keep the fp32 dS in its place
+              pr[cc + e] = __float_as_uint(d0);
+              pr[cc + e + 1] = __float_as_uint(d1);
+            }
+          }
+        }
+        // dS over the first 32 of this warpgroup's columns of its S buffer
+        tmem_st16(tSx, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        tmem_st16(tSx + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(ds_full(c & 1));
+        if constexpr (DS_OUT) {
+          // fp32 dS of this row's 64 keys while the dQ MMA runs; masked keys
+          // have P = 0 and so dS = 0.  Lanes 2m and 2m + 1 hold neighbouring
+          // rows; for every 8 keys they swap four values so that each store
+          // writes one whole 32-byte piece of a row from two lanes (the even
+          // lane's row first, then the odd lane's), rather than every lane
+          // half a piece of its own row.  Streaming stores: dS is not read
+          // again here and should not evict the K / V tiles that
+          // neighbouring heads reuse from L2.
+          const int64_t head_off = static_cast<int64_t>(b) * p.sd_b + static_cast<int64_t>(hq) * p.sd_h;
+          if (n0 + kBlk <= Lk) {
+            const bool odd = (lane & 1) != 0;
+            const int i_a = odd ? i - 1 : i;  // the even lane's row
+            const int i_b = odd ? i : i + 1;  // the odd lane's row
+            const int c_off = n0 + (odd ? 4 : 0);
+            float* row_a = p.ds_out + head_off + static_cast<int64_t>(i_a) * p.sd_i + c_off;
+            float* row_b = p.ds_out + head_off + static_cast<int64_t>(i_b) * p.sd_i + c_off;
+#pragma unroll
+            for (int g = 0; g < kBlk; g += 8) {
+              float lo[4], hi[4], got[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                lo[t] = __uint_as_float(pr[g + t]);
+                hi[t] = __uint_as_float(pr[g + 4 + t]);
+              }
+              // the even lane sends its keys g+4..g+7, the odd lane its g..g+3
+#pragma unroll
+              for (int t = 0; t < 4; ++t) got[t] = __shfl_xor_sync(0xffffffffu, odd ? lo[t] : hi[t], 1);
+              const float4 va = odd ? make_float4(got[0], got[1], got[2], got[3])
+                                    : make_float4(lo[0], lo[1], lo[2], lo[3]);
+              const float4 vb = odd ? make_float4(hi[0], hi[1], hi[2], hi[3])
+                                    : make_float4(got[0], got[1], got[2], got[3]);
+              if (i_a < Lq) __stcs(reinterpret_cast<float4*>(row_a + g), va);
+              if (i_b < Lq) __stcs(reinterpret_cast<float4*>(row_b + g), vb);
+            }
+          } else if (i < Lq) {
+            float* dst = p.ds_out + head_off + static_cast<int64_t>(i) * p.sd_i + n0;
+#pragma unroll
+            for (int e = 0; e < kBlk; ++e)
+              if (n0 + e < Lk) __stcs(dst + e, __uint_as_float(pr[e]));
+          }
+        }
+      }
+      // ----------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -----------
+      // Items without a visible key (none exist for the masks accepted at the
+      // boundary) store zeros without touching tensor memory.
+      if (nt > 0) {
+        if (ok) ok = mbar_wait(acc_done, u & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        ++u;
+      }
+      if (ok) {
+        uint32_t r[D / 2];
+        if (nt > 0) {
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 2; cc += 32)
+            tmem_ld32_sync(tmem + lane_bits + Lay::kDQCol + wg * (D / 2) + cc,
+                           *reinterpret_cast<uint32_t(*)[32]>(r + cc));
+        } else {
+#pragma unroll
+          for (int e = 0; e < D / 2; ++e) r[e] = 0u;
+        }
+        // lanes 2m, 2m + 1 hold rows i, i + 1 and trade halves of every 16
+        // columns, so each 16-byte store of the pair fills one 32-byte sector
+        const bool odd = (lane & 1) != 0;
+        const int ia = i - (odd ? 1 : 0);
+        __nv_bfloat16* dst_a = p.dq + static_cast<int64_t>(w.s.bc) * p.sq_b +
+                               static_cast<int64_t>(w.s.q0 + ia) * p.sq_l +
+                               static_cast<int64_t>(hq) * p.sq_h + wg * (D / 2) + (odd ? 8 : 0);
+        __nv_bfloat16* dst_b = dst_a + p.sq_l;
+#pragma unroll
+        for (int cc = 0; cc < D / 2; cc += 16) {
+          uint4 lo4, hi4;
+          pack16(r + cc, p.scale, lo4, hi4);
+          const uint4 got = shfl_xor_u4(odd ? lo4 : hi4, 1);
+          const uint4 va = odd ? got : lo4;  // row ia
+          const uint4 vb = odd ? hi4 : got;  // row ia + 1
+          if (ia < Lq) *reinterpret_cast<uint4*>(dst_a + cc) = va;
+          if (ia + 1 < Lq) *reinterpret_cast<uint4*>(dst_b + cc) = vb;
+        }
       }
     }
   }
@@ -935,54 +1109,58 @@ __global__ void __launch_bounds__(512, 1)
 
 // ------------------------------------------------------------- launchers
 // Launch selection bits of the backward (sdpa_bwd_phases).
-constexpr uint32_t kPhasePre = 1u, kPhaseGrads = 2u;
+constexpr uint32_t kPhasePre = 1u, kPhaseDq = 2u, kPhaseDkdv = 4u;
 
-// Workspace of the backward, in this order, each part 256-byte aligned:
-// D [rows] fp32 | turn counters [B * Hq * ceil(Lq / 128) * 4] u32 + the
-// ticket counter | dQ accumulator [rows * d] fp32, rows = the LSE rows
-// (B * Hq * Lq, or Hq * total rows when packed).
+// Workspace of the backward: D [rows] fp32, rows = the LSE rows
+// (B * Hq * Lq, or Hq * total rows when packed), 256-byte rounded.
 struct BwdWorkspace {
-  size_t d_off, turn_off, acc_off, total;
-  int64_t n_turns;
+  size_t d_off, total;
 };
 
-inline BwdWorkspace bwd_workspace_plan(int64_t rows, int64_t B, int64_t Hq, int64_t Lq, int64_t d) {
-  auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+inline BwdWorkspace bwd_workspace_plan(int64_t rows) {
   BwdWorkspace w;
-  w.n_turns = B * Hq * ((Lq + kTile - 1) / kTile) * 4;
   w.d_off = 0;
-  w.turn_off = r256(static_cast<size_t>(rows) * 4);
-  w.acc_off = w.turn_off + r256(static_cast<size_t>(w.n_turns + 1) * 4);
-  w.total = w.acc_off + r256(static_cast<size_t>(rows) * static_cast<size_t>(d) * 4);
+  w.total = (static_cast<size_t>(rows) * 4 + 255) / 256 * 256;
   return w;
 }
 
 template <int D, int BIAS>
 cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const CUtensorMap& mdo, uint32_t phases,
-                         int64_t n_axis, int64_t n_turns, cudaStream_t st) {
+                         const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mb,
+                         uint32_t phases, int64_t n_axis, cudaStream_t st) {
   if (phases & kPhasePre) {
-    const int64_t threads = std::max(n_axis * p.Hq * (D / 8), n_turns + 1);
+    const int64_t threads = n_axis * p.Hq * (D / 8);
     const int64_t blocks = (threads + 255) / 256;
-    bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, n_axis, n_turns);
+    bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, n_axis);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (phases & kPhaseGrads) {
-    using Lay = BwdLayout<D, BIAS>;
-    auto kern = bwd_kernel<D, BIAS, false>;
+  if (phases & kPhaseDq) {
+    using Lay = DqLayout<D, BIAS>;
+    auto kern = bwd_dq_kernel<D, BIAS>;
     if constexpr (BIAS != kBiasNone) {
-      if (p.ds_out) kern = bwd_kernel<D, BIAS, true>;
+      if (p.ds_out) kern = bwd_dq_kernel<D, BIAS, true>;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (or per work item, if fewer)
-    const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * ((p.Lk + kTile - 1) / kTile);
+    const int64_t items = static_cast<int64_t>((p.Lq + kTile - 1) / kTile) * p.Hq * p.B;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
     kern<<<static_cast<int>(items < sms ? items : sms), Lay::kThreads, Lay::kSmemAlloc, st>>>(
-        p, mq, mk, mv, mdo);
+        p, mq, mk, mv, mdo, mb);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (phases & kPhaseDkdv) {
+    using Lay = DkdvLayout<D, BIAS>;
+    auto kern = bwd_dkdv_kernel<D, BIAS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Lay::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    const int ntk = (p.Lk + kTile - 1) / kTile;
+    kern<<<dim3(ntk, p.Hkv, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(p, mq, mk, mv, mdo);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -991,12 +1169,12 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
 
 template <int D>
 cudaError_t launch_bwd_d(const AttnParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const CUtensorMap& mdo, uint32_t phases,
-                         int64_t n_axis, int64_t n_turns, cudaStream_t st) {
+                         const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mb,
+                         uint32_t phases, int64_t n_axis, cudaStream_t st) {
   switch (p.bias_kind) {
-    case kBiasDense: return launch_bwd_t<D, kBiasDense>(p, mq, mk, mv, mdo, phases, n_axis, n_turns, st);
-    case kBiasT5: return launch_bwd_t<D, kBiasT5>(p, mq, mk, mv, mdo, phases, n_axis, n_turns, st);
-    default: return launch_bwd_t<D, kBiasNone>(p, mq, mk, mv, mdo, phases, n_axis, n_turns, st);
+    case kBiasDense: return launch_bwd_t<D, kBiasDense>(p, mq, mk, mv, mdo, mb, phases, n_axis, st);
+    case kBiasT5: return launch_bwd_t<D, kBiasT5>(p, mq, mk, mv, mdo, mb, phases, n_axis, st);
+    default: return launch_bwd_t<D, kBiasNone>(p, mq, mk, mv, mdo, mb, phases, n_axis, st);
   }
 }
 

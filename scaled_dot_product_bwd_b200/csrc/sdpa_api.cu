@@ -311,9 +311,7 @@ sdpa_status_t run_fwd(const Geometry& g, const void* q, const void* k, const voi
 }
 
 // ------------------------------------------------------------ backward
-BwdWorkspace plan_of(const Geometry& g) {
-  return bwd_workspace_plan(g.rows(), g.B, g.Hq, g.Lq, g.d);
-}
+BwdWorkspace plan_of(const Geometry& g) { return bwd_workspace_plan(g.rows()); }
 
 // The backward's pointers, with its workspace (laid out by plan_of) at ws.
 sdpa_status_t bind_bwd(AttnParams& p, const Geometry& g, const void* o, const void* dout,
@@ -327,23 +325,20 @@ sdpa_status_t bind_bwd(AttnParams& p, const Geometry& g, const void* o, const vo
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dvec = reinterpret_cast<float*>(w + pl.d_off);
-  p.turns = reinterpret_cast<unsigned int*>(w + pl.turn_off);
-  p.tickets = p.turns + pl.n_turns;
-  p.dq_acc = reinterpret_cast<float*>(w + pl.acc_off);
   return SDPA_OK;
 }
 
 // Tensor maps, then the launches selected by `phases`.
 sdpa_status_t run_bwd(uint32_t phases, const AttnParams& p, const Geometry& g, const void* q,
                       const void* k, const void* v, const void* dout, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mb;
   if (!make_axis_map(&mq, q, g, true) || !make_axis_map(&mdo, dout, g, true) ||
       !make_axis_map(&mk, k, g, false) || !make_axis_map(&mv, v, g, false))
     return SDPA_ERR_CUDA;
-  const BwdWorkspace pl = plan_of(g);
-  cudaError_t e =
-      g.d == 128 ? launch_bwd_d<128>(p, mq, mk, mv, mdo, phases, g.axis_q(), pl.n_turns, stream)
-                 : launch_bwd_d<64>(p, mq, mk, mv, mdo, phases, g.axis_q(), pl.n_turns, stream);
+  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias dQ kernel at d = 64
+  if (p.bias_kind == kBiasDense && !make_bias_map(&mb, p)) return SDPA_ERR_CUDA;
+  cudaError_t e = g.d == 128 ? launch_bwd_d<128>(p, mq, mk, mv, mdo, mb, phases, g.axis_q(), stream)
+                             : launch_bwd_d<64>(p, mq, mk, mv, mdo, mb, phases, g.axis_q(), stream);
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
@@ -496,16 +491,6 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
     (void)mbar_wait(smem_u32(&bar_storage), 0, ctl);
   }
   __syncthreads();
-}
-
-// One dQ turn that nothing ever passes, waited on under the wait limit by
-// one warp, the way the backward's reducer warps wait for theirs.
-__global__ void turn_timeout_kernel(const unsigned int* ctr, uint64_t limit_ns) {
-  __shared__ int abort_flag;
-  if (threadIdx.x == 0) abort_flag = 0;
-  __syncwarp();
-  const WaitCtl ctl{&abort_flag, limit_ns};
-  (void)wait_turn(ctr, 0xffffffffu, ctl);
 }
 
 }  // namespace
@@ -791,12 +776,6 @@ sdpa_status_t sdpa_read_device_status(void* stream) {
 
 sdpa_status_t sdpa_debug_wait_timeout(void* stream) {
   wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_limit_ns);
-  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
-}
-
-sdpa_status_t sdpa_debug_turn_timeout(const uint32_t* counter, void* stream) {
-  if (!counter || (reinterpret_cast<uintptr_t>(counter) & 3u)) return SDPA_ERR_INVALID_ARG;
-  turn_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(counter, g_wait_limit_ns);
   return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 

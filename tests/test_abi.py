@@ -112,15 +112,11 @@ def test_bwd_rejects_bad_args(lib):
 
 
 def test_bwd_workspace_layout(lib):
-    # D (one float per LSE entry), the dQ turn counters (4 per 128 query rows
-    # of each head) plus the ticket word, and the float32 dQ accumulator
-    # (d floats per LSE entry), each rounded up to 256 bytes.
+    # D, one float per LSE entry, rounded up to 256 bytes.
     r256 = lambda x: (x + 255) // 256 * 256
     for B, L, Hq, d, Lk in ((1, 128, 4, 64, 0), (2, 300, 4, 128, 0), (3, 37, 2, 64, 1000)):
         s = _shape(B=B, L=L, Hq=Hq, d=d, Lk=Lk)
-        rows = B * Hq * L
-        turns = B * Hq * ((L + 127) // 128) * 4
-        want = r256(rows * 4) + r256((turns + 1) * 4) + r256(rows * d * 4)
+        want = r256(B * Hq * L * 4)
         assert lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1) == want
     assert lib.sdpa_bwd_workspace_size(ctypes.byref(_shape(Lk=-1)), 1) == 0
 
@@ -129,7 +125,7 @@ def test_bwd_phases_rejects_bad_bits(lib):
     s = _shape()
     m = binding.MaskSpec(1, -1, -1)
     ws = lib.sdpa_bwd_workspace_size(ctypes.byref(s), 1)
-    for ph in (0, 4, 7):
+    for ph in (0, 8, 9, 16, 0x80000007):
         assert lib.sdpa_bwd_phases(ph, ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
                                    ctypes.byref(m), 0.125, FAKE, FAKE, FAKE, 1, FAKE, ws,
                                    None) == 1
@@ -137,8 +133,9 @@ def test_bwd_phases_rejects_bad_bits(lib):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
     m = binding.MaskSpec(1, -1, -1)
-    big = _shape(B=1, L=65536, Hq=4, d=128, sq_b=65536 * 4 * 128, sq_l=4 * 128, sq_h=128,
-                 skv_b=65536 * 2 * 128, skv_l=2 * 128, skv_h=128)
+    L = 1 << 20  # B * Hq * L = 8M LSE entries: 32 MiB of D
+    big = _shape(B=1, L=L, Hq=8, d=64, sq_b=L * 8 * 64, sq_l=8 * 64, sq_h=64,
+                 skv_b=L * 2 * 64, skv_l=2 * 64, skv_h=64)
     assert lib.sdpa_bwd_workspace_size(ctypes.byref(big), 1) > binding.NOALLOC_SCRATCH_BYTES
     assert lib.sdpa_bwd_noalloc(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
                                 ctypes.byref(m), 0.1, FAKE, FAKE, FAKE, 1, None) == 3
@@ -167,11 +164,8 @@ def test_varlen_rejects_bad_args(lib):
     assert fwd(_varlen(), bias=_dense(0, 0, 300)) == 2       # no packed form of a dense bias
     assert fwd(_varlen(), shape=binding.Shape(3, 0, 4, 2, 96, 0, 4 * 96, 96, 0, 2 * 96, 96, 0)) == 2
     assert lib.sdpa_bwd_varlen_workspace_size(ctypes.byref(s), None) == 0
-    # rows of LSE, D and the dQ accumulator: Hq * total_q; counters per B * Hq * max tiles
-    r256 = lambda x: (x + 255) // 256 * 256
-    rows = 4 * 1000
-    turns = 3 * 4 * 3 * 4
-    want = r256(rows * 4) + r256((turns + 1) * 4) + r256(rows * 64 * 4)
+    # D, one float per LSE row: Hq * total_q rows
+    want = (4 * 1000 * 4 + 255) // 256 * 256
     assert lib.sdpa_bwd_varlen_workspace_size(ctypes.byref(s), ctypes.byref(_varlen())) == want
 
 

@@ -2,8 +2,7 @@
 that cannot allocate device memory around the call (kernel hosts that hand a
 library only its inputs and outputs, processes under a hard memory cap,
 latency-bound loops that avoid cudaMalloc / cudaFree).  Its workspace (the
-D vector, the dQ turn counters and the dQ accumulator) is a fixed array
-inside the library instead of caller memory; its results must match
+D vector) is a fixed array inside the library instead of caller memory; its results must match
 sdpa_bwd's bit for bit, call after call.
 
 Kept in its own file, named to be collected last.
@@ -58,11 +57,11 @@ def test_noalloc_matches_workspace_entry_point_twice(kw):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     dev = torch.device("cuda")
-    L = 40000                              # workspace ~ 2 * 40000 * 65 * 4 bytes > 16 MiB
-    q = torch.zeros(1, L, 2, 64, device=dev, dtype=torch.bfloat16)
+    L = 66000                              # workspace = 64 * 66000 * 4 bytes > 16 MiB
+    q = torch.zeros(1, L, 64, 64, device=dev, dtype=torch.bfloat16)
     k = torch.zeros(1, L, 1, 64, device=dev, dtype=torch.bfloat16)
     assert sdpa_bwd_workspace_size(q, k) > NOALLOC_SCRATCH_BYTES
-    lse = torch.zeros(1, 2, L, device=dev)
+    lse = torch.zeros(1, 64, L, device=dev)
     with pytest.raises(SdpaError) as e:
         sdpa_bwd_noalloc(q, k, k, q, q, lse, torch.empty_like(q), torch.empty_like(k),
                          torch.empty_like(k), causal=True)
