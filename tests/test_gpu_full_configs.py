@@ -54,14 +54,17 @@ def test_full_size_parity_and_repeatability(name):
     assert_close(got, ref)
 
 
-SWEEP = [(32, 512), (8, 512), (1, 2048), (8, 2048), (32, 8192), (1, 8192), (8, 16384)]
+SWEEP = [(hkv, L) for hkv in (32, 8, 1) for L in (512, 2048, 8192, 16384)]
 
 
 @pytest.mark.parametrize("hkv,L", SWEEP)
-def test_forward_sweep_parity(hkv, L):
+def test_forward_sweep_parity_and_repeatability(hkv, L):
     c = dict(B=32768 // L, Hq=32, Hkv=hkv, L=L, d=128, causal=True)
     inp = case_inputs(c)
     got = run_cuda(c, inp, backward=False)
+    again = run_cuda(c, inp, backward=False)
+    for n in got:
+        assert np.array_equal(got[n], again[n]), f"{n} not bitwise repeatable"
     # one (batch, KV group) unit; for long sequences a spread of query rows
     rows = None if L <= 2048 else np.unique(np.r_[0:64, L // 2 - 64:L // 2 + 64,
                                                   L - 200:L, np.linspace(0, L - 1, 97).astype(int)])
