@@ -523,30 +523,48 @@ def run_gpu(args, c):
     return 0
 
 
+def visited_tile_pairs(c):
+    """(query tile, key tile) pairs of one head that hold a visible (i, j)."""
+    L, n = c["L"], (c["L"] + 127) // 128
+    count = 0
+    for mi in range(n):
+        i0, i1 = mi * 128, min(L, mi * 128 + 128) - 1
+        lo = max(0, i0 - c["wl"]) if c["wl"] >= 0 else 0
+        hi = L - 1
+        if c["causal"]:
+            hi = min(hi, i1)
+        if c["wr"] >= 0:
+            hi = min(hi, i1 + c["wr"])
+        if hi >= lo:
+            count += hi // 128 - lo // 128 + 1
+    return count
+
+
 def bias_grad_extra_bytes(c):
-    """HBM bytes the bias gradient adds to the backward: the fp32 dS written
-    once, plus -- when it is staged (T5 table, broadcast dense bias) -- read
-    back once by the reduction and the gradient written."""
+    """HBM bytes the bias gradient adds to the backward.  A dense bias: the
+    fp32 dS written once (full shape), or written and read back by the
+    broadcast reduction.  T5 / ALiBi: the dQ kernel's per-warp diagonal sums
+    (1024 floats per visited tile pair) and the per-tile diagonals (256)
+    written and read back once, then the per-head totals and the result."""
     B, H, L = c["B"], c["Hq"], c["L"]
-    ds = B * H * L * L * 4
-    if c["bias"] == "t5":
-        return 2 * ds + 32 * H * 4
-    if c["bias"] == "alibi":
-        return 2 * ds + H * 4
-    return ds                      # a full-shape dense bias: dS goes straight out
+    if c["bias"] in ("t5", "alibi"):
+        tiles = B * H * visited_tile_pairs(c)
+        out = 32 * H * 4 if c["bias"] == "t5" else H * 4
+        return 2 * tiles * (1024 + 256) * 4 + 2 * H * (2 * L - 1) * 4 + out
+    return B * H * L * L * 4       # a full-shape dense bias: dS goes straight out
 
 
 def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
-    preprocess, the dQ kernel (with dS output) and the dK/dV kernel, the zero fill of
-    skipped key tiles under a mask, and the reductions (T5 / ALiBi: diagonal
-    sums, their fold and the per-bucket or per-slope sums; a full-shape dense
-    bias needs none)."""
+    preprocess, the dQ kernel (storing dS, or its diagonal sums) and the
+    dK/dV kernel; a dense bias under a mask adds the zero fill of skipped key
+    tiles; T5 / ALiBi add the per-tile fold, the per-head totals and the
+    per-bucket (or per-slope) sums."""
     n = 4
+    if c["bias"] in ("t5", "alibi"):
+        return n + 3
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1
-    if c["bias"] in ("t5", "alibi"):
-        n += 3
     return n
 
 

@@ -84,6 +84,9 @@ struct AttnParams {
   // element strides sd_b, sd_h, sd_i (multiples of 4), j contiguous
   float* ds_out;
   int64_t sd_b, sd_h, sd_i;
+  // optional per-warp sums of dS along the diagonals j - i (relative-position
+  // bias gradients); layout in bwd_dq_kernel's diagonal mode
+  float* diag_out;
   // bias
   int bias_kind;
   const float* bias;           // dense

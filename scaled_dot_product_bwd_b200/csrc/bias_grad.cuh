@@ -1,10 +1,12 @@
-// Bias gradients from the fp32 dS the dQ kernel stores (bwd_dq_kernel with
-// DS_OUT): the scores are linear in an additive bias, so a dense bias's
-// gradient is dS summed over each index the bias is broadcast along, and a
-// T5 table entry's gradient is dS summed over every (b, i, j) whose distance
-// j - i falls in its bucket (catie-aq/flashT5 README, "Full attention
-// biases" and "T5-like relative position encoding biases": a learnable
-// bias needs these to train).
+// Bias gradients.  The scores are linear in an additive bias, so a dense
+// bias's gradient is dS summed over each index the bias is broadcast along
+// (from the fp32 dS the dQ kernel stores in its store mode), a T5 table
+// entry's gradient is dS summed over every (b, i, j) whose distance j - i
+// falls in its bucket, and an ALiBi slope's is minus the sum of |j - i| dS
+// (both from the per-warp diagonal sums of dS the dQ kernel writes in its
+// diagonal mode; catie-aq/flashT5 README, "Full attention biases" and
+// "T5-like relative position encoding biases": a learnable bias needs these
+// to train).
 //
 // Every kernel here is bandwidth-bound and deterministic: each output is a
 // sum taken in one fixed order (fixed chunking of the reduced index, chunks
@@ -20,9 +22,6 @@ namespace sdpa {
 // not the device's SM count, so the chunking -- and with it the rounding of
 // every sum -- is the same on every device.
 constexpr int64_t kReduceTargetBlocks = 1184;
-
-// (b, i) rows per piece of the T5 diagonal sums.
-constexpr int64_t kT5RowsPerPiece = 128;
 
 // ---------------------------------------------------------------------
 // dS entries the backward never visits: for query row i, the key tiles
@@ -144,13 +143,9 @@ __global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseRedu
 // each side of 0, and the two sides use disjoint ids when bidirectional),
 // given to the last kernel as [lo, hi].
 struct T5Reduce {
-  const float* ds;               // [B, Hq, L, lp] fp32
-  int64_t ds_b, ds_h, ds_i;
-  int B, Hq, L;
-  int chunks;                    // pieces of the (b, i) range (grid z)
-  int64_t uchunk;                // (b, i) pairs per piece
-  float* partial;                // [chunks, Hq, 2L - 1]
-  float* out;                    // table gradient [num_buckets, Hq]
+  const float* partial;          // diagonal sums [Hq, 2L - 1]: partial[h, r + L - 1]
+  int Hq, L;
+  float* out;                    // table gradient [num_buckets, Hq], or slope gradient [Hq]
   int num_buckets;
 };
 
@@ -159,72 +154,69 @@ struct T5Ranges {
   int hi[128];                   // last r of bucket k; hi < lo: bucket unused
 };
 
-// partial[z, h, r + L - 1] = sum of dS[b, h, i, i + r] over the (b, i) of
-// piece z.  A thread walks only the rows that have a key at distance r, with
-// eight accumulators (the e-th of every eight consecutive rows goes to
-// accumulator e, an order fixed by the shape alone) so that eight loads are
-// in flight at a time.
-__global__ void __launch_bounds__(128) t5_diag_kernel(const T5Reduce a) {
+// ---------------------------------------------------------------------
+// The same diagonal sums from the dQ kernel's per-warp partials (its
+// diagonal mode), without the L x L dS: first each visited 128 x 128 tile's
+// 255 diagonals D = j - i - (n0 - m0) in [-127, 127], then the per-head
+// totals.  Both sum in an order fixed by the shape alone.
+struct DiagFold {
+  const float* warp_part;        // [B, Hq, nqt, ntk, 8 warps, 2 halves, 64]
+  float* tile_diag;              // [B, Hq, nqt, ntk, 256]
+  float* diag;                   // [Hq, 2L - 1]: diag[h, r + L - 1]
+  int B, Hq, L, nqt, ntk;
+};
+
+// One block per (query tile, key tile, b * Hq + h), thread D + 127: adds
+// the warp-half pieces that cover tile diagonal D, warps then halves in
+// index order.  Warp w (rows 32 (w % 4).., warpgroup w / 4 holding keys
+// 64 (w / 4)..) half h covers D = 64 (w / 4) + 32 h - 32 (w % 4) + t,
+// t in [-31, 31].  Tiles outside the mask band are skipped (never read).
+__global__ void __launch_bounds__(256) diag_tile_fold_kernel(const DiagFold a, const AttnParams p) {
+  const int mi = blockIdx.x, ni = blockIdx.y, bh = blockIdx.z;
+  int nlo, nhi;
+  key_tile_range(p, a.L, a.L, mi * kTile, kTile, nlo, nhi);
+  if (ni < nlo || ni >= nhi) return;
+  const int D = static_cast<int>(threadIdx.x) - 127;
+  if (D > 127) return;
+  const int64_t blk = (static_cast<int64_t>(bh) * a.nqt + mi) * a.ntk + ni;
+  const float* src = a.warp_part + blk * 1024;
+  float acc = 0.f;
+  for (int w = 0; w < 8; ++w) {
+    for (int h = 0; h < 2; ++h) {
+      const int t = D - 64 * (w >> 2) - 32 * h + 32 * (w & 3);
+      if (t < -31 || t > 31) continue;
+      acc += src[(w * 2 + h) * 64 + (t <= 0 ? t + 31 : 31 + t)];
+    }
+  }
+  a.tile_diag[blk * 256 + threadIdx.x] = acc;
+}
+
+// diag[h, r + L - 1] = sum over b, then query tile mi, then the (at most
+// two) visited key tiles ni with r - 128 (ni - mi) in [-127, 127], of the
+// tile diagonal there.
+__global__ void __launch_bounds__(128) diag_total_kernel(const DiagFold a, const AttnParams p) {
   const int nd = 2 * a.L - 1;
   const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
   if (dr >= nd) return;
   const int r = dr - (a.L - 1);
   const int h = blockIdx.y;
-  const int z = blockIdx.z;
-  const int row_lo = max(0, -r), row_hi = min(a.L, a.L - r);  // rows i with 0 <= i + r < L
-  const int64_t u0 = static_cast<int64_t>(z) * a.uchunk;
-  const int64_t u1 = min(static_cast<int64_t>(a.B) * a.L, u0 + a.uchunk);
-  const int b_first = static_cast<int>(u0 / a.L);
-  const int b_last = static_cast<int>((u1 - 1) / a.L);
-  const int64_t step = a.ds_i + 1;  // (i, i + r) -> (i + 1, i + 1 + r)
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int b = b_first; b <= b_last; ++b) {
-    int ia = row_lo, ib = row_hi;
-    if (b == b_first) ia = max(ia, static_cast<int>(u0 - static_cast<int64_t>(b) * a.L));
-    if (b == b_last) ib = min(ib, static_cast<int>(u1 - static_cast<int64_t>(b) * a.L));
-    const float* base = a.ds + static_cast<int64_t>(b) * a.ds_b +
-                        static_cast<int64_t>(h) * a.ds_h + r;
-    int i = ia;
-    for (; i + 8 <= ib; i += 8) {
-      float x[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = base[static_cast<int64_t>(i + e) * step];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += x[e];
+  float acc = 0.f;
+  for (int b = 0; b < a.B; ++b) {
+    for (int mi = 0; mi < a.nqt; ++mi) {
+      int nlo, nhi;
+      key_tile_range(p, a.L, a.L, mi * kTile, kTile, nlo, nhi);
+      // ni - mi in [ceil((r - 127) / 128), floor((r + 127) / 128)]
+      const int lo = mi + (r - 127 >= 0 ? (r - 127 + 127) / 128 : -((127 - r) / 128));
+      for (int ni = max(lo, nlo); ni < nhi; ++ni) {
+        const int Dv = r - kTile * (ni - mi);
+        if (Dv < -127) break;
+        if (Dv > 127) continue;
+        const int64_t blk = ((static_cast<int64_t>(b) * a.Hq + h) * a.nqt + mi) * a.ntk + ni;
+        acc += a.tile_diag[blk * 256 + Dv + 127];
+      }
     }
-#pragma unroll
-    for (int e = 0; e < 7; ++e)
-      if (i + e < ib) acc[e] += base[static_cast<int64_t>(i + e) * step];
   }
-  const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  a.partial[(static_cast<int64_t>(z) * a.Hq + h) * nd + dr] = sum;
-}
-
-// Folds the pieces: partial[0, h, dr] = sum over z of partial[z, h, dr], the
-// pieces taken in eight interleaved accumulators (piece z to accumulator
-// z mod 8) and the eight added in a fixed tree.  A thread owns one (h, dr)
-// across all pieces, so it may overwrite piece 0 in place.
-__global__ void __launch_bounds__(128) t5_piece_sum_kernel(const T5Reduce a) {
-  const int nd = 2 * a.L - 1;
-  const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
-  if (dr >= nd) return;
-  const int h = blockIdx.y;
-  const int64_t stride = static_cast<int64_t>(a.Hq) * nd;
-  const float* src = a.partial + static_cast<int64_t>(h) * nd + dr;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int z = 0;
-  for (; z + 8 <= a.chunks; z += 8) {
-    float x[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = src[(z + e) * stride];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += x[e];
-  }
-#pragma unroll
-  for (int e = 0; e < 7; ++e)
-    if (z + e < a.chunks) acc[e] += src[(z + e) * stride];
-  a.partial[static_cast<int64_t>(h) * nd + dr] =
-      ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  a.diag[static_cast<int64_t>(h) * nd + dr] = acc;
 }
 
 // out[k, h] = sum of the diagonal sums over bucket k's range of r: one block

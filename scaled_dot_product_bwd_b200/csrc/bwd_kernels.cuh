@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(352, 1)
       };
       load_vec(0);
       int issued_q[SQ], issued_o[SO];
-      for (int s = 0; s < SQ; ++s) issued_q[s] = -1;
-      for (int s = 0; s < SO; ++s) issued_o[s] = -1;
+      for (int e = 0; e < SQ; ++e) issued_q[e] = -1;
+      for (int e = 0; e < SO; ++e) issued_o[e] = -1;
       bool ok = true;
       for (int it = 0; it < total; ++it) {
         const int hq = g * p.G + it / nm;
@@ -303,10 +303,10 @@ __global__ void __launch_bounds__(352, 1)
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
         mbar_wait(kv_full, 0, ign);
-        for (int s = 0; s < SQ; ++s)
-          if (issued_q[s] >= 0) mbar_wait(q_full(s), issued_q[s], ign);
-        for (int s = 0; s < SO; ++s)
-          if (issued_o[s] >= 0) mbar_wait(o_full(s), issued_o[s], ign);
+        for (int e = 0; e < SQ; ++e)
+          if (issued_q[e] >= 0) mbar_wait(q_full(e), issued_q[e], ign);
+        for (int e = 0; e < SO; ++e)
+          if (issued_o[e] >= 0) mbar_wait(o_full(e), issued_o[e], ign);
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -558,7 +558,12 @@ __global__ void __launch_bounds__(352, 1)
 // its own, already loaded, S buffer: dP of block i + 1 can then be computed
 // as soon as block i's dP has been loaded, and S of block i + 2 waits only
 // for the dQ MMA of block i.
-template <int D, int BIAS>
+// DSM (what the kernel does with the fp32 dS besides the dQ MMA): 0 nothing,
+// 1 store it (dense-bias gradient), 2 store its per-warp sums along the
+// diagonals j - i (T5 / ALiBi gradients), staged through shared memory.
+constexpr int kDsNone = 0, kDsStore = 1, kDsDiag = 2;
+
+template <int D, int BIAS, int DSM = kDsNone>
 struct DqLayout {
   static constexpr int kTileBytes = kTile * D * 2;
   // Dense bias at d = 64: each block's 128 x 128 fp32 bias comes by TMA into
@@ -569,7 +574,8 @@ struct DqLayout {
   // K blocks are used until the block's dQ MMA, V blocks only until its dP
   // MMA: the K ring is the deeper one.
   static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : (kBiasTma ? 2 : 4);
-  static constexpr int kSV = (D == 128) ? 2 : (kBiasTma ? 2 : 3);
+  // (at d = 128 the diagonal staging area takes the second V stage)
+  static constexpr int kSV = (D == 128) ? (DSM == kDsDiag ? 1 : 2) : (kBiasTma ? 2 : 3);
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTileBytes;
   static constexpr int kKOff = 2 * kTileBytes;                // K ring
@@ -577,7 +583,10 @@ struct DqLayout {
   static constexpr int kBOff = kVOff + kSV * kTileBytes;      // bias ring (kBiasTma)
   static constexpr int kLutOff = kBOff + kSB * kBiasTileBytes;  // T5 only: 8 warps x 96 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
-  static constexpr int kBarOff = kLutOff + kLutBytes;
+  // DSM == 2: per warp, 32 rows x 32 keys of fp32 dS, row stride 33 floats
+  static constexpr int kDiagOff = kLutOff + kLutBytes;
+  static constexpr int kDiagBytes = (DSM == kDsDiag) ? 8 * 32 * 33 * 4 : 0;
+  static constexpr int kBarOff = kDiagOff + kDiagBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
   // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
   // b_full[2], b_empty[2]
@@ -590,13 +599,13 @@ struct DqLayout {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-// DS_OUT: also store dS in fp32 through p.ds_out (the bias gradient path).
-template <int D, int BIAS, bool DS_OUT = false>
+// DSM: see DqLayout (the bias-gradient paths).
+template <int D, int BIAS, int DSM = kDsNone>
 __global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
-  using Lay = DqLayout<D, BIAS>;
+  using Lay = DqLayout<D, BIAS, DSM>;
   constexpr int SK = Lay::kSK;
   constexpr int SV = Lay::kSV;
   extern __shared__ uint8_t smem[];
@@ -1002,7 +1011,7 @@ __global__ void __launch_bounds__(352, 1)
             const float d0 = __uint_as_float(pr[cc + e]) * (__uint_as_float(dr[e]) - dd);
             const float d1 = __uint_as_float(pr[cc + e + 1]) * (__uint_as_float(dr[e + 1]) - dd);
             pk[(cc + e) >> 1] = pack_bf16x2(d0, d1);
-            if constexpr (DS_OUT) {  // P is spent: keep the fp32 dS in its place
+            if constexpr (DSM != kDsNone) {  // P is spent: keep the fp32 dS in its place
               pr[cc + e] = __float_as_uint(d0);
               pr[cc + e + 1] = __float_as_uint(d1);
             }
@@ -1014,7 +1023,41 @@ __global__ void __launch_bounds__(352, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(ds_full(c & 1));
-        if constexpr (DS_OUT) {
+        if constexpr (DSM == kDsDiag) {
+          // Sums of this warp's 32 rows x 64 keys of dS along the diagonals,
+          // in two halves of 32 keys: each half is staged row by row
+          // (stride 33 floats: conflict-free both ways), then lane l adds up
+          // the diagonal t = c - r = l - 31 (rows 31 - l..31) and, for
+          // l < 31, t = l + 1 (rows 0..30 - l), one element per step, so a
+          // step's 32 reads hit 32 banks.  In absolute terms t is the
+          // distance j - i = n0 + 32 h - (m0 + 32 (warp % 4)) + t.  Per
+          // (batch, head, query tile, key tile): 8 warps x 2 halves x 64
+          // floats (t + 31 at 0..62 for t <= 0, 32 + t - 1 for t >= 1).
+          float* stg = reinterpret_cast<float*>(smem + Lay::kDiagOff) + warp * (32 * 33);
+          const int ntk = (p.Lk + kTile - 1) / kTile;
+          float* dst = p.diag_out +
+                       ((((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * ntk +
+                         (n0 - c0w) / kTile) * 8 + warp) * 128;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            __syncwarp();
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) stg[lane * 33 + cc] = __uint_as_float(pr[32 * h + cc]);
+            __syncwarp();
+            float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const bool first = k <= lane;
+              const int r = first ? 31 - lane + k : k - lane - 1;
+              const float v = stg[r * 33 + k];
+              s1 += first ? v : 0.f;
+              s2 += first ? 0.f : v;
+            }
+            dst[h * 64 + lane] = s1;
+            if (lane < 31) dst[h * 64 + 32 + lane] = s2;
+          }
+        }
+        if constexpr (DSM == kDsStore) {
           // fp32 dS of this row's 64 keys while the dQ MMA runs; masked keys
           // have P = 0 and so dS = 0.  Lanes 2m and 2m + 1 hold neighbouring
           // rows; for every 8 keys they swap four values so that each store
@@ -1136,19 +1179,27 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
     if (e != cudaSuccess) return e;
   }
   if (phases & kPhaseDq) {
-    using Lay = DqLayout<D, BIAS>;
     auto kern = bwd_dq_kernel<D, BIAS>;
-    if constexpr (BIAS != kBiasNone) {
-      if (p.ds_out) kern = bwd_dq_kernel<D, BIAS, true>;
+    int smem_bytes = DqLayout<D, BIAS>::kSmemAlloc;
+    if constexpr (BIAS == kBiasDense) {
+      if (p.ds_out) {
+        kern = bwd_dq_kernel<D, BIAS, kDsStore>;
+        smem_bytes = DqLayout<D, BIAS, kDsStore>::kSmemAlloc;
+      }
     }
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Lay::kSmemAlloc);
+    if constexpr (BIAS == kBiasT5) {
+      if (p.diag_out) {
+        kern = bwd_dq_kernel<D, BIAS, kDsDiag>;
+        smem_bytes = DqLayout<D, BIAS, kDsDiag>::kSmemAlloc;
+      }
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (or per work item, if fewer)
     const int64_t items = static_cast<int64_t>((p.Lq + kTile - 1) / kTile) * p.Hq * p.B;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    kern<<<static_cast<int>(items < sms ? items : sms), Lay::kThreads, Lay::kSmemAlloc, st>>>(
+    kern<<<static_cast<int>(items < sms ? items : sms), DqLayout<D, BIAS>::kThreads, smem_bytes, st>>>(
         p, mq, mk, mv, mdo, mb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -57,7 +57,6 @@ struct Geometry {
   int64_t sq_b, sq_l, sq_h, skv_b, skv_l, skv_h;
   // positions along the query / key sequence axis (per head)
   int64_t axis_q() const { return packed ? total_q : B * Lq; }
-  int64_t axis_k() const { return packed ? total_k : B * Lk; }
   // rows of LSE, D and the dQ accumulator
   int64_t rows() const { return Hq * axis_q(); }
 };
@@ -374,6 +373,10 @@ struct BiasGradPlan {
   int chunks = 1;         // pieces of the reduced index
   int64_t per_chunk = 0;  // reduced indices per piece
   size_t part_bytes = 0;  // partial sums of the pieces
+  // T5 / ALiBi: the dQ kernel's per-warp diagonal sums, then per-tile and
+  // per-head diagonal sums (no dS)
+  bool diag = false;
+  size_t warp_bytes = 0, tile_bytes = 0, diag_bytes = 0;
   size_t total = 0;
 };
 
@@ -422,17 +425,17 @@ sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, Bias
         pl.part_bytes = round256(static_cast<size_t>(pl.chunks * n_out * pl.lp) * sizeof(float));
     }
   } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_ALIBI) {
-    if (ds_elems > 1e17) return SDPA_ERR_UNSUPPORTED;
-    pl.ds_ws = true;
-    pl.ds_bytes = round256(static_cast<size_t>(B * Hq * L * pl.lp) * sizeof(float));
-    // pieces of kT5RowsPerPiece (b, i) rows: the diagonals near the middle
-    // hold L rows per batch entry and the outer ones few, so short pieces keep
-    // every thread's chain of loads short and the grid balanced; the
-    // partial sums are then 1/64 of dS or less
-    pl.per_chunk = kT5RowsPerPiece;
-    if ((B * L + pl.per_chunk - 1) / pl.per_chunk > 65535) pl.per_chunk = (B * L + 65534) / 65535;
-    pl.chunks = static_cast<int>((B * L + pl.per_chunk - 1) / pl.per_chunk);
-    pl.part_bytes = round256(static_cast<size_t>(pl.chunks * Hq * (2 * L - 1)) * sizeof(float));
+    // per (batch, head, query tile, key tile): 1024 per-warp sums and 256
+    // tile diagonals; per head: 2L - 1 diagonal totals
+    const int64_t nt = (L + kTile - 1) / kTile;
+    const double tiles = static_cast<double>(B) * Hq * nt * nt;
+    if (tiles * 1280.0 > 1e16 || nt > 65535 || B * Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+    pl.diag = true;
+    const size_t n_tiles = static_cast<size_t>(B * Hq * nt * nt);
+    pl.warp_bytes = round256(n_tiles * 1024 * sizeof(float));
+    pl.tile_bytes = round256(n_tiles * 256 * sizeof(float));
+    pl.diag_bytes = round256(static_cast<size_t>(Hq * (2 * L - 1)) * sizeof(float));
+    pl.part_bytes = pl.warp_bytes + pl.tile_bytes + pl.diag_bytes;
   } else {
     return SDPA_ERR_UNSUPPORTED;  // no bias: nothing to differentiate
   }
@@ -616,6 +619,40 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   bind_bwd(p, g, o, dout, lse, dq, dk, dv, ws);
   const int L = p.Lq;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (pl.diag) {
+    // T5 / ALiBi: per-warp diagonal sums from the dQ kernel, folded per
+    // tile, then per head, then per bucket (or weighed by -|r| per slope)
+    uint8_t* base = ws + pl.bwd_bytes;
+    DiagFold f;
+    f.warp_part = reinterpret_cast<const float*>(base);
+    f.tile_diag = reinterpret_cast<float*>(base + pl.warp_bytes);
+    f.diag = reinterpret_cast<float*>(base + pl.warp_bytes + pl.tile_bytes);
+    f.B = p.B;
+    f.Hq = p.Hq;
+    f.L = L;
+    f.nqt = f.ntk = (L + kTile - 1) / kTile;
+    p.diag_out = reinterpret_cast<float*>(base);
+    st = run_bwd(SDPA_BWD_ALL, p, g, q, k, v, dout, cs);
+    if (st != SDPA_OK) return st;
+    diag_tile_fold_kernel<<<dim3(f.nqt, f.ntk, p.B * p.Hq), 256, 0, cs>>>(f, p);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    const unsigned rblocks = static_cast<unsigned>((2 * L - 1 + 127) / 128);
+    diag_total_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(f, p);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    T5Reduce a;
+    std::memset(&a, 0, sizeof(a));
+    a.Hq = p.Hq;
+    a.L = L;
+    a.partial = f.diag;
+    a.out = dbias;
+    a.num_buckets = p.alibi ? 0 : bias->num_buckets;
+    if (p.alibi)
+      alibi_slope_grad_kernel<<<p.Hq, 256, 0, cs>>>(a);
+    else
+      t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  }
   if (pl.ds_ws) {
     p.ds_out = reinterpret_cast<float*>(ws + pl.bwd_bytes);
     p.sd_i = pl.lp;
@@ -627,7 +664,6 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     p.sd_h = p.sb_h;
     p.sd_i = p.sb_i;
   }
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int sms = sm_count();
   if (sms <= 0) return SDPA_ERR_CUDA;
   if (p.causal || p.wl >= 0 || p.wr >= 0) {
@@ -671,30 +707,6 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
       dense_bias_combine_kernel<<<static_cast<unsigned>(g1), 256, 0, cs>>>(a);
       if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     }
-  } else {
-    T5Reduce a;
-    a.ds = p.ds_out;
-    a.ds_b = p.sd_b;
-    a.ds_h = p.sd_h;
-    a.ds_i = p.sd_i;
-    a.B = p.B;
-    a.Hq = p.Hq;
-    a.L = L;
-    a.chunks = pl.chunks;
-    a.uchunk = pl.per_chunk;
-    a.partial = part;
-    a.out = dbias;
-    a.num_buckets = p.alibi ? 0 : bias->num_buckets;
-    const unsigned rblocks = static_cast<unsigned>((2 * L - 1 + 127) / 128);
-    t5_diag_kernel<<<dim3(rblocks, p.Hq, a.chunks), 128, 0, cs>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
-    t5_piece_sum_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
-    if (p.alibi)
-      alibi_slope_grad_kernel<<<p.Hq, 256, 0, cs>>>(a);
-    else
-      t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
-    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
   }
   return SDPA_OK;
 }

@@ -187,11 +187,15 @@ def test_bias_grad_workspace_size(lib):
     for b in (_dense(L * L, 0, L), _dense(0, L * L, L), _dense(0, 0, L)):
         n = ws(b)
         assert n >= d_bytes + ds_bytes and n % 256 == 0
+    # T5 / ALiBi: no dS; per (batch, head, query tile, key tile) 1024
+    # per-warp diagonal sums and 256 tile diagonals, per head 2L - 1 totals
+    r256 = lambda x: (x + 255) // 256 * 256
+    tiles = B * Hq * ((L + 127) // 128) ** 2
+    want = d_bytes + r256(tiles * 1024 * 4) + r256(tiles * 256 * 4) + r256(Hq * (2 * L - 1) * 4)
     t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
-    n = ws(t5)
-    assert n >= d_bytes + ds_bytes + Hq * (2 * L - 1) * 4 and n % 256 == 0
+    assert ws(t5) == want
     alibi = binding.BiasDesc(3, 0x10000, 0, 0, 0, 0, 0, 0)
-    assert ws(alibi) >= d_bytes + ds_bytes and ws(alibi) % 256 == 0
+    assert ws(alibi) == want
     assert ws(binding.BiasDesc(0, None, 0, 0, 0, 0, 0, 0)) == 0       # nothing to differentiate
     assert ws(_dense(L * L, L * L, L)) == 0                          # heads overlap batches
     assert ws(_dense(Hq * L * L, L * L, 0)) == 0                      # one row for all queries

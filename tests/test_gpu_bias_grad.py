@@ -185,7 +185,7 @@ def test_padded_dense_bias_gradient():
 
 
 @pytest.mark.parametrize("name", ["dense_full_window_d64", "dense_heads_bcast_d64",
-                                  "t5_bidir_d64"])
+                                  "t5_bidir_d64", "alibi_causal_gqa_d128"])
 def test_bias_grad_bitwise_repeatable(name):
     c = CASES[name]
     inp = case_inputs(c)
