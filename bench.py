@@ -558,11 +558,11 @@ def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
     preprocess, the dQ kernel (storing dS, or its diagonal sums) and the
     dK/dV kernel; a dense bias under a mask adds the zero fill of skipped key
-    tiles; T5 / ALiBi add the per-tile fold, the per-head totals and the
-    per-bucket (or per-slope) sums."""
+    tiles; T5 / ALiBi add the per-tile fold, the per-tile-offset sums, the
+    per-head totals and the per-bucket (or per-slope) sums."""
     n = 4
     if c["bias"] in ("t5", "alibi"):
-        return n + 3
+        return n + 4
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1
     return n

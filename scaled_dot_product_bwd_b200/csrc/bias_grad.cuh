@@ -162,6 +162,7 @@ struct T5Ranges {
 struct DiagFold {
   const float* warp_part;        // [B, Hq, nqt, ntk, 8 warps, 2 halves, 64]
   float* tile_diag;              // [B, Hq, nqt, ntk, 256]
+  float* band;                   // [B, Hq, 2 nqt - 1 tile offsets, 256]
   float* diag;                   // [Hq, 2L - 1]: diag[h, r + L - 1]
   int B, Hq, L, nqt, ntk;
 };
@@ -191,29 +192,51 @@ __global__ void __launch_bounds__(256) diag_tile_fold_kernel(const DiagFold a, c
   a.tile_diag[blk * 256 + threadIdx.x] = acc;
 }
 
-// diag[h, r + L - 1] = sum over b, then query tile mi, then the (at most
-// two) visited key tiles ni with r - 128 (ni - mi) in [-127, 127], of the
-// tile diagonal there.
-__global__ void __launch_bounds__(128) diag_total_kernel(const DiagFold a, const AttnParams p) {
+// band[b, h, dt + nt - 1, D + 127] = sum over query tiles mi (four
+// interleaved accumulators, mi % 4, added in a fixed tree) of the tile
+// diagonal D of tile (mi, mi + dt): one block per (tile offset dt, head,
+// batch entry), thread D + 127, so a warp reads 32 consecutive diagonals of
+// one tile.
+__global__ void __launch_bounds__(256) diag_band_kernel(const DiagFold a, const AttnParams p) {
+  const int nb = 2 * a.nqt - 1;
+  const int dt = static_cast<int>(blockIdx.x) - (a.nqt - 1);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int D = static_cast<int>(threadIdx.x);  // D + 127
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (D < 255) {
+    const int mi0 = max(0, -dt), mi1 = min(a.nqt, a.ntk - dt);
+#pragma unroll 4
+    for (int mi = mi0; mi < mi1; ++mi) {
+      int nlo, nhi;
+      key_tile_range(p, a.L, a.L, mi * kTile, kTile, nlo, nhi);
+      const int ni = mi + dt;
+      if (ni < nlo || ni >= nhi) continue;
+      const int64_t blk = ((static_cast<int64_t>(b) * a.Hq + h) * a.nqt + mi) * a.ntk + ni;
+      acc[mi & 3] += a.tile_diag[blk * 256 + D];
+    }
+  }
+  a.band[((static_cast<int64_t>(b) * a.Hq + h) * nb + blockIdx.x) * 256 + D] =
+      (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// diag[h, r + L - 1]: over b, the band sums of the (at most two) tile
+// offsets dt with r - 128 dt in [-127, 127], the lower dt first.
+__global__ void __launch_bounds__(128) diag_total_kernel(const DiagFold a) {
   const int nd = 2 * a.L - 1;
+  const int nb = 2 * a.nqt - 1;
   const int dr = blockIdx.x * 128 + static_cast<int>(threadIdx.x);
   if (dr >= nd) return;
   const int r = dr - (a.L - 1);
   const int h = blockIdx.y;
+  // lowest dt with r - 128 dt <= 127: ceil((r - 127) / 128)
+  const int dt0 = r - 127 >= 0 ? r / 128 : -((127 - r) / 128);
   float acc = 0.f;
   for (int b = 0; b < a.B; ++b) {
-    for (int mi = 0; mi < a.nqt; ++mi) {
-      int nlo, nhi;
-      key_tile_range(p, a.L, a.L, mi * kTile, kTile, nlo, nhi);
-      // ni - mi in [ceil((r - 127) / 128), floor((r + 127) / 128)]
-      const int lo = mi + (r - 127 >= 0 ? (r - 127 + 127) / 128 : -((127 - r) / 128));
-      for (int ni = max(lo, nlo); ni < nhi; ++ni) {
-        const int Dv = r - kTile * (ni - mi);
-        if (Dv < -127) break;
-        if (Dv > 127) continue;
-        const int64_t blk = ((static_cast<int64_t>(b) * a.Hq + h) * a.nqt + mi) * a.ntk + ni;
-        acc += a.tile_diag[blk * 256 + Dv + 127];
-      }
+    for (int dt = dt0; dt <= dt0 + 1; ++dt) {
+      const int Dv = r - kTile * dt;
+      if (Dv < -127 || dt < -(a.nqt - 1) || dt > a.nqt - 1) continue;
+      acc += a.band[((static_cast<int64_t>(b) * a.Hq + h) * nb + dt + a.nqt - 1) * 256 + Dv + 127];
     }
   }
   a.diag[static_cast<int64_t>(h) * nd + dr] = acc;

@@ -376,7 +376,7 @@ struct BiasGradPlan {
   // T5 / ALiBi: the dQ kernel's per-warp diagonal sums, then per-tile and
   // per-head diagonal sums (no dS)
   bool diag = false;
-  size_t warp_bytes = 0, tile_bytes = 0, diag_bytes = 0;
+  size_t warp_bytes = 0, tile_bytes = 0, band_bytes = 0, diag_bytes = 0;
   size_t total = 0;
 };
 
@@ -434,8 +434,9 @@ sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, Bias
     const size_t n_tiles = static_cast<size_t>(B * Hq * nt * nt);
     pl.warp_bytes = round256(n_tiles * 1024 * sizeof(float));
     pl.tile_bytes = round256(n_tiles * 256 * sizeof(float));
+    pl.band_bytes = round256(static_cast<size_t>(B * Hq * (2 * nt - 1) * 256) * sizeof(float));
     pl.diag_bytes = round256(static_cast<size_t>(Hq * (2 * L - 1)) * sizeof(float));
-    pl.part_bytes = pl.warp_bytes + pl.tile_bytes + pl.diag_bytes;
+    pl.part_bytes = pl.warp_bytes + pl.tile_bytes + pl.band_bytes + pl.diag_bytes;
   } else {
     return SDPA_ERR_UNSUPPORTED;  // no bias: nothing to differentiate
   }
@@ -622,12 +623,14 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (pl.diag) {
     // T5 / ALiBi: per-warp diagonal sums from the dQ kernel, folded per
-    // tile, then per head, then per bucket (or weighed by -|r| per slope)
+    // tile, per tile offset, then per head, then per bucket (or weighed by
+    // -|r| per slope)
     uint8_t* base = ws + pl.bwd_bytes;
     DiagFold f;
     f.warp_part = reinterpret_cast<const float*>(base);
     f.tile_diag = reinterpret_cast<float*>(base + pl.warp_bytes);
-    f.diag = reinterpret_cast<float*>(base + pl.warp_bytes + pl.tile_bytes);
+    f.band = reinterpret_cast<float*>(base + pl.warp_bytes + pl.tile_bytes);
+    f.diag = reinterpret_cast<float*>(base + pl.warp_bytes + pl.tile_bytes + pl.band_bytes);
     f.B = p.B;
     f.Hq = p.Hq;
     f.L = L;
@@ -637,8 +640,10 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     if (st != SDPA_OK) return st;
     diag_tile_fold_kernel<<<dim3(f.nqt, f.ntk, p.B * p.Hq), 256, 0, cs>>>(f, p);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    diag_band_kernel<<<dim3(2 * f.nqt - 1, p.Hq, p.B), 256, 0, cs>>>(f, p);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     const unsigned rblocks = static_cast<unsigned>((2 * L - 1 + 127) / 128);
-    diag_total_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(f, p);
+    diag_total_kernel<<<dim3(rblocks, p.Hq), 128, 0, cs>>>(f);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     T5Reduce a;
     std::memset(&a, 0, sizeof(a));

@@ -188,10 +188,13 @@ def test_bias_grad_workspace_size(lib):
         n = ws(b)
         assert n >= d_bytes + ds_bytes and n % 256 == 0
     # T5 / ALiBi: no dS; per (batch, head, query tile, key tile) 1024
-    # per-warp diagonal sums and 256 tile diagonals, per head 2L - 1 totals
+    # per-warp diagonal sums and 256 tile diagonals, per (batch, head, tile
+    # offset) 256 band sums, per head 2L - 1 totals
     r256 = lambda x: (x + 255) // 256 * 256
-    tiles = B * Hq * ((L + 127) // 128) ** 2
-    want = d_bytes + r256(tiles * 1024 * 4) + r256(tiles * 256 * 4) + r256(Hq * (2 * L - 1) * 4)
+    nt = (L + 127) // 128
+    tiles = B * Hq * nt * nt
+    want = (d_bytes + r256(tiles * 1024 * 4) + r256(tiles * 256 * 4) +
+            r256(B * Hq * (2 * nt - 1) * 256 * 4) + r256(Hq * (2 * L - 1) * 4))
     t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
     assert ws(t5) == want
     alibi = binding.BiasDesc(3, 0x10000, 0, 0, 0, 0, 0, 0)
