@@ -11,9 +11,12 @@ from .sdpa_oracle import (  # noqa: F401
     attention_forward_packed,
     attention_probs,
     dense_bias_gradient,
+    fire_gradients,
+    fire_table,
     head_scores,
     packed_positions,
     packed_visibility_mask,
+    rel_table_gradient,
     t5_relative_bucket,
     t5_table_gradient,
     visibility_mask,

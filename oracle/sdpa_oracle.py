@@ -45,6 +45,18 @@ What it computes, and where each piece comes from:
   m_h per query head given by the caller; under a causal mask this is the
   paper's -m_h (i - j), and the absolute value extends it to keys after the
   query.
+* A relative-position table (any per-head function of the distance j - i,
+  given as a table [Lq + Lk - 1, Hq], entry j - i + Lq - 1): the general form
+  of which T5 and ALiBi are special cases.
+* FIRE: the flashT5 README names it among the positional schemes it plans
+  to support, without a formula.  The oracle takes the bias of Li et al.
+  (2023, "Functional Interpolation for Relative Positions Improves Long
+  Context Transformers"): f(psi(i - j) / psi(max(T, i))) with
+  psi(x) = log(c x + 1) and f a one-hidden-layer ReLU MLP from the scalar to
+  one value per head.  Reading: the threshold T is at least the longest
+  query position (T >= Lq - 1), so max(T, i) = T on every row and the bias
+  is a function of the distance alone -- a relative-position table; keys
+  after the query (bidirectional use) take the same function of |i - j|.
 * Bias gradients: the scores are linear in the bias with coefficient 1, so
   the gradient of a dense bias is dS itself, summed over every index along
   which the bias is broadcast, and the gradient of a T5 table entry
@@ -87,6 +99,9 @@ __all__ = [
     "dense_bias_gradient",
     "t5_table_gradient",
     "alibi_slope_gradient",
+    "rel_table_gradient",
+    "fire_table",
+    "fire_gradients",
     "packed_positions",
     "packed_visibility_mask",
     "attention_forward_packed",
@@ -165,10 +180,15 @@ def _as64(x):
 
 
 def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
-                 t5_max_distance, t5_bidirectional, alibi_slopes=None, Lk=None):
+                 t5_max_distance, t5_bidirectional, alibi_slopes=None, Lk=None,
+                 rel_table=None):
     """Additive bias for one (batch, query head), [L, Lk] float64 (or 0)."""
     Lk = L if Lk is None else Lk
     out = 0.0
+    if rel_table is not None:
+        i = np.arange(L)[:, None]
+        j = np.arange(Lk)[None, :]
+        out = out + rel_table[j - i + L - 1, hq]
     if alibi_slopes is not None:
         i = np.arange(L)[:, None]
         j = np.arange(Lk)[None, :]
@@ -188,7 +208,7 @@ def _bias_matrix(b: int, hq: int, L: int, bias, t5_table, t5_num_buckets,
 def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
                 window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
                 t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None,
-                rows=None):
+                rel_table=None, rows=None):
     """Masked score matrix S for one (b, hq): scale * Q K^T + bias, -inf where
     masked.  q: [B, L, Hq, d], k: [B, Lk, Hkv, d] float64 arrays (Lk = L for
     self-attention; positions of both sequences count from 0).  With
@@ -199,9 +219,10 @@ def head_scores(q, k, b, hq, *, scale, causal=False, window_left=-1,
     g = hq // (Hq // Hkv)
     r = np.arange(L) if rows is None else np.asarray(rows)
     S = scale * (q[b, r, hq, :] @ k[b, :, g, :].T)
-    S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets,
-                         t5_max_distance, t5_bidirectional, alibi_slopes, Lk)[r] \
-        if (bias is not None or t5_table is not None or alibi_slopes is not None) else S
+    if bias is not None or t5_table is not None or alibi_slopes is not None or \
+            rel_table is not None:
+        S = S + _bias_matrix(b, hq, L, bias, t5_table, t5_num_buckets, t5_max_distance,
+                             t5_bidirectional, alibi_slopes, Lk, rel_table)[r]
     M = visibility_mask(L, causal, window_left, window_right, Lk)[r]
     S = np.where(M, S, -np.inf)
     return S
@@ -234,7 +255,7 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
     """Probability matrix P (rows sum to 1 over visible keys) for one head."""
     q = _as64(q)
     k = _as64(k)
-    for name in ("bias", "t5_table", "alibi_slopes"):
+    for name in ("bias", "t5_table", "alibi_slopes", "rel_table"):
         if name in mask_bias:
             mask_bias[name] = _as64(mask_bias[name])
     S = head_scores(q, k, b, hq, scale=_scale_of(q.shape[-1], scale), **mask_bias)
@@ -245,19 +266,21 @@ def attention_probs(q, k, b, hq, *, scale=None, **mask_bias):
 def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
                       window_right=-1, bias=None, t5_table=None,
                       t5_num_buckets=32, t5_max_distance=128,
-                      t5_bidirectional=True, alibi_slopes=None, batches=None,
-                      kv_heads=None, query_rows=None):
+                      t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+                      batches=None, kv_heads=None, query_rows=None):
     """O = softmax(scale Q K^T + bias, masked) V and LSE, in float64.
 
     q: [B, L, Hq, d]; k, v: [B, Lk, Hkv, d] (Lk = L for self-attention);
     bias: [B|1, Hq|1, L|1, Lk] or None;
-    t5_table: [num_buckets, Hq] or None; alibi_slopes: [Hq] or None.
+    t5_table: [num_buckets, Hq] or None; alibi_slopes: [Hq] or None;
+    rel_table: [L + Lk - 1, Hq] (row j - i + L - 1) or None.
     Returns O [B, L, Hq, d] and
     LSE [B, Hq, L]; when ``batches`` / ``kv_heads`` restrict the work to a
     subset, entries outside it are NaN.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
     bias, t5_table, alibi_slopes = _as64(bias), _as64(t5_table), _as64(alibi_slopes)
+    rel_table = _as64(rel_table)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     assert Hq % Hkv == 0
@@ -268,7 +291,7 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
               t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional,
-              alibi_slopes=alibi_slopes)
+              alibi_slopes=alibi_slopes, rel_table=rel_table)
     r = np.arange(L) if query_rows is None else np.asarray(query_rows)
     bs, gs = _select(B, Hkv, batches, kv_heads)
     for b in bs:
@@ -284,8 +307,8 @@ def attention_forward(q, k, v, *, scale=None, causal=False, window_left=-1,
 def attention_backward(q, k, v, do, *, scale=None, causal=False,
                        window_left=-1, window_right=-1, bias=None,
                        t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-                       t5_bidirectional=True, alibi_slopes=None, batches=None,
-                       kv_heads=None, return_dbias=False):
+                       t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+                       batches=None, kv_heads=None, return_dbias=False):
     """Gradients of sum(O * dO) with respect to Q, K, V (float64).
 
     Returns dQ [B, L, Hq, d], dK and dV [B, Lk, Hkv, d] (and, with
@@ -294,6 +317,7 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
     bias, t5_table, alibi_slopes = _as64(bias), _as64(t5_table), _as64(alibi_slopes)
+    rel_table = _as64(rel_table)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
@@ -305,7 +329,7 @@ def attention_backward(q, k, v, do, *, scale=None, causal=False,
     kw = dict(causal=causal, window_left=window_left, window_right=window_right,
               bias=bias, t5_table=t5_table, t5_num_buckets=t5_num_buckets,
               t5_max_distance=t5_max_distance, t5_bidirectional=t5_bidirectional,
-              alibi_slopes=alibi_slopes)
+              alibi_slopes=alibi_slopes, rel_table=rel_table)
     bs, gs = _select(B, Hkv, batches, kv_heads)
     for b in bs:
         for g in gs:
@@ -371,6 +395,58 @@ def alibi_slope_gradient(dS):
     L, Lk = dS.shape[2], dS.shape[3]
     dist = np.abs(np.arange(Lk)[None, :] - np.arange(L)[:, None])
     return -np.einsum("bhij,ij->h", dS, dist)
+
+
+def rel_table_gradient(dS):
+    """Gradient of a relative-position table [L + Lk - 1, Hq] from dS
+    [B, Hq, L, Lk]: entry j - i + L - 1 collects every dS[b, h, i, j] at that
+    distance (chain rule through the lookup; one explicit scatter-add)."""
+    dS = np.asarray(dS, dtype=np.float64)
+    B, Hq, L, Lk = dS.shape
+    row = (np.arange(Lk)[None, :] - np.arange(L)[:, None] + L - 1).ravel()
+    grad = np.zeros((L + Lk - 1, Hq))
+    for h in range(Hq):
+        np.add.at(grad[:, h], row, dS[:, h].sum(axis=0).ravel())
+    return grad
+
+
+def _fire_inputs(L, Lk, c, threshold):
+    """FIRE's normalized distance x = psi(|i - j|) / psi(threshold) for the
+    rows j - i = -(L - 1) .. Lk - 1, psi(t) = log(c t + 1)."""
+    if threshold < L - 1:
+        raise ValueError("the FIRE threshold must be at least the last query position")
+    dist = np.abs(np.arange(-(L - 1), Lk, dtype=np.float64))
+    return np.log(c * dist + 1.0) / np.log(c * threshold + 1.0), dist
+
+
+def fire_table(L, Lk, c, threshold, w1, b1, w2, b2):
+    """FIRE bias as a relative-position table [L + Lk - 1, H] (Li et al.
+    2023): f(x) = w2 relu(w1 x + b1) + b2 per head, x = psi(|i - j|) /
+    psi(threshold), psi(t) = log(c t + 1).  w1, b1: [W]; w2: [H, W]; b2: [H]."""
+    w1, b1, w2, b2 = (np.asarray(a, dtype=np.float64) for a in (w1, b1, w2, b2))
+    x, _ = _fire_inputs(L, Lk, c, threshold)
+    hidden = np.maximum(np.outer(x, w1) + b1[None, :], 0.0)      # [R, W]
+    return hidden @ w2.T + b2[None, :]                             # [R, H]
+
+
+def fire_gradients(d_table, L, Lk, c, threshold, w1, b1, w2, b2):
+    """Gradients of sum(d_table * fire_table(...)) with respect to w1, b1, w2,
+    b2, c and threshold (chain rule through the MLP and psi).  Returns a dict
+    of float64 arrays (c and threshold as scalars)."""
+    g = np.asarray(d_table, dtype=np.float64)                      # [R, H]
+    w1, b1, w2, b2 = (np.asarray(a, dtype=np.float64) for a in (w1, b1, w2, b2))
+    x, dist = _fire_inputs(L, Lk, c, threshold)
+    pre = np.outer(x, w1) + b1[None, :]
+    hidden = np.maximum(pre, 0.0)
+    d_hidden = g @ w2                                              # [R, W]
+    d_pre = np.where(pre > 0.0, d_hidden, 0.0)
+    dx = d_pre @ w1                                                # [R]
+    num = np.log(c * dist + 1.0)
+    den = np.log(c * threshold + 1.0)
+    dx_dc = (dist / (c * dist + 1.0)) / den - num * (threshold / (c * threshold + 1.0)) / den ** 2
+    dx_dt = -num * (c / (c * threshold + 1.0)) / den ** 2
+    return {"w1": d_pre.T @ x, "b1": d_pre.sum(axis=0), "w2": g.T @ hidden,
+            "b2": g.sum(axis=0), "c": float(dx @ dx_dc), "threshold": float(dx @ dx_dt)}
 
 
 # --------------------------------------------------------------------------

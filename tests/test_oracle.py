@@ -13,8 +13,9 @@ import pytest
 import torch
 
 from oracle import (alibi_slope_gradient, attention_backward, attention_forward,
-                    attention_probs, dense_bias_gradient, head_scores, t5_relative_bucket,
-                    t5_table_gradient, visibility_mask)
+                    attention_probs, dense_bias_gradient, fire_gradients, fire_table,
+                    head_scores, rel_table_gradient, t5_relative_bucket, t5_table_gradient,
+                    visibility_mask)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -709,3 +710,103 @@ def test_packed_gradients_central_differences():
             a[which][idx] -= 2 * h
             num[idx] = (up - loss(*a)) / (2 * h)
         assert np.allclose(grad, num, rtol=1e-6, atol=1e-8), which
+
+
+# ------------------------------------------- relative-position table, FIRE
+def test_rel_table_equals_the_dense_bias_it_expands_to():
+    # cross-attention shape, so a wrong offset or a swapped i / j shows
+    B, L, Lk, Hq, Hkv, d = 1, 6, 9, 2, 1, 4
+    q = rnd((B, L, Hq, d), 71)
+    k, v = rnd((B, Lk, Hkv, d), 72), rnd((B, Lk, Hkv, d), 73)
+    do = rnd((B, L, Hq, d), 74)
+    table = rnd((L + Lk - 1, Hq), 75)
+    dense = np.zeros((1, Hq, L, Lk))
+    for h in range(Hq):
+        for i in range(L):
+            for j in range(Lk):
+                dense[0, h, i, j] = table[j - i + L - 1, h]     # entry j - i + L - 1
+    for causal in (False, True):
+        O1, L1 = attention_forward(q, k, v, causal=causal, rel_table=table)
+        O2, L2 = attention_forward(q, k, v, causal=causal, bias=dense)
+        assert np.allclose(O1, O2, atol=1e-14) and np.allclose(L1, L2, atol=1e-14)
+        g1 = attention_backward(q, k, v, do, causal=causal, rel_table=table)
+        g2 = attention_backward(q, k, v, do, causal=causal, bias=dense)
+        for a, b_ in zip(g1, g2):
+            assert np.allclose(a, b_, atol=1e-13)
+
+
+def test_rel_table_of_t5_buckets_is_the_t5_bias():
+    # a table filled from the (golden-pinned) T5 buckets gives the T5 bias
+    q, k, v, do = qkv(B=1, L=10, Hq=2, Hkv=2, d=4, seed=81)
+    t5 = rnd((32, 2), 82)
+    rel = np.arange(-9, 10)
+    table = t5[t5_relative_bucket(rel, 32, 128, True), :]
+    O1, _ = attention_forward(q, k, v, rel_table=table)
+    O2, _ = attention_forward(q, k, v, t5_table=t5)
+    assert np.allclose(O1, O2, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rel_table_gradient_central_differences(causal):
+    B, L, Hq, Hkv, d = 2, 7, 2, 1, 3
+    q, k, v, do = qkv(B, L, Hq, Hkv, d, seed=91)
+    table = rnd((2 * L - 1, Hq), 92)
+    kw = dict(causal=causal, rel_table=table)
+    *_, dS = attention_backward(q, k, v, do, return_dbias=True, **kw)
+    g = rel_table_gradient(dS)
+    h = 1e-6
+    for r, hq in [(0, 0), (L - 1, 1), (L + 2, 0), (2 * L - 2, 1), (3, 1)]:
+        tp = table.copy(); tp[r, hq] += h
+        tm = table.copy(); tm[r, hq] -= h
+        num = (_loss(q, k, v, do, {**kw, "rel_table": tp})
+               - _loss(q, k, v, do, {**kw, "rel_table": tm})) / (2 * h)
+        assert abs(num - g[r, hq]) < 1e-7, (r, hq, num, g[r, hq])
+    if causal:
+        assert np.all(g[L:, :] == 0.0)          # keys after the query see nothing
+
+
+def test_fire_table_hand_worked():
+    # c = 1, threshold 15: psi(t) = log(t + 1), psi(15) = log 16, so the
+    # distances 0, 1, 3, 15 map to x = 0, 1/4, 1/2, 1 exactly.  With
+    # w1 = (1, -1), b1 = (0, 1/2), w2 = (2, 3), b2 = 1/4:
+    #   f(x) = 2 relu(x) + 3 relu(1/2 - x) + 1/4
+    #   f(0) = 1.75, f(1/4) = 0.5 + 0.75 + 0.25 = 1.5,
+    #   f(1/2) = 1 + 0 + 0.25 = 1.25, f(1) = 2 + 0 + 0.25 = 2.25
+    t = fire_table(16, 16, 1.0, 15.0, [1.0, -1.0], [0.0, 0.5], [[2.0, 3.0]], [0.25])
+    assert t.shape == (31, 1)
+    for dist, want in ((0, 1.75), (1, 1.5), (3, 1.25), (15, 2.25)):
+        assert abs(t[15 + dist, 0] - want) < 1e-12 and abs(t[15 - dist, 0] - want) < 1e-12
+
+
+def test_fire_threshold_reading():
+    # the threshold must cover every query position: max(T, i) = T then
+    fire_table(8, 8, 1.0, 7.0, [1.0], [0.0], [[1.0]], [0.0])
+    with pytest.raises(ValueError):
+        fire_table(8, 8, 1.0, 6.0, [1.0], [0.0], [[1.0]], [0.0])
+
+
+def test_fire_gradients_central_differences():
+    rng = np.random.default_rng(97)
+    L, Lk, W, H = 9, 12, 5, 3
+    params = dict(w1=rng.standard_normal(W), b1=rng.standard_normal(W) * 0.5,
+                  w2=rng.standard_normal((H, W)), b2=rng.standard_normal(H))
+    c, thr = 0.7, 11.0
+    g = rng.standard_normal((L + Lk - 1, H))
+
+    def loss(p, c_, t_):
+        return float(np.sum(g * fire_table(L, Lk, c_, t_, p["w1"], p["b1"], p["w2"], p["b2"])))
+
+    grads = fire_gradients(g, L, Lk, c, thr, **params)
+    h = 1e-6
+    for name in ("w1", "b1", "w2", "b2"):
+        flat = params[name].reshape(-1)
+        for idx in range(flat.size):
+            pp = {n: a.copy() for n, a in params.items()}
+            pm = {n: a.copy() for n, a in params.items()}
+            pp[name].reshape(-1)[idx] += h
+            pm[name].reshape(-1)[idx] -= h
+            num = (loss(pp, c, thr) - loss(pm, c, thr)) / (2 * h)
+            assert abs(num - grads[name].reshape(-1)[idx]) < 1e-6, (name, idx)
+    num_c = (loss(params, c + h, thr) - loss(params, c - h, thr)) / (2 * h)
+    num_t = (loss(params, c, thr + h) - loss(params, c, thr - h)) / (2 * h)
+    assert abs(num_c - grads["c"]) < 1e-6 and abs(num_t - grads["threshold"]) < 1e-6
