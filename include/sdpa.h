@@ -96,7 +96,8 @@ typedef enum sdpa_bias_kind {
   SDPA_BIAS_NONE = 0,
   SDPA_BIAS_DENSE = 1, /* additive float32 bias[b, h, i, j]                  */
   SDPA_BIAS_T5 = 2,    /* additive table[bucket(j - i), h], bucketed in-kernel */
-  SDPA_BIAS_ALIBI = 3  /* additive -slope[h] |j - i|, computed in-kernel       */
+  SDPA_BIAS_ALIBI = 3, /* additive -slope[h] |j - i|, computed in-kernel       */
+  SDPA_BIAS_REL = 4    /* additive table[j - i + Lq - 1, h] (any function of j - i) */
 } sdpa_bias_kind;
 
 /*
@@ -121,6 +122,13 @@ typedef enum sdpa_bias_kind {
  *          formula; this is the linear bias of Press et al. 2022 ("Train
  *          Short, Test Long"), equal to their -m (i - j) on the keys a causal
  *          mask leaves.  Strides and T5 fields are ignored.
+ *   REL:   ptr -> float32 table[Lq + Lk - 1][Hq] (row-major); bias[h, i, j]
+ *          = table[j - i + Lq - 1][h]: any per-head function of the
+ *          distance, looked up per tile like T5 (the general form of T5 and
+ *          ALiBi; FIRE enters this way through sdpa_fire_table).  Packed
+ *          batches index it with the longest lengths (max_seqlen_q - 1
+ *          offset, positions from 0 in each sequence).  Strides and T5
+ *          fields are ignored.
  */
 typedef struct sdpa_bias_desc {
   int32_t kind; /* sdpa_bias_kind */
@@ -298,13 +306,18 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
  *          16-byte aligned.
  *   ALIBI: dbias[h] = -sum of |j - i| dS[b, h, i, j] over every (b, i, j):
  *          the gradient of the slopes, float32 [Hq], 16-byte aligned.
+ *   REL:   dbias[(r + L - 1) * Hq + h] = sum of dS[b, h, i, i + r] over every
+ *          (b, i): float32 [2L - 1, Hq] like the table, 16-byte aligned.
  *   NONE:  SDPA_ERR_UNSUPPORTED.
  * dq, dk, dv as sdpa_bwd.  Deterministic: every sum is taken in one fixed
  * order, so repeated calls give identical bits.
  * workspace: at least sdpa_bwd_bias_grad_workspace_size(shape, bias) bytes,
- * 256-byte aligned, contents ignored on entry.  Except for a full-shape dense
- * bias, it holds an fp32 copy of dS, B * Hq * L rows of L floats padded to a
- * multiple of 8, that the gradient is reduced from.  dbias must not overlap any other argument.
+ * 256-byte aligned, contents ignored on entry.  A broadcast dense bias
+ * stages an fp32 copy of dS there (B * Hq * L rows of L floats padded to a
+ * multiple of 8) and reduces it; T5, ALiBi and REL stage no dS: the dQ
+ * kernel sums dS along the distances j - i per warp, 1280 floats per
+ * (batch, head, query tile, key tile), folded in fixed order.  A full-shape
+ * dense bias stages nothing.  dbias must not overlap any other argument.
  */
 size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias);
 sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,
@@ -354,6 +367,50 @@ void sdpa_set_wait_limit_ns(uint64_t ns);
  * afterwards.
  */
 sdpa_status_t sdpa_debug_wait_timeout(void* stream);
+
+/*
+ * FIRE relative-position bias as a REL table.  The catie-aq/flashT5 README
+ * names FIRE among the positional schemes it means to support and gives no
+ * formula; this is the bias of Li et al. 2023 ("Functional Interpolation for
+ * Relative Positions Improves Long Context Transformers"):
+ *   bias[h, i, j] = f_h(psi(|i - j|) / psi(threshold)),  psi(t) = log(c t + 1),
+ *   f(x) = w2 relu(w1 x + b1) + b2  (one hidden layer of `width` units).
+ * The paper divides by psi(max(threshold, i)); with threshold >= Lq - 1 (a
+ * requirement here, else SDPA_ERR_UNSUPPORTED) that is psi(threshold) on
+ * every row, so the bias depends on the distance alone; keys after the
+ * query take the same function of |i - j|.  All pointers are device float32:
+ * w1, b1 [width], w2 [heads][width], b2 [heads]; 1 <= width <= 1024,
+ * 1 <= heads <= 65535, c > 0.  Arithmetic in float32.
+ */
+typedef struct sdpa_fire {
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  float c;
+  float threshold;
+  int32_t width;
+  int32_t heads;
+} sdpa_fire;
+
+/* table [Lq + Lk - 1][heads] (device, caller-owned): the REL table of FIRE. */
+sdpa_status_t sdpa_fire_table(const sdpa_fire* fire, int64_t Lq, int64_t Lk, float* table,
+                              void* stream);
+
+/* Bytes of device workspace sdpa_fire_backward needs (0 for bad arguments). */
+size_t sdpa_fire_backward_workspace_size(const sdpa_fire* fire, int64_t Lq, int64_t Lk);
+
+/*
+ * Gradients of sum(d_table * table) with respect to FIRE's parameters, from
+ * the gradient of its table (sdpa_bwd_bias_grad with a REL bias returns
+ * it): d_w1, d_b1 [width], d_w2 [heads][width], d_b2 [heads], d_c_threshold
+ * [2] = (d/dc, d/dthreshold); all device float32, written in full.  Every
+ * output is a sum over the table rows in a fixed order (deterministic).
+ */
+sdpa_status_t sdpa_fire_backward(const sdpa_fire* fire, int64_t Lq, int64_t Lk,
+                                 const float* d_table, float* d_w1, float* d_b1, float* d_w2,
+                                 float* d_b2, float* d_c_threshold, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Static English text for a status code. */
 const char* sdpa_status_string(sdpa_status_t status);

@@ -21,6 +21,8 @@ from .binding import (  # noqa: F401
     sdpa_bwd_workspace_size,
     sdpa_debug_wait_timeout,
     sdpa_exp2_fma,
+    sdpa_fire_backward,
+    sdpa_fire_table,
     sdpa_fwd,
     sdpa_fwd_varlen,
     sdpa_read_device_status,

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsdpa_b200.so")
 SDPA_OK = 0
 STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTED",
                 3: "SDPA_ERR_WORKSPACE", 4: "SDPA_ERR_CUDA", 5: "SDPA_ERR_TIMEOUT"}
-BIAS_NONE, BIAS_DENSE, BIAS_T5, BIAS_ALIBI = 0, 1, 2, 3
+BIAS_NONE, BIAS_DENSE, BIAS_T5, BIAS_ALIBI, BIAS_REL = 0, 1, 2, 3, 4
 
 BWD_PREPROCESS, BWD_DQ, BWD_DKDV, BWD_ALL = 1, 2, 4, 7
 
@@ -30,7 +30,8 @@ EXPORTED = ("sdpa_fwd", "sdpa_fwd_varlen", "sdpa_bwd", "sdpa_bwd_phases", "sdpa_
             "sdpa_bwd_noalloc", "sdpa_bwd_workspace_size", "sdpa_bwd_varlen_workspace_size",
             "sdpa_bwd_bias_grad", "sdpa_bwd_bias_grad_workspace_size", "sdpa_t5_bucket",
             "sdpa_exp2_fma", "sdpa_read_device_status", "sdpa_set_wait_limit_ns",
-            "sdpa_debug_wait_timeout", "sdpa_status_string")
+            "sdpa_debug_wait_timeout", "sdpa_status_string", "sdpa_fire_table",
+            "sdpa_fire_backward_workspace_size", "sdpa_fire_backward")
 
 
 class SdpaError(RuntimeError):
@@ -49,6 +50,12 @@ class BiasDesc(ctypes.Structure):
                 ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64),
                 ("stride_i", ctypes.c_int64), ("num_buckets", ctypes.c_int32),
                 ("max_distance", ctypes.c_int32), ("bidirectional", ctypes.c_int32)]
+
+
+class Fire(ctypes.Structure):
+    _fields_ = [("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("b2", ctypes.c_void_p), ("c", ctypes.c_float), ("threshold", ctypes.c_float),
+                ("width", ctypes.c_int32), ("heads", ctypes.c_int32)]
 
 
 class Shape(ctypes.Structure):
@@ -110,6 +117,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.sdpa_set_wait_limit_ns.restype = None
     lib.sdpa_debug_wait_timeout.argtypes = [vp]
     lib.sdpa_debug_wait_timeout.restype = i32
+    fp = ctypes.POINTER(Fire)
+    lib.sdpa_fire_table.argtypes = [fp, i64, i64, vp, vp]
+    lib.sdpa_fire_table.restype = i32
+    lib.sdpa_fire_backward_workspace_size.argtypes = [fp, i64, i64]
+    lib.sdpa_fire_backward_workspace_size.restype = sz
+    lib.sdpa_fire_backward.argtypes = [fp, i64, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sdpa_fire_backward.restype = i32
     lib.sdpa_status_string.argtypes = [i32]
     lib.sdpa_status_string.restype = ctypes.c_char_p
     if path is None:
@@ -174,10 +188,23 @@ def make_mask(causal: bool, window_left: int, window_right: int) -> MaskSpec:
 
 def make_bias(bias: torch.Tensor | None, t5_table: torch.Tensor | None, num_buckets: int,
               max_distance: int, bidirectional: bool, dims: tuple | None = None,
-              alibi_slopes: torch.Tensor | None = None) -> BiasDesc:
+              alibi_slopes: torch.Tensor | None = None,
+              rel_table: torch.Tensor | None = None) -> BiasDesc:
     """Bias descriptor; ``dims`` = (B, Hq, L) of the attention checks the shapes."""
-    if sum(x is not None for x in (bias, t5_table, alibi_slopes)) > 1:
-        raise ValueError("give one of a dense bias, a T5 table or ALiBi slopes")
+    if sum(x is not None for x in (bias, t5_table, alibi_slopes, rel_table)) > 1:
+        raise ValueError("give one of a dense bias, a T5 table, ALiBi slopes or a relative table")
+    if rel_table is not None:
+        if (rel_table.dtype != torch.float32 or rel_table.dim() != 2
+                or not rel_table.is_contiguous()):
+            raise ValueError("relative table must be contiguous float32 [Lq + Lk - 1, Hq]")
+        if dims is not None:
+            if rel_table.shape[1] != dims[1]:
+                raise ValueError("relative table columns must equal the query heads")
+            if len(dims) > 2 and dims[2] > 0:
+                Lk = dims[3] if len(dims) > 3 else dims[2]
+                if rel_table.shape[0] != dims[2] + Lk - 1:
+                    raise ValueError("relative table must have Lq + Lk - 1 rows")
+        return BiasDesc(BIAS_REL, rel_table.data_ptr(), 0, 0, 0, 0, 0, 0)
     if alibi_slopes is not None:
         if (alibi_slopes.dtype != torch.float32 or alibi_slopes.dim() != 1
                 or not alibi_slopes.is_contiguous()):
@@ -217,7 +244,7 @@ def _same_layout(a: torch.Tensor, ref: torch.Tensor, name: str):
 
 def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=None,
              t5_table=None, t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
-             alibi_slopes=None, scale=None, out=None, lse=None):
+             alibi_slopes=None, rel_table=None, scale=None, out=None, lse=None):
     """O, LSE = attention forward (see sdpa_fwd in include/sdpa.h)."""
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -235,7 +262,7 @@ def sdpa_fwd(q, k, v, *, causal=False, window_left=-1, window_right=-1, bias=Non
         raise ValueError("lse must be contiguous float32 [B, Hq, L]")
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (B, Hq, L, k.shape[1]), alibi_slopes)
+                   (B, Hq, L, k.shape[1]), alibi_slopes, rel_table)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bd),
                       ctypes.byref(m), sc, _ptr(out), _ptr(lse), _stream(q))
@@ -251,7 +278,8 @@ def sdpa_bwd_workspace_size(q, k, deterministic: bool = True) -> int:
 
 def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
              bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-             t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None, dv=None,
+             t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+             scale=None, dq=None, dk=None, dv=None,
              workspace=None, deterministic=True, phases=BWD_ALL):
     """dQ, dK, dV = attention backward (see sdpa_bwd / sdpa_bwd_phases in include/sdpa.h).
 
@@ -276,7 +304,7 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes, rel_table)
     m = make_mask(causal, window_left, window_right)
     args = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
             ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq), _ptr(dk), _ptr(dv),
@@ -291,7 +319,8 @@ def sdpa_bwd(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=
 
 def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_left=-1,
                      window_right=-1, bias=None, t5_table=None, t5_num_buckets=32,
-                     t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None, scale=None):
+                     t5_max_distance=128, t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+                     scale=None):
     """Backward into caller-given dQ, dK, dV with no workspace and no allocation.
 
     For callers that cannot allocate device memory: the library's built-in
@@ -306,7 +335,7 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
         _same_layout(t, ref, n)
     sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes, rel_table)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_bwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do),
                               _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc, _ptr(dq),
@@ -318,7 +347,7 @@ def sdpa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, *, causal=False, window_le
 def sdpa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, *,
                     causal=False, window_left=-1, window_right=-1, t5_table=None,
                     t5_num_buckets=32, t5_max_distance=128, t5_bidirectional=True,
-                    alibi_slopes=None, scale=None, out=None, lse=None):
+                    alibi_slopes=None, rel_table=None, scale=None, out=None, lse=None):
     """O [total_q, Hq, d], LSE [Hq, total_q] of a packed batch (sdpa_fwd_varlen)."""
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -338,7 +367,7 @@ def sdpa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
         raise ValueError("lse must be contiguous float32 [Hq, total_q]")
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
     bd = make_bias(None, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (B, q.shape[1], 0, 0), alibi_slopes)
+                   (B, q.shape[1], 0, 0), alibi_slopes, rel_table)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_fwd_varlen(ctypes.byref(shape), ctypes.byref(vl), _ptr(q), _ptr(k), _ptr(v),
                              ctypes.byref(bd), ctypes.byref(m), sc, _ptr(out), _ptr(lse),
@@ -350,7 +379,8 @@ def sdpa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
 def sdpa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                     max_seqlen_k, *, causal=False, window_left=-1, window_right=-1,
                     t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-                    t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None,
+                    t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+                    scale=None, dq=None, dk=None,
                     dv=None, workspace=None):
     """dQ, dK, dV of a packed batch (sdpa_bwd_varlen)."""
     lib = load_library()
@@ -372,7 +402,7 @@ def sdpa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_
         workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
     sc = 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
     bd = make_bias(None, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (B, q.shape[1], 0, 0), alibi_slopes)
+                   (B, q.shape[1], 0, 0), alibi_slopes, rel_table)
     m = make_mask(causal, window_left, window_right)
     st = lib.sdpa_bwd_varlen(ctypes.byref(shape), ctypes.byref(vl), _ptr(q), _ptr(k), _ptr(v),
                              _ptr(o), _ptr(do), _ptr(lse), ctypes.byref(bd), ctypes.byref(m), sc,
@@ -384,17 +414,18 @@ def sdpa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_
 
 def sdpa_bwd_bias_grad_workspace_size(q, k, *, bias=None, t5_table=None, t5_num_buckets=32,
                                       t5_max_distance=128, t5_bidirectional=True,
-                                      alibi_slopes=None) -> int:
+                                      alibi_slopes=None, rel_table=None) -> int:
     lib = load_library()
     shape = make_shape(q, k)
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes, rel_table)
     return int(lib.sdpa_bwd_bias_grad_workspace_size(ctypes.byref(shape), ctypes.byref(bd)))
 
 
 def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, window_right=-1,
                        bias=None, t5_table=None, t5_num_buckets=32, t5_max_distance=128,
-                       t5_bidirectional=True, alibi_slopes=None, scale=None, dq=None, dk=None,
+                       t5_bidirectional=True, alibi_slopes=None, rel_table=None,
+                       scale=None, dq=None, dk=None,
                        dv=None, dbias=None, workspace=None):
     """dQ, dK, dV and the bias gradient (see sdpa_bwd_bias_grad in include/sdpa.h).
 
@@ -413,8 +444,8 @@ def sdpa_bwd_bias_grad(q, k, v, o, do, lse, *, causal=False, window_left=-1, win
     _same_layout(dk, k, "dk")
     _same_layout(dv, k, "dv")
     bd = make_bias(bias, t5_table, t5_num_buckets, t5_max_distance, t5_bidirectional,
-                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes)
-    ref = next((x for x in (bias, t5_table, alibi_slopes) if x is not None), None)
+                   (q.shape[0], q.shape[2], q.shape[1], k.shape[1]), alibi_slopes, rel_table)
+    ref = next((x for x in (bias, t5_table, alibi_slopes, rel_table) if x is not None), None)
     if ref is None:
         raise ValueError("a bias gradient needs a dense bias, a T5 table or ALiBi slopes")
     if dbias is None:
@@ -469,6 +500,48 @@ def sdpa_set_wait_limit_ns(ns: int):
 
 def sdpa_debug_wait_timeout():
     _check(load_library().sdpa_debug_wait_timeout(_stream()), "sdpa_debug_wait_timeout")
+
+
+def _fire_desc(w1, b1, w2, b2, c, threshold):
+    for t, n in ((w1, "w1"), (b1, "b1"), (w2, "w2"), (b2, "b2")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"FIRE {n} must be a contiguous float32 CUDA tensor")
+    W = w1.shape[0]
+    if w1.dim() != 1 or b1.shape != (W,) or w2.dim() != 2 or w2.shape[1] != W or \
+            b2.shape != (w2.shape[0],):
+        raise ValueError("FIRE weights must be w1 [W], b1 [W], w2 [H, W], b2 [H]")
+    return Fire(w1.data_ptr(), b1.data_ptr(), w2.data_ptr(), b2.data_ptr(), float(c),
+                float(threshold), int(W), int(w2.shape[0]))
+
+
+def sdpa_fire_table(w1, b1, w2, b2, c, threshold, Lq, Lk, out=None):
+    """FIRE bias as a relative-position table [Lq + Lk - 1, H] (see sdpa_fire_table in
+    include/sdpa.h); pass it as ``rel_table``."""
+    f = _fire_desc(w1, b1, w2, b2, c, threshold)
+    if out is None:
+        out = torch.empty(Lq + Lk - 1, f.heads, device=w1.device, dtype=torch.float32)
+    _check(load_library().sdpa_fire_table(ctypes.byref(f), int(Lq), int(Lk), _ptr(out),
+                                          _stream(w1)), "sdpa_fire_table")
+    return out
+
+
+def sdpa_fire_backward(w1, b1, w2, b2, c, threshold, Lq, Lk, d_table):
+    """Gradients of FIRE's parameters from its table's gradient: a dict with w1, b1, w2,
+    b2 and c_threshold (d/dc, d/dthreshold)."""
+    lib = load_library()
+    f = _fire_desc(w1, b1, w2, b2, c, threshold)
+    if d_table.dtype != torch.float32 or not d_table.is_contiguous() or \
+            tuple(d_table.shape) != (Lq + Lk - 1, f.heads):
+        raise ValueError("d_table must be contiguous float32 [Lq + Lk - 1, H]")
+    need = int(lib.sdpa_fire_backward_workspace_size(ctypes.byref(f), int(Lq), int(Lk)))
+    ws = torch.empty(max(need, 256), device=w1.device, dtype=torch.uint8)
+    g = {n: torch.empty_like(t) for n, t in (("w1", w1), ("b1", b1), ("w2", w2), ("b2", b2))}
+    g["c_threshold"] = torch.empty(2, device=w1.device, dtype=torch.float32)
+    _check(lib.sdpa_fire_backward(ctypes.byref(f), int(Lq), int(Lk), _ptr(d_table), _ptr(g["w1"]),
+                                  _ptr(g["b1"]), _ptr(g["w2"]), _ptr(g["b2"]),
+                                  _ptr(g["c_threshold"]), _ptr(ws), ws.numel(), _stream(w1)),
+           "sdpa_fire_backward")
+    return g
 
 
 def sdpa_status_string(status: int) -> str:

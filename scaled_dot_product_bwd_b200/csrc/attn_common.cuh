@@ -97,6 +97,10 @@ struct AttnParams {
   // that the kernels tabulate per tile
   int alibi;                   // 1: bias = -alibi_slopes[h] |j - i| instead of T5
   const float* alibi_slopes;   // [Hq]
+  // a relative-position table instead of T5 (when not null): bias =
+  // rel_table[(j - i + rel_off) * Hq + h], rows 0 .. rel_rows - 1
+  const float* rel_table;
+  int rel_off, rel_rows;
   uint64_t wait_limit_ns;
 };
 
@@ -142,9 +146,16 @@ __device__ __forceinline__ int64_t row_index(const AttnParams& p, const SeqView&
 // Relative-position bias of distance rel = j - i for query head hq, in log2
 // units (times log2 e), as the kBiasT5 kernels tabulate it per tile: the
 // T5 table entry of rel's bucket (catie-aq/flashT5 README, "T5-like relative
-// position encoding biases"), or ALiBi's -m_h |rel| (Press et al. 2022;
-// named by the same README among the supported positional schemes).
+// position encoding biases"), ALiBi's -m_h |rel| (Press et al. 2022; named
+// by the same README among the supported positional schemes), or a
+// caller's table entry for rel (the general form; FIRE's table).
 __device__ __forceinline__ float rel_bias_log2(const AttnParams& p, int rel, int hq) {
+  if (p.rel_table) {
+    // tables cover the in-range distances; the tile-wide lookup rows also
+    // span positions past the sequences, which the mask hides: clamp those
+    const int r = min(max(rel + p.rel_off, 0), p.rel_rows - 1);
+    return p.rel_table[static_cast<int64_t>(r) * p.Hq + hq] * kLog2e;
+  }
   if (p.alibi) return -(p.alibi_slopes[hq] * kLog2e) * fabsf(static_cast<float>(rel));
   return p.t5_table[t5_bucket(rel, p.t5) * p.Hq + hq] * kLog2e;
 }

@@ -260,6 +260,16 @@ __global__ void __launch_bounds__(256) t5_bucket_sum_kernel(const T5Reduce a, co
   if (threadIdx.x == 0) a.out[static_cast<int64_t>(k) * a.Hq + h] = red[0];
 }
 
+// REL: out[(r + L - 1) * Hq + h] = diagonal sum of r (a transpose).
+__global__ void __launch_bounds__(256) rel_table_grad_kernel(const T5Reduce a) {
+  const int nd = 2 * a.L - 1;
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<int64_t>(nd) * a.Hq) return;
+  const int row = static_cast<int>(idx / a.Hq);
+  const int h = static_cast<int>(idx - static_cast<int64_t>(row) * a.Hq);
+  a.out[idx] = a.partial[static_cast<int64_t>(h) * nd + row];
+}
+
 // ALiBi: the bias -m_h |r| is linear in the slope, so
 // out[h] = -sum over r of |r| times the diagonal sum of r; one block per
 // head, a fixed tree over its 256 threads.

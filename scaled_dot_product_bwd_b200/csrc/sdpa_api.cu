@@ -15,6 +15,7 @@
 #include "sdpa.h"
 #include "attn_common.cuh"
 #include "bias_grad.cuh"
+#include "fire.cuh"
 #include "bwd_kernels.cuh"
 #include "fwd_kernel.cuh"
 
@@ -251,6 +252,12 @@ sdpa_status_t prepare(const Geometry& g, const sdpa_bias_desc* bias, const sdpa_
       p.bias_kind = kBiasT5;  // the relative-position kernels, with the ALiBi table
       p.alibi = 1;
       p.alibi_slopes = bias->ptr;
+    } else if (bias->kind == SDPA_BIAS_REL) {
+      if (!bias->ptr) return SDPA_ERR_INVALID_ARG;
+      p.bias_kind = kBiasT5;  // the relative-position kernels, with the caller's table
+      p.rel_table = bias->ptr;
+      p.rel_off = p.Lq - 1;
+      p.rel_rows = p.Lq + p.Lk - 1;
     } else {
       return SDPA_ERR_INVALID_ARG;
     }
@@ -424,7 +431,8 @@ sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, Bias
       if (pl.chunks > 1)
         pl.part_bytes = round256(static_cast<size_t>(pl.chunks * n_out * pl.lp) * sizeof(float));
     }
-  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_ALIBI) {
+  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_ALIBI ||
+             bias->kind == SDPA_BIAS_REL) {
     // per (batch, head, query tile, key tile): 1024 per-warp sums and 256
     // tile diagonals; per head: 2L - 1 diagonal totals
     const int64_t nt = (L + kTile - 1) / kTile;
@@ -612,7 +620,8 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   st = plan_bias_grad(g, bias, pl);
   if (st != SDPA_OK) return st;
   T5Ranges rg;
-  if (p.bias_kind == kBiasT5 && !p.alibi && !t5_ranges(p.t5, p.Lq, bias->num_buckets, rg))
+  if (p.bias_kind == kBiasT5 && !p.alibi && !p.rel_table &&
+      !t5_ranges(p.t5, p.Lq, bias->num_buckets, rg))
     return SDPA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < pl.total)
@@ -622,9 +631,9 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   const int L = p.Lq;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (pl.diag) {
-    // T5 / ALiBi: per-warp diagonal sums from the dQ kernel, folded per
-    // tile, per tile offset, then per head, then per bucket (or weighed by
-    // -|r| per slope)
+    // T5 / ALiBi / REL: per-warp diagonal sums from the dQ kernel, folded
+    // per tile, per tile offset, then per head, then per bucket (weighed by
+    // -|r| per slope; one per table row)
     uint8_t* base = ws + pl.bwd_bytes;
     DiagFold f;
     f.warp_part = reinterpret_cast<const float*>(base);
@@ -652,10 +661,14 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.partial = f.diag;
     a.out = dbias;
     a.num_buckets = p.alibi ? 0 : bias->num_buckets;
-    if (p.alibi)
+    if (p.rel_table) {
+      const int64_t n = static_cast<int64_t>(2 * L - 1) * p.Hq;
+      rel_table_grad_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(a);
+    } else if (p.alibi) {
       alibi_slope_grad_kernel<<<p.Hq, 256, 0, cs>>>(a);
-    else
+    } else {
       t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
+    }
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
   }
   if (pl.ds_ws) {
@@ -793,6 +806,98 @@ sdpa_status_t sdpa_read_device_status(void* stream) {
 
 sdpa_status_t sdpa_debug_wait_timeout(void* stream) {
   wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_limit_ns);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ FIRE
+namespace {
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+sdpa_status_t fire_check(const sdpa_fire* f, int64_t Lq, int64_t Lk, FireArgs& a) {
+  if (!f || !f->w1 || !f->b1 || !f->w2 || !f->b2) return SDPA_ERR_INVALID_ARG;
+  if (!aligned4(f->w1) || !aligned4(f->b1) || !aligned4(f->w2) || !aligned4(f->b2))
+    return SDPA_ERR_INVALID_ARG;
+  if (f->width < 1 || f->width > 1024 || f->heads < 1 || f->heads > 65535)
+    return SDPA_ERR_INVALID_ARG;
+  if (!std::isfinite(f->c) || !(f->c > 0.f) || !std::isfinite(f->threshold))
+    return SDPA_ERR_INVALID_ARG;
+  if (Lq < 1 || Lk < 1 || Lq >= (1ll << 30) || Lk >= (1ll << 30)) return SDPA_ERR_INVALID_ARG;
+  if (static_cast<double>(f->threshold) < static_cast<double>(Lq - 1)) return SDPA_ERR_UNSUPPORTED;
+  a.w1 = f->w1;
+  a.b1 = f->b1;
+  a.w2 = f->w2;
+  a.b2 = f->b2;
+  a.c = f->c;
+  a.thr = f->threshold;
+  a.W = f->width;
+  a.H = f->heads;
+  a.Lq = static_cast<int>(Lq);
+  a.Lk = static_cast<int>(Lk);
+  return SDPA_OK;
+}
+
+struct FirePlan {
+  size_t hid, dpre, x, dxc, dxt, total;
+};
+
+FirePlan fire_plan(int64_t R, int W) {
+  FirePlan pl;
+  pl.hid = 0;
+  pl.dpre = round256(static_cast<size_t>(R) * W * sizeof(float));
+  pl.x = pl.dpre + pl.dpre;
+  pl.dxc = pl.x + round256(static_cast<size_t>(R) * sizeof(float));
+  pl.dxt = pl.dxc + round256(static_cast<size_t>(R) * sizeof(float));
+  pl.total = pl.dxt + round256(static_cast<size_t>(R) * sizeof(float));
+  return pl;
+}
+}  // namespace
+
+sdpa_status_t sdpa_fire_table(const sdpa_fire* fire, int64_t Lq, int64_t Lk, float* table,
+                              void* stream) {
+  FireArgs a;
+  sdpa_status_t st = fire_check(fire, Lq, Lk, a);
+  if (st != SDPA_OK) return st;
+  if (!table || !aligned4(table)) return SDPA_ERR_INVALID_ARG;
+  const int64_t n = (Lq + Lk - 1) * static_cast<int64_t>(a.H);
+  fire_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0,
+                      static_cast<cudaStream_t>(stream)>>>(a, table);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+size_t sdpa_fire_backward_workspace_size(const sdpa_fire* fire, int64_t Lq, int64_t Lk) {
+  FireArgs a;
+  if (fire_check(fire, Lq, Lk, a) != SDPA_OK) return 0;
+  return fire_plan(Lq + Lk - 1, a.W).total;
+}
+
+sdpa_status_t sdpa_fire_backward(const sdpa_fire* fire, int64_t Lq, int64_t Lk,
+                                 const float* d_table, float* d_w1, float* d_b1, float* d_w2,
+                                 float* d_b2, float* d_c_threshold, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  FireArgs a;
+  sdpa_status_t st = fire_check(fire, Lq, Lk, a);
+  if (st != SDPA_OK) return st;
+  const void* ptrs[] = {d_table, d_w1, d_b1, d_w2, d_b2, d_c_threshold};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned4(ptr)) return SDPA_ERR_INVALID_ARG;
+  const int64_t R = Lq + Lk - 1;
+  const FirePlan pl = fire_plan(R, a.W);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < pl.total)
+    return SDPA_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  FireWork ws;
+  ws.hid = reinterpret_cast<float*>(w + pl.hid);
+  ws.dpre = reinterpret_cast<float*>(w + pl.dpre);
+  ws.x = reinterpret_cast<float*>(w + pl.x);
+  ws.dxc = reinterpret_cast<float*>(w + pl.dxc);
+  ws.dxt = reinterpret_cast<float*>(w + pl.dxt);
+  FireOut out{d_w1, d_b1, d_w2, d_b2, d_c_threshold};
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  fire_rows_kernel<<<static_cast<unsigned>((R + 127) / 128), 128, 0, cs>>>(a, d_table, ws);
+  if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+  const int64_t n_out = static_cast<int64_t>(a.H) * a.W + a.H + 2 * a.W + 2;
+  fire_reduce_kernel<<<static_cast<unsigned>(n_out), 256, 0, cs>>>(a, d_table, ws, out);
   return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 

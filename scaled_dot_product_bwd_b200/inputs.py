@@ -29,15 +29,17 @@ class Inputs:
     t5_table: torch.Tensor | None = None
     bias: torch.Tensor | None = None
     alibi_slopes: torch.Tensor | None = None
+    rel_table: torch.Tensor | None = None
 
 
 def make_inputs(B: int, L: int, Hq: int, Hkv: int, d: int, *, seed: int = 0,
                 t5_buckets: int = 0, dense_bias: bool = False,
                 bias_shape: tuple | None = None, alibi: bool = False,
-                Lk: int | None = None) -> Inputs:
+                Lk: int | None = None, rel_table: bool = False) -> Inputs:
     """Draw Q, K, V, dO (bf16) and optionally a T5 table / dense bias (fp32).
 
-    K and V have Lk rows (default L).  ALiBi slopes are not drawn: they are
+    K and V have Lk rows (default L).  A relative-position table is
+    [L + Lk - 1, Hq] N(0,1) fp32, drawn last.  ALiBi slopes are not drawn: they are
     the geometric sequence of Press et al. 2022, 2^(-8 (h + 1) / Hq) for head
     h (fp32)."""
     g = torch.Generator().manual_seed(seed)
@@ -58,7 +60,20 @@ def make_inputs(B: int, L: int, Hq: int, Hkv: int, d: int, *, seed: int = 0,
     if alibi:
         slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)],
                               dtype=torch.float32)
-    return Inputs(q, k, v, do, table, bias, slopes)
+    rel = randn(L + Lk - 1, Hq) if rel_table else None
+    return Inputs(q, k, v, do, table, bias, slopes, rel)
+
+
+def make_fire_params(width: int, heads: int, *, seed: int = 0) -> dict:
+    """Seeded FIRE MLP weights (fp32): w1, b1 [width] ~ N(0,1) and N(0,1) / 2,
+    w2 [heads, width] ~ N(0,1) / sqrt(width), b2 [heads] ~ N(0,1) / 2."""
+    g = torch.Generator().manual_seed(seed)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+    return dict(w1=randn(width), b1=randn(width) * 0.5,
+                w2=randn(heads, width) * (1.0 / width ** 0.5), b2=randn(heads) * 0.5)
 
 
 # The workloads of the benchmark table, by name.  Each entry: shapes, mask and

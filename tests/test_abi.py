@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from scaled_dot_product_bwd_b200 import binding
 from scaled_dot_product_bwd_b200.build import LIB_PATH, build
@@ -268,3 +269,43 @@ def test_t5_bucket_rejects_bad_args(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         binding.load_library(str(tmp_path / "missing.so"))
+
+
+def test_fire_rejects_bad_args(lib):
+    def fire(**kw):
+        base = dict(w1=0x10000, b1=0x10000, w2=0x10000, b2=0x10000, c=0.5, threshold=300.0,
+                    width=32, heads=4)
+        base.update(kw)
+        return binding.Fire(*[base[n] for n, _ in binding.Fire._fields_])
+
+    def table(f, Lq=200, Lk=150, out=FAKE):
+        return lib.sdpa_fire_table(ctypes.byref(f) if f else None, Lq, Lk, out, None)
+    assert table(None) == 1
+    assert table(fire(w2=0)) == 1
+    assert table(fire(b1=0x10002)) == 1                   # not 4-byte aligned
+    for bad in (dict(width=0), dict(width=1025), dict(heads=0), dict(c=0.0), dict(c=-1.0),
+                dict(c=float("nan")), dict(threshold=float("inf"))):
+        assert table(fire(**bad)) == 1, bad
+    assert table(fire(), Lq=0) == 1
+    assert table(fire(), out=None) == 1
+    assert table(fire(threshold=198.0)) == 2             # below the last query position
+    # workspace: hidden activations and their gradients [R, W], then x, dx/dc, dx/dT [R]
+    r256 = lambda x: (x + 255) // 256 * 256
+    R = 200 + 150 - 1
+    want = 2 * r256(R * 32 * 4) + 3 * r256(R * 4)
+    assert lib.sdpa_fire_backward_workspace_size(ctypes.byref(fire()), 200, 150) == want
+    assert lib.sdpa_fire_backward_workspace_size(ctypes.byref(fire(threshold=10.0)), 200, 150) == 0
+    args = [FAKE] * 6
+    assert lib.sdpa_fire_backward(ctypes.byref(fire()), 200, 150, *args, FAKE, want - 1, None) == 3
+    assert lib.sdpa_fire_backward(ctypes.byref(fire()), 200, 150, *args, None, want, None) == 3
+    assert lib.sdpa_fire_backward(ctypes.byref(fire()), 200, 150, None, *args[1:], FAKE, want,
+                                  None) == 1
+
+
+def test_rel_table_bias_checks(lib):
+    s = _shape()
+    rel = binding.BiasDesc(4, None, 0, 0, 0, 0, 0, 0)
+    assert _fwd(lib, s, bias=rel) == 1                       # no table
+    with pytest.raises(ValueError):
+        binding.make_bias(None, None, 32, 128, True, (1, 4, 128), None,
+                          torch.zeros(200, 4))               # rows != L + Lk - 1

@@ -89,7 +89,7 @@ U_BF16 = 2.0 ** -8
 def row_error_scale(c, inp):
     """e_i of the module docstring, [B, Hq, L], from the oracle's O and dO."""
     kw = dict(mask_kw(c), bias=inp.bias, t5_table=inp.t5_table,
-              alibi_slopes=inp.alibi_slopes)
+              alibi_slopes=inp.alibi_slopes, rel_table=getattr(inp, "rel_table", None))
     O, _ = attention_forward(inp.q, inp.k, inp.v, **kw)          # [B, L, Hq, d]
     dO = inp.do.double().numpy()
     e = 4 * U_BF16 * np.sqrt(np.sum((dO * O) ** 2, axis=-1))     # [B, L, Hq]
