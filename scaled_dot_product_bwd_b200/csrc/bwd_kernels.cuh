@@ -320,20 +320,28 @@ __global__ void __launch_bounds__(352, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 keys x 128 queries
       constexpr uint32_t kIdG = idesc_bf16_f32(kTile, D, 0, 1);      // 128 keys x d
       const bool chain_s = (warp == 9);
+      // Descriptors are built once: one at shared-memory offset 0 per layout,
+      // plus the byte offset / 16 of each operand (the start-address field),
+      // so an MMA costs the issuing thread two adds.  The issuer shares its
+      // sub-partition with busy compute warps, so its instruction count is
+      // what its issue rate is spent on.
+      const uint64_t dk0 = smem_desc_sw128(sb, 16, 1024);            // K-major
+      const uint64_t dmn0 = smem_desc_sw128(sb, kTile * 128, 1024);  // MN-major, 64-wide halves
       bool ok = issuer_wait(kv_full, 0, ctl);
       for (int it = 0; it < total && ok; ++it) {
         const int sq = it % SQ, so = it % SO;
-        const uint32_t qs = sb + Lay::kQOff + sq * Lay::kTileBytes;
-        const uint32_t dos = sb + Lay::kDOOff + so * Lay::kTileBytes;
+        const uint64_t qk = dk0 + ((Lay::kQOff + sq * Lay::kTileBytes) >> 4);
+        const uint64_t qm = dmn0 + ((Lay::kQOff + sq * Lay::kTileBytes) >> 4);
+        const uint64_t od = dk0 + ((Lay::kDOOff + so * Lay::kTileBytes) >> 4);
+        const uint64_t om = dmn0 + ((Lay::kDOOff + so * Lay::kTileBytes) >> 4);
         if (chain_s) {
           if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
           if (it > 0 && !(ok = issuer_wait(s_free, (it - 1) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + Lay::kSCol,
-                   smem_desc_sw128(sb + Lay::kKOff + kmajor_koff(kk, kTile), 16, 1024),
-                   smem_desc_sw128(qs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + Lay::kSCol, dk0 + ((Lay::kKOff + kmajor_koff(kk, kTile)) >> 4),
+                   qk + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
           mma_commit(s_full);
           mma_commit(q_empty(sq));
           if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
@@ -341,9 +349,8 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk),
-                   smem_desc_sw128(dos + kk * 2048, kTile * 128, 1024), kIdG,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk), om + kk * (2048 >> 4),
+                   kIdG, (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(s_free);
           mma_commit(o_empty(so));
         } else {
@@ -352,9 +359,8 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + Lay::kDPCol,
-                   smem_desc_sw128(sb + Lay::kVOff + kmajor_koff(kk, kTile), 16, 1024),
-                   smem_desc_sw128(dos + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + Lay::kDPCol, dk0 + ((Lay::kVOff + kmajor_koff(kk, kTile)) >> 4),
+                   od + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
           mma_commit(dp_full);
           mma_commit(o_empty(so));
           if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
@@ -362,8 +368,8 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk),
-                   smem_desc_sw128(qs + kk * 2048, kTile * 128, 1024), kIdG,
+            mma_ts(tmem + Lay::kDKCol, split_a_col(tmem + Lay::kDPCol, kk), qm + kk * (2048 >> 4),
+                   kIdG,
                    (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(dp_free);
           mma_commit(q_empty(sq));
@@ -808,17 +814,20 @@ __global__ void __launch_bounds__(352, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
       const bool chain_s = (warp == 9);
+      // descriptors built once, plus byte offset / 16 per operand (see the
+      // dK/dV kernel's issuers)
+      const uint64_t dk0 = smem_desc_sw128(sb, 16, 1024);            // K-major
+      const uint64_t dmn0 = smem_desc_sw128(sb, kTile * 128, 1024);  // MN-major, 64-wide halves
       auto issue_dp = [&](int c) -> bool {
         const int sv = c % SV;
         if (!issuer_wait(v_full(sv), (c / SV) & 1, ctl)) return false;
         if (c > 0 && !issuer_wait(dp_used, (c - 1) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+        const uint64_t vd = dk0 + ((Lay::kVOff + sv * Lay::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + Lay::kDPCol,
-                 smem_desc_sw128(sb + Lay::kDOOff + kmajor_koff(kk, kTile), 16, 1024),
-                 smem_desc_sw128(vs + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + Lay::kDPCol, dk0 + ((Lay::kDOOff + kmajor_koff(kk, kTile)) >> 4),
+                 vd + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
         mma_commit(dp_full);
         mma_commit(v_empty(sv));
         return true;
@@ -834,16 +843,16 @@ __global__ void __launch_bounds__(352, 1)
         for (int it = 0; it < w.nt; ++it, ++c) {
           const int x = c & 1;
           const int sk = c % SK;
-          const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+          const uint64_t kd = dk0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
+          const uint64_t kmd = dmn0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
           if (chain_s) {
             if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
             if (c >= 2 && !(ok = issuer_wait(dq_done(x), ((c >> 1) - 1) & 1, ctl))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + kTile * x,
-                     smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
-                     smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS,
+              mma_ss(tmem + kTile * x, dk0 + ((Lay::kQOff + kmajor_koff(kk, kTile)) >> 4),
+                     kd + (kmajor_koff(kk, kTile) >> 4), kIdS,
                      kk > 0 ? 1u : 0u);
             mma_commit(s_full(x));
             mma_commit(k_empty(sk));
@@ -856,8 +865,8 @@ __global__ void __launch_bounds__(352, 1)
             // warpgroup thread read the previous item's dQ before marking dS ready
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk),
-                     smem_desc_sw128(ks + kk * 2048, kTile * 128, 1024), kIdQ,
+              mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk), kmd + kk * (2048 >> 4),
+                     kIdQ,
                      (it > 0 || kk > 0) ? 1u : 0u);
             mma_commit(dq_done(x));
             mma_commit(k_empty(sk));

@@ -271,6 +271,12 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_bf16_f32(kTile, D, 0, 1);      // V is N(=d)-major
       const bool chain_s = (warp == 9);
+      // Descriptors are built once: one at shared-memory offset 0 per layout,
+      // plus the byte offset / 16 of each operand (the start-address field),
+      // so an MMA costs the issuing thread two adds; it shares its
+      // sub-partition with busy softmax warps.
+      const uint64_t dk0 = smem_desc_sw128(sb, 16, 1024);            // K-major
+      const uint64_t dmn0 = smem_desc_sw128(sb, kTile * 128, 1024);  // MN-major, 64-wide halves
       int c = 0;  // tiles so far, over all items
       int u = 0;  // items with a non-empty band so far
       bool ok = true;
@@ -286,12 +292,11 @@ __global__ void __launch_bounds__(384, 1)
             // buffer x held P of tile c - NS: wait until its P V MMA is done
             if (c >= NS && !(ok = issuer_wait(pv_done(x), ((c / NS) - 1) & 1, ctl))) break;
             tc_fence_after();
-            const uint32_t ks = sb + Lay::kKOff + sk * Lay::kTileBytes;
+            const uint64_t kd = dk0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + x * kTile,
-                     smem_desc_sw128(sb + Lay::kQOff + kmajor_koff(kk, kTile), 16, 1024),
-                     smem_desc_sw128(ks + kmajor_koff(kk, kTile), 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + x * kTile, dk0 + ((Lay::kQOff + kmajor_koff(kk, kTile)) >> 4),
+                     kd + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
             mma_commit(s_full(x));
             mma_commit(k_empty(sk));
           } else {
@@ -301,11 +306,10 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = issuer_wait(v_full(sv), (c / SV) & 1, ctl))) break;
             if (!(ok = issuer_wait(p_full(x), (c / NS) & 1, ctl))) break;
             tc_fence_after();
-            const uint32_t vs = sb + Lay::kVOff + sv * Lay::kTileBytes;
+            const uint64_t vmd = dmn0 + ((Lay::kVOff + sv * Lay::kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_ts(tmem + Lay::kOCol, split_a_col(tmem + x * kTile, kk),
-                     smem_desc_sw128(vs + kk * 2048, kTile * 128, 1024), kIdO,
+              mma_ts(tmem + Lay::kOCol, split_a_col(tmem + x * kTile, kk), vmd + kk * (2048 >> 4), kIdO,
                      (it > 0 || kk > 0) ? 1u : 0u);
             mma_commit(pv_done(x));
             mma_commit(v_empty(sv));
