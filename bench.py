@@ -543,26 +543,36 @@ def visited_tile_pairs(c):
 def bias_grad_extra_bytes(c):
     """HBM bytes the bias gradient adds to the backward.  A dense bias: the
     fp32 dS written once (full shape), or written and read back by the
-    broadcast reduction.  T5 / ALiBi: the dQ kernel's per-warp diagonal sums
-    (1024 floats per visited tile pair) and the per-tile diagonals (256)
-    written and read back once, then the per-head totals and the result."""
+    broadcast reduction.  T5: the dQ kernel's per-warp diagonal sums (1024
+    floats per visited tile pair), the per-tile diagonals (256) and the
+    per-tile-offset sums (256 per offset), each written and read back once,
+    then the per-head totals and the result.  ALiBi: the dQ kernel's
+    per-warp sums of |j - i| dS (8 floats per visited tile pair) written and
+    read back once, then the result."""
     B, H, L = c["B"], c["Hq"], c["L"]
-    if c["bias"] in ("t5", "alibi"):
+    if c["bias"] == "t5":
         tiles = B * H * visited_tile_pairs(c)
-        out = 32 * H * 4 if c["bias"] == "t5" else H * 4
-        return 2 * tiles * (1024 + 256) * 4 + 2 * H * (2 * L - 1) * 4 + out
+        nt = (L + 127) // 128
+        return (2 * tiles * (1024 + 256) * 4 + 2 * B * H * (2 * nt - 1) * 256 * 4 +
+                2 * H * (2 * L - 1) * 4 + 32 * H * 4)
+    if c["bias"] == "alibi":
+        tiles = B * H * visited_tile_pairs(c)
+        return 2 * tiles * 8 * 4 + H * 4
     return B * H * L * L * 4       # a full-shape dense bias: dS goes straight out
 
 
 def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
-    preprocess, the dQ kernel (storing dS, or its diagonal sums) and the
-    dK/dV kernel; a dense bias under a mask adds the zero fill of skipped key
-    tiles; T5 / ALiBi add the per-tile fold, the per-tile-offset sums, the
-    per-head totals and the per-bucket (or per-slope) sums."""
+    preprocess, the dQ kernel (storing dS, its diagonal sums or its |j - i|
+    moments) and the dK/dV kernel; a dense bias under a mask adds the zero
+    fill of skipped key tiles; T5 adds the per-tile fold, the
+    per-tile-offset sums, the per-head totals and the per-bucket sums;
+    ALiBi the per-head sum of the moments."""
     n = 4
-    if c["bias"] in ("t5", "alibi"):
+    if c["bias"] == "t5":
         return n + 4
+    if c["bias"] == "alibi":
+        return n + 1
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1
     return n
@@ -650,7 +660,7 @@ def run_bias_grad(args, c):
                       "bwd_bias_grad": round(res[True]["bwd"], 4),
                       "bwd_plain": round(res[False]["bwd"], 4)},
         "bias_grad_extra_ms": round(extra_ms, 4),
-        "roofline": {"kernel": "bias-gradient extra (dS store + reduction)", "bound": "hbm",
+        "roofline": {"kernel": "bias-gradient extra (dS, its partial sums, reductions)", "bound": "hbm",
                      "achieved": None if ach is None else round(ach, 1),
                      "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": None if ach is None else round(ach / peaks["hbm"], 4),

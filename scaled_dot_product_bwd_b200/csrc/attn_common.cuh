@@ -31,6 +31,11 @@ struct T5Spec {
   int nthr;
   int bidirectional;
   int thr[kMaxT5Thresholds];
+  // Every rel <= one_lo_max lies in the capped bucket of keys before the
+  // query, every rel >= one_hi_min in one bucket too (the capped bucket of
+  // keys after it, or bucket 0 of a unidirectional table); INT_MIN /
+  // INT_MAX when no distance in range is capped.
+  int one_lo_max, one_hi_min;
 };
 
 __host__ __device__ __forceinline__ int t5_bucket(int rel, const T5Spec& s) {

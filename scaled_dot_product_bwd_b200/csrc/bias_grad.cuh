@@ -2,9 +2,10 @@
 // bias's gradient is dS summed over each index the bias is broadcast along
 // (from the fp32 dS the dQ kernel stores in its store mode), a T5 table
 // entry's gradient is dS summed over every (b, i, j) whose distance j - i
-// falls in its bucket, and an ALiBi slope's is minus the sum of |j - i| dS
+// falls in its bucket and a relative-position table row's over its distance
 // (both from the per-warp diagonal sums of dS the dQ kernel writes in its
-// diagonal mode; catie-aq/flashT5 README, "Full attention biases" and
+// diagonal modes), and an ALiBi slope's is minus the sum of |j - i| dS (from
+// the per-warp sums of its moment mode; catie-aq/flashT5 README, "Full attention biases" and
 // "T5-like relative position encoding biases": a learnable bias needs these
 // to train).
 //
@@ -136,16 +137,16 @@ __global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseRedu
 }
 
 // ---------------------------------------------------------------------
-// T5 table (and ALiBi slope) gradient.  The bias depends on j - i alone, so
-// first sum dS along each diagonal r = j - i (r in [-(L-1), L-1]), then add
-// up the diagonals of each bucket (or weigh them by -|r| for ALiBi).  Every
+// T5 table (and relative-position table) gradient.  The bias depends on
+// j - i alone, so first sum dS along each diagonal r = j - i (r in
+// [-(L-1), L-1]), then add up the diagonals of each bucket.  Every
 // bucket covers one contiguous range of r (the bucket is monotone in |r| on
 // each side of 0, and the two sides use disjoint ids when bidirectional),
 // given to the last kernel as [lo, hi].
 struct T5Reduce {
   const float* partial;          // diagonal sums [Hq, 2L - 1]: partial[h, r + L - 1]
   int Hq, L;
-  float* out;                    // table gradient [num_buckets, Hq], or slope gradient [Hq]
+  float* out;                    // table gradient [num_buckets, Hq] or [2L - 1, Hq]
   int num_buckets;
 };
 
@@ -270,19 +271,35 @@ __global__ void __launch_bounds__(256) rel_table_grad_kernel(const T5Reduce a) {
   a.out[idx] = a.partial[static_cast<int64_t>(h) * nd + row];
 }
 
-// ALiBi: the bias -m_h |r| is linear in the slope, so
-// out[h] = -sum over r of |r| times the diagonal sum of r; one block per
-// head, a fixed tree over its 256 threads.
-__global__ void __launch_bounds__(256) alibi_slope_grad_kernel(const T5Reduce a) {
-  __shared__ float red[256];
+// ALiBi: the bias -m_h |j - i| is linear in the slope, so its gradient is
+// -sum of |j - i| dS over (b, i, j).  The dQ kernel's moment mode writes
+// that sum per (b, h, query tile, key tile, warp) for the tiles in the
+// mask band; out[h] adds them up, one block per head: thread t takes the
+// entries t, t + 1024, ... in order (entries of tiles outside the band are
+// never written and are skipped), then a fixed tree over the threads.
+struct AlibiMoment {
+  const float* part;             // [B, Hq, nt, nt, 8]
+  float* out;                    // [Hq]
+  int B, Hq, L, nt;
+};
+
+__global__ void __launch_bounds__(1024) alibi_moment_kernel(const AlibiMoment a, const AttnParams p) {
+  __shared__ float red[1024];
   const int h = blockIdx.x;
-  const int nd = 2 * a.L - 1;
-  const float* diag = a.partial + static_cast<int64_t>(h) * nd;  // diag[r + L - 1]
+  const int64_t per_b = static_cast<int64_t>(a.nt) * a.nt * 8;
   float acc = 0.f;
-  for (int dr = static_cast<int>(threadIdx.x); dr < nd; dr += 256)
-    acc += fabsf(static_cast<float>(dr - (a.L - 1))) * diag[dr];
+  for (int64_t e = threadIdx.x; e < a.B * per_b; e += 1024) {
+    const int b = static_cast<int>(e / per_b);
+    const int64_t rem = e - b * per_b;
+    const int mi = static_cast<int>(rem / (a.nt * 8));
+    const int ni = static_cast<int>((rem / 8) % a.nt);
+    int nlo, nhi;
+    key_tile_range(p, a.L, a.L, mi * kTile, kTile, nlo, nhi);
+    if (ni < nlo || ni >= nhi) continue;
+    acc += a.part[(static_cast<int64_t>(b) * a.Hq + h) * per_b + rem];
+  }
   red[threadIdx.x] = acc;
-  for (int w = 128; w > 0; w >>= 1) {
+  for (int w = 512; w > 0; w >>= 1) {
     __syncthreads();
     if (static_cast<int>(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
   }

@@ -566,8 +566,11 @@ __global__ void __launch_bounds__(352, 1)
 // for the dQ MMA of block i.
 // DSM (what the kernel does with the fp32 dS besides the dQ MMA): 0 nothing,
 // 1 store it (dense-bias gradient), 2 store its per-warp sums along the
-// diagonals j - i (T5 / ALiBi gradients), staged through shared memory.
-constexpr int kDsNone = 0, kDsStore = 1, kDsDiag = 2;
+// diagonals j - i, staged through shared memory (relative-position table
+// gradient), 3 the same with one total for a piece of dS whose distances
+// share one T5 bucket (T5 table gradient), 4 store each warp's sum of
+// |j - i| dS (ALiBi slope gradient).
+constexpr int kDsNone = 0, kDsStore = 1, kDsDiag = 2, kDsDiagT5 = 3, kDsMoment = 4;
 
 template <int D, int BIAS, int DSM = kDsNone>
 struct DqLayout {
@@ -581,7 +584,8 @@ struct DqLayout {
   // MMA: the K ring is the deeper one.
   static constexpr int kSK = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : (kBiasTma ? 2 : 4);
   // (at d = 128 the diagonal staging area takes the second V stage)
-  static constexpr int kSV = (D == 128) ? (DSM == kDsDiag ? 1 : 2) : (kBiasTma ? 2 : 3);
+  static constexpr bool kStage = (DSM == kDsDiag || DSM == kDsDiagT5);
+  static constexpr int kSV = (D == 128) ? (kStage ? 1 : 2) : (kBiasTma ? 2 : 3);
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTileBytes;
   static constexpr int kKOff = 2 * kTileBytes;                // K ring
@@ -589,9 +593,9 @@ struct DqLayout {
   static constexpr int kBOff = kVOff + kSV * kTileBytes;      // bias ring (kBiasTma)
   static constexpr int kLutOff = kBOff + kSB * kBiasTileBytes;  // T5 only: 8 warps x 96 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
-  // DSM == 2: per warp, 32 rows x 32 keys of fp32 dS, row stride 33 floats
+  // diagonal sums: per warp, 32 rows x 32 keys of fp32 dS, row stride 33 floats
   static constexpr int kDiagOff = kLutOff + kLutBytes;
-  static constexpr int kDiagBytes = (DSM == kDsDiag) ? 8 * 32 * 33 * 4 : 0;
+  static constexpr int kDiagBytes = kStage ? 8 * 32 * 33 * 4 : 0;
   static constexpr int kBarOff = kDiagOff + kDiagBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
   // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
@@ -1032,7 +1036,23 @@ __global__ void __launch_bounds__(352, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(ds_full(c & 1));
-        if constexpr (DSM == kDsDiag) {
+        if constexpr (DSM == kDsMoment) {
+          // sum over this warp's 32 rows x 64 keys of |j - i| dS (distances
+          // are exact in fp32); one value per (batch, head, query tile, key
+          // tile, warp)
+          const float t0 = static_cast<float>(n0 - i);
+          float mom = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < kBlk; ++cc)
+            mom = fmaf(fabsf(t0 + static_cast<float>(cc)), __uint_as_float(pr[cc]), mom);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mom += __shfl_xor_sync(0xffffffffu, mom, o);
+          const int ntk = (p.Lk + kTile - 1) / kTile;
+          if (lane == 0)
+            p.diag_out[(((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * ntk +
+                        (n0 - c0w) / kTile) * 8 + warp] = mom;
+        }
+        if constexpr (DSM == kDsDiag || DSM == kDsDiagT5) {
           // Sums of this warp's 32 rows x 64 keys of dS along the diagonals,
           // in two halves of 32 keys: each half is staged row by row
           // (stride 33 floats: conflict-free both ways), then lane l adds up
@@ -1047,20 +1067,39 @@ __global__ void __launch_bounds__(352, 1)
           float* dst = p.diag_out +
                        ((((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * ntk +
                          (n0 - c0w) / kTile) * 8 + warp) * 128;
+          // With a T5 table only the sum over each bucket's distances is
+          // used.  A half whose distances t0 - 31 .. t0 + 31 all lie in the
+          // capped bucket of a side, or all at j >= i of a unidirectional
+          // table (bucket 0), needs only its total: it goes to the half's
+          // t = 0 slot and every other slot gets 0, which leaves every
+          // bucket's sum unchanged.  Most halves away from the diagonal are
+          // such.
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            __syncwarp();
-#pragma unroll
-            for (int cc = 0; cc < 32; ++cc) stg[lane * 33 + cc] = __uint_as_float(pr[32 * h + cc]);
-            __syncwarp();
+            const int t0 = n0 + 32 * h - m0 - (warp & 3) * 32;  // distance j - i at t = 0
+            bool one_bucket = false;
+            if constexpr (DSM == kDsDiagT5)
+              one_bucket = t0 + 31 <= p.t5.one_lo_max || t0 - 31 >= p.t5.one_hi_min;
             float s1 = 0.f, s2 = 0.f;
+            if (one_bucket) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const bool first = k <= lane;
-              const int r = first ? 31 - lane + k : k - lane - 1;
-              const float v = stg[r * 33 + k];
-              s1 += first ? v : 0.f;
-              s2 += first ? 0.f : v;
+              for (int cc = 0; cc < 32; ++cc) s1 += __uint_as_float(pr[32 * h + cc]);
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+              s1 = lane == 31 ? s1 : 0.f;
+            } else {
+              __syncwarp();
+#pragma unroll
+              for (int cc = 0; cc < 32; ++cc) stg[lane * 33 + cc] = __uint_as_float(pr[32 * h + cc]);
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                const bool first = k <= lane;
+                const int r = first ? 31 - lane + k : k - lane - 1;
+                const float v = stg[r * 33 + k];
+                s1 += first ? v : 0.f;
+                s2 += first ? 0.f : v;
+              }
             }
             dst[h * 64 + lane] = s1;
             if (lane < 31) dst[h * 64 + 32 + lane] = s2;
@@ -1197,9 +1236,15 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
       }
     }
     if constexpr (BIAS == kBiasT5) {
-      if (p.diag_out) {
+      if (p.diag_out && p.rel_table) {
         kern = bwd_dq_kernel<D, BIAS, kDsDiag>;
         smem_bytes = DqLayout<D, BIAS, kDsDiag>::kSmemAlloc;
+      } else if (p.diag_out && p.alibi) {
+        kern = bwd_dq_kernel<D, BIAS, kDsMoment>;
+        smem_bytes = DqLayout<D, BIAS, kDsMoment>::kSmemAlloc;
+      } else if (p.diag_out) {
+        kern = bwd_dq_kernel<D, BIAS, kDsDiagT5>;
+        smem_bytes = DqLayout<D, BIAS, kDsDiagT5>::kSmemAlloc;
       }
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);

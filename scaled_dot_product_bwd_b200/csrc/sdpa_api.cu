@@ -179,6 +179,10 @@ bool fill_t5(T5Spec& t, int nb, int md, int bidir) {
     t.thr[k] = (n < limit) ? static_cast<int>(n) : INT_MAX;
   }
   for (int k = K; k < kMaxT5Thresholds; ++k) t.thr[k] = INT_MAX;
+  // the capped bucket (half - 1) holds every n >= thr[K - 1]
+  const int sat = t.thr[K - 1];
+  t.one_lo_max = sat == INT_MAX ? INT_MIN : -sat;
+  t.one_hi_min = bidir ? sat : 0;
   return true;
 }
 
@@ -380,10 +384,12 @@ struct BiasGradPlan {
   int chunks = 1;         // pieces of the reduced index
   int64_t per_chunk = 0;  // reduced indices per piece
   size_t part_bytes = 0;  // partial sums of the pieces
-  // T5 / ALiBi: the dQ kernel's per-warp diagonal sums, then per-tile and
-  // per-head diagonal sums (no dS)
+  // T5 / relative-position table: the dQ kernel's per-warp diagonal sums,
+  // then per-tile and per-head diagonal sums (no dS)
   bool diag = false;
   size_t warp_bytes = 0, tile_bytes = 0, band_bytes = 0, diag_bytes = 0;
+  // ALiBi: the dQ kernel's per-warp sums of |j - i| dS
+  bool moment = false;
   size_t total = 0;
 };
 
@@ -431,8 +437,14 @@ sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, Bias
       if (pl.chunks > 1)
         pl.part_bytes = round256(static_cast<size_t>(pl.chunks * n_out * pl.lp) * sizeof(float));
     }
-  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_ALIBI ||
-             bias->kind == SDPA_BIAS_REL) {
+  } else if (bias->kind == SDPA_BIAS_ALIBI) {
+    // per (batch, head, query tile, key tile): 8 per-warp sums
+    const int64_t nt = (L + kTile - 1) / kTile;
+    const double tiles = static_cast<double>(B) * Hq * nt * nt;
+    if (tiles * 8.0 > 1e16) return SDPA_ERR_UNSUPPORTED;
+    pl.moment = true;
+    pl.part_bytes = round256(static_cast<size_t>(B * Hq * nt * nt) * 8 * sizeof(float));
+  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_REL) {
     // per (batch, head, query tile, key tile): 1024 per-warp sums and 256
     // tile diagonals; per head: 2L - 1 diagonal totals
     const int64_t nt = (L + kTile - 1) / kTile;
@@ -630,10 +642,24 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
   bind_bwd(p, g, o, dout, lse, dq, dk, dv, ws);
   const int L = p.Lq;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (pl.moment) {
+    // ALiBi: per-warp sums of |j - i| dS from the dQ kernel, then per head
+    AlibiMoment a;
+    a.part = reinterpret_cast<const float*>(ws + pl.bwd_bytes);
+    a.out = dbias;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.L = L;
+    a.nt = (L + kTile - 1) / kTile;
+    p.diag_out = reinterpret_cast<float*>(ws + pl.bwd_bytes);
+    st = run_bwd(SDPA_BWD_ALL, p, g, q, k, v, dout, cs);
+    if (st != SDPA_OK) return st;
+    alibi_moment_kernel<<<p.Hq, 1024, 0, cs>>>(a, p);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  }
   if (pl.diag) {
-    // T5 / ALiBi / REL: per-warp diagonal sums from the dQ kernel, folded
-    // per tile, per tile offset, then per head, then per bucket (weighed by
-    // -|r| per slope; one per table row)
+    // T5 / REL: per-warp diagonal sums from the dQ kernel, folded per tile,
+    // per tile offset, then per head, then per bucket (one per table row)
     uint8_t* base = ws + pl.bwd_bytes;
     DiagFold f;
     f.warp_part = reinterpret_cast<const float*>(base);
@@ -660,12 +686,10 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.L = L;
     a.partial = f.diag;
     a.out = dbias;
-    a.num_buckets = p.alibi ? 0 : bias->num_buckets;
+    a.num_buckets = bias->num_buckets;
     if (p.rel_table) {
       const int64_t n = static_cast<int64_t>(2 * L - 1) * p.Hq;
       rel_table_grad_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(a);
-    } else if (p.alibi) {
-      alibi_slope_grad_kernel<<<p.Hq, 256, 0, cs>>>(a);
     } else {
       t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
     }

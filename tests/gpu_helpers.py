@@ -15,7 +15,7 @@ LSE_ATOL = 1e-3
 
 def case_inputs(c):
     return make_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], c["d"], seed=c.get("seed", 0),
-                       t5_buckets=32 if c.get("bias") == "t5" else 0,
+                       t5_buckets=c.get("t5_nb", 32) if c.get("bias") == "t5" else 0,
                        dense_bias=c.get("bias") == "dense",
                        bias_shape=c.get("bias_shape"), alibi=c.get("bias") == "alibi",
                        Lk=c.get("Lk"))
@@ -29,6 +29,10 @@ def mask_kw(c):
         kw["scale"] = c["scale"]
     if "t5_bidirectional" in c:
         kw["t5_bidirectional"] = c["t5_bidirectional"]
+    if "t5_nb" in c:
+        kw["t5_num_buckets"] = c["t5_nb"]
+    if "t5_md" in c:
+        kw["t5_max_distance"] = c["t5_md"]
     return kw
 
 

@@ -188,7 +188,7 @@ def test_bias_grad_workspace_size(lib):
     for b in (_dense(L * L, 0, L), _dense(0, L * L, L), _dense(0, 0, L)):
         n = ws(b)
         assert n >= d_bytes + ds_bytes and n % 256 == 0
-    # T5 / ALiBi: no dS; per (batch, head, query tile, key tile) 1024
+    # T5 / REL: no dS; per (batch, head, query tile, key tile) 1024
     # per-warp diagonal sums and 256 tile diagonals, per (batch, head, tile
     # offset) 256 band sums, per head 2L - 1 totals
     r256 = lambda x: (x + 255) // 256 * 256
@@ -198,8 +198,9 @@ def test_bias_grad_workspace_size(lib):
             r256(B * Hq * (2 * nt - 1) * 256 * 4) + r256(Hq * (2 * L - 1) * 4))
     t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
     assert ws(t5) == want
+    # ALiBi: per (batch, head, query tile, key tile) 8 per-warp sums of |j - i| dS
     alibi = binding.BiasDesc(3, 0x10000, 0, 0, 0, 0, 0, 0)
-    assert ws(alibi) == want
+    assert ws(alibi) == d_bytes + r256(tiles * 8 * 4)
     assert ws(binding.BiasDesc(0, None, 0, 0, 0, 0, 0, 0)) == 0       # nothing to differentiate
     assert ws(_dense(L * L, L * L, L)) == 0                          # heads overlap batches
     assert ws(_dense(Hq * L * L, L * L, 0)) == 0                      # one row for all queries

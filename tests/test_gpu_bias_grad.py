@@ -52,6 +52,14 @@ CASES = {
     "t5_bidir_causal_gqa_d128": dict(B=1, Hq=2, Hkv=1, L=270, d=128, causal=True, bias="t5"),
     "t5_unidir_causal_d64": dict(B=2, Hq=2, Hkv=2, L=280, d=64, causal=True, bias="t5",
                                  t5_bidirectional=False),
+    # short max distances: the capped bucket starts at distance 16 (16
+    # buckets, max distance 24) or 14 (8 buckets, max distance 20), so most
+    # 32 x 32 pieces of dS lie in one bucket, on both sides of the diagonal
+    "t5_bidir_short_d64": dict(B=2, Hq=2, Hkv=2, L=330, d=64, bias="t5", t5_nb=16, t5_md=24),
+    "t5_unidir_short_d64": dict(B=1, Hq=2, Hkv=2, L=300, d=64, bias="t5", t5_nb=8, t5_md=20,
+                                t5_bidirectional=False),
+    "t5_unidir_short_causal_d128": dict(B=1, Hq=2, Hkv=1, L=300, d=128, causal=True, bias="t5",
+                                        t5_nb=8, t5_md=20, t5_bidirectional=False),
     # ALiBi slopes: dm_h = -sum |j - i| dS
     "alibi_bidir_d64": dict(B=2, Hq=4, Hkv=4, L=301, d=64, bias="alibi"),
     "alibi_causal_gqa_d128": dict(B=1, Hq=2, Hkv=1, L=270, d=128, causal=True, bias="alibi"),
@@ -118,17 +126,17 @@ def expected_bias_grad(c, inp, dS):
                 q2[h] += np.sum((e[b, h] * (P * dist).sum(axis=1)) ** 2)
         return alibi_slope_gradient(dS), q2
     bidir = c.get("t5_bidirectional", True)
-    nb = 32
+    nb, md = c.get("t5_nb", 32), c.get("t5_md", 128)
     i = np.arange(L)[:, None]
     j = np.arange(L)[None, :]
-    cell = (i * nb + t5_relative_bucket(j - i, nb, 128, bidir)).ravel()
+    cell = (i * nb + t5_relative_bucket(j - i, nb, md, bidir)).ravel()
     q2 = np.zeros((nb, Hq))
     for b in range(B):
         for h in range(Hq):
             P = attention_probs(inp.q, inp.k, b, h, **kw)
             mass = np.bincount(cell, weights=P.ravel(), minlength=L * nb).reshape(L, nb)
             q2[:, h] += np.sum((mass * e[b, h, :, None]) ** 2, axis=0)
-    return t5_table_gradient(dS, nb, 128, bidir), q2
+    return t5_table_gradient(dS, nb, md, bidir), q2
 
 
 def tolerance(ref, q2):
@@ -185,7 +193,7 @@ def test_padded_dense_bias_gradient():
 
 
 @pytest.mark.parametrize("name", ["dense_full_window_d64", "dense_heads_bcast_d64",
-                                  "t5_bidir_d64", "alibi_causal_gqa_d128"])
+                                  "t5_bidir_d64", "t5_bidir_short_d64", "alibi_causal_gqa_d128"])
 def test_bias_grad_bitwise_repeatable(name):
     c = CASES[name]
     inp = case_inputs(c)
