@@ -543,18 +543,15 @@ def visited_tile_pairs(c):
 def bias_grad_extra_bytes(c):
     """HBM bytes the bias gradient adds to the backward.  A dense bias: the
     fp32 dS written once (full shape), or written and read back by the
-    broadcast reduction.  T5: the dQ kernel's per-warp diagonal sums (1024
-    floats per visited tile pair), the per-tile diagonals (256) and the
-    per-tile-offset sums (256 per offset), each written and read back once,
-    then the per-head totals and the result.  ALiBi: the dQ kernel's
+    broadcast reduction.  T5: the dQ kernel's per-bucket sums (8 warps x 32
+    buckets per (batch, head, query tile)) written and read back once, then
+    the result.  ALiBi: the dQ kernel's
     per-warp sums of |j - i| dS (8 floats per visited tile pair) written and
     read back once, then the result."""
     B, H, L = c["B"], c["Hq"], c["L"]
     if c["bias"] == "t5":
-        tiles = B * H * visited_tile_pairs(c)
         nt = (L + 127) // 128
-        return (2 * tiles * (1024 + 256) * 4 + 2 * B * H * (2 * nt - 1) * 256 * 4 +
-                2 * H * (2 * L - 1) * 4 + 32 * H * 4)
+        return 2 * B * H * nt * 8 * 32 * 4 + 32 * H * 4
     if c["bias"] == "alibi":
         tiles = B * H * visited_tile_pairs(c)
         return 2 * tiles * 8 * 4 + H * 4
@@ -565,13 +562,10 @@ def bias_grad_launches(c):
     """Kernels one timed step of the bias-gradient leg launches: the forward,
     preprocess, the dQ kernel (storing dS, its diagonal sums or its |j - i|
     moments) and the dK/dV kernel; a dense bias under a mask adds the zero
-    fill of skipped key tiles; T5 adds the per-tile fold, the
-    per-tile-offset sums, the per-head totals and the per-bucket sums;
-    ALiBi the per-head sum of the moments."""
+    fill of skipped key tiles; T5 adds the per-(bucket, head) sum of the
+    per-bucket sums, ALiBi the per-head sum of the moments."""
     n = 4
-    if c["bias"] == "t5":
-        return n + 4
-    if c["bias"] == "alibi":
+    if c["bias"] in ("t5", "alibi"):
         return n + 1
     if c["causal"] or c["wl"] >= 0 or c["wr"] >= 0:
         n += 1

@@ -314,12 +314,14 @@ sdpa_status_t sdpa_bwd_noalloc(const sdpa_shape* shape, const void* q, const voi
  * workspace: at least sdpa_bwd_bias_grad_workspace_size(shape, bias) bytes,
  * 256-byte aligned, contents ignored on entry.  A broadcast dense bias
  * stages an fp32 copy of dS there (B * Hq * L rows of L floats padded to a
- * multiple of 8) and reduces it; T5 and REL stage no dS: the dQ kernel
- * sums dS along the distances j - i per warp, 1280 floats per (batch, head,
- * query tile, key tile), folded in fixed order; ALiBi neither: the dQ
- * kernel sums |j - i| dS per warp, 8 floats per (batch, head, query tile,
- * key tile).  A full-shape dense bias stages nothing.  dbias must not
- * overlap any other argument.
+ * multiple of 8) and reduces it; T5, ALiBi and REL stage no dS.  T5: the
+ * dQ kernel sums dS per bucket and warp over each query tile's key tiles,
+ * 8 * num_buckets floats per (batch, head, query tile); ALiBi: it sums
+ * |j - i| dS per warp, 8 floats per (batch, head, query tile, key tile);
+ * REL: it sums dS along the distances j - i per warp, 1280 floats per
+ * (batch, head, query tile, key tile), folded in fixed order.  A
+ * full-shape dense bias stages nothing.  dbias must not overlap any other
+ * argument.
  */
 size_t sdpa_bwd_bias_grad_workspace_size(const sdpa_shape* shape, const sdpa_bias_desc* bias);
 sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const void* k,

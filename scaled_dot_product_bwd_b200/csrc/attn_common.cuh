@@ -38,6 +38,13 @@ struct T5Spec {
   int one_lo_max, one_hi_min;
 };
 
+// The contiguous range [lo, hi] of distances r = j - i (within the
+// sequences) that falls in each T5 bucket; hi < lo: bucket unused.
+struct T5Ranges {
+  int lo[128];
+  int hi[128];
+};
+
 __host__ __device__ __forceinline__ int t5_bucket(int rel, const T5Spec& s) {
   int n, off = 0;
   if (s.bidirectional) {
@@ -89,8 +96,9 @@ struct AttnParams {
   // element strides sd_b, sd_h, sd_i (multiples of 4), j contiguous
   float* ds_out;
   int64_t sd_b, sd_h, sd_i;
-  // optional per-warp sums of dS along the diagonals j - i (relative-position
-  // bias gradients); layout in bwd_dq_kernel's diagonal mode
+  // optional per-warp sums of dS along the diagonals j - i, per T5 bucket
+  // or weighted by |j - i| (relative-position bias gradients); layouts in
+  // bwd_dq_kernel's diagonal, bucket and moment modes
   float* diag_out;
   // bias
   int bias_kind;
@@ -98,6 +106,7 @@ struct AttnParams {
   int64_t sb_b, sb_h, sb_i;
   const float* t5_table;       // [num_buckets, Hq]
   T5Spec t5;
+  T5Ranges t5r;                // the T5 table gradient only
   // ALiBi runs in the kBiasT5 kernels: both biases are functions of j - i
   // that the kernels tabulate per tile
   int alibi;                   // 1: bias = -alibi_slopes[h] |j - i| instead of T5

@@ -2,10 +2,11 @@
 // bias's gradient is dS summed over each index the bias is broadcast along
 // (from the fp32 dS the dQ kernel stores in its store mode), a T5 table
 // entry's gradient is dS summed over every (b, i, j) whose distance j - i
-// falls in its bucket and a relative-position table row's over its distance
-// (both from the per-warp diagonal sums of dS the dQ kernel writes in its
-// diagonal modes), and an ALiBi slope's is minus the sum of |j - i| dS (from
-// the per-warp sums of its moment mode; catie-aq/flashT5 README, "Full attention biases" and
+// falls in its bucket (from the per-bucket sums the dQ kernel writes in its
+// bucket mode), a relative-position table row's over its distance (from the
+// per-warp diagonal sums of its diagonal mode), and an ALiBi slope's is
+// minus the sum of |j - i| dS (from the per-warp sums of its moment mode;
+// catie-aq/flashT5 README, "Full attention biases" and
 // "T5-like relative position encoding biases": a learnable bias needs these
 // to train).
 //
@@ -137,22 +138,12 @@ __global__ void __launch_bounds__(256) dense_bias_combine_kernel(const DenseRedu
 }
 
 // ---------------------------------------------------------------------
-// T5 table (and relative-position table) gradient.  The bias depends on
-// j - i alone, so first sum dS along each diagonal r = j - i (r in
-// [-(L-1), L-1]), then add up the diagonals of each bucket.  Every
-// bucket covers one contiguous range of r (the bucket is monotone in |r| on
-// each side of 0, and the two sides use disjoint ids when bidirectional),
-// given to the last kernel as [lo, hi].
+// Relative-position table gradient.  The bias depends on j - i alone, so
+// sum dS along each diagonal r = j - i (r in [-(L-1), L-1]).
 struct T5Reduce {
   const float* partial;          // diagonal sums [Hq, 2L - 1]: partial[h, r + L - 1]
   int Hq, L;
-  float* out;                    // table gradient [num_buckets, Hq] or [2L - 1, Hq]
-  int num_buckets;
-};
-
-struct T5Ranges {
-  int lo[128];                   // first r of bucket k (r = j - i)
-  int hi[128];                   // last r of bucket k; hi < lo: bucket unused
+  float* out;                    // table gradient [2L - 1, Hq]
 };
 
 // ---------------------------------------------------------------------
@@ -243,16 +234,27 @@ __global__ void __launch_bounds__(128) diag_total_kernel(const DiagFold a) {
   a.diag[static_cast<int64_t>(h) * nd + dr] = acc;
 }
 
-// out[k, h] = sum of the diagonal sums over bucket k's range of r: one block
-// per (k, h), a fixed tree over its 256 threads.
-__global__ void __launch_bounds__(256) t5_bucket_sum_kernel(const T5Reduce a, const T5Ranges rg) {
+// T5: out[k, h] = sum over (b, query tile, warp) of the dQ kernel's per-bucket
+// partial sums (its bucket mode: per (b, h, query tile, warp) one sum per
+// bucket over every key tile); one block per (k, h), thread t adds the
+// entries t, t + 256, ... in order, then a fixed tree over the threads.
+struct T5BucketReduce {
+  const float* part;             // [B, Hq, nqt, 8, num_buckets]
+  float* out;                    // [num_buckets, Hq]
+  int B, Hq, nqt, num_buckets;
+};
+
+__global__ void __launch_bounds__(256) t5_bucket_reduce_kernel(const T5BucketReduce a) {
   __shared__ float red[256];
   const int k = blockIdx.x;
   const int h = blockIdx.y;
-  const int nd = 2 * a.L - 1;
-  const float* diag = a.partial + static_cast<int64_t>(h) * nd + (a.L - 1);  // diag[r]
+  const int per_b = a.nqt * 8;
   float acc = 0.f;
-  for (int r = rg.lo[k] + static_cast<int>(threadIdx.x); r <= rg.hi[k]; r += 256) acc += diag[r];
+  for (int e = static_cast<int>(threadIdx.x); e < a.B * per_b; e += 256) {
+    const int b = e / per_b;
+    const int rem = e - b * per_b;  // query tile * 8 + warp
+    acc += a.part[((static_cast<int64_t>(b) * a.Hq + h) * per_b + rem) * a.num_buckets + k];
+  }
   red[threadIdx.x] = acc;
   for (int w = 128; w > 0; w >>= 1) {
     __syncthreads();

@@ -567,9 +567,9 @@ __global__ void __launch_bounds__(352, 1)
 // DSM (what the kernel does with the fp32 dS besides the dQ MMA): 0 nothing,
 // 1 store it (dense-bias gradient), 2 store its per-warp sums along the
 // diagonals j - i, staged through shared memory (relative-position table
-// gradient), 3 the same with one total for a piece of dS whose distances
-// share one T5 bucket (T5 table gradient), 4 store each warp's sum of
-// |j - i| dS (ALiBi slope gradient).
+// gradient), 3 add those sums up per T5 bucket over the work item and store
+// one sum per bucket and warp (T5 table gradient), 4 store each warp's sum
+// of |j - i| dS (ALiBi slope gradient).
 constexpr int kDsNone = 0, kDsStore = 1, kDsDiag = 2, kDsDiagT5 = 3, kDsMoment = 4;
 
 template <int D, int BIAS, int DSM = kDsNone>
@@ -596,7 +596,10 @@ struct DqLayout {
   // diagonal sums: per warp, 32 rows x 32 keys of fp32 dS, row stride 33 floats
   static constexpr int kDiagOff = kLutOff + kLutBytes;
   static constexpr int kDiagBytes = kStage ? 8 * 32 * 33 * 4 : 0;
-  static constexpr int kBarOff = kDiagOff + kDiagBytes;
+  // bucket mode: per warp, 128 per-bucket sums
+  static constexpr int kBAccOff = kDiagOff + kDiagBytes;
+  static constexpr int kBAccBytes = (DSM == kDsDiagT5) ? 8 * 128 * 4 : 0;
+  static constexpr int kBarOff = kBAccOff + kBAccBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
   // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
   // b_full[2], b_empty[2]
@@ -896,6 +899,11 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
+    if constexpr (DSM == kDsDiagT5) {
+      // this warp's per-bucket sums; entry k is only ever touched by lane k % 32
+      float* bacc = reinterpret_cast<float*>(smem + Lay::kBAccOff) + warp * 128;
+      for (int k = lane; k < 128; k += 32) bacc[k] = 0.f;
+    }
     bool ok = true;
     int c = 0;  // key blocks so far, over all items
     int u = 0;  // items with a non-empty band so far
@@ -916,6 +924,9 @@ __global__ void __launch_bounds__(352, 1)
       if constexpr (BIAS == kBiasDense)
         brow = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
                static_cast<int64_t>(min(i, Lq - 1)) * p.sb_i;
+      // bucket mode: this row's sums of the halves inside the capped bucket
+      // of keys before / after the query (or bucket 0 of a unidirectional table)
+      float one_lo = 0.f, one_hi = 0.f;
       for (int it = 0; it < nt; ++it, ++c) {
         const int x = c & 1;
         const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup
@@ -1041,10 +1052,11 @@ __global__ void __launch_bounds__(352, 1)
           // are exact in fp32); one value per (batch, head, query tile, key
           // tile, warp)
           const float t0 = static_cast<float>(n0 - i);
-          float mom = 0.f;
+          float m4[4] = {0.f, 0.f, 0.f, 0.f};  // four chains: columns c % 4
 #pragma unroll
           for (int cc = 0; cc < kBlk; ++cc)
-            mom = fmaf(fabsf(t0 + static_cast<float>(cc)), __uint_as_float(pr[cc]), mom);
+            m4[cc & 3] = fmaf(fabsf(t0 + static_cast<float>(cc)), __uint_as_float(pr[cc]), m4[cc & 3]);
+          float mom = (m4[0] + m4[1]) + (m4[2] + m4[3]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mom += __shfl_xor_sync(0xffffffffu, mom, o);
           const int ntk = (p.Lk + kTile - 1) / kTile;
@@ -1059,21 +1071,20 @@ __global__ void __launch_bounds__(352, 1)
           // the diagonal t = c - r = l - 31 (rows 31 - l..31) and, for
           // l < 31, t = l + 1 (rows 0..30 - l), one element per step, so a
           // step's 32 reads hit 32 banks.  In absolute terms t is the
-          // distance j - i = n0 + 32 h - (m0 + 32 (warp % 4)) + t.  Per
-          // (batch, head, query tile, key tile): 8 warps x 2 halves x 64
-          // floats (t + 31 at 0..62 for t <= 0, 32 + t - 1 for t >= 1).
+          // distance j - i = n0 + 32 h - (m0 + 32 (warp % 4)) + t.
+          // Diagonal mode: per (batch, head, query tile, key tile), 8 warps
+          // x 2 halves x 64 floats (t + 31 at 0..62 for t <= 0, 32 + t - 1
+          // for t >= 1).  Bucket mode (T5 table): the 63 sums go to this
+          // warp's per-bucket accumulators in shared memory instead, lane k
+          // adding those of bucket k (and k + 32, ...), whose distances form
+          // one range [t5r.lo[k], t5r.hi[k]], as a difference of two prefix
+          // sums over the half's diagonals; a half whose distances all lie
+          // in the capped bucket of a side, or all at j >= i of a
+          // unidirectional table (bucket 0), skips the staging: each row
+          // adds its 32 values to a register sum for that bucket, which the
+          // warp reduces once per work item (most halves away from the
+          // diagonal are such).
           float* stg = reinterpret_cast<float*>(smem + Lay::kDiagOff) + warp * (32 * 33);
-          const int ntk = (p.Lk + kTile - 1) / kTile;
-          float* dst = p.diag_out +
-                       ((((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * ntk +
-                         (n0 - c0w) / kTile) * 8 + warp) * 128;
-          // With a T5 table only the sum over each bucket's distances is
-          // used.  A half whose distances t0 - 31 .. t0 + 31 all lie in the
-          // capped bucket of a side, or all at j >= i of a unidirectional
-          // table (bucket 0), needs only its total: it goes to the half's
-          // t = 0 slot and every other slot gets 0, which leaves every
-          // bucket's sum unchanged.  Most halves away from the diagonal are
-          // such.
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int t0 = n0 + 32 * h - m0 - (warp & 3) * 32;  // distance j - i at t = 0
@@ -1082,27 +1093,78 @@ __global__ void __launch_bounds__(352, 1)
               one_bucket = t0 + 31 <= p.t5.one_lo_max || t0 - 31 >= p.t5.one_hi_min;
             float s1 = 0.f, s2 = 0.f;
             if (one_bucket) {
+              // the row's 32 values as a pairwise tree, into the side's
+              // register sum (reduced over the warp once per item)
+              float v[16];
 #pragma unroll
-              for (int cc = 0; cc < 32; ++cc) s1 += __uint_as_float(pr[32 * h + cc]);
+              for (int q = 0; q < 16; ++q)
+                v[q] = __uint_as_float(pr[32 * h + 2 * q]) + __uint_as_float(pr[32 * h + 2 * q + 1]);
 #pragma unroll
-              for (int o = 16; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-              s1 = lane == 31 ? s1 : 0.f;
+              for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+                for (int q = 0; q < w2; ++q) v[q] = v[2 * q] + v[2 * q + 1];
+              if (t0 + 31 <= p.t5.one_lo_max)
+                one_lo += v[0];
+              else
+                one_hi += v[0];
+              continue;
             } else {
               __syncwarp();
 #pragma unroll
               for (int cc = 0; cc < 32; ++cc) stg[lane * 33 + cc] = __uint_as_float(pr[32 * h + cc]);
               __syncwarp();
+              // two chains per sum (even and odd steps), added at the end
+              float s1b = 0.f, s2b = 0.f;
 #pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                const bool first = k <= lane;
-                const int r = first ? 31 - lane + k : k - lane - 1;
-                const float v = stg[r * 33 + k];
-                s1 += first ? v : 0.f;
-                s2 += first ? 0.f : v;
+              for (int k = 0; k < 32; k += 2) {
+                const bool f0 = k <= lane, f1 = k + 1 <= lane;
+                const float v0 = stg[(f0 ? 31 - lane + k : k - lane - 1) * 33 + k];
+                const float v1 = stg[(f1 ? 32 - lane + k : k - lane) * 33 + k + 1];
+                s1 += f0 ? v0 : 0.f;
+                s2 += f0 ? 0.f : v0;
+                s1b += f1 ? v1 : 0.f;
+                s2b += f1 ? 0.f : v1;
+              }
+              s1 += s1b;
+              s2 += s2b;
+            }
+            if constexpr (DSM == kDsDiag) {
+              const int ntk = (p.Lk + kTile - 1) / kTile;
+              float* dst = p.diag_out +
+                           ((((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * ntk +
+                             (n0 - c0w) / kTile) * 8 + warp) * 128;
+              dst[h * 64 + lane] = s1;
+              if (lane < 31) dst[h * 64 + 32 + lane] = s2;
+            } else {
+              float* bacc = reinterpret_cast<float*>(smem + Lay::kBAccOff) + warp * 128;
+              {
+                // prefix sums over t = -31 .. 31 (s1 of lanes 0..31, then s2
+                // of lanes 0..30) at index t + 32 (index 0: the empty
+                // prefix); a bucket's sum is the difference of two of them
+                float a = s1, e = lane < 31 ? s2 : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                  const float xa = __shfl_up_sync(0xffffffffu, a, o);
+                  const float xe = __shfl_up_sync(0xffffffffu, e, o);
+                  if (lane >= o) {
+                    a += xa;
+                    e += xe;
+                  }
+                }
+                e += __shfl_sync(0xffffffffu, a, 31);
+                __syncwarp();
+                stg[lane + 1] = a;
+                if (lane < 31) stg[lane + 33] = e;
+                if (lane == 0) stg[0] = 0.f;
+                __syncwarp();
+                const int nbk = p.t5.bidirectional ? 2 * p.t5.half : p.t5.half;
+                for (int k = lane; k < nbk; k += 32) {
+                  const int lo = max(p.t5r.lo[k] - t0, -31);
+                  const int hi = min(p.t5r.hi[k] - t0, 31);
+                  if (lo <= hi) bacc[k] += stg[hi + 32] - stg[lo + 31];
+                }
               }
             }
-            dst[h * 64 + lane] = s1;
-            if (lane < 31) dst[h * 64 + 32 + lane] = s2;
           }
         }
         if constexpr (DSM == kDsStore) {
@@ -1146,6 +1208,27 @@ __global__ void __launch_bounds__(352, 1)
             for (int e = 0; e < kBlk; ++e)
               if (n0 + e < Lk) __stcs(dst + e, __uint_as_float(pr[e]));
           }
+        }
+      }
+      if constexpr (DSM == kDsDiagT5) {
+        // this warp's per-bucket sums over the item's key tiles, at
+        // [b, hq, query tile, warp, bucket]; the accumulators restart at 0
+        const int nbk = p.t5.bidirectional ? 2 * p.t5.half : p.t5.half;
+        float* bacc = reinterpret_cast<float*>(smem + Lay::kBAccOff) + warp * 128;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          one_lo += __shfl_xor_sync(0xffffffffu, one_lo, o);
+          one_hi += __shfl_xor_sync(0xffffffffu, one_hi, o);
+        }
+        const int k_lo = p.t5.half - 1;
+        const int k_hi = p.t5.bidirectional ? 2 * p.t5.half - 1 : 0;
+        if (lane == (k_lo & 31)) bacc[k_lo] += one_lo;
+        if (lane == (k_hi & 31)) bacc[k_hi] += one_hi;
+        float* dstb = p.diag_out +
+                      (((static_cast<int64_t>(b) * p.Hq + hq) * nqt + m0 / kTile) * 8 + warp) * nbk;
+        for (int k = lane; k < nbk; k += 32) {
+          dstb[k] = bacc[k];
+          bacc[k] = 0.f;
         }
       }
       // ----------- epilogue: warpgroup wg stores dQ columns [wg D/2, (wg+1) D/2) -----------

@@ -384,9 +384,11 @@ struct BiasGradPlan {
   int chunks = 1;         // pieces of the reduced index
   int64_t per_chunk = 0;  // reduced indices per piece
   size_t part_bytes = 0;  // partial sums of the pieces
-  // T5 / relative-position table: the dQ kernel's per-warp diagonal sums,
-  // then per-tile and per-head diagonal sums (no dS)
+  // relative-position table: the dQ kernel's per-warp diagonal sums, then
+  // per-tile and per-head diagonal sums (no dS)
   bool diag = false;
+  // T5 table: the dQ kernel's per-bucket sums per (batch, head, query tile, warp)
+  bool buckets = false;
   size_t warp_bytes = 0, tile_bytes = 0, band_bytes = 0, diag_bytes = 0;
   // ALiBi: the dQ kernel's per-warp sums of |j - i| dS
   bool moment = false;
@@ -444,7 +446,15 @@ sdpa_status_t plan_bias_grad(const Geometry& g, const sdpa_bias_desc* bias, Bias
     if (tiles * 8.0 > 1e16) return SDPA_ERR_UNSUPPORTED;
     pl.moment = true;
     pl.part_bytes = round256(static_cast<size_t>(B * Hq * nt * nt) * 8 * sizeof(float));
-  } else if (bias->kind == SDPA_BIAS_T5 || bias->kind == SDPA_BIAS_REL) {
+  } else if (bias->kind == SDPA_BIAS_T5) {
+    const int64_t nt = (L + kTile - 1) / kTile;
+    const int64_t nb = bias->num_buckets;
+    if (nb < 1 || nb > 128) return SDPA_ERR_INVALID_ARG;
+    if (static_cast<double>(B) * Hq * nt * 8 * nb > 1e15 || B * nt * 8 > (1ll << 30))
+      return SDPA_ERR_UNSUPPORTED;
+    pl.buckets = true;
+    pl.part_bytes = round256(static_cast<size_t>(B * Hq * nt * 8 * nb) * sizeof(float));
+  } else if (bias->kind == SDPA_BIAS_REL) {
     // per (batch, head, query tile, key tile): 1024 per-warp sums and 256
     // tile diagonals; per head: 2L - 1 diagonal totals
     const int64_t nt = (L + kTile - 1) / kTile;
@@ -657,9 +667,26 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     alibi_moment_kernel<<<p.Hq, 1024, 0, cs>>>(a, p);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
   }
+  if (pl.buckets) {
+    // T5: per-bucket sums per (batch, head, query tile, warp) from the dQ
+    // kernel, then per (bucket, head)
+    p.t5r = rg;
+    p.diag_out = reinterpret_cast<float*>(ws + pl.bwd_bytes);
+    st = run_bwd(SDPA_BWD_ALL, p, g, q, k, v, dout, cs);
+    if (st != SDPA_OK) return st;
+    T5BucketReduce a;
+    a.part = p.diag_out;
+    a.out = dbias;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.nqt = (L + kTile - 1) / kTile;
+    a.num_buckets = bias->num_buckets;
+    t5_bucket_reduce_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  }
   if (pl.diag) {
-    // T5 / REL: per-warp diagonal sums from the dQ kernel, folded per tile,
-    // per tile offset, then per head, then per bucket (one per table row)
+    // REL: per-warp diagonal sums from the dQ kernel, folded per tile, per
+    // tile offset, then per head, then transposed into the table's layout
     uint8_t* base = ws + pl.bwd_bytes;
     DiagFold f;
     f.warp_part = reinterpret_cast<const float*>(base);
@@ -686,13 +713,8 @@ sdpa_status_t sdpa_bwd_bias_grad(const sdpa_shape* shape, const void* q, const v
     a.L = L;
     a.partial = f.diag;
     a.out = dbias;
-    a.num_buckets = bias->num_buckets;
-    if (p.rel_table) {
-      const int64_t n = static_cast<int64_t>(2 * L - 1) * p.Hq;
-      rel_table_grad_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(a);
-    } else {
-      t5_bucket_sum_kernel<<<dim3(a.num_buckets, p.Hq), 256, 0, cs>>>(a, rg);
-    }
+    const int64_t n = static_cast<int64_t>(2 * L - 1) * p.Hq;
+    rel_table_grad_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(a);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
   }
   if (pl.ds_ws) {

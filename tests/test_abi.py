@@ -188,16 +188,19 @@ def test_bias_grad_workspace_size(lib):
     for b in (_dense(L * L, 0, L), _dense(0, L * L, L), _dense(0, 0, L)):
         n = ws(b)
         assert n >= d_bytes + ds_bytes and n % 256 == 0
-    # T5 / REL: no dS; per (batch, head, query tile, key tile) 1024
-    # per-warp diagonal sums and 256 tile diagonals, per (batch, head, tile
-    # offset) 256 band sums, per head 2L - 1 totals
+    # T5: no dS; per (batch, head, query tile) 8 warps x 32 per-bucket sums
     r256 = lambda x: (x + 255) // 256 * 256
     nt = (L + 127) // 128
     tiles = B * Hq * nt * nt
+    t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
+    assert ws(t5) == d_bytes + r256(B * Hq * nt * 8 * 32 * 4)
+    # REL: no dS; per (batch, head, query tile, key tile) 1024 per-warp
+    # diagonal sums and 256 tile diagonals, per (batch, head, tile offset)
+    # 256 band sums, per head 2L - 1 totals
     want = (d_bytes + r256(tiles * 1024 * 4) + r256(tiles * 256 * 4) +
             r256(B * Hq * (2 * nt - 1) * 256 * 4) + r256(Hq * (2 * L - 1) * 4))
-    t5 = binding.BiasDesc(2, 0x10000, 0, 0, 0, 32, 128, 1)
-    assert ws(t5) == want
+    rel = binding.BiasDesc(4, 0x10000, 0, 0, 0, 0, 0, 0)
+    assert ws(rel) == want
     # ALiBi: per (batch, head, query tile, key tile) 8 per-warp sums of |j - i| dS
     alibi = binding.BiasDesc(3, 0x10000, 0, 0, 0, 0, 0, 0)
     assert ws(alibi) == d_bytes + r256(tiles * 8 * 4)
