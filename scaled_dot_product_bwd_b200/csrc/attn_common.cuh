@@ -184,6 +184,19 @@ __device__ __forceinline__ constexpr bool emu_exp2(int c) {
   return BIAS != kBiasDense && (c & 7) >= MUFU_PER8;
 }
 
+// 2^x of columns c and c + 1, each on the unit emu_exp2 gives it; a pair
+// that both go to the FMA pipe takes the packed form (identical results).
+template <int BIAS, int MUFU_PER8>
+__device__ __forceinline__ void exp2_pair(int c, float x0, float x1, float& y0, float& y1) {
+  const bool f0 = emu_exp2<BIAS, MUFU_PER8>(c), f1 = emu_exp2<BIAS, MUFU_PER8>(c + 1);
+  if (f0 && f1) {
+    exp2_fma2(x0, x1, y0, y1);
+  } else {
+    y0 = f0 ? exp2_fma(x0) : fast_exp2(x0);
+    y1 = f1 ? exp2_fma(x1) : fast_exp2(x1);
+  }
+}
+
 // Key tiles [nlo, nhi) that hold any key visible from query rows
 // [m0, m0 + rows) (clipped to Lq), keys clipped to Lk.  Empty when nhi <= nlo.
 // Positions of both sequences count from 0.

@@ -119,7 +119,7 @@ struct DkdvLayout {
   static constexpr int kVOff = kTileBytes;
   static constexpr int kQOff = 2 * kTileBytes;                  // Q ring
   static constexpr int kDOOff = kQOff + kSQ * kTileBytes;       // dO ring
-  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;     // 2 x (lse2[128], D[128])
+  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;     // 2 x (-lse2[128], D[128])
   static constexpr int kLutOff = kVecOff + 2 * 2 * kTile * 4;   // T5 only: 8 warps x 96 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(352, 1)
           tma_load_4d(sb + Lay::kVOff + h * kTile * 128, &tmV, kv_full, h * 64, s.k0 + n0, g, s.bc);
         }
       }
-      // LSE (log2 units) and D of one block's 128 queries, four per lane,
+      // -LSE (log2 units) and D of one block's 128 queries, four per lane,
       // loaded one block ahead of the slot they go to.
       float l2v[4], ddv[4];
       auto load_vec = [&](int it) {
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(352, 1)
         float* lse2 = vec + x * 2 * kTile;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          lse2[lane + 32 * e] = l2v[e];
+          lse2[lane + 32 * e] = -l2v[e];
           lse2[kTile + lane + 32 * e] = ddv[e];
         }
         mbar_arrive(vec_full(x));
@@ -434,36 +434,50 @@ __global__ void __launch_bounds__(352, 1)
       const float* dvv = vec + x * 2 * kTile + kTile + c0w;
       uint32_t pr[64];  // S^T row, then P^T (fp32 bits)
       tmem_ld64_sync(tS, pr);
-      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+      // in pairs of columns: packed fp32 pair instructions for the affine
+      // step and the FMA-pipe exponentials (rounded as the scalar ones)
+      const float4* lse4 = reinterpret_cast<const float4*>(lse2);  // -LSE, log2 units
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
       if (full) {
 #pragma unroll
         for (int c4 = 0; c4 < kBlk / 4; ++c4) {
           const float4 l = lse4[c4];
-          const float lv[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {
             const int c = 4 * c4 + e;
-            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
-            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            uint64_t x2 = f2_fma(f2_pack(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1])), sc2,
+                                 e ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y));
+            if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[-c], lut_row[-c - 1]));
             if constexpr (BIAS == kBiasDense)
-              xv = fmaf(bcol[static_cast<int64_t>(c) * p.sb_i], kLog2e, xv);
-            pr[c] = __float_as_uint(emu_exp2<BIAS, kDkdvMufuPer8>(c) ? exp2_fma(xv) : fast_exp2(xv));
+              x2 = f2_fma(f2_pack(bcol[static_cast<int64_t>(c) * p.sb_i],
+                                  bcol[static_cast<int64_t>(c + 1) * p.sb_i]),
+                          f2_pack(kLog2e, kLog2e), x2);
+            float x0, x1, y0, y1;
+            f2_unpack(x2, x0, x1);
+            exp2_pair<BIAS, kDkdvMufuPer8>(c, x0, x1, y0, y1);
+            pr[c] = __float_as_uint(y0);
+            pr[c + 1] = __float_as_uint(y1);
           }
         }
       } else {
 #pragma unroll
         for (int c4 = 0; c4 < kBlk / 4; ++c4) {
           const float4 l = lse4[c4];
-          const float lv[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {
             const int c = 4 * c4 + e;
-            const bool vis = (c >= lo) && (c <= hi);
-            float xv = fmaf(__uint_as_float(pr[c]), p.scale_log2, -lv[e]);
-            if constexpr (BIAS == kBiasT5) xv += lut_row[-c];
+            const bool v0 = (c >= lo) && (c <= hi), v1 = (c + 1 >= lo) && (c + 1 <= hi);
+            uint64_t x2 = f2_fma(f2_pack(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1])), sc2,
+                                 e ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y));
+            if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[-c], lut_row[-c - 1]));
             if constexpr (BIAS == kBiasDense)
-              xv = fmaf(bcol[static_cast<int64_t>(vis ? c : 0) * p.sb_i], kLog2e, xv);
-            pr[c] = __float_as_uint(fast_exp2(vis ? xv : -INFINITY));
+              x2 = f2_fma(f2_pack(bcol[static_cast<int64_t>(v0 ? c : 0) * p.sb_i],
+                                  bcol[static_cast<int64_t>(v1 ? c + 1 : 0) * p.sb_i]),
+                          f2_pack(kLog2e, kLog2e), x2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            pr[c] = __float_as_uint(fast_exp2(v0 ? x0 : -INFINITY));
+            pr[c + 1] = __float_as_uint(fast_exp2(v1 ? x1 : -INFINITY));
           }
         }
       }
@@ -491,10 +505,16 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const float4 dv4 = d4v[c >> 2];
-          const float d0 = __uint_as_float(pr[cc + c]) * (__uint_as_float(dr[c]) - dv4.x);
-          const float d1 = __uint_as_float(pr[cc + c + 1]) * (__uint_as_float(dr[c + 1]) - dv4.y);
-          const float d2 = __uint_as_float(pr[cc + c + 2]) * (__uint_as_float(dr[c + 2]) - dv4.z);
-          const float d3 = __uint_as_float(pr[cc + c + 3]) * (__uint_as_float(dr[c + 3]) - dv4.w);
+          // dS = P (dP - D), two columns per instruction
+          const uint64_t a2 = f2_mul(
+              f2_pack(__uint_as_float(pr[cc + c]), __uint_as_float(pr[cc + c + 1])),
+              f2_sub(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), f2_pack(dv4.x, dv4.y)));
+          const uint64_t b2 = f2_mul(
+              f2_pack(__uint_as_float(pr[cc + c + 2]), __uint_as_float(pr[cc + c + 3])),
+              f2_sub(f2_pack(__uint_as_float(dr[c + 2]), __uint_as_float(dr[c + 3])), f2_pack(dv4.z, dv4.w)));
+          float d0, d1, d2, d3;
+          f2_unpack(a2, d0, d1);
+          f2_unpack(b2, d2, d3);
           pk[c >> 1] = pack_bf16x2(d0, d1);
           pk[(c >> 1) + 1] = pack_bf16x2(d2, d3);
         }
@@ -1001,11 +1021,19 @@ __global__ void __launch_bounds__(352, 1)
             }
           }
         } else if (full) {
+          // in pairs of columns: packed fp32 pair instructions for the
+          // affine step and the FMA-pipe exponentials (rounded as the scalar ones)
+          const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nl2 = f2_pack(-l2, -l2);
 #pragma unroll
-          for (int cc = 0; cc < kBlk; ++cc) {
-            float xv = fmaf(__uint_as_float(pr[cc]), p.scale_log2, -l2);
-            if constexpr (BIAS == kBiasT5) xv += lut_row[cc];
-            pr[cc] = __float_as_uint(emu_exp2<BIAS, kDqMufuPer8>(cc) ? exp2_fma(xv) : fast_exp2(xv));
+          for (int cc = 0; cc < kBlk; cc += 2) {
+            uint64_t x2 = f2_fma(f2_pack(__uint_as_float(pr[cc]), __uint_as_float(pr[cc + 1])), sc2, nl2);
+            if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[cc], lut_row[cc + 1]));
+            float x0, x1, y0, y1;
+            f2_unpack(x2, x0, x1);
+            exp2_pair<BIAS, kDqMufuPer8>(cc, x0, x1, y0, y1);
+            pr[cc] = __float_as_uint(y0);
+            pr[cc + 1] = __float_as_uint(y1);
           }
         } else {
 #pragma unroll
@@ -1032,8 +1060,12 @@ __global__ void __launch_bounds__(352, 1)
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float d0 = __uint_as_float(pr[cc + e]) * (__uint_as_float(dr[e]) - dd);
-            const float d1 = __uint_as_float(pr[cc + e + 1]) * (__uint_as_float(dr[e + 1]) - dd);
+            // dS = P (dP - D), two columns per instruction
+            const uint64_t d2 = f2_mul(
+                f2_pack(__uint_as_float(pr[cc + e]), __uint_as_float(pr[cc + e + 1])),
+                f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(dd, dd)));
+            float d0, d1;
+            f2_unpack(d2, d0, d1);
             pk[(cc + e) >> 1] = pack_bf16x2(d0, d1);
             if constexpr (DSM != kDsNone) {  // P is spent: keep the fp32 dS in its place
               pr[cc + e] = __float_as_uint(d0);

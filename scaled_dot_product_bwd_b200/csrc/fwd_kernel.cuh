@@ -495,10 +495,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int c = 0; c < 32; c += 2) {
               const uint64_t arg = f2_fma(
                   f2_pack(__uint_as_float(xs[c0 + c]), __uint_as_float(xs[c0 + c + 1])), c2, nm2);
-              float v0, v1;
+              float v0, v1, e0, e1;
               f2_unpack(arg, v0, v1);
-              const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
-              const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
+              exp2_pair<BIAS, kFwdMufuPer8>(c0 + c, v0, v1, e0, e1);
               acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(e0, e1));
               pk[c >> 1] = pack_bf16x2(e0, e1);
             }
@@ -521,8 +520,8 @@ __global__ void __launch_bounds__(384, 1)
               for (int c = 0; c < 32; c += 2) {
                 const float v0 = __uint_as_float(xs[c0 + c]) - m_sub;
                 const float v1 = __uint_as_float(xs[c0 + c + 1]) - m_sub;
-                const float e0 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c) ? exp2_fma(v0) : fast_exp2(v0);
-                const float e1 = emu_exp2<BIAS, kFwdMufuPer8>(c0 + c + 1) ? exp2_fma(v1) : fast_exp2(v1);
+                float e0, e1;
+                exp2_pair<BIAS, kFwdMufuPer8>(c0 + c, v0, v1, e0, e1);
                 sm[(c >> 1) & 3] += e0 + e1;
                 pk[c >> 1] = pack_bf16x2(e0, e1);
               }
