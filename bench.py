@@ -69,12 +69,12 @@ for _hkv, _tag in ((32, "mha"), (8, "gqa"), (1, "mqa")):
 # only while the library is built from exactly those sources.
 NCU_TRAFFIC = {
     # mistral4k_small (batch 2) capture, profiles/mistral4k_small_full_capture.md
-    ("mistral4k", "fwd"): {"bytes_per_batch": (100857088 + 37563136) / 2,
-        "source_hash": "eb1916b5659d374fedf09ed85336d41e2fcb78d24438cb38725bc99624eb0ebc"},
-    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171746048 + 44120832) / 2,
-        "source_hash": "eb1916b5659d374fedf09ed85336d41e2fcb78d24438cb38725bc99624eb0ebc"},
-    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170164224 + 23726080) / 2,
-        "source_hash": "eb1916b5659d374fedf09ed85336d41e2fcb78d24438cb38725bc99624eb0ebc"},
+    ("mistral4k", "fwd"): {"bytes_per_batch": (100943872 + 36961024) / 2,
+        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
+    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171795200 + 45393152) / 2,
+        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
+    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170254848 + 23896064) / 2,
+        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
 }
 
 
