@@ -236,8 +236,11 @@ __global__ void __launch_bounds__(352, 1)
           tma_load_4d(sb + Lay::kVOff + h * kTile * 128, &tmV, kv_full, h * 64, s.k0 + n0, g, s.bc);
         }
       }
-      // -LSE (log2 units) and D of one block's 128 queries, four per lane,
-      // loaded one block ahead of the slot they go to.
+      // LSE and D of one block's 128 queries, four per lane, loaded one
+      // block ahead of the slot they go to.  Nothing here uses the loaded
+      // values (a use would hold the warp until they arrive): they are
+      // converted where they are written, after the next block's copies
+      // have been issued.
       float l2v[4], ddv[4];
       auto load_vec = [&](int it) {
         const int hq = g * p.G + it / nm;
@@ -245,13 +248,12 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = m0 + lane + 32 * e;
-          l2v[e] = INFINITY;  // queries past the sequence: P = 0
+          l2v[e] = -INFINITY;  // queries past the sequence: P = 0
           ddv[e] = 0.f;
           if (i < Lq) {
             const int64_t idx = row_index(p, s, b, hq, i);
-            l2v[e] = p.lse[idx] * kLog2e;
+            l2v[e] = p.lse[idx];
             ddv[e] = p.dvec[idx];
-            if (l2v[e] == -INFINITY) l2v[e] = INFINITY;  // row with no visible key
           }
         }
       };
@@ -293,7 +295,9 @@ __global__ void __launch_bounds__(352, 1)
         float* lse2 = vec + x * 2 * kTile;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          lse2[lane + 32 * e] = -l2v[e];
+          // -LSE in log2 units; -inf (a row with no visible key, or past
+          // the sequence) gives P = 0
+          lse2[lane + 32 * e] = l2v[e] == -INFINITY ? -INFINITY : -l2v[e] * kLog2e;
           lse2[kTile + lane + 32 * e] = ddv[e];
         }
         mbar_arrive(vec_full(x));
