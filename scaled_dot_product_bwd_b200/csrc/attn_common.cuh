@@ -184,6 +184,25 @@ __device__ __forceinline__ constexpr bool emu_exp2(int c) {
   return BIAS != kBiasDense && (c & 7) >= MUFU_PER8;
 }
 
+// Compile-time flag for loops written once in two forms (a generic lambda
+// called with Flag<true>{} or Flag<false>{}).
+template <bool B>
+struct Flag {
+  static constexpr bool value = B;
+};
+
+// T5 table bias of a piece of a tile whose distances j - i are base ..
+// base + span: true, with the bias in log2 units in `bias`, when they all
+// lie in one capped bucket (or at j >= i of a unidirectional table), so the
+// bias is one constant over the piece.
+__device__ __forceinline__ bool t5_one_bucket(const AttnParams& p, int base, int span, int hq,
+                                              float& bias) {
+  if (p.rel_table != nullptr || p.alibi) return false;
+  if (base + span > p.t5.one_lo_max && base < p.t5.one_hi_min) return false;
+  bias = rel_bias_log2(p, base, hq);
+  return true;
+}
+
 // 2^x of columns c and c + 1, each on the unit emu_exp2 gives it; a pair
 // that both go to the FMA pipe takes the packed form (identical results).
 template <int BIAS, int MUFU_PER8>

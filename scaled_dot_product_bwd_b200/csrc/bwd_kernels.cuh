@@ -936,6 +936,14 @@ __global__ void __launch_bounds__(352, 1)
       if (!w.rows) continue;  // past this entry's query sequence: nothing to write
       const int m0 = w.m0, hq = w.hq, b = w.b, nt = w.nt;
       const int Lq = w.s.Lq, Lk = w.s.Lk;
+      // every key of the warpgroup's 64 from n0 is visible from all 128 rows
+      auto dq_tile_full = [&](int n0) {
+        bool f = n0 + kBlk <= Lk;
+        if (p.causal) f = f && (n0 + kBlk - 1 <= m0);
+        if (p.wl >= 0) f = f && (n0 >= m0 + kTile - 1 - p.wl);
+        if (p.wr >= 0) f = f && (n0 + kBlk - 1 <= m0 + p.wr);
+        return f;
+      };
       const int i = m0 + row;
       float l2 = INFINITY, dd = 0.f;
       if (i < Lq) {
@@ -955,20 +963,22 @@ __global__ void __launch_bounds__(352, 1)
         const int x = c & 1;
         const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup
         const float* lut_row = nullptr;
+        bool one_b = false;  // the warp's piece lies in one T5 bucket: bias ub throughout
+        float ub = 0.f;
         if constexpr (BIAS == kBiasT5) {
           // this warp's queries iw..iw+31 and keys n0..n0+63: j - i = (n0 - iw - 31) + e,
           // e in [0, 94]; the thread reads entry 31 - lane + cc for column cc
           const int base = n0 - m0 - (warp & 3) * 32 - 31;
-          __syncwarp();
-          for (int e = lane; e < 32 + kBlk - 1; e += 32) lut[e] = rel_bias_log2(p, base + e, hq);
-          __syncwarp();
+          one_b = dq_tile_full(n0) && t5_one_bucket(p, base, 32 + kBlk - 2, hq, ub);
+          if (!one_b) {
+            __syncwarp();
+            for (int e = lane; e < 32 + kBlk - 1; e += 32) lut[e] = rel_bias_log2(p, base + e, hq);
+            __syncwarp();
+          }
           lut_row = lut + 31 - lane;
         }
         int lo = 0, hi = kBlk - 1;
-        bool full = n0 + kBlk <= Lk;
-        if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
-        if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
-        if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
+        const bool full = dq_tile_full(n0);
         if (!full) {
           if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
           hi = min(hi, Lk - 1 - n0);
@@ -1026,19 +1036,27 @@ __global__ void __launch_bounds__(352, 1)
           }
         } else if (full) {
           // in pairs of columns: packed fp32 pair instructions for the
-          // affine step and the FMA-pipe exponentials (rounded as the scalar ones)
+          // affine step and the FMA-pipe exponentials (rounded as the scalar
+          // ones); a one-bucket T5 bias is folded into the row constant
           const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-          const uint64_t nl2 = f2_pack(-l2, -l2);
+          auto exp_full = [&](auto table) {
+            const float nl = one_b ? ub - l2 : -l2;
+            const uint64_t nl2 = f2_pack(nl, nl);
 #pragma unroll
-          for (int cc = 0; cc < kBlk; cc += 2) {
-            uint64_t x2 = f2_fma(f2_pack(__uint_as_float(pr[cc]), __uint_as_float(pr[cc + 1])), sc2, nl2);
-            if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[cc], lut_row[cc + 1]));
-            float x0, x1, y0, y1;
-            f2_unpack(x2, x0, x1);
-            exp2_pair<BIAS, kDqMufuPer8>(cc, x0, x1, y0, y1);
-            pr[cc] = __float_as_uint(y0);
-            pr[cc + 1] = __float_as_uint(y1);
-          }
+            for (int cc = 0; cc < kBlk; cc += 2) {
+              uint64_t x2 = f2_fma(f2_pack(__uint_as_float(pr[cc]), __uint_as_float(pr[cc + 1])), sc2, nl2);
+              if constexpr (decltype(table)::value) x2 = f2_add(x2, f2_pack(lut_row[cc], lut_row[cc + 1]));
+              float x0, x1, y0, y1;
+              f2_unpack(x2, x0, x1);
+              exp2_pair<BIAS, kDqMufuPer8>(cc, x0, x1, y0, y1);
+              pr[cc] = __float_as_uint(y0);
+              pr[cc + 1] = __float_as_uint(y1);
+            }
+          };
+          if (BIAS == kBiasT5 && !one_b)
+            exp_full(Flag<true>{});
+          else
+            exp_full(Flag<false>{});
         } else {
 #pragma unroll
           for (int cc = 0; cc < kBlk; ++cc) {

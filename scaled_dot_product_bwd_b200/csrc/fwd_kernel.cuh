@@ -361,28 +361,42 @@ __global__ void __launch_bounds__(384, 1)
         const int x = gc % NS;
         const int n0 = (w.nlo + it) * kTile + c0w;  // first key of this warpgroup's columns
         const uint32_t tS = tmem + lane_bits + x * kTile + c0w;
-        const float* lut_row = nullptr;
-        if constexpr (BIAS == kBiasT5) {
-          // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
-          float* lt = lut + (gc & 1) * 256;
-          const int base = n0 - m0 - (kTile - 1);
-          for (int r = row; r < kTile + kBlk - 1; r += kTile)
-            lt[r] = rel_bias_log2(p, base + r, hq);
-          named_barrier(1 + wg, kTile);
-          lut_row = lt + (kTile - 1) - row;
-        }
-        int lo = 0, hi = kBlk - 1;
         bool full = n0 + kBlk <= Lk;
         if (p.causal) full = full && (n0 + kBlk - 1 <= m0);
         if (p.wl >= 0) full = full && (n0 >= m0 + kTile - 1 - p.wl);
         if (p.wr >= 0) full = full && (n0 + kBlk - 1 <= m0 + p.wr);
+        const float* lut_row = nullptr;
+        // a fully visible piece of the warpgroup inside one T5 bucket: bias
+        // ub throughout, taken by the lean path below without a table
+        bool one_b = false;
+        float ub = 0.f;
+        if constexpr (BIAS == kBiasT5) {
+          // j - i = (n0 - m0) + (c - row): entry r = c - row + 127, r in [0, 190]
+          float* lt = lut + (gc & 1) * 256;
+          const int base = n0 - m0 - (kTile - 1);
+          // (the same for the whole warpgroup, so all or none of it takes the
+          // barrier; the table of tile gc - 2 is no longer read: every
+          // thread has passed the maximum exchange of tile gc - 1)
+          one_b = kFwdLeanSoftmax && full && p.scale_log2 > 0.f &&
+                  t5_one_bucket(p, base, kTile + kBlk - 2, hq, ub);
+          if (!one_b) {
+            for (int r = row; r < kTile + kBlk - 1; r += kTile)
+              lt[r] = rel_bias_log2(p, base + r, hq);
+            named_barrier(1 + wg, kTile);
+          }
+          lut_row = lt + (kTile - 1) - row;
+        }
+        int lo = 0, hi = kBlk - 1;
         if (!full) {
           if (p.wl >= 0) lo = max(lo, i - p.wl - n0);
           hi = min(hi, Lk - 1 - n0);
           if (p.causal) hi = min(hi, i - n0);
           if (p.wr >= 0) hi = min(hi, i + p.wr - n0);
         }
-        const bool lean = kFwdLeanSoftmax && BIAS == kBiasNone && full && p.scale_log2 > 0.f;
+        // lean: no bias, or a one-bucket T5 bias (a constant ub folded into
+        // the maximum and the exponent's offset)
+        const bool lean = kFwdLeanSoftmax && (BIAS == kBiasNone || (BIAS == kBiasT5 && one_b)) &&
+                          full && p.scale_log2 > 0.f;
 
         // ---- phase A: this warpgroup's half of S_j and its partial row max
         if (ok) ok = mbar_wait(s_full(x), (gc / NS) & 1, ctl);
@@ -403,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
               ma = fmax3(ma, __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
               mb = fmax3(mb, __uint_as_float(xs[c + 2]), __uint_as_float(xs[c + 3]));
             }
-            pmax = fmaxf(ma, mb) * p.scale_log2;
+            pmax = fmaf(fmaxf(ma, mb), p.scale_log2, ub);
           } else {
             float tm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             if constexpr (BT) {
@@ -486,7 +500,7 @@ __global__ void __launch_bounds__(384, 1)
         float sum;
         if (lean) {
           const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-          const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
+          const uint64_t nm2 = f2_pack(ub - m_sub, ub - m_sub);
           uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
           for (int c0 = 0; c0 < kBlk; c0 += 32) {
