@@ -124,15 +124,20 @@ struct DkdvLayout {
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], vec_full[2],
-  // vec_empty[2], s_full, dp_full, p_full, ds_full, s_free, dp_free, acc_done,
-  // drain[2]
-  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 9;
+  // vec_empty[2], s_full[2], dp_full, p_full[2], ds_full, s_free[2], dp_free,
+  // acc_done, drain[2]
+  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
   // 2 compute warpgroups, producer, two MMA issuers
   static constexpr int kThreads = 352;
   static constexpr int kTmemCols = 512;
   static constexpr int kSCol = 0, kDPCol = 128, kDVCol = 256, kDKCol = 256 + D;
+  // At d = 64, dV and dK take 128 columns: S^T gets a second buffer at 384,
+  // so S^T(i + 1) is computed while the warpgroups work on block i instead
+  // of waiting for dV(i) to read P^T(i) out of the one buffer.
+  static constexpr bool kSDouble = (D == 64);
+  static constexpr int kSCol1 = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
@@ -174,14 +179,23 @@ __global__ void __launch_bounds__(352, 1)
   constexpr int kB = 1 + 2 * SQ + 2 * SO;
   auto vec_full = [&](int x) { return bar(kB + x); };
   auto vec_empty = [&](int x) { return bar(kB + 2 + x); };
-  const uint32_t s_full = bar(kB + 4);
-  const uint32_t dp_full = bar(kB + 5);
-  const uint32_t p_full = bar(kB + 6);
-  const uint32_t ds_full = bar(kB + 7);
-  const uint32_t s_free = bar(kB + 8);
-  const uint32_t dp_free = bar(kB + 9);
-  const uint32_t acc_done = bar(kB + 10);
-  auto drain = [&](int x) { return bar(kB + 11 + x); };
+  // S^T ready, P^T ready, S^T buffer free: with two S^T buffers, block i's
+  // on barrier i % 2 with parity (i / 2) % 2 (S^T(i + 1) is issued before
+  // the wait for P^T(i), so the warpgroups may publish P^T(i + 1) first: one
+  // barrier would then complete two phases and lose a wakeup); else one
+  // barrier with parity i % 2
+  constexpr bool SD = Lay::kSDouble;
+  auto sb_of = [&](int i) { return SD ? (i & 1) : 0; };
+  auto sb_par = [&](int i) { return static_cast<uint32_t>(SD ? ((i >> 1) & 1) : (i & 1)); };
+  auto s_col = [&](int i) { return static_cast<uint32_t>(SD && (i & 1) ? Lay::kSCol1 : Lay::kSCol); };
+  auto s_full = [&](int x) { return bar(kB + 4 + x); };
+  const uint32_t dp_full = bar(kB + 6);
+  auto p_full = [&](int x) { return bar(kB + 7 + x); };
+  const uint32_t ds_full = bar(kB + 9);
+  auto s_free = [&](int x) { return bar(kB + 10 + x); };
+  const uint32_t dp_free = bar(kB + 12);
+  const uint32_t acc_done = bar(kB + 13);
+  auto drain = [&](int x) { return bar(kB + 14 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -201,11 +215,13 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(vec_full(x), 32);          // the producer warp's lanes
       mbar_init(vec_empty(x), 2 * kTile);  // both compute warpgroups
     }
-    mbar_init(s_full, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(p_full(x), 2 * kTile);
+      mbar_init(s_free(x), 1);
+    }
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 2 * kTile);
     mbar_init(ds_full, 2 * kTile);
-    mbar_init(s_free, 1);
     mbar_init(dp_free, 1);
     mbar_init(acc_done, 2);
     mbar_init(drain(0), 1);
@@ -334,28 +350,42 @@ __global__ void __launch_bounds__(352, 1)
       bool ok = issuer_wait(kv_full, 0, ctl);
       for (int it = 0; it < total && ok; ++it) {
         const int sq = it % SQ, so = it % SO;
-        const uint64_t qk = dk0 + ((Lay::kQOff + sq * Lay::kTileBytes) >> 4);
         const uint64_t qm = dmn0 + ((Lay::kQOff + sq * Lay::kTileBytes) >> 4);
         const uint64_t od = dk0 + ((Lay::kDOOff + so * Lay::kTileBytes) >> 4);
         const uint64_t om = dmn0 + ((Lay::kDOOff + so * Lay::kTileBytes) >> 4);
         if (chain_s) {
-          if (!(ok = issuer_wait(q_full(sq), (it / SQ) & 1, ctl))) break;
-          if (it > 0 && !(ok = issuer_wait(s_free, (it - 1) & 1, ctl))) break;
-          tc_fence_after();
+          // S^T(j) = K Q(j)^T into its buffer, once Q(j) has landed and dV
+          // has read P^T of the buffer's previous block
+          auto issue_s = [&](int j) -> bool {
+            const int sj = j % SQ;
+            if (!issuer_wait(q_full(sj), (j / SQ) & 1, ctl)) return false;
+            const int nbuf = SD ? 2 : 1;
+            if (j >= nbuf && !issuer_wait(s_free(sb_of(j - nbuf)), sb_par(j - nbuf), ctl)) return false;
+            tc_fence_after();
+            const uint64_t qkj = dk0 + ((Lay::kQOff + sj * Lay::kTileBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + Lay::kSCol, dk0 + ((Lay::kKOff + kmajor_koff(kk, kTile)) >> 4),
-                   qk + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
-          mma_commit(s_full);
-          mma_commit(q_empty(sq));
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + s_col(j), dk0 + ((Lay::kKOff + kmajor_koff(kk, kTile)) >> 4),
+                     qkj + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
+            mma_commit(s_full(sb_of(j)));
+            mma_commit(q_empty(sj));
+            return true;
+          };
+          if (SD) {
+            // S^T(it + 1) ahead of the wait for P^T(it)
+            if (it == 0 && !(ok = issue_s(0))) break;
+            if (it + 1 < total && !(ok = issue_s(it + 1))) break;
+          } else {
+            if (!(ok = issue_s(it))) break;
+          }
           if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
-          if (!(ok = issuer_wait(p_full, it & 1, ctl))) break;
+          if (!(ok = issuer_wait(p_full(sb_of(it)), sb_par(it), ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + Lay::kSCol, kk), om + kk * (2048 >> 4),
+            mma_ts(tmem + Lay::kDVCol, split_a_col(tmem + s_col(it), kk), om + kk * (2048 >> 4),
                    kIdG, (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(s_free);
+          mma_commit(s_free(sb_of(it)));
           mma_commit(o_empty(so));
         } else {
           if (!(ok = issuer_wait(o_full(so), (it / SO) & 1, ctl))) break;
@@ -394,7 +424,7 @@ __global__ void __launch_bounds__(352, 1)
     const int j = n0 + row;
     const int c0w = kBlk * wg;  // first query column of this warpgroup
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_bits + Lay::kSCol + c0w;
+    const uint32_t tS0 = tmem + lane_bits + c0w;  // + the block's S^T buffer column
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
     bool ok = true;
@@ -430,7 +460,8 @@ __global__ void __launch_bounds__(352, 1)
         bcol = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
                static_cast<int64_t>(min(m0, Lq - 1)) * p.sb_i + min(j, Lk - 1);
       if (ok) ok = mbar_wait(vec_full(x), (it >> 1) & 1, ctl);  // LSE / D staged
-      if (ok) ok = mbar_wait(s_full, it & 1, ctl);
+      const uint32_t tS = tS0 + s_col(it);
+      if (ok) ok = mbar_wait(s_full(sb_of(it)), sb_par(it), ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
@@ -495,7 +526,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(sb_of(it)));
       if (ok) ok = mbar_wait(dp_full, it & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;

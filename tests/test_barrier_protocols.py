@@ -251,9 +251,16 @@ def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True):
 
 
 # ---------------------------------------------------------------- dK / dV
-def dkdv_protocol(total, SQ, SO):
-    bars = {"kv_full": 1, "s_full": 1, "dp_full": 1, "p_full": 2, "ds_full": 2, "s_free": 1,
-            "dp_free": 1, "acc_done": 2}
+def dkdv_protocol(total, SQ, SO, s_double=False, p_double=True):
+    """s_double: S^T double-buffered (d = 64): S^T(i + 1) is issued before
+    the wait for P^T(i); s_full, p_full and s_free then go by block parity
+    (p_double=False models one P^T-ready barrier instead)."""
+    bars = {"kv_full": 1, "dp_full": 1, "ds_full": 2, "dp_free": 1, "acc_done": 2}
+    nb = 2 if s_double else 1
+    for x in range(nb):
+        bars[f"s_full{x}"] = 1
+        bars[f"p_full{x}"] = 2
+        bars[f"s_free{x}"] = 1
     for s in range(SQ):
         bars[f"q_full{s}"] = 1
         bars[f"q_empty{s}"] = 2
@@ -263,6 +270,12 @@ def dkdv_protocol(total, SQ, SO):
     for x in range(2):
         bars[f"vec_full{x}"] = 1
         bars[f"vec_empty{x}"] = 2
+
+    def par(name, it):
+        # (barrier, parity) of block it's phase
+        if s_double and (p_double or name != "p_full"):
+            return (f"{name}{it & 1}", (it >> 1) & 1)
+        return (f"{name}0", it & 1)
 
     def producer():
         yield ("async", "kv_full")
@@ -274,17 +287,26 @@ def dkdv_protocol(total, SQ, SO):
             yield ("wait", f"vec_empty{it & 1}", ((it >> 1) & 1) ^ 1)
             yield ("arrive", f"vec_full{it & 1}")
 
+    def issue_s(it):
+        yield ("wait", f"q_full{it % SQ}", (it // SQ) & 1)
+        if it >= nb:
+            yield ("wait",) + par("s_free", it - nb)
+        yield ("async", par("s_full", it)[0])
+        yield ("async", f"q_empty{it % SQ}")
+
     def chain_s():
         yield ("wait", "kv_full", 0)
+        if s_double and total > 0:
+            yield from issue_s(0)
         for it in range(total):
-            yield ("wait", f"q_full{it % SQ}", (it // SQ) & 1)
-            if it > 0:
-                yield ("wait", "s_free", (it - 1) & 1)
-            yield ("async", "s_full")
-            yield ("async", f"q_empty{it % SQ}")
+            if s_double:
+                if it + 1 < total:
+                    yield from issue_s(it + 1)
+            else:
+                yield from issue_s(it)
             yield ("wait", f"o_full{it % SO}", (it // SO) & 1)
-            yield ("wait", "p_full", it & 1)
-            yield ("async", "s_free")
+            yield ("wait",) + par("p_full", it)
+            yield ("async", par("s_free", it)[0])
             yield ("async", f"o_empty{it % SO}")
         yield ("async", "acc_done")
 
@@ -305,8 +327,8 @@ def dkdv_protocol(total, SQ, SO):
     def warpgroup():
         for it in range(total):
             yield ("wait", f"vec_full{it & 1}", (it >> 1) & 1)
-            yield ("wait", "s_full", it & 1)
-            yield ("arrive", "p_full")
+            yield ("wait",) + par("s_full", it)
+            yield ("arrive", par("p_full", it)[0])
             yield ("wait", "dp_full", it & 1)
             yield ("arrive", "ds_full")
             yield ("arrive", f"vec_empty{it & 1}")
@@ -350,10 +372,24 @@ def test_dq_protocol_with_one_ds_barrier_can_lose_a_wakeup():
     assert found
 
 
-@pytest.mark.parametrize("SQ,SO", [(3, 2), (2, 2), (4, 4)])
-def test_dkdv_protocol_has_no_deadlock(SQ, SO):
-    for total in (1, 2, 7, 40):
+def test_dkdv_double_s_with_one_p_barrier_can_lose_a_wakeup():
+    # with S^T(i + 1) issued before the wait for P^T(i), the warpgroups can
+    # publish P^T(i + 1) before the issuer looks for P^T(i): one barrier would
+    # then have completed two phases
+    found = False
+    for seed in range(200):
+        bars, roles = dkdv_protocol(40, 4, 4, s_double=True, p_double=False)
+        if explore(bars, roles, seed) is not None:
+            found = True
+            break
+    assert found
+
+
+@pytest.mark.parametrize("SQ,SO,s_double", [(3, 2, False), (2, 2, False), (4, 4, False),
+                                            (4, 4, True), (2, 2, True)])
+def test_dkdv_protocol_has_no_deadlock(SQ, SO, s_double):
+    for total in (1, 2, 3, 7, 40):
         for seed in SEEDS:
-            bars, roles = dkdv_protocol(total, SQ, SO)
+            bars, roles = dkdv_protocol(total, SQ, SO, s_double)
             blocked = explore(bars, roles, seed)
             assert blocked is None, (total, seed, blocked)
