@@ -36,6 +36,9 @@ struct T5Spec {
   // keys after it, or bucket 0 of a unidirectional table); INT_MIN /
   // INT_MAX when no distance in range is capped.
   int one_lo_max, one_hi_min;
+  // the closed form in float32 for the device's first guess:
+  // (half - max_exact) / log2(max_distance / max_exact) and 1 / max_exact
+  float log_scale, inv_max_exact;
 };
 
 // The contiguous range [lo, hi] of distances r = j - i (within the
@@ -57,9 +60,27 @@ __host__ __device__ __forceinline__ int t5_bucket(int rel, const T5Spec& s) {
   if (n < s.max_exact) {
     b = n;
   } else {
+#ifdef __CUDA_ARCH__
+    // The closed form max_exact + trunc(log2(n / max_exact) * log_scale) in
+    // float32 is within one of its float64 value; the integer thresholds
+    // then decide exactly: thr[k] <= n < thr[k + 1] is bucket max_exact + k,
+    // n >= thr[nthr - 1] the capped one.  (A loop over the thresholds reads
+    // them one after another and cost ~400 cycles per distance.)
+    const int K = s.nthr;
+    if (n >= s.thr[K - 1]) {
+      b = s.half - 1;
+    } else {
+      int k = static_cast<int>(__log2f(static_cast<float>(n) * s.inv_max_exact) * s.log_scale);
+      k = min(max(k, 0), K - 1);
+      if (k + 1 < K && n >= s.thr[k + 1]) ++k;
+      if (n < s.thr[k]) --k;
+      b = s.max_exact + k;
+    }
+#else
     b = s.max_exact - 1;
     for (int k = 0; k < s.nthr; ++k) b += (n >= s.thr[k]) ? 1 : 0;
     b = b < s.half - 1 ? b : s.half - 1;
+#endif
   }
   return b + off;
 }

@@ -332,7 +332,9 @@ __global__ void __launch_bounds__(352, 1)
   } else if (warp == 9 || warp == 10) {
     // ===================== MMA issuers (one thread each) =====================
     // Warp 9 owns the S^T chain: S^T(i), then dV(i) once P^T(i) is ready, then
-    // S^T(i+1) once dV(i) has read P^T(i) out of the S^T columns.  Warp 10 owns
+    // S^T(i+1) once dV(i) has read P^T(i) out of the S^T columns (at d = 64,
+    // with two S^T buffers, S^T(i+1) goes before the wait for P^T(i) and
+    // waits only for dV(i-1)).  Warp 10 owns
     // the dP^T chain: dP^T(i), dK(i) once dS^T(i) is ready, dP^T(i+1) once dK(i)
     // is done.  Neither waits on the other's barriers, so a stalled chain does
     // not hold up MMAs that are ready in the other.

@@ -183,6 +183,8 @@ bool fill_t5(T5Spec& t, int nb, int md, int bidir) {
   const int sat = t.thr[K - 1];
   t.one_lo_max = sat == INT_MAX ? INT_MIN : -sat;
   t.one_hi_min = bidir ? sat : 0;
+  t.log_scale = static_cast<float>(static_cast<double>(half - me) / std::log2(static_cast<double>(md) / me));
+  t.inv_max_exact = static_cast<float>(1.0 / me);
   return true;
 }
 

@@ -13,7 +13,9 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("nb,md,bidir", [(32, 128, True), (32, 128, False), (64, 256, True),
-                                         (16, 40, True), (128, 1000, False), (8, 20, True)])
+                                         (16, 40, True), (128, 1000, False), (8, 20, True),
+                                         (16, 24, True), (8, 20, False), (32, 4096, True),
+                                         (128, 20000, True), (64, 40, False), (128, 65, True)])
 def test_t5_buckets_bit_exact(nb, md, bidir):
     rel = np.arange(-20000, 20001, dtype=np.int32)
     got = sdpa_t5_bucket(torch.from_numpy(rel).cuda(), nb, md, bidir).cpu().numpy()
