@@ -658,12 +658,12 @@ struct DqLayout {
   static constexpr int kBAccBytes = (DSM == kDsDiagT5) ? 8 * 128 * 4 : 0;
   static constexpr int kBarOff = kBAccOff + kBAccBytes;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], dq_done[2],
-  // dp_full, dp_used, ds_full[2], acc_done, drain[2], q_empty, o_full, o_empty,
+  // dp_full, dp_used, ds_full[2], acc_done, drain[3], q_empty, o_full, o_empty,
   // b_full[2], b_empty[2]
-  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 18;
+  static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 19;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
-  static constexpr int kThreads = 352;  // 2 compute warpgroups, producer, two MMA issuers
+  static constexpr int kThreads = 384;  // 2 compute warpgroups, producer, three MMA issuers
   static constexpr int kTmemCols = 512;
   static constexpr int kDPCol = 256, kDQCol = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -671,7 +671,7 @@ struct DqLayout {
 
 // DSM: see DqLayout (the bias-gradient paths).
 template <int D, int BIAS, int DSM = kDsNone>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
@@ -729,13 +729,13 @@ __global__ void __launch_bounds__(352, 1)
   auto dq_done = [&](int x) { return bar(kB + 2 + x); };  // dQ MMA of a block in buffer x done
   const uint32_t dp_full = bar(kB + 4);
   const uint32_t dp_used = bar(kB + 5);
-  // dS of block i ready, by block parity: the dQ issuer issues dP(i + 1)
-  // before it waits for dS(i), so the warpgroups can finish dS(i + 1) before
-  // it looks; a single barrier would then have completed two phases and the
+  // dS of block i ready, by block parity: the warpgroups can finish dS(i + 1)
+  // (dP(i + 1) does not wait for the dQ MMAs) before the dQ issuer looks for
+  // dS(i); a single barrier would then have completed two phases and the
   // wait for block i's parity would never succeed.
   auto ds_full = [&](int x) { return x == 0 ? bar(kB + 6) : bar(kB + 13); };
   const uint32_t acc_done = bar(kB + 7);
-  auto drain = [&](int x) { return bar(kB + 8 + x); };
+  auto drain = [&](int x) { return x < 2 ? bar(kB + 8 + x) : bar(kB + 18); };
   // Q is read only by the score issuer, dO only by the dP issuer: each tile is
   // released as soon as its one reader is done with the item
   const uint32_t q_empty = bar(kB + 10);
@@ -777,6 +777,7 @@ __global__ void __launch_bounds__(352, 1)
     mbar_init(acc_done, 1);
     mbar_init(drain(0), 1);
     mbar_init(drain(1), 1);
+    mbar_init(drain(2), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -867,52 +868,39 @@ __global__ void __launch_bounds__(352, 1)
           if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
       }
     }
-  } else if (warp == 9 || warp == 10) {
+  } else if (warp >= 9 && warp <= 11) {
     // ===================== MMA issuers (one thread each) =====================
     // Warp 9 runs the score chain: S(i) into buffer i % 2 once K(i) has landed
     // and the dQ MMA of block i - 2 has read dS out of that buffer.  Warp 10
-    // runs dP one block ahead of dQ within an item: dP(i + 1) as soon as both
-    // warpgroups have loaded dP(i), then dQ(i) once dS(i) is ready.  Block
-    // indices run on across items.
+    // runs the dP chain: dP(i + 1) as soon as both warpgroups have loaded
+    // dP(i).  Warp 11 issues dQ(i) += dS(i) K(i) as soon as dS(i) is ready.
+    // With dP and dQ on one thread, dQ(i) waited behind the issue of
+    // dP(i + 1) (~1300 cycles on the mistral-shaped workload) and S(i + 2)
+    // behind dQ(i).  Block indices run on across items.
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
       constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
-      const bool chain_s = (warp == 9);
+      const int role = warp - 9;  // 0 scores, 1 dP, 2 dQ
       // descriptors built once, plus byte offset / 16 per operand (see the
       // dK/dV kernel's issuers)
       const uint64_t dk0 = smem_desc_sw128(sb, 16, 1024);            // K-major
       const uint64_t dmn0 = smem_desc_sw128(sb, kTile * 128, 1024);  // MN-major, 64-wide halves
-      auto issue_dp = [&](int c) -> bool {
-        const int sv = c % SV;
-        if (!issuer_wait(v_full(sv), (c / SV) & 1, ctl)) return false;
-        if (c > 0 && !issuer_wait(dp_used, (c - 1) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint64_t vd = dk0 + ((Lay::kVOff + sv * Lay::kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + Lay::kDPCol, dk0 + ((Lay::kDOOff + kmajor_koff(kk, kTile)) >> 4),
-                 vd + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
-        mma_commit(dp_full);
-        mma_commit(v_empty(sv));
-        return true;
-      };
       int c = 0;  // key blocks so far, over all items
       int u = 0;  // items with a non-empty band so far
       bool ok = true;
       for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
         const Item w = item_at(id);
         if (w.nt == 0) continue;
-        if (!(ok = issuer_wait(chain_s ? q_full : o_full, u & 1, ctl))) break;
-        if (!chain_s && !(ok = issue_dp(c))) break;
+        if (role == 0 && !(ok = issuer_wait(q_full, u & 1, ctl))) break;
+        if (role == 1 && !(ok = issuer_wait(o_full, u & 1, ctl))) break;
         for (int it = 0; it < w.nt; ++it, ++c) {
           const int x = c & 1;
           const int sk = c % SK;
-          const uint64_t kd = dk0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
-          const uint64_t kmd = dmn0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
-          if (chain_s) {
+          if (role == 0) {
             if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
             if (c >= 2 && !(ok = issuer_wait(dq_done(x), ((c >> 1) - 1) & 1, ctl))) break;
             tc_fence_after();
+            const uint64_t kd = dk0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + kTile * x, dk0 + ((Lay::kQOff + kmajor_koff(kk, kTile)) >> 4),
@@ -920,11 +908,23 @@ __global__ void __launch_bounds__(352, 1)
                      kk > 0 ? 1u : 0u);
             mma_commit(s_full(x));
             mma_commit(k_empty(sk));
+          } else if (role == 1) {
+            const int sv = c % SV;
+            if (!(ok = issuer_wait(v_full(sv), (c / SV) & 1, ctl))) break;
+            if (c > 0 && !(ok = issuer_wait(dp_used, (c - 1) & 1, ctl))) break;
+            tc_fence_after();
+            const uint64_t vd = dk0 + ((Lay::kVOff + sv * Lay::kTileBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + Lay::kDPCol, dk0 + ((Lay::kDOOff + kmajor_koff(kk, kTile)) >> 4),
+                     vd + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
+            mma_commit(dp_full);
+            mma_commit(v_empty(sv));
           } else {
-            if (it + 1 < w.nt && !(ok = issue_dp(c + 1))) break;
             if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
             if (!(ok = issuer_wait(ds_full(c & 1), (c >> 1) & 1, ctl))) break;
             tc_fence_after();
+            const uint64_t kmd = dmn0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
             // the item's first dQ MMA overwrites the accumulator: every
             // warpgroup thread read the previous item's dQ before marking dS ready
 #pragma unroll
@@ -937,15 +937,16 @@ __global__ void __launch_bounds__(352, 1)
           }
         }
         if (!ok) break;
-        mma_commit(chain_s ? q_empty : o_empty);  // the item's Q / dO is read
-        if (!chain_s) mma_commit(acc_done);
+        if (role == 0) mma_commit(q_empty);   // the item's Q is read
+        if (role == 1) mma_commit(o_empty);   // the item's dO is read
+        if (role == 2) mma_commit(acc_done);  // the item's dQ is complete
         ++u;
       }
       if (!ok) {
         volatile int never = 0;
         const WaitCtl ign{&never, p.wait_limit_ns};
-        mma_commit(drain(chain_s ? 0 : 1));
-        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
+        mma_commit(drain(role));
+        mbar_wait(drain(role), 0, ign);
       }
     }
   } else {

@@ -157,7 +157,9 @@ def fwd_protocol(items, SK, SV, NS=3, bias_ring=False, rng=None):
 
 
 # ------------------------------------------------------------------- dQ
-def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True):
+def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True, three_issuers=True):
+    """three_issuers: dP and dQ MMAs issued by threads of their own (the
+    kernel); else one thread issues dP(c + 1) and then dQ(c)."""
     bars = {"q_full": 1, "q_empty": 1, "o_full": 1, "o_empty": 1, "dp_full": 1, "dp_used": 2,
             "ds_full": 2, "ds_full0": 2, "ds_full1": 2, "acc_done": 1}
     for s in range(SK):
@@ -231,6 +233,30 @@ def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True):
             yield ("async", "o_empty")
             yield ("async", "acc_done")
 
+    def dp_issuer():
+        c = 0
+        for u, nt in enumerate(items):
+            yield ("wait", "o_full", u & 1)
+            for _ in range(nt):
+                yield ("wait", f"v_full{c % SV}", (c // SV) & 1)
+                if c > 0:
+                    yield ("wait", "dp_used", (c - 1) & 1)
+                yield ("async", "dp_full")
+                yield ("async", f"v_empty{c % SV}")
+                c += 1
+            yield ("async", "o_empty")
+
+    def dq_only_issuer():
+        c = 0
+        for u, nt in enumerate(items):
+            for _ in range(nt):
+                yield ("wait", f"k_full{c % SK}", (c // SK) & 1)
+                yield ("wait",) + ds(c)
+                yield ("async", f"dq_done{c & 1}")
+                yield ("async", f"k_empty{c % SK}")
+                c += 1
+            yield ("async", "acc_done")
+
     def warpgroup():
         c = 0
         for u, nt in enumerate(items):
@@ -245,8 +271,12 @@ def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True):
                 c += 1
             yield ("wait", "acc_done", u & 1)
 
-    roles = {"prod": producer(), "s": s_issuer(), "dq": dq_issuer(), "wg0": warpgroup(),
-             "wg1": warpgroup()}
+    if three_issuers:
+        roles = {"prod": producer(), "s": s_issuer(), "dp": dp_issuer(), "dq": dq_only_issuer(),
+                 "wg0": warpgroup(), "wg1": warpgroup()}
+    else:
+        roles = {"prod": producer(), "s": s_issuer(), "dq": dq_issuer(), "wg0": warpgroup(),
+                 "wg1": warpgroup()}
     return bars, roles
 
 
@@ -356,16 +386,17 @@ def test_forward_protocol_has_no_deadlock(SK, SV, bias_ring):
 def test_dq_protocol_has_no_deadlock(SK, SV, bias_ring):
     for items in ITEM_SETS:
         for seed in SEEDS:
-            bars, roles = dq_protocol(items, SK, SV, bias_ring=bias_ring)
-            blocked = explore(bars, roles, seed)
-            assert blocked is None, (items, seed, blocked)
+            for three in (True, False):
+                bars, roles = dq_protocol(items, SK, SV, bias_ring=bias_ring, three_issuers=three)
+                blocked = explore(bars, roles, seed)
+                assert blocked is None, (items, seed, three, blocked)
 
 
 def test_dq_protocol_with_one_ds_barrier_can_lose_a_wakeup():
     # The model catches the race the double-buffered dS barrier removes.
     found = False
     for seed in range(200):
-        bars, roles = dq_protocol([8, 8, 8], 4, 3, ds_double=False)
+        bars, roles = dq_protocol([8, 8, 8], 4, 3, ds_double=False, three_issuers=False)
         if explore(bars, roles, seed) is not None:
             found = True
             break
