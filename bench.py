@@ -69,12 +69,12 @@ for _hkv, _tag in ((32, "mha"), (8, "gqa"), (1, "mqa")):
 # only while the library is built from exactly those sources.
 NCU_TRAFFIC = {
     # mistral4k_small (batch 2) capture, profiles/mistral4k_small_full_capture.md
-    ("mistral4k", "fwd"): {"bytes_per_batch": (100943872 + 36961024) / 2,
-        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
-    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171795200 + 45393152) / 2,
-        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
-    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170254848 + 23896064) / 2,
-        "source_hash": "55d89616eea4a6549b0a6bac87542a4796d7201f71dfe928195a19f42500cc17"},
+    ("mistral4k", "fwd"): {"bytes_per_batch": (100941824 + 40003072) / 2,
+        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
+    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171728128 + 43235328) / 2,
+        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
+    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170409728 + 25851392) / 2,
+        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
 }
 
 
