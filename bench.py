@@ -70,11 +70,11 @@ for _hkv, _tag in ((32, "mha"), (8, "gqa"), (1, "mqa")):
 NCU_TRAFFIC = {
     # mistral4k_small (batch 2) capture, profiles/mistral4k_small_full_capture.md
     ("mistral4k", "fwd"): {"bytes_per_batch": (100941824 + 40003072) / 2,
-        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
+        "source_hash": "62dd73708300029ae96f352758e0b5b746047be67df999e80b967a9aa60f197a"},
     ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171728128 + 43235328) / 2,
-        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
+        "source_hash": "62dd73708300029ae96f352758e0b5b746047be67df999e80b967a9aa60f197a"},
     ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170409728 + 25851392) / 2,
-        "source_hash": "eb0592ea00c285a55cb351c74fc2d3ef1f1c3b0f8d1e84890e5aa7a7c8ace51a"},
+        "source_hash": "62dd73708300029ae96f352758e0b5b746047be67df999e80b967a9aa60f197a"},
 }
 
 

@@ -663,7 +663,12 @@ struct DqLayout {
   static constexpr int kNumBars = 1 + 2 * kSK + 2 * kSV + 19;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
-  static constexpr int kThreads = 384;  // 2 compute warpgroups, producer, three MMA issuers
+  // 2 compute warpgroups, producer, MMA issuers: three (scores, dP, dQ),
+  // or two (dP and dQ on one) for the diagonal-sum forms, whose warpgroups
+  // stage dS in shared memory every block (measured: a third issuer made
+  // those slower, every other form faster)
+  static constexpr int kIssuers = (DSM == kDsDiag || DSM == kDsDiagT5) ? 2 : 3;
+  static constexpr int kThreads = 288 + 32 * kIssuers;
   static constexpr int kTmemCols = 512;
   static constexpr int kDPCol = 256, kDQCol = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -671,7 +676,7 @@ struct DqLayout {
 
 // DSM: see DqLayout (the bias-gradient paths).
 template <int D, int BIAS, int DSM = kDsNone>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
@@ -868,7 +873,7 @@ __global__ void __launch_bounds__(384, 1)
           if (issued_v[s] >= 0) mbar_wait(v_full(s), issued_v[s], ign);
       }
     }
-  } else if (warp >= 9 && warp <= 11) {
+  } else if (Lay::kIssuers == 3 && warp >= 9 && warp <= 11) {
     // ===================== MMA issuers (one thread each) =====================
     // Warp 9 runs the score chain: S(i) into buffer i % 2 once K(i) has landed
     // and the dQ MMA of block i - 2 has read dS out of that buffer.  Warp 10
@@ -947,6 +952,87 @@ __global__ void __launch_bounds__(384, 1)
         const WaitCtl ign{&never, p.wait_limit_ns};
         mma_commit(drain(role));
         mbar_wait(drain(role), 0, ign);
+      }
+    }
+  } else if (Lay::kIssuers == 2 && (warp == 9 || warp == 10)) {
+    // ================ MMA issuers, bias-gradient forms (two threads) ================
+    // Warp 9 runs the score chain as above.  Warp 10 runs dP one block ahead
+    // of dQ within an item: dP(i + 1) as soon as both warpgroups have loaded
+    // dP(i), then dQ(i) once dS(i) is ready.  (A third issuer made these
+    // diagonal-sum forms slower: their warpgroups' extra work per block,
+    // not the dQ issue, bounds them.)
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTile, kTile, 0, 0);  // 128 queries x 128 keys
+      constexpr uint32_t kIdQ = idesc_bf16_f32(kTile, D, 0, 1);      // 128 queries x d
+      const bool chain_s = (warp == 9);
+      // descriptors built once, plus byte offset / 16 per operand (see the
+      // dK/dV kernel's issuers)
+      const uint64_t dk0 = smem_desc_sw128(sb, 16, 1024);            // K-major
+      const uint64_t dmn0 = smem_desc_sw128(sb, kTile * 128, 1024);  // MN-major, 64-wide halves
+      auto issue_dp = [&](int c) -> bool {
+        const int sv = c % SV;
+        if (!issuer_wait(v_full(sv), (c / SV) & 1, ctl)) return false;
+        if (c > 0 && !issuer_wait(dp_used, (c - 1) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint64_t vd = dk0 + ((Lay::kVOff + sv * Lay::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + Lay::kDPCol, dk0 + ((Lay::kDOOff + kmajor_koff(kk, kTile)) >> 4),
+                 vd + (kmajor_koff(kk, kTile) >> 4), kIdS, kk > 0 ? 1u : 0u);
+        mma_commit(dp_full);
+        mma_commit(v_empty(sv));
+        return true;
+      };
+      int c = 0;  // key blocks so far, over all items
+      int u = 0;  // items with a non-empty band so far
+      bool ok = true;
+      for (int id = blockIdx.x; id < n_items && ok; id += gridDim.x) {
+        const Item w = item_at(id);
+        if (w.nt == 0) continue;
+        if (!(ok = issuer_wait(chain_s ? q_full : o_full, u & 1, ctl))) break;
+        if (!chain_s && !(ok = issue_dp(c))) break;
+        for (int it = 0; it < w.nt; ++it, ++c) {
+          const int x = c & 1;
+          const int sk = c % SK;
+          const uint64_t kd = dk0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
+          const uint64_t kmd = dmn0 + ((Lay::kKOff + sk * Lay::kTileBytes) >> 4);
+          if (chain_s) {
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (c >= 2 && !(ok = issuer_wait(dq_done(x), ((c >> 1) - 1) & 1, ctl))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + kTile * x, dk0 + ((Lay::kQOff + kmajor_koff(kk, kTile)) >> 4),
+                     kd + (kmajor_koff(kk, kTile) >> 4), kIdS,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(s_full(x));
+            mma_commit(k_empty(sk));
+          } else {
+            if (it + 1 < w.nt && !(ok = issue_dp(c + 1))) break;
+            if (!(ok = issuer_wait(k_full(sk), (c / SK) & 1, ctl))) break;
+            if (!(ok = issuer_wait(ds_full(c & 1), (c >> 1) & 1, ctl))) break;
+            tc_fence_after();
+            // the item's first dQ MMA overwrites the accumulator: every
+            // warpgroup thread read the previous item's dQ before marking dS ready
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(tmem + Lay::kDQCol, split_a_col(tmem + kTile * x, kk), kmd + kk * (2048 >> 4),
+                     kIdQ,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(dq_done(x));
+            mma_commit(k_empty(sk));
+          }
+        }
+        if (!ok) break;
+        mma_commit(chain_s ? q_empty : o_empty);  // the item's Q / dO is read
+        if (!chain_s) mma_commit(acc_done);
+        ++u;
+      }
+      if (!ok) {
+        volatile int never = 0;
+        const WaitCtl ign{&never, p.wait_limit_ns};
+        mma_commit(drain(chain_s ? 0 : 1));
+        mbar_wait(drain(chain_s ? 0 : 1), 0, ign);
       }
     }
   } else {
@@ -1400,22 +1486,27 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
   if (phases & kPhaseDq) {
     auto kern = bwd_dq_kernel<D, BIAS>;
     int smem_bytes = DqLayout<D, BIAS>::kSmemAlloc;
+    int threads = DqLayout<D, BIAS>::kThreads;
     if constexpr (BIAS == kBiasDense) {
       if (p.ds_out) {
         kern = bwd_dq_kernel<D, BIAS, kDsStore>;
         smem_bytes = DqLayout<D, BIAS, kDsStore>::kSmemAlloc;
+        threads = DqLayout<D, BIAS, kDsStore>::kThreads;
       }
     }
     if constexpr (BIAS == kBiasT5) {
       if (p.diag_out && p.rel_table) {
         kern = bwd_dq_kernel<D, BIAS, kDsDiag>;
         smem_bytes = DqLayout<D, BIAS, kDsDiag>::kSmemAlloc;
+        threads = DqLayout<D, BIAS, kDsDiag>::kThreads;
       } else if (p.diag_out && p.alibi) {
         kern = bwd_dq_kernel<D, BIAS, kDsMoment>;
         smem_bytes = DqLayout<D, BIAS, kDsMoment>::kSmemAlloc;
+        threads = DqLayout<D, BIAS, kDsMoment>::kThreads;
       } else if (p.diag_out) {
         kern = bwd_dq_kernel<D, BIAS, kDsDiagT5>;
         smem_bytes = DqLayout<D, BIAS, kDsDiagT5>::kSmemAlloc;
+        threads = DqLayout<D, BIAS, kDsDiagT5>::kThreads;
       }
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
@@ -1424,7 +1515,7 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
     const int64_t items = static_cast<int64_t>((p.Lq + kTile - 1) / kTile) * p.Hq * p.B;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    kern<<<static_cast<int>(items < sms ? items : sms), DqLayout<D, BIAS>::kThreads, smem_bytes, st>>>(
+    kern<<<static_cast<int>(items < sms ? items : sms), threads, smem_bytes, st>>>(
         p, mq, mk, mv, mdo, mb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
