@@ -162,14 +162,25 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs.
+
+    A reader thread timestamps every sample.  ready() waits until nvidia-smi
+    is producing samples (its first one can take a second on a fresh box), so
+    that the timed region, bracketed by mark_start() / mark_end(), falls
+    inside the sampled stretch; the report keeps the samples taken during the
+    region, or the one nearest to it when the region is shorter than the
+    sampling interval."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu: int):
+        import threading
         self.proc = None
+        self.lines = []          # (monotonic time, line)
+        self.t0 = self.t1 = None
+        self.first = threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -177,34 +188,58 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line))
+            self.first.set()
+
+    def ready(self, timeout=5.0):
+        if self.proc is not None:
+            self.first.wait(timeout)
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.12)
+        time.sleep(0.06)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
+            self.proc.wait()
+        self.reader.join(timeout=5)
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.splitlines():
+        for t, line in self.lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                rows.append((t, float(f[1]), float(f[2]),
+                             {n for n, v in zip(names, f[5:9]) if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+        t0 = self.t0 if self.t0 is not None else rows[0][0]
+        t1 = self.t1 if self.t1 is not None else rows[-1][0]
+        inside = [r for r in rows if t0 <= r[0] <= t1 + 0.05]
+        if not inside:  # region shorter than the sampling interval: the nearest sample
+            mid = 0.5 * (t0 + t1)
+            inside = [min(rows, key=lambda r: abs(r[0] - mid))]
+        reasons = set().union(*(r[3] for r in inside))
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "samples": len(inside),
                 "reasons": sorted(reasons)}
 
 
@@ -382,12 +417,14 @@ def run_gpu(args, c):
         dist.barrier()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(local)
-    time.sleep(0.1)
+    sampler.ready()
+    sampler.mark_start()
     start.record(stream)
     for s in range(args.steps):
         step(evs[s])
     end.record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark_end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -624,10 +661,13 @@ def run_bias_grad(args, c):
                for _ in range(args.steps)]
         sampler = ClockSampler(0) if grad else None
         if sampler is not None:
-            time.sleep(0.1)
+            sampler.ready()
+            sampler.mark_start()
         for s_i in range(args.steps):
             step(grad, evs[s_i])
         torch.cuda.synchronize(dev)
+        if sampler is not None:
+            sampler.mark_end()
         clocks = sampler.stop() if sampler is not None else None
         res[grad] = dict(fwd=statistics.fmean(e[0].elapsed_time(e[1]) for e in evs),
                          bwd=statistics.fmean(e[1].elapsed_time(e[2]) for e in evs),
