@@ -1271,20 +1271,24 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
               one_bucket = t0 + 31 <= p.t5.one_lo_max || t0 - 31 >= p.t5.one_hi_min;
             float s1 = 0.f, s2 = 0.f;
             if (one_bucket) {
-              // the row's 32 values as a pairwise tree, into the side's
-              // register sum (reduced over the warp once per item)
-              float v[16];
+              // the row's 32 values as a pairwise tree of packed fp32 pair
+              // additions, into the side's register sum (reduced over the
+              // warp once per item)
+              uint64_t v[8];
 #pragma unroll
-              for (int q = 0; q < 16; ++q)
-                v[q] = __uint_as_float(pr[32 * h + 2 * q]) + __uint_as_float(pr[32 * h + 2 * q + 1]);
+              for (int q = 0; q < 8; ++q)
+                v[q] = f2_add(f2_pack(__uint_as_float(pr[32 * h + 4 * q]), __uint_as_float(pr[32 * h + 4 * q + 1])),
+                              f2_pack(__uint_as_float(pr[32 * h + 4 * q + 2]), __uint_as_float(pr[32 * h + 4 * q + 3])));
 #pragma unroll
-              for (int w2 = 8; w2 > 0; w2 >>= 1)
+              for (int w2 = 4; w2 > 0; w2 >>= 1)
 #pragma unroll
-                for (int q = 0; q < w2; ++q) v[q] = v[2 * q] + v[2 * q + 1];
+                for (int q = 0; q < w2; ++q) v[q] = f2_add(v[2 * q], v[2 * q + 1]);
+              float va, vb;
+              f2_unpack(v[0], va, vb);
               if (t0 + 31 <= p.t5.one_lo_max)
-                one_lo += v[0];
+                one_lo += va + vb;
               else
-                one_hi += v[0];
+                one_hi += va + vb;
               continue;
             } else {
               __syncwarp();
