@@ -50,8 +50,10 @@ namespace sdpa {
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 // Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all): with
 // both warpgroups on one tile, 6 of 8 on MUFU and 2 on the FMA pipe measured
-// fastest (5 and 4 were slower).
-constexpr int kFwdMufuPer8 = 6;
+// fastest at d = 128 (5 and 4 were slower); at d = 64, where P V takes half
+// as long, 5 of 8 (t5rpe forward 0.175 -> 0.173 ms).
+template <int D>
+constexpr int kFwdMufuPer8 = (D == 64) ? 5 : 6;
 // Full tiles without a bias take the lean path: the row max is taken on the
 // raw scores (scale > 0 preserves the order), the scale folds into the one
 // fused multiply-add that forms each exponent, and pairs of columns go
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(384, 1)
                   f2_pack(__uint_as_float(xs[c0 + c]), __uint_as_float(xs[c0 + c + 1])), c2, nm2);
               float v0, v1, e0, e1;
               f2_unpack(arg, v0, v1);
-              exp2_pair<BIAS, kFwdMufuPer8>(c0 + c, v0, v1, e0, e1);
+              exp2_pair<BIAS, kFwdMufuPer8<D>>(c0 + c, v0, v1, e0, e1);
               acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(e0, e1));
               pk[c >> 1] = pack_bf16x2(e0, e1);
             }
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(384, 1)
                 const float v0 = __uint_as_float(xs[c0 + c]) - m_sub;
                 const float v1 = __uint_as_float(xs[c0 + c + 1]) - m_sub;
                 float e0, e1;
-                exp2_pair<BIAS, kFwdMufuPer8>(c0 + c, v0, v1, e0, e1);
+                exp2_pair<BIAS, kFwdMufuPer8<D>>(c0 + c, v0, v1, e0, e1);
                 sm[(c >> 1) & 3] += e0 + e1;
                 pk[c >> 1] = pack_bf16x2(e0, e1);
               }
