@@ -39,14 +39,15 @@
 namespace sdpa {
 
 // Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all),
-// chosen by measurement per head dimension: at d = 128 the dK/dV kernel
-// gains from moving 3 of 8 to the FMA pipe and the dQ kernel from none; at
-// d = 64, where the MMAs take half as long for the same exponentials, 2 of
-// 8 in both (t5rpe dQ 0.176 -> 0.168 ms, dK/dV 0.212 -> 0.208 ms).
+// chosen by measurement: at d = 128 the dK/dV kernel gains from moving 3 of
+// 8 to the FMA pipe, the dQ kernel from none without a bias and from 2 with
+// a relative-position bias (alibi_causal_4k dQ 0.955 -> 0.933 ms); at d = 64,
+// where the MMAs take half as long for the same exponentials, 2 of 8 in both
+// (t5rpe dQ 0.176 -> 0.168 ms, dK/dV 0.212 -> 0.208 ms).
 template <int D>
 constexpr int kDkdvMufuPer8 = (D == 64) ? 6 : 5;
-template <int D>
-constexpr int kDqMufuPer8 = (D == 64) ? 6 : 8;
+template <int D, int BIAS>
+constexpr int kDqMufuPer8 = (D == 64 || BIAS == kBiasT5) ? 6 : 8;
 
 // ------------------------------------------------------------ preprocess
 // D = rowsum(dO * O) for every query row along the (padded or packed)
@@ -1172,7 +1173,7 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
               if constexpr (decltype(table)::value) x2 = f2_add(x2, f2_pack(lut_row[cc], lut_row[cc + 1]));
               float x0, x1, y0, y1;
               f2_unpack(x2, x0, x1);
-              exp2_pair<BIAS, kDqMufuPer8<D>>(cc, x0, x1, y0, y1);
+              exp2_pair<BIAS, kDqMufuPer8<D, BIAS>>(cc, x0, x1, y0, y1);
               pr[cc] = __float_as_uint(y0);
               pr[cc + 1] = __float_as_uint(y1);
             }
