@@ -39,13 +39,14 @@
 namespace sdpa {
 
 // Share of a full tile's exponentials on MUFU (per 8 columns; 8 = all),
-// chosen by measurement: at d = 128 the dK/dV kernel gains from moving 3 of
-// 8 to the FMA pipe, the dQ kernel from none without a bias and from 2 with
-// a relative-position bias (alibi_causal_4k dQ 0.955 -> 0.933 ms); at d = 64,
-// where the MMAs take half as long for the same exponentials, 2 of 8 in both
-// (t5rpe dQ 0.176 -> 0.168 ms, dK/dV 0.212 -> 0.208 ms).
-template <int D>
-constexpr int kDkdvMufuPer8 = (D == 64) ? 6 : 5;
+// chosen by measurement: at d = 128 without a bias the dK/dV kernel gains
+// from moving 3 of 8 to the FMA pipe and the dQ kernel from none; with a
+// relative-position bias (whose table adds FMA-pipe work per element) 2 of
+// 8 in both (alibi_causal_4k dQ 0.955 -> 0.933 ms, dK/dV 1.244 -> 1.200);
+// at d = 64, where the MMAs take half as long for the same exponentials, 2
+// of 8 in both (t5rpe dQ 0.176 -> 0.168 ms, dK/dV 0.212 -> 0.208 ms).
+template <int D, int BIAS>
+constexpr int kDkdvMufuPer8 = (D == 64 || BIAS == kBiasT5) ? 6 : 5;
 template <int D, int BIAS>
 constexpr int kDqMufuPer8 = (D == 64 || BIAS == kBiasT5) ? 6 : 8;
 
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(352, 1)
                           f2_pack(kLog2e, kLog2e), x2);
             float x0, x1, y0, y1;
             f2_unpack(x2, x0, x1);
-            exp2_pair<BIAS, kDkdvMufuPer8<D>>(c, x0, x1, y0, y1);
+            exp2_pair<BIAS, kDkdvMufuPer8<D, BIAS>>(c, x0, x1, y0, y1);
             pr[c] = __float_as_uint(y0);
             pr[c + 1] = __float_as_uint(y1);
           }
