@@ -116,23 +116,31 @@ __device__ __forceinline__ uint4 shfl_xor_u4(uint4 v, int m) {
 template <int D, int BIAS>
 struct DkdvLayout {
   static constexpr int kTileBytes = kTile * D * 2;  // 128 rows x d bf16
+  // A dense bias at d = 64 is staged by TMA: each block's 128 x 128 fp32
+  // tile (64 KB) in a two-slot ring, loaded one block ahead, in place of
+  // 64 scattered global loads per thread that the exponentials wait for.
+  static constexpr bool kBiasTma = (BIAS == kBiasDense && D == 64);
+  static constexpr int kBiasTileBytes = kTile * kTile * 4;
+  static constexpr int kSB = kBiasTma ? 2 : 0;
   // Q blocks are used until the block's dK MMA, dO blocks only until its dV
   // MMA: the Q ring is the deeper one.  At d = 128 without a T5 table this
-  // fills the 227 KB of shared memory to the last kilobyte.
-  static constexpr int kSQ = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : 4;
-  static constexpr int kSO = (D == 128) ? 2 : 4;
+  // fills the 227 KB of shared memory to the last kilobyte; so does the
+  // bias ring with two-slot Q and dO rings at d = 64.
+  static constexpr int kSQ = (D == 128) ? (BIAS == kBiasT5 ? 2 : 3) : (kBiasTma ? 2 : 4);
+  static constexpr int kSO = (D == 128) ? 2 : (kBiasTma ? 2 : 4);
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
   static constexpr int kQOff = 2 * kTileBytes;                  // Q ring
   static constexpr int kDOOff = kQOff + kSQ * kTileBytes;       // dO ring
-  static constexpr int kVecOff = kDOOff + kSO * kTileBytes;     // 2 x (-lse2[128], D[128])
+  static constexpr int kBOff = kDOOff + kSO * kTileBytes;       // bias ring (kBiasTma), 1 KB aligned
+  static constexpr int kVecOff = kBOff + kSB * kBiasTileBytes;  // 2 x (-lse2[128], D[128])
   static constexpr int kLutOff = kVecOff + 2 * 2 * kTile * 4;   // T5 only: 8 warps x 96 floats
   static constexpr int kLutBytes = (BIAS == kBiasT5) ? 8 * 96 * 4 : 0;
   static constexpr int kBarOff = kLutOff + kLutBytes;
   // kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], vec_full[2],
   // vec_empty[2], s_full[2], dp_full, p_full[2], ds_full, s_free[2], dp_free,
-  // acc_done, drain[2]
-  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 12;
+  // acc_done, drain[2], then with the bias ring b_full[2], b_empty[2]
+  static constexpr int kNumBars = 1 + 2 * kSQ + 2 * kSO + 4 + 12 + (kBiasTma ? 4 : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemAlloc = kMiscOff + 16;
   // 2 compute warpgroups, producer, two MMA issuers
@@ -145,6 +153,7 @@ struct DkdvLayout {
   static constexpr bool kSDouble = (D == 64);
   static constexpr int kSCol1 = 384;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(kBOff % 1024 == 0, "128-byte swizzled TMA boxes start on 1 KB");
 };
 
 
@@ -152,7 +161,7 @@ template <int D, int BIAS>
 __global__ void __launch_bounds__(352, 1)
     bwd_dkdv_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    const __grid_constant__ CUtensorMap tmDO) {
+                    const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmB) {
   using Lay = DkdvLayout<D, BIAS>;
   constexpr int SQ = Lay::kSQ;
   constexpr int SO = Lay::kSO;
@@ -202,11 +211,20 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t dp_free = bar(kB + 12);
   const uint32_t acc_done = bar(kB + 13);
   auto drain = [&](int x) { return bar(kB + 14 + x); };
+  constexpr bool BT = Lay::kBiasTma;
+  auto b_full = [&](int x) { return bar(kB + 16 + x); };
+  auto b_empty = [&](int x) { return bar(kB + 18 + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    if constexpr (BT) {
+      for (int x = 0; x < 2; ++x) {
+        mbar_init(b_full(x), 1);
+        mbar_init(b_empty(x), 2 * kTile);  // both compute warpgroups
+      }
+    }
     // Q blocks are read by both issuers (S^T and dK), dO blocks too (dP^T and
     // dV): a slot is free once each issuer's last MMA on it has completed.
     for (int s = 0; s < SQ; ++s) {
@@ -280,7 +298,7 @@ __global__ void __launch_bounds__(352, 1)
         }
       };
       load_vec(0);
-      int issued_q[SQ], issued_o[SO];
+      int issued_q[SQ], issued_o[SO], issued_b[2] = {-1, -1};
       for (int e = 0; e < SQ; ++e) issued_q[e] = -1;
       for (int e = 0; e < SO; ++e) issued_o[e] = -1;
       bool ok = true;
@@ -288,11 +306,28 @@ __global__ void __launch_bounds__(352, 1)
         const int hq = g * p.G + it / nm;
         const int m0 = (mlo + it % nm) * kTile;
         const int x = it & 1;
-        // The Q / dO copies go first: they wait only for their ring slots,
-        // not for the compute warps, so they run as far ahead as the rings allow.
+        // The copies go first: they wait only for their ring slots, not for
+        // the LSE / D slot, so they run as far ahead as the rings allow.
         if (lane == 0) {
           const int sq = it % SQ, so = it % SO;
-          ok = mbar_wait(q_empty(sq), ((it / SQ) & 1) ^ 1, ctl);
+          if constexpr (BT) {
+            // ahead of Q: its slot frees once the warpgroups have formed P of
+            // the block two back, before that block's dK MMA frees Q's slot.
+            // Rows m0.. (queries) and keys n0.. of (b, hq): 4 boxes of 32
+            // keys; past either sequence the box reads zeros (those pairs
+            // are masked)
+            const uint32_t bph = (it >> 1) & 1;
+            ok = mbar_wait(b_empty(x), bph ^ 1, ctl);
+            if (ok) {
+              mbar_expect_tx(b_full(x), Lay::kBiasTileBytes);
+              const int hb = p.sb_h ? hq : 0, bb = p.sb_b ? b : 0;
+              for (int q4 = 0; q4 < 4; ++q4)
+                tma_load_4d(sb + Lay::kBOff + x * Lay::kBiasTileBytes + q4 * (kTile * 128), &tmB,
+                            b_full(x), n0 + 32 * q4, m0, hb, bb);
+              issued_b[x] = static_cast<int>(bph);
+            }
+          }
+          if (ok) ok = mbar_wait(q_empty(sq), ((it / SQ) & 1) ^ 1, ctl);
           if (ok) {
             mbar_expect_tx(q_full(sq), Lay::kTileBytes);
             for (int h = 0; h < D / 64; ++h)
@@ -333,6 +368,8 @@ __global__ void __launch_bounds__(352, 1)
           if (issued_q[e] >= 0) mbar_wait(q_full(e), issued_q[e], ign);
         for (int e = 0; e < SO; ++e)
           if (issued_o[e] >= 0) mbar_wait(o_full(e), issued_o[e], ign);
+        for (int e = 0; e < 2; ++e)
+          if (issued_b[e] >= 0) mbar_wait(b_full(e), issued_b[e], ign);
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -435,6 +472,14 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tS0 = tmem + lane_bits + c0w;  // + the block's S^T buffer column
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
+    // Staged bias: this warp's keys are box warp % 4 of the block; query
+    // column c is the box's row c0w + c, 128 bytes whose 16-byte chunks sit
+    // at chunk ^ (row % 8) (128-byte swizzle).  The warp reads one whole row
+    // per column: no bank conflicts.
+    const uint8_t* bbox = smem + Lay::kBOff + (warp & 3) * (kTile * 128) + c0w * 128;
+    uint32_t boff[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) boff[k] = (((lane >> 2) ^ k) << 4) | ((lane & 3) << 2);
     bool ok = true;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1;
@@ -464,12 +509,21 @@ __global__ void __launch_bounds__(352, 1)
         if (j >= Lk) hi = -1;  // past the key sequence: no query sees it
       }
       const float* bcol = nullptr;
-      if constexpr (BIAS == kBiasDense)
+      if constexpr (BIAS == kBiasDense && !BT)
         bcol = p.bias + static_cast<int64_t>(b) * p.sb_b + static_cast<int64_t>(hq) * p.sb_h +
                static_cast<int64_t>(min(m0, Lq - 1)) * p.sb_i + min(j, Lk - 1);
+      const uint8_t* bt = bbox + x * Lay::kBiasTileBytes;
+      // bias of query column c (every column of the staged box is in range)
+      auto bias_at = [&](int c, bool valid) -> float {
+        if constexpr (BT) return *reinterpret_cast<const float*>(bt + c * 128 + boff[c & 7]);
+        else return bcol[static_cast<int64_t>(valid ? c : 0) * p.sb_i];
+      };
       if (ok) ok = mbar_wait(vec_full(x), (it >> 1) & 1, ctl);  // LSE / D staged
       const uint32_t tS = tS0 + s_col(it);
       if (ok) ok = mbar_wait(s_full(sb_of(it)), sb_par(it), ctl);
+      if constexpr (BT) {
+        if (ok) ok = mbar_wait(b_full(x), (it >> 1) & 1, ctl);
+      }
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
@@ -492,9 +546,7 @@ __global__ void __launch_bounds__(352, 1)
                                  e ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y));
             if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[-c], lut_row[-c - 1]));
             if constexpr (BIAS == kBiasDense)
-              x2 = f2_fma(f2_pack(bcol[static_cast<int64_t>(c) * p.sb_i],
-                                  bcol[static_cast<int64_t>(c + 1) * p.sb_i]),
-                          f2_pack(kLog2e, kLog2e), x2);
+              x2 = f2_fma(f2_pack(bias_at(c, true), bias_at(c + 1, true)), f2_pack(kLog2e, kLog2e), x2);
             float x0, x1, y0, y1;
             f2_unpack(x2, x0, x1);
             exp2_pair<BIAS, kDkdvMufuPer8<D, BIAS>>(c, x0, x1, y0, y1);
@@ -514,9 +566,7 @@ __global__ void __launch_bounds__(352, 1)
                                  e ? f2_pack(l.z, l.w) : f2_pack(l.x, l.y));
             if constexpr (BIAS == kBiasT5) x2 = f2_add(x2, f2_pack(lut_row[-c], lut_row[-c - 1]));
             if constexpr (BIAS == kBiasDense)
-              x2 = f2_fma(f2_pack(bcol[static_cast<int64_t>(v0 ? c : 0) * p.sb_i],
-                                  bcol[static_cast<int64_t>(v1 ? c + 1 : 0) * p.sb_i]),
-                          f2_pack(kLog2e, kLog2e), x2);
+              x2 = f2_fma(f2_pack(bias_at(c, v0), bias_at(c + 1, v1)), f2_pack(kLog2e, kLog2e), x2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
             pr[c] = __float_as_uint(fast_exp2(v0 ? x0 : -INFINITY));
@@ -524,6 +574,7 @@ __global__ void __launch_bounds__(352, 1)
           }
         }
       }
+      if constexpr (BT) mbar_arrive(b_empty(x));  // the bias block is read
 #pragma unroll
       for (int cc = 0; cc < kBlk; cc += 32) {
         uint32_t pk[16];
@@ -1537,7 +1588,7 @@ cudaError_t launch_bwd_t(const AttnParams& p, const CUtensorMap& mq, const CUten
                                          Lay::kSmemAlloc);
     if (e != cudaSuccess) return e;
     const int ntk = (p.Lk + kTile - 1) / kTile;
-    kern<<<dim3(ntk, p.Hkv, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(p, mq, mk, mv, mdo);
+    kern<<<dim3(ntk, p.Hkv, p.B), Lay::kThreads, Lay::kSmemAlloc, st>>>(p, mq, mk, mv, mdo, mb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

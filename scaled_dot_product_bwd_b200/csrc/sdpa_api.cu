@@ -347,7 +347,7 @@ sdpa_status_t run_bwd(uint32_t phases, const AttnParams& p, const Geometry& g, c
   if (!make_axis_map(&mq, q, g, true) || !make_axis_map(&mdo, dout, g, true) ||
       !make_axis_map(&mk, k, g, false) || !make_axis_map(&mv, v, g, false))
     return SDPA_ERR_CUDA;
-  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias dQ kernel at d = 64
+  std::memset(&mb, 0, sizeof(mb));  // read only by the dense-bias kernels at d = 64
   if (p.bias_kind == kBiasDense && !make_bias_map(&mb, p)) return SDPA_ERR_CUDA;
   cudaError_t e = g.d == 128 ? launch_bwd_d<128>(p, mq, mk, mv, mdo, mb, phases, g.axis_q(), stream)
                              : launch_bwd_d<64>(p, mq, mk, mv, mdo, mb, phases, g.axis_q(), stream);

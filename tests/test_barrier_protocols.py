@@ -281,11 +281,17 @@ def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True, three_issuers=Tr
 
 
 # ---------------------------------------------------------------- dK / dV
-def dkdv_protocol(total, SQ, SO, s_double=False, p_double=True):
+def dkdv_protocol(total, SQ, SO, s_double=False, p_double=True, bias_ring=False):
     """s_double: S^T double-buffered (d = 64): S^T(i + 1) is issued before
     the wait for P^T(i); s_full, p_full and s_free then go by block parity
-    (p_double=False models one P^T-ready barrier instead)."""
+    (p_double=False models one P^T-ready barrier instead).  bias_ring: the
+    dense bias staged by TMA in two slots, issued ahead of each block's Q,
+    released by the warpgroups once P^T is formed."""
     bars = {"kv_full": 1, "dp_full": 1, "ds_full": 2, "dp_free": 1, "acc_done": 2}
+    if bias_ring:
+        for x in range(2):
+            bars[f"b_full{x}"] = 1
+            bars[f"b_empty{x}"] = 2
     nb = 2 if s_double else 1
     for x in range(nb):
         bars[f"s_full{x}"] = 1
@@ -310,6 +316,9 @@ def dkdv_protocol(total, SQ, SO, s_double=False, p_double=True):
     def producer():
         yield ("async", "kv_full")
         for it in range(total):
+            if bias_ring:
+                yield ("wait", f"b_empty{it & 1}", ((it >> 1) & 1) ^ 1)
+                yield ("async", f"b_full{it & 1}")
             yield ("wait", f"q_empty{it % SQ}", ((it // SQ) & 1) ^ 1)
             yield ("async", f"q_full{it % SQ}")
             yield ("wait", f"o_empty{it % SO}", ((it // SO) & 1) ^ 1)
@@ -358,6 +367,9 @@ def dkdv_protocol(total, SQ, SO, s_double=False, p_double=True):
         for it in range(total):
             yield ("wait", f"vec_full{it & 1}", (it >> 1) & 1)
             yield ("wait",) + par("s_full", it)
+            if bias_ring:
+                yield ("wait", f"b_full{it & 1}", (it >> 1) & 1)
+                yield ("arrive", f"b_empty{it & 1}")
             yield ("arrive", par("p_full", it)[0])
             yield ("wait", "dp_full", it & 1)
             yield ("arrive", "ds_full")
@@ -416,11 +428,12 @@ def test_dkdv_double_s_with_one_p_barrier_can_lose_a_wakeup():
     assert found
 
 
-@pytest.mark.parametrize("SQ,SO,s_double", [(3, 2, False), (2, 2, False), (4, 4, False),
-                                            (4, 4, True), (2, 2, True)])
-def test_dkdv_protocol_has_no_deadlock(SQ, SO, s_double):
+@pytest.mark.parametrize("SQ,SO,s_double,bias_ring",
+                         [(3, 2, False, False), (2, 2, False, False), (4, 4, False, False),
+                          (4, 4, True, False), (2, 2, True, False), (2, 2, True, True)])
+def test_dkdv_protocol_has_no_deadlock(SQ, SO, s_double, bias_ring):
     for total in (1, 2, 3, 7, 40):
         for seed in SEEDS:
-            bars, roles = dkdv_protocol(total, SQ, SO, s_double)
+            bars, roles = dkdv_protocol(total, SQ, SO, s_double, bias_ring=bias_ring)
             blocked = explore(bars, roles, seed)
             assert blocked is None, (total, seed, blocked)
