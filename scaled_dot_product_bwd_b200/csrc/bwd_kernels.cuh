@@ -888,14 +888,10 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
         for (int it = 0; it < w.nt; ++it, ++c) {
           const int sk = c % SK, sv = c % SV;
           const int n0 = (w.nlo + it) * kTile;
-          if (!(ok = mbar_wait(k_empty(sk), ((c / SK) & 1) ^ 1, ctl))) break;
-          mbar_expect_tx(k_full(sk), Lay::kTileBytes);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
-                        k_full(sk), h * 64, w.s.k0 + n0, w.g, w.s.bc);
-          issued_k[sk] = (c / SK) & 1;
           if constexpr (BT) {
-            // this block's bias: rows m0.., keys n0.. of (b, hq), 4 boxes
+            // this block's bias: rows m0.., keys n0.. of (b, hq), 4 boxes.
+            // Ahead of K: its slot frees once the warpgroups have formed P
+            // of the block two back, K's only after that block's dQ MMA.
             const int x = c & 1;
             const uint32_t bph = (c >> 1) & 1;
             if (!(ok = mbar_wait(b_empty(x), bph ^ 1, ctl))) break;
@@ -905,9 +901,14 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
               tma_load_4d(sb + Lay::kBOff + x * Lay::kBiasTileBytes + q4 * (kTile * 128), &tmB,
                           b_full(x), n0 + 32 * q4, w.m0, hb, bb);
             b_issued[x] = static_cast<int>(bph);
-          } else if constexpr (BIAS == kBiasDense) {
-            prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
           }
+          if (!(ok = mbar_wait(k_empty(sk), ((c / SK) & 1) ^ 1, ctl))) break;
+          mbar_expect_tx(k_full(sk), Lay::kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(sb + Lay::kKOff + sk * Lay::kTileBytes + h * kTile * 128, &tmK,
+                        k_full(sk), h * 64, w.s.k0 + n0, w.g, w.s.bc);
+          issued_k[sk] = (c / SK) & 1;
+          if constexpr (BIAS == kBiasDense && !BT) prefetch_bias_tile(p, w.b, w.hq, w.m0, n0);
           if (!(ok = mbar_wait(v_empty(sv), ((c / SV) & 1) ^ 1, ctl))) break;
           mbar_expect_tx(v_full(sv), Lay::kTileBytes);
           for (int h = 0; h < D / 64; ++h)

@@ -187,11 +187,11 @@ def dq_protocol(items, SK, SV, bias_ring=False, ds_double=True, three_issuers=Tr
                 yield ("wait", "o_empty", (u - 1) & 1)
             yield ("async", "o_full")
             for _ in range(nt):
-                yield ("wait", f"k_empty{c % SK}", ((c // SK) & 1) ^ 1)
-                yield ("async", f"k_full{c % SK}")
-                if bias_ring:
+                if bias_ring:  # the bias block goes ahead of K
                     yield ("wait", f"b_empty{c & 1}", ((c >> 1) & 1) ^ 1)
                     yield ("async", f"b_full{c & 1}")
+                yield ("wait", f"k_empty{c % SK}", ((c // SK) & 1) ^ 1)
+                yield ("async", f"k_full{c % SK}")
                 yield ("wait", f"v_empty{c % SV}", ((c // SV) & 1) ^ 1)
                 yield ("async", f"v_full{c % SV}")
                 c += 1
