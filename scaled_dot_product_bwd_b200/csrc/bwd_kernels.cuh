@@ -1101,10 +1101,22 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tDP = tmem + lane_bits + Lay::kDPCol + c0w;
     float* lut = reinterpret_cast<float*>(smem + Lay::kLutOff) + warp * 96;
+    // Bucket mode: lane l's buckets l, l + 32, ... and their distance ranges,
+    // read from the parameters once (lanes reading different entries of a
+    // parameter array are served one address at a time); a bucket past the
+    // table's count gets an empty range.
+    int rlo[4], rhi[4];
     if constexpr (DSM == kDsDiagT5) {
       // this warp's per-bucket sums; entry k is only ever touched by lane k % 32
       float* bacc = reinterpret_cast<float*>(smem + Lay::kBAccOff) + warp * 128;
       for (int k = lane; k < 128; k += 32) bacc[k] = 0.f;
+      const int nbk = p.t5.bidirectional ? 2 * p.t5.half : p.t5.half;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = lane + 32 * q;
+        rlo[q] = k < nbk ? p.t5r.lo[k] : (1 << 29);
+        rhi[q] = k < nbk ? p.t5r.hi[k] : -(1 << 29);
+      }
     }
     bool ok = true;
     int c = 0;  // key blocks so far, over all items
@@ -1394,10 +1406,12 @@ __global__ void __launch_bounds__(DqLayout<D, BIAS, DSM>::kThreads, 1)
                 if (lane == 0) stg[0] = 0.f;
                 __syncwarp();
                 const int nbk = p.t5.bidirectional ? 2 * p.t5.half : p.t5.half;
-                for (int k = lane; k < nbk; k += 32) {
-                  const int lo = max(p.t5r.lo[k] - t0, -31);
-                  const int hi = min(p.t5r.hi[k] - t0, 31);
-                  if (lo <= hi) bacc[k] += stg[hi + 32] - stg[lo + 31];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  if (32 * q >= nbk) break;
+                  const int lo = max(rlo[q] - t0, -31);
+                  const int hi = min(rhi[q] - t0, 31);
+                  if (lo <= hi) bacc[lane + 32 * q] += stg[hi + 32] - stg[lo + 31];
                 }
               }
             }
