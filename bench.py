@@ -69,12 +69,12 @@ for _hkv, _tag in ((32, "mha"), (8, "gqa"), (1, "mqa")):
 # only while the library is built from exactly those sources.
 NCU_TRAFFIC = {
     # mistral4k_small (batch 2) capture, profiles/mistral4k_small_full_capture.md
-    ("mistral4k", "fwd"): {"bytes_per_batch": (100761344 + 37730048) / 2,
-        "source_hash": "ebe599b0fe77bbafe016cd00822503210ca4b90ba29aff9824298b76c72d9da1"},
-    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (170876672 + 43709440) / 2,
-        "source_hash": "ebe599b0fe77bbafe016cd00822503210ca4b90ba29aff9824298b76c72d9da1"},
-    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (169953792 + 23550720) / 2,
-        "source_hash": "ebe599b0fe77bbafe016cd00822503210ca4b90ba29aff9824298b76c72d9da1"},
+    ("mistral4k", "fwd"): {"bytes_per_batch": (100771328 + 37383168) / 2,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
+    ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171738624 + 45638144) / 2,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
+    ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170260224 + 24276224) / 2,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
 }
 
 

@@ -51,6 +51,12 @@ CASES = {
     "cross_shorter_keys_causal_d128": dict(B=1, Hq=2, Hkv=1, L=300, Lk=140, d=128, causal=True),
     "cross_t5_d64": dict(B=2, Hq=2, Hkv=2, L=130, Lk=260, d=64, bias="t5"),
     "cross_dense_bias_d64": dict(B=1, Hq=2, Hkv=2, L=150, Lk=200, d=64, bias="dense"),
+    # queries outnumber keys under a causal mask with a dense bias staged by
+    # TMA: the bias boxes of the last tiles reach past both sequences, and
+    # two query heads share each key tile (Lk a multiple of 4: bias rows
+    # are read in 16-byte pieces)
+    "cross_dense_bias_causal_gqa_d64": dict(B=2, Hq=4, Hkv=2, L=330, Lk=148, d=64, causal=True,
+                                            bias="dense"),
     # (keys outnumber queries: with 257 queries over 129 keys under a causal
     # mask and ALiBi slope 1/4, the last key collects a probability mass of
     # ~24 and bf16 rounding of P alone moves its dV past the fixed bound)
