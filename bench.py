@@ -49,6 +49,10 @@ CONFIGS = {
     # the t5rpe shape at batch 4: the case the bias-gradient ncu capture runs
     # on (its fp32 dS, 200 MB, still larger than L2)
     "t5rpe_small": dict(B=4, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1, bias="t5"),
+    # the t5dense shape at batch 4: the case its ncu capture runs on (the
+    # fp32 bias, 200 MB, still larger than L2)
+    "t5dense_small": dict(B=4, Hq=12, Hkv=12, L=1024, d=64, causal=False, wl=-1, wr=-1,
+                          bias="dense"),
     # the mistral4k shape at batch 2: the case the ncu captures run on (inputs
     # still larger than L2, a few hundred MB on the device)
     "mistral4k_small": dict(B=2, Hq=32, Hkv=8, L=4096, d=128, causal=True, wl=4096, wr=-1,
@@ -74,6 +78,13 @@ NCU_TRAFFIC = {
     ("mistral4k", "bwd_dq"): {"bytes_per_batch": (171738624 + 45638144) / 2,
         "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
     ("mistral4k", "bwd_dkdv"): {"bytes_per_batch": (170260224 + 24276224) / 2,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
+    # t5dense_small (batch 4) capture, profiles/t5dense_small_capture.md
+    ("t5dense", "fwd"): {"bytes_per_batch": (233312768 + 5899776) / 4,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
+    ("t5dense", "bwd_dq"): {"bytes_per_batch": (241260288 + 6072064) / 4,
+        "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
+    ("t5dense", "bwd_dkdv"): {"bytes_per_batch": (227603456 + 8563200) / 4,
         "source_hash": "99e2ec3349212877272f08c8b7b1e98abfcf74474ee83ea1a209a2e3e5a6bec4"},
 }
 
