@@ -75,7 +75,8 @@ def assert_close(got: dict, ref: dict, names=("o", "lse", "dq", "dk", "dv")):
         assert sel.any(), n
         rs, gs = r[sel], g[sel]
         both_inf = np.isinf(rs) & (rs == gs)
-        err = np.where(both_inf, 0.0, np.abs(gs.astype(np.float64) - rs))
+        with np.errstate(invalid="ignore"):  # inf - inf where both agree: masked below
+            err = np.where(both_inf, 0.0, np.abs(gs.astype(np.float64) - rs))
         if n == "lse":
             tol = np.full_like(rs, LSE_ATOL)
         else:
