@@ -173,25 +173,38 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs.
+    """SM clock and clock-event (throttle) reasons sampled while the timed
+    region runs.
 
-    A reader thread timestamps every sample.  ready() waits until nvidia-smi
-    is producing samples (its first one can take a second on a fresh box), so
-    that the timed region, bracketed by mark_start() / mark_end(), falls
-    inside the sampled stretch; the report keeps the samples taken during the
-    region, or the one nearest to it when the region is shorter than the
-    sampling interval."""
+    NVML is polled from a thread every ~2 ms on the GPU that CUDA device
+    `gpu` is (found by its UUID, so CUDA_VISIBLE_DEVICES cannot point it at
+    another GPU); where NVML cannot be used, nvidia-smi's query loop is read
+    instead.  Every sample is timestamped.  ready() waits for the first
+    sample, so that the timed region, bracketed by mark_start() /
+    mark_end(), falls inside the sampled stretch; the report keeps the
+    samples taken during the region, or the one nearest to it when the
+    region is shorter than the sampling interval.  Only reads settings."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, gpu: int):
         import threading
         self.proc = None
-        self.lines = []          # (monotonic time, line)
+        self.nvml = None
+        self.rows = []           # (monotonic time, sm MHz, max sm MHz, {reasons})
+        self.lines = []          # nvidia-smi: (monotonic time, line)
         self.t0 = self.t1 = None
         self.first = threading.Event()
+        self.halt = threading.Event()
+        self.reader = None
+        if self._open_nvml(gpu):
+            self.reader = threading.Thread(target=self._poll, daemon=True)
+            self.reader.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -203,13 +216,50 @@ class ClockSampler:
         self.reader = threading.Thread(target=self._read, daemon=True)
         self.reader.start()
 
+    def _open_nvml(self, gpu):
+        try:
+            import pynvml
+            import torch
+            uuid = str(torch.cuda.get_device_properties(gpu).uuid)
+            pynvml.nvmlInit()
+        except Exception:
+            return False
+        try:
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.reasons_of = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.reasons_of(h)
+            pre = ("nvmlClocksEventReason" if hasattr(pynvml, "nvmlClocksEventReasonHwSlowdown")
+                   else "nvmlClocksThrottleReason")
+            self.bits = {n: getattr(pynvml, pre + b) for n, b in zip(
+                self.NAMES, ("HwSlowdown", "HwThermalSlowdown", "SwThermalSlowdown", "SwPowerCap"))}
+        except Exception:
+            pynvml.nvmlShutdown()
+            return False
+        self.nvml, self.handle = pynvml, h
+        return True
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while not self.halt.is_set():
+            t = time.monotonic()
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = int(self.reasons_of(h))
+            except Exception:
+                break
+            self.rows.append((t, sm, self.max_mhz, {n for n, b in self.bits.items() if r & b}))
+            self.first.set()
+            self.halt.wait(self.PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append((time.monotonic(), line))
             self.first.set()
 
     def ready(self, timeout=5.0):
-        if self.proc is not None:
+        if self.reader is not None:
             self.first.wait(timeout)
 
     def mark_start(self):
@@ -219,39 +269,47 @@ class ClockSampler:
         self.t1 = time.monotonic()
 
     def stop(self):
-        if self.proc is None:
+        if self.reader is None:
             return None
-        time.sleep(0.06)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            self.proc.wait()
-        self.reader.join(timeout=5)
-        rows = []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for t, line in self.lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
+        if self.nvml is not None:
+            self.halt.set()
+            self.reader.join(timeout=5)
+            self.nvml.nvmlShutdown()
+            rows, source = self.rows, "nvml"
+        else:
+            time.sleep(0.06)
+            self.proc.terminate()
             try:
-                rows.append((t, float(f[1]), float(f[2]),
-                             {n for n, v in zip(names, f[5:9]) if v.lower().startswith("active")}))
-            except ValueError:
-                continue
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.proc.wait()
+            self.reader.join(timeout=5)
+            rows, source = [], "nvidia-smi"
+            for t, line in self.lines:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    rows.append((t, float(f[1]), float(f[2]),
+                                 {n for n, v in zip(self.NAMES, f[5:9])
+                                  if v.lower().startswith("active")}))
+                except ValueError:
+                    continue
         if not rows:
             return None
         t0 = self.t0 if self.t0 is not None else rows[0][0]
         t1 = self.t1 if self.t1 is not None else rows[-1][0]
-        inside = [r for r in rows if t0 <= r[0] <= t1 + 0.05]
+        # nvidia-smi lines are stamped when read, a little after they were taken
+        slack = 0.05 if source == "nvidia-smi" else 0.0
+        inside = [r for r in rows if t0 <= r[0] <= t1 + slack]
         if not inside:  # region shorter than the sampling interval: the nearest sample
             mid = 0.5 * (t0 + t1)
             inside = [min(rows, key=lambda r: abs(r[0] - mid))]
         reasons = set().union(*(r[3] for r in inside))
         return {"sm_mhz": statistics.median(r[1] for r in inside),
                 "sm_max_mhz": max(r[2] for r in inside), "samples": len(inside),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "source": source}
 
 
 def make_case(c, seed):
