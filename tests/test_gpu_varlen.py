@@ -66,7 +66,8 @@ def rounding_allowance(q, k, do, O, P, dS, scale):
 def _close(name, got, ref, atol, extra=0.0):
     got = got.float().cpu().numpy()
     both_inf = np.isinf(ref) & (ref == got)
-    err = np.where(both_inf, 0.0, np.abs(got - ref))
+    with np.errstate(invalid="ignore"):  # inf - inf where both agree: masked below
+        err = np.where(both_inf, 0.0, np.abs(got - ref))
     tol = atol + (RTOL * np.abs(ref) if atol == ATOL else 0.0) + extra
     bad = ~(err <= tol)
     where = [tuple(int(x) for x in ix) for ix in np.argwhere(bad)[:6]]
